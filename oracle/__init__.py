@@ -1,0 +1,151 @@
+"""CPU oracle for the multi-adapter LoRA linear layer (ctypes wrapper).
+
+TEST INFRASTRUCTURE ONLY. Only tests/, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` may import this package. The product path
+(the CUDA library and its binding) never imports it and shares no code with it.
+
+Functions follow the definitions cited in ``lora_oracle.c``; all arithmetic
+is fp64 over exactly widened bf16 inputs. Parity pins live in
+``tests/test_oracle.py``.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "lora_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+
+_i64 = ctypes.c_int64
+_i32 = ctypes.c_int32
+_u64 = ctypes.c_uint64
+_dbl = ctypes.c_double
+_vp = ctypes.c_void_p
+
+
+def build(force: bool = False) -> str:
+    """Compile the oracle with gcc (-O2, OpenMP, no fast-math)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        subprocess.check_call(["gcc", "-O2", "-fopenmp", "-fPIC", "-shared", "-std=c11",
+                               "-o", _LIB, _SRC, "-lm"])
+    return _LIB
+
+
+_lib = None
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        build()
+        L = ctypes.CDLL(_LIB)
+        L.oracle_splitmix64_at.restype = _u64
+        L.oracle_splitmix64_at.argtypes = [_u64, _u64]
+        L.oracle_splitmix64_next.restype = _u64
+        L.oracle_splitmix64_next.argtypes = [ctypes.POINTER(_u64)]
+        L.oracle_drop_threshold.restype = _u64
+        L.oracle_drop_threshold.argtypes = [_dbl]
+        L.oracle_mask.restype = None
+        L.oracle_mask.argtypes = [_u64, _dbl, _i64, _i64, _vp]
+        L.oracle_plan.restype = ctypes.c_int
+        L.oracle_plan.argtypes = [_vp, _i64, _i32, _vp, _vp, _vp]
+        L.oracle_fwd.restype = None
+        L.oracle_fwd.argtypes = [_i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _dbl, _u64, _vp, _i64, _vp, _vp, _i64]
+        L.oracle_bwd.restype = None
+        L.oracle_bwd.argtypes = [_i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
+                                 _dbl, _u64, _vp, _vp, _i64, _vp, _vp, _vp]
+        L.oracle_num_threads.restype = ctypes.c_int
+        L.oracle_num_threads.argtypes = []
+        _lib = L
+    return _lib
+
+
+def _p(a):
+    return None if a is None else a.ctypes.data_as(_vp)
+
+
+def _c(a, dt):
+    return np.ascontiguousarray(a, dtype=dt)
+
+
+def num_threads() -> int:
+    return int(lib().oracle_num_threads())
+
+
+def splitmix64_at(seed: int, n: int) -> int:
+    return int(lib().oracle_splitmix64_at(seed & (2**64 - 1), n))
+
+
+def splitmix64_stream(seed: int, count: int) -> list[int]:
+    st = _u64(seed & (2**64 - 1))
+    return [int(lib().oracle_splitmix64_next(ctypes.byref(st))) for _ in range(count)]
+
+
+def drop_threshold(p: float) -> int:
+    return int(lib().oracle_drop_threshold(float(p)))
+
+
+def mask(seed: int, p: float, T: int, d_in: int) -> np.ndarray:
+    """uint8 [T, d_in]: 1 where the LoRA-branch input element is dropped."""
+    out = np.empty((T, d_in), dtype=np.uint8)
+    lib().oracle_mask(seed, float(p), T, d_in, _p(out))
+    return out
+
+
+def plan(ids, n_adapters: int):
+    """(perm int32[T], segments int32[n_seg, 3] of (adapter, start, length))."""
+    ids = _c(ids, np.int32)
+    T = ids.shape[0]
+    perm = np.empty(T, dtype=np.int32)
+    seg = np.empty((max(1, min(T, n_adapters)), 3), dtype=np.int32)
+    ns = _i32(0)
+    rc = lib().oracle_plan(_p(ids), T, n_adapters, _p(perm), _p(seg), ctypes.cast(ctypes.pointer(ns), _vp))
+    if rc != 0:
+        raise ValueError("adapter id out of range")
+    return perm, seg[: ns.value].copy()
+
+
+def _common(inp):
+    return (_c(inp.ids, np.int32), _c(inp.ranks, np.int32), _c(inp.scale, np.float32),
+            _c(inp.X, np.uint16), _c(inp.W, np.uint16), _c(inp.A_pool, np.uint16),
+            _c(inp.B_pool, np.uint16))
+
+
+def forward(inp, rows=None, p=None, seed=None, want_u=False):
+    """Y (fp64 [n_rows, d_out]) and optionally U (fp64 [n_rows, r_max]) for the
+    given original token rows (default: all)."""
+    ids, ranks, scale, X, W, A, B = _common(inp)
+    rows = np.arange(inp.T, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    p = inp.p_drop if p is None else p
+    seed = inp.mask_seed if seed is None else seed
+    Y = np.empty((rows.shape[0], inp.d_out), dtype=np.float64)
+    rmax = int(ranks.max()) if ranks.size else 1
+    U = np.empty((rows.shape[0], rmax), dtype=np.float64) if want_u else None
+    lib().oracle_fwd(inp.T, inp.d_in, inp.d_out, ranks.shape[0], _p(ids), _p(ranks), _p(scale),
+                     _p(X), _p(W), _p(A), _p(B), float(p), seed, _p(rows), rows.shape[0],
+                     _p(Y), _p(U), rmax)
+    return (Y, U) if want_u else Y
+
+
+def backward(inp, rows=None, p=None, seed=None, dY=None, want_dAB=True):
+    """dX rows (fp64 [n_rows, d_in]), dA_pool (fp64 [sum r, d_in]) and
+    dB_pool (fp64 [sum r, d_out])."""
+    ids, ranks, scale, X, W, A, B = _common(inp)
+    dY = _c(inp.dY if dY is None else dY, np.uint16)
+    rows = np.arange(inp.T, dtype=np.int64) if rows is None else _c(rows, np.int64)
+    p = inp.p_drop if p is None else p
+    seed = inp.mask_seed if seed is None else seed
+    R = int(ranks.sum())
+    dX = np.empty((rows.shape[0], inp.d_in), dtype=np.float64)
+    dA = np.empty((R, inp.d_in), dtype=np.float64) if want_dAB else None
+    dB = np.empty((R, inp.d_out), dtype=np.float64) if want_dAB else None
+    lib().oracle_bwd(inp.T, inp.d_in, inp.d_out, ranks.shape[0], _p(ids), _p(ranks), _p(scale),
+                     _p(X), _p(W), _p(A), _p(B), float(p), seed, _p(dY), _p(rows), rows.shape[0],
+                     _p(dX), _p(dA), _p(dB))
+    return dX, dA, dB
