@@ -1,0 +1,460 @@
+"""Benchmark of the multi-adapter LoRA linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl lora|reference]
+
+One step = one pass of the layer's whole hot path over one batch: the shrink
+(U = (D ⊙ X)·A_a per token) and the fused tcgen05 GEMM (Y = X·W + s_a·U·B_a)
+over a plan built once per batch (and, for the fine-tuning workload, the
+backward dU -> dX GEMM -> dA, dB). Inputs are resident in HBM; steps rotate
+over several input copies whose total exceeds the 126 MB L2, so no step reads
+its operands from a warm L2. Steps are CUDA-graph replays (one graph per input
+copy) timed with CUDA events on the replay stream, max over ranks.
+
+Prints one JSON line (rank 0). `value` = tokens of all ranks / max-over-ranks
+device time of the K timed steps. `e2e` is the same metric through the public
+API with host buffers: per step the plan is built from host ids, X is copied
+from pinned host memory, the forward runs, Y is copied back.
+
+Under torchrun each rank processes its own batch of the same workload (weak
+scaling, no collective on the data path).
+
+--impl reference times the CPU oracle (fp64 loops, all host cores) on a
+bounded sample of the same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from lora_adapter_execution_b200 import workloads as wl  # noqa: E402
+
+METRIC = "tokens/s per fused multi-LoRA linear at 1 B200; % of bf16 TC peak / HBM roofline"
+L2_BYTES = 126 * 1024 * 1024
+DEFAULT_STEPS = {"tiny": 2000, "decode": 3000, "prefill": 200, "fleet": 1000, "finetune": 100}
+DEFAULT_WARMUP = 5
+WORKLOAD_TEXT = {
+    "tiny": "tiny: T=64, d_in=d_out=256, 4 adapters ranks {4,8,8,16}, s=16/r, ids uniform",
+    "decode": "decode: T=256, d_in=d_out=4096, 64 adapters rank 16, s=2, ids uniform (unsorted)",
+    "prefill": "prefill: T=8192, d_in=4096, d_out=11008, 200 adapters ranks {8,16,32,64}, Zipf(1.0) per 512-token request",
+    "fleet": "fleet: T=4096, d_in=d_out=4096, 1000 adapters ranks 1..21, B rows x 1/k, Zipf(1.2) per token",
+    "finetune": "finetune: T=16384, d_in=d_out=4096, 1 adapter rank 16, s=2, dropout 0.1; forward + backward",
+}
+KERNEL_SOURCES = ["lora_adapter_execution_b200/csrc/gemm.cuh", "lora_adapter_execution_b200/csrc/common.cuh"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=None)
+    ap.add_argument("--warmup", type=int, default=DEFAULT_WARMUP)
+    ap.add_argument("--config", default="decode", choices=list(wl.WORKLOADS))
+    ap.add_argument("--impl", default="lora", choices=["lora", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    a = ap.parse_args()
+    if a.steps is None:
+        a.steps = DEFAULT_STEPS[a.config]
+    a.warmup = max(3, a.warmup)
+    return a
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except Exception:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+            self.t.join(timeout=2)
+
+    def summary(self):
+        sm, smax, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax = float(f[2])
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- helpers
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d["hbm_gbs"], d["bf16_tflops"], d.get("bf16_tflops_sustained"), "measured"
+    return 6650.0, 1590.0, 1400.0, "fallback"
+
+
+def kernel_src_sha():
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        h.update(open(os.path.join(ROOT, f), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(config):
+    """dram bytes per launch of the fused GEMM from a committed ncu capture, if the
+    kernel source has not changed since (profiles/traffic.json)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(config)
+    if not d or d.get("src_sha") != kernel_src_sha():
+        return None
+    return d.get("traffic_bytes_per_launch")
+
+
+def algorithmic(inp, info):
+    """Per-launch algorithmic bytes and flops of the fused GEMM, and of the whole
+    layer (forward): bytes read or written at least once, flops of the dense math
+    without block-diagonal padding."""
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    R_used, R_tok = info["sum_r_used"], info["sum_r_tokens"]
+    gemm_bytes = 2 * (T * di + di * do + do * R_used + T * do)
+    gemm_flops = 2 * T * di * do + 2 * do * R_tok
+    layer_bytes = 2 * (T * di + di * do + T * do + (di + do) * R_used)
+    layer_flops = 2 * T * di * do + 2 * (di + do) * R_tok
+    return gemm_bytes, gemm_flops, layer_bytes, layer_flops
+
+
+# ----------------------------------------------------------------------------- reference arm
+def oracle_sample(inp, rows_budget_s: float, rank_info=None):
+    """Time the oracle on a bounded sample; returns (tokens, seconds, sample text)."""
+    import oracle
+    if inp.dY is not None:
+        # forward + backward on the first Ts tokens (a smaller batch of the same workload)
+        def run(Ts):
+            sub = wl.Inputs(spec=inp.spec, T=Ts, d_in=inp.d_in, d_out=inp.d_out, ranks=inp.ranks,
+                            ids=inp.ids[:Ts].copy(), scale=inp.scale, X=inp.X[:Ts].copy(), W=inp.W,
+                            A_pool=inp.A_pool, B_pool=inp.B_pool, dY=inp.dY[:Ts].copy(), p_drop=inp.p_drop,
+                            mask_seed=inp.mask_seed, offsets=inp.offsets)
+            t0 = time.perf_counter()
+            oracle.forward(sub)
+            oracle.backward(sub)
+            return time.perf_counter() - t0
+        Ts = 4
+        dt = run(Ts)
+        Ts = int(max(4, min(inp.T, Ts * rows_budget_s / max(dt, 1e-3))))
+        dt = run(Ts)
+        return Ts, dt, f"forward+backward of the first {Ts} tokens (sub-batch of the same workload)"
+    rows = np.arange(min(inp.T, 8), dtype=np.int64)
+    t0 = time.perf_counter()
+    oracle.forward(inp, rows=rows)
+    dt = time.perf_counter() - t0
+    n = int(max(8, min(inp.T, 8 * rows_budget_s / max(dt, 1e-3))))
+    rows = np.linspace(0, inp.T - 1, n).astype(np.int64)
+    t0 = time.perf_counter()
+    oracle.forward(inp, rows=rows)
+    dt = time.perf_counter() - t0
+    return n, dt, f"forward of {n} evenly spaced tokens of the batch"
+
+
+def run_reference(a):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return
+    import oracle
+    inp = wl.make_inputs(a.config)
+    oracle.build()
+    cores = oracle.num_threads()
+    budget = max(2.0, 120.0 / max(1, a.steps + a.warmup))
+    for _ in range(a.warmup):
+        oracle_sample(inp, budget / 4)
+    tok = 0
+    secs = 0.0
+    sample = ""
+    for _ in range(a.steps):
+        n, dt, sample = oracle_sample(inp, budget)
+        tok += n
+        secs += dt
+    v = tok / secs
+    out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
+           "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * secs / a.steps,
+           "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": WORKLOAD_TEXT[a.config]},
+           "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+           "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+# ----------------------------------------------------------------------------- lora arm
+def run_lora(a):
+    import torch
+    import torch.distributed as dist
+
+    import lora_adapter_execution_b200 as lora
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+    lora.load_library()
+
+    # each rank its own batch (tokens and ids) of the same layer
+    inp = wl.make_inputs(a.config, seed=rank)
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    finetune = inp.dY is not None
+
+    def d(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+
+    per_copy = 2 * (T * di + di * do + T * do) + 2 * (di + do) * int(inp.offsets[-1])
+    if finetune:
+        per_copy += 2 * (T * do + 2 * T * di)
+    n_copies = max(2, min(8, math.ceil(3 * L2_BYTES / per_copy)))
+    plan = lora.Plan(inp.ids, inp.ranks, di, do)
+    info = plan.info()
+    r_max = info["r_max"]
+    scale = torch.from_numpy(inp.scale).to(dev)
+    copies = []
+    for c in range(n_copies):
+        cp = dict(X=d(inp.X), W=d(inp.W), A=d(inp.A_pool), B=d(inp.B_pool),
+                  Y=torch.empty(T, do, dtype=torch.bfloat16, device=dev),
+                  U=torch.empty(T, r_max, dtype=torch.bfloat16, device=dev) if finetune else None)
+        if finetune:
+            r = int(inp.ranks[0])
+            cp.update(dY=d(inp.dY), dX=torch.empty(T, di, dtype=torch.bfloat16, device=dev),
+                      dA=torch.empty(r, di, dtype=torch.float32, device=dev),
+                      dB=torch.empty(r, do, dtype=torch.float32, device=dev),
+                      ws=torch.empty(lora.bwd_workspace_size(T, di, do, r), dtype=torch.uint8, device=dev))
+        copies.append(cp)
+
+    # one graph per copy; the plan (and its scratch) is shared, steps run in order
+    def step(cp):
+        lora.linear_shrink(plan, cp["X"], cp["A"], scale, p_drop=inp.p_drop, seed=inp.mask_seed, U_save=cp["U"])
+        lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
+        if finetune:
+            lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"], cp["dX"],
+                            cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed)
+
+    launches_per_step = 2 + (6 if finetune else 0)
+    stream = torch.cuda.Stream(device=dev)
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        step(copies[0])  # first call sets kernel attributes outside any capture
+    torch.cuda.synchronize()
+    graphs, ggraphs, bgraphs = [], [], []
+    for cp in copies:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(cp)
+        graphs.append(g)
+        g2 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g2, stream=stream):
+            lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
+        ggraphs.append(g2)
+        g3 = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g3, stream=stream):
+            lora.base_gemm(cp["X"], cp["W"], cp["Y"])
+        bgraphs.append(g3)
+    torch.cuda.synchronize()
+    assert lora.device_status() == 0
+
+    def timed(gs, K, sampler_index=None):
+        for i in range(a.warmup):
+            gs[i % len(gs)].replay()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for i in range(K):
+                gs[i % len(gs)].replay()
+            e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        ms = e0.elapsed_time(e1)
+        if world > 1:
+            t = torch.tensor([ms], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ms = float(t.item())
+        return ms
+
+    K = a.steps
+    with ClockSampler(local_rank) as clk:
+        ms_total = timed(graphs, K)
+    clocks = clk.summary()
+    ms_gemm = timed(ggraphs, K)
+    ms_base = timed(bgraphs, K)
+    assert lora.device_status() == 0
+
+    # torch.matmul base for the overhead reference (cuBLAS, same shape and rotation)
+    tgraphs = []
+    for cp in copies:
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            torch.matmul(cp["X"], cp["W"], out=cp["Y"])
+        tgraphs.append(g)
+    ms_torch = timed(tgraphs, K)
+
+    value = world * T * K / (ms_total * 1e-3)
+    hbm, tc_burst, tc_sust, src = peaks()
+    gb, gf, lb, lf = algorithmic(inp, info)
+    t_gemm = ms_gemm * 1e-3 / K
+    if a.config in ("decode", "tiny"):
+        achieved = gb / t_gemm / 1e9
+        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
+                "peak_kind": f"{src} hbm_gbs (burst copy)"}
+    else:
+        achieved = gf / t_gemm / 1e12
+        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_burst, "unit": "TFLOP/s",
+                "frac": achieved / tc_burst, "peak_kind": f"{src} bf16_tflops (burst)"}
+    roof.update({"traffic": recorded_traffic(a.config), "kernel": "lora_gemm_kernel (fused base + adapter GEMM)",
+                 "algorithmic_per_launch": gb if roof["bound"] == "hbm" else gf,
+                 "avg_launch_us": t_gemm * 1e6})
+
+    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+           "warmup": a.warmup, "ms_per_step": ms_total / K, "higher_is_better": True, "scaling": "weak",
+           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+           "config": {"workload": WORKLOAD_TEXT[a.config], "tokens_per_rank": T,
+                      "l2": f"inputs rotate over {n_copies} copies ({n_copies * per_copy / 2**20:.0f} MiB > 126 MiB L2)",
+                      "timing": "CUDA-graph replays, CUDA events on the replay stream, max over ranks",
+                      "parallelism": f"dp{world} (independent batches)",
+                      "plan": "built once per batch outside the timed region (reused by every layer)"},
+           "roofline": roof,
+           "gpu_launches": launches_per_step * K,
+           "clocks": clocks,
+           "layer": {"fused_gemm_us": t_gemm * 1e6, "base_gemm_us": ms_base * 1e3 / K,
+                     "torch_matmul_us": ms_torch * 1e3 / K, "step_us": ms_total * 1e3 / K,
+                     "overhead_vs_base": (ms_total / min(ms_base, ms_torch)) - 1.0 if not finetune else None,
+                     "layer_alg_bytes": lb, "layer_alg_flops": lf,
+                     "segments": info["n_segments"], "aug_k_total": info["aug_k_total"]}}
+
+    # ---- end to end through the public API with host buffers
+    if not a.no_e2e:
+        pin_X = torch.from_numpy(inp.X.view(np.int16)).view(torch.bfloat16).pin_memory()
+        pin_Y = torch.empty(T, do, dtype=torch.bfloat16).pin_memory()
+        cp = copies[0]
+        h2d = pin_X.numel() * 2 + inp.ids.nbytes
+        d2h = pin_Y.numel() * 2
+        extra = {}
+        if finetune:
+            pin_dY = torch.from_numpy(inp.dY.view(np.int16)).view(torch.bfloat16).pin_memory()
+            pin_dX = torch.empty(T, di, dtype=torch.bfloat16).pin_memory()
+            h2d += pin_dY.numel() * 2
+            d2h += pin_dX.numel() * 2
+        Ke = max(3, min(K, 200 if not finetune else 20))
+
+        def e2e_step():
+            p = lora.Plan(inp.ids, inp.ranks, di, do, stream=stream)
+            with torch.cuda.stream(stream):
+                cp["X"].copy_(pin_X, non_blocking=True)
+                lora.linear_fwd(p, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["Y"], p_drop=inp.p_drop,
+                                seed=inp.mask_seed, U_save=cp["U"])
+                if finetune:
+                    cp["dY"].copy_(pin_dY, non_blocking=True)
+                    lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"],
+                                    cp["dX"], cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed)
+                    pin_dX.copy_(cp["dX"], non_blocking=True)
+                pin_Y.copy_(cp["Y"], non_blocking=True)
+            stream.synchronize()
+            p.destroy()
+
+        for _ in range(2):
+            e2e_step()
+        if world > 1:
+            dist.barrier()
+        t0 = time.perf_counter()
+        for _ in range(Ke):
+            e2e_step()
+        dt = time.perf_counter() - t0
+        if world > 1:
+            t = torch.tensor([dt], device=dev, dtype=torch.float64)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            dt = float(t.item())
+        out["e2e"] = {"value": world * T * Ke / dt, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+                      "d2h_bytes_per_step": int(d2h), "steps": Ke,
+                      "what": "plan from host ids + H2D of X (pinned) + forward" + (" + backward" if finetune else "")
+                              + " + D2H of the result, host wall clock per step"}
+
+    # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
+    if rank == 0 and world == 1 and not a.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        n, dt, sample = oracle_sample(inp, 15.0)
+        out["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+                               "kind": "oracle", "sample": sample}
+
+    for cp in copies:
+        cp.clear()
+    del graphs, ggraphs, bgraphs, tgraphs
+    plan.destroy()
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def main():
+    a = parse()
+    if a.impl == "reference":
+        run_reference(a)
+    else:
+        run_lora(a)
+
+
+if __name__ == "__main__":
+    main()

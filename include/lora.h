@@ -1,0 +1,236 @@
+/*
+ * lora.h — C ABI of the B200 (sm_100a) heterogeneous multi-adapter LoRA linear layer.
+ *
+ * The layer computes, for every token t carrying adapter id a = ids[t],
+ *
+ *     Y[t] = X[t]·W + s_a·((D ⊙ X)[t]·A_a)·B_a
+ *
+ * with W frozen and each adapter keeping its own rank r_a (no padding to a
+ * common rank), D an optional dropout mask on the LoRA-branch input.
+ *  - The LoRA reparameterisation Y = X·W + X·(A·B) with A in R^{d x r},
+ *    B in R^{r x k}, W frozen: "LoRAFusion：消除冗余内存访问的多 LoRA 高效微调系统",
+ *    section 解决什么真问题 (what problem it solves), item 1.
+ *  - Computing xAB on the fly for a batch mixing many adapters, base part
+ *    batched, without padding: "S-LoRA：一个GPU运行数千大模型成为可能",
+ *    section 批处理 (batching).
+ *  - Rank-exact factor storage (a rank-R weight occupies R vectors of the
+ *    hidden size): same S-LoRA article, section Unified Paging.
+ *  - Keeping each adapter at its retained rank instead of padding or
+ *    re-expanding: "LoRAForge：压缩与执行协同，让多LoRA服务更高效",
+ *    section 核心设计 (core design).
+ *  - Dropout is one of the small memory-bound ops between the GEMMs of a LoRA
+ *    forward: LoRAFusion explainer, section 解决什么真问题, item 1.
+ *
+ * Conventions for every entry point:
+ *  - bf16 tensors are passed as `uint16_t*` holding bf16 bit patterns, row-major,
+ *    contiguous, in DEVICE memory, 16-byte aligned. Sizes are element counts.
+ *  - The caller owns every tensor buffer. A plan owns its own small device and
+ *    host arrays (and its forward scratch) until lora_plan_destroy.
+ *  - Every call that launches work is asynchronous and ordered on `stream`
+ *    (a cudaStream_t; NULL is the legacy default stream). Nothing synchronises
+ *    the host except lora_plan_build (which copies the plan to the device) and
+ *    lora_device_status.
+ *  - Return value: LORA_OK (0) or a negative LORA_ERR_* code. Arguments are
+ *    validated on the host before any launch; on an error nothing is launched.
+ *    No exception crosses the ABI.
+ *  - Kernels never trap: a device-side bounds violation or a wait that runs
+ *    out of time sets a per-device status word (see lora_device_status) and the
+ *    kernel returns early.
+ */
+#ifndef LORA_B200_H
+#define LORA_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st *lora_stream_t; /* identical to cudaStream_t */
+typedef struct lora_plan *lora_plan_t;
+
+enum lora_status {
+    LORA_OK = 0,
+    LORA_ERR_ARG = -1,         /* null pointer, non-positive size, size not a multiple of 8, misaligned pointer */
+    LORA_ERR_ID = -2,          /* an adapter id outside [0, n_adapters) */
+    LORA_ERR_RANK = -3,        /* a rank outside [1, LORA_MAX_RANK] */
+    LORA_ERR_CUDA = -4,        /* a CUDA runtime or driver call failed */
+    LORA_ERR_DEVICE = -5,      /* the device status word was set (bounds or wait timeout) */
+    LORA_ERR_UNSUPPORTED = -6, /* the current device is not sm_100 */
+    LORA_ERR_NOMEM = -7,       /* a plan allocation failed */
+    LORA_ERR_WORKSPACE = -8    /* workspace pointer null or smaller than required */
+};
+
+#define LORA_MAX_RANK 256
+#define LORA_TILE_M 128 /* tokens per output tile of the fused GEMM */
+
+/* Device status word bits (lora_device_status). */
+#define LORA_DEV_TIMEOUT 0x1u /* a bounded wait inside a kernel ran out of time */
+#define LORA_DEV_BOUNDS 0x2u  /* a kernel saw an index outside its buffers and skipped it */
+
+/* ------------------------------------------------------------------------
+ * lora_plan_build — group a batch's tokens by adapter (once per batch).
+ *
+ * Sorts the T tokens by adapter id (stable: ties keep their original order)
+ * into segments of consecutive tokens sharing one adapter, cuts the sorted
+ * order into 128-token output tiles, and lists for each tile the adapters it
+ * touches with their ranks and factor-pool offsets (off_a = sum of ranks of
+ * adapters 0..a-1). A plan depends only on (ids, ranks, d_in, d_out) and can be
+ * reused by every LoRA linear layer of one batch that shares them; deciding the
+ * routing once per batch and reusing it across layers follows the token-level
+ * pre-gating idea of "AdaFuse: Accelerating Dynamic Adapter Inference via
+ * Token-Level Pre-Gating and Fused Kernel Optimization", 方法详解 (method),
+ * 整体框架 (framework).
+ *
+ *   ids_host    int32[T] host: adapter id of each token, in [0, n_adapters)
+ *   T           number of tokens, >= 1
+ *   ranks_host  int32[n_adapters] host: r_a in [1, LORA_MAX_RANK]
+ *   n_adapters  >= 1
+ *   d_in, d_out input / output width, multiples of 8, >= 8
+ *   stream      stream for the plan's host-to-device copy; the call
+ *               synchronises it, so the plan is on the device on return (and
+ *               the host arrays may be freed)
+ *   out         receives the plan; unchanged on error
+ * Errors: LORA_ERR_ARG, LORA_ERR_ID, LORA_ERR_RANK, LORA_ERR_NOMEM, LORA_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
+                    int32_t n_adapters, int64_t d_in, int64_t d_out, lora_stream_t stream,
+                    lora_plan_t *out);
+
+/* Host-only variant of lora_plan_build: the same grouping and tile layout,
+ * but no device buffers (no CUDA call at all). Such a plan can be inspected
+ * with lora_plan_get / lora_plan_info and destroyed; lora_linear_fwd rejects
+ * it with LORA_ERR_ARG. Errors: LORA_ERR_ARG, LORA_ERR_ID, LORA_ERR_RANK,
+ * LORA_ERR_NOMEM. */
+int lora_plan_build_host(const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
+                         int32_t n_adapters, int64_t d_in, int64_t d_out, lora_plan_t *out);
+
+/* Copy the plan's grouping to host memory.
+ *   perm_host   int32[T] or NULL: perm[i] = original index of the token at sorted position i
+ *   seg_host    int32[n_seg*3] or NULL: (adapter, start, length) per segment, ascending
+ *               adapter id, start = first sorted position; adapters without tokens have none
+ *   n_seg       int32* or NULL: number of segments
+ * Errors: LORA_ERR_ARG (null plan). */
+int lora_plan_get(lora_plan_t plan, int32_t *perm_host, int32_t *seg_host, int32_t *n_seg);
+
+typedef struct lora_plan_info {
+    int64_t T, d_in, d_out;
+    int32_t n_adapters;
+    int32_t n_segments;
+    int32_t n_tiles;        /* ceil(T / LORA_TILE_M) */
+    int32_t r_max;          /* largest rank among adapters that own tokens */
+    int64_t sum_r_used;     /* sum of ranks of adapters that own tokens */
+    int64_t sum_r_tokens;   /* sum over tokens of their adapter's rank */
+    int64_t aug_k_total;    /* sum over tiles of the tile's augmented K (multiples of 16) */
+    int64_t scratch_bytes;  /* device scratch owned by the plan */
+} lora_plan_info_t;
+
+/* Errors: LORA_ERR_ARG. */
+int lora_plan_info(lora_plan_t plan, lora_plan_info_t *info);
+
+/* Free the plan (waits for nothing; the caller must not free a plan that queued
+ * work still uses). NULL is ignored. */
+void lora_plan_destroy(lora_plan_t plan);
+
+/* ------------------------------------------------------------------------
+ * lora_linear_fwd — Y = X·W + s_a·((D ⊙ X)·A_a)·B_a for every token.
+ *
+ *   X       bf16 [T, d_in]     tokens in their original order
+ *   W       bf16 [d_in, d_out] frozen base weight
+ *   A_pool  bf16 [R, d_in]     R = sum of all ranks; row off_a + k is column k of A_a
+ *   B_pool  bf16 [R, d_out]    row off_a + k is row k of B_a
+ *   scale   f32  [n_adapters]  DEVICE array of s_a
+ *   p_drop  dropout probability on the LoRA-branch input, in [0, 1); 0 disables.
+ *           Element (t, i) of X (t = original token index) is dropped iff
+ *           h < floor(p_drop * 2^64), where h is output number t*d_in + i
+ *           (0-based) of the SplitMix64 generator seeded with `seed`; kept
+ *           elements are scaled by 1/(1 - p_drop). The base term X·W never sees
+ *           dropout.
+ *   seed    dropout seed
+ *   Y       bf16 [T, d_out]    output, original token order (fp32 accumulation,
+ *           rounded once to bf16)
+ *   U_save  bf16 [T, r_max] or NULL: U[t,k] = ((D ⊙ X)[t]·A_a)[k] for k < r_a,
+ *           zero for k >= r_a (r_max from lora_plan_info); the backward's input
+ *   stream  launch stream
+ * The plan's scratch holds s_a·U rounded to bf16 between the two kernels, so
+ * two forwards with one plan must not run concurrently.
+ * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
+                    const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed,
+                    uint16_t *Y, uint16_t *U_save, lora_stream_t stream);
+
+/* The forward's two phases, for callers that schedule or time them apart
+ * (lora_linear_fwd is exactly lora_linear_shrink followed by lora_fused_gemm
+ * on one stream).
+ *
+ * lora_linear_shrink: U = (D ⊙ X)·A_a for every token, written as s_a·U in
+ * bf16 into the plan's scratch (in the layout the fused GEMM reads) and, if
+ * U_save is not NULL, as U into U_save. Arguments as in lora_linear_fwd.
+ *
+ * lora_fused_gemm: Y = X·W + (s_a·U)·B_a from the plan's scratch, which must
+ * hold the output of a lora_linear_shrink with the same plan that is ordered
+ * before this call on the stream.
+ * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA. */
+int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_pool, const float *scale,
+                       double p_drop, uint64_t seed, uint16_t *U_save, lora_stream_t stream);
+int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *B_pool,
+                    uint16_t *Y, lora_stream_t stream);
+
+/* Y = X·W only (no adapter term), through the same tcgen05 GEMM kernel: the
+ * base-only reference the adapter overhead is measured against.
+ * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA. */
+int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T, int64_t d_in,
+                   int64_t d_out, lora_stream_t stream);
+
+/* ------------------------------------------------------------------------
+ * lora_linear_bwd — backward of the forward for one adapter (fine-tuning;
+ * every token uses it), W frozen so no dW. Plain chain rule:
+ *   dU = s·dY·B^T                       [T, r]
+ *   dB = s·U^T·dY                       [r, d_out]
+ *   dA = ((D ⊙ X)^T·dU)^T, stored [r, d_in] (row k = column k of dA)
+ *   dX = dY·W^T + D ⊙ (dU·A^T)          [T, d_in], D = keep mask / (1 - p)
+ *
+ *   X, W, A (bf16 [r, d_in], rows = columns of A), B (bf16 [r, d_out]),
+ *   scale, p_drop, seed    as in the forward (same mask)
+ *   U_save  bf16 [T, r]    the forward's U_save
+ *   dY      bf16 [T, d_out]
+ *   dX      bf16 [T, d_in]  output
+ *   dA      f32 [r, d_in]   output
+ *   dB      f32 [r, d_out]  output
+ *   workspace, workspace_bytes  device scratch of at least
+ *           lora_linear_bwd_workspace_size(T, d_in, d_out, r) bytes, 256-byte
+ *           aligned, owned by the caller; contents on entry are ignored.
+ * Reductions over tokens use a fixed split and a fixed summation order, so
+ * results are deterministic run to run.
+ * Errors: LORA_ERR_ARG, LORA_ERR_RANK, LORA_ERR_WORKSPACE, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+size_t lora_linear_bwd_workspace_size(int64_t T, int64_t d_in, int64_t d_out, int32_t r);
+
+int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B,
+                    float scale, double p_drop, uint64_t seed, const uint16_t *U_save,
+                    const uint16_t *dY, uint16_t *dX, float *dA, float *dB, int64_t T,
+                    int64_t d_in, int64_t d_out, int32_t r, void *workspace,
+                    size_t workspace_bytes, lora_stream_t stream);
+
+/* Test hook: write the dropout mask the forward and backward use.
+ *   mask_dev  uint8 [T, d_in] device: 1 where X[t, i] is dropped, else 0.
+ * Errors: LORA_ERR_ARG, LORA_ERR_CUDA. */
+int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint8_t *mask_dev,
+                      lora_stream_t stream);
+
+/* Synchronise `stream`, then read and clear the current device's status word.
+ *   status_host  receives the LORA_DEV_* bits (0 if all kernels ran cleanly); may be NULL
+ * Returns LORA_OK if the word was 0, LORA_ERR_DEVICE if any bit was set,
+ * LORA_ERR_CUDA if the synchronisation failed. */
+int lora_device_status(lora_stream_t stream, uint32_t *status_host);
+
+/* Static string for a status code (never NULL). */
+const char *lora_status_string(int code);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* LORA_B200_H */

@@ -1,0 +1,11 @@
+"""B200 (sm_100a) heterogeneous multi-adapter LoRA linear layer.
+
+The compute lives in the in-tree CUDA library ``liblora_b200.so`` behind the C
+ABI declared in ``include/lora.h``; ``lora_adapter_execution_b200.abi`` is a
+thin ctypes binding with the same names (argument marshalling only). There is
+no CPU fallback: if the library is missing, every call raises.
+"""
+
+from . import abi  # noqa: F401
+from .abi import (LoraError, Plan, base_gemm, bwd_workspace_size, device_status, dropout_mask,  # noqa: F401
+                  fused_gemm, linear_bwd, linear_fwd, linear_shrink, load_library)

@@ -1,0 +1,212 @@
+"""ctypes binding of include/lora.h (argument marshalling only).
+
+Tensors are torch CUDA tensors (bf16 where the ABI says bf16); each call passes
+their raw device pointers and the current torch stream to the library. Nothing
+here computes any part of the layer.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import os
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "liblora_b200.so")
+
+LORA_OK = 0
+STATUS_NAMES = {0: "LORA_OK", -1: "LORA_ERR_ARG", -2: "LORA_ERR_ID", -3: "LORA_ERR_RANK",
+                -4: "LORA_ERR_CUDA", -5: "LORA_ERR_DEVICE", -6: "LORA_ERR_UNSUPPORTED",
+                -7: "LORA_ERR_NOMEM", -8: "LORA_ERR_WORKSPACE"}
+
+_vp = ctypes.c_void_p
+_i32 = ctypes.c_int32
+_i64 = ctypes.c_int64
+_u64 = ctypes.c_uint64
+_dbl = ctypes.c_double
+_f32 = ctypes.c_float
+_sz = ctypes.c_size_t
+
+
+class LoraError(RuntimeError):
+    def __init__(self, code: int, what: str):
+        self.code = code
+        super().__init__(f"{what}: {STATUS_NAMES.get(code, code)} ({_lib_or_none_str(code)})")
+
+
+class _Info(ctypes.Structure):
+    _fields_ = [("T", _i64), ("d_in", _i64), ("d_out", _i64), ("n_adapters", _i32),
+                ("n_segments", _i32), ("n_tiles", _i32), ("r_max", _i32), ("sum_r_used", _i64),
+                ("sum_r_tokens", _i64), ("aug_k_total", _i64), ("scratch_bytes", _i64)]
+
+
+_lib = None
+
+
+def _lib_or_none_str(code):
+    try:
+        return load_library().lora_status_string(code).decode()
+    except Exception:  # pragma: no cover
+        return "?"
+
+
+def load_library():
+    """Load liblora_b200.so; raises if it has not been built (no fallback)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"CUDA library not built: {LIB_PATH} (run python -m lora_adapter_execution_b200.build)")
+    L = ctypes.CDLL(LIB_PATH)
+    sig = {
+        "lora_plan_build": (ctypes.c_int, [_vp, _i64, _vp, _i32, _i64, _i64, _vp, ctypes.POINTER(_vp)]),
+        "lora_plan_build_host": (ctypes.c_int, [_vp, _i64, _vp, _i32, _i64, _i64, ctypes.POINTER(_vp)]),
+        "lora_plan_get": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
+        "lora_plan_info": (ctypes.c_int, [_vp, ctypes.POINTER(_Info)]),
+        "lora_plan_destroy": (None, [_vp]),
+        "lora_linear_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp]),
+        "lora_linear_shrink": (ctypes.c_int, [_vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp]),
+        "lora_fused_gemm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
+        "lora_base_gemm": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp]),
+        "lora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
+        "lora_linear_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _f32, _dbl, _u64, _vp, _vp, _vp, _vp, _vp,
+                                           _i64, _i64, _i64, _i32, _vp, _sz, _vp]),
+        "lora_dropout_mask": (ctypes.c_int, [_u64, _dbl, _i64, _i64, _vp, _vp]),
+        "lora_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+        "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(L, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = L
+    return L
+
+
+def _check(rc: int, what: str):
+    if rc != LORA_OK:
+        raise LoraError(rc, what)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    if stream is None:
+        import torch
+        return ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    if isinstance(stream, int):
+        return ctypes.c_void_p(stream)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _host_i32(a):
+    a = a.cpu().numpy() if hasattr(a, "cpu") else a
+    return np.ascontiguousarray(a, dtype=np.int32)
+
+
+class Plan:
+    """A batch's token-by-adapter grouping (lora_plan_build / lora_plan_build_host)."""
+
+    def __init__(self, ids, ranks, d_in: int, d_out: int, *, stream=None, host_only: bool = False):
+        L = load_library()
+        self._ids = _host_i32(ids)
+        self._ranks = _host_i32(ranks)
+        h = _vp()
+        T, n = self._ids.shape[0], self._ranks.shape[0]
+        if host_only:
+            rc = L.lora_plan_build_host(self._ids.ctypes.data_as(_vp), T, self._ranks.ctypes.data_as(_vp), n,
+                                        d_in, d_out, ctypes.byref(h))
+        else:
+            rc = L.lora_plan_build(self._ids.ctypes.data_as(_vp), T, self._ranks.ctypes.data_as(_vp), n,
+                                   d_in, d_out, _stream(stream), ctypes.byref(h))
+        _check(rc, "lora_plan_build")
+        self._h = h
+        self.T, self.d_in, self.d_out, self.n_adapters = T, d_in, d_out, n
+
+    @property
+    def handle(self):
+        return self._h
+
+    def info(self) -> dict:
+        inf = _Info()
+        _check(load_library().lora_plan_info(self._h, ctypes.byref(inf)), "lora_plan_info")
+        return {f: getattr(inf, f) for f, _ in _Info._fields_}
+
+    def grouping(self):
+        L = load_library()
+        ns = _i32(0)
+        _check(L.lora_plan_get(self._h, None, None, ctypes.byref(ns)), "lora_plan_get")
+        perm = np.empty(self.T, dtype=np.int32)
+        seg = np.empty((max(ns.value, 1), 3), dtype=np.int32)
+        _check(L.lora_plan_get(self._h, perm.ctypes.data_as(_vp), seg.ctypes.data_as(_vp), None), "lora_plan_get")
+        return perm, seg[: ns.value].copy()
+
+    def destroy(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            load_library().lora_plan_destroy(self._h)
+            self._h = _vp()
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass
+
+
+def linear_fwd(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.0, seed: int = 0,
+               U_save=None, stream=None):
+    _check(load_library().lora_linear_fwd(plan.handle, _ptr(X), _ptr(W), _ptr(A_pool), _ptr(B_pool), _ptr(scale),
+                                          float(p_drop), int(seed) & (2**64 - 1), _ptr(Y), _ptr(U_save),
+                                          _stream(stream)), "lora_linear_fwd")
+
+
+def linear_shrink(plan: Plan, X, A_pool, scale, *, p_drop: float = 0.0, seed: int = 0, U_save=None, stream=None):
+    _check(load_library().lora_linear_shrink(plan.handle, _ptr(X), _ptr(A_pool), _ptr(scale), float(p_drop),
+                                             int(seed) & (2**64 - 1), _ptr(U_save), _stream(stream)),
+           "lora_linear_shrink")
+
+
+def fused_gemm(plan: Plan, X, W, B_pool, Y, *, stream=None):
+    _check(load_library().lora_fused_gemm(plan.handle, _ptr(X), _ptr(W), _ptr(B_pool), _ptr(Y), _stream(stream)),
+           "lora_fused_gemm")
+
+
+def base_gemm(X, W, Y, *, stream=None):
+    T, d_in = X.shape
+    d_out = W.shape[1]
+    _check(load_library().lora_base_gemm(_ptr(X), _ptr(W), _ptr(Y), T, d_in, d_out, _stream(stream)),
+           "lora_base_gemm")
+
+
+def bwd_workspace_size(T: int, d_in: int, d_out: int, r: int) -> int:
+    return int(load_library().lora_linear_bwd_workspace_size(T, d_in, d_out, r))
+
+
+def linear_bwd(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, workspace, *, p_drop: float = 0.0,
+               seed: int = 0, stream=None):
+    T, d_in = X.shape
+    d_out = W.shape[1]
+    r = A.shape[0]
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load_library().lora_linear_bwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), float(scale), float(p_drop),
+                                          int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY), _ptr(dX), _ptr(dA),
+                                          _ptr(dB), T, d_in, d_out, r, _ptr(workspace), nbytes, _stream(stream)),
+           "lora_linear_bwd")
+
+
+def dropout_mask(seed: int, p_drop: float, mask, *, stream=None):
+    T, d_in = mask.shape
+    _check(load_library().lora_dropout_mask(int(seed) & (2**64 - 1), float(p_drop), T, d_in, _ptr(mask),
+                                            _stream(stream)), "lora_dropout_mask")
+
+
+def device_status(stream=None) -> int:
+    """Synchronise the stream and return (and clear) the device status word."""
+    v = ctypes.c_uint32(0)
+    rc = load_library().lora_device_status(_stream(stream), ctypes.byref(v))
+    if rc not in (LORA_OK, -5):
+        raise LoraError(rc, "lora_device_status")
+    return int(v.value)

@@ -1,0 +1,65 @@
+// Host/device shared layout of a plan. Plain structs only (no CUDA types), so the
+// host planner (plan.cpp, g++) and the kernels (lora_b200.cu, nvcc) agree on it.
+#pragma once
+
+#include <stdint.h>
+
+#include <vector>
+
+namespace lora {
+
+constexpr int kTileM = 128;      // tokens per fused-GEMM output tile
+constexpr int kAugBlock = 64;    // augmented-K columns per shrink-output block
+constexpr int kAugBlockBytes = kTileM * kAugBlock * 2;  // 16 KB, one swizzled smem image
+constexpr int kShrinkN = 64;     // rank columns per shrink work unit
+
+// One 128-token output tile of the sorted order.
+struct TileDesc {
+  int32_t row0;    // first sorted position
+  int32_t rows;    // valid rows (<= 128)
+  int32_t chunk0;  // first ChunkDesc of this tile
+  int32_t nchunk;  // adapters touching the tile
+  int32_t kaug;    // augmented K = sum of the chunks' kc (multiple of 16)
+  int32_t contig;  // original index of row 0 if the tile's tokens are consecutive originals, else -1
+  int64_t uofs;    // byte offset of the tile's s*U image in the plan scratch
+};
+
+// One adapter's run of rows inside one tile: its K slice of the augmented contraction.
+struct ChunkDesc {
+  int32_t adapter;
+  int32_t pool_row;  // off_a: first row of the adapter in A_pool / B_pool
+  int32_t rank;      // r_a
+  int32_t kc;        // r_a rounded up to 16 (MMA K step)
+  int32_t kofs;      // first augmented-K column of the chunk within its tile
+  int32_t lo, hi;    // tile-local rows [lo, hi) owned by the adapter
+  int32_t tile;
+};
+
+// Shrink work unit: rank columns [n0, n0+nn) of one chunk.
+struct UnitDesc {
+  int32_t chunk;
+  int32_t n0;
+  int32_t nn;
+  int32_t last;  // 1 if this is the chunk's last piece (it also zero-fills U_save up to r_max)
+};
+
+struct HostPlan {
+  int64_t T = 0, d_in = 0, d_out = 0;
+  int32_t n_adapters = 0;
+  std::vector<int32_t> perm;     // sorted position -> original token
+  std::vector<int32_t> seg;      // n_seg x 3: adapter, start, length
+  std::vector<int64_t> offsets;  // n_adapters + 1
+  std::vector<TileDesc> tiles;
+  std::vector<ChunkDesc> chunks;
+  std::vector<UnitDesc> units;
+  int32_t r_max = 0;
+  int64_t sum_r_used = 0, sum_r_tokens = 0, aug_k_total = 0;
+  int64_t scratch_bytes = 0;
+  int32_t max_chunk_rows = 0;
+};
+
+// Returns LORA_OK or a LORA_ERR_* code; fills `hp` on success.
+int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t n_adapters,
+                    int64_t d_in, int64_t d_out, HostPlan &hp);
+
+}  // namespace lora

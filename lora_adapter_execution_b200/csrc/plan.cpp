@@ -1,0 +1,122 @@
+// Host planner: group a batch's tokens by adapter and lay out the fused GEMM's
+// augmented-K work.
+//
+// Grouping requests by adapter so the base GEMM runs batched while each
+// adapter's xAB is computed for its own tokens without padding follows the
+// batching section (批处理) of "S-LoRA：一个GPU运行数千大模型成为可能"; the
+// rank-exact pool offsets follow its Unified Paging section (a rank-R weight
+// occupies R vectors). Building the grouping once per batch and reusing it in
+// every layer follows the decide-once framework (整体框架) of "AdaFuse:
+// Accelerating Dynamic Adapter Inference via Token-Level Pre-Gating and Fused
+// Kernel Optimization".
+#include <algorithm>
+
+#include "../../include/lora.h"
+#include "internal.h"
+
+namespace lora {
+
+int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t n_adapters,
+                    int64_t d_in, int64_t d_out, HostPlan &hp) {
+  if (!ids || !ranks || T <= 0 || n_adapters <= 0 || d_in < 8 || d_out < 8 || (d_in % 8) ||
+      (d_out % 8))
+    return LORA_ERR_ARG;
+  if (T > (int64_t)1 << 30 || d_in > (int64_t)1 << 30 || d_out > (int64_t)1 << 30)
+    return LORA_ERR_ARG;
+  for (int32_t a = 0; a < n_adapters; ++a)
+    if (ranks[a] < 1 || ranks[a] > LORA_MAX_RANK) return LORA_ERR_RANK;
+  for (int64_t t = 0; t < T; ++t)
+    if (ids[t] < 0 || ids[t] >= n_adapters) return LORA_ERR_ID;
+
+  hp = HostPlan();
+  hp.T = T;
+  hp.d_in = d_in;
+  hp.d_out = d_out;
+  hp.n_adapters = n_adapters;
+
+  hp.offsets.assign(n_adapters + 1, 0);
+  for (int32_t a = 0; a < n_adapters; ++a) hp.offsets[a + 1] = hp.offsets[a] + ranks[a];
+  if (hp.offsets[n_adapters] >= ((int64_t)1 << 31) - 256) return LORA_ERR_ARG;
+
+  // Stable counting sort by adapter id.
+  std::vector<int64_t> count(n_adapters + 1, 0);
+  for (int64_t t = 0; t < T; ++t) ++count[ids[t] + 1];
+  for (int32_t a = 0; a < n_adapters; ++a) count[a + 1] += count[a];  // count[a] = start of a
+  std::vector<int64_t> cursor(count.begin(), count.end() - 1);
+  hp.perm.assign(T, 0);
+  for (int64_t t = 0; t < T; ++t) hp.perm[cursor[ids[t]]++] = (int32_t)t;
+
+  // Segments, ascending adapter id, adapters without tokens skipped.
+  for (int32_t a = 0; a < n_adapters; ++a) {
+    int64_t len = count[a + 1] - count[a];
+    if (len == 0) continue;
+    hp.seg.push_back(a);
+    hp.seg.push_back((int32_t)count[a]);
+    hp.seg.push_back((int32_t)len);
+    hp.r_max = std::max(hp.r_max, ranks[a]);
+    hp.sum_r_used += ranks[a];
+    hp.sum_r_tokens += (int64_t)ranks[a] * len;
+  }
+  const int32_t n_seg = (int32_t)(hp.seg.size() / 3);
+
+  // Tiles of 128 sorted positions; each adapter run inside a tile is a chunk
+  // whose K slice is the adapter's rank rounded up to the 16-wide MMA step.
+  const int64_t n_tiles = (T + kTileM - 1) / kTileM;
+  int32_t s = 0;  // current segment
+  int64_t uofs = 0;
+  for (int64_t m = 0; m < n_tiles; ++m) {
+    TileDesc td{};
+    td.row0 = (int32_t)(m * kTileM);
+    td.rows = (int32_t)std::min<int64_t>(kTileM, T - m * kTileM);
+    td.chunk0 = (int32_t)hp.chunks.size();
+    int32_t kofs = 0;
+    const int64_t r_end = td.row0 + td.rows;
+    while (s < n_seg && hp.seg[3 * s + 1] < r_end) {
+      const int32_t a = hp.seg[3 * s + 0];
+      const int64_t s_beg = hp.seg[3 * s + 1];
+      const int64_t s_end = s_beg + hp.seg[3 * s + 2];
+      ChunkDesc cd{};
+      cd.adapter = a;
+      cd.pool_row = (int32_t)hp.offsets[a];
+      cd.rank = ranks[a];
+      cd.kc = (ranks[a] + 15) / 16 * 16;
+      cd.kofs = kofs;
+      cd.lo = (int32_t)(std::max<int64_t>(s_beg, td.row0) - td.row0);
+      cd.hi = (int32_t)(std::min<int64_t>(s_end, r_end) - td.row0);
+      cd.tile = (int32_t)m;
+      kofs += cd.kc;
+      hp.max_chunk_rows = std::max(hp.max_chunk_rows, cd.hi - cd.lo);
+      hp.chunks.push_back(cd);
+      if (s_end <= r_end) ++s;  // segment finished inside this tile
+      else break;               // segment continues into the next tile
+    }
+    td.nchunk = (int32_t)hp.chunks.size() - td.chunk0;
+    td.kaug = kofs;
+    // consecutive originals?
+    bool contig = true;
+    for (int32_t i = 1; i < td.rows && contig; ++i)
+      contig = hp.perm[td.row0 + i] == hp.perm[td.row0] + i;
+    td.contig = contig ? hp.perm[td.row0] : -1;
+    td.uofs = uofs;
+    uofs += (int64_t)((td.kaug + kAugBlock - 1) / kAugBlock) * kAugBlockBytes;
+    hp.aug_k_total += td.kaug;
+    hp.tiles.push_back(td);
+  }
+  hp.scratch_bytes = uofs;
+
+  // Shrink units: each chunk's rank columns in pieces of at most 64.
+  for (int32_t c = 0; c < (int32_t)hp.chunks.size(); ++c) {
+    const ChunkDesc &cd = hp.chunks[c];
+    for (int32_t n0 = 0; n0 < cd.kc; n0 += kShrinkN) {
+      UnitDesc u{};
+      u.chunk = c;
+      u.n0 = n0;
+      u.nn = std::min(kShrinkN, cd.kc - n0);
+      u.last = (n0 + kShrinkN >= cd.kc) ? 1 : 0;
+      hp.units.push_back(u);
+    }
+  }
+  return LORA_OK;
+}
+
+}  // namespace lora

@@ -1,0 +1,559 @@
+// Skinny contractions around the fused GEMM, all memory-bound: the rank
+// dimension r_a is 1..256 against d_in, d_out in the thousands.
+//
+//  * lora_shrink_kernel: U[t, k] = sum_i In[t, i] * F[k, i] over the rows of one
+//    adapter run (forward: In = X with the dropout mask, F = A_pool rows of the
+//    adapter; backward: In = dY, F = B rows). Each X tile is read once through
+//    TMA into shared memory; warp-level MMA (mma.sync m16n8k16, bf16 -> fp32)
+//    works on the skinny rank dimension. The d_in contraction is split across
+//    the CTAs of a thread-block cluster and summed through distributed shared
+//    memory, so a small adapter run still spreads its bytes over several SMs.
+//    Forward output: the tile's s·U block, already in the 128-byte-swizzled
+//    shared-memory image the fused GEMM's MMA reads, plus U for the backward.
+//  * lora_tcontract_kernel: partial[q][k][n] = sum_{t in split q} G[t, k] * In[t, n]
+//    (dB with G = U, In = dY; dA with G = dU, In = masked X), fixed token splits.
+//  * lora_reduce_splits_kernel: sums the splits in a fixed order (deterministic).
+//  * lora_mask_kernel: the dropout mask itself (test hook).
+//
+// Where the LoRA shrink sits in the layer: the X·A product of the LoRA branch
+// next to the frozen base GEMM, "LoRAFusion：消除冗余内存访问的多 LoRA 高效微调系统",
+// 解决什么真问题, item 1; dropout of the branch input is one of the small ops
+// listed there.
+#pragma once
+
+#include "common.cuh"
+#include "internal.h"
+
+namespace lora {
+
+constexpr int kSkConsumerWarps = 8;
+constexpr int kSkThreads = (kSkConsumerWarps + 1) * 32;  // + 1 producer warp
+constexpr int kSkBK = 64;                                 // columns per stage (one 128-byte swizzled row)
+constexpr int kSkPool = 72 * 1024;                        // stage ring (also the reduction scratch)
+constexpr int kSkMaxStages = 16;
+constexpr int kSkFinBytes = kTileM * kShrinkN * 4;        // CTA partial [128 x 64] fp32
+constexpr int kSkSmem = 1024 + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64;
+
+struct ShrinkParams {
+  int32_t mode;     // 0: forward shrink over plan units; 1: backward dU over consecutive tiles
+  int32_t T, K;     // tokens, contraction length
+  int32_t ksplit;   // cluster size along the contraction
+  int32_t kslice;   // contraction columns per cluster rank (multiple of kSkBK)
+  // forward
+  const UnitDesc *units;
+  const ChunkDesc *chunks;
+  const TileDesc *tiles;
+  const int32_t *perm;
+  const float *scale;
+  uint64_t seed, thr;
+  float inv_keep;
+  uint8_t *uimg;
+  __nv_bfloat16 *U_save;
+  int32_t r_max;
+  // backward
+  int32_t r;
+  int32_t npieces;
+  float scale1;
+  float *dU;                 // [T, r] fp32
+  __nv_bfloat16 *dU_bf16;    // [T, r]
+};
+
+struct UnitGeom {
+  int32_t rows;      // valid rows (<= 128)
+  int32_t row0;      // first sorted position (forward) or first token (backward)
+  int32_t contig;    // original index of the first row if rows are consecutive originals, else -1
+  int32_t frow;      // first F row of the piece
+  int32_t nn;        // piece width (multiple of 16, <= 64)
+  int32_t nvalid;    // columns of the piece that are real ranks (rest are zero)
+  // forward only
+  int32_t tile, lo, kcol, adapter, n0, last;
+};
+
+__device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
+  UnitGeom g;
+  if (p.mode == 0) {
+    const UnitDesc ud = p.units[u];
+    const ChunkDesc cd = p.chunks[ud.chunk];
+    const TileDesc td = p.tiles[cd.tile];
+    g.rows = cd.hi - cd.lo;
+    g.row0 = td.row0 + cd.lo;
+    g.contig = td.contig >= 0 ? td.contig + cd.lo : -1;
+    g.frow = cd.pool_row + ud.n0;
+    g.nn = ud.nn;
+    g.nvalid = max(0, min(ud.nn, cd.rank - ud.n0));
+    g.tile = cd.tile;
+    g.lo = cd.lo;
+    g.kcol = cd.kofs + ud.n0;
+    g.adapter = cd.adapter;
+    g.n0 = ud.n0;
+    g.last = ud.last;
+  } else {
+    const int m = u / p.npieces;
+    const int piece = u % p.npieces;
+    g.rows = min(kTileM, p.T - m * kTileM);
+    g.row0 = m * kTileM;
+    g.contig = g.row0;
+    g.n0 = piece * kShrinkN;
+    g.nn = min(kShrinkN, ((p.r + 15) / 16) * 16 - g.n0);
+    g.frow = g.n0;
+    g.nvalid = max(0, min(g.nn, p.r - g.n0));
+    g.tile = m;
+    g.lo = 0;
+    g.kcol = 0;
+    g.adapter = 0;
+    g.last = 0;
+  }
+  return g;
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                        uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t &r0, uint32_t &r1, uint32_t &r2,
+                                          uint32_t &r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0,%1,%2,%3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void mma_bf16_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+      "{%0,%1,%2,%3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+// zero the bf16 halves of a packed pair whose mask bit says "dropped"
+__device__ __forceinline__ uint32_t mask_pair(uint32_t v, bool keep_lo, bool keep_hi) {
+  return (keep_lo ? (v & 0xFFFFu) : 0u) | (keep_hi ? (v & 0xFFFF0000u) : 0u);
+}
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_sync_all() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                   : "memory");
+}
+__device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
+  float v;
+  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+  return v;
+}
+
+// Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
+// its rank q contracts columns [q*kslice, (q+1)*kslice).
+__global__ void __launch_bounds__(kSkThreads, 1)
+    lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows, box {64, 16}
+                       const __grid_constant__ CUtensorMap mapInG,   // In rows, box {64, 1} (gather4)
+                       const __grid_constant__ CUtensorMap mapF16,   // F rows, box {64, 16}
+                       const ShrinkParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const uint32_t pool = smem_u32(smem);
+  float *fin = reinterpret_cast<float *>(smem + kSkPool);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSkPool + kSkFinBytes);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * kSkMaxStages;
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kSkMaxStages);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int unit = blockIdx.x / p.ksplit;
+  const uint32_t crank = cluster_ctarank();
+  const UnitGeom g = unit_geom(p, unit);
+
+  const int Rp = ((g.rows + 15) / 16) * 16;  // rows rounded to the MMA M step
+  const int mb = Rp / 16;
+  const int stage_bytes = (Rp + g.nn) * 128;  // X rows then F rows, 128 B (64 bf16) each
+  const int nstage = min(kSkMaxStages, kSkPool / stage_bytes);
+  const int kbeg = static_cast<int>(crank) * p.kslice;
+  const int kend = min(p.K, kbeg + p.kslice);
+  const int nblk = kend > kbeg ? (kend - kbeg + kSkBK - 1) / kSkBK : 0;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < nstage; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, kSkConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  // warp work split: MW warps along rows (m-blocks), KW along the k16 steps of a stage
+  int MW = 1;
+  while (MW * 2 <= mb && MW < kSkConsumerWarps) MW *= 2;
+  const int KW = kSkConsumerWarps / MW;
+  const int nb8 = g.nn / 8;
+
+  float acc[2][8][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+
+  if (warp == kSkConsumerWarps) {
+    // -------------------------------------------------------------- producer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int b = 0; b < nblk; ++b) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
+        const uint32_t fb = full0 + 8 * stage;
+        mbar_arrive_expect_tx(fb, stage_bytes);
+        const uint32_t xb = pool + stage * stage_bytes;
+        const uint32_t fbuf = xb + Rp * 128;
+        const int col = kbeg + b * kSkBK;
+        if (g.contig >= 0) {
+          for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, g.contig + r16);
+        } else {
+          for (int r4 = 0; r4 < Rp; r4 += 4) {
+            int rr[4];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) rr[j] = p.perm[g.row0 + min(r4 + j, g.rows - 1)];
+            tma_gather4(xb + r4 * 128, &mapInG, fb, col, rr[0], rr[1], rr[2], rr[3]);
+          }
+        }
+        for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
+        if (++stage == nstage) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- consumers
+    const int mphase = warp % MW;
+    const int kphase = warp / MW;
+    // original token index of the two rows this lane's fragments touch, per m-block slot
+    int64_t orow[2][2];
+#pragma unroll
+    for (int i = 0; i < 2; ++i)
+#pragma unroll
+      for (int h = 0; h < 2; ++h) {
+        const int r = (mphase + i * MW) * 16 + (lane >> 2) + 8 * h;
+        const int rc = min(r, g.rows - 1);
+        orow[i][h] = g.contig >= 0 ? static_cast<int64_t>(g.contig + rc)
+                                   : (p.mode == 0 ? static_cast<int64_t>(p.perm[g.row0 + rc]) : 0);
+      }
+    const bool masked = p.mode == 0 && p.thr != 0;
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int b = 0; b < nblk; ++b) {
+      if (!mbar_wait(full0 + 8 * stage, phase)) { *abort_flag = 1; break; }
+      const uint32_t xb = pool + stage * stage_bytes;
+      const uint32_t fbuf = xb + Rp * 128;
+      for (int ks = kphase; ks < 4; ks += KW) {  // k16 steps of the stage
+        const int colbase = kbeg + b * kSkBK + ks * 16;
+#pragma unroll
+        for (int i = 0; i < 2; ++i) {
+          const int mblk = mphase + i * MW;
+          if (mblk >= mb) break;
+          uint32_t a0, a1, a2, a3;
+          {
+            const int mi = lane >> 3;
+            const int r = mblk * 16 + (mi & 1) * 8 + (lane & 7);
+            const int chunk = ks * 2 + (mi >> 1);
+            ldsm_x4(xb + r * 128 + (((chunk ^ (r & 7)) & 7) << 4), a0, a1, a2, a3);
+          }
+          if (masked) {
+            const int c0 = colbase + 2 * (lane & 3);
+            a0 = mask_pair(a0, keep_elem(p.seed, p.thr, orow[i][0], c0, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 1, p.K));
+            a1 = mask_pair(a1, keep_elem(p.seed, p.thr, orow[i][1], c0, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 1, p.K));
+            a2 = mask_pair(a2, keep_elem(p.seed, p.thr, orow[i][0], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 9, p.K));
+            a3 = mask_pair(a3, keep_elem(p.seed, p.thr, orow[i][1], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 9, p.K));
+          }
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            if (2 * jj >= nb8) break;
+            uint32_t b0, b1, b2, b3;
+            const int mi = lane >> 3;
+            const int nr = jj * 16 + (mi >> 1) * 8 + (lane & 7);
+            const int chunk = ks * 2 + (mi & 1);
+            ldsm_x4(fbuf + nr * 128 + (((chunk ^ (nr & 7)) & 7) << 4), b0, b1, b2, b3);
+            mma_bf16_16816(acc[i][2 * jj], a0, a1, a2, a3, b0, b1);
+            mma_bf16_16816(acc[i][2 * jj + 1], a0, a1, a2, a3, b2, b3);
+          }
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+      if (++stage == nstage) { stage = 0; phase ^= 1; }
+    }
+  }
+  __syncthreads();  // every TMA landed and was consumed: the pool is free for the reduction
+
+  // ---------------------------------------------------------------- CTA reduction
+  // red[w][slot*16 + row][col], fp32, in the (now idle) stage pool
+  float *red = reinterpret_cast<float *>(smem);
+  if (warp < kSkConsumerWarps) {
+    const int mphase = warp % MW;
+#pragma unroll
+    for (int i = 0; i < 2; ++i) {
+      const int mblk = mphase + i * MW;
+      if (mblk >= mb) break;
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        if (j >= nb8) break;
+        const int r = i * 16 + (lane >> 2);
+        const int c = j * 8 + 2 * (lane & 3);
+        float *base = red + (warp * 32) * kShrinkN;
+        base[r * kShrinkN + c] = acc[i][j][0];
+        base[r * kShrinkN + c + 1] = acc[i][j][1];
+        base[(r + 8) * kShrinkN + c] = acc[i][j][2];
+        base[(r + 8) * kShrinkN + c + 1] = acc[i][j][3];
+      }
+    }
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < Rp * g.nn; e += blockDim.x) {
+    const int r = e / g.nn, c = e % g.nn;
+    const int mblk = r / 16;
+    const int mphase = mblk % MW;
+    const int slot = mblk / MW;
+    float s = 0.f;
+    for (int kp = 0; kp < KW; ++kp) {
+      const int w = kp * MW + mphase;
+      s += red[(w * 32 + slot * 16 + (r & 15)) * kShrinkN + c];
+    }
+    fin[r * kShrinkN + c] = s;
+  }
+  cluster_sync_all();  // every rank's fin is final
+
+  if (crank == 0) {
+    if (p.ksplit > 1) {
+      for (int e = threadIdx.x; e < Rp * g.nn; e += blockDim.x) {
+        const int r = e / g.nn, c = e % g.nn;
+        const uint32_t la = smem_u32(fin + r * kShrinkN + c);
+        float s = fin[r * kShrinkN + c];
+        for (uint32_t q = 1; q < static_cast<uint32_t>(p.ksplit); ++q) s += ld_dsmem_f32(map_to_rank(la, q));
+        fin[r * kShrinkN + c] = s;
+      }
+    }
+    // the peers only read their own fin below this point; rank 0 owns fin now
+  }
+  cluster_sync_all();  // peers may exit only after rank 0 has read their fin
+
+  if (crank == 0) {
+    if (p.mode == 0) {
+      const float s_a = p.scale[g.adapter] * p.inv_keep;
+      // s·U block of the tile: all 128 rows of columns [kcol, kcol + nn)
+      uint8_t *img = p.uimg + p.tiles[g.tile].uofs;
+      for (int e = threadIdx.x; e < kTileM * (g.nn / 8); e += blockDim.x) {
+        const int row = e / (g.nn / 8);
+        const int c8 = (e % (g.nn / 8)) * 8;
+        const int lr = row - g.lo;
+        const bool mine = lr >= 0 && lr < g.rows;
+        uint32_t w[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float v0 = 0.f, v1 = 0.f;
+          if (mine) {
+            if (c8 + 2 * j < g.nvalid) v0 = fin[lr * kShrinkN + c8 + 2 * j] * s_a;
+            if (c8 + 2 * j + 1 < g.nvalid) v1 = fin[lr * kShrinkN + c8 + 2 * j + 1] * s_a;
+          }
+          w[j] = pack_bf16x2(v0, v1);
+        }
+        const int col = g.kcol + c8;
+        uint8_t *dst = img + (col / kAugBlock) * kAugBlockBytes + sw128_offset(row, col % kAugBlock);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+      }
+      if (p.U_save) {
+        const int cend = g.last ? p.r_max : min(p.r_max, g.n0 + g.nn);
+        const int ncol = max(0, cend - g.n0);
+        for (int e = threadIdx.x; e < g.rows * ncol; e += blockDim.x) {
+          const int lr = e / ncol, c = e % ncol;
+          const int64_t orig = g.contig >= 0 ? g.contig + lr : p.perm[g.row0 + lr];
+          const float v = c < g.nvalid ? fin[lr * kShrinkN + c] * p.inv_keep : 0.f;
+          p.U_save[orig * p.r_max + g.n0 + c] = __float2bfloat16_rn(v);
+        }
+      }
+    } else {
+      for (int e = threadIdx.x; e < g.rows * g.nvalid; e += blockDim.x) {
+        const int lr = e / g.nvalid, c = e % g.nvalid;
+        const int64_t t = g.row0 + lr;
+        const float v = fin[lr * kShrinkN + c] * p.scale1;
+        p.dU[t * p.r + g.n0 + c] = v;
+        p.dU_bf16[t * p.r + g.n0 + c] = __float2bfloat16_rn(v);
+      }
+    }
+  }
+}
+
+// ------------------------------------------------------------------ token contraction
+constexpr int kTcThreads = 288;   // 8 consumer warps + producer warp
+constexpr int kTcStages = 6;
+constexpr int kTcTok = 64;        // tokens per stage
+constexpr int kTcCols = 128;      // columns per CTA
+constexpr int kTcMaxR = 64;
+
+struct TcParams {
+  int32_t T, N, r;
+  int32_t splits, tsplit;  // token splits, tokens per split (multiple of 64)
+  uint64_t seed, thr;      // mask on In (dA); thr = 0 for none
+  float *partial;          // [splits][r][N]
+};
+
+// partial[q][k][n] = sum_{t in split q} G[t, k] * In[t, n] (In masked if thr != 0).
+// Grid (N / 128, splits).
+__global__ void __launch_bounds__(kTcThreads, 1)
+    lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N], box {64, 64}, swizzle 128B
+                          const __grid_constant__ CUtensorMap mapG,   // G [T, r], box {r, 64}, no swizzle
+                          const TcParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  const int in_bytes = kTcTok * kTcCols * 2;    // 16 KB (two 8 KB halves)
+  const int g_bytes = kTcTok * p.r * 2;         // <= 8 KB
+  const int g_pad = ((g_bytes + 1023) & ~1023) + 1024;  // slack: rank-8 fragments read one row past
+  const int stage_bytes = in_bytes + g_pad;
+  const uint32_t pool = smem_u32(smem);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kTcStages * stage_bytes);
+  const uint32_t full0 = smem_u32(bars);
+  const uint32_t empty0 = full0 + 8 * kTcStages;
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int n0 = blockIdx.x * kTcCols;
+  const int t0 = blockIdx.y * p.tsplit;
+  const int t1 = min(p.T, t0 + p.tsplit);
+  const int nblk = t1 > t0 ? (t1 - t0 + kTcTok - 1) / kTcTok : 0;
+  const int mblocks = (p.r + 15) / 16;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kTcStages; ++s) {
+      mbar_init(full0 + 8 * s, 1);
+      mbar_init(empty0 + 8 * s, 8);
+    }
+    fence_mbar_init();
+  }
+  __syncthreads();
+
+  float acc[4][2][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 2; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+
+  if (warp == 8) {
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int b = 0; b < nblk; ++b) {
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) break;
+        const uint32_t fb = full0 + 8 * stage;
+        const uint32_t sb = pool + stage * stage_bytes;
+        const int t = t0 + b * kTcTok;
+        mbar_arrive_expect_tx(fb, in_bytes + g_bytes);
+        tma_load_2d(sb, &mapIn, fb, n0, t);
+        tma_load_2d(sb + 8192, &mapIn, fb, n0 + 64, t);
+        tma_load_2d(sb + in_bytes, &mapG, fb, 0, t);
+        if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+      }
+    }
+  } else {
+    // warp w owns columns [16w, 16w + 16) of the CTA's 128
+    const int cw = warp * 16;
+    const int h = cw / 64;        // which 64-column half
+    const int cin = cw % 64;      // column offset inside the half
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int b = 0; b < nblk; ++b) {
+      if (!mbar_wait(full0 + 8 * stage, phase)) break;
+      const uint32_t sb = pool + stage * stage_bytes;
+      const uint32_t inb = sb + h * 8192;
+      const uint32_t gb = sb + in_bytes;
+      const int tbase = t0 + b * kTcTok;
+#pragma unroll
+      for (int ks = 0; ks < kTcTok / 16; ++ks) {
+        // B fragments (tokens x columns) for the warp's two n8 blocks
+        uint32_t b0, b1, b2, b3;
+        {
+          const int mi = lane >> 3;
+          const int tr = ks * 16 + (mi & 1) * 8 + (lane & 7);
+          const int chunk = (cin >> 3) + (mi >> 1);
+          ldsm_x4_t(inb + tr * 128 + (((chunk ^ (tr & 7)) & 7) << 4), b0, b1, b2, b3);
+        }
+        if (p.thr != 0) {
+          // b0: tokens ks*16 + 2*(lane&3) + {0,1}, column cw + lane/4; b1: tokens + 8;
+          // b2, b3: column + 8
+          const int tk = tbase + ks * 16 + 2 * (lane & 3);
+          const int c = n0 + cw + (lane >> 2);
+          b0 = mask_pair(b0, keep_elem(p.seed, p.thr, tk, c, p.N), keep_elem(p.seed, p.thr, tk + 1, c, p.N));
+          b1 = mask_pair(b1, keep_elem(p.seed, p.thr, tk + 8, c, p.N), keep_elem(p.seed, p.thr, tk + 9, c, p.N));
+          b2 = mask_pair(b2, keep_elem(p.seed, p.thr, tk, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 1, c + 8, p.N));
+          b3 = mask_pair(b3, keep_elem(p.seed, p.thr, tk + 8, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 9, c + 8, p.N));
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i >= mblocks) break;
+          // A fragment = G^T (ranks x tokens) from G stored [token][rank]
+          uint32_t a0, a1, a2, a3;
+          const int mi = lane >> 3;
+          const int tr = ks * 16 + (mi >> 1) * 8 + (lane & 7);
+          const int rcol = i * 16 + (mi & 1) * 8;
+          ldsm_x4_t(gb + tr * (p.r * 2) + rcol * 2, a0, a1, a2, a3);
+          mma_bf16_16816(acc[i][0], a0, a1, a2, a3, b0, b1);
+          mma_bf16_16816(acc[i][1], a0, a1, a2, a3, b2, b3);
+        }
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+      if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+    }
+    // write partial[q][k][n]
+    float *out = p.partial + static_cast<int64_t>(blockIdx.y) * p.r * p.N;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      if (i >= mblocks) break;
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int k = i * 16 + (lane >> 2);
+        const int c = n0 + cw + j * 8 + 2 * (lane & 3);
+        if (c < p.N) {
+          if (k < p.r) {
+            out[static_cast<int64_t>(k) * p.N + c] = acc[i][j][0];
+            out[static_cast<int64_t>(k) * p.N + c + 1] = acc[i][j][1];
+          }
+          if (k + 8 < p.r) {
+            out[static_cast<int64_t>(k + 8) * p.N + c] = acc[i][j][2];
+            out[static_cast<int64_t>(k + 8) * p.N + c + 1] = acc[i][j][3];
+          }
+        }
+      }
+    }
+  }
+}
+
+// out[e] = factor * sum_q partial[q][e], q in order 0..splits-1.
+__global__ void lora_reduce_splits_kernel(const float *__restrict__ partial, int splits, int64_t n,
+                                          float factor, float *__restrict__ out) {
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    float s = 0.f;
+    for (int q = 0; q < splits; ++q) s += partial[static_cast<int64_t>(q) * n + e];
+    out[e] = s * factor;
+  }
+}
+
+__global__ void lora_mask_kernel(uint64_t seed, uint64_t thr, int64_t T, int64_t d_in, uint8_t *mask) {
+  const int64_t n = T * d_in;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    mask[e] = keep_elem(seed, thr, e / d_in, e % d_in, d_in) ? 0 : 1;
+}
+
+}  // namespace lora

@@ -163,14 +163,17 @@ void oracle_fwd(int64_t T, int64_t d_in, int64_t d_out, int32_t n_adapters,
             const uint16_t *wrow = W + i * d_out;
             for (int64_t j = 0; j < d_out; ++j) y[j] += x * bf(wrow[j]);
         }
-        /* shrink: U = Xd * A_a */
+        /* shrink: U = Xd * A_a, Xd[i] = X[t,i] * keep(t,i) */
+        double *xd = (double *)malloc(sizeof(double) * (size_t)d_in);
+        for (int64_t i = 0; i < d_in; ++i)
+            xd[i] = bf(X[t * d_in + i]) * keep_factor(seed, thr, p, t, i, d_in);
         for (int32_t k = 0; k < r; ++k) {
             const uint16_t *arow = A_pool + (off[a] + k) * d_in;
             double acc = 0.0;
-            for (int64_t i = 0; i < d_in; ++i)
-                acc += bf(X[t * d_in + i]) * keep_factor(seed, thr, p, t, i, d_in) * bf(arow[i]);
+            for (int64_t i = 0; i < d_in; ++i) acc += xd[i] * bf(arow[i]);
             u[k] = acc;
         }
+        free(xd);
         /* expand: Y += s * U * B_a */
         for (int64_t j = 0; j < d_out; ++j) {
             double acc = 0.0;
@@ -216,17 +219,20 @@ void oracle_bwd(int64_t T, int64_t d_in, int64_t d_out, int32_t n_adapters,
         for (int64_t t = 0; t < T; ++t) {
             int32_t a = ids[t];
             double s = (double)scale[a];
+            double *xd = (double *)malloc(sizeof(double) * (size_t)d_in);
+            for (int64_t i = 0; i < d_in; ++i)
+                xd[i] = bf(X[t * d_in + i]) * keep_factor(seed, thr, p, t, i, d_in);
             for (int32_t k = 0; k < ranks[a]; ++k) {
                 const uint16_t *arow = A_pool + (off[a] + k) * d_in;
                 const uint16_t *brow = B_pool + (off[a] + k) * d_out;
                 double acc = 0.0;
-                for (int64_t i = 0; i < d_in; ++i)
-                    acc += bf(X[t * d_in + i]) * keep_factor(seed, thr, p, t, i, d_in) * bf(arow[i]);
+                for (int64_t i = 0; i < d_in; ++i) acc += xd[i] * bf(arow[i]);
                 U[t * rmax + k] = acc;
                 double g = 0.0;
                 for (int64_t j = 0; j < d_out; ++j) g += bf(dY[t * d_out + j]) * bf(brow[j]);
                 dU[t * rmax + k] = s * g;
             }
+            free(xd);
         }
     }
     if (dB_pool) {

@@ -1,0 +1,95 @@
+"""C-ABI library checks that need no GPU: it loads, exports every function the
+header declares, maps status codes to strings, and validates arguments on the
+host before touching CUDA."""
+
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import lora_adapter_execution_b200 as lora
+from lora_adapter_execution_b200 import abi
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "lora.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_\s\*]*?\b(lora_[a-z0-9_]+)\s*\(", src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_library_exports_every_header_function():
+    L = abi.load_library()
+    names = header_functions()
+    assert len(names) >= 12
+    for n in names:
+        assert hasattr(L, n), n
+
+
+def test_nm_exports():
+    import subprocess
+    out = subprocess.run(["nm", "-D", "--defined-only", abi.LIB_PATH], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\bT (lora_[a-z0-9_]+)", out))
+    assert set(header_functions()) <= exported
+
+
+def test_status_strings():
+    L = abi.load_library()
+    for code in list(abi.STATUS_NAMES) + [-99]:
+        s = L.lora_status_string(code)
+        assert isinstance(s, bytes) and len(s) > 0
+
+
+def _host_plan(ids, ranks, d_in=64, d_out=64):
+    L = abi.load_library()
+    ids = np.ascontiguousarray(ids, dtype=np.int32)
+    ranks = np.ascontiguousarray(ranks, dtype=np.int32)
+    h = ctypes.c_void_p()
+    rc = L.lora_plan_build_host(ids.ctypes.data_as(ctypes.c_void_p), ids.shape[0],
+                                ranks.ctypes.data_as(ctypes.c_void_p), ranks.shape[0], d_in, d_out,
+                                ctypes.byref(h))
+    if rc == 0:
+        L.lora_plan_destroy(h)
+    return rc
+
+
+def test_plan_argument_errors():
+    assert _host_plan([0, 1, 2], [4, 4, 4]) == 0
+    assert _host_plan([0, 3], [4, 4, 4]) == -2           # id out of range
+    assert _host_plan([-1], [4]) == -2
+    assert _host_plan([0], [0]) == -3                     # rank 0
+    assert _host_plan([0], [257]) == -3                   # rank above the maximum
+    assert _host_plan([0], [4], d_in=12) == -1            # not a multiple of 8
+    assert _host_plan([0], [4], d_out=0) == -1
+    L = abi.load_library()
+    assert L.lora_plan_build_host(None, 1, None, 1, 64, 64, ctypes.byref(ctypes.c_void_p())) == -1
+
+
+def test_null_plan_calls():
+    L = abi.load_library()
+    assert L.lora_plan_get(None, None, None, None) == -1
+    assert L.lora_plan_info(None, None) == -1
+    L.lora_plan_destroy(None)  # ignored
+    assert L.lora_linear_fwd(None, None, None, None, None, None, 0.0, 0, None, None, None) == -1
+
+
+def test_bwd_workspace_size_monotone():
+    a = lora.bwd_workspace_size(4096, 4096, 4096, 16)
+    b = lora.bwd_workspace_size(16384, 4096, 4096, 16)
+    assert 0 < a < b
+    assert lora.bwd_workspace_size(0, 4096, 4096, 16) == 0
+
+
+def test_bwd_rejects_bad_rank_before_cuda():
+    L = abi.load_library()
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 12, p, 1 << 20, None)
+    assert rc == -3
+    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 16, None, 0, None)
+    assert rc == -8

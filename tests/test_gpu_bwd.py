@@ -1,0 +1,99 @@
+"""GPU parity of the single-adapter backward (dU -> dX GEMM with the masked
+adapter term -> token contractions for dA, dB) against the fp64 oracle."""
+
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+from lora_adapter_execution_b200 import workloads as wl
+
+from helpers import check_close, dev_bf16, host_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import lora_adapter_execution_b200 as lora
+    lora.load_library()
+    yield
+    assert lora.device_status() == 0
+
+
+def run_fwd_bwd(inp):
+    """Forward (for U_save) then backward, all through the C ABI."""
+    import lora_adapter_execution_b200 as lora
+    r = int(inp.ranks[0])
+    plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out)
+    X, W = dev_bf16(inp.X), dev_bf16(inp.W)
+    A, B = dev_bf16(inp.A_pool), dev_bf16(inp.B_pool)
+    dY = dev_bf16(inp.dY)
+    scale = torch.from_numpy(inp.scale).cuda()
+    Y = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+    U = torch.empty(inp.T, r, dtype=torch.bfloat16, device="cuda")
+    lora.linear_fwd(plan, X, W, A, B, scale, Y, p_drop=inp.p_drop, seed=inp.mask_seed, U_save=U)
+    dX = torch.empty(inp.T, inp.d_in, dtype=torch.bfloat16, device="cuda")
+    dA = torch.empty(r, inp.d_in, dtype=torch.float32, device="cuda")
+    dB = torch.empty(r, inp.d_out, dtype=torch.float32, device="cuda")
+    ws = torch.empty(lora.bwd_workspace_size(inp.T, inp.d_in, inp.d_out, r), dtype=torch.uint8, device="cuda")
+    lora.linear_bwd(X, W, A, B, float(inp.scale[0]), U, dY, dX, dA, dB, ws, p_drop=inp.p_drop,
+                    seed=inp.mask_seed)
+    assert lora.device_status() == 0
+    plan.destroy()
+    return host_f64(dX), host_f64(dA), host_f64(dB)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T=390, d_in=264, d_out=200, p_drop=0.0),
+    dict(T=390, d_in=264, d_out=200, p_drop=0.1),
+    dict(T=1000, d_in=520, d_out=264, p_drop=0.3),
+])
+def test_bwd_small_vs_oracle(kw):
+    inp = wl.make_inputs("finetune", **kw)
+    dX, dA, dB = run_fwd_bwd(inp)
+    rdX, rdA, rdB = oracle.backward(inp)
+    check_close(dX, rdX, "dX")
+    check_close(dA, rdA, "dA")
+    check_close(dB, rdB, "dB")
+
+
+@pytest.mark.parametrize("r", [8, 32, 64])
+def test_bwd_ranks(r):
+    inp = wl.make_inputs("finetune", T=300, d_in=256, d_out=136, p_drop=0.1)
+    rng = np.random.default_rng(r)
+    A = wl.f32_to_bf16_bits(rng.standard_normal((r, inp.d_in)).astype(np.float32) / 16)
+    B = wl.f32_to_bf16_bits(rng.standard_normal((r, inp.d_out)).astype(np.float32) / np.sqrt(r))
+    inp = dataclasses.replace(inp, ranks=np.array([r], dtype=np.int32), A_pool=A, B_pool=B,
+                              offsets=np.array([0, r]))
+    dX, dA, dB = run_fwd_bwd(inp)
+    rdX, rdA, rdB = oracle.backward(inp)
+    check_close(dX, rdX, f"dX r={r}")
+    check_close(dA, rdA, f"dA r={r}")
+    check_close(dB, rdB, f"dB r={r}")
+
+
+def test_bwd_full_finetune_vs_oracle():
+    inp = wl.make_inputs("finetune")
+    dX, dA, dB = run_fwd_bwd(inp)
+    rng = np.random.default_rng(0)
+    rows = np.unique(np.concatenate([[0, 127, 128, inp.T - 1], rng.choice(inp.T, 40, replace=False)]))
+    rdX, rdA, rdB = oracle.backward(inp, rows=rows.astype(np.int64))
+    check_close(dX[rows], rdX, "dX")
+    check_close(dA, rdA, "dA")
+    check_close(dB, rdB, "dB")
+
+
+def test_bwd_deterministic():
+    inp = wl.make_inputs("finetune", T=2100, d_in=256, d_out=264, p_drop=0.1)
+    a = run_fwd_bwd(inp)
+    b = run_fwd_bwd(inp)
+    for x, y in zip(a, b):
+        assert (x == y).all()

@@ -1,0 +1,197 @@
+"""GPU parity of the forward path (plan -> shrink -> fused tcgen05 GEMM) against
+the fp64 CPU oracle, element by element, through the C ABI.
+
+Tolerance (bf16 I/O, fp32 accumulation): rel-Frobenius <= 5e-3 and
+|err| <= 3e-2 * max(1, |ref|) per element; bit-exact where the inputs make the
+arithmetic exact; the plan and the dropout mask bit-exact."""
+
+from __future__ import annotations
+
+import dataclasses
+
+import numpy as np
+import pytest
+
+import oracle
+from lora_adapter_execution_b200 import workloads as wl
+
+from helpers import check_close, dev_bf16, host_bits, host_f64
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    import lora_adapter_execution_b200 as lora
+    lora.load_library()
+    yield
+    assert lora.device_status() == 0
+
+
+def run_fwd(inp, want_u=True, p=None, seed=None):
+    import lora_adapter_execution_b200 as lora
+    p = inp.p_drop if p is None else p
+    seed = inp.mask_seed if seed is None else seed
+    plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out)
+    X, W = dev_bf16(inp.X), dev_bf16(inp.W)
+    A, B = dev_bf16(inp.A_pool), dev_bf16(inp.B_pool)
+    scale = torch.from_numpy(inp.scale).cuda()
+    Y = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+    rmax = plan.info()["r_max"]
+    U = torch.full((inp.T, rmax), float("nan"), dtype=torch.bfloat16, device="cuda") if want_u else None
+    lora.linear_fwd(plan, X, W, A, B, scale, Y, p_drop=p, seed=seed, U_save=U)
+    assert lora.device_status() == 0
+    out = (host_f64(Y), host_f64(U) if want_u else None)
+    plan.destroy()
+    return out
+
+
+SMALL_CASES = {
+    # ragged everywhere: T not a multiple of 128, d_in not of 64, d_out not of 256
+    "tiny": dict(name="tiny", kw={}),
+    "decode_small": dict(name="decode", kw=dict(T=300, d_in=328, d_out=264, n_adapters=40)),
+    "prefill_small": dict(name="prefill", kw=dict(T=1100, d_in=256, d_out=520, n_adapters=12)),
+    "fleet_small": dict(name="fleet", kw=dict(T=700, d_in=320, d_out=296, n_adapters=200)),
+    "finetune_small": dict(name="finetune", kw=dict(T=390, d_in=264, d_out=200, with_dy=False)),
+    "rank_256": dict(name="tiny", kw=dict(T=200, d_in=192, d_out=136, n_adapters=3)),
+}
+
+
+@pytest.mark.parametrize("case", list(SMALL_CASES))
+def test_fwd_small_vs_oracle(case):
+    c = SMALL_CASES[case]
+    inp = wl.make_inputs(c["name"], **c["kw"])
+    if case == "rank_256":
+        # extreme ranks: the maximum (256, four shrink pieces), 1, and a non-multiple of 16
+        ranks = np.array([256, 1, 130], dtype=np.int32)
+        off = np.concatenate([[0], np.cumsum(ranks)])
+        rng = np.random.default_rng(3)
+        A = wl.f32_to_bf16_bits(rng.standard_normal((off[-1], inp.d_in)).astype(np.float32) / 14)
+        B = wl.f32_to_bf16_bits(rng.standard_normal((off[-1], inp.d_out)).astype(np.float32) / 8)
+        inp = dataclasses.replace(inp, ranks=ranks, A_pool=A, B_pool=B, offsets=off,
+                                  scale=np.array([0.25, 3.0, -0.5], dtype=np.float32))
+    Y, U = run_fwd(inp)
+    Yr, Ur = oracle.forward(inp, want_u=True)
+    check_close(Y, Yr, f"{case} Y")
+    check_close(U, Ur[:, :U.shape[1]], f"{case} U")
+
+
+def test_fwd_dropout_small():
+    inp = wl.make_inputs("fleet", T=520, d_in=256, d_out=264, n_adapters=60, p_drop=0.1)
+    inp = dataclasses.replace(inp, mask_seed=1234)
+    Y, U = run_fwd(inp)
+    Yr, Ur = oracle.forward(inp, want_u=True)
+    check_close(Y, Yr, "dropout Y")
+    check_close(U, Ur[:, :U.shape[1]], "dropout U")
+
+
+def test_fwd_integer_bit_exact():
+    # |U| <= 64*4 = 256 (exact in bf16) and every fp32 partial sum is an exact
+    # integer, so the GPU result is exactly the oracle's value rounded once.
+    rng = np.random.default_rng(7)
+    T, d_in, d_out = 260, 64, 272
+    ranks = [16, 5, 32, 1]
+    ids = rng.integers(0, 4, size=T)
+    inp = wl.integer_inputs(T, d_in, d_out, ranks, ids, seed=5, lo=-2, hi=2)
+    Y, U = run_fwd(inp)
+    Yr, Ur = oracle.forward(inp, want_u=True)
+    want = wl.bf16_bits_to_f32(wl.f32_to_bf16_bits(Yr.astype(np.float32))).astype(np.float64)
+    assert np.abs(Yr).max() < 2**24
+    assert (Y == want).all(), np.argwhere(Y != want)[:5]
+    assert (U == Ur[:, :U.shape[1]]).all()
+
+
+def test_fwd_B_zero_equals_base_gemm():
+    import lora_adapter_execution_b200 as lora
+    inp = wl.make_inputs("decode", T=384, d_in=512, d_out=512, n_adapters=16)
+    inp = dataclasses.replace(inp, B_pool=np.zeros_like(inp.B_pool))
+    Y, _ = run_fwd(inp, want_u=False)
+    Yb = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+    lora.base_gemm(dev_bf16(inp.X), dev_bf16(inp.W), Yb)
+    Yb = host_f64(Yb)
+    # every tile's tokens are gathered in another order, but each output row is
+    # the same dot products in the same K order: identical values
+    assert (Y == Yb).all()
+    check_close(Yb, oracle.forward(inp), "base")
+
+
+def test_base_gemm_ragged_vs_oracle():
+    import lora_adapter_execution_b200 as lora
+    inp = wl.make_inputs("decode", T=333, d_in=200, d_out=776, n_adapters=2)
+    Yb = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+    lora.base_gemm(dev_bf16(inp.X), dev_bf16(inp.W), Yb)
+    z = dataclasses.replace(inp, B_pool=np.zeros_like(inp.B_pool))
+    check_close(host_f64(Yb), oracle.forward(z), "base ragged")
+
+
+def test_fwd_token_permutation_invariance():
+    inp = wl.make_inputs("fleet", T=600, d_in=256, d_out=256, n_adapters=90)
+    Y, _ = run_fwd(inp, want_u=False)
+    pi = np.random.default_rng(2).permutation(inp.T)
+    inp2 = dataclasses.replace(inp, X=inp.X[pi].copy(), ids=inp.ids[pi].copy())
+    Y2, _ = run_fwd(inp2, want_u=False)
+    check_close(Y2, Y[pi], "permuted")
+
+
+def test_plan_on_device_matches_oracle():
+    import lora_adapter_execution_b200 as lora
+    inp = wl.make_inputs("fleet", d_in=16, d_out=16)
+    plan = lora.Plan(inp.ids, inp.ranks, 4096, 4096)
+    perm, seg = plan.grouping()
+    operm, oseg = oracle.plan(inp.ids, inp.n_adapters)
+    assert (perm == operm).all() and (seg == oseg).all()
+
+
+@pytest.mark.parametrize("p,seed", [(0.1, 0), (0.5, 77), (0.0, 3)])
+def test_dropout_mask_bit_exact(p, seed):
+    import lora_adapter_execution_b200 as lora
+    T, d = 333, 264
+    m = torch.empty(T, d, dtype=torch.uint8, device="cuda")
+    lora.dropout_mask(seed, p, m)
+    assert (m.cpu().numpy() == oracle.mask(seed, p, T, d)).all()
+
+
+def _sample_rows(T, n, seed=0):
+    rng = np.random.default_rng(seed)
+    edge = [0, 1, 127, 128, T - 1, T - 2, T // 2]
+    return np.unique(np.concatenate([edge, rng.choice(T, size=n, replace=False)])).astype(np.int64)
+
+
+@pytest.mark.parametrize("name,nrows", [("decode", None), ("prefill", 48), ("fleet", 96), ("finetune", 32)])
+def test_fwd_full_size_vs_oracle(name, nrows):
+    inp = wl.make_inputs(name, with_dy=False)
+    Y, U = run_fwd(inp)
+    rows = np.arange(inp.T) if nrows is None else _sample_rows(inp.T, nrows)
+    Yr, Ur = oracle.forward(inp, rows=rows, want_u=True)
+    check_close(Y[rows], Yr, f"{name} Y")
+    check_close(U[rows], Ur[:, :U.shape[1]], f"{name} U")
+
+
+def test_fwd_repeatable_bitwise():
+    inp = wl.make_inputs("fleet", T=900, d_in=256, d_out=264, n_adapters=100)
+    Y1, U1 = run_fwd(inp)
+    Y2, U2 = run_fwd(inp)
+    assert (Y1 == Y2).all() and (U1 == U2).all()
+
+
+def test_fwd_argument_errors():
+    import lora_adapter_execution_b200 as lora
+    inp = wl.make_inputs("tiny")
+    plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out)
+    X, W = dev_bf16(inp.X), dev_bf16(inp.W)
+    A, B = dev_bf16(inp.A_pool), dev_bf16(inp.B_pool)
+    scale = torch.from_numpy(inp.scale).cuda()
+    Y = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(lora.LoraError):
+        lora.linear_fwd(plan, X, W, A, B, scale, Y, p_drop=1.0)
+    Xo = torch.empty(inp.T * inp.d_in + 1, dtype=torch.bfloat16, device="cuda")[1:].view(inp.T, inp.d_in)
+    with pytest.raises(lora.LoraError):
+        lora.linear_fwd(plan, Xo, W, A, B, scale, Y)
+    host_plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out, host_only=True)
+    with pytest.raises(lora.LoraError):
+        lora.linear_fwd(host_plan, X, W, A, B, scale, Y)
+    assert lora.device_status() == 0
