@@ -268,7 +268,7 @@ def run_lora(a):
     for c in range(n_copies):
         cp = dict(X=d(inp.X), W=d(inp.W), A=d(inp.A_pool), B=d(inp.B_pool),
                   Y=torch.empty(T, do, dtype=torch.bfloat16, device=dev),
-                  U=torch.empty(T, r_max, dtype=torch.bfloat16, device=dev) if finetune else None)
+                  U=torch.empty(T, r_max, dtype=torch.float32, device=dev) if finetune else None)
         if finetune:
             r = int(inp.ranks[0])
             cp.update(dY=d(inp.dY), dX=torch.empty(T, di, dtype=torch.bfloat16, device=dev),
@@ -341,6 +341,9 @@ def run_lora(a):
     assert lora.device_status() == 0
 
     # torch.matmul base for the overhead reference (cuBLAS, same shape and rotation)
+    with torch.cuda.stream(stream):
+        torch.matmul(copies[0]["X"], copies[0]["W"], out=copies[0]["Y"])  # create the cuBLAS handle outside capture
+    torch.cuda.synchronize()
     tgraphs = []
     for cp in copies:
         g = torch.cuda.CUDAGraph()

@@ -150,8 +150,10 @@ void lora_plan_destroy(lora_plan_t plan);
  *   seed    dropout seed
  *   Y       bf16 [T, d_out]    output, original token order (fp32 accumulation,
  *           rounded once to bf16)
- *   U_save  bf16 [T, r_max] or NULL: U[t,k] = ((D ⊙ X)[t]·A_a)[k] for k < r_a,
- *           zero for k >= r_a (r_max from lora_plan_info); the backward's input
+ *   U_save  f32 [T, r_max] or NULL: U[t,k] = ((D ⊙ X)[t]·A_a)[k] for k < r_a,
+ *           zero for k >= r_a (r_max from lora_plan_info); the backward's input.
+ *           Kept in fp32: the backward reduces it over all tokens, where a bf16
+ *           rounding of every term would dominate the error of small sums.
  *   stream  launch stream
  * The plan's scratch holds s_a·U rounded to bf16 between the two kernels, so
  * two forwards with one plan must not run concurrently.
@@ -159,7 +161,7 @@ void lora_plan_destroy(lora_plan_t plan);
  * ------------------------------------------------------------------------ */
 int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
                     const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed,
-                    uint16_t *Y, uint16_t *U_save, lora_stream_t stream);
+                    uint16_t *Y, float *U_save, lora_stream_t stream);
 
 /* The forward's two phases, for callers that schedule or time them apart
  * (lora_linear_fwd is exactly lora_linear_shrink followed by lora_fused_gemm
@@ -174,7 +176,7 @@ int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
  * before this call on the stream.
  * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA. */
 int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_pool, const float *scale,
-                       double p_drop, uint64_t seed, uint16_t *U_save, lora_stream_t stream);
+                       double p_drop, uint64_t seed, float *U_save, lora_stream_t stream);
 int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *B_pool,
                     uint16_t *Y, lora_stream_t stream);
 
@@ -194,7 +196,7 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
  *
  *   X, W, A (bf16 [r, d_in], rows = columns of A), B (bf16 [r, d_out]),
  *   scale, p_drop, seed    as in the forward (same mask)
- *   U_save  bf16 [T, r]    the forward's U_save
+ *   U_save  f32 [T, r]     the forward's U_save
  *   dY      bf16 [T, d_out]
  *   dX      bf16 [T, d_in]  output
  *   dA      f32 [r, d_in]   output
@@ -209,7 +211,7 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
 size_t lora_linear_bwd_workspace_size(int64_t T, int64_t d_in, int64_t d_out, int32_t r);
 
 int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B,
-                    float scale, double p_drop, uint64_t seed, const uint16_t *U_save,
+                    float scale, double p_drop, uint64_t seed, const float *U_save,
                     const uint16_t *dY, uint16_t *dX, float *dA, float *dB, int64_t T,
                     int64_t d_in, int64_t d_out, int32_t r, void *workspace,
                     size_t workspace_bytes, lora_stream_t stream);
@@ -219,6 +221,15 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
  * Errors: LORA_ERR_ARG, LORA_ERR_CUDA. */
 int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint8_t *mask_dev,
                       lora_stream_t stream);
+
+/* Test hook for failure detection: launch one thread that waits on an mbarrier
+ * nothing will complete, with a wait limit of `limit_us` microseconds (1 ..
+ * 10^6). The wait runs out, sets LORA_DEV_TIMEOUT in the status word and the
+ * kernel returns normally, so the context stays usable; `*waited_ok_dev`
+ * (device int) receives 0. This is the same bounded wait every kernel of the
+ * library uses on its pipeline barriers.
+ * Errors: LORA_ERR_ARG, LORA_ERR_CUDA. */
+int lora_selftest_bounded_wait(uint32_t limit_us, int *waited_ok_dev, lora_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the current device's status word.
  *   status_host  receives the LORA_DEV_* bits (0 if all kernels ran cleanly); may be NULL

@@ -74,6 +74,7 @@ def load_library():
                                            _i64, _i64, _i64, _i32, _vp, _sz, _vp]),
         "lora_dropout_mask": (ctypes.c_int, [_u64, _dbl, _i64, _i64, _vp, _vp]),
         "lora_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
+        "lora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _vp, _vp]),
         "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -210,3 +211,9 @@ def device_status(stream=None) -> int:
     if rc not in (LORA_OK, -5):
         raise LoraError(rc, "lora_device_status")
     return int(v.value)
+
+
+def selftest_bounded_wait(limit_us: int, waited_ok, *, stream=None):
+    """Run the bounded-wait self-test (see include/lora.h)."""
+    _check(load_library().lora_selftest_bounded_wait(int(limit_us), _ptr(waited_ok), _stream(stream)),
+           "lora_selftest_bounded_wait")

@@ -62,19 +62,22 @@ __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   return ok != 0;
 }
 // Wait for the phase of `parity` to complete. Returns false (after flagging
-// LORA_DEV_TIMEOUT) if it has not completed within kWaitLimitNs.
-__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+// LORA_DEV_TIMEOUT) if it has not completed within `limit_ns`.
+__device__ __forceinline__ bool mbar_wait_for(uint32_t bar, uint32_t parity, uint64_t limit_ns) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer();
   while (true) {
 #pragma unroll 1
     for (int i = 0; i < 64; ++i)
       if (mbar_try_wait(bar, parity)) return true;
-    if (globaltimer() - t0 > kWaitLimitNs) {
+    if (globaltimer() - t0 > limit_ns) {
       flag_status(LORA_DEV_TIMEOUT);
       return false;
     }
   }
+}
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+  return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
 // ------------------------------------------------------------------ TMA / bulk copies
@@ -104,6 +107,17 @@ __device__ __forceinline__ void bulk_g2s(uint32_t dst, const void *src, uint32_t
           dst),
       "l"(src), "r"(bytes), "r"(bar)
       : "memory");
+}
+
+// 16-byte global -> shared async copy; src_bytes = 0 fills the 16 bytes with zeros.
+__device__ __forceinline__ void cp_async_16(uint32_t dst, const void *src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+// Arrive on `bar` once every cp.async this thread issued so far has landed (the
+// arrival is counted in the barrier's expected count).
+__device__ __forceinline__ void cp_async_arrive_noinc(uint32_t bar) {
+  asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(bar) : "memory");
 }
 
 // ------------------------------------------------------------------ tcgen05
@@ -206,6 +220,25 @@ __host__ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64
 __device__ __forceinline__ bool keep_elem(uint64_t seed, uint64_t thr, int64_t t, int64_t col,
                                           int64_t d_in) {
   return thr == 0 || splitmix64_at(seed, static_cast<uint64_t>(t * d_in + col)) >= thr;
+}
+
+// Keep bits of 32 consecutive mask positions idx0 .. idx0+31 (bit i set if kept):
+// the same SplitMix64 outputs as splitmix64_at, with the state advanced by one
+// increment per position instead of recomputed.
+__device__ __forceinline__ uint32_t keep_mask32(uint64_t seed, uint64_t thr, uint64_t idx0) {
+  if (thr == 0) return 0xFFFFFFFFu;
+  uint64_t z = seed + (idx0 + 1ull) * 0x9E3779B97F4A7C15ull;
+  uint32_t m = 0;
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    uint64_t x = z;
+    x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
+    x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
+    x ^= x >> 31;
+    m |= (x >= thr ? 1u : 0u) << i;
+    z += 0x9E3779B97F4A7C15ull;
+  }
+  return m;
 }
 
 // ------------------------------------------------------------------ bf16 packing

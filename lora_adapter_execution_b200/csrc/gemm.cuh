@@ -13,9 +13,10 @@
 // 数千大模型成为可能" without padding adapters to a common rank.
 //
 // Structure: persistent CTAs (one per SM), 6 warps:
-//   warp 0      TMA producer (one thread): X rows (tile load, or gather4 by the
-//               plan's permutation), W tile, then the tile's s·U images (bulk
-//               copy) and the matching rows of B_pool (tile loads)
+//   warp 0      producer: X rows (one TMA box when the tile's tokens are
+//               consecutive, else 16-byte cp.async row copies by the plan's
+//               permutation from all 32 lanes), W tile (TMA), then the tile's
+//               s·U images (bulk copy) and the matching B_pool rows (TMA)
 //   warp 1      MMA issuer (one thread) + TMEM owner: 128x256 fp32 accumulator,
 //               double-buffered in TMEM (512 columns) so the epilogue of tile i
 //               overlaps the main loop of tile i+1
@@ -40,9 +41,10 @@ constexpr int kStageB = kBN * kBK * 2;            // 32 KB
 constexpr int kStageBytes = kStageA + kStageB;    // 48 KB
 constexpr int kGemmThreads = 192;
 constexpr int kGemmBarBytes = 256;
-constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 4;
+constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 4 + kBM * 16;
 
 enum GemmEpi { kEpiStore = 0, kEpiBwdLora = 1 };
+constexpr int kEpiRankRegs = 16;  // dU values per row kept in registers by the backward epilogue
 
 struct GemmParams {
   int32_t T;       // rows (tokens)
@@ -54,6 +56,7 @@ struct GemmParams {
   const ChunkDesc *chunks;
   const int32_t *perm;
   const uint8_t *uimg;  // s·U images, one 16 KB block per 64 augmented columns
+  const uint16_t *Aptr; // the A operand's rows (X or dY), row stride K, for gathered tiles
   __nv_bfloat16 *out;   // [T, N]
   // backward epilogue: out += keep(t, col) / (1 - p) * sum_k dU[t, k] * A[k, col]
   const float *dU;      // [T, r]
@@ -61,7 +64,52 @@ struct GemmParams {
   int32_t r;
   uint64_t seed, thr;
   float inv_keep;
+  // K split: 1 = persistent CTAs over all tiles; S > 1 = one tile per cluster of
+  // S CTAs, CTA q takes base K blocks [q*KB/S, (q+1)*KB/S) and adapter blocks
+  // q, q+S, ...; partial accumulators are summed through distributed shared
+  // memory and CTA q stores output columns [q*256/S, (q+1)*256/S).
+  int32_t ksplit;
 };
+
+constexpr int kRedStride = kBN + 4;  // fp32 row stride of the split-K partial in smem (padded)
+
+// The K blocks one CTA contributes to one tile.
+struct BlockRange {
+  int kb_lo, nbase;  // base blocks kb_lo .. kb_lo + nbase - 1
+  int q, S, nlb;     // adapter blocks q, q + S, ... < nlb
+  __device__ __forceinline__ int count() const { return nbase + (q < nlb ? (nlb - q + S - 1) / S : 0); }
+  // index into the tile's block sequence: < KB base, >= KB adapter block (blk - KB)
+  __device__ __forceinline__ int block(int i, int KB) const {
+    return i < nbase ? kb_lo + i : KB + q + (i - nbase) * S;
+  }
+};
+
+__device__ __forceinline__ BlockRange block_range(int KB, int nlb, int q, int S) {
+  BlockRange br;
+  br.kb_lo = KB * q / S;
+  br.nbase = KB * (q + 1) / S - br.kb_lo;
+  br.q = q;
+  br.S = S;
+  br.nlb = nlb;
+  return br;
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+  uint32_t r;
+  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+  return r;
+}
+__device__ __forceinline__ void cluster_barrier() {
+  asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void ld_dsmem_v4(uint32_t local_addr, uint32_t rank, float (&v)[4]) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
+               : "r"(ra)
+               : "memory");
+}
 
 __device__ __forceinline__ TileDesc regular_tile(int mt, int T) {
   TileDesc td;
@@ -95,13 +143,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGemmStages + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   int32_t *rowcache = reinterpret_cast<int32_t *>(smem + kGemmStages * kStageBytes + kGemmBarBytes);
+  int4 *chunkcache = reinterpret_cast<int4 *>(smem + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
-      mbar_init(full0 + 8 * s, 1);
+      mbar_init(full0 + 8 * s, 33);  // producer lane 0 (expect_tx) + one arrival per producer lane
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -123,63 +172,100 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int n_tiles = p.n_mt * p.n_nt;
   const int KB = (p.K + kBK - 1) / kBK;
   const bool has_plan = p.tiles != nullptr;
+  const bool split = p.ksplit > 1;
+  const int S = split ? p.ksplit : 1;
+  const int q = split ? static_cast<int>(cluster_rank()) : 0;
+  const int tile0 = split ? static_cast<int>(blockIdx.x) / S : static_cast<int>(blockIdx.x);
+  const int tile_step = split ? n_tiles : static_cast<int>(gridDim.x);
 
   if (warp == 0) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ producer
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
-        const int mt = tile % p.n_mt;
-        const int nt = tile / p.n_mt;
-        const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
-        const int n0 = nt * kBN;
-        if (td.contig < 0) {
-          for (int i = 0; i < kBM; ++i) {
-            const int rr = i < td.rows ? i : td.rows - 1;  // pad rows repeat a valid row
-            rowcache[i] = p.perm[td.row0 + rr];
-          }
+    // -------------------------------------------------------------- producer
+    // The whole warp stages each tile's gather rows and adapter table in shared
+    // memory (no dependent global loads inside the K loop); lane 0 issues TMA.
+    int stage = 0;
+    uint32_t phase = 0;
+    for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
+      const int mt = tile % p.n_mt;
+      const int nt = tile / p.n_mt;
+      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      const int n0 = nt * kBN;
+      if (td.contig < 0) {
+        for (int i = lane; i < kBM; i += 32) {
+          const int rr = i < td.rows ? i : td.rows - 1;  // pad rows repeat a valid row
+          rowcache[i] = p.perm[td.row0 + rr];
         }
-        const int nlb = (td.kaug + kAugBlock - 1) / kAugBlock;
-        for (int blk = 0; blk < KB + nlb; ++blk) {
-          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
-          const uint32_t a_dst = stage0 + stage * kStageBytes;
-          const uint32_t b_dst = a_dst + kStageA;
-          const uint32_t fb = full0 + 8 * stage;
-          if (blk < KB) {
-            const int k0 = blk * kBK;
-            mbar_arrive_expect_tx(fb, kStageA + kStageB);
-            if (td.contig >= 0) {
-              tma_load_2d(a_dst, &mapA, fb, k0, td.contig);
-            } else {
-              for (int g = 0; g < kBM / 4; ++g)
-                tma_gather4(a_dst + g * 512, &mapAg, fb, k0, rowcache[4 * g], rowcache[4 * g + 1],
-                            rowcache[4 * g + 2], rowcache[4 * g + 3]);
-            }
+      }
+      for (int c = lane; c < td.nchunk; c += 32) {
+        const ChunkDesc cd = p.chunks[td.chunk0 + c];
+        chunkcache[c] = make_int4(cd.pool_row, cd.kofs, cd.kc, 0);
+      }
+      __syncwarp();
+      // Every lane runs the K loop. Each stage's full barrier expects 33 arrivals:
+      // lane 0's expect_tx arrival (TMA bytes) plus one per lane, made by the
+      // completion of the lane's cp.async row copies (gathered tiles) or by a
+      // plain arrive (everything else).
+      const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
+      const int nblk = br.count();
+      const bool gathered = td.contig < 0;
+      int c = 0;  // chunk cursor over the tile's adapter table (lane 0)
+      for (int i = 0; i < nblk; ++i) {
+        const int blk = br.block(i, KB);
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
+        const uint32_t a_dst = stage0 + stage * kStageBytes;
+        const uint32_t b_dst = a_dst + kStageA;
+        const uint32_t fb = full0 + 8 * stage;
+        if (blk < KB) {
+          const int k0 = blk * kBK;
+          if (lane == 0) {
+            mbar_arrive_expect_tx(fb, (gathered ? 0 : kStageA) + kStageB);
+            if (!gathered) tma_load_2d(a_dst, &mapA, fb, k0, td.contig);
             if (B_KMAJOR) {
               tma_load_2d(b_dst, &mapB, fb, k0, n0);
             } else {
               for (int j = 0; j < kBN / 64; ++j) tma_load_2d(b_dst + j * 8192, &mapB, fb, n0 + j * 64, k0);
             }
+          }
+          if (gathered) {
+            // 128 rows x 8 16-byte chunks; a warp instruction covers 4 whole rows.
+            // Placed with the 128-byte swizzle the MMA descriptor expects.
+            const int chunk = lane & 7;
+            const bool inside = k0 + chunk * 8 < p.K;
+#pragma unroll 4
+            for (int it = 0; it < kBM / 4; ++it) {
+              const int row = it * 4 + (lane >> 3);
+              const uint16_t *src = p.Aptr + static_cast<int64_t>(rowcache[row]) * p.K + (inside ? k0 + chunk * 8 : 0);
+              cp_async_16(a_dst + row * 128 + (((chunk ^ (row & 7)) & 7) << 4), src, inside ? 16u : 0u);
+            }
+            cp_async_arrive_noinc(fb);
           } else {
-            // adapter K block: 64 augmented columns (up to 4 MMA K steps)
+            mbar_arrive(fb);
+          }
+        } else {
+          if (lane == 0) {
+            // adapter K block: 64 augmented columns (up to 4 MMA K steps). Each
+            // chunk spans 2*kc columns: s*U rounded to bf16 (hi), then the
+            // rounding remainder (lo); both multiply the same B rows.
             const int lb = blk - KB;
             const int steps = min(4, (td.kaug - lb * kAugBlock) / 16);
             mbar_arrive_expect_tx(fb, kStageA + steps * (kBN / 64) * 2048);
             bulk_g2s(a_dst, p.uimg + td.uofs + static_cast<int64_t>(lb) * kAugBlockBytes, kAugBlockBytes,
                      fb);
-            int c = td.chunk0;
-            for (int q = 0; q < steps; ++q) {
-              const int kq = lb * kAugBlock + q * 16;
-              while (c + 1 < td.chunk0 + td.nchunk && kq >= p.chunks[c].kofs + p.chunks[c].kc) ++c;
-              const int prow = p.chunks[c].pool_row + (kq - p.chunks[c].kofs);
+            for (int qq = 0; qq < steps; ++qq) {
+              const int kq = lb * kAugBlock + qq * 16;
+              while (c + 1 < td.nchunk && kq >= chunkcache[c].y + 2 * chunkcache[c].z) ++c;
+              const int4 cc = chunkcache[c];
+              int o = kq - cc.y;
+              if (o >= cc.z) o -= cc.z;
+              const int prow = cc.x + o;
               for (int j = 0; j < kBN / 64; ++j)
-                tma_load_2d(b_dst + j * 8192 + q * 2048, &mapBl, fb, n0 + j * 64, prow);
+                tma_load_2d(b_dst + j * 8192 + qq * 2048, &mapBl, fb, n0 + j * 64, prow);
             }
           }
-          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
+          mbar_arrive(fb);
         }
+        if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
       }
+      __syncwarp();
     }
   } else if (warp == 1) {
     if (lane == 0) {
@@ -189,25 +275,28 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t aphase = 0;
-      for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
+      for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
         const int mt = tile % p.n_mt;
         const int kaug = has_plan ? p.tiles[mt].kaug : 0;
-        const int nlb = (kaug + kAugBlock - 1) / kAugBlock;
+        const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const int nblk = br.count();
         if (!mbar_wait(acce0 + 8 * acc, aphase ^ 1)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
         bool ok = true;
-        for (int blk = 0; blk < KB + nlb; ++blk) {
+        for (int i = 0; i < nblk; ++i) {
+          const int blk = br.block(i, KB);
           if (!mbar_wait(full0 + 8 * stage, phase)) { *abort_flag = 1; ok = false; break; }
           tc_fence_after();
+          fence_proxy_async_smem();  // rows written by cp.async (generic proxy) -> MMA operand reads
           const uint32_t a_s = stage0 + stage * kStageBytes;
           const uint32_t b_s = a_s + kStageA;
           const int steps = blk < KB ? 4 : min(4, (kaug - (blk - KB) * kAugBlock) / 16);
-          for (int q = 0; q < steps; ++q) {
-            const uint64_t ad = sdesc_sw128(a_s + q * 32, 16, 1024);
-            const uint64_t bd = B_KMAJOR ? sdesc_sw128(b_s + q * 32, 16, 1024)
-                                         : sdesc_sw128(b_s + q * 2048, 8192, 1024);
-            umma_bf16(d_tmem, ad, bd, kIdesc, (blk > 0 || q > 0) ? 1u : 0u);
+          for (int qq = 0; qq < steps; ++qq) {
+            const uint64_t ad = sdesc_sw128(a_s + qq * 32, 16, 1024);
+            const uint64_t bd = B_KMAJOR ? sdesc_sw128(b_s + qq * 32, 16, 1024)
+                                         : sdesc_sw128(b_s + qq * 2048, 8192, 1024);
+            umma_bf16(d_tmem, ad, bd, kIdesc, (i > 0 || qq > 0) ? 1u : 0u);
           }
           umma_commit(empty0 + 8 * stage);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
@@ -223,15 +312,41 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int row = quarter * 32 + lane;
     int acc = 0;
     uint32_t aphase = 0;
-    for (int tile = blockIdx.x; tile < n_tiles && !*abort_flag; tile += gridDim.x) {
+    for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
       const int mt = tile % p.n_mt;
       const int nt = tile / p.n_mt;
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       if (!mbar_wait(accf0 + 8 * acc, aphase)) { *abort_flag = 1; break; }
       tc_fence_after();
+      if (split) {
+        // partial accumulator -> shared memory (the stage ring is idle: every MMA
+        // of this CTA's only tile has completed); zeros if this CTA had no blocks
+        const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
+        float *red = reinterpret_cast<float *>(smem) + row * kRedStride;
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem_base + ((quarter * 32) << 16) + acc * kBN + c * 32, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            float4 o = any ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                         __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(red + c * 32 + 4 * j) = o;
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(acce0 + 8 * acc);
+        break;
+      }
       const bool valid = row < td.rows;
       int64_t orig = 0;
       if (valid) orig = has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
+      float du[kEpiRankRegs];  // backward: this row's dU, loaded once per tile (ranks <= kEpiRankRegs)
+      if (EPI == kEpiBwdLora) {
+#pragma unroll
+        for (int k = 0; k < kEpiRankRegs; ++k) du[k] = (valid && k < p.r) ? p.dU[orig * p.r + k] : 0.f;
+      }
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];
         tmem_ld32(tmem_base + ((quarter * 32) << 16) + acc * kBN + c * 32, v);
@@ -245,29 +360,30 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             float l[32];
 #pragma unroll
             for (int i = 0; i < 32; ++i) l[i] = 0.f;
-            for (int k = 0; k < p.r; ++k) {
-              const float du = p.dU[orig * p.r + k];
+            auto add_rank = [&](int k, float d) {
               const uint4 *arow = reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(k) * p.N + col0);
 #pragma unroll
               for (int j = 0; j < 4; ++j) {
                 if (col0 + 8 * j < p.N) {
-                  const uint4 w = __ldg(arow + j);
-                  l[8 * j + 0] += du * bf16_lo(w.x);
-                  l[8 * j + 1] += du * bf16_hi(w.x);
-                  l[8 * j + 2] += du * bf16_lo(w.y);
-                  l[8 * j + 3] += du * bf16_hi(w.y);
-                  l[8 * j + 4] += du * bf16_lo(w.z);
-                  l[8 * j + 5] += du * bf16_hi(w.z);
-                  l[8 * j + 6] += du * bf16_lo(w.w);
-                  l[8 * j + 7] += du * bf16_hi(w.w);
+                  const uint4 w = __ldg(arow + j);  // same address across the warp: one broadcast
+                  l[8 * j + 0] += d * bf16_lo(w.x);
+                  l[8 * j + 1] += d * bf16_hi(w.x);
+                  l[8 * j + 2] += d * bf16_lo(w.y);
+                  l[8 * j + 3] += d * bf16_hi(w.y);
+                  l[8 * j + 4] += d * bf16_lo(w.z);
+                  l[8 * j + 5] += d * bf16_hi(w.z);
+                  l[8 * j + 6] += d * bf16_lo(w.w);
+                  l[8 * j + 7] += d * bf16_hi(w.w);
                 }
               }
-            }
+            };
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-              const bool keep = keep_elem(p.seed, p.thr, orig, col0 + i, p.N);
-              f[i] += keep ? p.inv_keep * l[i] : 0.f;
-            }
+            for (int k = 0; k < kEpiRankRegs; ++k)
+              if (k < p.r) add_rank(k, du[k]);
+            for (int k = kEpiRankRegs; k < p.r; ++k) add_rank(k, p.dU[orig * p.r + k]);
+            const uint32_t keep = keep_mask32(p.seed, p.thr, static_cast<uint64_t>(orig * p.N + col0));
+#pragma unroll
+            for (int i = 0; i < 32; ++i) f[i] += ((keep >> i) & 1u) ? p.inv_keep * l[i] : 0.f;
           }
           uint4 *dst = reinterpret_cast<uint4 *>(p.out + orig * p.N + col0);
 #pragma unroll
@@ -291,6 +407,46 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   tc_fence_before();
   __syncthreads();
+  if (split) {
+    // --------------------------------------------------- split-K cluster reduction
+    cluster_barrier();  // every CTA's partial is in its shared memory
+    if (warp >= 2 && tile0 < n_tiles && !*abort_flag) {
+      const int row = (warp & 3) * 32 + lane;
+      const int mt = tile0 % p.n_mt;
+      const int nt = tile0 / p.n_mt;
+      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      if (row < td.rows) {
+        const int64_t orig = has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
+        const int width = kBN / S;
+        const int c0 = q * width;
+        const uint32_t rbase = smem_u32(smem) + static_cast<uint32_t>(row * kRedStride + c0) * 4u;
+        for (int cc = 0; cc < width; cc += 8) {
+          const int col = nt * kBN + c0 + cc;
+          if (col >= p.N) break;
+          float s[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) s[e] = 0.f;
+          for (int pr = 0; pr < S; ++pr) {
+            float a[4], b[4];
+            ld_dsmem_v4(rbase + cc * 4, pr, a);
+            ld_dsmem_v4(rbase + cc * 4 + 16, pr, b);
+#pragma unroll
+            for (int e = 0; e < 4; ++e) {
+              s[e] += a[e];
+              s[4 + e] += b[e];
+            }
+          }
+          uint4 o;
+          o.x = pack_bf16x2(s[0], s[1]);
+          o.y = pack_bf16x2(s[2], s[3]);
+          o.z = pack_bf16x2(s[4], s[5]);
+          o.w = pack_bf16x2(s[6], s[7]);
+          *reinterpret_cast<uint4 *>(p.out + orig * p.N + col) = o;
+        }
+      }
+    }
+    cluster_barrier();  // peers keep their shared memory until every read is done
+  }
   if (warp == 1) {
     __syncwarp();
     tc_fence_after();

@@ -19,7 +19,7 @@ struct TileDesc {
   int32_t rows;    // valid rows (<= 128)
   int32_t chunk0;  // first ChunkDesc of this tile
   int32_t nchunk;  // adapters touching the tile
-  int32_t kaug;    // augmented K = sum of the chunks' kc (multiple of 16)
+  int32_t kaug;    // augmented K = sum of the chunks' 2*kc (multiple of 32)
   int32_t contig;  // original index of row 0 if the tile's tokens are consecutive originals, else -1
   int64_t uofs;    // byte offset of the tile's s*U image in the plan scratch
 };
@@ -30,7 +30,8 @@ struct ChunkDesc {
   int32_t pool_row;  // off_a: first row of the adapter in A_pool / B_pool
   int32_t rank;      // r_a
   int32_t kc;        // r_a rounded up to 16 (MMA K step)
-  int32_t kofs;      // first augmented-K column of the chunk within its tile
+  int32_t kofs;      // first augmented-K column of the chunk within its tile (hi part;
+                     // the lo part starts at kofs + kc)
   int32_t lo, hi;    // tile-local rows [lo, hi) owned by the adapter
   int32_t tile;
 };

@@ -84,9 +84,56 @@ bool make_map(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint
   return r == CUDA_SUCCESS;
 }
 
+// 2-D fp32 tensor map over a row-major [rows x cols] matrix, no swizzle.
+bool make_map_f32(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint32_t box_cols,
+                  uint32_t box_rows) {
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * 4};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void *>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA; }
+
+// Forward GEMM launch: persistent CTAs when there are enough output tiles to
+// fill the GPU; otherwise clusters of S CTAs split the K loop of each tile
+// (S a power of two, S * tiles <= SMs, S <= number of K blocks).
+int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const CUtensorMap &ag,
+                    const CUtensorMap &b, const CUtensorMap &bl, lora_stream_t stream) {
+  const int n_tiles = gp.n_mt * gp.n_nt;
+  const int KB = (gp.K + kBK - 1) / kBK;
+  int S = 1;
+  while (S < 4 && 2 * S * n_tiles <= ds->num_sms && 2 * S <= KB) S *= 2;
+  gp.ksplit = S;
+  if (S == 1) {
+    const int grid = std::min(ds->num_sms, n_tiles);
+    lora_gemm_kernel<false, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(a, ag, b, bl, gp);
+    return launch_status();
+  }
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_tiles * S));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = S;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, lora_gemm_kernel<false, kEpiStore>, a, ag, b, bl, gp) != cudaSuccess) {
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  return LORA_OK;
+}
 
 }  // namespace
 
@@ -229,7 +276,7 @@ void lora_plan_destroy(lora_plan_t plan) {
 }
 
 int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_pool, const float *scale,
-                       double p_drop, uint64_t seed, uint16_t *U_save, lora_stream_t stream) {
+                       double p_drop, uint64_t seed, float *U_save, lora_stream_t stream) {
   if (!plan || !plan->dev || !X || !A_pool || !scale) return LORA_ERR_ARG;
   if (!aligned16(X) || !aligned16(A_pool)) return LORA_ERR_ARG;
   if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
@@ -264,7 +311,8 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   sp.seed = seed;
   sp.inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
   sp.uimg = plan->scratch;
-  sp.U_save = reinterpret_cast<__nv_bfloat16 *>(U_save);
+  sp.In = X;
+  sp.U_save = U_save;
   sp.r_max = hp.r_max;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(n_units * ks));
@@ -311,15 +359,14 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   gp.chunks = plan->d_chunks;
   gp.perm = plan->d_perm;
   gp.uimg = plan->scratch;
+  gp.Aptr = X;
   gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
-  const int grid = std::min(ds->num_sms, gp.n_mt * gp.n_nt);
-  lora_gemm_kernel<false, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(mX128, mXg, mW, mBl, gp);
-  return launch_status();
+  return launch_fwd_gemm(ds, gp, mX128, mXg, mW, mBl, stream);
 }
 
 int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
                     const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed, uint16_t *Y,
-                    uint16_t *U_save, lora_stream_t stream) {
+                    float *U_save, lora_stream_t stream) {
   if (!plan || !plan->dev || !X || !W || !A_pool || !B_pool || !scale || !Y) return LORA_ERR_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(A_pool) || !aligned16(B_pool) || !aligned16(Y))
     return LORA_ERR_ARG;
@@ -347,13 +394,12 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
   gp.N = static_cast<int32_t>(d_out);
   gp.n_mt = static_cast<int32_t>((T + kBM - 1) / kBM);
   gp.n_nt = static_cast<int32_t>((d_out + kBN - 1) / kBN);
+  gp.Aptr = X;
   gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
-  const int grid = std::min(ds->num_sms, gp.n_mt * gp.n_nt);
-  lora_gemm_kernel<false, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(mX128, mX128, mW, mW, gp);
-  return launch_status();
+  return launch_fwd_gemm(ds, gp, mX128, mX128, mW, mW, stream);
 }
 
-// Workspace layout: dU f32 [T, r] | dU bf16 [T, r] | dB partial [S, r, d_out] | dA partial [S, r, d_in]
+// Workspace layout: dU f32 [T, r] | dB partial [S, r, d_out] | dA partial [S, r, d_in]
 static int64_t bwd_splits(int64_t T, int64_t d_in) {
   (void)d_in;
   int64_t s = (T + 2047) / 2048;  // ~2048 tokens per split
@@ -364,11 +410,11 @@ size_t lora_linear_bwd_workspace_size(int64_t T, int64_t d_in, int64_t d_out, in
   if (T <= 0 || d_in <= 0 || d_out <= 0 || r <= 0) return 0;
   auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
   const int64_t S = bwd_splits(T, d_in);
-  return static_cast<size_t>(up(T * r * 4) + up(T * r * 2) + up(S * r * d_out * 4) + up(S * r * d_in * 4));
+  return static_cast<size_t>(up(T * r * 4) + up(S * r * d_out * 4) + up(S * r * d_in * 4));
 }
 
 int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B, float scale,
-                    double p_drop, uint64_t seed, const uint16_t *U_save, const uint16_t *dY, uint16_t *dX,
+                    double p_drop, uint64_t seed, const float *U_save, const uint16_t *dY, uint16_t *dX,
                     float *dA, float *dB, int64_t T, int64_t d_in, int64_t d_out, int32_t r, void *workspace,
                     size_t workspace_bytes, lora_stream_t stream) {
   if (!X || !W || !A || !B || !U_save || !dY || !dX || !dA || !dB) return LORA_ERR_ARG;
@@ -390,9 +436,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
   const int64_t S = bwd_splits(T, d_in);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   float *dU = reinterpret_cast<float *>(ws);
-  __nv_bfloat16 *dU16 = reinterpret_cast<__nv_bfloat16 *>(ws + up(T * r * 4));
-  float *pdB = reinterpret_cast<float *>(ws + up(T * r * 4) + up(T * r * 2));
-  float *pdA = reinterpret_cast<float *>(ws + up(T * r * 4) + up(T * r * 2) + up(S * r * d_out * 4));
+  float *pdB = reinterpret_cast<float *>(ws + up(T * r * 4));
+  float *pdA = reinterpret_cast<float *>(ws + up(T * r * 4) + up(S * r * d_out * 4));
 
   const uint64_t thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
   const float inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
@@ -404,8 +449,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
   ok &= make_map(&mdY128, dY, d_out, T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mWt, W, d_out, d_in, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mdY64, dY, d_out, T, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&mU, U_save, r, T, r, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
-  ok &= make_map(&mdU, dU16, r, T, r, 64, CU_TENSOR_MAP_SWIZZLE_NONE);
+  ok &= make_map_f32(&mU, U_save, r, T, r, 64);
+  ok &= make_map_f32(&mdU, dU, r, T, r, 64);
   ok &= make_map(&mX64, X, d_in, T, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return LORA_ERR_ARG;
 
@@ -418,8 +463,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     sp.r = r;
     sp.npieces = (((r + 15) / 16) * 16 + kShrinkN - 1) / kShrinkN;
     sp.scale1 = scale;
+    sp.In = dY;
     sp.dU = dU;
-    sp.dU_bf16 = dU16;
     const int n_units = static_cast<int>((T + kTileM - 1) / kTileM) * sp.npieces;
     int ks = std::max(1, std::min(4, (2 * ds->num_sms + n_units - 1) / n_units));
     ks = std::min<int>(ks, static_cast<int>((d_out + kSkBK - 1) / kSkBK));
@@ -452,6 +497,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.N = static_cast<int32_t>(d_in);
     gp.n_mt = static_cast<int32_t>((T + kBM - 1) / kBM);
     gp.n_nt = static_cast<int32_t>((d_in + kBN - 1) / kBN);
+    gp.Aptr = dY;
     gp.out = reinterpret_cast<__nv_bfloat16 *>(dX);
     gp.dU = dU;
     gp.A = A;
@@ -459,6 +505,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.seed = seed;
     gp.thr = thr;
     gp.inv_keep = inv_keep;
+    gp.ksplit = 1;
     const int grid = std::min(ds->num_sms, gp.n_mt * gp.n_nt);
     lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mdY128, mWt, mWt, gp);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
@@ -466,8 +513,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
   // K3c: dB = s * U^T * dY and dA = (D ⊙ X)^T * dU, split over tokens, then reduced
   {
     const int64_t tsplit = ((T + S - 1) / S + kTcTok - 1) / kTcTok * kTcTok;
-    const int g_bytes = kTcTok * r * 2;
-    const int stage_bytes = kTcTok * kTcCols * 2 + ((g_bytes + 1023) & ~1023) + 1024;
+    const int g_bytes = kTcTok * r * 4;
+    const int stage_bytes = kTcTok * kTcCols * 2 + ((g_bytes + 1023) & ~1023);
     const int smem = 1024 + kTcStages * stage_bytes + 2 * kTcStages * 8;
     // note: the kernel lays stages out with the same formula
     TcParams tp{};
@@ -506,6 +553,12 @@ int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uin
   const int64_t n = T * d_in;
   const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 65535));
   lora_mask_kernel<<<blocks, 256, 0, stream>>>(seed, thr, T, d_in, mask_dev);
+  return launch_status();
+}
+
+int lora_selftest_bounded_wait(uint32_t limit_us, int *waited_ok_dev, lora_stream_t stream) {
+  if (!waited_ok_dev || limit_us < 1 || limit_us > 1000000) return LORA_ERR_ARG;
+  lora_wait_selftest_kernel<<<1, 32, 0, stream>>>(static_cast<uint64_t>(limit_us) * 1000ull, waited_ok_dev);
   return launch_status();
 }
 

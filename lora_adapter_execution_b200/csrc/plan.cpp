@@ -60,7 +60,9 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
   const int32_t n_seg = (int32_t)(hp.seg.size() / 3);
 
   // Tiles of 128 sorted positions; each adapter run inside a tile is a chunk
-  // whose K slice is the adapter's rank rounded up to the 16-wide MMA step.
+  // whose K slice is twice the adapter's rank rounded up to the 16-wide MMA
+  // step: s*U enters the MMA as bf16 hi + lo parts against the same B rows,
+  // so the adapter term keeps ~16 mantissa bits whatever the scale.
   const int64_t n_tiles = (T + kTileM - 1) / kTileM;
   int32_t s = 0;  // current segment
   int64_t uofs = 0;
@@ -84,7 +86,7 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
       cd.lo = (int32_t)(std::max<int64_t>(s_beg, td.row0) - td.row0);
       cd.hi = (int32_t)(std::min<int64_t>(s_end, r_end) - td.row0);
       cd.tile = (int32_t)m;
-      kofs += cd.kc;
+      kofs += 2 * cd.kc;  // bf16 hi part, then the bf16 lo part of s*U
       hp.max_chunk_rows = std::max(hp.max_chunk_rows, cd.hi - cd.lo);
       hp.chunks.push_back(cd);
       if (s_end <= r_end) ++s;  // segment finished inside this tile

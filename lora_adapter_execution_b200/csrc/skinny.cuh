@@ -12,6 +12,8 @@
 //    shared-memory image the fused GEMM's MMA reads, plus U for the backward.
 //  * lora_tcontract_kernel: partial[q][k][n] = sum_{t in split q} G[t, k] * In[t, n]
 //    (dB with G = U, In = dY; dA with G = dU, In = masked X), fixed token splits.
+//    G stays fp32 and enters the MMA as a hi + lo pair of bf16 (two MMAs), so the
+//    reduction over thousands of tokens keeps ~16 mantissa bits per term.
 //  * lora_reduce_splits_kernel: sums the splits in a fixed order (deterministic).
 //  * lora_mask_kernel: the dropout mask itself (test hook).
 //
@@ -32,13 +34,14 @@ constexpr int kSkBK = 64;                                 // columns per stage (
 constexpr int kSkPool = 72 * 1024;                        // stage ring (also the reduction scratch)
 constexpr int kSkMaxStages = 16;
 constexpr int kSkFinBytes = kTileM * kShrinkN * 4;        // CTA partial [128 x 64] fp32
-constexpr int kSkSmem = 1024 + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64;
+constexpr int kSkSmem = 1024 + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64 + kTileM * 4;
 
 struct ShrinkParams {
   int32_t mode;     // 0: forward shrink over plan units; 1: backward dU over consecutive tiles
   int32_t T, K;     // tokens, contraction length
   int32_t ksplit;   // cluster size along the contraction
   int32_t kslice;   // contraction columns per cluster rank (multiple of kSkBK)
+  const uint16_t *In;  // rows of the contracted input (X or dY), row stride K
   // forward
   const UnitDesc *units;
   const ChunkDesc *chunks;
@@ -48,14 +51,13 @@ struct ShrinkParams {
   uint64_t seed, thr;
   float inv_keep;
   uint8_t *uimg;
-  __nv_bfloat16 *U_save;
+  float *U_save;
   int32_t r_max;
   // backward
   int32_t r;
   int32_t npieces;
   float scale1;
   float *dU;                 // [T, r] fp32
-  __nv_bfloat16 *dU_bf16;    // [T, r]
 };
 
 struct UnitGeom {
@@ -66,7 +68,7 @@ struct UnitGeom {
   int32_t nn;        // piece width (multiple of 16, <= 64)
   int32_t nvalid;    // columns of the piece that are real ranks (rest are zero)
   // forward only
-  int32_t tile, lo, kcol, adapter, n0, last;
+  int32_t tile, lo, kcol, kc, adapter, n0, last;
 };
 
 __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
@@ -84,6 +86,7 @@ __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
     g.tile = cd.tile;
     g.lo = cd.lo;
     g.kcol = cd.kofs + ud.n0;
+    g.kc = cd.kc;
     g.adapter = cd.adapter;
     g.n0 = ud.n0;
     g.last = ud.last;
@@ -100,6 +103,7 @@ __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
     g.tile = m;
     g.lo = 0;
     g.kcol = 0;
+    g.kc = 0;
     g.adapter = 0;
     g.last = 0;
   }
@@ -153,9 +157,9 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
 
 // Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
 // its rank q contracts columns [q*kslice, (q+1)*kslice).
-__global__ void __launch_bounds__(kSkThreads, 1)
+__global__ void __launch_bounds__(kSkThreads, 2)
     lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows, box {64, 16}
-                       const __grid_constant__ CUtensorMap mapInG,   // In rows, box {64, 1} (gather4)
+                       const __grid_constant__ CUtensorMap mapInG,   // unused (kept for the launch signature)
                        const __grid_constant__ CUtensorMap mapF16,   // F rows, box {64, 16}
                        const ShrinkParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -167,6 +171,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * kSkMaxStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kSkMaxStages);
+  int32_t *rowcache = reinterpret_cast<int32_t *>(smem + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -184,7 +189,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
-      mbar_init(full0 + 8 * s, 1);
+      mbar_init(full0 + 8 * s, 33);
       mbar_init(empty0 + 8 * s, kSkConsumerWarps);
     }
     *abort_flag = 0;
@@ -208,29 +213,40 @@ __global__ void __launch_bounds__(kSkThreads, 1)
 
   if (warp == kSkConsumerWarps) {
     // -------------------------------------------------------------- producer
-    if (lane == 0) {
-      int stage = 0;
-      uint32_t phase = 0;
-      for (int b = 0; b < nblk; ++b) {
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
-        const uint32_t fb = full0 + 8 * stage;
-        mbar_arrive_expect_tx(fb, stage_bytes);
-        const uint32_t xb = pool + stage * stage_bytes;
-        const uint32_t fbuf = xb + Rp * 128;
-        const int col = kbeg + b * kSkBK;
-        if (g.contig >= 0) {
+    if (g.contig < 0) {
+      for (int i = lane; i < Rp; i += 32) rowcache[i] = p.perm[g.row0 + min(i, g.rows - 1)];
+    }
+    __syncwarp();
+    // all lanes run the stage loop: lane 0 issues the TMA boxes (F rows, and X
+    // rows of consecutive tokens); gathered X rows are 16-byte cp.async copies
+    // from every lane. Full barriers expect 33 arrivals (see the GEMM producer).
+    int stage = 0;
+    uint32_t phase = 0;
+    const bool gathered = g.contig < 0;
+    for (int b = 0; b < nblk; ++b) {
+      if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
+      const uint32_t fb = full0 + 8 * stage;
+      const uint32_t xb = pool + stage * stage_bytes;
+      const uint32_t fbuf = xb + Rp * 128;
+      const int col = kbeg + b * kSkBK;
+      if (lane == 0) {
+        mbar_arrive_expect_tx(fb, (gathered ? 0 : Rp * 128) + g.nn * 128);
+        if (!gathered)
           for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, g.contig + r16);
-        } else {
-          for (int r4 = 0; r4 < Rp; r4 += 4) {
-            int rr[4];
-#pragma unroll
-            for (int j = 0; j < 4; ++j) rr[j] = p.perm[g.row0 + min(r4 + j, g.rows - 1)];
-            tma_gather4(xb + r4 * 128, &mapInG, fb, col, rr[0], rr[1], rr[2], rr[3]);
-          }
-        }
         for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
-        if (++stage == nstage) { stage = 0; phase ^= 1; }
       }
+      if (gathered) {
+        const int chunk = lane & 7;
+        const bool inside = col + chunk * 8 < p.K;
+        for (int row = lane >> 3; row < Rp; row += 4) {
+          const uint16_t *src = p.In + static_cast<int64_t>(rowcache[row]) * p.K + (inside ? col + chunk * 8 : 0);
+          cp_async_16(xb + row * 128 + (((chunk ^ (row & 7)) & 7) << 4), src, inside ? 16u : 0u);
+        }
+        cp_async_arrive_noinc(fb);
+      } else {
+        mbar_arrive(fb);
+      }
+      if (++stage == nstage) { stage = 0; phase ^= 1; }
     }
   } else {
     // -------------------------------------------------------------- consumers
@@ -348,14 +364,15 @@ __global__ void __launch_bounds__(kSkThreads, 1)
   if (crank == 0) {
     if (p.mode == 0) {
       const float s_a = p.scale[g.adapter] * p.inv_keep;
-      // s·U block of the tile: all 128 rows of columns [kcol, kcol + nn)
+      // s·U of the tile, all 128 rows of columns [kcol, kcol + nn) (bf16 hi part)
+      // and [kcol + kc, kcol + kc + nn) (bf16 lo part: the rounding remainder)
       uint8_t *img = p.uimg + p.tiles[g.tile].uofs;
       for (int e = threadIdx.x; e < kTileM * (g.nn / 8); e += blockDim.x) {
         const int row = e / (g.nn / 8);
         const int c8 = (e % (g.nn / 8)) * 8;
         const int lr = row - g.lo;
         const bool mine = lr >= 0 && lr < g.rows;
-        uint32_t w[4];
+        uint32_t hi[4], lo[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
           float v0 = 0.f, v1 = 0.f;
@@ -363,11 +380,15 @@ __global__ void __launch_bounds__(kSkThreads, 1)
             if (c8 + 2 * j < g.nvalid) v0 = fin[lr * kShrinkN + c8 + 2 * j] * s_a;
             if (c8 + 2 * j + 1 < g.nvalid) v1 = fin[lr * kShrinkN + c8 + 2 * j + 1] * s_a;
           }
-          w[j] = pack_bf16x2(v0, v1);
+          hi[j] = pack_bf16x2(v0, v1);
+          lo[j] = pack_bf16x2(v0 - bf16_lo(hi[j]), v1 - bf16_hi(hi[j]));
         }
         const int col = g.kcol + c8;
         uint8_t *dst = img + (col / kAugBlock) * kAugBlockBytes + sw128_offset(row, col % kAugBlock);
-        *reinterpret_cast<uint4 *>(dst) = make_uint4(w[0], w[1], w[2], w[3]);
+        *reinterpret_cast<uint4 *>(dst) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+        const int col2 = col + g.kc;
+        uint8_t *dst2 = img + (col2 / kAugBlock) * kAugBlockBytes + sw128_offset(row, col2 % kAugBlock);
+        *reinterpret_cast<uint4 *>(dst2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
       if (p.U_save) {
         const int cend = g.last ? p.r_max : min(p.r_max, g.n0 + g.nn);
@@ -376,7 +397,7 @@ __global__ void __launch_bounds__(kSkThreads, 1)
           const int lr = e / ncol, c = e % ncol;
           const int64_t orig = g.contig >= 0 ? g.contig + lr : p.perm[g.row0 + lr];
           const float v = c < g.nvalid ? fin[lr * kShrinkN + c] * p.inv_keep : 0.f;
-          p.U_save[orig * p.r_max + g.n0 + c] = __float2bfloat16_rn(v);
+          p.U_save[orig * p.r_max + g.n0 + c] = v;
         }
       }
     } else {
@@ -385,7 +406,6 @@ __global__ void __launch_bounds__(kSkThreads, 1)
         const int64_t t = g.row0 + lr;
         const float v = fin[lr * kShrinkN + c] * p.scale1;
         p.dU[t * p.r + g.n0 + c] = v;
-        p.dU_bf16[t * p.r + g.n0 + c] = __float2bfloat16_rn(v);
       }
     }
   }
@@ -405,18 +425,24 @@ struct TcParams {
   float *partial;          // [splits][r][N]
 };
 
+// split fp32 values into bf16 hi + lo (hi = rn(v), lo = rn(v - hi)), packed in pairs
+__device__ __forceinline__ void split_pair(float v0, float v1, uint32_t &hi, uint32_t &lo) {
+  hi = pack_bf16x2(v0, v1);
+  lo = pack_bf16x2(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
+}
+
 // partial[q][k][n] = sum_{t in split q} G[t, k] * In[t, n] (In masked if thr != 0).
 // Grid (N / 128, splits).
 __global__ void __launch_bounds__(kTcThreads, 1)
-    lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N], box {64, 64}, swizzle 128B
-                          const __grid_constant__ CUtensorMap mapG,   // G [T, r], box {r, 64}, no swizzle
+    lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N] bf16, box {64, 64}, swizzle 128B
+                          const __grid_constant__ CUtensorMap mapG,   // G [T, r] fp32, box {r, 64}, no swizzle
                           const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   const int in_bytes = kTcTok * kTcCols * 2;    // 16 KB (two 8 KB halves)
-  const int g_bytes = kTcTok * p.r * 2;         // <= 8 KB
-  const int g_pad = ((g_bytes + 1023) & ~1023) + 1024;  // slack: rank-8 fragments read one row past
+  const int g_bytes = kTcTok * p.r * 4;         // <= 16 KB
+  const int g_pad = (g_bytes + 1023) & ~1023;
   const int stage_bytes = in_bytes + g_pad;
   const uint32_t pool = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kTcStages * stage_bytes);
@@ -500,14 +526,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           if (i >= mblocks) break;
-          // A fragment = G^T (ranks x tokens) from G stored [token][rank]
-          uint32_t a0, a1, a2, a3;
-          const int mi = lane >> 3;
-          const int tr = ks * 16 + (mi >> 1) * 8 + (lane & 7);
-          const int rcol = i * 16 + (mi & 1) * 8;
-          ldsm_x4_t(gb + tr * (p.r * 2) + rcol * 2, a0, a1, a2, a3);
-          mma_bf16_16816(acc[i][0], a0, a1, a2, a3, b0, b1);
-          mma_bf16_16816(acc[i][1], a0, a1, a2, a3, b2, b3);
+          // A fragment = G^T (ranks x tokens) from G stored [token][rank] fp32:
+          // element (m, k) of the 16x16 fragment is G[ks*16 + k][i*16 + m]
+          const int m = i * 16 + (lane >> 2);
+          const int k = ks * 16 + 2 * (lane & 3);
+          const float *gf = reinterpret_cast<const float *>(smem + (gb - pool));
+          auto gv = [&](int kk, int mm) { return mm < p.r ? gf[kk * p.r + mm] : 0.f; };
+          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+          split_pair(gv(k, m), gv(k + 1, m), h0, l0);
+          split_pair(gv(k, m + 8), gv(k + 1, m + 8), h1, l1);
+          split_pair(gv(k + 8, m), gv(k + 9, m), h2, l2);
+          split_pair(gv(k + 8, m + 8), gv(k + 9, m + 8), h3, l3);
+          mma_bf16_16816(acc[i][0], h0, h1, h2, h3, b0, b1);
+          mma_bf16_16816(acc[i][1], h0, h1, h2, h3, b2, b3);
+          mma_bf16_16816(acc[i][0], l0, l1, l2, l3, b0, b1);
+          mma_bf16_16816(acc[i][1], l0, l1, l2, l3, b2, b3);
         }
       }
       __syncwarp();
@@ -546,6 +579,18 @@ __global__ void lora_reduce_splits_kernel(const float *__restrict__ partial, int
     float s = 0.f;
     for (int q = 0; q < splits; ++q) s += partial[static_cast<int64_t>(q) * n + e];
     out[e] = s * factor;
+  }
+}
+
+// Self-test of the bounded wait: one thread waits on an mbarrier that nothing
+// will ever complete; the wait gives up after `limit_ns`, flags LORA_DEV_TIMEOUT
+// and the kernel returns normally.
+__global__ void lora_wait_selftest_kernel(uint64_t limit_ns, int *result) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    fence_mbar_init();
+    *result = mbar_wait_for(smem_u32(&bar), 0, limit_ns) ? 1 : 0;
   }
 }
 

@@ -38,7 +38,7 @@ def run_fwd_bwd(inp):
     dY = dev_bf16(inp.dY)
     scale = torch.from_numpy(inp.scale).cuda()
     Y = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
-    U = torch.empty(inp.T, r, dtype=torch.bfloat16, device="cuda")
+    U = torch.empty(inp.T, r, dtype=torch.float32, device="cuda")
     lora.linear_fwd(plan, X, W, A, B, scale, Y, p_drop=inp.p_drop, seed=inp.mask_seed, U_save=U)
     dX = torch.empty(inp.T, inp.d_in, dtype=torch.bfloat16, device="cuda")
     dA = torch.empty(r, inp.d_in, dtype=torch.float32, device="cuda")

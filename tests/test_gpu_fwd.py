@@ -42,7 +42,7 @@ def run_fwd(inp, want_u=True, p=None, seed=None):
     scale = torch.from_numpy(inp.scale).cuda()
     Y = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
     rmax = plan.info()["r_max"]
-    U = torch.full((inp.T, rmax), float("nan"), dtype=torch.bfloat16, device="cuda") if want_u else None
+    U = torch.full((inp.T, rmax), float("nan"), dtype=torch.float32, device="cuda") if want_u else None
     lora.linear_fwd(plan, X, W, A, B, scale, Y, p_drop=p, seed=seed, U_save=U)
     assert lora.device_status() == 0
     out = (host_f64(Y), host_f64(U) if want_u else None)

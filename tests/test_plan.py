@@ -43,12 +43,13 @@ def test_plan_fuzz():
         operm, oseg = oracle.plan(ids, n)
         assert (perm == operm).all() and (seg == oseg).all()
         info = p.info()
-        # augmented K: every tile adds its adapters' ranks rounded up to 16
+        # augmented K: every tile adds, per adapter present, twice its rank
+        # rounded up to 16 (bf16 hi and lo parts of s*U)
         kaug = 0
         for m in range(info["n_tiles"]):
             pos = perm[m * 128:(m + 1) * 128]
             for a in np.unique(ids[pos]):
-                kaug += -(-int(ranks[a]) // 16) * 16
+                kaug += 2 * (-(-int(ranks[a]) // 16) * 16)
         assert info["aug_k_total"] == kaug
         assert info["scratch_bytes"] % 16384 == 0
 
