@@ -169,7 +169,9 @@ int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
  *
  * lora_linear_shrink: U = (D ⊙ X)·A_a for every token, written as s_a·U in
  * bf16 into the plan's scratch (in the layout the fused GEMM reads) and, if
- * U_save is not NULL, as U into U_save. Arguments as in lora_linear_fwd.
+ * U_save is not NULL, as U into U_save. When the plan's tiles are not runs of
+ * consecutive tokens, it first copies X's rows in sorted order into the plan's
+ * scratch (a sorted copy both kernels read). Arguments as in lora_linear_fwd.
  *
  * lora_fused_gemm: Y = X·W + (s_a·U)·B_a from the plan's scratch, which must
  * hold the output of a lora_linear_shrink with the same plan that is ordered

@@ -13,10 +13,10 @@
 // 数千大模型成为可能" without padding adapters to a common rank.
 //
 // Structure: persistent CTAs (one per SM), 6 warps:
-//   warp 0      producer: X rows (one TMA box when the tile's tokens are
-//               consecutive, else 16-byte cp.async row copies by the plan's
-//               permutation from all 32 lanes), W tile (TMA), then the tile's
-//               s·U images (bulk copy) and the matching B_pool rows (TMA)
+//   warp 0      TMA producer (lane 0): a 128-row box of X (original rows when a
+//               tile's tokens are consecutive, else the sorted copy of X the
+//               shrink wrote while gathering), the W tile, then the tile's s·U
+//               images (bulk copy) and the matching B_pool rows
 //   warp 1      MMA issuer (one thread) + TMEM owner: 128x256 fp32 accumulator,
 //               double-buffered in TMEM (512 columns) so the epilogue of tile i
 //               overlaps the main loop of tile i+1
@@ -41,7 +41,7 @@ constexpr int kStageB = kBN * kBK * 2;            // 32 KB
 constexpr int kStageBytes = kStageA + kStageB;    // 48 KB
 constexpr int kGemmThreads = 192;
 constexpr int kGemmBarBytes = 256;
-constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 4 + kBM * 16;
+constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16;
 
 enum GemmEpi { kEpiStore = 0, kEpiBwdLora = 1 };
 constexpr int kEpiRankRegs = 16;  // dU values per row kept in registers by the backward epilogue
@@ -56,7 +56,8 @@ struct GemmParams {
   const ChunkDesc *chunks;
   const int32_t *perm;
   const uint8_t *uimg;  // s·U images, one 16 KB block per 64 augmented columns
-  const uint16_t *Aptr; // the A operand's rows (X or dY), row stride K, for gathered tiles
+  int32_t a_sorted;     // 1: A rows are stored in the plan's sorted order (row td.row0 of the
+                        // A tensor map), as written by the shrink; 0: tiles are consecutive originals
   __nv_bfloat16 *out;   // [T, N]
   // backward epilogue: out += keep(t, col) / (1 - p) * sum_k dU[t, k] * A[k, col]
   const float *dU;      // [T, r]
@@ -64,6 +65,7 @@ struct GemmParams {
   int32_t r;
   uint64_t seed, thr;
   float inv_keep;
+  const int32_t *mt_order;  // m-tile visiting order (heaviest adapter work first), or null
   // K split: 1 = persistent CTAs over all tiles; S > 1 = one tile per cluster of
   // S CTAs, CTA q takes base K blocks [q*KB/S, (q+1)*KB/S) and adapter blocks
   // q, q+S, ...; partial accumulators are summed through distributed shared
@@ -71,16 +73,30 @@ struct GemmParams {
   int32_t ksplit;
 };
 
-constexpr int kRedStride = kBN + 4;  // fp32 row stride of the split-K partial in smem (padded)
+// Split-K receive slots: slot s (one per cluster rank) holds rank s's partial for
+// this CTA's 256/S columns, 128 rows, rows padded by 16 bytes so the
+// row-per-thread reads are bank-conflict free: S * 128 * (256/S + 4) * 4 bytes,
+// at most 139 KB (S = 4), inside the idle stage ring.
+__host__ __device__ constexpr int slot_stride(int S) { return kBN / S + 4; }
+__host__ __device__ constexpr int slot_bytes(int S) { return kBM * slot_stride(S) * 4; }
+constexpr int kTStride = 36;  // fp32 row stride of a warp's 32x32 transposition block
+static_assert(2 * slot_bytes(2) + 4 * 32 * kTStride * 4 <= kGemmStages * kStageBytes,
+              "receive slots and transposition blocks must fit the stage ring");
+static_assert(4 * slot_bytes(4) + 4 * 32 * kTStride * 4 <= kGemmStages * kStageBytes,
+              "receive slots and transposition blocks must fit the stage ring");
 
 // The K blocks one CTA contributes to one tile.
 struct BlockRange {
   int kb_lo, nbase;  // base blocks kb_lo .. kb_lo + nbase - 1
   int q, S, nlb;     // adapter blocks q, q + S, ... < nlb
-  __device__ __forceinline__ int count() const { return nbase + (q < nlb ? (nlb - q + S - 1) / S : 0); }
-  // index into the tile's block sequence: < KB base, >= KB adapter block (blk - KB)
+  __device__ __forceinline__ int naug() const { return q < nlb ? (nlb - q + S - 1) / S : 0; }
+  __device__ __forceinline__ int count() const { return nbase + naug(); }
+  // index into the tile's block sequence: < KB base, >= KB adapter block (blk - KB).
+  // Adapter blocks come first: their scattered B-row loads then overlap the base
+  // K loop instead of draining the pipeline at the end of the tile.
   __device__ __forceinline__ int block(int i, int KB) const {
-    return i < nbase ? kb_lo + i : KB + q + (i - nbase) * S;
+    const int na = naug();
+    return i < na ? KB + q + i * S : kb_lo + (i - na);
   }
 };
 
@@ -101,6 +117,13 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 }
 __device__ __forceinline__ void cluster_barrier() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
+}
+__device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, float4 v) {
+  uint32_t ra;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "f"(v.x), "f"(v.y), "f"(v.z),
+               "f"(v.w)
+               : "memory");
 }
 __device__ __forceinline__ void ld_dsmem_v4(uint32_t local_addr, uint32_t rank, float (&v)[4]) {
   uint32_t ra;
@@ -126,8 +149,7 @@ __device__ __forceinline__ TileDesc regular_tile(int mt, int T) {
 // B_KMAJOR: the B operand tile is K-major (backward: W^T); otherwise MN-major (W).
 template <bool B_KMAJOR, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
-    lora_gemm_kernel(const __grid_constant__ CUtensorMap mapA,    // rows of X/dY, box {64, 128}
-                     const __grid_constant__ CUtensorMap mapAg,   // rows of X, box {64, 1} (gather4)
+    lora_gemm_kernel(const __grid_constant__ CUtensorMap mapA,    // A rows (X, sorted X or dY), box {64, 128}
                      const __grid_constant__ CUtensorMap mapB,    // W
                      const __grid_constant__ CUtensorMap mapBl,   // B_pool rows, box {64, 16}
                      const GemmParams p) {
@@ -142,15 +164,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t acce0 = accf0 + 16;                        // [2]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGemmStages + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
-  int32_t *rowcache = reinterpret_cast<int32_t *>(smem + kGemmStages * kStageBytes + kGemmBarBytes);
-  int4 *chunkcache = reinterpret_cast<int4 *>(smem + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 4);
+  int4 *chunkcache = reinterpret_cast<int4 *>(smem + kGemmStages * kStageBytes + kGemmBarBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < kGemmStages; ++s) {
-      mbar_init(full0 + 8 * s, 33);  // producer lane 0 (expect_tx) + one arrival per producer lane
+      mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, 1);
     }
     for (int b = 0; b < 2; ++b) {
@@ -180,68 +201,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // -------------------------------------------------------------- producer
-    // The whole warp stages each tile's gather rows and adapter table in shared
-    // memory (no dependent global loads inside the K loop); lane 0 issues TMA.
+    // The warp stages each tile's adapter table in shared memory (no dependent
+    // global loads inside the K loop); lane 0 issues every TMA copy.
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
-      const int mt = tile % p.n_mt;
+      const int mt = p.mt_order ? p.mt_order[tile % p.n_mt] : tile % p.n_mt;
       const int nt = tile / p.n_mt;
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       const int n0 = nt * kBN;
-      if (td.contig < 0) {
-        for (int i = lane; i < kBM; i += 32) {
-          const int rr = i < td.rows ? i : td.rows - 1;  // pad rows repeat a valid row
-          rowcache[i] = p.perm[td.row0 + rr];
-        }
-      }
+      // A rows: the sorted copy written by the shrink (rows in tile order), or the
+      // original rows when the tile's tokens are consecutive originals
+      const int arow = p.a_sorted ? td.row0 : td.contig;
       for (int c = lane; c < td.nchunk; c += 32) {
         const ChunkDesc cd = p.chunks[td.chunk0 + c];
         chunkcache[c] = make_int4(cd.pool_row, cd.kofs, cd.kc, 0);
       }
       __syncwarp();
-      // Every lane runs the K loop. Each stage's full barrier expects 33 arrivals:
-      // lane 0's expect_tx arrival (TMA bytes) plus one per lane, made by the
-      // completion of the lane's cp.async row copies (gathered tiles) or by a
-      // plain arrive (everything else).
-      const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
-      const int nblk = br.count();
-      const bool gathered = td.contig < 0;
-      int c = 0;  // chunk cursor over the tile's adapter table (lane 0)
-      for (int i = 0; i < nblk; ++i) {
-        const int blk = br.block(i, KB);
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
-        const uint32_t a_dst = stage0 + stage * kStageBytes;
-        const uint32_t b_dst = a_dst + kStageA;
-        const uint32_t fb = full0 + 8 * stage;
-        if (blk < KB) {
-          const int k0 = blk * kBK;
-          if (lane == 0) {
-            mbar_arrive_expect_tx(fb, (gathered ? 0 : kStageA) + kStageB);
-            if (!gathered) tma_load_2d(a_dst, &mapA, fb, k0, td.contig);
+      if (lane == 0) {
+        if (arow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; }
+        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const int nblk = arow < 0 ? 0 : br.count();
+        int c = 0;  // chunk cursor over the tile's adapter table
+        for (int i = 0; i < nblk; ++i) {
+          const int blk = br.block(i, KB);
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
+          const uint32_t a_dst = stage0 + stage * kStageBytes;
+          const uint32_t b_dst = a_dst + kStageA;
+          const uint32_t fb = full0 + 8 * stage;
+          if (blk < KB) {
+            const int k0 = blk * kBK;
+            mbar_arrive_expect_tx(fb, kStageA + kStageB);
+            tma_load_2d(a_dst, &mapA, fb, k0, arow);
             if (B_KMAJOR) {
               tma_load_2d(b_dst, &mapB, fb, k0, n0);
             } else {
               for (int j = 0; j < kBN / 64; ++j) tma_load_2d(b_dst + j * 8192, &mapB, fb, n0 + j * 64, k0);
             }
-          }
-          if (gathered) {
-            // 128 rows x 8 16-byte chunks; a warp instruction covers 4 whole rows.
-            // Placed with the 128-byte swizzle the MMA descriptor expects.
-            const int chunk = lane & 7;
-            const bool inside = k0 + chunk * 8 < p.K;
-#pragma unroll 4
-            for (int it = 0; it < kBM / 4; ++it) {
-              const int row = it * 4 + (lane >> 3);
-              const uint16_t *src = p.Aptr + static_cast<int64_t>(rowcache[row]) * p.K + (inside ? k0 + chunk * 8 : 0);
-              cp_async_16(a_dst + row * 128 + (((chunk ^ (row & 7)) & 7) << 4), src, inside ? 16u : 0u);
-            }
-            cp_async_arrive_noinc(fb);
           } else {
-            mbar_arrive(fb);
-          }
-        } else {
-          if (lane == 0) {
             // adapter K block: 64 augmented columns (up to 4 MMA K steps). Each
             // chunk spans 2*kc columns: s*U rounded to bf16 (hi), then the
             // rounding remainder (lo); both multiply the same B rows.
@@ -261,9 +258,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 tma_load_2d(b_dst + j * 8192 + qq * 2048, &mapBl, fb, n0 + j * 64, prow);
             }
           }
-          mbar_arrive(fb);
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
         }
-        if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
       }
       __syncwarp();
     }
@@ -276,7 +272,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t aphase = 0;
       for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
-        const int mt = tile % p.n_mt;
+        const int mt = p.mt_order ? p.mt_order[tile % p.n_mt] : tile % p.n_mt;
         const int kaug = has_plan ? p.tiles[mt].kaug : 0;
         const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
         const int nblk = br.count();
@@ -288,7 +284,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int blk = br.block(i, KB);
           if (!mbar_wait(full0 + 8 * stage, phase)) { *abort_flag = 1; ok = false; break; }
           tc_fence_after();
-          fence_proxy_async_smem();  // rows written by cp.async (generic proxy) -> MMA operand reads
           const uint32_t a_s = stage0 + stage * kStageBytes;
           const uint32_t b_s = a_s + kStageA;
           const int steps = blk < KB ? 4 : min(4, (kaug - (blk - KB) * kAugBlock) / 16);
@@ -313,32 +308,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t aphase = 0;
     for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
-      const int mt = tile % p.n_mt;
+      const int mt = p.mt_order ? p.mt_order[tile % p.n_mt] : tile % p.n_mt;
       const int nt = tile / p.n_mt;
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       if (!mbar_wait(accf0 + 8 * acc, aphase)) { *abort_flag = 1; break; }
       tc_fence_after();
-      if (split) {
-        // partial accumulator -> shared memory (the stage ring is idle: every MMA
-        // of this CTA's only tile has completed); zeros if this CTA had no blocks
-        const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
-        float *red = reinterpret_cast<float *>(smem) + row * kRedStride;
-        for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem_base + ((quarter * 32) << 16) + acc * kBN + c * 32, v);
-          tmem_wait_ld();
-#pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            float4 o = any ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                         __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
-                           : make_float4(0.f, 0.f, 0.f, 0.f);
-            *reinterpret_cast<float4 *>(red + c * 32 + 4 * j) = o;
-          }
-        }
-        tc_fence_before();
-        mbar_arrive(acce0 + 8 * acc);
-        break;
-      }
+      if (split) break;  // the cluster reduction below handles the single tile
       const bool valid = row < td.rows;
       int64_t orig = 0;
       if (valid) orig = has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
@@ -409,43 +384,100 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (split) {
     // --------------------------------------------------- split-K cluster reduction
-    cluster_barrier();  // every CTA's partial is in its shared memory
+    // slot s of CTA q's shared memory holds CTA s's partial for the columns q
+    // owns; the barrier's release/acquire makes every pushed store visible
+    // barrier 1: every CTA's MMAs are complete, so every stage ring is idle
+    cluster_barrier();
+    const int width = kBN / S;
     if (warp >= 2 && tile0 < n_tiles && !*abort_flag) {
-      const int row = (warp & 3) * 32 + lane;
-      const int mt = tile0 % p.n_mt;
+      // push this CTA's partial sums for the column slices other CTAs own
+      // straight from TMEM into their receive slots (fire-and-forget stores);
+      // the slice this CTA owns stays in TMEM
+      tc_fence_after();
+      const int quarter = warp & 3;
+      const int row = quarter * 32 + lane;
+      const int mt = p.mt_order ? p.mt_order[tile0 % p.n_mt] : tile0 % p.n_mt;
+      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
+      // a warp's 32 rows x 32 columns pass through a small shared-memory block so
+      // that each remote store instruction writes 4 whole 128-byte row pieces
+      // (coalesced) instead of 32 scattered 16-byte pieces
+      float *tb = reinterpret_cast<float *>(smem + S * slot_bytes(S)) + (warp - 2) * 32 * kTStride;
+      for (int c = 0; c < kBN / 32; ++c) {
+        const int owner = (c * 32) / width;
+        if (owner == q) continue;
+        uint32_t v[32];
+        tmem_ld32(tmem_base + ((quarter * 32) << 16) + c * 32, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+          *reinterpret_cast<float4 *>(tb + lane * kTStride + 4 * j) =
+              any ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        __syncwarp();
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+          const int r = 4 * j + (lane >> 3);  // row within the warp's 32
+          const int cc = (lane & 7) * 4;      // column within the 32-column chunk
+          const float4 o = *reinterpret_cast<const float4 *>(tb + r * kTStride + cc);
+          const uint32_t dst = smem_u32(smem) +
+                               static_cast<uint32_t>(q * slot_bytes(S) + (quarter * 32 + r) * slot_stride(S) * 4 +
+                                                     (c * 32 - owner * width + cc) * 4);
+          st_dsmem_v4(dst, static_cast<uint32_t>(owner), o);
+        }
+        __syncwarp();
+      }
+    }
+    // barrier 2: every pushed store is visible to its owner (release / acquire)
+    cluster_barrier();
+    if (warp >= 2 && tile0 < n_tiles && !*abort_flag) {
+      const int quarter = warp & 3;
+      const int row = quarter * 32 + lane;
+      const int mt = p.mt_order ? p.mt_order[tile0 % p.n_mt] : tile0 % p.n_mt;
       const int nt = tile0 / p.n_mt;
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
-      if (row < td.rows) {
-        const int64_t orig = has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
-        const int width = kBN / S;
-        const int c0 = q * width;
-        const uint32_t rbase = smem_u32(smem) + static_cast<uint32_t>(row * kRedStride + c0) * 4u;
-        for (int cc = 0; cc < width; cc += 8) {
-          const int col = nt * kBN + c0 + cc;
-          if (col >= p.N) break;
-          float s[8];
+      const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
+      const bool valid = row < td.rows;
+      const int64_t orig = !valid ? 0 : has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
+      for (int c0 = 0; c0 < width; c0 += 32) {
+        uint32_t v[32];
+        tmem_ld32(tmem_base + ((quarter * 32) << 16) + q * width + c0, v);  // own partial
+        tmem_wait_ld();
+        float s[32];
 #pragma unroll
-          for (int e = 0; e < 8; ++e) s[e] = 0.f;
-          for (int pr = 0; pr < S; ++pr) {
-            float a[4], b[4];
-            ld_dsmem_v4(rbase + cc * 4, pr, a);
-            ld_dsmem_v4(rbase + cc * 4 + 16, pr, b);
+        for (int e = 0; e < 32; ++e) s[e] = any ? __uint_as_float(v[e]) : 0.f;
+        // add the other ranks' partials in rank order (fixed order: deterministic)
+        for (int src = 0; src < S; ++src) {
+          if (src == q) continue;
+          const float4 *slot = reinterpret_cast<const float4 *>(
+              smem + src * slot_bytes(S) + (row * slot_stride(S) + c0) * 4);
 #pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              s[e] += a[e];
-              s[4 + e] += b[e];
+          for (int j = 0; j < 8; ++j) {
+            const float4 t = slot[j];
+            s[4 * j + 0] += t.x;
+            s[4 * j + 1] += t.y;
+            s[4 * j + 2] += t.z;
+            s[4 * j + 3] += t.w;
+          }
+        }
+        const int col = nt * kBN + q * width + c0;
+        if (valid) {
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            if (col + 8 * h < p.N) {
+              uint4 o;
+              o.x = pack_bf16x2(s[8 * h + 0], s[8 * h + 1]);
+              o.y = pack_bf16x2(s[8 * h + 2], s[8 * h + 3]);
+              o.z = pack_bf16x2(s[8 * h + 4], s[8 * h + 5]);
+              o.w = pack_bf16x2(s[8 * h + 6], s[8 * h + 7]);
+              *reinterpret_cast<uint4 *>(p.out + orig * p.N + col + 8 * h) = o;
             }
           }
-          uint4 o;
-          o.x = pack_bf16x2(s[0], s[1]);
-          o.y = pack_bf16x2(s[2], s[3]);
-          o.z = pack_bf16x2(s[4], s[5]);
-          o.w = pack_bf16x2(s[6], s[7]);
-          *reinterpret_cast<uint4 *>(p.out + orig * p.N + col) = o;
         }
       }
     }
-    cluster_barrier();  // peers keep their shared memory until every read is done
+    cluster_barrier();  // barrier 3: no CTA exits while a peer may still read it
   }
   if (warp == 1) {
     __syncwarp();

@@ -53,9 +53,11 @@ struct HostPlan {
   std::vector<TileDesc> tiles;
   std::vector<ChunkDesc> chunks;
   std::vector<UnitDesc> units;
+  std::vector<int32_t> mt_order;  // m-tiles by decreasing adapter work (stable)
   int32_t r_max = 0;
   int64_t sum_r_used = 0, sum_r_tokens = 0, aug_k_total = 0;
   int64_t scratch_bytes = 0;
+  int64_t xs_offset = -1;  // byte offset of the sorted copy of X in the scratch (-1: not needed)
   int32_t max_chunk_rows = 0;
 };
 

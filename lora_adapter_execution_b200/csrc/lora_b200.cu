@@ -104,16 +104,16 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_
 // Forward GEMM launch: persistent CTAs when there are enough output tiles to
 // fill the GPU; otherwise clusters of S CTAs split the K loop of each tile
 // (S a power of two, S * tiles <= SMs, S <= number of K blocks).
-int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const CUtensorMap &ag,
-                    const CUtensorMap &b, const CUtensorMap &bl, lora_stream_t stream) {
+int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const CUtensorMap &b,
+                    const CUtensorMap &bl, lora_stream_t stream) {
   const int n_tiles = gp.n_mt * gp.n_nt;
   const int KB = (gp.K + kBK - 1) / kBK;
   int S = 1;
-  while (S < 4 && 2 * S * n_tiles <= ds->num_sms && 2 * S <= KB) S *= 2;
+  while (S < 4 && 2 * S * n_tiles <= ds->num_sms && 2 * S <= KB) S *= 2;  // S in {1, 2, 4}
   gp.ksplit = S;
   if (S == 1) {
     const int grid = std::min(ds->num_sms, n_tiles);
-    lora_gemm_kernel<false, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(a, ag, b, bl, gp);
+    lora_gemm_kernel<false, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(a, b, bl, gp);
     return launch_status();
   }
   cudaLaunchConfig_t cfg{};
@@ -128,7 +128,7 @@ int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const 
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, lora_gemm_kernel<false, kEpiStore>, a, ag, b, bl, gp) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, lora_gemm_kernel<false, kEpiStore>, a, b, bl, gp) != cudaSuccess) {
     cudaGetLastError();
     return LORA_ERR_CUDA;
   }
@@ -145,6 +145,7 @@ struct lora_plan {
   const TileDesc *d_tiles = nullptr;
   const ChunkDesc *d_chunks = nullptr;
   const UnitDesc *d_units = nullptr;
+  const int32_t *d_mt_order = nullptr;
   int device = 0;
 };
 
@@ -188,7 +189,8 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   const size_t b_tiles = up(sizeof(TileDesc) * hp.tiles.size());
   const size_t b_chunks = up(sizeof(ChunkDesc) * hp.chunks.size());
   const size_t b_units = up(sizeof(UnitDesc) * hp.units.size());
-  const size_t total = b_perm + b_tiles + b_chunks + b_units;
+  const size_t b_order = up(sizeof(int32_t) * hp.mt_order.size());
+  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order;
   if (cudaMalloc(&pl->dev, total) != cudaSuccess) {
     cudaGetLastError();
     delete pl;
@@ -205,6 +207,7 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   pl->d_tiles = reinterpret_cast<const TileDesc *>(base + b_perm);
   pl->d_chunks = reinterpret_cast<const ChunkDesc *>(base + b_perm + b_tiles);
   pl->d_units = reinterpret_cast<const UnitDesc *>(base + b_perm + b_tiles + b_chunks);
+  pl->d_mt_order = reinterpret_cast<const int32_t *>(base + b_perm + b_tiles + b_chunks + b_units);
   bool ok = true;
   ok &= cudaMemcpyAsync(base, hp.perm.data(), sizeof(int32_t) * hp.perm.size(), cudaMemcpyHostToDevice,
                         stream) == cudaSuccess;
@@ -214,6 +217,8 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
                         cudaMemcpyHostToDevice, stream) == cudaSuccess;
   ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks, hp.units.data(), sizeof(UnitDesc) * hp.units.size(),
                         cudaMemcpyHostToDevice, stream) == cudaSuccess;
+  ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks + b_units, hp.mt_order.data(),
+                        sizeof(int32_t) * hp.mt_order.size(), cudaMemcpyHostToDevice, stream) == cudaSuccess;
   // the copies read host vectors that the plan keeps alive; make sure they have
   // been consumed before returning so the caller may reuse its stream freely
   ok &= cudaStreamSynchronize(stream) == cudaSuccess;
@@ -285,10 +290,10 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   if (rc != LORA_OK) return rc;
   const HostPlan &hp = plan->hp;
   const int64_t R = hp.offsets[hp.n_adapters];
-  CUtensorMap mXg, mX16, mA16;
+  CUtensorMap mX16, mA16;
+  uint16_t *Xs = hp.xs_offset >= 0 ? reinterpret_cast<uint16_t *>(plan->scratch + hp.xs_offset) : nullptr;
   bool ok = true;
-  ok &= make_map(&mXg, X, hp.d_in, hp.T, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&mX16, X, hp.d_in, hp.T, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&mX16, Xs ? Xs : X, hp.d_in, hp.T, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mA16, A_pool, hp.d_in, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return LORA_ERR_ARG;
   ShrinkParams sp{};
@@ -311,7 +316,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   sp.seed = seed;
   sp.inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
   sp.uimg = plan->scratch;
-  sp.In = X;
+  sp.x_sorted = Xs ? 1 : 0;
   sp.U_save = U_save;
   sp.r_max = hp.r_max;
   cudaLaunchConfig_t cfg{};
@@ -326,7 +331,14 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mX16, mXg, mA16, sp) != cudaSuccess) {
+  if (Xs) {
+    // sorted copy of X first (the shrink and the fused GEMM read token tiles from it)
+    const int64_t pieces = hp.T * (hp.d_in / 8);
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((pieces + 255) / 256, 8 * ds->num_sms));
+    lora_gather_rows_kernel<<<blocks, 256, 0, stream>>>(X, plan->d_perm, Xs, hp.T, hp.d_in);
+    if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+  }
+  if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mX16, mA16, sp) != cudaSuccess) {
     cudaGetLastError();
     return LORA_ERR_CUDA;
   }
@@ -342,10 +354,11 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   if (rc != LORA_OK) return rc;
   const HostPlan &hp = plan->hp;
   const int64_t R = hp.offsets[hp.n_adapters];
-  CUtensorMap mX128, mXg, mW, mBl;
+  CUtensorMap mX128, mW, mBl;
+  const bool sorted = hp.xs_offset >= 0;
+  const void *Asrc = sorted ? static_cast<const void *>(plan->scratch + hp.xs_offset) : static_cast<const void *>(X);
   bool ok = true;
-  ok &= make_map(&mX128, X, hp.d_in, hp.T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&mXg, X, hp.d_in, hp.T, 64, 1, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&mX128, Asrc, hp.d_in, hp.T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mW, W, hp.d_out, hp.d_in, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mBl, B_pool, hp.d_out, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return LORA_ERR_ARG;
@@ -359,9 +372,10 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   gp.chunks = plan->d_chunks;
   gp.perm = plan->d_perm;
   gp.uimg = plan->scratch;
-  gp.Aptr = X;
+  gp.mt_order = plan->d_mt_order;
+  gp.a_sorted = sorted ? 1 : 0;
   gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
-  return launch_fwd_gemm(ds, gp, mX128, mXg, mW, mBl, stream);
+  return launch_fwd_gemm(ds, gp, mX128, mW, mBl, stream);
 }
 
 int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
@@ -394,9 +408,9 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
   gp.N = static_cast<int32_t>(d_out);
   gp.n_mt = static_cast<int32_t>((T + kBM - 1) / kBM);
   gp.n_nt = static_cast<int32_t>((d_out + kBN - 1) / kBN);
-  gp.Aptr = X;
+  gp.a_sorted = 0;
   gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
-  return launch_fwd_gemm(ds, gp, mX128, mX128, mW, mW, stream);
+  return launch_fwd_gemm(ds, gp, mX128, mW, mW, stream);
 }
 
 // Workspace layout: dU f32 [T, r] | dB partial [S, r, d_out] | dA partial [S, r, d_in]
@@ -463,7 +477,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     sp.r = r;
     sp.npieces = (((r + 15) / 16) * 16 + kShrinkN - 1) / kShrinkN;
     sp.scale1 = scale;
-    sp.In = dY;
+    sp.x_sorted = 0;
     sp.dU = dU;
     const int n_units = static_cast<int>((T + kTileM - 1) / kTileM) * sp.npieces;
     int ks = std::max(1, std::min(4, (2 * ds->num_sms + n_units - 1) / n_units));
@@ -484,7 +498,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mdY16, mdY16, mB16, sp) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mdY16, mB16, sp) != cudaSuccess) {
       cudaGetLastError();
       return LORA_ERR_CUDA;
     }
@@ -497,7 +511,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.N = static_cast<int32_t>(d_in);
     gp.n_mt = static_cast<int32_t>((T + kBM - 1) / kBM);
     gp.n_nt = static_cast<int32_t>((d_in + kBN - 1) / kBN);
-    gp.Aptr = dY;
+    gp.a_sorted = 0;
     gp.out = reinterpret_cast<__nv_bfloat16 *>(dX);
     gp.dU = dU;
     gp.A = A;
@@ -507,7 +521,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.inv_keep = inv_keep;
     gp.ksplit = 1;
     const int grid = std::min(ds->num_sms, gp.n_mt * gp.n_nt);
-    lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mdY128, mWt, mWt, gp);
+    lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mWt, gp);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
   // K3c: dB = s * U^T * dY and dA = (D ⊙ X)^T * dU, split over tokens, then reduced

@@ -104,7 +104,22 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
     hp.aug_k_total += td.kaug;
     hp.tiles.push_back(td);
   }
+  // Tiles whose tokens are not consecutive originals read X through a sorted
+  // copy that the shrink writes while it gathers the rows anyway.
+  bool any_gathered = false;
+  for (const TileDesc &td : hp.tiles) any_gathered |= td.contig < 0;
+  if (any_gathered) {
+    hp.xs_offset = (uofs + 255) / 256 * 256;
+    uofs = hp.xs_offset + T * d_in * 2;
+  }
   hp.scratch_bytes = uofs;
+
+  // Visiting order of m-tiles for the persistent GEMM: most augmented K first, so
+  // the heavy tiles (many small adapters) start early instead of ending last.
+  hp.mt_order.resize(hp.tiles.size());
+  for (size_t m = 0; m < hp.tiles.size(); ++m) hp.mt_order[m] = (int32_t)m;
+  std::stable_sort(hp.mt_order.begin(), hp.mt_order.end(),
+                   [&](int32_t a, int32_t b) { return hp.tiles[a].kaug > hp.tiles[b].kaug; });
 
   // Shrink units: each chunk's rank columns in pieces of at most 64.
   for (int32_t c = 0; c < (int32_t)hp.chunks.size(); ++c) {

@@ -8,6 +8,8 @@
 //    works on the skinny rank dimension. The d_in contraction is split across
 //    the CTAs of a thread-block cluster and summed through distributed shared
 //    memory, so a small adapter run still spreads its bytes over several SMs.
+//    Tokens of one adapter are consecutive rows either of X or of the sorted
+//    copy of X that lora_gather_rows_kernel writes first.
 //    Forward output: the tile's s·U block, already in the 128-byte-swizzled
 //    shared-memory image the fused GEMM's MMA reads, plus U for the backward.
 //  * lora_tcontract_kernel: partial[q][k][n] = sum_{t in split q} G[t, k] * In[t, n]
@@ -34,14 +36,14 @@ constexpr int kSkBK = 64;                                 // columns per stage (
 constexpr int kSkPool = 72 * 1024;                        // stage ring (also the reduction scratch)
 constexpr int kSkMaxStages = 16;
 constexpr int kSkFinBytes = kTileM * kShrinkN * 4;        // CTA partial [128 x 64] fp32
-constexpr int kSkSmem = 1024 + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64 + kTileM * 4;
+constexpr int kSkSmem = 1024 + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64;
 
 struct ShrinkParams {
   int32_t mode;     // 0: forward shrink over plan units; 1: backward dU over consecutive tiles
   int32_t T, K;     // tokens, contraction length
   int32_t ksplit;   // cluster size along the contraction
   int32_t kslice;   // contraction columns per cluster rank (multiple of kSkBK)
-  const uint16_t *In;  // rows of the contracted input (X or dY), row stride K
+  int32_t x_sorted;   // 1: the In tensor map covers the plan's sorted copy of X (unit rows at g.row0)
   // forward
   const UnitDesc *units;
   const ChunkDesc *chunks;
@@ -158,8 +160,7 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
 // Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
 // its rank q contracts columns [q*kslice, (q+1)*kslice).
 __global__ void __launch_bounds__(kSkThreads, 2)
-    lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows, box {64, 16}
-                       const __grid_constant__ CUtensorMap mapInG,   // unused (kept for the launch signature)
+    lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows (X, sorted X or dY), box {64, 16}
                        const __grid_constant__ CUtensorMap mapF16,   // F rows, box {64, 16}
                        const ShrinkParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -171,7 +172,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * kSkMaxStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kSkMaxStages);
-  int32_t *rowcache = reinterpret_cast<int32_t *>(smem + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
-      mbar_init(full0 + 8 * s, 33);
+      mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, kSkConsumerWarps);
     }
     *abort_flag = 0;
@@ -213,40 +213,25 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 
   if (warp == kSkConsumerWarps) {
     // -------------------------------------------------------------- producer
-    if (g.contig < 0) {
-      for (int i = lane; i < Rp; i += 32) rowcache[i] = p.perm[g.row0 + min(i, g.rows - 1)];
-    }
-    __syncwarp();
-    // all lanes run the stage loop: lane 0 issues the TMA boxes (F rows, and X
-    // rows of consecutive tokens); gathered X rows are 16-byte cp.async copies
-    // from every lane. Full barriers expect 33 arrivals (see the GEMM producer).
-    int stage = 0;
-    uint32_t phase = 0;
-    const bool gathered = g.contig < 0;
-    for (int b = 0; b < nblk; ++b) {
-      if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
-      const uint32_t fb = full0 + 8 * stage;
-      const uint32_t xb = pool + stage * stage_bytes;
-      const uint32_t fbuf = xb + Rp * 128;
-      const int col = kbeg + b * kSkBK;
-      if (lane == 0) {
-        mbar_arrive_expect_tx(fb, (gathered ? 0 : Rp * 128) + g.nn * 128);
-        if (!gathered)
-          for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, g.contig + r16);
+    // Lane 0 streams the unit's X rows (16-row TMA boxes: the rows are
+    // consecutive either in X itself or in the plan's sorted copy of X) and
+    // the adapter's F rows through the stage ring.
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0;
+      const int xrow = p.x_sorted ? g.row0 : g.contig;
+      for (int b = 0; b < nblk; ++b) {
+        if (xrow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; break; }
+        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
+        const uint32_t fb = full0 + 8 * stage;
+        const uint32_t xb = pool + stage * stage_bytes;
+        const uint32_t fbuf = xb + Rp * 128;
+        const int col = kbeg + b * kSkBK;
+        mbar_arrive_expect_tx(fb, stage_bytes);
+        for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, xrow + r16);
         for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
+        if (++stage == nstage) { stage = 0; phase ^= 1; }
       }
-      if (gathered) {
-        const int chunk = lane & 7;
-        const bool inside = col + chunk * 8 < p.K;
-        for (int row = lane >> 3; row < Rp; row += 4) {
-          const uint16_t *src = p.In + static_cast<int64_t>(rowcache[row]) * p.K + (inside ? col + chunk * 8 : 0);
-          cp_async_16(xb + row * 128 + (((chunk ^ (row & 7)) & 7) << 4), src, inside ? 16u : 0u);
-        }
-        cp_async_arrive_noinc(fb);
-      } else {
-        mbar_arrive(fb);
-      }
-      if (++stage == nstage) { stage = 0; phase ^= 1; }
     }
   } else {
     // -------------------------------------------------------------- consumers
@@ -568,6 +553,22 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
       }
     }
+  }
+}
+
+// Xs[i, :] = X[perm[i], :]: the plan's sorted copy of X, so every later load of a
+// token tile (shrink and fused GEMM) is one TMA box instead of a row gather.
+// Each thread copies 16-byte pieces; consecutive threads cover consecutive
+// pieces of a row, so reads and writes are fully coalesced.
+__global__ void lora_gather_rows_kernel(const uint16_t *__restrict__ X, const int32_t *__restrict__ perm,
+                                        uint16_t *__restrict__ Xs, int64_t T, int64_t d) {
+  const int64_t per_row = d / 8;
+  const int64_t n = T * per_row;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / per_row, c = e % per_row;
+    const uint4 v = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<int64_t>(perm[i]) * d) + c);
+    reinterpret_cast<uint4 *>(Xs + i * d)[c] = v;
   }
 }
 

@@ -46,12 +46,19 @@ def test_plan_fuzz():
         # augmented K: every tile adds, per adapter present, twice its rank
         # rounded up to 16 (bf16 hi and lo parts of s*U)
         kaug = 0
+        images = 0
+        gathered = False
         for m in range(info["n_tiles"]):
             pos = perm[m * 128:(m + 1) * 128]
-            for a in np.unique(ids[pos]):
-                kaug += 2 * (-(-int(ranks[a]) // 16) * 16)
+            kt = sum(2 * (-(-int(ranks[a]) // 16) * 16) for a in np.unique(ids[pos]))
+            kaug += kt
+            images += -(-kt // 64) * 16384
+            gathered |= not (np.diff(pos) == 1).all()
         assert info["aug_k_total"] == kaug
-        assert info["scratch_bytes"] % 16384 == 0
+        # scratch: the s*U images, then (if some tile's tokens are not consecutive
+        # originals) a sorted copy of X (T x d_in bf16), 256-byte aligned
+        want = images if not gathered else -(-images // 256) * 256 + T * 64 * 2
+        assert info["scratch_bytes"] == want
 
 
 def test_workload_tile_statistics():
