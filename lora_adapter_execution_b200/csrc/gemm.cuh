@@ -395,7 +395,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // the slice this CTA owns stays in TMEM
       tc_fence_after();
       const int quarter = warp & 3;
-      const int row = quarter * 32 + lane;
       const int mt = p.mt_order ? p.mt_order[tile0 % p.n_mt] : tile0 % p.n_mt;
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
