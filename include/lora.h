@@ -218,6 +218,41 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
                     int64_t d_in, int64_t d_out, int32_t r, void *workspace,
                     size_t workspace_bytes, lora_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * lora_linear_bwd_static — lora_linear_bwd without a caller workspace.
+ *
+ * No counterpart on the pages: this is an integration aid. Some callers cannot
+ * allocate device memory at the point where they run the backward: a process
+ * whose whole device memory is owned by another allocator (a framework's
+ * caching allocator, or an arena a serving process reserves at start-up), where
+ * an extra cudaMalloc fails or fragments that pool; plugins hosted by a program
+ * that gives them no allocator; and code that must not allocate once it is
+ * running (fixed-memory or real-time deployments). This entry point takes the
+ * same arguments as lora_linear_bwd except the workspace and allocates nothing:
+ * its scratch is a file-scope device array of LORA_BWD_STATIC_SCRATCH_BYTES
+ * bytes inside the library, which every GPU that loads the library holds until
+ * the process exits.
+ *
+ *  - Requests whose workspace need (lora_linear_bwd_workspace_size) exceeds
+ *    LORA_BWD_STATIC_SCRATCH_BYTES are rejected with LORA_ERR_WORKSPACE before
+ *    anything is launched.
+ *  - The first call on a device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before any stream capture on the device.
+ *  - Every call shares the one array, and the array keeps what the last call
+ *    left in it. Nothing in it needs to start at zero: each call writes every
+ *    scratch byte it later reads. Calls that overlap on the GPU (different
+ *    streams, or different host threads, without ordering between them) race
+ *    on the array and give wrong results; order them.
+ * Errors: as lora_linear_bwd.
+ * ------------------------------------------------------------------------ */
+#define LORA_BWD_STATIC_SCRATCH_BYTES ((size_t)8 << 20) /* 8 MiB */
+
+int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B,
+                           float scale, double p_drop, uint64_t seed, const float *U_save,
+                           const uint16_t *dY, uint16_t *dX, float *dA, float *dB, int64_t T,
+                           int64_t d_in, int64_t d_out, int32_t r, lora_stream_t stream);
+
 /* Test hook: write the dropout mask the forward and backward use.
  *   mask_dev  uint8 [T, d_in] device: 1 where X[t, i] is dropped, else 0.
  * Errors: LORA_ERR_ARG, LORA_ERR_CUDA. */

@@ -72,6 +72,8 @@ def load_library():
         "lora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
         "lora_linear_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _f32, _dbl, _u64, _vp, _vp, _vp, _vp, _vp,
                                            _i64, _i64, _i64, _i32, _vp, _sz, _vp]),
+        "lora_linear_bwd_static": (ctypes.c_int, [_vp, _vp, _vp, _vp, _f32, _dbl, _u64, _vp, _vp, _vp, _vp, _vp,
+                                                  _i64, _i64, _i64, _i32, _vp]),
         "lora_dropout_mask": (ctypes.c_int, [_u64, _dbl, _i64, _i64, _vp, _vp]),
         "lora_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
         "lora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _vp, _vp]),
@@ -196,6 +198,20 @@ def linear_bwd(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, workspace, *, p
                                           int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY), _ptr(dX), _ptr(dA),
                                           _ptr(dB), T, d_in, d_out, r, _ptr(workspace), nbytes, _stream(stream)),
            "lora_linear_bwd")
+
+
+def linear_bwd_static(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, *, p_drop: float = 0.0,
+                      seed: int = 0, stream=None):
+    """lora_linear_bwd_static: the backward without a caller workspace (for callers
+    that cannot allocate device memory); see include/lora.h for its limit and
+    sharing rules."""
+    T, d_in = X.shape
+    d_out = W.shape[1]
+    r = A.shape[0]
+    _check(load_library().lora_linear_bwd_static(_ptr(X), _ptr(W), _ptr(A), _ptr(B), float(scale), float(p_drop),
+                                                 int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY), _ptr(dX),
+                                                 _ptr(dA), _ptr(dB), T, d_in, d_out, r, _stream(stream)),
+           "lora_linear_bwd_static")
 
 
 def dropout_mask(seed: int, p_drop: float, mask, *, stream=None):

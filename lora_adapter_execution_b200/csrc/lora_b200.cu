@@ -557,6 +557,39 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
   return launch_status();
 }
 
+}  // extern "C"
+
+// Scratch of lora_linear_bwd_static: one array per device, shared by every
+// call; host code must not use its name as an address (that is a host-side
+// stand-in), so the device address is looked up once per device below.
+static __device__ __align__(256) uint8_t g_bwd_static_scratch[LORA_BWD_STATIC_SCRATCH_BYTES];
+static void *g_bwd_static_ptr[kMaxDevices];
+
+extern "C" {
+
+int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B,
+                           float scale, double p_drop, uint64_t seed, const float *U_save, const uint16_t *dY,
+                           uint16_t *dX, float *dA, float *dB, int64_t T, int64_t d_in, int64_t d_out, int32_t r,
+                           lora_stream_t stream) {
+  const size_t need = lora_linear_bwd_workspace_size(T, d_in, d_out, r);
+  if (need > LORA_BWD_STATIC_SCRATCH_BYTES) return LORA_ERR_WORKSPACE;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_ERR_CUDA;
+  if (!g_bwd_static_ptr[dev]) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_bwd_static_ptr[dev]) {
+      void *ptr = nullptr;
+      if (cudaGetSymbolAddress(&ptr, g_bwd_static_scratch) != cudaSuccess || !ptr) {
+        cudaGetLastError();
+        return LORA_ERR_CUDA;
+      }
+      g_bwd_static_ptr[dev] = ptr;
+    }
+  }
+  return lora_linear_bwd(X, W, A, B, scale, p_drop, seed, U_save, dY, dX, dA, dB, T, d_in, d_out, r,
+                         g_bwd_static_ptr[dev], LORA_BWD_STATIC_SCRATCH_BYTES, stream);
+}
+
 int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint8_t *mask_dev,
                       lora_stream_t stream) {
   if (!mask_dev || T <= 0 || d_in <= 0 || !(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
