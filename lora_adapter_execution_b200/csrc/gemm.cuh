@@ -39,6 +39,9 @@ constexpr int kGemmStages = 4;
 constexpr int kStageA = kBM * kBK * 2;            // 16 KB
 constexpr int kStageB = kBN * kBK * 2;            // 32 KB
 constexpr int kStageBytes = kStageA + kStageB;    // 48 KB
+// An adapter block's B operand: up to four 8 KB slots, each one 16-row slice of
+// B_pool over the tile's 256 columns, stored [4 column blocks][16 rows][64 cols].
+constexpr int kBSlot = 4 * 16 * 128;
 constexpr int kGemmThreads = 192;
 constexpr int kGemmBarBytes = 256;
 constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16;
@@ -66,6 +69,9 @@ struct GemmParams {
   uint64_t seed, thr;
   float inv_keep;
   const int32_t *mt_order;  // m-tile visiting order (heaviest adapter work first), or null
+  int32_t group_m;          // m-tiles per group of the tile visiting order (>= 1)
+  int32_t b3d;              // 1: mapBl is the 3-D view {64, rows, N/64} (N % 64 == 0) and one
+                            // copy fills a B slot; 0: mapBl is 2-D {64, 16}, four copies per slot
   // K split: 1 = persistent CTAs over all tiles; S > 1 = one tile per cluster of
   // S CTAs, CTA q takes base K blocks [q*KB/S, (q+1)*KB/S) and adapter blocks
   // q, q+S, ...; partial accumulators are summed through distributed shared
@@ -134,6 +140,24 @@ __device__ __forceinline__ void ld_dsmem_v4(uint32_t local_addr, uint32_t rank, 
                : "memory");
 }
 
+// Output tile visiting order: tiles come in groups of group_m m-tiles; inside a
+// group the m index runs fastest. The CTAs that run at the same time then share
+// a few row blocks of A and a few column blocks of B through L2, and a group's A
+// rows stay in L2 while its n-tiles are swept (A read from DRAM about once, B
+// about n_mt / group_m times). The m-tile index goes through mt_order when the
+// plan has one.
+__device__ __forceinline__ void tile_coords(int tile, const GemmParams &p, int &mt, int &nt) {
+  const int G = p.group_m;
+  const int per_group = G * p.n_nt;
+  const int g = tile / per_group;
+  const int r = tile - g * per_group;
+  const int m0 = g * G;
+  const int gm = min(G, p.n_mt - m0);
+  const int mi = m0 + r % gm;
+  nt = r / gm;
+  mt = p.mt_order ? p.mt_order[mi] : mi;
+}
+
 __device__ __forceinline__ TileDesc regular_tile(int mt, int T) {
   TileDesc td;
   td.row0 = mt * kBM;
@@ -151,7 +175,7 @@ template <bool B_KMAJOR, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     lora_gemm_kernel(const __grid_constant__ CUtensorMap mapA,    // A rows (X, sorted X or dY), box {64, 128}
                      const __grid_constant__ CUtensorMap mapB,    // W
-                     const __grid_constant__ CUtensorMap mapBl,   // B_pool rows, box {64, 16}
+                     const __grid_constant__ CUtensorMap mapBl,   // B_pool rows, box {64, 16(, 4)}
                      const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -164,6 +188,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const uint32_t acce0 = accf0 + 16;                        // [2]
   uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(bars + 2 * kGemmStages + 4);
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
+  // per stage: the B slot each K step of an adapter block reads (2 bits per step)
+  volatile uint32_t *bmap = tmem_slot + 2;
   int4 *chunkcache = reinterpret_cast<int4 *>(smem + kGemmStages * kStageBytes + kGemmBarBytes);
 
   const int warp = threadIdx.x >> 5;
@@ -206,8 +232,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int stage = 0;
     uint32_t phase = 0;
     for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
-      const int mt = p.mt_order ? p.mt_order[tile % p.n_mt] : tile % p.n_mt;
-      const int nt = tile / p.n_mt;
+      int mt, nt;
+      tile_coords(tile, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       const int n0 = nt * kBN;
       // A rows: the sorted copy written by the shrink (rows in tile order), or the
@@ -241,21 +267,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           } else {
             // adapter K block: 64 augmented columns (up to 4 MMA K steps). Each
             // chunk spans 2*kc columns: s*U rounded to bf16 (hi), then the
-            // rounding remainder (lo); both multiply the same B rows.
+            // rounding remainder (lo); both multiply the same B rows, so each
+            // distinct 16-row slice of B_pool is copied once, into its own slot.
             const int lb = blk - KB;
             const int steps = min(4, (td.kaug - lb * kAugBlock) / 16);
-            mbar_arrive_expect_tx(fb, kStageA + steps * (kBN / 64) * 2048);
+            int prow_s[4] = {0, 0, 0, 0};
+            int nslot = 0;
+            uint32_t map = 0;
+#pragma unroll
+            for (int qq = 0; qq < 4; ++qq) {
+              if (qq < steps) {
+                const int kq = lb * kAugBlock + qq * 16;
+                while (c + 1 < td.nchunk && kq >= chunkcache[c].y + 2 * chunkcache[c].z) ++c;
+                const int4 cc = chunkcache[c];
+                int o = kq - cc.y;
+                if (o >= cc.z) o -= cc.z;
+                const int prow = cc.x + o;
+                int s = nslot;
+#pragma unroll
+                for (int u = 0; u < 4; ++u)
+                  if (u < nslot && prow_s[u] == prow && s == nslot) s = u;
+                if (s == nslot) {
+#pragma unroll
+                  for (int u = 0; u < 4; ++u)
+                    if (u == nslot) prow_s[u] = prow;
+                  ++nslot;
+                }
+                map |= static_cast<uint32_t>(s) << (2 * qq);
+              }
+            }
+            bmap[stage] = map;  // published to the MMA thread by the release arrive below
+            mbar_arrive_expect_tx(fb, kStageA + nslot * kBSlot);
             bulk_g2s(a_dst, p.uimg + td.uofs + static_cast<int64_t>(lb) * kAugBlockBytes, kAugBlockBytes,
                      fb);
-            for (int qq = 0; qq < steps; ++qq) {
-              const int kq = lb * kAugBlock + qq * 16;
-              while (c + 1 < td.nchunk && kq >= chunkcache[c].y + 2 * chunkcache[c].z) ++c;
-              const int4 cc = chunkcache[c];
-              int o = kq - cc.y;
-              if (o >= cc.z) o -= cc.z;
-              const int prow = cc.x + o;
-              for (int j = 0; j < kBN / 64; ++j)
-                tma_load_2d(b_dst + j * 8192 + qq * 2048, &mapBl, fb, n0 + j * 64, prow);
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+              if (u < nslot) {
+                if (p.b3d) {
+                  tma_load_3d(b_dst + u * kBSlot, &mapBl, fb, 0, prow_s[u], n0 / 64);
+                } else {
+                  for (int j = 0; j < kBN / 64; ++j)
+                    tma_load_2d(b_dst + u * kBSlot + j * 2048, &mapBl, fb, n0 + j * 64, prow_s[u]);
+                }
+              }
             }
           }
           if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
@@ -272,7 +326,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       int acc = 0;
       uint32_t aphase = 0;
       for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
-        const int mt = p.mt_order ? p.mt_order[tile % p.n_mt] : tile % p.n_mt;
+        int mt, nt;
+        tile_coords(tile, p, mt, nt);
         const int kaug = has_plan ? p.tiles[mt].kaug : 0;
         const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
         const int nblk = br.count();
@@ -286,11 +341,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           tc_fence_after();
           const uint32_t a_s = stage0 + stage * kStageBytes;
           const uint32_t b_s = a_s + kStageA;
-          const int steps = blk < KB ? 4 : min(4, (kaug - (blk - KB) * kAugBlock) / 16);
+          const bool aug = blk >= KB;
+          const int steps = aug ? min(4, (kaug - (blk - KB) * kAugBlock) / 16) : 4;
+          const uint32_t map = aug ? bmap[stage] : 0u;
           for (int qq = 0; qq < steps; ++qq) {
             const uint64_t ad = sdesc_sw128(a_s + qq * 32, 16, 1024);
-            const uint64_t bd = B_KMAJOR ? sdesc_sw128(b_s + qq * 32, 16, 1024)
-                                         : sdesc_sw128(b_s + qq * 2048, 8192, 1024);
+            // MN-major B: base blocks are [4 column blocks][64 rows][64 cols]
+            // (column-block stride 8 KB); adapter slots are [4][16][64] (2 KB)
+            const uint64_t bd =
+                B_KMAJOR ? sdesc_sw128(b_s + qq * 32, 16, 1024)
+                : aug    ? sdesc_sw128(b_s + ((map >> (2 * qq)) & 3u) * kBSlot, 2048, 1024)
+                         : sdesc_sw128(b_s + qq * 2048, 8192, 1024);
             umma_bf16(d_tmem, ad, bd, kIdesc, (i > 0 || qq > 0) ? 1u : 0u);
           }
           umma_commit(empty0 + 8 * stage);
@@ -308,8 +369,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     int acc = 0;
     uint32_t aphase = 0;
     for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
-      const int mt = p.mt_order ? p.mt_order[tile % p.n_mt] : tile % p.n_mt;
-      const int nt = tile / p.n_mt;
+      int mt, nt;
+      tile_coords(tile, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       if (!mbar_wait(accf0 + 8 * acc, aphase)) { *abort_flag = 1; break; }
       tc_fence_after();
@@ -395,7 +456,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // the slice this CTA owns stays in TMEM
       tc_fence_after();
       const int quarter = warp & 3;
-      const int mt = p.mt_order ? p.mt_order[tile0 % p.n_mt] : tile0 % p.n_mt;
+      int mt, nt;
+      tile_coords(tile0, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
       // a warp's 32 rows x 32 columns pass through a small shared-memory block so
@@ -433,8 +495,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (warp >= 2 && tile0 < n_tiles && !*abort_flag) {
       const int quarter = warp & 3;
       const int row = quarter * 32 + lane;
-      const int mt = p.mt_order ? p.mt_order[tile0 % p.n_mt] : tile0 % p.n_mt;
-      const int nt = tile0 / p.n_mt;
+      int mt, nt;
+      tile_coords(tile0, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
       const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
       const bool valid = row < td.rows;

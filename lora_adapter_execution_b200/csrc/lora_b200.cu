@@ -97,7 +97,32 @@ bool make_map_f32(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, 
   return r == CUDA_SUCCESS;
 }
 
+// 3-D view {64, rows, cols / 64} of a row-major bf16 [rows x cols] matrix
+// (cols % 64 == 0): one box {64, box_rows, blocks} copies `blocks` consecutive
+// 64-column blocks of `box_rows` rows, each block stored as [box_rows][64].
+bool make_map_blocks(CUtensorMap *m, const void *base, int64_t cols, int64_t rows, uint32_t box_rows,
+                     uint32_t blocks) {
+  cuuint64_t dims[3] = {64, static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(cols / 64)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(cols) * 2, 128};
+  cuuint32_t box[3] = {64, box_rows, blocks};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = g_encode(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+                        estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// m-tiles per group of the GEMM tile order: a group's 128-row blocks of A take
+// about 16 MB, so they stay in L2 while its n-tiles run (on 8192 x 4096 x 11008
+// this cut DRAM reads of the base GEMM from 853 MB to 428 MB; on 16384 x 4096 x
+// 4096 from 1.9 GB to 283 MB).
+int default_group_m(int n_mt, int64_t K) {
+  const int64_t per_mtile = static_cast<int64_t>(kBM) * K * 2;
+  const int64_t g = (16ll << 20) / per_mtile;
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g, n_mt)));
+}
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA; }
 
@@ -108,6 +133,7 @@ int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const 
                     const CUtensorMap &bl, lora_stream_t stream) {
   const int n_tiles = gp.n_mt * gp.n_nt;
   const int KB = (gp.K + kBK - 1) / kBK;
+  gp.group_m = default_group_m(gp.n_mt, gp.K);
   int S = 1;
   while (S < 4 && 2 * S * n_tiles <= ds->num_sms && 2 * S <= KB) S *= 2;  // S in {1, 2, 4}
   gp.ksplit = S;
@@ -360,9 +386,12 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   bool ok = true;
   ok &= make_map(&mX128, Asrc, hp.d_in, hp.T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mW, W, hp.d_out, hp.d_in, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&mBl, B_pool, hp.d_out, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  const bool b3d = hp.d_out % 64 == 0;
+  ok &= b3d ? make_map_blocks(&mBl, B_pool, hp.d_out, R, 16, kBN / 64)
+            : make_map(&mBl, B_pool, hp.d_out, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return LORA_ERR_ARG;
   GemmParams gp{};
+  gp.b3d = b3d ? 1 : 0;
   gp.T = static_cast<int32_t>(hp.T);
   gp.K = static_cast<int32_t>(hp.d_in);
   gp.N = static_cast<int32_t>(hp.d_out);
@@ -520,6 +549,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.thr = thr;
     gp.inv_keep = inv_keep;
     gp.ksplit = 1;
+    gp.group_m = default_group_m(gp.n_mt, gp.K);
     const int grid = std::min(ds->num_sms, gp.n_mt * gp.n_nt);
     lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mWt, gp);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
