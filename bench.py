@@ -52,7 +52,8 @@ WORKLOAD_TEXT = {
     "fleet": "fleet: T=4096, d_in=d_out=4096, 1000 adapters ranks 1..21, B rows x 1/k, Zipf(1.2) per token",
     "finetune": "finetune: T=16384, d_in=d_out=4096, 1 adapter rank 16, s=2, dropout 0.1; forward + backward",
 }
-KERNEL_SOURCES = ["lora_adapter_execution_b200/csrc/gemm.cuh", "lora_adapter_execution_b200/csrc/common.cuh"]
+KERNEL_SOURCES = ["lora_adapter_execution_b200/csrc/gemm.cuh", "lora_adapter_execution_b200/csrc/common.cuh",
+                  "lora_adapter_execution_b200/csrc/lora_b200.cu"]
 
 
 def parse():
@@ -64,6 +65,8 @@ def parse():
     ap.add_argument("--impl", default="lora", choices=["lora", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-layer", action="store_true",
+                    help="time only the full step (no GEMM-alone, base or torch timings; for profiler runs)")
     a = ap.parse_args()
     if a.steps is None:
         a.steps = DEFAULT_STEPS[a.config]
@@ -336,6 +339,17 @@ def run_lora(a):
     with ClockSampler(local_rank) as clk:
         ms_total = timed(graphs, K)
     clocks = clk.summary()
+    if a.no_layer:
+        value = world * T * K / (ms_total * 1e-3)
+        if rank == 0:
+            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+                              "warmup": a.warmup, "ms_per_step": ms_total / K, "note": "--no-layer run"}))
+        del graphs, ggraphs, bgraphs
+        plan.destroy()
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+        return
     ms_gemm = timed(ggraphs, K)
     ms_base = timed(bgraphs, K)
     assert lora.device_status() == 0
