@@ -48,6 +48,10 @@ constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM
 
 enum GemmEpi { kEpiStore = 0, kEpiBwdLora = 1 };
 constexpr int kEpiRankRegs = 16;  // dU values per row kept in registers by the backward epilogue
+// backward epilogue: the tile's slice of A (ranks < kEpiRankRegs, 256 columns) as
+// fp32 in shared memory, behind the adapter tables
+constexpr int kEpiAsBytes = kEpiRankRegs * kBN * 4;  // 16 KB
+constexpr int kGemmSmemBwd = kGemmSmem + kEpiAsBytes;
 
 struct GemmParams {
   int32_t T;       // rows (tokens)
@@ -157,6 +161,23 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams &p, int &
   nt = r / gm;
   mt = p.mt_order ? p.mt_order[mi] : mi;
 }
+
+// Barrier 1 over the 4 epilogue warps (128 threads). The OR form returns, to every
+// participant, whether any of them passed true: the warps then leave the tile
+// loop together, so none is left waiting at the next barrier.
+__device__ __forceinline__ bool epi_bar_or(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.or.pred p, 1, 128, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v))
+      : "memory");
+  return r != 0;
+}
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
 __device__ __forceinline__ TileDesc regular_tile(int mt, int T) {
   TileDesc td;
@@ -366,13 +387,35 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // -------------------------------------------------------------- epilogue
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
+    float *as = reinterpret_cast<float *>(smem + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16);
     int acc = 0;
     uint32_t aphase = 0;
-    for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
+    // the backward's warps leave together (epi_bar_or), so its loop ignores the
+    // flag here and tests it at the barrier
+    for (int tile = tile0; tile < n_tiles && (EPI == kEpiBwdLora || !*abort_flag); tile += tile_step) {
       int mt, nt;
       tile_coords(tile, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
-      if (!mbar_wait(accf0 + 8 * acc, aphase)) { *abort_flag = 1; break; }
+      if (EPI == kEpiBwdLora) {
+        // stage A[k][nt*256 .. +256) for k < min(r, 16) as fp32 (zero past r or N):
+        // 8 threads per rank, 32 columns each
+        const int et = static_cast<int>(threadIdx.x) - 64;
+        const int k = et >> 3;
+        const int cb = (et & 7) * 32;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int col = nt * kBN + cb + 8 * j;
+          uint4 w = make_uint4(0, 0, 0, 0);
+          if (k < p.r && col < p.N) w = __ldg(reinterpret_cast<const uint4 *>(p.A + static_cast<int64_t>(k) * p.N + col));
+          float4 *d4 = reinterpret_cast<float4 *>(as + k * kBN + cb + 8 * j);
+          d4[0] = make_float4(bf16_lo(w.x), bf16_hi(w.x), bf16_lo(w.y), bf16_hi(w.y));
+          d4[1] = make_float4(bf16_lo(w.z), bf16_hi(w.z), bf16_lo(w.w), bf16_hi(w.w));
+        }
+        const bool waited = mbar_wait(accf0 + 8 * acc, aphase);
+        if (epi_bar_or(!waited || *abort_flag)) { *abort_flag = 1; break; }
+      } else {
+        if (!mbar_wait(accf0 + 8 * acc, aphase)) { *abort_flag = 1; break; }
+      }
       tc_fence_after();
       if (split) break;  // the cluster reduction below handles the single tile
       const bool valid = row < td.rows;
@@ -414,8 +457,20 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             };
 #pragma unroll
-            for (int k = 0; k < kEpiRankRegs; ++k)
-              if (k < p.r) add_rank(k, du[k]);
+            for (int k = 0; k < kEpiRankRegs; ++k) {
+              if (k < p.r) {
+                const float4 *ar = reinterpret_cast<const float4 *>(as + k * kBN + c * 32);  // broadcast reads
+                const float d = du[k];
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                  const float4 a4 = ar[j];
+                  l[4 * j + 0] += d * a4.x;
+                  l[4 * j + 1] += d * a4.y;
+                  l[4 * j + 2] += d * a4.z;
+                  l[4 * j + 3] += d * a4.w;
+                }
+              }
+            }
             for (int k = kEpiRankRegs; k < p.r; ++k) add_rank(k, p.dU[orig * p.r + k]);
             const uint32_t keep = keep_mask32(p.seed, p.thr, static_cast<uint64_t>(orig * p.N + col0));
 #pragma unroll
@@ -438,6 +493,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       tc_fence_before();
       mbar_arrive(acce0 + 8 * acc);
       if (++acc == 2) { acc = 0; aphase ^= 1; }
+      if (EPI == kEpiBwdLora) epi_bar();  // every read of the A slice is done before it is replaced
     }
   }
 

@@ -56,7 +56,7 @@ int device_state(DeviceState **out) {
           ok &= cudaFuncSetAttribute(lora_gemm_kernel<false, kEpiStore>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_gemm_kernel<true, kEpiBwdLora>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBwd) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kSkSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_tcontract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -551,7 +551,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.ksplit = 1;
     gp.group_m = default_group_m(gp.n_mt, gp.K);
     const int grid = std::min(ds->num_sms, gp.n_mt * gp.n_nt);
-    lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mWt, gp);
+    lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmemBwd, stream>>>(mdY128, mWt, mWt, gp);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
   // K3c: dB = s * U^T * dY and dA = (D ⊙ X)^T * dU, split over tokens, then reduced
