@@ -83,17 +83,23 @@ struct GemmParams {
   int32_t ksplit;
 };
 
-// Split-K receive slots: slot s (one per cluster rank) holds rank s's partial for
-// this CTA's 256/S columns, 128 rows, rows padded by 16 bytes so the
-// row-per-thread reads are bank-conflict free: S * 128 * (256/S + 4) * 4 bytes,
-// at most 139 KB (S = 4), inside the idle stage ring.
-__host__ __device__ constexpr int slot_stride(int S) { return kBN / S + 4; }
-__host__ __device__ constexpr int slot_bytes(int S) { return kBM * slot_stride(S) * 4; }
-constexpr int kTStride = 36;  // fp32 row stride of a warp's 32x32 transposition block
-static_assert(2 * slot_bytes(2) + 4 * 32 * kTStride * 4 <= kGemmStages * kStageBytes,
-              "receive slots and transposition blocks must fit the stage ring");
-static_assert(4 * slot_bytes(4) + 4 * 32 * kTStride * 4 <= kGemmStages * kStageBytes,
-              "receive slots and transposition blocks must fit the stage ring");
+// Split-K exchange, inside the idle stage ring once every MMA of the cluster is
+// done. Each CTA q owns output columns [q*w, (q+1)*w), w = 256/S. Partials move
+// as 4 KB blocks (32 rows x 32 columns fp32, one epilogue warp's TMEM lanes)
+// with bulk shared-to-shared copies that complete on the owner's receive
+// barrier. Inside a block, row r's 16-byte column group j sits at group
+// j ^ (r & 7), so both the row-per-thread writes and reads are conflict-free.
+//   [0, (S-1)*w*512)  receive slots, one per other rank (rank order, own skipped),
+//                     each [w/32 column blocks][4 warps][4 KB]
+//   then              outgoing blocks: per warp (256-w)/32 blocks of 4 KB
+constexpr int kXBlock = 32 * 32 * 4;
+__host__ __device__ constexpr int xslot_bytes(int S) { return (kBN / S) * kBM * 4; }
+__host__ __device__ constexpr int xstage_bytes(int S) { return 4 * ((kBN - kBN / S) / 32) * kXBlock; }
+static_assert((2 - 1) * xslot_bytes(2) + xstage_bytes(2) <= kGemmStages * kStageBytes,
+              "split-K exchange (S = 2) must fit the stage ring");
+static_assert((4 - 1) * xslot_bytes(4) + xstage_bytes(4) <= kGemmStages * kStageBytes,
+              "split-K exchange (S = 4) must fit the stage ring");
+__host__ __device__ constexpr uint32_t xswz(int row, int j) { return static_cast<uint32_t>(row * 128 + ((j ^ (row & 7)) * 16)); }
 
 // The K blocks one CTA contributes to one tile.
 struct BlockRange {
@@ -128,20 +134,10 @@ __device__ __forceinline__ uint32_t cluster_rank() {
 __device__ __forceinline__ void cluster_barrier() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::: "memory");
 }
-__device__ __forceinline__ void st_dsmem_v4(uint32_t local_addr, uint32_t rank, float4 v) {
+__device__ __forceinline__ uint32_t map_rank(uint32_t local_addr, uint32_t rank) {
   uint32_t ra;
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
-  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(ra), "f"(v.x), "f"(v.y), "f"(v.z),
-               "f"(v.w)
-               : "memory");
-}
-__device__ __forceinline__ void ld_dsmem_v4(uint32_t local_addr, uint32_t rank, float (&v)[4]) {
-  uint32_t ra;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(ra) : "r"(local_addr), "r"(rank));
-  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
-               : "=f"(v[0]), "=f"(v[1]), "=f"(v[2]), "=f"(v[3])
-               : "r"(ra)
-               : "memory");
+  return ra;
 }
 
 // Output tile visiting order: tiles come in groups of group_m m-tiles; inside a
@@ -211,6 +207,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile int *abort_flag = reinterpret_cast<volatile int *>(tmem_slot + 1);
   // per stage: the B slot each K step of an adapter block reads (2 bits per step)
   volatile uint32_t *bmap = tmem_slot + 2;
+  const uint32_t recv_bar = full0 + 128;  // split-K: the other ranks' partials have landed
   int4 *chunkcache = reinterpret_cast<int4 *>(smem + kGemmStages * kStageBytes + kGemmBarBytes);
 
   const int warp = threadIdx.x >> 5;
@@ -225,6 +222,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(accf0 + 8 * b, 1);
       mbar_init(acce0 + 8 * b, 128);
     }
+    mbar_init(recv_bar, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -501,100 +499,104 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (split) {
     // --------------------------------------------------- split-K cluster reduction
-    // slot s of CTA q's shared memory holds CTA s's partial for the columns q
-    // owns; the barrier's release/acquire makes every pushed store visible
-    // barrier 1: every CTA's MMAs are complete, so every stage ring is idle
+    // barrier: every CTA's MMAs are complete, so every stage ring is idle and may
+    // receive; it also orders the receive barriers' initialisation before any
+    // remote completion
     cluster_barrier();
     const int width = kBN / S;
+    const uint32_t slot0 = smem_u32(smem);
+    const uint32_t out0 = slot0 + (S - 1) * xslot_bytes(S);
+    if (threadIdx.x == 64) mbar_arrive_expect_tx(recv_bar, (S - 1) * xslot_bytes(S));
     if (warp >= 2 && tile0 < n_tiles && !*abort_flag) {
-      // push this CTA's partial sums for the column slices other CTAs own
-      // straight from TMEM into their receive slots (fire-and-forget stores);
-      // the slice this CTA owns stays in TMEM
-      tc_fence_after();
       const int quarter = warp & 3;
       int mt, nt;
       tile_coords(tile0, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      // a CTA with no K blocks for this tile contributes zeros (its TMEM was never written)
       const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
-      // a warp's 32 rows x 32 columns pass through a small shared-memory block so
-      // that each remote store instruction writes 4 whole 128-byte row pieces
-      // (coalesced) instead of 32 scattered 16-byte pieces
-      float *tb = reinterpret_cast<float *>(smem + S * slot_bytes(S)) + (warp - 2) * 32 * kTStride;
+      tc_fence_after();
+      // send: TMEM -> registers -> a 4 KB outgoing block -> bulk copy into the owner's slot
+      int nout = 0;
       for (int c = 0; c < kBN / 32; ++c) {
         const int owner = (c * 32) / width;
         if (owner == q) continue;
         uint32_t v[32];
         tmem_ld32(tmem_base + ((quarter * 32) << 16) + c * 32, v);
         tmem_wait_ld();
+        const uint32_t blk = out0 + static_cast<uint32_t>((quarter * ((kBN - width) / 32) + nout) * kXBlock);
+        uint8_t *blkp = smem + (blk - slot0);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4 *>(tb + lane * kTStride + 4 * j) =
+          *reinterpret_cast<float4 *>(blkp + xswz(lane, j)) =
               any ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
                                 __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
                   : make_float4(0.f, 0.f, 0.f, 0.f);
+        fence_proxy_async_smem();  // the bulk copy (async proxy) reads what these stores wrote
         __syncwarp();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int r = 4 * j + (lane >> 3);  // row within the warp's 32
-          const int cc = (lane & 7) * 4;      // column within the 32-column chunk
-          const float4 o = *reinterpret_cast<const float4 *>(tb + r * kTStride + cc);
-          const uint32_t dst = smem_u32(smem) +
-                               static_cast<uint32_t>(q * slot_bytes(S) + (quarter * 32 + r) * slot_stride(S) * 4 +
-                                                     (c * 32 - owner * width + cc) * 4);
-          st_dsmem_v4(dst, static_cast<uint32_t>(owner), o);
+        if (lane == 0) {
+          const int jq = q < owner ? q : q - 1;  // this rank's slot at the owner
+          const int cc = (c * 32 - owner * width) / 32;
+          const uint32_t dst = slot0 + static_cast<uint32_t>(jq * xslot_bytes(S) + (cc * 4 + quarter) * kXBlock);
+          bulk_s2s_cluster(map_rank(dst, static_cast<uint32_t>(owner)), blk, kXBlock,
+                           map_rank(recv_bar, static_cast<uint32_t>(owner)));
         }
-        __syncwarp();
+        ++nout;
       }
-    }
-    // barrier 2: every pushed store is visible to its owner (release / acquire)
-    cluster_barrier();
-    if (warp >= 2 && tile0 < n_tiles && !*abort_flag) {
-      const int quarter = warp & 3;
-      const int row = quarter * 32 + lane;
-      int mt, nt;
-      tile_coords(tile0, p, mt, nt);
-      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
-      const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
-      const bool valid = row < td.rows;
-      const int64_t orig = !valid ? 0 : has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
-      for (int c0 = 0; c0 < width; c0 += 32) {
-        uint32_t v[32];
-        tmem_ld32(tmem_base + ((quarter * 32) << 16) + q * width + c0, v);  // own partial
-        tmem_wait_ld();
-        float s[32];
+      if (lane == 0) {
+        bulk_commit();
+        bulk_wait_read_all();  // the outgoing blocks are read before this CTA can exit
+      }
+      __syncwarp();
+      // receive: own partial from TMEM + the other ranks' blocks in rank order
+      // (a fixed order, so the result is deterministic)
+      if (!mbar_wait(recv_bar, 0)) {
+        *abort_flag = 1;
+      } else {
+        const int row = quarter * 32 + lane;
+        const bool valid = row < td.rows;
+        const int64_t orig =
+            !valid ? 0 : has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
+        for (int cc = 0; cc < width / 32; ++cc) {
+          uint32_t v[32];
+          tmem_ld32(tmem_base + ((quarter * 32) << 16) + q * width + cc * 32, v);
+          tmem_wait_ld();
+          float s[32];
 #pragma unroll
-        for (int e = 0; e < 32; ++e) s[e] = any ? __uint_as_float(v[e]) : 0.f;
-        // add the other ranks' partials in rank order (fixed order: deterministic)
-        for (int src = 0; src < S; ++src) {
-          if (src == q) continue;
-          const float4 *slot = reinterpret_cast<const float4 *>(
-              smem + src * slot_bytes(S) + (row * slot_stride(S) + c0) * 4);
+          for (int e = 0; e < 32; ++e) s[e] = any ? __uint_as_float(v[e]) : 0.f;
+          for (int src = 0; src < S; ++src) {
+            if (src == q) continue;
+            const int js = src < q ? src : src - 1;
+            const uint8_t *bp = smem + js * xslot_bytes(S) + (cc * 4 + quarter) * kXBlock;
 #pragma unroll
-          for (int j = 0; j < 8; ++j) {
-            const float4 t = slot[j];
-            s[4 * j + 0] += t.x;
-            s[4 * j + 1] += t.y;
-            s[4 * j + 2] += t.z;
-            s[4 * j + 3] += t.w;
+            for (int j = 0; j < 8; ++j) {
+              const float4 t = *reinterpret_cast<const float4 *>(bp + xswz(lane, j));
+              s[4 * j + 0] += t.x;
+              s[4 * j + 1] += t.y;
+              s[4 * j + 2] += t.z;
+              s[4 * j + 3] += t.w;
+            }
           }
-        }
-        const int col = nt * kBN + q * width + c0;
-        if (valid) {
+          const int col = nt * kBN + q * width + cc * 32;
+          if (valid) {
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            if (col + 8 * h < p.N) {
-              uint4 o;
-              o.x = pack_bf16x2(s[8 * h + 0], s[8 * h + 1]);
-              o.y = pack_bf16x2(s[8 * h + 2], s[8 * h + 3]);
-              o.z = pack_bf16x2(s[8 * h + 4], s[8 * h + 5]);
-              o.w = pack_bf16x2(s[8 * h + 6], s[8 * h + 7]);
-              *reinterpret_cast<uint4 *>(p.out + orig * p.N + col + 8 * h) = o;
+            for (int h = 0; h < 4; ++h) {
+              if (col + 8 * h < p.N) {
+                uint4 o;
+                o.x = pack_bf16x2(s[8 * h + 0], s[8 * h + 1]);
+                o.y = pack_bf16x2(s[8 * h + 2], s[8 * h + 3]);
+                o.z = pack_bf16x2(s[8 * h + 4], s[8 * h + 5]);
+                o.w = pack_bf16x2(s[8 * h + 6], s[8 * h + 7]);
+                *reinterpret_cast<uint4 *>(p.out + orig * p.N + col + 8 * h) = o;
+              }
             }
           }
         }
       }
     }
-    cluster_barrier();  // barrier 3: no CTA exits while a peer may still read it
+    // every TMEM read is done before warp 1 frees it; every block bound for this
+    // CTA has landed (the receive barrier) and every outgoing block has been read
+    tc_fence_before();
+    __syncthreads();
   }
   if (warp == 1) {
     __syncwarp();
