@@ -282,13 +282,14 @@ def run_lora(a):
 
     # one graph per copy; the plan (and its scratch) is shared, steps run in order
     def step(cp):
-        lora.linear_shrink(plan, cp["X"], cp["A"], scale, p_drop=inp.p_drop, seed=inp.mask_seed, U_save=cp["U"])
-        lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
+        lora.linear_fwd(plan, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["Y"], p_drop=inp.p_drop,
+                        seed=inp.mask_seed, U_save=cp["U"])
         if finetune:
             lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"], cp["dX"],
                             cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed)
 
-    launches_per_step = 2 + (6 if finetune else 0)
+    # the forward: [row gather] + shrink + fused GEMM; the backward: dU, dX GEMM, 2 x (contraction + reduce)
+    launches_per_step = 2 + int(info["gathers_x"]) + (6 if finetune else 0)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):

@@ -124,6 +124,9 @@ typedef struct lora_plan_info {
     int64_t sum_r_tokens;   /* sum over tokens of their adapter's rank */
     int64_t aug_k_total;    /* sum over tiles of the tile's augmented K (multiples of 16) */
     int64_t scratch_bytes;  /* device scratch owned by the plan */
+    int32_t gathers_x;      /* 1 if the forward first writes the adapter-sorted copy of X
+                               into the scratch (some tile is not a run of consecutive
+                               tokens): one more kernel launch per forward */
 } lora_plan_info_t;
 
 /* Errors: LORA_ERR_ARG. */

@@ -38,7 +38,8 @@ class LoraError(RuntimeError):
 class _Info(ctypes.Structure):
     _fields_ = [("T", _i64), ("d_in", _i64), ("d_out", _i64), ("n_adapters", _i32),
                 ("n_segments", _i32), ("n_tiles", _i32), ("r_max", _i32), ("sum_r_used", _i64),
-                ("sum_r_tokens", _i64), ("aug_k_total", _i64), ("scratch_bytes", _i64)]
+                ("sum_r_tokens", _i64), ("aug_k_total", _i64), ("scratch_bytes", _i64),
+                ("gathers_x", _i32)]
 
 
 _lib = None

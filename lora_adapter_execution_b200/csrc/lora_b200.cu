@@ -296,6 +296,7 @@ int lora_plan_info(lora_plan_t plan, lora_plan_info_t *info) {
   info->sum_r_tokens = hp.sum_r_tokens;
   info->aug_k_total = hp.aug_k_total;
   info->scratch_bytes = hp.scratch_bytes;
+  info->gathers_x = hp.xs_offset >= 0 ? 1 : 0;
   return LORA_OK;
 }
 
