@@ -340,6 +340,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false, !B_KMAJOR);
+      // stage 0's descriptors: A K-major (SW128, 8-row groups 1 KB apart, a K16
+      // step 32 bytes on); B K-major likewise, or MN-major with 64-column blocks
+      // 8 KB apart and a K16 step 16 rows (2 KB) on
+      const uint64_t adesc0 = sdesc_sw128(stage0, 16, 1024);
+      const uint64_t bdesc0 = B_KMAJOR ? sdesc_sw128(stage0 + kStageA, 16, 1024)
+                                       : sdesc_sw128(stage0 + kStageA, 8192, 1024);
+      constexpr uint64_t kAStep = 32 >> 4;
+      constexpr uint64_t kBStep = B_KMAJOR ? (32 >> 4) : (2048 >> 4);
       int stage = 0;
       uint32_t phase = 0;
       int acc = 0;
@@ -358,20 +366,27 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const int blk = br.block(i, KB);
           if (!mbar_wait(full0 + 8 * stage, phase)) { *abort_flag = 1; ok = false; break; }
           tc_fence_after();
-          const uint32_t a_s = stage0 + stage * kStageBytes;
-          const uint32_t b_s = a_s + kStageA;
-          const bool aug = blk >= KB;
-          const int steps = aug ? min(4, (kaug - (blk - KB) * kAugBlock) / 16) : 4;
-          const uint32_t map = aug ? bmap[stage] : 0u;
-          for (int qq = 0; qq < steps; ++qq) {
-            const uint64_t ad = sdesc_sw128(a_s + qq * 32, 16, 1024);
-            // MN-major B: base blocks are [4 column blocks][64 rows][64 cols]
-            // (column-block stride 8 KB); adapter slots are [4][16][64] (2 KB)
-            const uint64_t bd =
-                B_KMAJOR ? sdesc_sw128(b_s + qq * 32, 16, 1024)
-                : aug    ? sdesc_sw128(b_s + ((map >> (2 * qq)) & 3u) * kBSlot, 2048, 1024)
-                         : sdesc_sw128(b_s + qq * 2048, 8192, 1024);
-            umma_bf16(d_tmem, ad, bd, kIdesc, (i > 0 || qq > 0) ? 1u : 0u);
+          // One thread issues every MMA, so its instruction count per K block
+          // bounds the tensor pipe: the descriptors of a stage are the stage's
+          // base descriptors plus constants (address field in 16-byte units).
+          const uint64_t ad = adesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
+          if (blk < KB) {
+            umma_bf16(d_tmem, ad, bd, kIdesc, i > 0 ? 1u : 0u);
+            umma_bf16_acc(d_tmem, ad + kAStep, bd + kBStep, kIdesc);
+            umma_bf16_acc(d_tmem, ad + 2 * kAStep, bd + 2 * kBStep, kIdesc);
+            umma_bf16_acc(d_tmem, ad + 3 * kAStep, bd + 3 * kBStep, kIdesc);
+          } else {
+            // adapter block (MN-major B slots [4 column blocks][16 rows][64 cols],
+            // column-block stride 2 KB; the slot of each K step from bmap)
+            const int steps = min(4, (kaug - (blk - KB) * kAugBlock) / 16);
+            const uint32_t map = bmap[stage];
+            const uint32_t b_s = stage0 + stage * kStageBytes + kStageA;
+            for (int qq = 0; qq < steps; ++qq) {
+              const uint64_t bq = B_KMAJOR ? bd + qq * kAStep
+                                           : sdesc_sw128(b_s + ((map >> (2 * qq)) & 3u) * kBSlot, 2048, 1024);
+              umma_bf16(d_tmem, ad + qq * kAStep, bq, kIdesc, (i > 0 || qq > 0) ? 1u : 0u);
+            }
           }
           umma_commit(empty0 + 8 * stage);
           if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
