@@ -74,6 +74,8 @@ struct GemmParams {
   float inv_keep;
   const int32_t *mt_order;  // m-tile visiting order (heaviest adapter work first), or null
   int32_t group_m;          // m-tiles per group of the tile visiting order (>= 1)
+  int32_t w3d;              // 1 (MN-major B only): mapB is the 3-D view {64, K, N/64} of W
+                            // (N % 64 == 0), one copy per K block; 0: 2-D {64, 64}, four copies
   int32_t b3d;              // 1: mapBl is the 3-D view {64, rows, N/64} (N % 64 == 0) and one
                             // copy fills a B slot; 0: mapBl is 2-D {64, 16}, four copies per slot
   // K split: 1 = persistent CTAs over all tiles; S > 1 = one tile per cluster of
@@ -191,7 +193,7 @@ __device__ __forceinline__ TileDesc regular_tile(int mt, int T) {
 template <bool B_KMAJOR, int EPI>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     lora_gemm_kernel(const __grid_constant__ CUtensorMap mapA,    // A rows (X, sorted X or dY), box {64, 128}
-                     const __grid_constant__ CUtensorMap mapB,    // W
+                     const __grid_constant__ CUtensorMap mapB,    // W (2-D or 3-D, see GemmParams::w3d)
                      const __grid_constant__ CUtensorMap mapBl,   // B_pool rows, box {64, 16(, 4)}
                      const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -280,6 +282,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             tma_load_2d(a_dst, &mapA, fb, k0, arow);
             if (B_KMAJOR) {
               tma_load_2d(b_dst, &mapB, fb, k0, n0);
+            } else if (p.w3d) {
+              tma_load_3d(b_dst, &mapB, fb, 0, k0, n0 / 64);  // the four 64-column blocks in one copy
             } else {
               for (int j = 0; j < kBN / 64; ++j) tma_load_2d(b_dst + j * 8192, &mapB, fb, n0 + j * 64, k0);
             }

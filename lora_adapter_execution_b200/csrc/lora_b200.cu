@@ -386,13 +386,15 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   const void *Asrc = sorted ? static_cast<const void *>(plan->scratch + hp.xs_offset) : static_cast<const void *>(X);
   bool ok = true;
   ok &= make_map(&mX128, Asrc, hp.d_in, hp.T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map(&mW, W, hp.d_out, hp.d_in, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   const bool b3d = hp.d_out % 64 == 0;
+  ok &= b3d ? make_map_blocks(&mW, W, hp.d_out, hp.d_in, 64, kBN / 64)
+            : make_map(&mW, W, hp.d_out, hp.d_in, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= b3d ? make_map_blocks(&mBl, B_pool, hp.d_out, R, 16, kBN / 64)
             : make_map(&mBl, B_pool, hp.d_out, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return LORA_ERR_ARG;
   GemmParams gp{};
   gp.b3d = b3d ? 1 : 0;
+  gp.w3d = b3d ? 1 : 0;
   gp.T = static_cast<int32_t>(hp.T);
   gp.K = static_cast<int32_t>(hp.d_in);
   gp.N = static_cast<int32_t>(hp.d_out);
@@ -429,10 +431,13 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
   int rc = device_state(&ds);
   if (rc != LORA_OK) return rc;
   CUtensorMap mX128, mW;
+  const bool w3d = d_out % 64 == 0;
   bool ok = make_map(&mX128, X, d_in, T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
-            make_map(&mW, W, d_out, d_in, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+            (w3d ? make_map_blocks(&mW, W, d_out, d_in, 64, kBN / 64)
+                 : make_map(&mW, W, d_out, d_in, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B));
   if (!ok) return LORA_ERR_ARG;
   GemmParams gp{};
+  gp.w3d = w3d ? 1 : 0;
   gp.T = static_cast<int32_t>(T);
   gp.K = static_cast<int32_t>(d_in);
   gp.N = static_cast<int32_t>(d_out);
