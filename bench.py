@@ -277,19 +277,25 @@ def run_lora(a):
             cp.update(dY=d(inp.dY), dX=torch.empty(T, di, dtype=torch.bfloat16, device=dev),
                       dA=torch.empty(r, di, dtype=torch.float32, device=dev),
                       dB=torch.empty(r, do, dtype=torch.float32, device=dev),
-                      ws=torch.empty(lora.bwd_workspace_size(T, di, do, r), dtype=torch.uint8, device=dev))
+                      ws=torch.empty(lora.bwd_workspace_size(T, di, do, r), dtype=torch.uint8, device=dev),
+                      bits=torch.empty(T, -(-di // 32), dtype=torch.int32, device=dev))
         copies.append(cp)
 
     # one graph per copy; the plan (and its scratch) is shared, steps run in order
     def step(cp):
+        bits = None
+        if finetune and inp.p_drop > 0:
+            # the step's dropout mask, written once and read by the forward and the backward
+            bits = cp["bits"]
+            lora.dropout_keep_bits(inp.mask_seed, inp.p_drop, bits, di)
         lora.linear_fwd(plan, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["Y"], p_drop=inp.p_drop,
-                        seed=inp.mask_seed, U_save=cp["U"])
+                        seed=inp.mask_seed, U_save=cp["U"], keep_bits=bits)
         if finetune:
             lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"], cp["dX"],
-                            cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed)
+                            cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed, keep_bits=bits)
 
     # the forward: [row gather] + shrink + fused GEMM; the backward: dU, dX GEMM, 2 x (contraction + reduce)
-    launches_per_step = 2 + int(info["gathers_x"]) + (6 if finetune else 0)
+    launches_per_step = 2 + int(info["gathers_x"]) + (6 if finetune else 0) + (1 if finetune and inp.p_drop > 0 else 0)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
@@ -419,12 +425,17 @@ def run_lora(a):
             p = lora.Plan(inp.ids, inp.ranks, di, do, stream=stream)
             with torch.cuda.stream(stream):
                 cp["X"].copy_(pin_X, non_blocking=True)
+                bits = None
+                if finetune and inp.p_drop > 0:
+                    bits = cp["bits"]
+                    lora.dropout_keep_bits(inp.mask_seed, inp.p_drop, bits, di, stream=stream)
                 lora.linear_fwd(p, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["Y"], p_drop=inp.p_drop,
-                                seed=inp.mask_seed, U_save=cp["U"])
+                                seed=inp.mask_seed, U_save=cp["U"], keep_bits=bits)
                 if finetune:
                     cp["dY"].copy_(pin_dY, non_blocking=True)
                     lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"],
-                                    cp["dX"], cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed)
+                                    cp["dX"], cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed,
+                                    keep_bits=bits)
                     pin_dX.copy_(cp["dX"], non_blocking=True)
                 pin_Y.copy_(cp["Y"], non_blocking=True)
             stream.synchronize()

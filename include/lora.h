@@ -157,6 +157,11 @@ void lora_plan_destroy(lora_plan_t plan);
  *           zero for k >= r_a (r_max from lora_plan_info); the backward's input.
  *           Kept in fp32: the backward reduces it over all tokens, where a bf16
  *           rounding of every term would dominate the error of small sums.
+ *   keep_bits  u32 [T, ceil(d_in/32)] DEVICE array or NULL: the dropout mask as
+ *           written by lora_dropout_keep_bits(seed, p_drop, T, d_in) (4-byte
+ *           aligned). Read instead of re-deriving each bit from the generator;
+ *           ignored when p_drop is 0. The caller guarantees it matches seed and
+ *           p_drop. One mask array serves a forward and its backward.
  *   stream  launch stream
  * The plan's scratch holds s_a·U rounded to bf16 between the two kernels, so
  * two forwards with one plan must not run concurrently.
@@ -164,7 +169,7 @@ void lora_plan_destroy(lora_plan_t plan);
  * ------------------------------------------------------------------------ */
 int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
                     const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed,
-                    uint16_t *Y, float *U_save, lora_stream_t stream);
+                    uint16_t *Y, float *U_save, const uint32_t *keep_bits, lora_stream_t stream);
 
 /* The forward's two phases, for callers that schedule or time them apart
  * (lora_linear_fwd is exactly lora_linear_shrink followed by lora_fused_gemm
@@ -181,7 +186,8 @@ int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
  * before this call on the stream.
  * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA. */
 int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_pool, const float *scale,
-                       double p_drop, uint64_t seed, float *U_save, lora_stream_t stream);
+                       double p_drop, uint64_t seed, float *U_save, const uint32_t *keep_bits,
+                       lora_stream_t stream);
 int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *B_pool,
                     uint16_t *Y, lora_stream_t stream);
 
@@ -209,6 +215,7 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
  *   workspace, workspace_bytes  device scratch of at least
  *           lora_linear_bwd_workspace_size(T, d_in, d_out, r) bytes, 256-byte
  *           aligned, owned by the caller; contents on entry are ignored.
+ *   keep_bits  NULL or the mask as in lora_linear_fwd (the forward's own array)
  * Reductions over tokens use a fixed split and a fixed summation order, so
  * results are deterministic run to run.
  * Errors: LORA_ERR_ARG, LORA_ERR_RANK, LORA_ERR_WORKSPACE, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA.
@@ -219,7 +226,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
                     float scale, double p_drop, uint64_t seed, const float *U_save,
                     const uint16_t *dY, uint16_t *dX, float *dA, float *dB, int64_t T,
                     int64_t d_in, int64_t d_out, int32_t r, void *workspace,
-                    size_t workspace_bytes, lora_stream_t stream);
+                    size_t workspace_bytes, const uint32_t *keep_bits, lora_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * lora_linear_bwd_static — lora_linear_bwd without a caller workspace.
@@ -254,13 +261,26 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
 int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B,
                            float scale, double p_drop, uint64_t seed, const float *U_save,
                            const uint16_t *dY, uint16_t *dX, float *dA, float *dB, int64_t T,
-                           int64_t d_in, int64_t d_out, int32_t r, lora_stream_t stream);
+                           int64_t d_in, int64_t d_out, int32_t r, const uint32_t *keep_bits,
+                           lora_stream_t stream);
 
 /* Test hook: write the dropout mask the forward and backward use.
  *   mask_dev  uint8 [T, d_in] device: 1 where X[t, i] is dropped, else 0.
  * Errors: LORA_ERR_ARG, LORA_ERR_CUDA. */
 int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint8_t *mask_dev,
                       lora_stream_t stream);
+
+/* The same mask as keep bits, for lora_linear_fwd / lora_linear_bwd's
+ * keep_bits argument: word t*ceil(d_in/32) + w of bits_dev (u32, DEVICE,
+ * 4-byte aligned, caller-owned) holds columns 32w .. 32w+31 of token t, bit i
+ * set iff column 32w+i is KEPT; bits past d_in are 0. One pass of the generator
+ * over the T x d_in elements, so that the forward's shrink, the backward's dX
+ * epilogue and its dA contraction read the mask instead of each re-deriving it
+ * (the dropout definition is the one under lora_linear_fwd's p_drop; the pages
+ * fix no generator, this one is a reading of them, not a counterpart).
+ * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA. */
+int lora_dropout_keep_bits(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint32_t *bits_dev,
+                           lora_stream_t stream);
 
 /* Test hook for failure detection: launch one thread that waits on an mbarrier
  * nothing will complete, with a wait limit of `limit_us` microseconds (1 ..

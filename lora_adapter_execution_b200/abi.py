@@ -66,16 +66,17 @@ def load_library():
         "lora_plan_get": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
         "lora_plan_info": (ctypes.c_int, [_vp, ctypes.POINTER(_Info)]),
         "lora_plan_destroy": (None, [_vp]),
-        "lora_linear_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp]),
-        "lora_linear_shrink": (ctypes.c_int, [_vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp]),
+        "lora_linear_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp, _vp]),
+        "lora_linear_shrink": (ctypes.c_int, [_vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp]),
         "lora_fused_gemm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
         "lora_base_gemm": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp]),
         "lora_linear_bwd_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
         "lora_linear_bwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _f32, _dbl, _u64, _vp, _vp, _vp, _vp, _vp,
-                                           _i64, _i64, _i64, _i32, _vp, _sz, _vp]),
+                                           _i64, _i64, _i64, _i32, _vp, _sz, _vp, _vp]),
         "lora_linear_bwd_static": (ctypes.c_int, [_vp, _vp, _vp, _vp, _f32, _dbl, _u64, _vp, _vp, _vp, _vp, _vp,
-                                                  _i64, _i64, _i64, _i32, _vp]),
+                                                  _i64, _i64, _i64, _i32, _vp, _vp]),
         "lora_dropout_mask": (ctypes.c_int, [_u64, _dbl, _i64, _i64, _vp, _vp]),
+        "lora_dropout_keep_bits": (ctypes.c_int, [_u64, _dbl, _i64, _i64, _vp, _vp]),
         "lora_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
         "lora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _vp, _vp]),
         "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -161,15 +162,17 @@ class Plan:
 
 
 def linear_fwd(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.0, seed: int = 0,
-               U_save=None, stream=None):
+               U_save=None, keep_bits=None, stream=None):
     _check(load_library().lora_linear_fwd(plan.handle, _ptr(X), _ptr(W), _ptr(A_pool), _ptr(B_pool), _ptr(scale),
                                           float(p_drop), int(seed) & (2**64 - 1), _ptr(Y), _ptr(U_save),
-                                          _stream(stream)), "lora_linear_fwd")
+                                          _ptr(keep_bits), _stream(stream)), "lora_linear_fwd")
 
 
-def linear_shrink(plan: Plan, X, A_pool, scale, *, p_drop: float = 0.0, seed: int = 0, U_save=None, stream=None):
+def linear_shrink(plan: Plan, X, A_pool, scale, *, p_drop: float = 0.0, seed: int = 0, U_save=None,
+                  keep_bits=None, stream=None):
     _check(load_library().lora_linear_shrink(plan.handle, _ptr(X), _ptr(A_pool), _ptr(scale), float(p_drop),
-                                             int(seed) & (2**64 - 1), _ptr(U_save), _stream(stream)),
+                                             int(seed) & (2**64 - 1), _ptr(U_save), _ptr(keep_bits),
+                                             _stream(stream)),
            "lora_linear_shrink")
 
 
@@ -190,19 +193,20 @@ def bwd_workspace_size(T: int, d_in: int, d_out: int, r: int) -> int:
 
 
 def linear_bwd(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, workspace, *, p_drop: float = 0.0,
-               seed: int = 0, stream=None):
+               seed: int = 0, keep_bits=None, stream=None):
     T, d_in = X.shape
     d_out = W.shape[1]
     r = A.shape[0]
     nbytes = workspace.numel() * workspace.element_size()
     _check(load_library().lora_linear_bwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), float(scale), float(p_drop),
                                           int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY), _ptr(dX), _ptr(dA),
-                                          _ptr(dB), T, d_in, d_out, r, _ptr(workspace), nbytes, _stream(stream)),
+                                          _ptr(dB), T, d_in, d_out, r, _ptr(workspace), nbytes, _ptr(keep_bits),
+                                          _stream(stream)),
            "lora_linear_bwd")
 
 
 def linear_bwd_static(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, *, p_drop: float = 0.0,
-                      seed: int = 0, stream=None):
+                      seed: int = 0, keep_bits=None, stream=None):
     """lora_linear_bwd_static: the backward without a caller workspace (for callers
     that cannot allocate device memory); see include/lora.h for its limit and
     sharing rules."""
@@ -211,7 +215,8 @@ def linear_bwd_static(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, *, p_dro
     r = A.shape[0]
     _check(load_library().lora_linear_bwd_static(_ptr(X), _ptr(W), _ptr(A), _ptr(B), float(scale), float(p_drop),
                                                  int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY), _ptr(dX),
-                                                 _ptr(dA), _ptr(dB), T, d_in, d_out, r, _stream(stream)),
+                                                 _ptr(dA), _ptr(dB), T, d_in, d_out, r, _ptr(keep_bits),
+                                                 _stream(stream)),
            "lora_linear_bwd_static")
 
 
@@ -219,6 +224,16 @@ def dropout_mask(seed: int, p_drop: float, mask, *, stream=None):
     T, d_in = mask.shape
     _check(load_library().lora_dropout_mask(int(seed) & (2**64 - 1), float(p_drop), T, d_in, _ptr(mask),
                                             _stream(stream)), "lora_dropout_mask")
+
+
+def dropout_keep_bits(seed: int, p_drop: float, bits, d_in: int, *, stream=None):
+    """Write the dropout keep bits of a [T, d_in] input into `bits` (int32 device
+    tensor [T, ceil(d_in / 32)]), for linear_fwd / linear_bwd's keep_bits."""
+    T, wpr = bits.shape
+    if wpr != -(-d_in // 32):
+        raise ValueError("bits must have ceil(d_in / 32) columns")
+    _check(load_library().lora_dropout_keep_bits(int(seed) & (2**64 - 1), float(p_drop), T, d_in, _ptr(bits),
+                                                 _stream(stream)), "lora_dropout_keep_bits")
 
 
 def device_status(stream=None) -> int:

@@ -72,6 +72,8 @@ struct GemmParams {
   int32_t r;
   uint64_t seed, thr;
   float inv_keep;
+  const uint32_t *keep_bits;  // precomputed keep bits (null: hash), word t * wpr + col / 32
+  int64_t wpr;
   const int32_t *mt_order;  // m-tile visiting order (heaviest adapter work first), or null
   int32_t group_m;          // m-tiles per group of the tile visiting order (>= 1)
   int32_t w3d;              // 1 (MN-major B only): mapB is the 3-D view {64, K, N/64} of W
@@ -489,7 +491,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               }
             }
             for (int k = kEpiRankRegs; k < p.r; ++k) add_rank(k, p.dU[orig * p.r + k]);
-            const uint32_t keep = keep_mask32(p.seed, p.thr, static_cast<uint64_t>(orig * p.N + col0));
+            const uint32_t keep = p.keep_bits ? __ldg(p.keep_bits + orig * p.wpr + (col0 >> 5))
+                                              : keep_mask32(p.seed, p.thr, static_cast<uint64_t>(orig * p.N + col0));
 #pragma unroll
             for (int i = 0; i < 32; ++i) f[i] += ((keep >> i) & 1u) ? p.inv_keep * l[i] : 0.f;
           }

@@ -308,9 +308,11 @@ void lora_plan_destroy(lora_plan_t plan) {
 }
 
 int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_pool, const float *scale,
-                       double p_drop, uint64_t seed, float *U_save, lora_stream_t stream) {
+                       double p_drop, uint64_t seed, float *U_save, const uint32_t *keep_bits,
+                       lora_stream_t stream) {
   if (!plan || !plan->dev || !X || !A_pool || !scale) return LORA_ERR_ARG;
   if (!aligned16(X) || !aligned16(A_pool)) return LORA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(keep_bits) & 3u) return LORA_ERR_ARG;
   if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
   DeviceState *ds = nullptr;
   int rc = device_state(&ds);
@@ -340,6 +342,8 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   sp.perm = plan->d_perm;
   sp.scale = scale;
   sp.thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
+  sp.keep_bits = sp.thr ? keep_bits : nullptr;  // no mask without dropout
+  sp.wpr = (hp.d_in + 31) / 32;
   sp.seed = seed;
   sp.inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
   sp.uimg = plan->scratch;
@@ -412,12 +416,12 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
 
 int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
                     const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed, uint16_t *Y,
-                    float *U_save, lora_stream_t stream) {
+                    float *U_save, const uint32_t *keep_bits, lora_stream_t stream) {
   if (!plan || !plan->dev || !X || !W || !A_pool || !B_pool || !scale || !Y) return LORA_ERR_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(A_pool) || !aligned16(B_pool) || !aligned16(Y))
     return LORA_ERR_ARG;
   if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
-  const int rc = lora_linear_shrink(plan, X, A_pool, scale, p_drop, seed, U_save, stream);
+  const int rc = lora_linear_shrink(plan, X, A_pool, scale, p_drop, seed, U_save, keep_bits, stream);
   if (rc != LORA_OK) return rc;
   return lora_fused_gemm(plan, X, W, B_pool, Y, stream);
 }
@@ -465,8 +469,9 @@ size_t lora_linear_bwd_workspace_size(int64_t T, int64_t d_in, int64_t d_out, in
 int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B, float scale,
                     double p_drop, uint64_t seed, const float *U_save, const uint16_t *dY, uint16_t *dX,
                     float *dA, float *dB, int64_t T, int64_t d_in, int64_t d_out, int32_t r, void *workspace,
-                    size_t workspace_bytes, lora_stream_t stream) {
+                    size_t workspace_bytes, const uint32_t *keep_bits, lora_stream_t stream) {
   if (!X || !W || !A || !B || !U_save || !dY || !dX || !dA || !dB) return LORA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(keep_bits) & 3u) return LORA_ERR_ARG;
   if (T <= 0 || d_in < 8 || d_out < 8 || (d_in % 8) || (d_out % 8)) return LORA_ERR_ARG;
   if (T > (int64_t)1 << 30 || d_in > (int64_t)1 << 30 || d_out > (int64_t)1 << 30) return LORA_ERR_ARG;
   if (r < 8 || r > kTcMaxR || (r % 8)) return LORA_ERR_RANK;
@@ -553,6 +558,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.r = r;
     gp.seed = seed;
     gp.thr = thr;
+    gp.keep_bits = thr ? keep_bits : nullptr;
+    gp.wpr = (d_in + 31) / 32;
     gp.inv_keep = inv_keep;
     gp.ksplit = 1;
     gp.group_m = default_group_m(gp.n_mt, gp.K);
@@ -574,12 +581,17 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     tp.tsplit = static_cast<int32_t>(tsplit);
     tp.N = static_cast<int32_t>(d_out);
     tp.thr = 0;
+    tp.keep_bits = nullptr;
     tp.partial = pdB;
     dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
     lora_tcontract_kernel<<<grid_b, kTcThreads, smem, stream>>>(mdY64, mU, tp);
     tp.N = static_cast<int32_t>(d_in);
     tp.thr = thr;
     tp.seed = seed;
+    // the contraction re-derives the mask: its bit reads would be scattered per
+    // fragment (measured slower than hashing on 16384 x 4096)
+    tp.keep_bits = nullptr;
+    tp.wpr = (d_in + 31) / 32;
     tp.partial = pdA;
     dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
     lora_tcontract_kernel<<<grid_a, kTcThreads, smem, stream>>>(mX64, mdU, tp);
@@ -606,7 +618,7 @@ extern "C" {
 int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B,
                            float scale, double p_drop, uint64_t seed, const float *U_save, const uint16_t *dY,
                            uint16_t *dX, float *dA, float *dB, int64_t T, int64_t d_in, int64_t d_out, int32_t r,
-                           lora_stream_t stream) {
+                           const uint32_t *keep_bits, lora_stream_t stream) {
   const size_t need = lora_linear_bwd_workspace_size(T, d_in, d_out, r);
   if (need > LORA_BWD_STATIC_SCRATCH_BYTES) return LORA_ERR_WORKSPACE;
   int dev = 0;
@@ -623,7 +635,7 @@ int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t 
     }
   }
   return lora_linear_bwd(X, W, A, B, scale, p_drop, seed, U_save, dY, dX, dA, dB, T, d_in, d_out, r,
-                         g_bwd_static_ptr[dev], LORA_BWD_STATIC_SCRATCH_BYTES, stream);
+                         g_bwd_static_ptr[dev], LORA_BWD_STATIC_SCRATCH_BYTES, keep_bits, stream);
 }
 
 int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint8_t *mask_dev,
@@ -636,6 +648,21 @@ int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uin
   const int64_t n = T * d_in;
   const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 65535));
   lora_mask_kernel<<<blocks, 256, 0, stream>>>(seed, thr, T, d_in, mask_dev);
+  return launch_status();
+}
+
+int lora_dropout_keep_bits(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint32_t *bits_dev,
+                           lora_stream_t stream) {
+  if (!bits_dev || T <= 0 || d_in <= 0 || !(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
+  if ((reinterpret_cast<uintptr_t>(bits_dev) & 3u) != 0) return LORA_ERR_ARG;
+  DeviceState *ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LORA_OK) return rc;
+  const uint64_t thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
+  const int64_t wpr = (d_in + 31) / 32;
+  const int64_t n = T * wpr;
+  const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 16 * ds->num_sms));
+  lora_keep_bits_kernel<<<blocks, 256, 0, stream>>>(seed, thr, T, d_in, wpr, bits_dev);
   return launch_status();
 }
 

@@ -52,6 +52,9 @@ struct ShrinkParams {
   const float *scale;
   uint64_t seed, thr;
   float inv_keep;
+  // precomputed keep bits (null: hash each element): word t * wpr + col / 32, bit col % 32
+  const uint32_t *keep_bits;
+  int64_t wpr;
   uint8_t *uimg;
   float *U_save;
   int32_t r_max;
@@ -270,10 +273,22 @@ __global__ void __launch_bounds__(kSkThreads, 2)
           }
           if (masked) {
             const int c0 = colbase + 2 * (lane & 3);
-            a0 = mask_pair(a0, keep_elem(p.seed, p.thr, orow[i][0], c0, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 1, p.K));
-            a1 = mask_pair(a1, keep_elem(p.seed, p.thr, orow[i][1], c0, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 1, p.K));
-            a2 = mask_pair(a2, keep_elem(p.seed, p.thr, orow[i][0], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 9, p.K));
-            a3 = mask_pair(a3, keep_elem(p.seed, p.thr, orow[i][1], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 9, p.K));
+            if (p.keep_bits) {
+              // colbase is a multiple of 16, so c0 .. c0 + 9 share one 32-bit word
+              // (columns past K are zero in the stage; their bits are not read)
+              const bool in = colbase < p.K;
+              const uint32_t w0 = in ? __ldg(p.keep_bits + orow[i][0] * p.wpr + (colbase >> 5)) >> (c0 & 31) : 0u;
+              const uint32_t w1 = in ? __ldg(p.keep_bits + orow[i][1] * p.wpr + (colbase >> 5)) >> (c0 & 31) : 0u;
+              a0 = mask_pair(a0, w0 & 1u, (w0 >> 1) & 1u);
+              a1 = mask_pair(a1, w1 & 1u, (w1 >> 1) & 1u);
+              a2 = mask_pair(a2, (w0 >> 8) & 1u, (w0 >> 9) & 1u);
+              a3 = mask_pair(a3, (w1 >> 8) & 1u, (w1 >> 9) & 1u);
+            } else {
+              a0 = mask_pair(a0, keep_elem(p.seed, p.thr, orow[i][0], c0, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 1, p.K));
+              a1 = mask_pair(a1, keep_elem(p.seed, p.thr, orow[i][1], c0, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 1, p.K));
+              a2 = mask_pair(a2, keep_elem(p.seed, p.thr, orow[i][0], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 9, p.K));
+              a3 = mask_pair(a3, keep_elem(p.seed, p.thr, orow[i][1], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 9, p.K));
+            }
           }
 #pragma unroll
           for (int jj = 0; jj < 4; ++jj) {
@@ -407,6 +422,8 @@ struct TcParams {
   int32_t T, N, r;
   int32_t splits, tsplit;  // token splits, tokens per split (multiple of 64)
   uint64_t seed, thr;      // mask on In (dA); thr = 0 for none
+  const uint32_t *keep_bits;  // precomputed keep bits of In (null: hash), word t * wpr + col / 32
+  int64_t wpr;
   float *partial;          // [splits][r][N]
 };
 
@@ -503,10 +520,26 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           // b2, b3: column + 8
           const int tk = tbase + ks * 16 + 2 * (lane & 3);
           const int c = n0 + cw + (lane >> 2);
-          b0 = mask_pair(b0, keep_elem(p.seed, p.thr, tk, c, p.N), keep_elem(p.seed, p.thr, tk + 1, c, p.N));
-          b1 = mask_pair(b1, keep_elem(p.seed, p.thr, tk + 8, c, p.N), keep_elem(p.seed, p.thr, tk + 9, c, p.N));
-          b2 = mask_pair(b2, keep_elem(p.seed, p.thr, tk, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 1, c + 8, p.N));
-          b3 = mask_pair(b3, keep_elem(p.seed, p.thr, tk + 8, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 9, c + 8, p.N));
+          if (p.keep_bits) {
+            // c % 32 <= 23 (n0 multiple of 128, cw of 16, lane / 4 < 8): c and c + 8
+            // share one word of each token's row
+            const uint32_t *kb = p.keep_bits + (c >> 5);
+            const int sh = c & 31;
+            const bool cin_ = c < p.N;  // columns past N are zero in the stage
+            const uint32_t w0 = cin_ && tk < p.T ? __ldg(kb + static_cast<int64_t>(tk) * p.wpr) >> sh : 0u;
+            const uint32_t w1 = cin_ && tk + 1 < p.T ? __ldg(kb + static_cast<int64_t>(tk + 1) * p.wpr) >> sh : 0u;
+            const uint32_t w8 = cin_ && tk + 8 < p.T ? __ldg(kb + static_cast<int64_t>(tk + 8) * p.wpr) >> sh : 0u;
+            const uint32_t w9 = cin_ && tk + 9 < p.T ? __ldg(kb + static_cast<int64_t>(tk + 9) * p.wpr) >> sh : 0u;
+            b0 = mask_pair(b0, w0 & 1u, w1 & 1u);
+            b1 = mask_pair(b1, w8 & 1u, w9 & 1u);
+            b2 = mask_pair(b2, (w0 >> 8) & 1u, (w1 >> 8) & 1u);
+            b3 = mask_pair(b3, (w8 >> 8) & 1u, (w9 >> 8) & 1u);
+          } else {
+            b0 = mask_pair(b0, keep_elem(p.seed, p.thr, tk, c, p.N), keep_elem(p.seed, p.thr, tk + 1, c, p.N));
+            b1 = mask_pair(b1, keep_elem(p.seed, p.thr, tk + 8, c, p.N), keep_elem(p.seed, p.thr, tk + 9, c, p.N));
+            b2 = mask_pair(b2, keep_elem(p.seed, p.thr, tk, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 1, c + 8, p.N));
+            b3 = mask_pair(b3, keep_elem(p.seed, p.thr, tk + 8, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 9, c + 8, p.N));
+          }
         }
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
@@ -592,6 +625,21 @@ __global__ void lora_wait_selftest_kernel(uint64_t limit_ns, int *result) {
     mbar_init(smem_u32(&bar), 1);
     fence_mbar_init();
     *result = mbar_wait_for(smem_u32(&bar), 0, limit_ns) ? 1 : 0;
+  }
+}
+
+// keep bits of the dropout mask: word t * wpr + w holds columns 32w .. 32w + 31 of
+// token t (bit i set if column 32w + i is kept; bits past d_in are 0)
+__global__ void lora_keep_bits_kernel(uint64_t seed, uint64_t thr, int64_t T, int64_t d_in, int64_t wpr,
+                                      uint32_t *bits) {
+  const int64_t n = T * wpr;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = e / wpr, w = e % wpr;
+    const int64_t col0 = 32 * w;
+    uint32_t m = keep_mask32(seed, thr, static_cast<uint64_t>(t * d_in + col0));
+    if (d_in - col0 < 32) m &= (1u << (d_in - col0)) - 1u;
+    bits[e] = m;
   }
 }
 

@@ -76,7 +76,7 @@ def test_null_plan_calls():
     assert L.lora_plan_get(None, None, None, None) == -1
     assert L.lora_plan_info(None, None) == -1
     L.lora_plan_destroy(None)  # ignored
-    assert L.lora_linear_fwd(None, None, None, None, None, None, 0.0, 0, None, None, None) == -1
+    assert L.lora_linear_fwd(None, None, None, None, None, None, 0.0, 0, None, None, None, None) == -1
 
 
 def test_bwd_workspace_size_monotone():
@@ -89,7 +89,7 @@ def test_bwd_workspace_size_monotone():
 def test_bwd_rejects_bad_rank_before_cuda():
     L = abi.load_library()
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
-    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 12, p, 1 << 20, None)
+    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 12, p, 1 << 20, None, None)
     assert rc == -3
-    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 16, None, 0, None)
+    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 16, None, 0, None, None)
     assert rc == -8

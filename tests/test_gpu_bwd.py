@@ -28,10 +28,15 @@ def _cuda():
     assert lora.device_status() == 0
 
 
-def run_fwd_bwd(inp):
-    """Forward (for U_save) then backward, all through the C ABI."""
+def run_fwd_bwd(inp, keep_bits=False, outputs=False):
+    """Forward (for U_save) then backward, all through the C ABI; with
+    keep_bits the dropout mask is written once and read by both."""
     import lora_adapter_execution_b200 as lora
     r = int(inp.ranks[0])
+    bits = None
+    if keep_bits:
+        bits = torch.empty(inp.T, -(-inp.d_in // 32), dtype=torch.int32, device="cuda")
+        lora.dropout_keep_bits(inp.mask_seed, inp.p_drop, bits, inp.d_in)
     plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out)
     X, W = dev_bf16(inp.X), dev_bf16(inp.W)
     A, B = dev_bf16(inp.A_pool), dev_bf16(inp.B_pool)
@@ -39,16 +44,34 @@ def run_fwd_bwd(inp):
     scale = torch.from_numpy(inp.scale).cuda()
     Y = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
     U = torch.empty(inp.T, r, dtype=torch.float32, device="cuda")
-    lora.linear_fwd(plan, X, W, A, B, scale, Y, p_drop=inp.p_drop, seed=inp.mask_seed, U_save=U)
+    lora.linear_fwd(plan, X, W, A, B, scale, Y, p_drop=inp.p_drop, seed=inp.mask_seed, U_save=U, keep_bits=bits)
     dX = torch.empty(inp.T, inp.d_in, dtype=torch.bfloat16, device="cuda")
     dA = torch.empty(r, inp.d_in, dtype=torch.float32, device="cuda")
     dB = torch.empty(r, inp.d_out, dtype=torch.float32, device="cuda")
     ws = torch.empty(lora.bwd_workspace_size(inp.T, inp.d_in, inp.d_out, r), dtype=torch.uint8, device="cuda")
     lora.linear_bwd(X, W, A, B, float(inp.scale[0]), U, dY, dX, dA, dB, ws, p_drop=inp.p_drop,
-                    seed=inp.mask_seed)
+                    seed=inp.mask_seed, keep_bits=bits)
     assert lora.device_status() == 0
     plan.destroy()
+    if outputs:
+        return [t.cpu() for t in (Y, U, dX, dA, dB)]
     return host_f64(dX), host_f64(dA), host_f64(dB)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(T=390, d_in=264, d_out=200, p_drop=0.1),
+    dict(T=1000, d_in=520, d_out=264, p_drop=0.3),
+    dict(T=700, d_in=256, d_out=256, p_drop=0.0),
+])
+def test_keep_bits_path_identical(kw):
+    """Reading the mask from keep bits gives bit-identical Y, U, dX, dA, dB to
+    re-deriving it from the generator in every kernel."""
+    inp = wl.make_inputs("finetune", **kw)
+    a = run_fwd_bwd(inp, keep_bits=False, outputs=True)
+    b = run_fwd_bwd(inp, keep_bits=True, outputs=True)
+    for x, y in zip(a, b):
+        assert torch.equal(x.view(torch.int32) if x.dtype == torch.float32 else x.view(torch.int16),
+                           y.view(torch.int32) if y.dtype == torch.float32 else y.view(torch.int16))
 
 
 @pytest.mark.parametrize("kw", [

@@ -155,6 +155,22 @@ def test_dropout_mask_bit_exact(p, seed):
     assert (m.cpu().numpy() == oracle.mask(seed, p, T, d)).all()
 
 
+@pytest.mark.parametrize("p,seed,d", [(0.1, 0, 264), (0.5, 77, 200), (0.0, 3, 256), (0.3, 9, 37)])
+def test_dropout_keep_bits_bit_exact(p, seed, d):
+    """The keep bits (1 = kept) against the oracle's dropped mask, element by
+    element; bits past d_in are 0."""
+    import lora_adapter_execution_b200 as lora
+    T = 301
+    wpr = -(-d // 32)
+    bits = torch.empty(T, wpr, dtype=torch.int32, device="cuda")
+    lora.dropout_keep_bits(seed, p, bits, d)
+    words = bits.cpu().numpy().view(np.uint32)
+    unpacked = ((words[:, :, None] >> np.arange(32, dtype=np.uint32)) & 1).reshape(T, wpr * 32)
+    keep = 1 - oracle.mask(seed, p, T, d).astype(np.uint32)
+    assert (unpacked[:, :d] == keep).all()
+    assert (unpacked[:, d:] == 0).all()
+
+
 def _sample_rows(T, n, seed=0):
     rng = np.random.default_rng(seed)
     edge = [0, 1, 127, 128, T - 1, T - 2, T // 2]

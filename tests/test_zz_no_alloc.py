@@ -80,7 +80,7 @@ def test_static_scratch_backward_rejects_oversized_requests():
     t = torch.empty(16, dtype=torch.uint8, device="cuda")
     p = abi._ptr(t)
     L = lora.load_library()
-    rc = L.lora_linear_bwd_static(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, T, d_in, d_out, r,
+    rc = L.lora_linear_bwd_static(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, T, d_in, d_out, r, None,
                                   abi._stream(None))
     assert rc == -8  # LORA_ERR_WORKSPACE, nothing launched
     assert lora.device_status() == 0
