@@ -537,38 +537,49 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // a CTA with no K blocks for this tile contributes zeros (its TMEM was never written)
       const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
       tc_fence_after();
-      // send: TMEM -> registers -> a 4 KB outgoing block -> bulk copy into the owner's slot
+      // send: TMEM -> registers -> this warp's 4 KB outgoing blocks (column pairs
+      // of one owner: width >= 64), one proxy fence, then the bulk copies into
+      // the owners' slots; they are waited for (read) only before exit
       int nout = 0;
-      for (int c = 0; c < kBN / 32; ++c) {
+      for (int c = 0; c < kBN / 32; c += 2) {
         const int owner = (c * 32) / width;
         if (owner == q) continue;
-        uint32_t v[32];
-        tmem_ld32(tmem_base + ((quarter * 32) << 16) + c * 32, v);
+        uint32_t v0[32], v1[32];
+        tmem_ld32(tmem_base + ((quarter * 32) << 16) + c * 32, v0);
+        tmem_ld32(tmem_base + ((quarter * 32) << 16) + (c + 1) * 32, v1);
         tmem_wait_ld();
-        const uint32_t blk = out0 + static_cast<uint32_t>((quarter * ((kBN - width) / 32) + nout) * kXBlock);
-        uint8_t *blkp = smem + (blk - slot0);
+        uint8_t *b0 = smem + (out0 - slot0) + (quarter * ((kBN - width) / 32) + nout) * kXBlock;
+        uint8_t *b1 = b0 + kXBlock;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          *reinterpret_cast<float4 *>(blkp + xswz(lane, j)) =
-              any ? make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]))
+        for (int j = 0; j < 8; ++j) {
+          *reinterpret_cast<float4 *>(b0 + xswz(lane, j)) =
+              any ? make_float4(__uint_as_float(v0[4 * j]), __uint_as_float(v0[4 * j + 1]),
+                                __uint_as_float(v0[4 * j + 2]), __uint_as_float(v0[4 * j + 3]))
                   : make_float4(0.f, 0.f, 0.f, 0.f);
-        fence_proxy_async_smem();  // the bulk copy (async proxy) reads what these stores wrote
-        __syncwarp();
-        if (lane == 0) {
+          *reinterpret_cast<float4 *>(b1 + xswz(lane, j)) =
+              any ? make_float4(__uint_as_float(v1[4 * j]), __uint_as_float(v1[4 * j + 1]),
+                                __uint_as_float(v1[4 * j + 2]), __uint_as_float(v1[4 * j + 3]))
+                  : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
+        nout += 2;
+      }
+      fence_proxy_async_smem();  // the bulk copies (async proxy) read what these stores wrote
+      __syncwarp();
+      if (lane == 0) {
+        int k = 0;
+        for (int c = 0; c < kBN / 32; ++c) {
+          const int owner = (c * 32) / width;
+          if (owner == q) continue;
+          const uint32_t blk = out0 + static_cast<uint32_t>((quarter * ((kBN - width) / 32) + k) * kXBlock);
           const int jq = q < owner ? q : q - 1;  // this rank's slot at the owner
           const int cc = (c * 32 - owner * width) / 32;
           const uint32_t dst = slot0 + static_cast<uint32_t>(jq * xslot_bytes(S) + (cc * 4 + quarter) * kXBlock);
           bulk_s2s_cluster(map_rank(dst, static_cast<uint32_t>(owner)), blk, kXBlock,
                            map_rank(recv_bar, static_cast<uint32_t>(owner)));
+          ++k;
         }
-        ++nout;
-      }
-      if (lane == 0) {
         bulk_commit();
-        bulk_wait_read_all();  // the outgoing blocks are read before this CTA can exit
       }
-      __syncwarp();
       // receive: own partial from TMEM + the other ranks' blocks in rank order
       // (a fixed order, so the result is deterministic)
       if (!mbar_wait(recv_bar, 0)) {
@@ -614,6 +625,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           }
         }
       }
+      if (lane == 0) bulk_wait_read_all();  // the outgoing blocks are read before this CTA can exit
+      __syncwarp();
     }
     // every TMEM read is done before warp 1 frees it; every block bound for this
     // CTA has landed (the receive barrier) and every outgoing block has been read

@@ -190,20 +190,22 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   const int kend = min(p.K, kbeg + p.kslice);
   const int nblk = kend > kbeg ? (kend - kbeg + kSkBK - 1) / kSkBK : 0;
 
+  // warp work split: MW warps along rows (m-blocks), KW along the stages (warp
+  // group kphase takes stages kphase, kphase + KW, ...), so the stages of a small
+  // unit are consumed in parallel instead of one after another
+  int MW = 1;
+  while (MW * 2 <= mb && MW < kSkConsumerWarps) MW *= 2;
+  const int KW = kSkConsumerWarps / MW;
+
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, kSkConsumerWarps);
+      mbar_init(empty0 + 8 * s, MW);  // the MW warps that consume the stage
     }
     *abort_flag = 0;
     fence_mbar_init();
   }
   __syncthreads();
-
-  // warp work split: MW warps along rows (m-blocks), KW along the k16 steps of a stage
-  int MW = 1;
-  while (MW * 2 <= mb && MW < kSkConsumerWarps) MW *= 2;
-  const int KW = kSkConsumerWarps / MW;
   const int nb8 = g.nn / 8;
 
   float acc[2][8][4];
@@ -252,13 +254,13 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                                    : (p.mode == 0 ? static_cast<int64_t>(p.perm[g.row0 + rc]) : 0);
       }
     const bool masked = p.mode == 0 && p.thr != 0;
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int b = 0; b < nblk; ++b) {
+    for (int b = kphase; b < nblk; b += KW) {
+      const int stage = b % nstage;
+      const uint32_t phase = static_cast<uint32_t>(b / nstage) & 1u;
       if (!mbar_wait(full0 + 8 * stage, phase)) { *abort_flag = 1; break; }
       const uint32_t xb = pool + stage * stage_bytes;
       const uint32_t fbuf = xb + Rp * 128;
-      for (int ks = kphase; ks < 4; ks += KW) {  // k16 steps of the stage
+      for (int ks = 0; ks < 4; ++ks) {  // k16 steps of the stage
         const int colbase = kbeg + b * kSkBK + ks * 16;
 #pragma unroll
         for (int i = 0; i < 2; ++i) {
@@ -305,7 +307,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       }
       __syncwarp();
       if (lane == 0) mbar_arrive(empty0 + 8 * stage);
-      if (++stage == nstage) { stage = 0; phase ^= 1; }
     }
   }
   __syncthreads();  // every TMA landed and was consumed: the pool is free for the reduction
