@@ -238,6 +238,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // inputs written by the previous kernels of the forward (s·U images, the
+  // sorted copy of X) and the output are touched only after they completed
+  pdl_wait();
 
   const int n_tiles = p.n_mt * p.n_nt;
   const int KB = (p.K + kBK - 1) / kBK;

@@ -137,23 +137,22 @@ int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const 
   int S = 1;
   while (S < 4 && 2 * S * n_tiles <= ds->num_sms && 2 * S <= KB) S *= 2;  // S in {1, 2, 4}
   gp.ksplit = S;
-  if (S == 1) {
-    const int grid = std::min(ds->num_sms, n_tiles);
-    lora_gemm_kernel<false, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(a, b, bl, gp);
-    return launch_status();
-  }
   cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(n_tiles * S));
+  cfg.gridDim = dim3(static_cast<unsigned>(S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S));
   cfg.blockDim = dim3(kGemmThreads);
   cfg.dynamicSmemBytes = kGemmSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = S;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
+  // programmatic serialization: the GEMM's setup overlaps the end of the
+  // kernel before it (the shrink), whose results it waits for in pdl_wait
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = S;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = S == 1 ? 1 : 2;
   if (cudaLaunchKernelEx(&cfg, lora_gemm_kernel<false, kEpiStore>, a, b, bl, gp) != cudaSuccess) {
     cudaGetLastError();
     return LORA_ERR_CUDA;
@@ -355,13 +354,18 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   cfg.blockDim = dim3(kSkThreads);
   cfg.dynamicSmemBytes = kSkSmem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  // programmatic serialization: the shrink's setup (barriers, its plan entry)
+  // overlaps the end of the kernel before it; it waits in pdl_wait before
+  // touching X or any output
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = ks;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
+  cfg.numAttrs = 2;
   if (Xs) {
     // sorted copy of X first (the shrink and the fused GEMM read token tiles from it)
     const int64_t pieces = hp.T * (hp.d_in / 8);

@@ -180,7 +180,8 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   const int lane = threadIdx.x & 31;
   const int unit = blockIdx.x / p.ksplit;
   const uint32_t crank = cluster_ctarank();
-  const UnitGeom g = unit_geom(p, unit);
+  pdl_launch_dependents();  // the fused GEMM may set itself up meanwhile
+  const UnitGeom g = unit_geom(p, unit);  // plan tables: written before any kernel of the forward
 
   const int Rp = ((g.rows + 15) / 16) * 16;  // rows rounded to the MMA M step
   const int mb = Rp / 16;
@@ -206,6 +207,9 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     fence_mbar_init();
   }
   __syncthreads();
+  // X (or its sorted copy from the row gather) and everything else the launch
+  // reads or writes come after the previous kernel on the stream has completed
+  pdl_wait();
   const int nb8 = g.nn / 8;
 
   float acc[2][8][4];
@@ -596,6 +600,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 // pieces of a row, so reads and writes are fully coalesced.
 __global__ void lora_gather_rows_kernel(const uint16_t *__restrict__ X, const int32_t *__restrict__ perm,
                                         uint16_t *__restrict__ Xs, int64_t T, int64_t d) {
+  pdl_launch_dependents();  // the shrink may set itself up meanwhile
   const int64_t per_row = d / 8;
   const int64_t n = T * per_row;
   for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
