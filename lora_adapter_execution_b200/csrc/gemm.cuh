@@ -75,6 +75,7 @@ struct GemmParams {
   const uint32_t *keep_bits;  // precomputed keep bits (null: hash), word t * wpr + col / 32
   int64_t wpr;
   const int32_t *mt_order;  // m-tile visiting order (heaviest adapter work first), or null
+  const AugBlockDesc *augblocks;  // the plan's adapter K blocks (TileDesc::aug0 + block)
   int32_t group_m;          // m-tiles per group of the tile visiting order (>= 1)
   int32_t w3d;              // 1 (MN-major B only): mapB is the 3-D view {64, K, N/64} of W
                             // (N % 64 == 0), one copy per K block; 0: 2-D {64, 64}, four copies
@@ -212,7 +213,6 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // per stage: the B slot each K step of an adapter block reads (2 bits per step)
   volatile uint32_t *bmap = tmem_slot + 2;
   const uint32_t recv_bar = full0 + 128;  // split-K: the other ranks' partials have landed
-  int4 *chunkcache = reinterpret_cast<int4 *>(smem + kGemmStages * kStageBytes + kGemmBarBytes);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -265,16 +265,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // A rows: the sorted copy written by the shrink (rows in tile order), or the
       // original rows when the tile's tokens are consecutive originals
       const int arow = p.a_sorted ? td.row0 : td.contig;
-      for (int c = lane; c < td.nchunk; c += 32) {
-        const ChunkDesc cd = p.chunks[td.chunk0 + c];
-        chunkcache[c] = make_int4(cd.pool_row, cd.kofs, cd.kc, 0);
-      }
-      __syncwarp();
       if (lane == 0) {
         if (arow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; }
         const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
         const int nblk = arow < 0 ? 0 : br.count();
-        int c = 0;  // chunk cursor over the tile's adapter table
+        // adapter block descriptors, one load ahead of their use (the adapter
+        // blocks come first: block i < naug is adapter block q + i * S)
+        const int na = br.naug();
+        int4 nprow = make_int4(0, 0, 0, 0);
+        int ninfo = 0;
+        if (na > 0) {
+          nprow = __ldg(reinterpret_cast<const int4 *>(p.augblocks + td.aug0 + q));
+          ninfo = __ldg(&p.augblocks[td.aug0 + q].info);
+        }
         for (int i = 0; i < nblk; ++i) {
           const int blk = br.block(i, KB);
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
@@ -296,33 +299,15 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // adapter K block: 64 augmented columns (up to 4 MMA K steps). Each
             // chunk spans 2*kc columns: s*U rounded to bf16 (hi), then the
             // rounding remainder (lo); both multiply the same B rows, so each
-            // distinct 16-row slice of B_pool is copied once, into its own slot.
+            // distinct 16-row slice of B_pool is copied once, into its own slot
+            // (the planner's descriptor lists the slices and each step's slot).
             const int lb = blk - KB;
-            const int steps = min(4, (td.kaug - lb * kAugBlock) / 16);
-            int prow_s[4] = {0, 0, 0, 0};
-            int nslot = 0;
-            uint32_t map = 0;
-#pragma unroll
-            for (int qq = 0; qq < 4; ++qq) {
-              if (qq < steps) {
-                const int kq = lb * kAugBlock + qq * 16;
-                while (c + 1 < td.nchunk && kq >= chunkcache[c].y + 2 * chunkcache[c].z) ++c;
-                const int4 cc = chunkcache[c];
-                int o = kq - cc.y;
-                if (o >= cc.z) o -= cc.z;
-                const int prow = cc.x + o;
-                int s = nslot;
-#pragma unroll
-                for (int u = 0; u < 4; ++u)
-                  if (u < nslot && prow_s[u] == prow && s == nslot) s = u;
-                if (s == nslot) {
-#pragma unroll
-                  for (int u = 0; u < 4; ++u)
-                    if (u == nslot) prow_s[u] = prow;
-                  ++nslot;
-                }
-                map |= static_cast<uint32_t>(s) << (2 * qq);
-              }
+            const int prow_s[4] = {nprow.x, nprow.y, nprow.z, nprow.w};
+            const int nslot = ninfo & 15;
+            const uint32_t map = static_cast<uint32_t>(ninfo >> 4) & 0xFFu;
+            if (i + 1 < na) {
+              nprow = __ldg(reinterpret_cast<const int4 *>(p.augblocks + td.aug0 + lb + S));
+              ninfo = __ldg(&p.augblocks[td.aug0 + lb + S].info);
             }
             bmap[stage] = map;  // published to the MMA thread by the release arrive below
             mbar_arrive_expect_tx(fb, kStageA + nslot * kBSlot);

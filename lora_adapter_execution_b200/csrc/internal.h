@@ -22,6 +22,17 @@ struct TileDesc {
   int32_t kaug;    // augmented K = sum of the chunks' 2*kc (multiple of 32)
   int32_t contig;  // original index of row 0 if the tile's tokens are consecutive originals, else -1
   int64_t uofs;    // byte offset of the tile's s*U image in the plan scratch
+  int32_t aug0;    // first AugBlockDesc of the tile (one per 64 augmented columns)
+  int32_t pad_;
+};
+
+// One adapter K block of a tile (64 augmented columns, up to 4 MMA K steps of 16):
+// the distinct 16-row slices of B_pool it reads and which slice each K step uses.
+// Precomputed by the planner so the GEMM's copy-issuing thread only reads it.
+struct AugBlockDesc {
+  int32_t prow[4];  // first B_pool row of slot 0..nslot-1 (0 past nslot)
+  int32_t info;     // nslot | slot of K step q at bits 4 + 2q | steps << 12
+  int32_t pad_[3];
 };
 
 // One adapter's run of rows inside one tile: its K slice of the augmented contraction.
@@ -53,6 +64,7 @@ struct HostPlan {
   std::vector<TileDesc> tiles;
   std::vector<ChunkDesc> chunks;
   std::vector<UnitDesc> units;
+  std::vector<AugBlockDesc> augblocks;
   std::vector<int32_t> mt_order;  // m-tiles by decreasing adapter work (stable)
   int32_t r_max = 0;
   int64_t sum_r_used = 0, sum_r_tokens = 0, aug_k_total = 0;

@@ -171,6 +171,7 @@ struct lora_plan {
   const ChunkDesc *d_chunks = nullptr;
   const UnitDesc *d_units = nullptr;
   const int32_t *d_mt_order = nullptr;
+  const AugBlockDesc *d_augblocks = nullptr;
   int device = 0;
 };
 
@@ -215,7 +216,8 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   const size_t b_chunks = up(sizeof(ChunkDesc) * hp.chunks.size());
   const size_t b_units = up(sizeof(UnitDesc) * hp.units.size());
   const size_t b_order = up(sizeof(int32_t) * hp.mt_order.size());
-  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order;
+  const size_t b_aug = up(sizeof(AugBlockDesc) * hp.augblocks.size());
+  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug;
   if (cudaMalloc(&pl->dev, total) != cudaSuccess) {
     cudaGetLastError();
     delete pl;
@@ -233,6 +235,8 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   pl->d_chunks = reinterpret_cast<const ChunkDesc *>(base + b_perm + b_tiles);
   pl->d_units = reinterpret_cast<const UnitDesc *>(base + b_perm + b_tiles + b_chunks);
   pl->d_mt_order = reinterpret_cast<const int32_t *>(base + b_perm + b_tiles + b_chunks + b_units);
+  pl->d_augblocks =
+      reinterpret_cast<const AugBlockDesc *>(base + b_perm + b_tiles + b_chunks + b_units + b_order);
   bool ok = true;
   ok &= cudaMemcpyAsync(base, hp.perm.data(), sizeof(int32_t) * hp.perm.size(), cudaMemcpyHostToDevice,
                         stream) == cudaSuccess;
@@ -244,6 +248,10 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
                         cudaMemcpyHostToDevice, stream) == cudaSuccess;
   ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks + b_units, hp.mt_order.data(),
                         sizeof(int32_t) * hp.mt_order.size(), cudaMemcpyHostToDevice, stream) == cudaSuccess;
+  if (!hp.augblocks.empty())
+    ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks + b_units + b_order, hp.augblocks.data(),
+                          sizeof(AugBlockDesc) * hp.augblocks.size(), cudaMemcpyHostToDevice,
+                          stream) == cudaSuccess;
   // the copies read host vectors that the plan keeps alive; make sure they have
   // been consumed before returning so the caller may reuse its stream freely
   ok &= cudaStreamSynchronize(stream) == cudaSuccess;
@@ -413,6 +421,7 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   gp.perm = plan->d_perm;
   gp.uimg = plan->scratch;
   gp.mt_order = plan->d_mt_order;
+  gp.augblocks = plan->d_augblocks;
   gp.a_sorted = sorted ? 1 : 0;
   gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
   return launch_fwd_gemm(ds, gp, mX128, mW, mBl, stream);
