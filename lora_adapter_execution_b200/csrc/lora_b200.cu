@@ -124,6 +124,25 @@ int default_group_m(int n_mt, int64_t K) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(g, n_mt)));
 }
 
+// Cluster size of the shrink (CTAs that split one unit's contraction): the
+// choice in 1..4 with the fewest stages on the critical path, counting whole
+// waves of 2 CTAs per SM (a second, mostly empty wave costs a full one).
+int shrink_split(int n_units, int64_t K, int num_sms) {
+  const int64_t kb = (K + kSkBK - 1) / kSkBK;
+  const int64_t slots = 2 * static_cast<int64_t>(num_sms);
+  int best = 1;
+  int64_t best_cost = -1;
+  for (int ks = 1; ks <= 4 && ks <= kb; ++ks) {
+    const int64_t waves = (static_cast<int64_t>(n_units) * ks + slots - 1) / slots;
+    const int64_t cost = waves * ((kb + ks - 1) / ks);
+    if (best_cost < 0 || cost < best_cost) {
+      best = ks;
+      best_cost = cost;
+    }
+  }
+  return best;
+}
+
 int launch_status() { return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA; }
 
 // Forward GEMM launch: persistent CTAs when there are enough output tiles to
@@ -337,8 +356,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   sp.T = static_cast<int32_t>(hp.T);
   sp.K = static_cast<int32_t>(hp.d_in);
   const int n_units = static_cast<int>(hp.units.size());
-  int ks = std::max(1, std::min(4, (2 * ds->num_sms + n_units - 1) / n_units));
-  ks = std::min<int>(ks, static_cast<int>((hp.d_in + kSkBK - 1) / kSkBK));
+  const int ks = shrink_split(n_units, hp.d_in, ds->num_sms);
   int64_t slice = (hp.d_in + ks - 1) / ks;
   slice = (slice + kSkBK - 1) / kSkBK * kSkBK;
   sp.ksplit = ks;
@@ -533,8 +551,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     sp.x_sorted = 0;
     sp.dU = dU;
     const int n_units = static_cast<int>((T + kTileM - 1) / kTileM) * sp.npieces;
-    int ks = std::max(1, std::min(4, (2 * ds->num_sms + n_units - 1) / n_units));
-    ks = std::min<int>(ks, static_cast<int>((d_out + kSkBK - 1) / kSkBK));
+    const int ks = shrink_split(n_units, d_out, ds->num_sms);
     int64_t slice = (d_out + ks - 1) / ks;
     slice = (slice + kSkBK - 1) / kSkBK * kSkBK;
     sp.ksplit = ks;
