@@ -603,7 +603,21 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     const int g_bytes = kTcTok * r * 4;
     const int stage_bytes = kTcTok * kTcCols * 2 + ((g_bytes + 1023) & ~1023);
     const int smem = 1024 + kTcStages * stage_bytes + 2 * kTcStages * 8;
+    // keep bits in the dA contraction need a 16-byte row stride (d_in % 128 == 0);
+    // otherwise it re-derives the mask from the generator
+    bool use_bits = thr != 0 && keep_bits != nullptr && ((d_in + 31) / 32) % 4 == 0;
     // note: the kernel lays stages out with the same formula
+    CUtensorMap mBits = mX64;  // unused unless the dA contraction reads keep bits
+    if (use_bits) {
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>((d_in + 31) / 32), static_cast<cuuint64_t>(T)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>((d_in + 31) / 32) * 4};
+      cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcCols / 32), static_cast<cuuint32_t>(kTcTok)};
+      cuuint32_t estr[2] = {1, 1};
+      if (g_encode(&mBits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(keep_bits), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        use_bits = false;
+    }
     TcParams tp{};
     tp.T = static_cast<int32_t>(T);
     tp.r = r;
@@ -614,17 +628,17 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     tp.keep_bits = nullptr;
     tp.partial = pdB;
     dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
-    lora_tcontract_kernel<<<grid_b, kTcThreads, smem, stream>>>(mdY64, mU, tp);
+    lora_tcontract_kernel<<<grid_b, kTcThreads, smem, stream>>>(mdY64, mU, mBits, tp);
     tp.N = static_cast<int32_t>(d_in);
     tp.thr = thr;
     tp.seed = seed;
-    // the contraction re-derives the mask: its bit reads would be scattered per
-    // fragment (measured slower than hashing on 16384 x 4096)
-    tp.keep_bits = nullptr;
+    // with keep bits, each stage's bits come through the copy engine with its tile
+    tp.keep_bits = use_bits ? keep_bits : nullptr;
+    const int smem_a = smem + (use_bits ? kTcStages * kTcTok * (kTcCols / 32) * 4 : 0);
     tp.wpr = (d_in + 31) / 32;
     tp.partial = pdA;
     dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
-    lora_tcontract_kernel<<<grid_a, kTcThreads, smem, stream>>>(mX64, mdU, tp);
+    lora_tcontract_kernel<<<grid_a, kTcThreads, smem_a, stream>>>(mX64, mdU, mBits, tp);
     const int64_t nb = static_cast<int64_t>(r) * d_out;
     const int64_t na = static_cast<int64_t>(r) * d_in;
     lora_reduce_splits_kernel<<<static_cast<unsigned>(std::min<int64_t>((nb + 255) / 256, 4096)), 256, 0, stream>>>(

@@ -443,6 +443,7 @@ __device__ __forceinline__ void split_pair(float v0, float v1, uint32_t &hi, uin
 __global__ void __launch_bounds__(kTcThreads, 1)
     lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N] bf16, box {64, 64}, swizzle 128B
                           const __grid_constant__ CUtensorMap mapG,   // G [T, r] fp32, box {r, 64}, no swizzle
+                          const __grid_constant__ CUtensorMap mapBits,  // keep bits [T, wpr] u32, box {4, 64}
                           const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -450,7 +451,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int in_bytes = kTcTok * kTcCols * 2;    // 16 KB (two 8 KB halves)
   const int g_bytes = kTcTok * p.r * 4;         // <= 16 KB
   const int g_pad = (g_bytes + 1023) & ~1023;
-  const int stage_bytes = in_bytes + g_pad;
+  const int bits_bytes = p.keep_bits ? kTcTok * (kTcCols / 32) * 4 : 0;  // 1 KB: the stage's keep bits
+  const int stage_bytes = in_bytes + g_pad + bits_bytes;
   const uint32_t pool = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kTcStages * stage_bytes);
   const uint32_t full0 = smem_u32(bars);
@@ -490,10 +492,11 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         const uint32_t fb = full0 + 8 * stage;
         const uint32_t sb = pool + stage * stage_bytes;
         const int t = t0 + b * kTcTok;
-        mbar_arrive_expect_tx(fb, in_bytes + g_bytes);
+        mbar_arrive_expect_tx(fb, in_bytes + g_bytes + bits_bytes);
         tma_load_2d(sb, &mapIn, fb, n0, t);
         tma_load_2d(sb + 8192, &mapIn, fb, n0 + 64, t);
         tma_load_2d(sb + in_bytes, &mapG, fb, 0, t);
+        if (bits_bytes) tma_load_2d(sb + in_bytes + g_pad, &mapBits, fb, n0 / 32, t);
         if (++stage == kTcStages) { stage = 0; phase ^= 1; }
       }
     }
@@ -526,15 +529,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           const int tk = tbase + ks * 16 + 2 * (lane & 3);
           const int c = n0 + cw + (lane >> 2);
           if (p.keep_bits) {
-            // c % 32 <= 23 (n0 multiple of 128, cw of 16, lane / 4 < 8): c and c + 8
-            // share one word of each token's row
-            const uint32_t *kb = p.keep_bits + (c >> 5);
+            // the stage's bits, [64 tokens][4 words] for its 128 columns; c % 32 <= 23
+            // (n0 multiple of 128, cw of 16, lane / 4 < 8), so c and c + 8 share a word
+            const uint32_t *bs = reinterpret_cast<const uint32_t *>(smem + (sb - pool) + in_bytes + g_pad);
+            const int tl = ks * 16 + 2 * (lane & 3);
+            const int wd = (c - n0) >> 5;
             const int sh = c & 31;
-            const bool cin_ = c < p.N;  // columns past N are zero in the stage
-            const uint32_t w0 = cin_ && tk < p.T ? __ldg(kb + static_cast<int64_t>(tk) * p.wpr) >> sh : 0u;
-            const uint32_t w1 = cin_ && tk + 1 < p.T ? __ldg(kb + static_cast<int64_t>(tk + 1) * p.wpr) >> sh : 0u;
-            const uint32_t w8 = cin_ && tk + 8 < p.T ? __ldg(kb + static_cast<int64_t>(tk + 8) * p.wpr) >> sh : 0u;
-            const uint32_t w9 = cin_ && tk + 9 < p.T ? __ldg(kb + static_cast<int64_t>(tk + 9) * p.wpr) >> sh : 0u;
+            const uint32_t w0 = bs[tl * 4 + wd] >> sh;
+            const uint32_t w1 = bs[(tl + 1) * 4 + wd] >> sh;
+            const uint32_t w8 = bs[(tl + 8) * 4 + wd] >> sh;
+            const uint32_t w9 = bs[(tl + 9) * 4 + wd] >> sh;
             b0 = mask_pair(b0, w0 & 1u, w1 & 1u);
             b1 = mask_pair(b1, w8 & 1u, w9 & 1u);
             b2 = mask_pair(b2, (w0 >> 8) & 1u, (w1 >> 8) & 1u);
