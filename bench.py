@@ -176,35 +176,40 @@ def algorithmic(inp, info):
 
 
 # ----------------------------------------------------------------------------- reference arm
-def oracle_sample(inp, rows_budget_s: float, rank_info=None):
-    """Time the oracle on a bounded sample; returns (tokens, seconds, sample text)."""
+def _oracle_runner(inp):
+    """(run(n) -> seconds, what) for the oracle on n tokens of the workload: the
+    forward of n evenly spaced tokens, or (fine-tuning) forward + backward of a
+    sub-batch of the first n tokens."""
     import oracle
     if inp.dY is not None:
-        # forward + backward on the first Ts tokens (a smaller batch of the same workload)
-        def run(Ts):
-            sub = wl.Inputs(spec=inp.spec, T=Ts, d_in=inp.d_in, d_out=inp.d_out, ranks=inp.ranks,
-                            ids=inp.ids[:Ts].copy(), scale=inp.scale, X=inp.X[:Ts].copy(), W=inp.W,
-                            A_pool=inp.A_pool, B_pool=inp.B_pool, dY=inp.dY[:Ts].copy(), p_drop=inp.p_drop,
+        def run(n):
+            sub = wl.Inputs(spec=inp.spec, T=n, d_in=inp.d_in, d_out=inp.d_out, ranks=inp.ranks,
+                            ids=inp.ids[:n].copy(), scale=inp.scale, X=inp.X[:n].copy(), W=inp.W,
+                            A_pool=inp.A_pool, B_pool=inp.B_pool, dY=inp.dY[:n].copy(), p_drop=inp.p_drop,
                             mask_seed=inp.mask_seed, offsets=inp.offsets)
             t0 = time.perf_counter()
             oracle.forward(sub)
             oracle.backward(sub)
             return time.perf_counter() - t0
-        Ts = 4
-        dt = run(Ts)
-        Ts = int(max(4, min(inp.T, Ts * rows_budget_s / max(dt, 1e-3))))
-        dt = run(Ts)
-        return Ts, dt, f"forward+backward of the first {Ts} tokens (sub-batch of the same workload)"
-    rows = np.arange(min(inp.T, 8), dtype=np.int64)
-    t0 = time.perf_counter()
-    oracle.forward(inp, rows=rows)
-    dt = time.perf_counter() - t0
-    n = int(max(8, min(inp.T, 8 * rows_budget_s / max(dt, 1e-3))))
-    rows = np.linspace(0, inp.T - 1, n).astype(np.int64)
-    t0 = time.perf_counter()
-    oracle.forward(inp, rows=rows)
-    dt = time.perf_counter() - t0
-    return n, dt, f"forward of {n} evenly spaced tokens of the batch"
+        return run, "forward+backward of the first {n} tokens (sub-batch of the same workload)"
+
+    def run(n):
+        rows = np.linspace(0, inp.T - 1, n).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.forward(inp, rows=rows)
+        return time.perf_counter() - t0
+    return run, "forward of {n} evenly spaced tokens of the batch"
+
+
+def oracle_sample(inp, budget_s: float):
+    """Time the oracle on a bounded sample of about budget_s seconds; returns
+    (tokens, seconds, sample text)."""
+    run, what = _oracle_runner(inp)
+    n0 = 4
+    dt = run(n0)
+    n = int(max(1, min(inp.T, n0 * budget_s / max(dt, 1e-6))))
+    dt = run(n)
+    return n, dt, what.format(n=n)
 
 
 def run_reference(a):
@@ -215,17 +220,22 @@ def run_reference(a):
     inp = wl.make_inputs(a.config)
     oracle.build()
     cores = oracle.num_threads()
-    budget = max(2.0, 120.0 / max(1, a.steps + a.warmup))
+    # the whole run (warm-up + K steps) takes about 90 s of oracle time: each
+    # step is a bounded sample sized once from a calibration run
+    run, what = _oracle_runner(inp)
+    per_step = 90.0 / max(1, a.steps + a.warmup)
+    n0 = 2
+    dt0 = run(n0)
+    n = int(max(1, min(inp.T, n0 * per_step / max(dt0, 1e-6))))
     for _ in range(a.warmup):
-        oracle_sample(inp, budget / 4)
+        run(n)
     tok = 0
     secs = 0.0
-    sample = ""
     for _ in range(a.steps):
-        n, dt, sample = oracle_sample(inp, budget)
+        secs += run(n)
         tok += n
-        secs += dt
     v = tok / secs
+    sample = what.format(n=n)
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
            "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * secs / a.steps,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
@@ -421,8 +431,10 @@ def run_lora(a):
             d2h += pin_dX.numel() * 2
         Ke = max(3, min(K, 200 if not finetune else 20))
 
+        p = lora.Plan(inp.ids, inp.ranks, di, do, stream=stream)
+
         def e2e_step():
-            p = lora.Plan(inp.ids, inp.ranks, di, do, stream=stream)
+            p.rebuild(inp.ids, stream=stream)  # the batch's plan from its host ids (buffers reused)
             with torch.cuda.stream(stream):
                 cp["X"].copy_(pin_X, non_blocking=True)
                 bits = None
@@ -439,7 +451,6 @@ def run_lora(a):
                     pin_dX.copy_(cp["dX"], non_blocking=True)
                 pin_Y.copy_(cp["Y"], non_blocking=True)
             stream.synchronize()
-            p.destroy()
 
         for _ in range(2):
             e2e_step()
@@ -449,6 +460,7 @@ def run_lora(a):
         for _ in range(Ke):
             e2e_step()
         dt = time.perf_counter() - t0
+        p.destroy()
         if world > 1:
             t = torch.tensor([dt], device=dev, dtype=torch.float64)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)

@@ -98,6 +98,19 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
                     int32_t n_adapters, int64_t d_in, int64_t d_out, lora_stream_t stream,
                     lora_plan_t *out);
 
+/* Refill an existing device plan with a new batch (arguments as in
+ * lora_plan_build). The plan's device tables and scratch are reused when they
+ * are large enough and reallocated otherwise, so a serving loop that builds one
+ * plan per batch does not allocate device memory per batch. No work that uses
+ * the plan may be in flight on any stream (the caller orders it, as for any
+ * buffer it overwrites); the call returns after the tables have reached the
+ * device. On LORA_ERR_ARG / LORA_ERR_ID / LORA_ERR_RANK the plan is unchanged;
+ * after LORA_ERR_NOMEM or LORA_ERR_CUDA it holds no device memory and is only
+ * good for lora_plan_destroy. No counterpart in the pages (the plan's device
+ * lifetime is this library's design). */
+int lora_plan_rebuild(lora_plan_t plan, const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
+                      int32_t n_adapters, int64_t d_in, int64_t d_out, lora_stream_t stream);
+
 /* Host-only variant of lora_plan_build: the same grouping and tile layout,
  * but no device buffers (no CUDA call at all). Such a plan can be inspected
  * with lora_plan_get / lora_plan_info and destroyed; lora_linear_fwd rejects

@@ -62,6 +62,7 @@ def load_library():
     L = ctypes.CDLL(LIB_PATH)
     sig = {
         "lora_plan_build": (ctypes.c_int, [_vp, _i64, _vp, _i32, _i64, _i64, _vp, ctypes.POINTER(_vp)]),
+        "lora_plan_rebuild": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _i64, _i64, _vp]),
         "lora_plan_build_host": (ctypes.c_int, [_vp, _i64, _vp, _i32, _i64, _i64, ctypes.POINTER(_vp)]),
         "lora_plan_get": (ctypes.c_int, [_vp, _vp, _vp, _vp]),
         "lora_plan_info": (ctypes.c_int, [_vp, ctypes.POINTER(_Info)]),
@@ -130,6 +131,18 @@ class Plan:
         _check(rc, "lora_plan_build")
         self._h = h
         self.T, self.d_in, self.d_out, self.n_adapters = T, d_in, d_out, n
+
+    def rebuild(self, ids, *, ranks=None, stream=None):
+        """lora_plan_rebuild: the same plan object for a new batch (device buffers
+        reused when they fit); no work using the plan may be in flight."""
+        self._ids = _host_i32(ids)
+        if ranks is not None:
+            self._ranks = _host_i32(ranks)
+        T, n = self._ids.shape[0], self._ranks.shape[0]
+        _check(load_library().lora_plan_rebuild(self._h, self._ids.ctypes.data_as(_vp), T,
+                                                self._ranks.ctypes.data_as(_vp), n, self.d_in, self.d_out,
+                                                _stream(stream)), "lora_plan_rebuild")
+        self.T, self.n_adapters = T, n
 
     @property
     def handle(self):

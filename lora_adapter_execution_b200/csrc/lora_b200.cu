@@ -191,6 +191,7 @@ struct lora_plan {
   const UnitDesc *d_units = nullptr;
   const int32_t *d_mt_order = nullptr;
   const AugBlockDesc *d_augblocks = nullptr;
+  size_t dev_cap = 0, scratch_cap = 0;  // allocated bytes (a rebuild reuses them when they fit)
   int device = 0;
 };
 
@@ -211,22 +212,17 @@ const char *lora_status_string(int code) {
   }
 }
 
-int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_host, int32_t n_adapters,
-                    int64_t d_in, int64_t d_out, lora_stream_t stream, lora_plan_t *out) {
-  if (!out) return LORA_ERR_ARG;
-  lora_plan *pl = new (std::nothrow) lora_plan();
-  if (!pl) return LORA_ERR_NOMEM;
-  int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, pl->hp);
-  if (rc != LORA_OK) {
-    delete pl;
-    return rc;
-  }
+}  // extern "C"
+
+namespace {
+// Device side of a plan: (re)allocate its table block and scratch when they are
+// smaller than the plan needs (kept otherwise, so a rebuilt plan reuses them),
+// then upload the tables. Returns LORA_OK or an error; on error the plan keeps
+// no device memory.
+int upload_plan(lora_plan *pl, lora_stream_t stream) {
   DeviceState *ds = nullptr;
-  rc = device_state(&ds);
-  if (rc != LORA_OK) {
-    delete pl;
-    return rc;
-  }
+  int rc = device_state(&ds);
+  if (rc != LORA_OK) return rc;
   cudaGetDevice(&pl->device);
   const HostPlan &hp = pl->hp;
   auto up = [](size_t b) { return (b + 255) & ~static_cast<size_t>(255); };
@@ -237,16 +233,35 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   const size_t b_order = up(sizeof(int32_t) * hp.mt_order.size());
   const size_t b_aug = up(sizeof(AugBlockDesc) * hp.augblocks.size());
   const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug;
-  if (cudaMalloc(&pl->dev, total) != cudaSuccess) {
-    cudaGetLastError();
-    delete pl;
-    return LORA_ERR_NOMEM;
+  auto release = [&]() {
+    if (pl->dev) cudaFree(pl->dev);
+    if (pl->scratch) cudaFree(pl->scratch);
+    pl->dev = nullptr;
+    pl->scratch = nullptr;
+    pl->dev_cap = 0;
+    pl->scratch_cap = 0;
+  };
+  if (total > pl->dev_cap) {
+    if (pl->dev) cudaFree(pl->dev);
+    pl->dev = nullptr;
+    pl->dev_cap = 0;
+    if (cudaMalloc(&pl->dev, total) != cudaSuccess) {
+      cudaGetLastError();
+      release();
+      return LORA_ERR_NOMEM;
+    }
+    pl->dev_cap = total;
   }
-  if (hp.scratch_bytes > 0 && cudaMalloc(reinterpret_cast<void **>(&pl->scratch), hp.scratch_bytes) != cudaSuccess) {
-    cudaGetLastError();
-    cudaFree(pl->dev);
-    delete pl;
-    return LORA_ERR_NOMEM;
+  if (static_cast<size_t>(hp.scratch_bytes) > pl->scratch_cap) {
+    if (pl->scratch) cudaFree(pl->scratch);
+    pl->scratch = nullptr;
+    pl->scratch_cap = 0;
+    if (cudaMalloc(reinterpret_cast<void **>(&pl->scratch), hp.scratch_bytes) != cudaSuccess) {
+      cudaGetLastError();
+      release();
+      return LORA_ERR_NOMEM;
+    }
+    pl->scratch_cap = static_cast<size_t>(hp.scratch_bytes);
   }
   uint8_t *base = static_cast<uint8_t *>(pl->dev);
   pl->d_perm = reinterpret_cast<const int32_t *>(base);
@@ -276,13 +291,38 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   ok &= cudaStreamSynchronize(stream) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
-    cudaFree(pl->dev);
-    cudaFree(pl->scratch);
-    delete pl;
+    release();
     return LORA_ERR_CUDA;
+  }
+  return LORA_OK;
+}
+}  // namespace
+
+extern "C" {
+
+int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_host, int32_t n_adapters,
+                    int64_t d_in, int64_t d_out, lora_stream_t stream, lora_plan_t *out) {
+  if (!out) return LORA_ERR_ARG;
+  lora_plan *pl = new (std::nothrow) lora_plan();
+  if (!pl) return LORA_ERR_NOMEM;
+  int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, pl->hp);
+  if (rc == LORA_OK) rc = upload_plan(pl, stream);
+  if (rc != LORA_OK) {
+    delete pl;
+    return rc;
   }
   *out = pl;
   return LORA_OK;
+}
+
+int lora_plan_rebuild(lora_plan_t plan, const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
+                      int32_t n_adapters, int64_t d_in, int64_t d_out, lora_stream_t stream) {
+  if (!plan || !plan->dev) return LORA_ERR_ARG;
+  HostPlan hp;
+  int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, hp);
+  if (rc != LORA_OK) return rc;  // the plan is unchanged
+  plan->hp = std::move(hp);
+  return upload_plan(plan, stream);
 }
 
 int lora_plan_build_host(const int32_t *ids_host, int64_t T, const int32_t *ranks_host, int32_t n_adapters,

@@ -171,6 +171,33 @@ def test_dropout_keep_bits_bit_exact(p, seed, d):
     assert (unpacked[:, d:] == 0).all()
 
 
+def test_plan_rebuild_matches_fresh_plan():
+    """A plan rebuilt for another batch (smaller: buffers reused; larger:
+    reallocated) gives bit-identical Y to a freshly built plan, and its grouping
+    equals the oracle's."""
+    import lora_adapter_execution_b200 as lora
+    first = wl.make_inputs("fleet", T=700, d_in=256, d_out=264, n_adapters=90, seed=1)
+    plan = lora.Plan(first.ids, first.ranks, first.d_in, first.d_out)
+    for T, seed in [(300, 2), (1500, 3)]:
+        inp = wl.make_inputs("fleet", T=T, d_in=256, d_out=264, n_adapters=90, seed=seed)
+        plan.rebuild(inp.ids, ranks=inp.ranks)
+        perm, seg = plan.grouping()
+        operm, oseg = oracle.plan(inp.ids, inp.n_adapters)
+        assert (perm == operm).all() and (seg == oseg).all()
+        X, W, A, B = dev_bf16(inp.X), dev_bf16(inp.W), dev_bf16(inp.A_pool), dev_bf16(inp.B_pool)
+        scale = torch.from_numpy(inp.scale).cuda()
+        Y1 = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+        Y2 = torch.empty_like(Y1)
+        lora.linear_fwd(plan, X, W, A, B, scale, Y1)
+        fresh = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out)
+        lora.linear_fwd(fresh, X, W, A, B, scale, Y2)
+        torch.cuda.synchronize()
+        fresh.destroy()
+        assert torch.equal(Y1.view(torch.int16), Y2.view(torch.int16))
+    plan.destroy()
+    assert lora.device_status() == 0
+
+
 def _sample_rows(T, n, seed=0):
     rng = np.random.default_rng(seed)
     edge = [0, 1, 127, 128, T - 1, T - 2, T // 2]
