@@ -12,6 +12,7 @@ constexpr int kTileM = 128;      // tokens per fused-GEMM output tile
 constexpr int kAugBlock = 64;    // augmented-K columns per shrink-output block
 constexpr int kAugBlockBytes = kTileM * kAugBlock * 2;  // 16 KB, one swizzled smem image
 constexpr int kShrinkN = 64;     // rank columns per shrink work unit
+constexpr int kUnitRows = 32;    // token rows per shrink work unit (a chunk's rows are split)
 
 // One 128-token output tile of the sorted order.
 struct TileDesc {
@@ -47,12 +48,18 @@ struct ChunkDesc {
   int32_t tile;
 };
 
-// Shrink work unit: rank columns [n0, n0+nn) of one chunk.
+// Shrink work unit: rank columns [n0, n0+nn) of one chunk, over the chunk's
+// tile-local rows [r0, r1) (at most kUnitRows: small units keep more stages of
+// the shrink's ring in flight).
 struct UnitDesc {
   int32_t chunk;
   int32_t n0;
   int32_t nn;
-  int32_t last;  // 1 if this is the chunk's last piece (it also zero-fills U_save up to r_max)
+  int32_t last;       // 1 if this is the chunk's last rank piece (it also zero-fills U_save up to r_max)
+  int32_t r0, r1;     // tile-local rows
+  int32_t zero_fill;  // 1: the unit also writes the zeros of its image columns in the
+                      // tile rows outside the chunk (one row piece per chunk does)
+  int32_t pad_;
 };
 
 struct HostPlan {

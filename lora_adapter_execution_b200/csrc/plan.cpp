@@ -146,16 +146,35 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
   std::stable_sort(hp.mt_order.begin(), hp.mt_order.end(),
                    [&](int32_t a, int32_t b) { return hp.tiles[a].kaug > hp.tiles[b].kaug; });
 
-  // Shrink units: each chunk's rank columns in pieces of at most 64.
+  // Shrink units: each chunk's rank columns in pieces of at most 64. When chunk
+  // sizes are uneven (the largest has at least 4x the rows of the median, as
+  // with a few popular adapters among many rare ones), chunk rows are also cut
+  // into pieces of at most kUnitRows, so the big chunks do not set the length of
+  // the whole kernel; even chunks stay whole (fewer re-reads of A).
+  int32_t piece_rows = kTileM;
+  if (!hp.chunks.empty()) {
+    std::vector<int32_t> rows;
+    rows.reserve(hp.chunks.size());
+    for (const ChunkDesc &cd : hp.chunks) rows.push_back(cd.hi - cd.lo);
+    const int32_t max_rows = *std::max_element(rows.begin(), rows.end());
+    std::nth_element(rows.begin(), rows.begin() + rows.size() / 2, rows.end());
+    const int32_t median = std::max(1, rows[rows.size() / 2]);
+    if (max_rows >= 4 * median) piece_rows = kUnitRows;
+  }
   for (int32_t c = 0; c < (int32_t)hp.chunks.size(); ++c) {
     const ChunkDesc &cd = hp.chunks[c];
-    for (int32_t n0 = 0; n0 < cd.kc; n0 += kShrinkN) {
-      UnitDesc u{};
-      u.chunk = c;
-      u.n0 = n0;
-      u.nn = std::min(kShrinkN, cd.kc - n0);
-      u.last = (n0 + kShrinkN >= cd.kc) ? 1 : 0;
-      hp.units.push_back(u);
+    for (int32_t r0 = cd.lo; r0 < cd.hi; r0 += piece_rows) {
+      for (int32_t n0 = 0; n0 < cd.kc; n0 += kShrinkN) {
+        UnitDesc u{};
+        u.chunk = c;
+        u.n0 = n0;
+        u.nn = std::min(kShrinkN, cd.kc - n0);
+        u.last = (n0 + kShrinkN >= cd.kc) ? 1 : 0;
+        u.r0 = r0;
+        u.r1 = std::min(cd.hi, r0 + piece_rows);
+        u.zero_fill = r0 == cd.lo ? 1 : 0;
+        hp.units.push_back(u);
+      }
     }
   }
   return LORA_OK;

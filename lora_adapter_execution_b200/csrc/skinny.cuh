@@ -72,8 +72,8 @@ struct UnitGeom {
   int32_t frow;      // first F row of the piece
   int32_t nn;        // piece width (multiple of 16, <= 64)
   int32_t nvalid;    // columns of the piece that are real ranks (rest are zero)
-  // forward only
-  int32_t tile, lo, kcol, kc, adapter, n0, last;
+  // forward only (lo: tile-local first row of the unit; clo, chi: the chunk's rows)
+  int32_t tile, lo, kcol, kc, adapter, n0, last, clo, chi, zero_fill;
 };
 
 __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
@@ -82,14 +82,17 @@ __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
     const UnitDesc ud = p.units[u];
     const ChunkDesc cd = p.chunks[ud.chunk];
     const TileDesc td = p.tiles[cd.tile];
-    g.rows = cd.hi - cd.lo;
-    g.row0 = td.row0 + cd.lo;
-    g.contig = td.contig >= 0 ? td.contig + cd.lo : -1;
+    g.rows = ud.r1 - ud.r0;
+    g.row0 = td.row0 + ud.r0;
+    g.contig = td.contig >= 0 ? td.contig + ud.r0 : -1;
     g.frow = cd.pool_row + ud.n0;
     g.nn = ud.nn;
     g.nvalid = max(0, min(ud.nn, cd.rank - ud.n0));
     g.tile = cd.tile;
-    g.lo = cd.lo;
+    g.lo = ud.r0;
+    g.clo = cd.lo;
+    g.chi = cd.hi;
+    g.zero_fill = ud.zero_fill;
     g.kcol = cd.kofs + ud.n0;
     g.kc = cd.kc;
     g.adapter = cd.adapter;
@@ -111,6 +114,9 @@ __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
     g.kc = 0;
     g.adapter = 0;
     g.last = 0;
+    g.clo = 0;
+    g.chi = 0;
+    g.zero_fill = 0;
   }
   return g;
 }
@@ -369,14 +375,17 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   if (crank == 0) {
     if (p.mode == 0) {
       const float s_a = p.scale[g.adapter] * p.inv_keep;
-      // s·U of the tile, all 128 rows of columns [kcol, kcol + nn) (bf16 hi part)
-      // and [kcol + kc, kcol + kc + nn) (bf16 lo part: the rounding remainder)
+      // s·U of the tile in columns [kcol, kcol + nn) (bf16 hi part) and
+      // [kcol + kc, kcol + kc + nn) (bf16 lo part: the rounding remainder): the
+      // unit's rows, and (one row piece per chunk) the zeros of the tile rows
+      // outside the chunk; the chunk's other rows belong to its other pieces
       uint8_t *img = p.uimg + p.tiles[g.tile].uofs;
       for (int e = threadIdx.x; e < kTileM * (g.nn / 8); e += blockDim.x) {
         const int row = e / (g.nn / 8);
         const int c8 = (e % (g.nn / 8)) * 8;
         const int lr = row - g.lo;
         const bool mine = lr >= 0 && lr < g.rows;
+        if (!mine && !(g.zero_fill && (row < g.clo || row >= g.chi))) continue;
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
