@@ -509,112 +509,117 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   __syncthreads();
   if (split) {
     // --------------------------------------------------- split-K cluster reduction
+    // The tile's table entry and the output rows are fetched before the barrier,
+    // so their global latency overlaps the wait for the slowest peer.
+    const int width = kBN / S;
+    const uint32_t slot0 = smem_u32(smem);
+    const uint32_t out0 = slot0 + (S - 1) * xslot_bytes(S);
+    int mt = 0, nt = 0;
+    tile_coords(tile0 < n_tiles ? tile0 : 0, p, mt, nt);
+    const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+    // a CTA with no K blocks for this tile contributes zeros (its TMEM was never written)
+    const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const bool valid = warp >= 2 && row < td.rows;
+    const int64_t orig =
+        !valid ? 0 : has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
     // barrier: every CTA's MMAs are complete, so every stage ring is idle and may
     // receive; it also orders the receive barriers' initialisation before any
     // remote completion
     cluster_barrier();
-    const int width = kBN / S;
-    const uint32_t slot0 = smem_u32(smem);
-    const uint32_t out0 = slot0 + (S - 1) * xslot_bytes(S);
     if (threadIdx.x == 64) mbar_arrive_expect_tx(recv_bar, (S - 1) * xslot_bytes(S));
-    if (warp >= 2 && tile0 < n_tiles && !*abort_flag) {
-      const int quarter = warp & 3;
-      int mt, nt;
-      tile_coords(tile0, p, mt, nt);
-      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
-      // a CTA with no K blocks for this tile contributes zeros (its TMEM was never written)
-      const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
-      tc_fence_after();
-      // send: TMEM -> registers -> this warp's 4 KB outgoing blocks (column pairs
-      // of one owner: width >= 64), one proxy fence, then the bulk copies into
-      // the owners' slots; they are waited for (read) only before exit
-      int nout = 0;
-      for (int c = 0; c < kBN / 32; c += 2) {
-        const int owner = (c * 32) / width;
-        if (owner == q) continue;
-        uint32_t v0[32], v1[32];
-        tmem_ld32(tmem_base + ((quarter * 32) << 16) + c * 32, v0);
-        tmem_ld32(tmem_base + ((quarter * 32) << 16) + (c + 1) * 32, v1);
-        tmem_wait_ld();
-        uint8_t *b0 = smem + (out0 - slot0) + (quarter * ((kBN - width) / 32) + nout) * kXBlock;
-        uint8_t *b1 = b0 + kXBlock;
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          *reinterpret_cast<float4 *>(b0 + xswz(lane, j)) =
-              any ? make_float4(__uint_as_float(v0[4 * j]), __uint_as_float(v0[4 * j + 1]),
-                                __uint_as_float(v0[4 * j + 2]), __uint_as_float(v0[4 * j + 3]))
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-          *reinterpret_cast<float4 *>(b1 + xswz(lane, j)) =
-              any ? make_float4(__uint_as_float(v1[4 * j]), __uint_as_float(v1[4 * j + 1]),
-                                __uint_as_float(v1[4 * j + 2]), __uint_as_float(v1[4 * j + 3]))
-                  : make_float4(0.f, 0.f, 0.f, 0.f);
-        }
-        nout += 2;
-      }
-      fence_proxy_async_smem();  // the bulk copies (async proxy) read what these stores wrote
-      __syncwarp();
-      if (lane == 0) {
-        int k = 0;
-        for (int c = 0; c < kBN / 32; ++c) {
-          const int owner = (c * 32) / width;
+    bool go = false;
+    if (warp >= 2) {
+      go = tile0 < n_tiles && !*abort_flag;
+      if (go) {
+        // send, step 1: TMEM -> registers -> 4 KB blocks laid out per owner as the
+        // owner's receive slot is ([column block][warp][32 rows x 32 fp32])
+        tc_fence_after();
+        for (int c = 0; c < kBN / 32; c += 2) {
+          const int owner = (c * 32) / width;  // width >= 64: columns c, c + 1 share an owner
           if (owner == q) continue;
-          const uint32_t blk = out0 + static_cast<uint32_t>((quarter * ((kBN - width) / 32) + k) * kXBlock);
-          const int jq = q < owner ? q : q - 1;  // this rank's slot at the owner
+          const int oidx = owner < q ? owner : owner - 1;
           const int cc = (c * 32 - owner * width) / 32;
-          const uint32_t dst = slot0 + static_cast<uint32_t>(jq * xslot_bytes(S) + (cc * 4 + quarter) * kXBlock);
-          bulk_s2s_cluster(map_rank(dst, static_cast<uint32_t>(owner)), blk, kXBlock,
+          uint32_t v0[32], v1[32];
+          tmem_ld32(tmem_base + ((quarter * 32) << 16) + c * 32, v0);
+          tmem_ld32(tmem_base + ((quarter * 32) << 16) + (c + 1) * 32, v1);
+          tmem_wait_ld();
+          uint8_t *b0 = smem + (out0 - slot0) + oidx * xslot_bytes(S) + (cc * 4 + quarter) * kXBlock;
+          uint8_t *b1 = b0 + 4 * kXBlock;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) {
+            *reinterpret_cast<float4 *>(b0 + xswz(lane, j)) =
+                any ? make_float4(__uint_as_float(v0[4 * j]), __uint_as_float(v0[4 * j + 1]),
+                                  __uint_as_float(v0[4 * j + 2]), __uint_as_float(v0[4 * j + 3]))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+            *reinterpret_cast<float4 *>(b1 + xswz(lane, j)) =
+                any ? make_float4(__uint_as_float(v1[4 * j]), __uint_as_float(v1[4 * j + 1]),
+                                  __uint_as_float(v1[4 * j + 2]), __uint_as_float(v1[4 * j + 3]))
+                    : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+        }
+        fence_proxy_async_smem();  // the bulk copies (async proxy) read what these stores wrote
+      }
+      // step 2: once all 4 warps have written, one thread sends each owner its
+      // whole slot (width x 128 fp32) in one bulk copy; the reducing barrier
+      // makes the warps agree on whether to go on
+      go = !epi_bar_or(!go);
+      if (go && threadIdx.x == 64) {
+        for (int owner = 0; owner < S; ++owner) {
+          if (owner == q) continue;
+          const int oidx = owner < q ? owner : owner - 1;
+          const int jq = q < owner ? q : q - 1;  // this rank's slot at the owner
+          bulk_s2s_cluster(map_rank(slot0 + static_cast<uint32_t>(jq * xslot_bytes(S)), static_cast<uint32_t>(owner)),
+                           out0 + static_cast<uint32_t>(oidx * xslot_bytes(S)), xslot_bytes(S),
                            map_rank(recv_bar, static_cast<uint32_t>(owner)));
-          ++k;
         }
         bulk_commit();
       }
       // receive: own partial from TMEM + the other ranks' blocks in rank order
       // (a fixed order, so the result is deterministic)
-      if (!mbar_wait(recv_bar, 0)) {
-        *abort_flag = 1;
-      } else {
-        const int row = quarter * 32 + lane;
-        const bool valid = row < td.rows;
-        const int64_t orig =
-            !valid ? 0 : has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
-        for (int cc = 0; cc < width / 32; ++cc) {
-          uint32_t v[32];
-          tmem_ld32(tmem_base + ((quarter * 32) << 16) + q * width + cc * 32, v);
-          tmem_wait_ld();
-          float s[32];
+      if (go) {
+        if (!mbar_wait(recv_bar, 0)) {
+          *abort_flag = 1;
+        } else {
+          for (int cc = 0; cc < width / 32; ++cc) {
+            uint32_t v[32];
+            tmem_ld32(tmem_base + ((quarter * 32) << 16) + q * width + cc * 32, v);
+            tmem_wait_ld();
+            float s[32];
 #pragma unroll
-          for (int e = 0; e < 32; ++e) s[e] = any ? __uint_as_float(v[e]) : 0.f;
-          for (int src = 0; src < S; ++src) {
-            if (src == q) continue;
-            const int js = src < q ? src : src - 1;
-            const uint8_t *bp = smem + js * xslot_bytes(S) + (cc * 4 + quarter) * kXBlock;
+            for (int e = 0; e < 32; ++e) s[e] = any ? __uint_as_float(v[e]) : 0.f;
+            for (int src = 0; src < S; ++src) {
+              if (src == q) continue;
+              const int js = src < q ? src : src - 1;
+              const uint8_t *bp = smem + js * xslot_bytes(S) + (cc * 4 + quarter) * kXBlock;
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const float4 t = *reinterpret_cast<const float4 *>(bp + xswz(lane, j));
-              s[4 * j + 0] += t.x;
-              s[4 * j + 1] += t.y;
-              s[4 * j + 2] += t.z;
-              s[4 * j + 3] += t.w;
+              for (int j = 0; j < 8; ++j) {
+                const float4 t = *reinterpret_cast<const float4 *>(bp + xswz(lane, j));
+                s[4 * j + 0] += t.x;
+                s[4 * j + 1] += t.y;
+                s[4 * j + 2] += t.z;
+                s[4 * j + 3] += t.w;
+              }
             }
-          }
-          const int col = nt * kBN + q * width + cc * 32;
-          if (valid) {
+            const int col = nt * kBN + q * width + cc * 32;
+            if (valid) {
 #pragma unroll
-            for (int h = 0; h < 4; ++h) {
-              if (col + 8 * h < p.N) {
-                uint4 o;
-                o.x = pack_bf16x2(s[8 * h + 0], s[8 * h + 1]);
-                o.y = pack_bf16x2(s[8 * h + 2], s[8 * h + 3]);
-                o.z = pack_bf16x2(s[8 * h + 4], s[8 * h + 5]);
-                o.w = pack_bf16x2(s[8 * h + 6], s[8 * h + 7]);
-                *reinterpret_cast<uint4 *>(p.out + orig * p.N + col + 8 * h) = o;
+              for (int h = 0; h < 4; ++h) {
+                if (col + 8 * h < p.N) {
+                  uint4 o;
+                  o.x = pack_bf16x2(s[8 * h + 0], s[8 * h + 1]);
+                  o.y = pack_bf16x2(s[8 * h + 2], s[8 * h + 3]);
+                  o.z = pack_bf16x2(s[8 * h + 4], s[8 * h + 5]);
+                  o.w = pack_bf16x2(s[8 * h + 6], s[8 * h + 7]);
+                  *reinterpret_cast<uint4 *>(p.out + orig * p.N + col + 8 * h) = o;
+                }
               }
             }
           }
         }
+        if (threadIdx.x == 64) bulk_wait_read_all();  // the outgoing slots are read before this CTA can exit
       }
-      if (lane == 0) bulk_wait_read_all();  // the outgoing blocks are read before this CTA can exit
-      __syncwarp();
     }
     // every TMEM read is done before warp 1 frees it; every block bound for this
     // CTA has landed (the receive barrier) and every outgoing block has been read
