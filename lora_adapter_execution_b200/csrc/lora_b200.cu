@@ -409,6 +409,19 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   sp.thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
   sp.keep_bits = sp.thr ? keep_bits : nullptr;  // no mask without dropout
   sp.wpr = (hp.d_in + 31) / 32;
+  // units of consecutive tokens copy their keep bits with each stage when the
+  // bit array's rows are 16-byte multiples (d_in % 128 == 0)
+  CUtensorMap mBits16 = mX16;
+  if (sp.keep_bits && sp.wpr % 4 == 0) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(sp.wpr), static_cast<cuuint64_t>(hp.T)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(sp.wpr) * 4};
+    cuuint32_t box[2] = {4, 16};
+    cuuint32_t estr[2] = {1, 1};
+    sp.bits_tma = g_encode(&mBits16, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(sp.keep_bits), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (!sp.bits_tma) mBits16 = mX16;
+  }
   sp.seed = seed;
   sp.inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
   sp.uimg = plan->scratch;
@@ -439,7 +452,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
     lora_gather_rows_kernel<<<blocks, 256, 0, stream>>>(X, plan->d_perm, Xs, hp.T, hp.d_in);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
-  if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mX16, mA16, sp) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mX16, mA16, mBits16, sp) != cudaSuccess) {
     cudaGetLastError();
     return LORA_ERR_CUDA;
   }
@@ -608,7 +621,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mdY16, mB16, sp) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mdY16, mB16, mdY16, sp) != cudaSuccess) {
       cudaGetLastError();
       return LORA_ERR_CUDA;
     }

@@ -55,6 +55,7 @@ struct ShrinkParams {
   // precomputed keep bits (null: hash each element): word t * wpr + col / 32, bit col % 32
   const uint32_t *keep_bits;
   int64_t wpr;
+  int32_t bits_tma;  // 1: units of consecutive tokens copy their bits with each stage (mapBits16)
   uint8_t *uimg;
   float *U_save;
   int32_t r_max;
@@ -171,6 +172,7 @@ __device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
 __global__ void __launch_bounds__(kSkThreads, 2)
     lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows (X, sorted X or dY), box {64, 16}
                        const __grid_constant__ CUtensorMap mapF16,   // F rows, box {64, 16}
+                       const __grid_constant__ CUtensorMap mapBits16,  // keep bits [T, wpr] u32, box {4, 16}
                        const ShrinkParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -191,7 +193,10 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 
   const int Rp = ((g.rows + 15) / 16) * 16;  // rows rounded to the MMA M step
   const int mb = Rp / 16;
-  const int stage_bytes = (Rp + g.nn) * 128;  // X rows then F rows, 128 B (64 bf16) each
+  // a unit of consecutive tokens reads its keep bits from the stage: 4 words
+  // (128 columns, the 16-byte-aligned span holding the stage's 64) per row
+  const bool stage_bits = p.mode == 0 && p.thr != 0 && p.bits_tma && g.contig >= 0;
+  const int stage_bytes = (Rp + g.nn) * 128 + (stage_bits ? Rp * 16 : 0);  // X rows, F rows (, bits)
   const int nstage = min(kSkMaxStages, kSkPool / stage_bytes);
   const int kbeg = static_cast<int>(crank) * p.kslice;
   const int kend = min(p.K, kbeg + p.kslice);
@@ -245,6 +250,11 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         mbar_arrive_expect_tx(fb, stage_bytes);
         for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, xrow + r16);
         for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
+        if (stage_bits) {
+          const uint32_t bb = fbuf + g.nn * 128;
+          for (int r16 = 0; r16 < Rp; r16 += 16)
+            tma_load_2d(bb + r16 * 16, &mapBits16, fb, (col >> 7) * 4, g.contig + r16);
+        }
         if (++stage == nstage) { stage = 0; phase ^= 1; }
       }
     }
@@ -285,7 +295,20 @@ __global__ void __launch_bounds__(kSkThreads, 2)
           }
           if (masked) {
             const int c0 = colbase + 2 * (lane & 3);
-            if (p.keep_bits) {
+            if (stage_bits) {
+              // the stage's bits: [Rp rows][4 words], word (colbase >> 5) & 3 of the
+              // 128-column span; c0 .. c0 + 9 share one word (colbase % 16 == 0)
+              const uint32_t *bs = reinterpret_cast<const uint32_t *>(smem + (fbuf - pool) + g.nn * 128);
+              const int wd = (colbase >> 5) & 3;
+              const int r0 = min(mblk * 16 + (lane >> 2), g.rows - 1);
+              const int r1 = min(mblk * 16 + (lane >> 2) + 8, g.rows - 1);
+              const uint32_t w0 = bs[r0 * 4 + wd] >> (c0 & 31);
+              const uint32_t w1 = bs[r1 * 4 + wd] >> (c0 & 31);
+              a0 = mask_pair(a0, w0 & 1u, (w0 >> 1) & 1u);
+              a1 = mask_pair(a1, w1 & 1u, (w1 >> 1) & 1u);
+              a2 = mask_pair(a2, (w0 >> 8) & 1u, (w0 >> 9) & 1u);
+              a3 = mask_pair(a3, (w1 >> 8) & 1u, (w1 >> 9) & 1u);
+            } else if (p.keep_bits) {
               // colbase is a multiple of 16, so c0 .. c0 + 9 share one 32-bit word
               // (columns past K are zero in the stage; their bits are not read)
               const bool in = colbase < p.K;
