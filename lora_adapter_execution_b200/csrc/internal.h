@@ -50,8 +50,9 @@ struct ChunkDesc {
 
 // Shrink work unit: rank columns [n0, n0+nn) of one chunk, over the chunk's
 // tile-local rows [r0, r1) (at most kUnitRows: small units keep more stages of
-// the shrink's ring in flight).
-struct UnitDesc {
+// the shrink's ring in flight). The fields after zero_fill repeat what the unit's
+// chunk and tile hold, so the shrink reads its whole geometry in one access.
+struct alignas(16) UnitDesc {
   int32_t chunk;
   int32_t n0;
   int32_t nn;
@@ -59,7 +60,17 @@ struct UnitDesc {
   int32_t r0, r1;     // tile-local rows
   int32_t zero_fill;  // 1: the unit also writes the zeros of its image columns in the
                       // tile rows outside the chunk (one row piece per chunk does)
+  int32_t row0;       // sorted position of row r0 (tile row0 + r0)
+  int32_t contig;     // original index of row r0 if the tile's tokens are consecutive, else -1
+  int32_t frow;       // first A_pool row of the piece (the adapter's pool_row + n0)
+  int32_t nvalid;     // columns of the piece that are real ranks
+  int32_t tile;
+  int32_t clo, chi;   // the chunk's tile-local rows
+  int32_t kcol;       // augmented-K column of the piece's hi part (chunk kofs + n0)
+  int32_t kc;         // the chunk's rank rounded up to 16 (hi-to-lo column distance)
+  int32_t adapter;
   int32_t pad_;
+  int64_t uofs;       // byte offset of the tile's s*U image in the plan scratch
 };
 
 struct HostPlan {

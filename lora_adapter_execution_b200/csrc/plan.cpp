@@ -173,6 +173,18 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
         u.r0 = r0;
         u.r1 = std::min(cd.hi, r0 + piece_rows);
         u.zero_fill = r0 == cd.lo ? 1 : 0;
+        const TileDesc &td = hp.tiles[cd.tile];
+        u.row0 = td.row0 + r0;
+        u.contig = td.contig >= 0 ? td.contig + r0 : -1;
+        u.frow = cd.pool_row + n0;
+        u.nvalid = std::max(0, std::min(u.nn, cd.rank - n0));
+        u.tile = cd.tile;
+        u.clo = cd.lo;
+        u.chi = cd.hi;
+        u.kcol = cd.kofs + n0;
+        u.kc = cd.kc;
+        u.adapter = cd.adapter;
+        u.uofs = td.uofs;
         hp.units.push_back(u);
       }
     }

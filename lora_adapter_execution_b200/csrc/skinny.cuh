@@ -30,13 +30,17 @@
 
 namespace lora {
 
-constexpr int kSkConsumerWarps = 8;
+constexpr int kSkConsumerWarps = 4;
 constexpr int kSkThreads = (kSkConsumerWarps + 1) * 32;  // + 1 producer warp
 constexpr int kSkBK = 64;                                 // columns per stage (one 128-byte swizzled row)
-constexpr int kSkPool = 72 * 1024;                        // stage ring (also the reduction scratch)
+constexpr int kSkPool = 108 * 1024;                       // stage ring (also the reduction scratch)
 constexpr int kSkMaxStages = 16;
+constexpr int kSkRedBytes = kSkConsumerWarps * 32 * kShrinkN * 4;  // per-warp partials, fp32
 constexpr int kSkFinBytes = kTileM * kShrinkN * 4;        // CTA partial [128 x 64] fp32
-constexpr int kSkSmem = 1024 + kSkPool + kSkFinBytes + 2 * kSkMaxStages * 8 + 64;
+constexpr int kSkSmem = 1024 + kSkPool + 2 * kSkMaxStages * 8 + 64;
+// the partials and the CTA sum reuse the idle ring; two CTAs fit on an SM
+static_assert(kSkRedBytes + kSkFinBytes <= kSkPool, "shrink reduction scratch exceeds the stage pool");
+static_assert(2 * (kSkSmem + 1024) <= 228 * 1024, "two shrink CTAs must fit on an SM");
 
 struct ShrinkParams {
   int32_t mode;     // 0: forward shrink over plan units; 1: backward dU over consecutive tiles
@@ -75,30 +79,30 @@ struct UnitGeom {
   int32_t nvalid;    // columns of the piece that are real ranks (rest are zero)
   // forward only (lo: tile-local first row of the unit; clo, chi: the chunk's rows)
   int32_t tile, lo, kcol, kc, adapter, n0, last, clo, chi, zero_fill;
+  int64_t uofs;  // the tile's image offset
 };
 
 __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
   UnitGeom g;
   if (p.mode == 0) {
-    const UnitDesc ud = p.units[u];
-    const ChunkDesc cd = p.chunks[ud.chunk];
-    const TileDesc td = p.tiles[cd.tile];
+    const UnitDesc ud = p.units[u];  // one 80-byte record
     g.rows = ud.r1 - ud.r0;
-    g.row0 = td.row0 + ud.r0;
-    g.contig = td.contig >= 0 ? td.contig + ud.r0 : -1;
-    g.frow = cd.pool_row + ud.n0;
+    g.row0 = ud.row0;
+    g.contig = ud.contig;
+    g.frow = ud.frow;
     g.nn = ud.nn;
-    g.nvalid = max(0, min(ud.nn, cd.rank - ud.n0));
-    g.tile = cd.tile;
+    g.nvalid = ud.nvalid;
+    g.tile = ud.tile;
     g.lo = ud.r0;
-    g.clo = cd.lo;
-    g.chi = cd.hi;
+    g.clo = ud.clo;
+    g.chi = ud.chi;
     g.zero_fill = ud.zero_fill;
-    g.kcol = cd.kofs + ud.n0;
-    g.kc = cd.kc;
-    g.adapter = cd.adapter;
+    g.kcol = ud.kcol;
+    g.kc = ud.kc;
+    g.adapter = ud.adapter;
     g.n0 = ud.n0;
     g.last = ud.last;
+    g.uofs = ud.uofs;
   } else {
     const int m = u / p.npieces;
     const int piece = u % p.npieces;
@@ -118,6 +122,7 @@ __device__ __forceinline__ UnitGeom unit_geom(const ShrinkParams &p, int u) {
     g.clo = 0;
     g.chi = 0;
     g.zero_fill = 0;
+    g.uofs = 0;
   }
   return g;
 }
@@ -161,10 +166,160 @@ __device__ __forceinline__ uint32_t map_to_rank(uint32_t saddr, uint32_t rank) {
   asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(saddr), "r"(rank));
   return r;
 }
-__device__ __forceinline__ float ld_dsmem_f32(uint32_t addr) {
-  float v;
-  asm volatile("ld.shared::cluster.f32 %0, [%1];" : "=f"(v) : "r"(addr) : "memory");
+__device__ __forceinline__ float4 ld_dsmem_f32x4(uint32_t addr) {
+  float4 v;
+  asm volatile("ld.shared::cluster.v4.f32 {%0, %1, %2, %3}, [%4];"
+               : "=f"(v.x), "=f"(v.y), "=f"(v.z), "=f"(v.w)
+               : "r"(addr)
+               : "memory");
   return v;
+}
+
+// AND the A-fragment registers v01 (columns c, c + 1) and v89 (c + 8, c + 9)
+// of one row with that row's keep bits x (bit 0 = column c): the two shifts put
+// the bits on byte sign positions and prmt's sign-replicate selectors widen
+// each to a 16-bit all-ones / all-zeros lane mask.
+__device__ __forceinline__ void apply_keep(uint32_t &v01, uint32_t &v89, uint32_t x) {
+  const uint32_t a = x << 7, b = x << 14;
+  uint32_t m01, m89;
+  asm("prmt.b32 %0, %1, %2, 0xDD88;" : "=r"(m01) : "r"(a), "r"(b));
+  asm("prmt.b32 %0, %1, %2, 0xEE99;" : "=r"(m89) : "r"(a), "r"(b));
+  v01 &= m01;
+  v89 &= m89;
+}
+
+// What one consumer warp of the shrink needs to walk the stage ring.
+struct ShrinkWarp {
+  uint32_t pool, full0, empty0;
+  int stage_bytes, nstage, nblk, kbeg, Rp, mb, MW, KW, mphase, kphase;
+  int mask;  // dropout on X: 0 none, 1 keep bits staged with the rows, 2 keep bits from HBM, 3 hash
+};
+
+constexpr int kSkConsumerBar = 1;  // named barrier of the 256 consumer threads
+
+// One consumer warp: m16n8k16 MMAs of its m-blocks (mphase and, when the unit
+// has more, mphase + MW) over the stages kphase, kphase + KW, ... against the
+// NB16 16-column blocks of the F rows. The ldmatrix offsets inside a stage are
+// the same for every stage (128-byte swizzle, 1024-byte aligned stage parts),
+// so they are computed once. After the last stage the warp writes its partial
+// sums to red[warp][slot * 16 + row][col] in the freed stage pool.
+template <int NB16>
+__device__ __forceinline__ void shrink_consume(const ShrinkWarp &w, const ShrinkParams &p, const UnitGeom &g,
+                                               const int64_t (&orow)[2][2], const uint8_t *smem,
+                                               volatile int *abort_flag, float *red, int warp, int lane) {
+  float acc[2][2 * NB16][4];
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int j = 0; j < 2 * NB16; ++j)
+#pragma unroll
+      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
+
+  const int l7 = lane & 7, mi = lane >> 3;
+  uint32_t aoff[4], boff[4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    // ldmatrix x4: lanes 8q .. 8q + 7 address the rows of matrix q; a row's
+    // 16-byte chunk c sits at chunk c ^ (row & 7), and row & 7 == lane & 7
+    aoff[ks] = ((mi & 1) * 8 + l7) * 128 + ((((2 * ks + (mi >> 1)) ^ l7) & 7) << 4);
+    boff[ks] = ((mi >> 1) * 8 + l7) * 128 + ((((2 * ks + (mi & 1)) ^ l7) & 7) << 4);
+  }
+  const bool two = w.mphase + w.MW < w.mb;  // the warp has a second m-block
+  const int q2 = 2 * (lane & 3);
+  int rr[2][2];  // unit rows of the lane's fragments, clamped to the valid rows
+#pragma unroll
+  for (int i = 0; i < 2; ++i)
+#pragma unroll
+    for (int h = 0; h < 2; ++h) rr[i][h] = min((w.mphase + i * w.MW) * 16 + (lane >> 2) + 8 * h, g.rows - 1);
+
+  for (int b = w.kphase; b < w.nblk; b += w.KW) {
+    const int stage = b % w.nstage;
+    const uint32_t phase = static_cast<uint32_t>(b / w.nstage) & 1u;
+    if (!mbar_wait(w.full0 + 8 * stage, phase)) { *abort_flag = 1; break; }
+    const uint32_t xb = w.pool + stage * w.stage_bytes;
+    const uint32_t fbuf = xb + w.Rp * 128;
+    const int col = w.kbeg + b * kSkBK;  // first column of the stage, a multiple of 64
+    // keep bits of the lane's rows for the stage's 64 columns: words
+    // col / 32 and col / 32 + 1 of each row
+    uint32_t kw[2][2][2];
+    if (w.mask == 1) {
+      // the stage holds words 4 * (col / 128) .. + 3 of every row; ours are
+      // words (col / 32) & 3 (0 or 2) and the next
+      const uint32_t *bs = reinterpret_cast<const uint32_t *>(smem + (fbuf - w.pool) + g.nn * 128);
+      const int wd = (col >> 5) & 3;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (i == 1 && !two) break;
+          const uint2 v = *reinterpret_cast<const uint2 *>(bs + rr[i][h] * 4 + wd);
+          kw[i][h][0] = v.x;
+          kw[i][h][1] = v.y;
+        }
+    } else if (w.mask == 2) {
+      // columns past K are zero in the stage: their bits are not read
+      const bool second = col + 32 < p.K;
+#pragma unroll
+      for (int i = 0; i < 2; ++i)
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          if (i == 1 && !two) break;
+          const uint32_t *src = p.keep_bits + orow[i][h] * p.wpr + (col >> 5);
+          kw[i][h][0] = __ldg(src);
+          kw[i][h][1] = second ? __ldg(src + 1) : 0u;
+        }
+    }
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t bf[NB16][4];
+#pragma unroll
+      for (int jj = 0; jj < NB16; ++jj)
+        ldsm_x4(fbuf + boff[ks] + jj * 2048, bf[jj][0], bf[jj][1], bf[jj][2], bf[jj][3]);
+#pragma unroll
+      for (int i = 0; i < 2; ++i) {
+        if (i == 1 && !two) break;
+        const int mblk = w.mphase + i * w.MW;
+        uint32_t a0, a1, a2, a3;
+        ldsm_x4(xb + aoff[ks] + mblk * 2048, a0, a1, a2, a3);
+        if (w.mask == 1 || w.mask == 2) {
+          const int s = (ks & 1) * 16 + q2;
+          apply_keep(a0, a2, kw[i][0][ks >> 1] >> s);
+          apply_keep(a1, a3, kw[i][1][ks >> 1] >> s);
+        } else if (w.mask == 3) {
+          const int c0 = col + ks * 16 + q2;
+          a0 = mask_pair(a0, keep_elem(p.seed, p.thr, orow[i][0], c0, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 1, p.K));
+          a1 = mask_pair(a1, keep_elem(p.seed, p.thr, orow[i][1], c0, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 1, p.K));
+          a2 = mask_pair(a2, keep_elem(p.seed, p.thr, orow[i][0], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 9, p.K));
+          a3 = mask_pair(a3, keep_elem(p.seed, p.thr, orow[i][1], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 9, p.K));
+        }
+#pragma unroll
+        for (int jj = 0; jj < NB16; ++jj) {
+          mma_bf16_16816(acc[i][2 * jj], a0, a1, a2, a3, bf[jj][0], bf[jj][1]);
+          mma_bf16_16816(acc[i][2 * jj + 1], a0, a1, a2, a3, bf[jj][2], bf[jj][3]);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(w.empty0 + 8 * stage);
+  }
+
+  // every consumer warp is past its last stage: every TMA of the ring has
+  // landed and been read, so the pool may be overwritten
+  asm volatile("bar.sync %0, %1;" ::"n"(kSkConsumerBar), "n"(kSkConsumerWarps * 32) : "memory");
+  float *base = red + (warp * 32) * kShrinkN;
+#pragma unroll
+  for (int i = 0; i < 2; ++i) {
+    if (i == 1 && !two) break;
+#pragma unroll
+    for (int j = 0; j < 2 * NB16; ++j) {
+      const int r = i * 16 + (lane >> 2);
+      const int c = j * 8 + q2;
+      base[r * kShrinkN + c] = acc[i][j][0];
+      base[r * kShrinkN + c + 1] = acc[i][j][1];
+      base[(r + 8) * kShrinkN + c] = acc[i][j][2];
+      base[(r + 8) * kShrinkN + c + 1] = acc[i][j][3];
+    }
+  }
 }
 
 // Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
@@ -178,8 +333,8 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
   const uint32_t pool = smem_u32(smem);
-  float *fin = reinterpret_cast<float *>(smem + kSkPool);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSkPool + kSkFinBytes);
+  float *fin = reinterpret_cast<float *>(smem + kSkRedBytes);  // in the pool, after the partials
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSkPool);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * kSkMaxStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kSkMaxStages);
@@ -189,6 +344,11 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   const int unit = blockIdx.x / p.ksplit;
   const uint32_t crank = cluster_ctarank();
   pdl_launch_dependents();  // the fused GEMM may set itself up meanwhile
+  if (warp == kSkConsumerWarps && lane == 0) {
+    prefetch_tmap(&mapIn16);
+    prefetch_tmap(&mapF16);
+    if (p.bits_tma) prefetch_tmap(&mapBits16);
+  }
   const UnitGeom g = unit_geom(p, unit);  // plan tables: written before any kernel of the forward
 
   const int Rp = ((g.rows + 15) / 16) * 16;  // rows rounded to the MMA M step
@@ -196,7 +356,10 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   // a unit of consecutive tokens reads its keep bits from the stage: 4 words
   // (128 columns, the 16-byte-aligned span holding the stage's 64) per row
   const bool stage_bits = p.mode == 0 && p.thr != 0 && p.bits_tma && g.contig >= 0;
-  const int stage_bytes = (Rp + g.nn) * 128 + (stage_bits ? Rp * 16 : 0);  // X rows, F rows (, bits)
+  // a stage: X rows, F rows (, bits); the next stage starts on a 1024-byte
+  // boundary, as the 128-byte swizzle of its TMA boxes requires
+  const int stage_tx = (Rp + g.nn) * 128 + (stage_bits ? Rp * 16 : 0);
+  const int stage_bytes = (stage_tx + 1023) & ~1023;
   const int nstage = min(kSkMaxStages, kSkPool / stage_bytes);
   const int kbeg = static_cast<int>(crank) * p.kslice;
   const int kend = min(p.K, kbeg + p.kslice);
@@ -221,15 +384,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   // X (or its sorted copy from the row gather) and everything else the launch
   // reads or writes come after the previous kernel on the stream has completed
   pdl_wait();
-  const int nb8 = g.nn / 8;
-
-  float acc[2][8][4];
-#pragma unroll
-  for (int i = 0; i < 2; ++i)
-#pragma unroll
-    for (int j = 0; j < 8; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
 
   if (warp == kSkConsumerWarps) {
     // -------------------------------------------------------------- producer
@@ -247,7 +401,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         const uint32_t xb = pool + stage * stage_bytes;
         const uint32_t fbuf = xb + Rp * 128;
         const int col = kbeg + b * kSkBK;
-        mbar_arrive_expect_tx(fb, stage_bytes);
+        mbar_arrive_expect_tx(fb, stage_tx);
         for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, xrow + r16);
         for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
         if (stage_bits) {
@@ -260,165 +414,149 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     }
   } else {
     // -------------------------------------------------------------- consumers
-    const int mphase = warp % MW;
-    const int kphase = warp / MW;
+    ShrinkWarp w;
+    w.pool = pool;
+    w.full0 = full0;
+    w.empty0 = empty0;
+    w.stage_bytes = stage_bytes;
+    w.nstage = nstage;
+    w.nblk = nblk;
+    w.kbeg = kbeg;
+    w.Rp = Rp;
+    w.mb = mb;
+    w.MW = MW;
+    w.KW = KW;
+    w.mphase = warp % MW;
+    w.kphase = warp / MW;
+    w.mask = (p.mode != 0 || p.thr == 0) ? 0 : (stage_bits ? 1 : (p.keep_bits ? 2 : 3));
     // original token index of the two rows this lane's fragments touch, per m-block slot
     int64_t orow[2][2];
 #pragma unroll
     for (int i = 0; i < 2; ++i)
 #pragma unroll
       for (int h = 0; h < 2; ++h) {
-        const int r = (mphase + i * MW) * 16 + (lane >> 2) + 8 * h;
+        const int r = (w.mphase + i * MW) * 16 + (lane >> 2) + 8 * h;
         const int rc = min(r, g.rows - 1);
         orow[i][h] = g.contig >= 0 ? static_cast<int64_t>(g.contig + rc)
                                    : (p.mode == 0 ? static_cast<int64_t>(p.perm[g.row0 + rc]) : 0);
       }
-    const bool masked = p.mode == 0 && p.thr != 0;
-    for (int b = kphase; b < nblk; b += KW) {
-      const int stage = b % nstage;
-      const uint32_t phase = static_cast<uint32_t>(b / nstage) & 1u;
-      if (!mbar_wait(full0 + 8 * stage, phase)) { *abort_flag = 1; break; }
-      const uint32_t xb = pool + stage * stage_bytes;
-      const uint32_t fbuf = xb + Rp * 128;
-      for (int ks = 0; ks < 4; ++ks) {  // k16 steps of the stage
-        const int colbase = kbeg + b * kSkBK + ks * 16;
-#pragma unroll
-        for (int i = 0; i < 2; ++i) {
-          const int mblk = mphase + i * MW;
-          if (mblk >= mb) break;
-          uint32_t a0, a1, a2, a3;
-          {
-            const int mi = lane >> 3;
-            const int r = mblk * 16 + (mi & 1) * 8 + (lane & 7);
-            const int chunk = ks * 2 + (mi >> 1);
-            ldsm_x4(xb + r * 128 + (((chunk ^ (r & 7)) & 7) << 4), a0, a1, a2, a3);
-          }
-          if (masked) {
-            const int c0 = colbase + 2 * (lane & 3);
-            if (stage_bits) {
-              // the stage's bits: [Rp rows][4 words], word (colbase >> 5) & 3 of the
-              // 128-column span; c0 .. c0 + 9 share one word (colbase % 16 == 0)
-              const uint32_t *bs = reinterpret_cast<const uint32_t *>(smem + (fbuf - pool) + g.nn * 128);
-              const int wd = (colbase >> 5) & 3;
-              const int r0 = min(mblk * 16 + (lane >> 2), g.rows - 1);
-              const int r1 = min(mblk * 16 + (lane >> 2) + 8, g.rows - 1);
-              const uint32_t w0 = bs[r0 * 4 + wd] >> (c0 & 31);
-              const uint32_t w1 = bs[r1 * 4 + wd] >> (c0 & 31);
-              a0 = mask_pair(a0, w0 & 1u, (w0 >> 1) & 1u);
-              a1 = mask_pair(a1, w1 & 1u, (w1 >> 1) & 1u);
-              a2 = mask_pair(a2, (w0 >> 8) & 1u, (w0 >> 9) & 1u);
-              a3 = mask_pair(a3, (w1 >> 8) & 1u, (w1 >> 9) & 1u);
-            } else if (p.keep_bits) {
-              // colbase is a multiple of 16, so c0 .. c0 + 9 share one 32-bit word
-              // (columns past K are zero in the stage; their bits are not read)
-              const bool in = colbase < p.K;
-              const uint32_t w0 = in ? __ldg(p.keep_bits + orow[i][0] * p.wpr + (colbase >> 5)) >> (c0 & 31) : 0u;
-              const uint32_t w1 = in ? __ldg(p.keep_bits + orow[i][1] * p.wpr + (colbase >> 5)) >> (c0 & 31) : 0u;
-              a0 = mask_pair(a0, w0 & 1u, (w0 >> 1) & 1u);
-              a1 = mask_pair(a1, w1 & 1u, (w1 >> 1) & 1u);
-              a2 = mask_pair(a2, (w0 >> 8) & 1u, (w0 >> 9) & 1u);
-              a3 = mask_pair(a3, (w1 >> 8) & 1u, (w1 >> 9) & 1u);
-            } else {
-              a0 = mask_pair(a0, keep_elem(p.seed, p.thr, orow[i][0], c0, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 1, p.K));
-              a1 = mask_pair(a1, keep_elem(p.seed, p.thr, orow[i][1], c0, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 1, p.K));
-              a2 = mask_pair(a2, keep_elem(p.seed, p.thr, orow[i][0], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][0], c0 + 9, p.K));
-              a3 = mask_pair(a3, keep_elem(p.seed, p.thr, orow[i][1], c0 + 8, p.K), keep_elem(p.seed, p.thr, orow[i][1], c0 + 9, p.K));
-            }
-          }
-#pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            if (2 * jj >= nb8) break;
-            uint32_t b0, b1, b2, b3;
-            const int mi = lane >> 3;
-            const int nr = jj * 16 + (mi >> 1) * 8 + (lane & 7);
-            const int chunk = ks * 2 + (mi & 1);
-            ldsm_x4(fbuf + nr * 128 + (((chunk ^ (nr & 7)) & 7) << 4), b0, b1, b2, b3);
-            mma_bf16_16816(acc[i][2 * jj], a0, a1, a2, a3, b0, b1);
-            mma_bf16_16816(acc[i][2 * jj + 1], a0, a1, a2, a3, b2, b3);
-          }
-        }
-      }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+    float *red = reinterpret_cast<float *>(smem);
+    switch (g.nn >> 4) {
+      case 1: shrink_consume<1>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+      case 2: shrink_consume<2>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+      case 3: shrink_consume<3>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+      default: shrink_consume<4>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
     }
   }
-  __syncthreads();  // every TMA landed and was consumed: the pool is free for the reduction
 
   // ---------------------------------------------------------------- CTA reduction
-  // red[w][slot*16 + row][col], fp32, in the (now idle) stage pool
+  // the consumers left their partial sums in red[w][slot*16 + row][col] (fp32,
+  // the idle stage pool); fin[row][col] = the sum over the KW warps of a row.
+  // Threads work on float4 column groups: nq per row, rpp rows per pass.
   float *red = reinterpret_cast<float *>(smem);
-  if (warp < kSkConsumerWarps) {
-    const int mphase = warp % MW;
-#pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int mblk = mphase + i * MW;
-      if (mblk >= mb) break;
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        if (j >= nb8) break;
-        const int r = i * 16 + (lane >> 2);
-        const int c = j * 8 + 2 * (lane & 3);
-        float *base = red + (warp * 32) * kShrinkN;
-        base[r * kShrinkN + c] = acc[i][j][0];
-        base[r * kShrinkN + c + 1] = acc[i][j][1];
-        base[(r + 8) * kShrinkN + c] = acc[i][j][2];
-        base[(r + 8) * kShrinkN + c + 1] = acc[i][j][3];
-      }
-    }
-  }
   __syncthreads();
-  for (int e = threadIdx.x; e < Rp * g.nn; e += blockDim.x) {
-    const int r = e / g.nn, c = e % g.nn;
-    const int mblk = r / 16;
-    const int mphase = mblk % MW;
-    const int slot = mblk / MW;
-    float s = 0.f;
-    for (int kp = 0; kp < KW; ++kp) {
-      const int w = kp * MW + mphase;
-      s += red[(w * 32 + slot * 16 + (r & 15)) * kShrinkN + c];
+  const int nq = g.nn >> 2;
+  const int rpp = static_cast<int>(blockDim.x) / nq;
+  const int tq = static_cast<int>(threadIdx.x) % nq;
+  const int tr = static_cast<int>(threadIdx.x) / nq;
+  int lmw = 0;
+  while ((1 << lmw) < MW) ++lmw;
+  if (tr < rpp) {
+    for (int r = tr; r < Rp; r += rpp) {
+      const int mblk = r >> 4;
+      const int row_in = ((mblk >> lmw) << 4) + (r & 15);  // slot * 16 + row in the m-block
+      float4 s4 = make_float4(0.f, 0.f, 0.f, 0.f);
+      for (int kp = 0; kp < KW; ++kp) {
+        const int w = kp * MW + (mblk & (MW - 1));
+        const float4 v = *reinterpret_cast<const float4 *>(red + (w * 32 + row_in) * kShrinkN + tq * 4);
+        s4.x += v.x;
+        s4.y += v.y;
+        s4.z += v.z;
+        s4.w += v.w;
+      }
+      *reinterpret_cast<float4 *>(fin + r * kShrinkN + tq * 4) = s4;
     }
-    fin[r * kShrinkN + c] = s;
   }
-  cluster_sync_all();  // every rank's fin is final
 
-  if (crank == 0) {
-    if (p.ksplit > 1) {
-      for (int e = threadIdx.x; e < Rp * g.nn; e += blockDim.x) {
-        const int r = e / g.nn, c = e % g.nn;
-        const uint32_t la = smem_u32(fin + r * kShrinkN + c);
-        float s = fin[r * kShrinkN + c];
-        for (uint32_t q = 1; q < static_cast<uint32_t>(p.ksplit); ++q) s += ld_dsmem_f32(map_to_rank(la, q));
-        fin[r * kShrinkN + c] = s;
+  // ---------------------------------------------------------------- cluster reduction
+  // rank q completes the tile rows [tr0, tr1): it sums those of the unit's rows
+  // over the ranks (in rank order, so the result does not depend on which rank
+  // sums) and writes their outputs; the ranks' shares run in parallel
+  const int ksp = p.ksplit;
+  const int tr0 = static_cast<int>(crank) * kTileM / ksp;
+  const int tr1 = (static_cast<int>(crank) + 1) * kTileM / ksp;
+  const int lr0 = max(0, tr0 - g.lo);
+  const int lr1 = min(g.rows, tr1 - g.lo);
+  if (ksp > 1) {
+    cluster_sync_all();  // every rank's fin is final
+    if (tr < rpp) {
+      for (int lr = lr0 + tr; lr < lr1; lr += 4 * rpp) {
+        // up to 4 rows per thread with their remote loads in flight together
+        float4 part[4][4];  // [row][rank]
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int rr = min(lr + u * rpp, lr1 - 1);
+          const uint32_t la = smem_u32(fin + rr * kShrinkN + tq * 4);
+#pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            if (q >= ksp) break;
+            part[u][q] = q == static_cast<int>(crank) ? *reinterpret_cast<const float4 *>(fin + rr * kShrinkN + tq * 4)
+                                                     : ld_dsmem_f32x4(map_to_rank(la, static_cast<uint32_t>(q)));
+          }
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int rr = lr + u * rpp;
+          if (rr >= lr1) break;
+          float4 s4 = part[u][0];
+#pragma unroll
+          for (int q = 1; q < 4; ++q) {
+            if (q >= ksp) break;
+            s4.x += part[u][q].x;
+            s4.y += part[u][q].y;
+            s4.z += part[u][q].z;
+            s4.w += part[u][q].w;
+          }
+          // only this rank reads these rows of fin from here on
+          *reinterpret_cast<float4 *>(fin + rr * kShrinkN + tq * 4) = s4;
+        }
       }
     }
-    // the peers only read their own fin below this point; rank 0 owns fin now
+    cluster_sync_all();  // the peers' fin was read: every rank may go on and exit
   }
-  cluster_sync_all();  // peers may exit only after rank 0 has read their fin
 
-  if (crank == 0) {
-    if (p.mode == 0) {
-      const float s_a = p.scale[g.adapter] * p.inv_keep;
-      // s·U of the tile in columns [kcol, kcol + nn) (bf16 hi part) and
-      // [kcol + kc, kcol + kc + nn) (bf16 lo part: the rounding remainder): the
-      // unit's rows, and (one row piece per chunk) the zeros of the tile rows
-      // outside the chunk; the chunk's other rows belong to its other pieces
-      uint8_t *img = p.uimg + p.tiles[g.tile].uofs;
-      for (int e = threadIdx.x; e < kTileM * (g.nn / 8); e += blockDim.x) {
-        const int row = e / (g.nn / 8);
-        const int c8 = (e % (g.nn / 8)) * 8;
+  if (p.mode == 0) {
+    const float s_a = p.scale[g.adapter] * p.inv_keep;
+    // s·U of the tile in columns [kcol, kcol + nn) (bf16 hi part) and
+    // [kcol + kc, kcol + kc + nn) (bf16 lo part: the rounding remainder): the
+    // unit's rows, and (one row piece per chunk) the zeros of the tile rows
+    // outside the chunk; the chunk's other rows belong to its other pieces
+    uint8_t *img = p.uimg + g.uofs;
+    const int n8 = g.nn >> 3;
+    const int rp8 = static_cast<int>(blockDim.x) / n8;
+    const int t8 = static_cast<int>(threadIdx.x) % n8;
+    const int trow = static_cast<int>(threadIdx.x) / n8;
+    if (trow < rp8) {
+      const int c8 = t8 * 8;
+      for (int row = tr0 + trow; row < tr1; row += rp8) {
         const int lr = row - g.lo;
         const bool mine = lr >= 0 && lr < g.rows;
         if (!mine && !(g.zero_fill && (row < g.clo || row >= g.chi))) continue;
+        float v[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j) v[j] = 0.f;
+        if (mine) {
+          const float4 x0 = *reinterpret_cast<const float4 *>(fin + lr * kShrinkN + c8);
+          const float4 x1 = *reinterpret_cast<const float4 *>(fin + lr * kShrinkN + c8 + 4);
+          const float xs[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = c8 + j < g.nvalid ? xs[j] * s_a : 0.f;
+        }
         uint32_t hi[4], lo[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          float v0 = 0.f, v1 = 0.f;
-          if (mine) {
-            if (c8 + 2 * j < g.nvalid) v0 = fin[lr * kShrinkN + c8 + 2 * j] * s_a;
-            if (c8 + 2 * j + 1 < g.nvalid) v1 = fin[lr * kShrinkN + c8 + 2 * j + 1] * s_a;
-          }
-          hi[j] = pack_bf16x2(v0, v1);
-          lo[j] = pack_bf16x2(v0 - bf16_lo(hi[j]), v1 - bf16_hi(hi[j]));
+          hi[j] = pack_bf16x2(v[2 * j], v[2 * j + 1]);
+          lo[j] = pack_bf16x2(v[2 * j] - bf16_lo(hi[j]), v[2 * j + 1] - bf16_hi(hi[j]));
         }
         const int col = g.kcol + c8;
         uint8_t *dst = img + (col / kAugBlock) * kAugBlockBytes + sw128_offset(row, col % kAugBlock);
@@ -427,23 +565,24 @@ __global__ void __launch_bounds__(kSkThreads, 2)
         uint8_t *dst2 = img + (col2 / kAugBlock) * kAugBlockBytes + sw128_offset(row, col2 % kAugBlock);
         *reinterpret_cast<uint4 *>(dst2) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
       }
-      if (p.U_save) {
-        const int cend = g.last ? p.r_max : min(p.r_max, g.n0 + g.nn);
-        const int ncol = max(0, cend - g.n0);
-        for (int e = threadIdx.x; e < g.rows * ncol; e += blockDim.x) {
-          const int lr = e / ncol, c = e % ncol;
-          const int64_t orig = g.contig >= 0 ? g.contig + lr : p.perm[g.row0 + lr];
-          const float v = c < g.nvalid ? fin[lr * kShrinkN + c] * p.inv_keep : 0.f;
-          p.U_save[orig * p.r_max + g.n0 + c] = v;
-        }
+    }
+    if (p.U_save) {
+      // one warp per row: columns n0 .. cend of the token's U_save row (zeros
+      // past the adapter's rank up to r_max on the chunk's last piece)
+      const int cend = g.last ? p.r_max : min(p.r_max, g.n0 + g.nn);
+      const int ncol = max(0, cend - g.n0);
+      const int nw = static_cast<int>(blockDim.x) >> 5;
+      for (int lr = lr0 + warp; lr < lr1; lr += nw) {
+        const int64_t orig = g.contig >= 0 ? static_cast<int64_t>(g.contig + lr) : p.perm[g.row0 + lr];
+        float *dst = p.U_save + orig * p.r_max + g.n0;
+        for (int c = lane; c < ncol; c += 32) dst[c] = c < g.nvalid ? fin[lr * kShrinkN + c] * p.inv_keep : 0.f;
       }
-    } else {
-      for (int e = threadIdx.x; e < g.rows * g.nvalid; e += blockDim.x) {
-        const int lr = e / g.nvalid, c = e % g.nvalid;
-        const int64_t t = g.row0 + lr;
-        const float v = fin[lr * kShrinkN + c] * p.scale1;
-        p.dU[t * p.r + g.n0 + c] = v;
-      }
+    }
+  } else {
+    const int nw = static_cast<int>(blockDim.x) >> 5;
+    for (int lr = lr0 + warp; lr < lr1; lr += nw) {
+      float *dst = p.dU + static_cast<int64_t>(g.row0 + lr) * p.r + g.n0;
+      for (int c = lane; c < g.nvalid; c += 32) dst[c] = fin[lr * kShrinkN + c] * p.scale1;
     }
   }
 }
