@@ -12,11 +12,15 @@
 // multi-adapter batch of the batching section (批处理) of "S-LoRA：一个GPU运行
 // 数千大模型成为可能" without padding adapters to a common rank.
 //
-// Structure: persistent CTAs (one per SM), 6 warps:
+// Structure: persistent CTAs (one per SM), 7 warps:
 //   warp 0      TMA producer (lane 0): a 128-row box of X (original rows when a
 //               tile's tokens are consecutive, else the sorted copy of X the
-//               shrink wrote while gathering), the W tile, then the tile's s·U
-//               images (bulk copy) and the matching B_pool rows
+//               shrink wrote while gathering), then the tile's s·U images (bulk
+//               copy) and the matching B_pool rows
+//   warp 6      TMA producer (lane 0) of the W tiles of the base K blocks. With
+//               every SM loading, one thread's copies complete one after another
+//               (a few hundred ns each, nearly independent of their size), so
+//               two issuing threads double the rate at which stages fill
 //   warp 1      MMA issuer (one thread) + TMEM owner: 128x256 fp32 accumulator,
 //               double-buffered in TMEM (512 columns) so the epilogue of tile i
 //               overlaps the main loop of tile i+1
@@ -42,7 +46,8 @@ constexpr int kStageBytes = kStageA + kStageB;    // 48 KB
 // An adapter block's B operand: up to four 8 KB slots, each one 16-row slice of
 // B_pool over the tile's 256 columns, stored [4 column blocks][16 rows][64 cols].
 constexpr int kBSlot = 4 * 16 * 128;
-constexpr int kGemmThreads = 192;
+constexpr int kGemmThreads = 224;
+constexpr int kGemmWarpW = 6;  // the W-copy warp
 constexpr int kGemmBarBytes = 256;
 constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16;
 
@@ -239,8 +244,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // inputs written by the previous kernels of the forward (s·U images, the
-  // sorted copy of X) and the output are touched only after they completed
-  pdl_wait();
+  // sorted copy of X) and the output are touched only after they completed;
+  // the W copies read only the weights and the plan's tables (written before
+  // those kernels ran), so their warp starts streaming at once
+  if (warp != kGemmWarpW) pdl_wait();
 
   const int n_tiles = p.n_mt * p.n_nt;
   const int KB = (p.K + kBK - 1) / kBK;
@@ -253,6 +260,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // -------------------------------------------------------------- producer
+    if (lane == 0) {
+      prefetch_tmap(&mapA);
+      if (has_plan) prefetch_tmap(&mapBl);
+    }
     // The warp stages each tile's adapter table in shared memory (no dependent
     // global loads inside the K loop); lane 0 issues every TMA copy.
     int stage = 0;
@@ -285,16 +296,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint32_t b_dst = a_dst + kStageA;
           const uint32_t fb = full0 + 8 * stage;
           if (blk < KB) {
-            const int k0 = blk * kBK;
+            // the W tile of this stage comes from warp kGemmWarpW's copy; the
+            // expected bytes cover both (a copy may land before this arrive:
+            // the phase cannot complete while the arrival is pending)
             mbar_arrive_expect_tx(fb, kStageA + kStageB);
-            tma_load_2d(a_dst, &mapA, fb, k0, arow);
-            if (B_KMAJOR) {
-              tma_load_2d(b_dst, &mapB, fb, k0, n0);
-            } else if (p.w3d) {
-              tma_load_3d(b_dst, &mapB, fb, 0, k0, n0 / 64);  // the four 64-column blocks in one copy
-            } else {
-              for (int j = 0; j < kBN / 64; ++j) tma_load_2d(b_dst + j * 8192, &mapB, fb, n0 + j * 64, k0);
-            }
+            tma_load_2d(a_dst, &mapA, fb, blk * kBK, arow);
           } else {
             // adapter K block: 64 augmented columns (up to 4 MMA K steps). Each
             // chunk spans 2*kc columns: s*U rounded to bf16 (hi), then the
@@ -330,6 +336,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
       __syncwarp();
     }
+  } else if (warp == kGemmWarpW) {
+    // ------------------------------------------------------------ W producer
+    // Walks the same block sequence as warp 0 and fills the B half of each base
+    // block's stage once the stage is free. It waits for every stage in turn,
+    // adapter blocks' too: a parity wait is only exact while the waiter is at
+    // most one phase ahead of the barrier.
+    if (lane == 0) {
+      prefetch_tmap(&mapB);
+      int stage = 0;
+      uint32_t phase = 0;
+      for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
+        int mt, nt;
+        tile_coords(tile, p, mt, nt);
+        const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+        const int n0 = nt * kBN;
+        const int arow = p.a_sorted ? td.row0 : td.contig;
+        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const int nblk = arow < 0 ? 0 : br.count();
+        for (int i = 0; i < nblk; ++i) {
+          const int blk = br.block(i, KB);
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
+          if (blk < KB) {
+            const uint32_t b_dst = stage0 + stage * kStageBytes + kStageA;
+            const uint32_t fb = full0 + 8 * stage;
+            const int k0 = blk * kBK;
+            if (B_KMAJOR) {
+              tma_load_2d(b_dst, &mapB, fb, k0, n0);
+            } else if (p.w3d) {
+              tma_load_3d(b_dst, &mapB, fb, 0, k0, n0 / 64);  // the four 64-column blocks in one copy
+            } else {
+              for (int j = 0; j < kBN / 64; ++j) tma_load_2d(b_dst + j * 8192, &mapB, fb, n0 + j * 64, k0);
+            }
+          }
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
+        }
+      }
+    }
+    __syncwarp();
   } else if (warp == 1) {
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
@@ -391,7 +435,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
   } else {
-    // -------------------------------------------------------------- epilogue
+    // -------------------------------------------------------------- epilogue (warps 2..5)
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
     float *as = reinterpret_cast<float *>(smem + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16);
@@ -521,7 +565,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const bool valid = warp >= 2 && row < td.rows;
+    const bool epi = warp >= 2 && warp < 6;
+    const bool valid = epi && row < td.rows;
     const int64_t orig =
         !valid ? 0 : has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
     // barrier: every CTA's MMAs are complete, so every stage ring is idle and may
@@ -530,7 +575,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     cluster_barrier();
     if (threadIdx.x == 64) mbar_arrive_expect_tx(recv_bar, (S - 1) * xslot_bytes(S));
     bool go = false;
-    if (warp >= 2) {
+    if (epi) {
       go = tile0 < n_tiles && !*abort_flag;
       if (go) {
         // send, step 1: TMEM -> registers -> 4 KB blocks laid out per owner as the
