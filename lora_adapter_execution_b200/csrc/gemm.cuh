@@ -257,6 +257,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const int q = split ? static_cast<int>(cluster_rank()) : 0;
   const int tile0 = split ? static_cast<int>(blockIdx.x) / S : static_cast<int>(blockIdx.x);
   const int tile_step = split ? n_tiles : static_cast<int>(gridDim.x);
+  // split-K tail inputs, set by the epilogue warps before their wait
+  int split_rows = 0, split_nt = 0, split_kaug = 0;
+  int64_t split_orig = 0;
 
   if (warp == 0) {
     // -------------------------------------------------------------- producer
@@ -441,6 +444,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     float *as = reinterpret_cast<float *>(smem + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16);
     int acc = 0;
     uint32_t aphase = 0;
+    if (split) {
+      // the split-K tail's table entry and output row, loaded while the K loop runs
+      int mt = 0, nt = 0;
+      tile_coords(tile0 < n_tiles ? tile0 : 0, p, mt, nt);
+      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      split_rows = td.rows;
+      split_nt = nt;
+      split_kaug = td.kaug;
+      split_orig = row >= td.rows ? 0
+                   : has_plan    ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row])
+                                 : td.row0 + row;
+    }
     // the backward's warps leave together (epi_bar_or), so its loop ignores the
     // flag here and tests it at the barrier
     for (int tile = tile0; tile < n_tiles && (EPI == kEpiBwdLora || !*abort_flag); tile += tile_step) {
@@ -558,17 +573,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int width = kBN / S;
     const uint32_t slot0 = smem_u32(smem);
     const uint32_t out0 = slot0 + (S - 1) * xslot_bytes(S);
-    int mt = 0, nt = 0;
-    tile_coords(tile0 < n_tiles ? tile0 : 0, p, mt, nt);
-    const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+    const int nt = split_nt;
     // a CTA with no K blocks for this tile contributes zeros (its TMEM was never written)
-    const bool any = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
+    const bool any = block_range(KB, (split_kaug + kAugBlock - 1) / kAugBlock, q, S).count() > 0;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const bool epi = warp >= 2 && warp < 6;
-    const bool valid = epi && row < td.rows;
-    const int64_t orig =
-        !valid ? 0 : has_plan ? (td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row]) : td.row0 + row;
+    const bool valid = epi && row < split_rows;
+    const int64_t orig = valid ? split_orig : 0;
     // barrier: every CTA's MMAs are complete, so every stage ring is idle and may
     // receive; it also orders the receive barriers' initialisation before any
     // remote completion
