@@ -60,7 +60,7 @@ int device_state(DeviceState **out) {
           ok &= cudaFuncSetAttribute(lora_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      kSkSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_tcontract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     200 * 1024) == cudaSuccess;
+                                     1024 + kTcSmemBudget + 2 * kTcMaxStages * 8) == cudaSuccess;
           if (!ok) d.status = LORA_ERR_CUDA;
         }
       }
@@ -537,16 +537,19 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
 }
 
 // Workspace layout: dU f32 [T, r] | dB partial [S, r, d_out] | dA partial [S, r, d_in]
-static int64_t bwd_splits(int64_t T, int64_t d_in) {
-  (void)d_in;
-  int64_t s = (T + 2047) / 2048;  // ~2048 tokens per split
+// Token splits of the backward contractions: about two CTAs per SM of a B200
+// (148 SMs) over the wider of the two column ranges, at least 64 tokens each.
+static int64_t bwd_splits(int64_t T, int64_t d_in, int64_t d_out) {
+  const int64_t cols = (std::max(d_in, d_out) + kTcCols - 1) / kTcCols;
+  int64_t s = (2 * 148 + cols / 2) / cols;
+  s = std::min<int64_t>(s, (T + kTcTok - 1) / kTcTok);
   return std::max<int64_t>(1, std::min<int64_t>(s, 16));
 }
 
 size_t lora_linear_bwd_workspace_size(int64_t T, int64_t d_in, int64_t d_out, int32_t r) {
   if (T <= 0 || d_in <= 0 || d_out <= 0 || r <= 0) return 0;
   auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
-  const int64_t S = bwd_splits(T, d_in);
+  const int64_t S = bwd_splits(T, d_in, d_out);
   return static_cast<size_t>(up(T * r * 4) + up(S * r * d_out * 4) + up(S * r * d_in * 4));
 }
 
@@ -571,7 +574,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
   if (rc != LORA_OK) return rc;
 
   auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
-  const int64_t S = bwd_splits(T, d_in);
+  const int64_t S = bwd_splits(T, d_in, d_out);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   float *dU = reinterpret_cast<float *>(ws);
   float *pdB = reinterpret_cast<float *>(ws + up(T * r * 4));
@@ -653,13 +656,9 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
   // K3c: dB = s * U^T * dY and dA = (D ⊙ X)^T * dU, split over tokens, then reduced
   {
     const int64_t tsplit = ((T + S - 1) / S + kTcTok - 1) / kTcTok * kTcTok;
-    const int g_bytes = kTcTok * r * 4;
-    const int stage_bytes = kTcTok * kTcCols * 2 + ((g_bytes + 1023) & ~1023);
-    const int smem = 1024 + kTcStages * stage_bytes + 2 * kTcStages * 8;
     // keep bits in the dA contraction need a 16-byte row stride (d_in % 128 == 0);
     // otherwise it re-derives the mask from the generator
     bool use_bits = thr != 0 && keep_bits != nullptr && ((d_in + 31) / 32) % 4 == 0;
-    // note: the kernel lays stages out with the same formula
     CUtensorMap mBits = mX64;  // unused unless the dA contraction reads keep bits
     if (use_bits) {
       cuuint64_t dims[2] = {static_cast<cuuint64_t>((d_in + 31) / 32), static_cast<cuuint64_t>(T)};
@@ -681,13 +680,14 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     tp.keep_bits = nullptr;
     tp.partial = pdB;
     dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
-    lora_tcontract_kernel<<<grid_b, kTcThreads, smem, stream>>>(mdY64, mU, mBits, tp);
+    const int smem_b = 1024 + tc_stages(r, false) * tc_stage_bytes(r, false) + 2 * kTcMaxStages * 8;
+    lora_tcontract_kernel<<<grid_b, kTcThreads, smem_b, stream>>>(mdY64, mU, mBits, tp);
     tp.N = static_cast<int32_t>(d_in);
     tp.thr = thr;
     tp.seed = seed;
     // with keep bits, each stage's bits come through the copy engine with its tile
     tp.keep_bits = use_bits ? keep_bits : nullptr;
-    const int smem_a = smem + (use_bits ? kTcStages * kTcTok * (kTcCols / 32) * 4 : 0);
+    const int smem_a = 1024 + tc_stages(r, use_bits) * tc_stage_bytes(r, use_bits) + 2 * kTcMaxStages * 8;
     tp.wpr = (d_in + 31) / 32;
     tp.partial = pdA;
     dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));

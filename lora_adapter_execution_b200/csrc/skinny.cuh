@@ -588,11 +588,26 @@ __global__ void __launch_bounds__(kSkThreads, 2)
 }
 
 // ------------------------------------------------------------------ token contraction
-constexpr int kTcThreads = 288;   // 8 consumer warps + producer warp
-constexpr int kTcStages = 6;
+constexpr int kTcConsumerWarps = 4;
+constexpr int kTcThreads = (kTcConsumerWarps + 1) * 32;  // + producer warp
+constexpr int kTcMaxStages = 6;
 constexpr int kTcTok = 64;        // tokens per stage
-constexpr int kTcCols = 128;      // columns per CTA
+constexpr int kTcCols = 128;      // columns per CTA (32 per consumer warp)
 constexpr int kTcMaxR = 64;
+constexpr int kTcSmemBudget = 110 * 1024;  // stage ring per CTA: two CTAs share an SM
+
+// Bytes of one stage of the token contraction: In [64 tokens][128 columns] as two
+// 64-column halves (128-byte swizzle), G [64 tokens][r] fp32 as copied, the
+// stage's keep bits [64 tokens][4 words] when read, and G^T split into bf16 hi
+// and lo parts, [16 * mblocks ranks][64 tokens] each (128-byte rows, swizzled).
+__host__ __device__ inline int tc_stage_bytes(int r, bool bits) {
+  const int mblocks = (r + 15) / 16;
+  return kTcTok * kTcCols * 2 + ((kTcTok * r * 4 + 1023) & ~1023) + (bits ? 1024 : 0) + 2 * mblocks * 2048;
+}
+__host__ __device__ inline int tc_stages(int r, bool bits) {
+  const int n = kTcSmemBudget / tc_stage_bytes(r, bits);
+  return n < kTcMaxStages ? n : kTcMaxStages;
+}
 
 struct TcParams {
   int32_t T, N, r;
@@ -609,9 +624,22 @@ __device__ __forceinline__ void split_pair(float v0, float v1, uint32_t &hi, uin
   lo = pack_bf16x2(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
 }
 
+// Mask of a transposed B fragment register: its two bf16 halves are tokens t
+// and t + 1 of one column, whose keep bits are bit 0 of xa and xb (sel 0xCC88)
+// or bit 8 (the column 8 further on, sel 0xDD99).
+template <uint32_t kSel>
+__device__ __forceinline__ uint32_t keep_pair_t(uint32_t xa, uint32_t xb) {
+  uint32_t m;
+  asm("prmt.b32 %0, %1, %2, %3;" : "=r"(m) : "r"(xa << 7), "r"(xb << 7), "n"(kSel));
+  return m;
+}
+
 // partial[q][k][n] = sum_{t in split q} G[t, k] * In[t, n] (In masked if thr != 0).
-// Grid (N / 128, splits).
-__global__ void __launch_bounds__(kTcThreads, 1)
+// Grid (N / 128, splits). Warp w < 4 owns columns [32w, 32w + 32) of the CTA's
+// 128. The consumer warps first turn the stage's fp32 G into its transposed hi
+// and lo bf16 images (once for all warps), then each k16 step takes two
+// transposed In fragments and, per 16 ranks, two G^T fragments and eight MMAs.
+__global__ void __launch_bounds__(kTcThreads, 2)
     lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N] bf16, box {64, 64}, swizzle 128B
                           const __grid_constant__ CUtensorMap mapG,   // G [T, r] fp32, box {r, 64}, no swizzle
                           const __grid_constant__ CUtensorMap mapBits,  // keep bits [T, wpr] u32, box {4, 64}
@@ -619,15 +647,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
+  const bool bits = p.keep_bits != nullptr;
+  const int mblocks = (p.r + 15) / 16;
   const int in_bytes = kTcTok * kTcCols * 2;    // 16 KB (two 8 KB halves)
   const int g_bytes = kTcTok * p.r * 4;         // <= 16 KB
   const int g_pad = (g_bytes + 1023) & ~1023;
-  const int bits_bytes = p.keep_bits ? kTcTok * (kTcCols / 32) * 4 : 0;  // 1 KB: the stage's keep bits
-  const int stage_bytes = in_bytes + g_pad + bits_bytes;
+  const int bits_bytes = bits ? 1024 : 0;       // the stage's keep bits
+  const int conv_off = in_bytes + g_pad + bits_bytes;  // G^T hi, then lo (mblocks * 2 KB each)
+  const int stage_bytes = tc_stage_bytes(p.r, bits);
+  const int nstage = tc_stages(p.r, bits);
   const uint32_t pool = smem_u32(smem);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kTcStages * stage_bytes);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + nstage * stage_bytes);
   const uint32_t full0 = smem_u32(bars);
-  const uint32_t empty0 = full0 + 8 * kTcStages;
+  const uint32_t empty0 = full0 + 8 * kTcMaxStages;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -635,27 +667,21 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   const int t0 = blockIdx.y * p.tsplit;
   const int t1 = min(p.T, t0 + p.tsplit);
   const int nblk = t1 > t0 ? (t1 - t0 + kTcTok - 1) / kTcTok : 0;
-  const int mblocks = (p.r + 15) / 16;
 
   if (threadIdx.x == 0) {
-    for (int s = 0; s < kTcStages; ++s) {
+    for (int s = 0; s < nstage; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, 8);
+      mbar_init(empty0 + 8 * s, kTcConsumerWarps);
     }
     fence_mbar_init();
   }
   __syncthreads();
 
-  float acc[4][2][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 2; ++j)
-#pragma unroll
-      for (int e = 0; e < 4; ++e) acc[i][j][e] = 0.f;
-
-  if (warp == 8) {
+  if (warp == kTcConsumerWarps) {
     if (lane == 0) {
+      prefetch_tmap(&mapIn);
+      prefetch_tmap(&mapG);
+      if (bits) prefetch_tmap(&mapBits);
       int stage = 0;
       uint32_t phase = 0;
       for (int b = 0; b < nblk; ++b) {
@@ -667,105 +693,171 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         tma_load_2d(sb, &mapIn, fb, n0, t);
         tma_load_2d(sb + 8192, &mapIn, fb, n0 + 64, t);
         tma_load_2d(sb + in_bytes, &mapG, fb, 0, t);
-        if (bits_bytes) tma_load_2d(sb + in_bytes + g_pad, &mapBits, fb, n0 / 32, t);
-        if (++stage == kTcStages) { stage = 0; phase ^= 1; }
+        if (bits) tma_load_2d(sb + in_bytes + g_pad, &mapBits, fb, n0 / 32, t);
+        if (++stage == nstage) { stage = 0; phase ^= 1; }
       }
     }
-  } else {
-    // warp w owns columns [16w, 16w + 16) of the CTA's 128
-    const int cw = warp * 16;
-    const int h = cw / 64;        // which 64-column half
-    const int cin = cw % 64;      // column offset inside the half
-    int stage = 0;
-    uint32_t phase = 0;
-    for (int b = 0; b < nblk; ++b) {
-      if (!mbar_wait(full0 + 8 * stage, phase)) break;
-      const uint32_t sb = pool + stage * stage_bytes;
-      const uint32_t inb = sb + h * 8192;
-      const uint32_t gb = sb + in_bytes;
-      const int tbase = t0 + b * kTcTok;
+    return;  // no block-wide barrier follows
+  }
+
+  // ------------------------------------------------------------------ consumers
+  const int cw = warp * 32;     // the warp's first column of the CTA's 128
+  const int half = cw / 64;     // which 64-column half of the stage
+  const int cin = cw % 64;      // column offset inside the half (0 or 32)
+  const int mi = lane >> 3;
+  const int l7 = lane & 7;
+  // transposed In fragments of column group g (16 columns) at k16 step ks:
+  // lanes 8q .. 8q + 7 address tokens ks*16 + (q & 1)*8 + (lane & 7) of chunk
+  // cin/8 + 2g + (q >> 1)
+  uint32_t boff[4][2];
 #pragma unroll
-      for (int ks = 0; ks < kTcTok / 16; ++ks) {
-        // B fragments (tokens x columns) for the warp's two n8 blocks
-        uint32_t b0, b1, b2, b3;
-        {
-          const int mi = lane >> 3;
-          const int tr = ks * 16 + (mi & 1) * 8 + (lane & 7);
-          const int chunk = (cin >> 3) + (mi >> 1);
-          ldsm_x4_t(inb + tr * 128 + (((chunk ^ (tr & 7)) & 7) << 4), b0, b1, b2, b3);
+  for (int ks = 0; ks < 4; ++ks)
+#pragma unroll
+    for (int g = 0; g < 2; ++g) {
+      const int tr = ks * 16 + (mi & 1) * 8 + l7;
+      const int chunk = (cin >> 3) + 2 * g + (mi >> 1);
+      boff[ks][g] = half * 8192 + tr * 128 + (((chunk ^ (tr & 7)) & 7) << 4);
+    }
+  // G^T fragments (ranks x tokens, row-major) from the hi / lo images: rank rows
+  // (q & 1)*8 + (lane & 7) of the 16-rank block, token chunk ks*2 + (q >> 1)
+  uint32_t aoff[4];
+#pragma unroll
+  for (int ks = 0; ks < 4; ++ks) {
+    const int m = (mi & 1) * 8 + l7;
+    aoff[ks] = m * 128 + ((((2 * ks + (mi >> 1)) ^ (m & 7)) & 7) << 4);
+  }
+  const int q2 = 2 * (lane & 3);
+  const int tid = static_cast<int>(threadIdx.x);  // 0 .. 127
+
+  float acc[4][2][2][4];  // [m-block][column group][n8][fragment]
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
+#pragma unroll
+      for (int j = 0; j < 2; ++j)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[i][g][j][e] = 0.f;
+
+  int stage = 0;
+  uint32_t phase = 0;
+  for (int b = 0; b < nblk; ++b) {
+    if (!mbar_wait(full0 + 8 * stage, phase)) break;
+    const uint32_t sb = pool + stage * stage_bytes;
+    uint8_t *const sbp = smem + (sb - pool);
+    // G^T images of this stage. Work item = (token pair tp, 4 consecutive ranks
+    // from k4): G[2tp][k4 .. k4 + 3] and G[2tp + 1][k4 .. k4 + 3] as two 16-byte
+    // reads (consecutive threads take consecutive ranks, so the reads do not
+    // collide on banks), written as (hi, lo) bf16 pairs at rank rows k4 .. k4 + 3,
+    // tokens 2tp and 2tp + 1. Rank rows from r to 16 * mblocks are zero.
+    {
+      const float *graw = reinterpret_cast<const float *>(sbp + in_bytes);
+      uint8_t *ghi = sbp + conv_off;
+      uint8_t *glo = ghi + mblocks * 2048;
+      const int q4 = mblocks * 4;  // 4-rank groups per token pair
+      for (int item = tid; item < 32 * q4; item += kTcConsumerWarps * 32) {
+        const int tp = item / q4;
+        const int k4 = (item - tp * q4) * 4;
+        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+        if (k4 < p.r) {  // r % 8 == 0: a group is all in or all out
+          v0 = *reinterpret_cast<const float4 *>(graw + (2 * tp) * p.r + k4);
+          v1 = *reinterpret_cast<const float4 *>(graw + (2 * tp + 1) * p.r + k4);
         }
-        if (p.thr != 0) {
-          // b0: tokens ks*16 + 2*(lane&3) + {0,1}, column cw + lane/4; b1: tokens + 8;
-          // b2, b3: column + 8
-          const int tk = tbase + ks * 16 + 2 * (lane & 3);
-          const int c = n0 + cw + (lane >> 2);
-          if (p.keep_bits) {
-            // the stage's bits, [64 tokens][4 words] for its 128 columns; c % 32 <= 23
-            // (n0 multiple of 128, cw of 16, lane / 4 < 8), so c and c + 8 share a word
-            const uint32_t *bs = reinterpret_cast<const uint32_t *>(smem + (sb - pool) + in_bytes + g_pad);
-            const int tl = ks * 16 + 2 * (lane & 3);
-            const int wd = (c - n0) >> 5;
-            const int sh = c & 31;
-            const uint32_t w0 = bs[tl * 4 + wd] >> sh;
-            const uint32_t w1 = bs[(tl + 1) * 4 + wd] >> sh;
-            const uint32_t w8 = bs[(tl + 8) * 4 + wd] >> sh;
-            const uint32_t w9 = bs[(tl + 9) * 4 + wd] >> sh;
-            b0 = mask_pair(b0, w0 & 1u, w1 & 1u);
-            b1 = mask_pair(b1, w8 & 1u, w9 & 1u);
-            b2 = mask_pair(b2, (w0 >> 8) & 1u, (w1 >> 8) & 1u);
-            b3 = mask_pair(b3, (w8 >> 8) & 1u, (w9 >> 8) & 1u);
-          } else {
-            b0 = mask_pair(b0, keep_elem(p.seed, p.thr, tk, c, p.N), keep_elem(p.seed, p.thr, tk + 1, c, p.N));
-            b1 = mask_pair(b1, keep_elem(p.seed, p.thr, tk + 8, c, p.N), keep_elem(p.seed, p.thr, tk + 9, c, p.N));
-            b2 = mask_pair(b2, keep_elem(p.seed, p.thr, tk, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 1, c + 8, p.N));
-            b3 = mask_pair(b3, keep_elem(p.seed, p.thr, tk + 8, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 9, c + 8, p.N));
+        const float a0[4] = {v0.x, v0.y, v0.z, v0.w};
+        const float a1[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int k = k4 + u;
+          uint32_t hi, lo;
+          split_pair(a0[u], a1[u], hi, lo);
+          const uint32_t off = k * 128 + ((((tp >> 2) ^ (k & 7)) & 7) << 4) + (tp & 3) * 4;
+          *reinterpret_cast<uint32_t *>(ghi + off) = hi;
+          *reinterpret_cast<uint32_t *>(glo + off) = lo;
+        }
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kTcConsumerWarps * 32) : "memory");
+    const uint32_t ghi_s = sb + conv_off;
+    const uint32_t glo_s = ghi_s + mblocks * 2048;
+    const uint32_t *bs = reinterpret_cast<const uint32_t *>(sbp + in_bytes + g_pad);
+    const int tbase = t0 + b * kTcTok;
+#pragma unroll
+    for (int ks = 0; ks < 4; ++ks) {
+      uint32_t bf[2][4];
+#pragma unroll
+      for (int g = 0; g < 2; ++g) ldsm_x4_t(sb + boff[ks][g], bf[g][0], bf[g][1], bf[g][2], bf[g][3]);
+      if (p.thr != 0) {
+        // bf[g][0]: tokens tl, tl + 1 of column c = n0 + cw + 16g + lane/4;
+        // [1]: tokens + 8; [2], [3]: column + 8
+        const int tl = ks * 16 + q2;
+        if (bits) {
+          // the stage's bits: [64 tokens][4 words] for its 128 columns; the
+          // warp's 32 columns are word cw / 32, and c, c + 8 share it
+          const int wd = cw >> 5;
+          const uint32_t w0 = bs[tl * 4 + wd], w1 = bs[(tl + 1) * 4 + wd];
+          const uint32_t w8 = bs[(tl + 8) * 4 + wd], w9 = bs[(tl + 9) * 4 + wd];
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const int sh = 16 * g + (lane >> 2);
+            const uint32_t x0 = w0 >> sh, x1 = w1 >> sh, x8 = w8 >> sh, x9 = w9 >> sh;
+            bf[g][0] &= keep_pair_t<0xCC88>(x0, x1);
+            bf[g][1] &= keep_pair_t<0xCC88>(x8, x9);
+            bf[g][2] &= keep_pair_t<0xDD99>(x0, x1);
+            bf[g][3] &= keep_pair_t<0xDD99>(x8, x9);
+          }
+        } else {
+          const int tk = tbase + tl;
+#pragma unroll
+          for (int g = 0; g < 2; ++g) {
+            const int c = n0 + cw + 16 * g + (lane >> 2);
+            bf[g][0] = mask_pair(bf[g][0], keep_elem(p.seed, p.thr, tk, c, p.N), keep_elem(p.seed, p.thr, tk + 1, c, p.N));
+            bf[g][1] = mask_pair(bf[g][1], keep_elem(p.seed, p.thr, tk + 8, c, p.N), keep_elem(p.seed, p.thr, tk + 9, c, p.N));
+            bf[g][2] = mask_pair(bf[g][2], keep_elem(p.seed, p.thr, tk, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 1, c + 8, p.N));
+            bf[g][3] = mask_pair(bf[g][3], keep_elem(p.seed, p.thr, tk + 8, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 9, c + 8, p.N));
           }
         }
+      }
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          if (i >= mblocks) break;
-          // A fragment = G^T (ranks x tokens) from G stored [token][rank] fp32:
-          // element (m, k) of the 16x16 fragment is G[ks*16 + k][i*16 + m]
-          const int m = i * 16 + (lane >> 2);
-          const int k = ks * 16 + 2 * (lane & 3);
-          const float *gf = reinterpret_cast<const float *>(smem + (gb - pool));
-          auto gv = [&](int kk, int mm) { return mm < p.r ? gf[kk * p.r + mm] : 0.f; };
-          uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
-          split_pair(gv(k, m), gv(k + 1, m), h0, l0);
-          split_pair(gv(k, m + 8), gv(k + 1, m + 8), h1, l1);
-          split_pair(gv(k + 8, m), gv(k + 9, m), h2, l2);
-          split_pair(gv(k + 8, m + 8), gv(k + 9, m + 8), h3, l3);
-          mma_bf16_16816(acc[i][0], h0, h1, h2, h3, b0, b1);
-          mma_bf16_16816(acc[i][1], h0, h1, h2, h3, b2, b3);
-          mma_bf16_16816(acc[i][0], l0, l1, l2, l3, b0, b1);
-          mma_bf16_16816(acc[i][1], l0, l1, l2, l3, b2, b3);
+      for (int i = 0; i < 4; ++i) {
+        if (i >= mblocks) break;
+        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+        ldsm_x4(ghi_s + i * 2048 + aoff[ks], h0, h1, h2, h3);
+        ldsm_x4(glo_s + i * 2048 + aoff[ks], l0, l1, l2, l3);
+#pragma unroll
+        for (int g = 0; g < 2; ++g) {
+          mma_bf16_16816(acc[i][g][0], h0, h1, h2, h3, bf[g][0], bf[g][1]);
+          mma_bf16_16816(acc[i][g][1], h0, h1, h2, h3, bf[g][2], bf[g][3]);
+          mma_bf16_16816(acc[i][g][0], l0, l1, l2, l3, bf[g][0], bf[g][1]);
+          mma_bf16_16816(acc[i][g][1], l0, l1, l2, l3, bf[g][2], bf[g][3]);
         }
       }
-      __syncwarp();
-      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
-      if (++stage == kTcStages) { stage = 0; phase ^= 1; }
     }
-    // write partial[q][k][n]
-    float *out = p.partial + static_cast<int64_t>(blockIdx.y) * p.r * p.N;
+    __syncwarp();
+    if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+    if (++stage == nstage) { stage = 0; phase ^= 1; }
+  }
+  // write partial[q][k][n]
+  float *out = p.partial + static_cast<int64_t>(blockIdx.y) * p.r * p.N;
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      if (i >= mblocks) break;
+  for (int i = 0; i < 4; ++i) {
+    if (i >= mblocks) break;
+#pragma unroll
+    for (int g = 0; g < 2; ++g)
 #pragma unroll
       for (int j = 0; j < 2; ++j) {
         const int k = i * 16 + (lane >> 2);
-        const int c = n0 + cw + j * 8 + 2 * (lane & 3);
+        const int c = n0 + cw + 16 * g + j * 8 + q2;
         if (c < p.N) {
           if (k < p.r) {
-            out[static_cast<int64_t>(k) * p.N + c] = acc[i][j][0];
-            out[static_cast<int64_t>(k) * p.N + c + 1] = acc[i][j][1];
+            out[static_cast<int64_t>(k) * p.N + c] = acc[i][g][j][0];
+            out[static_cast<int64_t>(k) * p.N + c + 1] = acc[i][g][j][1];
           }
           if (k + 8 < p.r) {
-            out[static_cast<int64_t>(k + 8) * p.N + c] = acc[i][j][2];
-            out[static_cast<int64_t>(k + 8) * p.N + c + 1] = acc[i][j][3];
+            out[static_cast<int64_t>(k + 8) * p.N + c] = acc[i][g][j][2];
+            out[static_cast<int64_t>(k + 8) * p.N + c + 1] = acc[i][g][j][3];
           }
         }
       }
-    }
   }
 }
 
