@@ -245,10 +245,27 @@ __host__ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64
   z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
   return z ^ (z >> 31);
 }
+// splitmix64 output of state z (the state after its increment) >= thr, i.e. the
+// element is kept. The comparison needs only the high word of the output unless
+// it ties with the high word of thr (a 2^-32 event): the last product's low word
+// and the last shift's low half are formed only then.
+__device__ __forceinline__ bool keep_state(uint64_t z, uint64_t thr) {
+  const uint64_t x = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
+  const uint64_t u = x ^ (x >> 27);
+  constexpr uint64_t kM2 = 0x94D049BB133111EBull;
+  const uint32_t ul = static_cast<uint32_t>(u), uh = static_cast<uint32_t>(u >> 32);
+  const uint32_t ph = __umulhi(ul, static_cast<uint32_t>(kM2)) + ul * static_cast<uint32_t>(kM2 >> 32) +
+                      uh * static_cast<uint32_t>(kM2);  // high word of u * kM2
+  const uint32_t oh = ph ^ (ph >> 31);                   // high word of the output
+  const uint32_t th = static_cast<uint32_t>(thr >> 32);
+  if (oh != th) return oh > th;
+  const uint64_t p = u * kM2;
+  return (p ^ (p >> 31)) >= thr;
+}
 // true if element (t, col) of the LoRA-branch input is kept.
 __device__ __forceinline__ bool keep_elem(uint64_t seed, uint64_t thr, int64_t t, int64_t col,
                                           int64_t d_in) {
-  return thr == 0 || splitmix64_at(seed, static_cast<uint64_t>(t * d_in + col)) >= thr;
+  return thr == 0 || keep_state(seed + (static_cast<uint64_t>(t * d_in + col) + 1ull) * 0x9E3779B97F4A7C15ull, thr);
 }
 
 // Keep bits of 32 consecutive mask positions idx0 .. idx0+31 (bit i set if kept):
@@ -260,11 +277,7 @@ __device__ __forceinline__ uint32_t keep_mask32(uint64_t seed, uint64_t thr, uin
   uint32_t m = 0;
 #pragma unroll
   for (int i = 0; i < 32; ++i) {
-    uint64_t x = z;
-    x = (x ^ (x >> 30)) * 0xBF58476D1CE4E5B9ull;
-    x = (x ^ (x >> 27)) * 0x94D049BB133111EBull;
-    x ^= x >> 31;
-    m |= (x >= thr ? 1u : 0u) << i;
+    m |= (keep_state(z, thr) ? 1u : 0u) << i;
     z += 0x9E3779B97F4A7C15ull;
   }
   return m;
