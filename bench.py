@@ -78,6 +78,24 @@ def dist_env():
     return int(os.environ.get("RANK", 0)), int(os.environ.get("LOCAL_RANK", 0)), int(os.environ.get("WORLD_SIZE", 1))
 
 
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest of the ranks' values (a device time): an all-reduce MAX over the
+    process group, the value itself on one rank."""
+    if world <= 1:
+        return float(x)
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank: int, steps: int, world: int, ms: float) -> float:
+    """Whole-job tokens/s: every rank processed steps x tokens_per_rank tokens of
+    its own batch (weak scaling) in ms, the max over ranks."""
+    return world * tokens_per_rank * steps / (ms * 1e-3)
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
@@ -262,7 +280,7 @@ def run_lora(a):
     lora.load_library()
 
     # each rank its own batch (tokens and ids) of the same layer
-    inp = wl.make_inputs(a.config, seed=rank)
+    inp = wl.make_rank_inputs(a.config, rank)
     T, di, do = inp.T, inp.d_in, inp.d_out
     finetune = inp.dY is not None
 
@@ -345,19 +363,14 @@ def run_lora(a):
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
-        ms = e0.elapsed_time(e1)
-        if world > 1:
-            t = torch.tensor([ms], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ms = float(t.item())
-        return ms
+        return max_over_ranks(e0.elapsed_time(e1), world, dev)
 
     K = a.steps
     with ClockSampler(local_rank) as clk:
         ms_total = timed(graphs, K)
     clocks = clk.summary()
     if a.no_layer:
-        value = world * T * K / (ms_total * 1e-3)
+        value = job_throughput(T, K, world, ms_total)
         if rank == 0:
             print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
                               "warmup": a.warmup, "ms_per_step": ms_total / K, "note": "--no-layer run"}))
@@ -383,7 +396,7 @@ def run_lora(a):
         tgraphs.append(g)
     ms_torch = timed(tgraphs, K)
 
-    value = world * T * K / (ms_total * 1e-3)
+    value = job_throughput(T, K, world, ms_total)
     hbm, tc_burst, tc_sust, src = peaks()
     gb, gf, lb, lf = algorithmic(inp, info)
     t_gemm = ms_gemm * 1e-3 / K
@@ -461,11 +474,8 @@ def run_lora(a):
             e2e_step()
         dt = time.perf_counter() - t0
         p.destroy()
-        if world > 1:
-            t = torch.tensor([dt], device=dev, dtype=torch.float64)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            dt = float(t.item())
-        out["e2e"] = {"value": world * T * Ke / dt, "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+        dt = max_over_ranks(dt, world, dev)
+        out["e2e"] = {"value": job_throughput(T, Ke, world, dt * 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                       "d2h_bytes_per_step": int(d2h), "steps": Ke,
                       "what": "plan from host ids + H2D of X (pinned) + forward" + (" + backward" if finetune else "")
                               + " + D2H of the result, host wall clock per step"}

@@ -219,3 +219,21 @@ def integer_inputs(T: int, d_in: int, d_out: int, ranks, ids, seed: int = 0,
                   scale=np.ones(n, dtype=np.float32), X=ints((T, d_in)), W=ints((d_in, d_out)),
                   A_pool=ints((R, d_in)), B_pool=ints((R, d_out)), dY=ints((T, d_out)),
                   p_drop=0.0, mask_seed=0, offsets=offsets)
+
+
+def make_rank_inputs(spec: Spec | str, rank: int, **kw) -> Inputs:
+    """Rank `rank`'s share of a data-parallel run: the same layer (ranks, scales,
+    W, A_pool, B_pool) on every rank, and a batch of its own (ids, X, dY and the
+    dropout seed) drawn with the workload's recipe. Rank 0's batch is the
+    workload's own draw."""
+    if isinstance(spec, str):
+        spec = SPECS[spec]
+    base = make_inputs(spec, **kw)
+    if rank == 0:
+        return base
+    kw2 = dict(kw)
+    kw2["seed"] = (spec.seed if kw.get("seed") is None else kw["seed"]) + 7919 * rank
+    other = make_inputs(spec, **kw2)
+    return Inputs(spec=spec, T=base.T, d_in=base.d_in, d_out=base.d_out, ranks=base.ranks, ids=other.ids,
+                  scale=base.scale, X=other.X, W=base.W, A_pool=base.A_pool, B_pool=base.B_pool, dY=other.dY,
+                  p_drop=base.p_drop, mask_seed=base.mask_seed + rank, offsets=base.offsets)

@@ -1,0 +1,86 @@
+"""The multi-rank host logic of bench.py on CPU: world_size 2 over gloo.
+
+Weak scaling: every rank runs the same layer on a batch of its own, the step
+time is the max over ranks of the device times, and the job's throughput counts
+every rank's tokens. No GPU is needed for any of this."""
+import os
+import socket
+import subprocess
+import sys
+
+import numpy as np
+import pytest
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from lora_adapter_execution_b200 import workloads as wl  # noqa: E402
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _rank_main(rank, world, port, q):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    import datetime
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=60))
+    try:
+        ms = bench.max_over_ranks(1.5 + 2.0 * rank, world)
+        inp = wl.make_rank_inputs("tiny", rank)
+        q.put((rank, ms, int(inp.ids.sum()), float(np.asarray(inp.X, dtype=np.float64).sum())))
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_batches_gloo():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_main, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = [q.get(timeout=120) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    got.sort()
+    # every rank sees the slowest rank's time
+    assert [g[1] for g in got] == [3.5, 3.5]
+    # the two ranks ran different batches
+    assert got[0][2:] != got[1][2:]
+
+
+def test_rank_inputs_share_the_layer():
+    a = wl.make_rank_inputs("fleet", 0, T=300, d_in=64, d_out=64, n_adapters=40)
+    b = wl.make_rank_inputs("fleet", 1, T=300, d_in=64, d_out=64, n_adapters=40)
+    ref = wl.make_inputs("fleet", T=300, d_in=64, d_out=64, n_adapters=40)
+    for f in ("ranks", "scale", "W", "A_pool", "B_pool", "offsets"):
+        assert np.array_equal(getattr(a, f), getattr(b, f)), f
+    assert np.array_equal(a.X, ref.X) and np.array_equal(a.ids, ref.ids)
+    assert not np.array_equal(a.X, b.X)
+    assert not np.array_equal(a.ids, b.ids)
+    assert b.ids.min() >= 0 and b.ids.max() < len(b.ranks)
+    assert a.mask_seed != b.mask_seed
+
+
+def test_job_throughput_counts_every_rank():
+    assert bench.job_throughput(256, 10, 1, 2.0) == pytest.approx(256 * 10 / 2e-3)
+    assert bench.job_throughput(256, 10, 4, 2.0) == pytest.approx(4 * 256 * 10 / 2e-3)
+    assert bench.max_over_ranks(3.25, 1) == 3.25
+
+
+def test_reference_arm_other_ranks_exit_quietly():
+    env = dict(os.environ, RANK="1", LOCAL_RANK="1", WORLD_SIZE="2")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--gpus", "2",
+                        "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == ""
