@@ -98,18 +98,53 @@ def job_throughput(tokens_per_rank: int, steps: int, world: int, ms: float) -> f
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """nvidia-smi sampling of SM clocks and throttle reasons during the timed region."""
+    """SM clocks and throttle reasons sampled during the timed region: NVML every
+    2 ms (the device found by its UUID), else nvidia-smi every 100 ms. Reads only."""
 
     Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    # NVML clock event reason bits
+    REASONS = {"sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40}
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
         self.lines = []
+        self.nv = None
+        self.samples = []  # (sm MHz, max sm MHz, reason bits)
+        self.stop = threading.Event()
+
+    def _nvml_handle(self):
+        import pynvml
+        pynvml.nvmlInit()
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(self.index).uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(("GPU-" + uuid).encode())
+        except Exception:
+            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.index)
+
+    def _poll(self):
+        nv, h = self.nv
+        smax = nv.nvmlDeviceGetMaxClockInfo(h, nv.NVML_CLOCK_SM)
+        get_reasons = getattr(nv, "nvmlDeviceGetCurrentClocksEventReasons", None) or \
+            nv.nvmlDeviceGetCurrentClocksThrottleReasons
+        while not self.stop.is_set():
+            try:
+                self.samples.append((nv.nvmlDeviceGetClockInfo(h, nv.NVML_CLOCK_SM), smax, get_reasons(h)))
+            except Exception:
+                break
+            time.sleep(0.002)
 
     def __enter__(self):
+        try:
+            self.nv = self._nvml_handle()
+            self.t = threading.Thread(target=self._poll, daemon=True)
+            self.t.start()
+            return self
+        except Exception:
+            self.nv = None
         try:
             self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.Q}",
                                           "--format=csv,noheader,nounits", "-lms", "100"],
@@ -125,6 +160,9 @@ class ClockSampler:
             self.lines.append(line.strip())
 
     def __exit__(self, *a):
+        if self.nv is not None:
+            self.stop.set()
+            self.t.join(timeout=2)
         if self.proc is not None:
             self.proc.terminate()
             try:
@@ -134,7 +172,14 @@ class ClockSampler:
             self.t.join(timeout=2)
 
     def summary(self):
-        sm, smax, reasons = [], None, set()
+        sm, smax, reasons, any_bits = [], None, set(), 0
+        for mhz, mx, bits in self.samples:
+            sm.append(float(mhz))
+            smax = float(mx)
+            any_bits |= int(bits)
+            for n, b in self.REASONS.items():
+                if bits & b:
+                    reasons.add(n)
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         for ln in self.lines:
             f = [x.strip() for x in ln.split(",")]
@@ -149,7 +194,9 @@ class ClockSampler:
                 if v.lower() == "active":
                     reasons.add(n)
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": smax,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "source": "nvml" if self.samples else ("nvidia-smi" if self.lines else None),
+                "nvml_reason_bits": hex(any_bits) if self.samples else None}
 
 
 # ----------------------------------------------------------------------------- helpers
@@ -309,31 +356,53 @@ def run_lora(a):
                       bits=torch.empty(T, -(-di // 32), dtype=torch.int32, device=dev))
         copies.append(cp)
 
-    # one graph per copy; the plan (and its scratch) is shared, steps run in order
-    def step(cp):
-        bits = None
-        if finetune and inp.p_drop > 0:
-            # the step's dropout mask, written once and read by the forward and the backward
-            bits = cp["bits"]
-            lora.dropout_keep_bits(inp.mask_seed, inp.p_drop, bits, di)
-        lora.linear_fwd(plan, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["Y"], p_drop=inp.p_drop,
-                        seed=inp.mask_seed, U_save=cp["U"], keep_bits=bits)
+    # one graph per copy; the plan (and its scratch) is shared, steps run in order.
+    # With dropout, copy c's batch has its own mask seed; its keep bits depend on
+    # the seed only, so each step writes the next copy's bits on a second stream
+    # while its own forward GEMM runs (the bits kernel needs no shared memory and
+    # fits beside the GEMM's CTAs), and joins that stream before it ends.
+    masked = finetune and inp.p_drop > 0
+    side = torch.cuda.Stream(device=dev)
+    ev_fork = torch.cuda.Event()
+    ev_join = torch.cuda.Event()
+
+    def seed_of(c):
+        return inp.mask_seed + c
+
+    def step(c):
+        cp, nxt = copies[c], (c + 1) % len(copies)
+        bits = cp["bits"] if masked else None
+        lora.linear_shrink(plan, cp["X"], cp["A"], scale, p_drop=inp.p_drop, seed=seed_of(c), U_save=cp["U"],
+                           keep_bits=bits)
+        cur = torch.cuda.current_stream()
+        if masked:
+            ev_fork.record(cur)
+            side.wait_event(ev_fork)
+            with torch.cuda.stream(side):
+                lora.dropout_keep_bits(seed_of(nxt), inp.p_drop, copies[nxt]["bits"], di)
+            ev_join.record(side)
+        lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
         if finetune:
             lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"], cp["dX"],
-                            cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed, keep_bits=bits)
+                            cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=seed_of(c), keep_bits=bits)
+        if masked:
+            cur.wait_event(ev_join)
 
     # the forward: [row gather] + shrink + fused GEMM; the backward: dU, dX GEMM, 2 x (contraction + reduce)
     launches_per_step = 2 + int(info["gathers_x"]) + (6 if finetune else 0) + (1 if finetune and inp.p_drop > 0 else 0)
     stream = torch.cuda.Stream(device=dev)
     torch.cuda.synchronize()
     with torch.cuda.stream(stream):
-        step(copies[0])  # first call sets kernel attributes outside any capture
+        if masked:  # every copy's keep bits exist before its first step
+            for c in range(len(copies)):
+                lora.dropout_keep_bits(seed_of(c), inp.p_drop, copies[c]["bits"], di)
+        step(0)  # first call sets kernel attributes outside any capture
     torch.cuda.synchronize()
     graphs, ggraphs, bgraphs = [], [], []
-    for cp in copies:
+    for c, cp in enumerate(copies):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=stream):
-            step(cp)
+            step(c)
         graphs.append(g)
         g2 = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g2, stream=stream):
