@@ -232,11 +232,8 @@ __device__ __forceinline__ void shrink_consume(const ShrinkWarp &w, const Shrink
 #pragma unroll
     for (int h = 0; h < 2; ++h) rr[i][h] = min((w.mphase + i * w.MW) * 16 + (lane >> 2) + 8 * h, g.rows - 1);
 
-  for (int b = w.kphase; b < w.nblk; b += w.KW) {
-    const int stage = b % w.nstage;
-    const uint32_t phase = static_cast<uint32_t>(b / w.nstage) & 1u;
-    if (!mbar_wait(w.full0 + 8 * stage, phase)) { *abort_flag = 1; break; }
-    const uint32_t xb = w.pool + stage * w.stage_bytes;
+  // the MMAs of 64-column block b, whose X rows start at xb
+  auto consume = [&](int b, uint32_t xb) {
     const uint32_t fbuf = xb + w.Rp * 128;
     const int col = w.kbeg + b * kSkBK;  // first column of the stage, a multiple of 64
     // keep bits of the lane's rows for the stage's 64 columns: words
@@ -299,6 +296,18 @@ __device__ __forceinline__ void shrink_consume(const ShrinkWarp &w, const Shrink
         }
       }
     }
+  };
+
+  // stage S of the ring holds blocks S*KW .. S*KW + KW - 1 (KW blocks of
+  // stage_bytes each); warp group kphase takes block S*KW + kphase, and every
+  // consumer warp releases the stage
+  const int nsuper = (w.nblk + w.KW - 1) / w.KW;
+  for (int S = 0; S < nsuper; ++S) {
+    const int stage = S % w.nstage;
+    const uint32_t phase = static_cast<uint32_t>(S / w.nstage) & 1u;
+    if (!mbar_wait(w.full0 + 8 * stage, phase)) { *abort_flag = 1; break; }
+    const int b = S * w.KW + w.kphase;
+    if (b < w.nblk) consume(b, w.pool + stage * w.KW * w.stage_bytes + w.kphase * w.stage_bytes);
     __syncwarp();
     if (lane == 0) mbar_arrive(w.empty0 + 8 * stage);
   }
@@ -360,7 +369,6 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   // boundary, as the 128-byte swizzle of its TMA boxes requires
   const int stage_tx = (Rp + g.nn) * 128 + (stage_bits ? Rp * 16 : 0);
   const int stage_bytes = (stage_tx + 1023) & ~1023;
-  const int nstage = min(kSkMaxStages, kSkPool / stage_bytes);
   const int kbeg = static_cast<int>(crank) * p.kslice;
   const int kend = min(p.K, kbeg + p.kslice);
   const int nblk = kend > kbeg ? (kend - kbeg + kSkBK - 1) / kSkBK : 0;
@@ -371,11 +379,15 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   int MW = 1;
   while (MW * 2 <= mb && MW < kSkConsumerWarps) MW *= 2;
   const int KW = kSkConsumerWarps / MW;
+  // a ring stage holds KW consecutive 64-column blocks, one per warp group, so a
+  // small unit's copies come in groups (a lone 16-row block pair per barrier
+  // round trip kept too few bytes moving)
+  const int nstage = min(kSkMaxStages, kSkPool / (KW * stage_bytes));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
       mbar_init(full0 + 8 * s, 1);
-      mbar_init(empty0 + 8 * s, MW);  // the MW warps that consume the stage
+      mbar_init(empty0 + 8 * s, kSkConsumerWarps);  // every consumer warp releases a stage
     }
     *abort_flag = 0;
     fence_mbar_init();
@@ -394,20 +406,24 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       int stage = 0;
       uint32_t phase = 0;
       const int xrow = p.x_sorted ? g.row0 : g.contig;
-      for (int b = 0; b < nblk; ++b) {
+      const int nsuper = (nblk + KW - 1) / KW;
+      for (int S = 0; S < nsuper; ++S) {
         if (xrow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; break; }
         if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
         const uint32_t fb = full0 + 8 * stage;
-        const uint32_t xb = pool + stage * stage_bytes;
-        const uint32_t fbuf = xb + Rp * 128;
-        const int col = kbeg + b * kSkBK;
-        mbar_arrive_expect_tx(fb, stage_tx);
-        for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, xrow + r16);
-        for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
-        if (stage_bits) {
-          const uint32_t bb = fbuf + g.nn * 128;
-          for (int r16 = 0; r16 < Rp; r16 += 16)
-            tma_load_2d(bb + r16 * 16, &mapBits16, fb, (col >> 7) * 4, g.contig + r16);
+        const int nb = min(KW, nblk - S * KW);  // blocks in this stage
+        mbar_arrive_expect_tx(fb, nb * stage_tx);
+        for (int j = 0; j < nb; ++j) {
+          const uint32_t xb = pool + (stage * KW + j) * stage_bytes;
+          const uint32_t fbuf = xb + Rp * 128;
+          const int col = kbeg + (S * KW + j) * kSkBK;
+          for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, xrow + r16);
+          for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
+          if (stage_bits) {
+            const uint32_t bb = fbuf + g.nn * 128;
+            for (int r16 = 0; r16 < Rp; r16 += 16)
+              tma_load_2d(bb + r16 * 16, &mapBits16, fb, (col >> 7) * 4, g.contig + r16);
+          }
         }
         if (++stage == nstage) { stage = 0; phase ^= 1; }
       }
