@@ -192,6 +192,7 @@ __device__ __forceinline__ void apply_keep(uint32_t &v01, uint32_t &v89, uint32_
 struct ShrinkWarp {
   uint32_t pool, full0, empty0;
   int stage_bytes, nstage, nblk, kbeg, Rp, mb, MW, KW, mphase, kphase;
+  int NB;  // 64-column blocks per ring stage (a multiple of KW)
   int mask;  // dropout on X: 0 none, 1 keep bits staged with the rows, 2 keep bits from HBM, 3 hash
 };
 
@@ -298,16 +299,18 @@ __device__ __forceinline__ void shrink_consume(const ShrinkWarp &w, const Shrink
     }
   };
 
-  // stage S of the ring holds blocks S*KW .. S*KW + KW - 1 (KW blocks of
-  // stage_bytes each); warp group kphase takes block S*KW + kphase, and every
-  // consumer warp releases the stage
-  const int nsuper = (w.nblk + w.KW - 1) / w.KW;
+  // stage S of the ring holds blocks S*NB .. S*NB + NB - 1 (NB blocks of
+  // stage_bytes each, NB a multiple of KW); warp group kphase takes blocks
+  // kphase, kphase + KW, ... of it, and every consumer warp releases the stage
+  const int nsuper = (w.nblk + w.NB - 1) / w.NB;
   for (int S = 0; S < nsuper; ++S) {
     const int stage = S % w.nstage;
     const uint32_t phase = static_cast<uint32_t>(S / w.nstage) & 1u;
     if (!mbar_wait(w.full0 + 8 * stage, phase)) { *abort_flag = 1; break; }
-    const int b = S * w.KW + w.kphase;
-    if (b < w.nblk) consume(b, w.pool + stage * w.KW * w.stage_bytes + w.kphase * w.stage_bytes);
+    for (int j = w.kphase; j < w.NB; j += w.KW) {
+      const int b = S * w.NB + j;
+      if (b < w.nblk) consume(b, w.pool + (stage * w.NB + j) * w.stage_bytes);
+    }
     __syncwarp();
     if (lane == 0) mbar_arrive(w.empty0 + 8 * stage);
   }
@@ -379,10 +382,12 @@ __global__ void __launch_bounds__(kSkThreads, 2)
   int MW = 1;
   while (MW * 2 <= mb && MW < kSkConsumerWarps) MW *= 2;
   const int KW = kSkConsumerWarps / MW;
-  // a ring stage holds KW consecutive 64-column blocks, one per warp group, so a
-  // small unit's copies come in groups (a lone 16-row block pair per barrier
-  // round trip kept too few bytes moving)
-  const int nstage = min(kSkMaxStages, kSkPool / (KW * stage_bytes));
+  // a ring stage holds NB consecutive 64-column blocks: small units (at most 32
+  // rows) take four, shared out over the KW warp groups, so their copies come in
+  // groups (a lone 16-row block pair per barrier round trip kept too few bytes
+  // moving); larger units one
+  const int NB = Rp <= 32 ? 4 : KW;
+  const int nstage = min(kSkMaxStages, kSkPool / (NB * stage_bytes));
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
@@ -406,17 +411,17 @@ __global__ void __launch_bounds__(kSkThreads, 2)
       int stage = 0;
       uint32_t phase = 0;
       const int xrow = p.x_sorted ? g.row0 : g.contig;
-      const int nsuper = (nblk + KW - 1) / KW;
+      const int nsuper = (nblk + NB - 1) / NB;
       for (int S = 0; S < nsuper; ++S) {
         if (xrow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; break; }
         if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
         const uint32_t fb = full0 + 8 * stage;
-        const int nb = min(KW, nblk - S * KW);  // blocks in this stage
+        const int nb = min(NB, nblk - S * NB);  // blocks in this stage
         mbar_arrive_expect_tx(fb, nb * stage_tx);
         for (int j = 0; j < nb; ++j) {
-          const uint32_t xb = pool + (stage * KW + j) * stage_bytes;
+          const uint32_t xb = pool + (stage * NB + j) * stage_bytes;
           const uint32_t fbuf = xb + Rp * 128;
-          const int col = kbeg + (S * KW + j) * kSkBK;
+          const int col = kbeg + (S * NB + j) * kSkBK;
           for (int r16 = 0; r16 < Rp; r16 += 16) tma_load_2d(xb + r16 * 128, &mapIn16, fb, col, xrow + r16);
           for (int n16 = 0; n16 < g.nn; n16 += 16) tma_load_2d(fbuf + n16 * 128, &mapF16, fb, col, g.frow + n16);
           if (stage_bits) {
@@ -442,6 +447,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
     w.mb = mb;
     w.MW = MW;
     w.KW = KW;
+    w.NB = NB;
     w.mphase = warp % MW;
     w.kphase = warp / MW;
     w.mask = (p.mode != 0 || p.thr == 0) ? 0 : (stage_bits ? 1 : (p.keep_bits ? 2 : 3));
