@@ -91,6 +91,10 @@ struct GemmParams {
   // q, q+S, ...; partial accumulators are summed through distributed shared
   // memory and CTA q stores output columns [q*256/S, (q+1)*256/S).
   int32_t ksplit;
+  // persistent mode: CTA b runs tiles sched_tiles[sched_off[b] .. sched_off[b+1])
+  // (indices in the visiting order); null: round robin
+  const int32_t *sched_off;
+  const int32_t *sched_tiles;
 };
 
 // Split-K exchange, inside the idle stage ring once every MMA of the cluster is
@@ -156,16 +160,35 @@ __device__ __forceinline__ uint32_t map_rank(uint32_t local_addr, uint32_t rank)
 // rows stay in L2 while its n-tiles are swept (A read from DRAM about once, B
 // about n_mt / group_m times). The m-tile index goes through mt_order when the
 // plan has one.
-__device__ __forceinline__ void tile_coords(int tile, const GemmParams &p, int &mt, int &nt) {
-  const int G = p.group_m;
-  const int per_group = G * p.n_nt;
+__host__ __device__ inline void tile_mn(int tile, int n_mt, int n_nt, int G, int &mi, int &nt) {
+  const int per_group = G * n_nt;
   const int g = tile / per_group;
   const int r = tile - g * per_group;
   const int m0 = g * G;
-  const int gm = min(G, p.n_mt - m0);
-  const int mi = m0 + r % gm;
+  const int gm = G < n_mt - m0 ? G : n_mt - m0;
+  mi = m0 + r % gm;
   nt = r / gm;
+}
+__device__ __forceinline__ void tile_coords(int tile, const GemmParams &p, int &mt, int &nt) {
+  int mi;
+  tile_mn(tile, p.n_mt, p.n_nt, p.group_m, mi, nt);
   mt = p.mt_order ? p.mt_order[mi] : mi;
+}
+
+// The k-th tile (in the visiting order above) of this CTA in persistent mode:
+// the plan's schedule lists each CTA's tiles when it has one (tiles of unequal
+// adapter work spread over the CTAs by estimated cost), else the CTA takes
+// tiles blockIdx.x, blockIdx.x + gridDim.x, ...
+__device__ __forceinline__ bool cta_tile(const GemmParams &p, int k, int tile0, int tile_step, int n_tiles,
+                                         int &tile) {
+  if (p.sched_off) {
+    const int i = p.sched_off[blockIdx.x] + k;
+    if (i >= p.sched_off[blockIdx.x + 1]) return false;
+    tile = p.sched_tiles[i];
+    return true;
+  }
+  tile = tile0 + k * tile_step;
+  return tile < n_tiles;
 }
 
 // Barrier 1 over the 4 epilogue warps (128 threads). The OR form returns, to every
@@ -271,7 +294,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // global loads inside the K loop); lane 0 issues every TMA copy.
     int stage = 0;
     uint32_t phase = 0;
-    for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
+    int tile;
+    for (int k = 0; !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
       int mt, nt;
       tile_coords(tile, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
@@ -349,7 +373,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       prefetch_tmap(&mapB);
       int stage = 0;
       uint32_t phase = 0;
-      for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
+      int tile;
+      for (int k = 0; !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
         int mt, nt;
         tile_coords(tile, p, mt, nt);
         const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
@@ -393,7 +418,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint32_t phase = 0;
       int acc = 0;
       uint32_t aphase = 0;
-      for (int tile = tile0; tile < n_tiles && !*abort_flag; tile += tile_step) {
+      int tile;
+      for (int k = 0; !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
         int mt, nt;
         tile_coords(tile, p, mt, nt);
         const int kaug = has_plan ? p.tiles[mt].kaug : 0;
@@ -458,7 +484,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     // the backward's warps leave together (epi_bar_or), so its loop ignores the
     // flag here and tests it at the barrier
-    for (int tile = tile0; tile < n_tiles && (EPI == kEpiBwdLora || !*abort_flag); tile += tile_step) {
+    int tile;
+    for (int k = 0; (EPI == kEpiBwdLora || !*abort_flag) && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
       int mt, nt;
       tile_coords(tile, p, mt, nt);
       const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);

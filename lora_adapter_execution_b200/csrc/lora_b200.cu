@@ -3,6 +3,8 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <queue>
+#include <utility>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
@@ -148,14 +150,69 @@ int launch_status() { return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_
 // Forward GEMM launch: persistent CTAs when there are enough output tiles to
 // fill the GPU; otherwise clusters of S CTAs split the K loop of each tile
 // (S a power of two, S * tiles <= SMs, S <= number of K blocks).
+int fwd_ksplit(int n_tiles, int KB, int num_sms) {
+  int S = 1;
+  while (S < 4 && 2 * S * n_tiles <= num_sms && 2 * S <= KB) S *= 2;  // S in {1, 2, 4}
+  return S;
+}
+
+// Tiles of the persistent fused GEMM per CTA: in the kernel's visiting order,
+// each tile goes to the CTA with the least estimated work so far (greedy list
+// scheduling). A tile costs its base K blocks plus 1.3x its adapter K blocks
+// (per-CTA timings: an adapter block takes about 1.3 times a base block). With
+// equal costs this is the round robin the kernel would do by itself; with the
+// uneven adapter work of many small adapters per tile it evens out the CTAs'
+// loads. Output: off[grid + 1] then the tile indices, CTA by CTA, or nothing
+// when the round robin is about as even.
+void build_schedule(const HostPlan &hp, int grid, int group_m, std::vector<int32_t> &out) {
+  const int n_mt = static_cast<int>(hp.tiles.size());
+  const int n_nt = static_cast<int>((hp.d_out + kBN - 1) / kBN);
+  const int KB = static_cast<int>((hp.d_in + kBK - 1) / kBK);
+  const int n_tiles = n_mt * n_nt;
+  std::vector<std::vector<int32_t>> lists(grid);
+  using Load = std::pair<int64_t, int>;  // (work so far, CTA): ties go to the lowest CTA
+  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> q;
+  for (int b = 0; b < grid; ++b) q.push({0, b});
+  for (int t = 0; t < n_tiles; ++t) {
+    int mi, nt;
+    tile_mn(t, n_mt, n_nt, group_m, mi, nt);
+    const int mt = hp.mt_order.empty() ? mi : hp.mt_order[mi];
+    const int naug = (hp.tiles[mt].kaug + kAugBlock - 1) / kAugBlock;
+    const Load l = q.top();
+    q.pop();
+    lists[l.second].push_back(t);
+    q.push({l.first + 10 * KB + 13 * naug, l.second});
+  }
+  // keep it only where it shortens the heaviest CTA by more than 2 % against the
+  // round robin (whose tile order keeps more operands shared through L2)
+  int64_t greedy_max = 0;
+  while (!q.empty()) {
+    greedy_max = std::max(greedy_max, q.top().first);
+    q.pop();
+  }
+  std::vector<int64_t> rr(grid, 0);
+  for (int t = 0; t < n_tiles; ++t) {
+    int mi, nt;
+    tile_mn(t, n_mt, n_nt, group_m, mi, nt);
+    const int mt = hp.mt_order.empty() ? mi : hp.mt_order[mi];
+    rr[t % grid] += 10 * KB + 13 * ((hp.tiles[mt].kaug + kAugBlock - 1) / kAugBlock);
+  }
+  const int64_t rr_max = *std::max_element(rr.begin(), rr.end());
+  out.clear();
+  if (greedy_max * 100 > rr_max * 98) return;
+  out.assign(grid + 1, 0);
+  for (int b = 0; b < grid; ++b) out[b + 1] = out[b] + static_cast<int32_t>(lists[b].size());
+  for (int b = 0; b < grid; ++b) out.insert(out.end(), lists[b].begin(), lists[b].end());
+}
+
 int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const CUtensorMap &b,
                     const CUtensorMap &bl, lora_stream_t stream) {
   const int n_tiles = gp.n_mt * gp.n_nt;
   const int KB = (gp.K + kBK - 1) / kBK;
   gp.group_m = default_group_m(gp.n_mt, gp.K);
-  int S = 1;
-  while (S < 4 && 2 * S * n_tiles <= ds->num_sms && 2 * S <= KB) S *= 2;  // S in {1, 2, 4}
+  const int S = fwd_ksplit(n_tiles, KB, ds->num_sms);
   gp.ksplit = S;
+  if (S > 1) gp.sched_off = gp.sched_tiles = nullptr;  // one tile per cluster
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S));
   cfg.blockDim = dim3(kGemmThreads);
@@ -191,6 +248,8 @@ struct lora_plan {
   const UnitDesc *d_units = nullptr;
   const int32_t *d_mt_order = nullptr;
   const AugBlockDesc *d_augblocks = nullptr;
+  std::vector<int32_t> sched;           // the fused GEMM's per-CTA tiles (build_schedule), if persistent
+  const int32_t *d_sched = nullptr;     // off[grid + 1] | tiles
   size_t dev_cap = 0, scratch_cap = 0;  // allocated bytes (a rebuild reuses them when they fit)
   int device = 0;
 };
@@ -232,7 +291,17 @@ int upload_plan(lora_plan *pl, lora_stream_t stream) {
   const size_t b_units = up(sizeof(UnitDesc) * hp.units.size());
   const size_t b_order = up(sizeof(int32_t) * hp.mt_order.size());
   const size_t b_aug = up(sizeof(AugBlockDesc) * hp.augblocks.size());
-  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug;
+  // the persistent fused GEMM's tile schedule (its grid and tile order as launched)
+  pl->sched.clear();
+  {
+    const int n_mt = static_cast<int>(hp.tiles.size());
+    const int n_tiles = n_mt * static_cast<int>((hp.d_out + kBN - 1) / kBN);
+    const int KB = static_cast<int>((hp.d_in + kBK - 1) / kBK);
+    if (n_tiles > 0 && fwd_ksplit(n_tiles, KB, ds->num_sms) == 1)
+      build_schedule(hp, std::min(ds->num_sms, n_tiles), default_group_m(n_mt, hp.d_in), pl->sched);
+  }
+  const size_t b_sched = up(sizeof(int32_t) * pl->sched.size());
+  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug + b_sched;
   auto release = [&]() {
     if (pl->dev) cudaFree(pl->dev);
     if (pl->scratch) cudaFree(pl->scratch);
@@ -271,6 +340,8 @@ int upload_plan(lora_plan *pl, lora_stream_t stream) {
   pl->d_mt_order = reinterpret_cast<const int32_t *>(base + b_perm + b_tiles + b_chunks + b_units);
   pl->d_augblocks =
       reinterpret_cast<const AugBlockDesc *>(base + b_perm + b_tiles + b_chunks + b_units + b_order);
+  uint8_t *sched_dst = base + b_perm + b_tiles + b_chunks + b_units + b_order + b_aug;
+  pl->d_sched = pl->sched.empty() ? nullptr : reinterpret_cast<const int32_t *>(sched_dst);
   bool ok = true;
   ok &= cudaMemcpyAsync(base, hp.perm.data(), sizeof(int32_t) * hp.perm.size(), cudaMemcpyHostToDevice,
                         stream) == cudaSuccess;
@@ -285,6 +356,9 @@ int upload_plan(lora_plan *pl, lora_stream_t stream) {
   if (!hp.augblocks.empty())
     ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks + b_units + b_order, hp.augblocks.data(),
                           sizeof(AugBlockDesc) * hp.augblocks.size(), cudaMemcpyHostToDevice,
+                          stream) == cudaSuccess;
+  if (!pl->sched.empty())
+    ok &= cudaMemcpyAsync(sched_dst, pl->sched.data(), sizeof(int32_t) * pl->sched.size(), cudaMemcpyHostToDevice,
                           stream) == cudaSuccess;
   // the copies read host vectors that the plan keeps alive; make sure they have
   // been consumed before returning so the caller may reuse its stream freely
@@ -493,6 +567,11 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   gp.uimg = plan->scratch;
   gp.mt_order = plan->d_mt_order;
   gp.augblocks = plan->d_augblocks;
+  if (plan->d_sched) {
+    const int grid = static_cast<int>(plan->sched.size()) - gp.n_mt * gp.n_nt - 1;
+    gp.sched_off = plan->d_sched;
+    gp.sched_tiles = plan->d_sched + grid + 1;
+  }
   gp.a_sorted = sorted ? 1 : 0;
   gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
   return launch_fwd_gemm(ds, gp, mX128, mW, mBl, stream);
