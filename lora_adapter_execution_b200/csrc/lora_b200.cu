@@ -568,9 +568,14 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   gp.mt_order = plan->d_mt_order;
   gp.augblocks = plan->d_augblocks;
   if (plan->d_sched) {
-    const int grid = static_cast<int>(plan->sched.size()) - gp.n_mt * gp.n_nt - 1;
-    gp.sched_off = plan->d_sched;
-    gp.sched_tiles = plan->d_sched + grid + 1;
+    // the lists were made for the persistent grid of the plan's device; they
+    // apply only to a launch of that same grid
+    const int n_tiles = gp.n_mt * gp.n_nt;
+    const int grid = static_cast<int>(plan->sched.size()) - n_tiles - 1;
+    if (grid == std::min(ds->num_sms, n_tiles)) {
+      gp.sched_off = plan->d_sched;
+      gp.sched_tiles = plan->d_sched + grid + 1;
+    }
   }
   gp.a_sorted = sorted ? 1 : 0;
   gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
