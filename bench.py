@@ -13,7 +13,8 @@ copy) timed with CUDA events on the replay stream, max over ranks.
 Prints one JSON line (rank 0). `value` = tokens of all ranks / max-over-ranks
 device time of the K timed steps. `e2e` is the same metric through the public
 API with host buffers: per step the plan is built from host ids, X is copied
-from pinned host memory, the forward runs, Y is copied back.
+from pinned host memory, the forward runs, Y is copied back; consecutive steps
+overlap (copy-in, compute and copy-out streams over two slots of buffers).
 
 Under torchrun each rank processes its own batch of the same workload (weak
 scaling, no collective on the data path).
@@ -513,41 +514,73 @@ def run_lora(a):
             d2h += pin_dX.numel() * 2
         Ke = max(3, min(K, 200 if not finetune else 20))
 
-        p = lora.Plan(inp.ids, inp.ranks, di, do, stream=stream)
+        # Steps run as a pipeline over two slots (device buffers, plan, pinned
+        # results): step i copies its inputs in on one stream, computes on a
+        # second and copies its results out on a third, so the copies of one step
+        # overlap the compute of its neighbours. Each step still builds its plan
+        # from the host ids and moves all of its own inputs and results.
+        s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+        slots = copies[:2]
+        plans = [lora.Plan(inp.ids, inp.ranks, di, do, stream=s_in) for _ in range(2)]
+        pin_Ys = [pin_Y, torch.empty(T, do, dtype=torch.bfloat16).pin_memory()]
+        pin_dXs = [pin_dX, torch.empty(T, di, dtype=torch.bfloat16).pin_memory()] if finetune else None
+        ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "comp", "out")}
 
-        def e2e_step():
-            p.rebuild(inp.ids, stream=stream)  # the batch's plan from its host ids (buffers reused)
-            with torch.cuda.stream(stream):
-                cp["X"].copy_(pin_X, non_blocking=True)
+        def e2e_step(i):
+            s = i % 2
+            c, p = slots[s], plans[s]
+            if i >= 2:
+                s_in.wait_event(ev["comp"][s])  # step i - 2 is done with this slot's inputs and plan
+            p.rebuild(inp.ids, stream=s_in)  # the batch's plan from its host ids (buffers reused)
+            with torch.cuda.stream(s_in):
+                c["X"].copy_(pin_X, non_blocking=True)
+                if finetune:
+                    c["dY"].copy_(pin_dY, non_blocking=True)
+                ev["in"][s].record(s_in)
+            s_comp.wait_event(ev["in"][s])
+            if i >= 2:
+                s_comp.wait_event(ev["out"][s])  # step i - 2's results have left this slot
+            with torch.cuda.stream(s_comp):
                 bits = None
                 if finetune and inp.p_drop > 0:
-                    bits = cp["bits"]
-                    lora.dropout_keep_bits(inp.mask_seed, inp.p_drop, bits, di, stream=stream)
-                lora.linear_fwd(p, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["Y"], p_drop=inp.p_drop,
-                                seed=inp.mask_seed, U_save=cp["U"], keep_bits=bits)
+                    bits = c["bits"]
+                    lora.dropout_keep_bits(inp.mask_seed, inp.p_drop, bits, di, stream=s_comp)
+                lora.linear_fwd(p, c["X"], c["W"], c["A"], c["B"], scale, c["Y"], p_drop=inp.p_drop,
+                                seed=inp.mask_seed, U_save=c["U"], keep_bits=bits)
                 if finetune:
-                    cp["dY"].copy_(pin_dY, non_blocking=True)
-                    lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"],
-                                    cp["dX"], cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=inp.mask_seed,
+                    lora.linear_bwd(c["X"], c["W"], c["A"], c["B"], float(inp.scale[0]), c["U"], c["dY"],
+                                    c["dX"], c["dA"], c["dB"], c["ws"], p_drop=inp.p_drop, seed=inp.mask_seed,
                                     keep_bits=bits)
-                    pin_dX.copy_(cp["dX"], non_blocking=True)
-                pin_Y.copy_(cp["Y"], non_blocking=True)
-            stream.synchronize()
+                ev["comp"][s].record(s_comp)
+            s_out.wait_event(ev["comp"][s])
+            with torch.cuda.stream(s_out):
+                pin_Ys[s].copy_(c["Y"], non_blocking=True)
+                if finetune:
+                    pin_dXs[s].copy_(c["dX"], non_blocking=True)
+                ev["out"][s].record(s_out)
 
-        for _ in range(2):
-            e2e_step()
+        def drain():
+            for st in (s_in, s_comp, s_out):
+                st.synchronize()
+
+        for i in range(2):
+            e2e_step(i)
+        drain()
         if world > 1:
             dist.barrier()
         t0 = time.perf_counter()
-        for _ in range(Ke):
-            e2e_step()
+        for i in range(Ke):
+            e2e_step(2 + i)
+        drain()
         dt = time.perf_counter() - t0
-        p.destroy()
+        for p in plans:
+            p.destroy()
         dt = max_over_ranks(dt, world, dev)
         out["e2e"] = {"value": job_throughput(T, Ke, world, dt * 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
                       "d2h_bytes_per_step": int(d2h), "steps": Ke,
-                      "what": "plan from host ids + H2D of X (pinned) + forward" + (" + backward" if finetune else "")
-                              + " + D2H of the result, host wall clock per step"}
+                      "what": "per step: plan from host ids + H2D of X (pinned) + forward" + (" + backward" if finetune else "")
+                              + " + D2H of the result; steps pipelined over two slots (copy-in, compute and"
+                              " copy-out streams); host wall clock over the steps"}
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
