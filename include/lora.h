@@ -101,9 +101,15 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
 /* Refill an existing device plan with a new batch (arguments as in
  * lora_plan_build). The plan's device tables and scratch are reused when they
  * are large enough and reallocated otherwise, so a serving loop that builds one
- * plan per batch does not allocate device memory per batch. No work that uses
- * the plan may be in flight on any stream (the caller orders it, as for any
- * buffer it overwrites); the call returns after the tables have reached the
+ * plan per batch does not allocate device memory per batch. The tables are
+ * copied to the device on `stream` from one of two pinned host staging buffers
+ * the plan owns (used in turn; a buffer is refilled only after its previous copy
+ * has completed), and the call returns without waiting for that copy: work that
+ * uses the rebuilt plan must run on `stream` or after it, and work on other
+ * streams that uses the plan's previous contents must be finished before the
+ * call or ordered before `stream` by the caller (work earlier on `stream` is
+ * ordered by the stream). The host arrays may be freed on return. When the
+ * plan's device buffers must grow they are reallocated, which waits for the
  * device. On LORA_ERR_ARG / LORA_ERR_ID / LORA_ERR_RANK the plan is unchanged;
  * after LORA_ERR_NOMEM or LORA_ERR_CUDA it holds no device memory and is only
  * good for lora_plan_destroy. No counterpart in the pages (the plan's device

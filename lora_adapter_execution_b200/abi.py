@@ -134,7 +134,9 @@ class Plan:
 
     def rebuild(self, ids, *, ranks=None, stream=None):
         """lora_plan_rebuild: the same plan object for a new batch (device buffers
-        reused when they fit); no work using the plan may be in flight."""
+        reused when they fit). Stream-ordered on `stream` (default: the current
+        torch stream): run the plan's work there or after it; work on other
+        streams that still uses the old tables must be ordered first."""
         self._ids = _host_i32(ids)
         if ranks is not None:
             self._ranks = _host_i32(ranks)

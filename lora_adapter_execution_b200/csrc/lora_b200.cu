@@ -250,6 +250,10 @@ struct lora_plan {
   const AugBlockDesc *d_augblocks = nullptr;
   std::vector<int32_t> sched;           // the fused GEMM's per-CTA tiles (build_schedule), if persistent
   const int32_t *d_sched = nullptr;     // off[grid + 1] | tiles
+  void *stage[2] = {nullptr, nullptr};  // pinned host staging of the tables, used in turn
+  size_t stage_cap[2] = {0, 0};
+  cudaEvent_t stage_ev[2] = {nullptr, nullptr};  // the last copy out of each staging buffer
+  int stage_next = 0;
   size_t dev_cap = 0, scratch_cap = 0;  // allocated bytes (a rebuild reuses them when they fit)
   int device = 0;
 };
@@ -278,7 +282,8 @@ namespace {
 // smaller than the plan needs (kept otherwise, so a rebuilt plan reuses them),
 // then upload the tables. Returns LORA_OK or an error; on error the plan keeps
 // no device memory.
-int upload_plan(lora_plan *pl, lora_stream_t stream) {
+// sync: wait until the tables are on the device before returning.
+int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
   DeviceState *ds = nullptr;
   int rc = device_state(&ds);
   if (rc != LORA_OK) return rc;
@@ -342,27 +347,43 @@ int upload_plan(lora_plan *pl, lora_stream_t stream) {
       reinterpret_cast<const AugBlockDesc *>(base + b_perm + b_tiles + b_chunks + b_units + b_order);
   uint8_t *sched_dst = base + b_perm + b_tiles + b_chunks + b_units + b_order + b_aug;
   pl->d_sched = pl->sched.empty() ? nullptr : reinterpret_cast<const int32_t *>(sched_dst);
+  // The tables go to the device in one copy from one of the plan's two pinned
+  // staging buffers, laid out as the device buffer. A staging buffer is refilled
+  // only after its previous copy has completed (its event), so consecutive
+  // rebuilds need no stream synchronisation.
   bool ok = true;
-  ok &= cudaMemcpyAsync(base, hp.perm.data(), sizeof(int32_t) * hp.perm.size(), cudaMemcpyHostToDevice,
-                        stream) == cudaSuccess;
-  ok &= cudaMemcpyAsync(base + b_perm, hp.tiles.data(), sizeof(TileDesc) * hp.tiles.size(),
-                        cudaMemcpyHostToDevice, stream) == cudaSuccess;
-  ok &= cudaMemcpyAsync(base + b_perm + b_tiles, hp.chunks.data(), sizeof(ChunkDesc) * hp.chunks.size(),
-                        cudaMemcpyHostToDevice, stream) == cudaSuccess;
-  ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks, hp.units.data(), sizeof(UnitDesc) * hp.units.size(),
-                        cudaMemcpyHostToDevice, stream) == cudaSuccess;
-  ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks + b_units, hp.mt_order.data(),
-                        sizeof(int32_t) * hp.mt_order.size(), cudaMemcpyHostToDevice, stream) == cudaSuccess;
-  if (!hp.augblocks.empty())
-    ok &= cudaMemcpyAsync(base + b_perm + b_tiles + b_chunks + b_units + b_order, hp.augblocks.data(),
-                          sizeof(AugBlockDesc) * hp.augblocks.size(), cudaMemcpyHostToDevice,
-                          stream) == cudaSuccess;
-  if (!pl->sched.empty())
-    ok &= cudaMemcpyAsync(sched_dst, pl->sched.data(), sizeof(int32_t) * pl->sched.size(), cudaMemcpyHostToDevice,
-                          stream) == cudaSuccess;
-  // the copies read host vectors that the plan keeps alive; make sure they have
-  // been consumed before returning so the caller may reuse its stream freely
-  ok &= cudaStreamSynchronize(stream) == cudaSuccess;
+  const int k = pl->stage_next;
+  if (pl->stage_ev[k]) ok &= cudaEventSynchronize(pl->stage_ev[k]) == cudaSuccess;
+  else ok &= cudaEventCreateWithFlags(&pl->stage_ev[k], cudaEventDisableTiming) == cudaSuccess;
+  if (ok && total > pl->stage_cap[k]) {
+    if (pl->stage[k]) cudaFreeHost(pl->stage[k]);
+    pl->stage[k] = nullptr;
+    pl->stage_cap[k] = 0;
+    if (cudaHostAlloc(&pl->stage[k], total, cudaHostAllocDefault) != cudaSuccess) {
+      cudaGetLastError();
+      release();
+      return LORA_ERR_NOMEM;
+    }
+    pl->stage_cap[k] = total;
+  }
+  if (ok) {
+    uint8_t *h = static_cast<uint8_t *>(pl->stage[k]);
+    auto put = [&](size_t off, const void *src, size_t bytes) {
+      if (bytes) std::memcpy(h + off, src, bytes);
+    };
+    put(0, hp.perm.data(), sizeof(int32_t) * hp.perm.size());
+    put(b_perm, hp.tiles.data(), sizeof(TileDesc) * hp.tiles.size());
+    put(b_perm + b_tiles, hp.chunks.data(), sizeof(ChunkDesc) * hp.chunks.size());
+    put(b_perm + b_tiles + b_chunks, hp.units.data(), sizeof(UnitDesc) * hp.units.size());
+    put(b_perm + b_tiles + b_chunks + b_units, hp.mt_order.data(), sizeof(int32_t) * hp.mt_order.size());
+    put(b_perm + b_tiles + b_chunks + b_units + b_order, hp.augblocks.data(),
+        sizeof(AugBlockDesc) * hp.augblocks.size());
+    put(static_cast<size_t>(sched_dst - base), pl->sched.data(), sizeof(int32_t) * pl->sched.size());
+    ok &= cudaMemcpyAsync(base, h, total, cudaMemcpyHostToDevice, stream) == cudaSuccess;
+    ok &= cudaEventRecord(pl->stage_ev[k], stream) == cudaSuccess;
+    pl->stage_next = k ^ 1;
+  }
+  if (ok && sync) ok &= cudaStreamSynchronize(stream) == cudaSuccess;
   if (!ok) {
     cudaGetLastError();
     release();
@@ -380,7 +401,7 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   lora_plan *pl = new (std::nothrow) lora_plan();
   if (!pl) return LORA_ERR_NOMEM;
   int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, pl->hp);
-  if (rc == LORA_OK) rc = upload_plan(pl, stream);
+  if (rc == LORA_OK) rc = upload_plan(pl, stream, true);
   if (rc != LORA_OK) {
     delete pl;
     return rc;
@@ -396,7 +417,7 @@ int lora_plan_rebuild(lora_plan_t plan, const int32_t *ids_host, int64_t T, cons
   int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, hp);
   if (rc != LORA_OK) return rc;  // the plan is unchanged
   plan->hp = std::move(hp);
-  return upload_plan(plan, stream);
+  return upload_plan(plan, stream, false);
 }
 
 int lora_plan_build_host(const int32_t *ids_host, int64_t T, const int32_t *ranks_host, int32_t n_adapters,
@@ -442,6 +463,13 @@ int lora_plan_info(lora_plan_t plan, lora_plan_info_t *info) {
 
 void lora_plan_destroy(lora_plan_t plan) {
   if (!plan) return;
+  for (int k = 0; k < 2; ++k) {
+    if (plan->stage_ev[k]) {
+      cudaEventSynchronize(plan->stage_ev[k]);  // its copy may still read the staging buffer
+      cudaEventDestroy(plan->stage_ev[k]);
+    }
+    if (plan->stage[k]) cudaFreeHost(plan->stage[k]);
+  }
   if (plan->dev) cudaFree(plan->dev);
   if (plan->scratch) cudaFree(plan->scratch);
   delete plan;
