@@ -95,6 +95,10 @@ struct GemmParams {
   // (indices in the visiting order); null: round robin
   const int32_t *sched_off;
   const int32_t *sched_tiles;
+  // split-K exchange through L2: slot (tile, src, owner) at
+  // xws + ((tile * S + src) * S + owner) * xslot_bytes(S); null: through
+  // distributed shared memory
+  uint8_t *xws;
 };
 
 // Split-K exchange, inside the idle stage ring once every MMA of the cluster is
@@ -608,11 +612,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const bool epi = warp >= 2 && warp < 6;
     const bool valid = epi && row < split_rows;
     const int64_t orig = valid ? split_orig : 0;
-    // barrier: every CTA's MMAs are complete, so every stage ring is idle and may
-    // receive; it also orders the receive barriers' initialisation before any
-    // remote completion
-    cluster_barrier();
-    if (threadIdx.x == 64) mbar_arrive_expect_tx(recv_bar, (S - 1) * xslot_bytes(S));
+    // Two ways to move the partials. Through distributed shared memory: after a
+    // cluster barrier (every CTA's MMAs are complete, so every stage ring is idle
+    // and may receive; it also orders the receive barriers' initialisation before
+    // any remote completion) each CTA copies its blocks into the owners' rings.
+    // Through L2 (the plan's workspace): each CTA writes its blocks to global
+    // memory, and after the cluster barrier each owner copies its blocks in; the
+    // peers' rings are never written, and this measured faster.
+    const bool via_l2 = p.xws != nullptr;
+    if (!via_l2) {
+      cluster_barrier();
+      if (threadIdx.x == 64) mbar_arrive_expect_tx(recv_bar, (S - 1) * xslot_bytes(S));
+    }
     bool go = false;
     if (epi) {
       go = tile0 < n_tiles && !*abort_flag;
@@ -653,13 +664,37 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         for (int owner = 0; owner < S; ++owner) {
           if (owner == q) continue;
           const int oidx = owner < q ? owner : owner - 1;
-          const int jq = q < owner ? q : q - 1;  // this rank's slot at the owner
-          bulk_s2s_cluster(map_rank(slot0 + static_cast<uint32_t>(jq * xslot_bytes(S)), static_cast<uint32_t>(owner)),
-                           out0 + static_cast<uint32_t>(oidx * xslot_bytes(S)), xslot_bytes(S),
-                           map_rank(recv_bar, static_cast<uint32_t>(owner)));
+          const uint32_t src = out0 + static_cast<uint32_t>(oidx * xslot_bytes(S));
+          if (via_l2) {
+            bulk_s2g(p.xws + (static_cast<int64_t>(tile0 * S + q) * S + owner) * xslot_bytes(S), src, xslot_bytes(S));
+          } else {
+            const int jq = q < owner ? q : q - 1;  // this rank's slot at the owner
+            bulk_s2s_cluster(map_rank(slot0 + static_cast<uint32_t>(jq * xslot_bytes(S)), static_cast<uint32_t>(owner)),
+                             src, xslot_bytes(S), map_rank(recv_bar, static_cast<uint32_t>(owner)));
+          }
         }
         bulk_commit();
+        if (via_l2) {
+          bulk_wait_all();  // the partials are in global memory before the barrier releases them
+          fence_proxy_async_global();
+        }
       }
+    }
+    if (via_l2) {
+      cluster_barrier();  // every rank's partials are written
+      if (go && threadIdx.x == 64) {
+        fence_proxy_async_global();
+        mbar_arrive_expect_tx(recv_bar, (S - 1) * xslot_bytes(S));
+        for (int src = 0; src < S; ++src) {
+          if (src == q) continue;
+          const int js = src < q ? src : src - 1;
+          bulk_g2s(slot0 + static_cast<uint32_t>(js * xslot_bytes(S)),
+                   p.xws + (static_cast<int64_t>(tile0 * S + src) * S + q) * xslot_bytes(S), xslot_bytes(S),
+                   recv_bar);
+        }
+      }
+    }
+    if (epi) {
       // receive: own partial from TMEM + the other ranks' blocks in rank order
       // (a fixed order, so the result is deterministic)
       if (go) {

@@ -254,6 +254,8 @@ struct lora_plan {
   size_t stage_cap[2] = {0, 0};
   cudaEvent_t stage_ev[2] = {nullptr, nullptr};  // the last copy out of each staging buffer
   int stage_next = 0;
+  int xws_S = 0;          // split of the fused GEMM whose exchange workspace the scratch holds (0: none)
+  size_t xws_offset = 0;  // its byte offset in the scratch
   size_t dev_cap = 0, scratch_cap = 0;  // allocated bytes (a rebuild reuses them when they fit)
   int device = 0;
 };
@@ -326,16 +328,31 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
     }
     pl->dev_cap = total;
   }
-  if (static_cast<size_t>(hp.scratch_bytes) > pl->scratch_cap) {
+  // a split-K fused GEMM exchanges its partial sums through a workspace behind
+  // the scratch's images (and sorted X): [tiles][S][S] slots of xslot_bytes(S)
+  pl->xws_S = 0;
+  pl->xws_offset = 0;
+  size_t scratch_total = static_cast<size_t>(hp.scratch_bytes);
+  {
+    const int n_tiles = static_cast<int>(hp.tiles.size()) * static_cast<int>((hp.d_out + kBN - 1) / kBN);
+    const int KB = static_cast<int>((hp.d_in + kBK - 1) / kBK);
+    const int S = n_tiles > 0 ? fwd_ksplit(n_tiles, KB, ds->num_sms) : 1;
+    if (S > 1) {
+      pl->xws_S = S;
+      pl->xws_offset = up(scratch_total);
+      scratch_total = pl->xws_offset + static_cast<size_t>(n_tiles) * S * S * xslot_bytes(S);
+    }
+  }
+  if (scratch_total > pl->scratch_cap) {
     if (pl->scratch) cudaFree(pl->scratch);
     pl->scratch = nullptr;
     pl->scratch_cap = 0;
-    if (cudaMalloc(reinterpret_cast<void **>(&pl->scratch), hp.scratch_bytes) != cudaSuccess) {
+    if (cudaMalloc(reinterpret_cast<void **>(&pl->scratch), scratch_total) != cudaSuccess) {
       cudaGetLastError();
       release();
       return LORA_ERR_NOMEM;
     }
-    pl->scratch_cap = static_cast<size_t>(hp.scratch_bytes);
+    pl->scratch_cap = scratch_total;
   }
   uint8_t *base = static_cast<uint8_t *>(pl->dev);
   pl->d_perm = reinterpret_cast<const int32_t *>(base);
@@ -595,6 +612,11 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   gp.uimg = plan->scratch;
   gp.mt_order = plan->d_mt_order;
   gp.augblocks = plan->d_augblocks;
+  {
+    const int KB = (gp.K + kBK - 1) / kBK;
+    if (plan->xws_S > 1 && fwd_ksplit(gp.n_mt * gp.n_nt, KB, ds->num_sms) == plan->xws_S)
+      gp.xws = plan->scratch + plan->xws_offset;
+  }
   if (plan->d_sched) {
     // the lists were made for the persistent grid of the plan's device; they
     // apply only to a launch of that same grid
