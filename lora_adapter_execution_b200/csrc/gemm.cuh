@@ -88,8 +88,9 @@ struct GemmParams {
                             // copy fills a B slot; 0: mapBl is 2-D {64, 16}, four copies per slot
   // K split: 1 = persistent CTAs over all tiles; S > 1 = one tile per cluster of
   // S CTAs, CTA q takes base K blocks [q*KB/S, (q+1)*KB/S) and adapter blocks
-  // q, q+S, ...; partial accumulators are summed through distributed shared
-  // memory and CTA q stores output columns [q*256/S, (q+1)*256/S).
+  // q, q+S, ...; partial accumulators are exchanged (through the L2 workspace
+  // xws when given, else distributed shared memory) and CTA q sums and stores
+  // output columns [q*256/S, (q+1)*256/S).
   int32_t ksplit;
   // persistent mode: CTA b runs tiles sched_tiles[sched_off[b] .. sched_off[b+1])
   // (indices in the visiting order); null: round robin
@@ -103,9 +104,11 @@ struct GemmParams {
 
 // Split-K exchange, inside the idle stage ring once every MMA of the cluster is
 // done. Each CTA q owns output columns [q*w, (q+1)*w), w = 256/S. Partials move
-// as 4 KB blocks (32 rows x 32 columns fp32, one epilogue warp's TMEM lanes)
-// with bulk shared-to-shared copies that complete on the owner's receive
-// barrier. Inside a block, row r's 16-byte column group j sits at group
+// as 4 KB blocks (32 rows x 32 columns fp32, one epilogue warp's TMEM lanes),
+// staged per owner and moved whole: by bulk shared-to-shared copies that
+// complete on the owner's receive barrier, or through a global workspace (bulk
+// store by the sender, bulk load by the owner into the same receive slot, with a
+// cluster barrier between). Inside a block, row r's 16-byte column group j sits at group
 // j ^ (r & 7), so both the row-per-thread writes and reads are conflict-free.
 //   [0, (S-1)*w*512)  receive slots, one per other rank (rank order, own skipped),
 //                     each [w/32 column blocks][4 warps][4 KB]
