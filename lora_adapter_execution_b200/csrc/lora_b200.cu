@@ -59,8 +59,10 @@ int device_state(DeviceState **out) {
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_gemm_kernel<true, kEpiBwdLora>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBwd) == cudaSuccess;
-          ok &= cudaFuncSetAttribute(lora_shrink_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     kSkSmem) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_shrink_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sk_smem(4)) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_shrink_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     sk_smem(2)) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_tcontract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      1024 + kTcSmemBudget + 2 * kTcMaxStages * 8) == cudaSuccess;
           if (!ok) d.status = LORA_ERR_CUDA;
@@ -127,22 +129,43 @@ int default_group_m(int n_mt, int64_t K) {
 }
 
 // Cluster size of the shrink (CTAs that split one unit's contraction): the
-// choice in 1..4 with the fewest stages on the critical path, counting whole
-// waves of 2 CTAs per SM (a second, mostly empty wave costs a full one).
-int shrink_split(int n_units, int64_t K, int num_sms) {
+// choice in 1..4 with the least work on the critical path, counting whole waves
+// of ctas_per_sm CTAs per SM (a second, mostly empty wave costs a full one) and,
+// per CTA, its 64-column blocks plus a fixed cost of its setup and tail (about
+// 2.8 us in per-CTA timelines, some 32 blocks' worth at ~0.09 us per block).
+int shrink_split(int n_units, int64_t K, int num_sms, int ctas_per_sm, int64_t *cost_out = nullptr) {
   const int64_t kb = (K + kSkBK - 1) / kSkBK;
-  const int64_t slots = 2 * static_cast<int64_t>(num_sms);
+  const int64_t slots = static_cast<int64_t>(ctas_per_sm) * num_sms;
   int best = 1;
   int64_t best_cost = -1;
   for (int ks = 1; ks <= 4 && ks <= kb; ++ks) {
     const int64_t waves = (static_cast<int64_t>(n_units) * ks + slots - 1) / slots;
-    const int64_t cost = waves * ((kb + ks - 1) / ks);
+    const int64_t cost = waves * ((kb + ks - 1) / ks + 32);
     if (best_cost < 0 || cost < best_cost) {
       best = ks;
       best_cost = cost;
     }
   }
+  if (cost_out) *cost_out = best_cost;
   return best;
+}
+
+// The shrink build for a launch: the small-piece build (three CTAs per SM, a
+// smaller ring) only when every piece allows it and it leaves fewer stages on
+// the critical path than the two-per-SM build (more CTAs per SM alone gave no
+// gain to a launch that needs the same number of waves either way).
+int shrink_build(int n_units, int64_t K, int num_sms, int max_nn, int *ks_out) {
+  int64_t cost_big = 0, cost_small = 0;
+  const int ks_big = shrink_split(n_units, K, num_sms, sk_ctas_per_sm(4), &cost_big);
+  if (max_nn <= 32) {
+    const int ks_small = shrink_split(n_units, K, num_sms, sk_ctas_per_sm(2), &cost_small);
+    if (cost_small < cost_big) {
+      *ks_out = ks_small;
+      return 2;
+    }
+  }
+  *ks_out = ks_big;
+  return 4;
 }
 
 int launch_status() { return cudaGetLastError() == cudaSuccess ? LORA_OK : LORA_ERR_CUDA; }
@@ -515,7 +538,11 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   sp.T = static_cast<int32_t>(hp.T);
   sp.K = static_cast<int32_t>(hp.d_in);
   const int n_units = static_cast<int>(hp.units.size());
-  const int ks = shrink_split(n_units, hp.d_in, ds->num_sms);
+  // the build (and cluster size) with the fewest stages on the critical path
+  int max_nn = 0;
+  for (const UnitDesc &u : hp.units) max_nn = std::max(max_nn, static_cast<int>(u.nn));
+  int ks = 1;
+  const int max_nb16 = shrink_build(n_units, hp.d_in, ds->num_sms, max_nn, &ks);
   int64_t slice = (hp.d_in + ks - 1) / ks;
   slice = (slice + kSkBK - 1) / kSkBK * kSkBK;
   sp.ksplit = ks;
@@ -550,7 +577,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(static_cast<unsigned>(n_units * ks));
   cfg.blockDim = dim3(kSkThreads);
-  cfg.dynamicSmemBytes = kSkSmem;
+  cfg.dynamicSmemBytes = sk_smem(max_nb16);
   cfg.stream = stream;
   // programmatic serialization: the shrink's setup (barriers, its plan entry)
   // overlaps the end of the kernel before it; it waits in pdl_wait before
@@ -571,7 +598,8 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
     lora_gather_rows_kernel<<<blocks, 256, 0, stream>>>(X, plan->d_perm, Xs, hp.T, hp.d_in);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
-  if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mX16, mA16, mBits16, sp) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, max_nb16 <= 2 ? lora_shrink_kernel<2> : lora_shrink_kernel<4>, mX16, mA16, mBits16,
+                         sp) != cudaSuccess) {
     cudaGetLastError();
     return LORA_ERR_CUDA;
   }
@@ -741,7 +769,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     sp.x_sorted = 0;
     sp.dU = dU;
     const int n_units = static_cast<int>((T + kTileM - 1) / kTileM) * sp.npieces;
-    const int ks = shrink_split(n_units, d_out, ds->num_sms);
+    int ks = 1;
+    const int max_nb16 = shrink_build(n_units, d_out, ds->num_sms, std::min(kShrinkN, ((r + 15) / 16) * 16), &ks);
     int64_t slice = (d_out + ks - 1) / ks;
     slice = (slice + kSkBK - 1) / kSkBK * kSkBK;
     sp.ksplit = ks;
@@ -749,7 +778,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     cudaLaunchConfig_t cfg{};
     cfg.gridDim = dim3(static_cast<unsigned>(n_units * ks));
     cfg.blockDim = dim3(kSkThreads);
-    cfg.dynamicSmemBytes = kSkSmem;
+    cfg.dynamicSmemBytes = sk_smem(max_nb16);
     cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -758,7 +787,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    if (cudaLaunchKernelEx(&cfg, lora_shrink_kernel, mdY16, mB16, mdY16, sp) != cudaSuccess) {
+    if (cudaLaunchKernelEx(&cfg, max_nb16 <= 2 ? lora_shrink_kernel<2> : lora_shrink_kernel<4>, mdY16, mB16, mdY16,
+                           sp) != cudaSuccess) {
       cudaGetLastError();
       return LORA_ERR_CUDA;
     }

@@ -33,14 +33,20 @@ namespace lora {
 constexpr int kSkConsumerWarps = 4;
 constexpr int kSkThreads = (kSkConsumerWarps + 1) * 32;  // + 1 producer warp
 constexpr int kSkBK = 64;                                 // columns per stage (one 128-byte swizzled row)
-constexpr int kSkPool = 108 * 1024;                       // stage ring (also the reduction scratch)
 constexpr int kSkMaxStages = 16;
 constexpr int kSkRedBytes = kSkConsumerWarps * 32 * kShrinkN * 4;  // per-warp partials, fp32
 constexpr int kSkFinBytes = kTileM * kShrinkN * 4;        // CTA partial [128 x 64] fp32
-constexpr int kSkSmem = 1024 + kSkPool + 2 * kSkMaxStages * 8 + 64;
-// the partials and the CTA sum reuse the idle ring; two CTAs fit on an SM
-static_assert(kSkRedBytes + kSkFinBytes <= kSkPool, "shrink reduction scratch exceeds the stage pool");
-static_assert(2 * (kSkSmem + 1024) <= 228 * 1024, "two shrink CTAs must fit on an SM");
+// Two builds of the shrink: for pieces of up to 64 rank columns (four 16-column
+// blocks), two CTAs per SM with a 108 KB stage ring; for pieces of at most 32
+// (two blocks: fewer accumulator registers), three CTAs per SM with 72 KB, so
+// runs of many small adapters fill the GPU in fewer waves.
+__host__ __device__ constexpr int sk_ctas_per_sm(int max_nb16) { return max_nb16 <= 2 ? 3 : 2; }
+__host__ __device__ constexpr int sk_pool(int max_nb16) { return max_nb16 <= 2 ? 72 * 1024 : 108 * 1024; }
+__host__ __device__ constexpr int sk_smem(int max_nb16) { return 1024 + sk_pool(max_nb16) + 2 * kSkMaxStages * 8 + 64; }
+// the partials and the CTA sum reuse the idle ring; the CTAs fit on an SM
+static_assert(kSkRedBytes + kSkFinBytes <= sk_pool(2), "shrink reduction scratch exceeds the stage pool");
+static_assert(2 * (sk_smem(4) + 1024) <= 228 * 1024, "two shrink CTAs must fit on an SM");
+static_assert(3 * (sk_smem(2) + 1024) <= 228 * 1024, "three small-piece shrink CTAs must fit on an SM");
 
 struct ShrinkParams {
   int32_t mode;     // 0: forward shrink over plan units; 1: backward dU over consecutive tiles
@@ -336,7 +342,8 @@ __device__ __forceinline__ void shrink_consume(const ShrinkWarp &w, const Shrink
 
 // Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
 // its rank q contracts columns [q*kslice, (q+1)*kslice).
-__global__ void __launch_bounds__(kSkThreads, 2)
+template <int kMaxNB16>
+__global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
     lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows (X, sorted X or dY), box {64, 16}
                        const __grid_constant__ CUtensorMap mapF16,   // F rows, box {64, 16}
                        const __grid_constant__ CUtensorMap mapBits16,  // keep bits [T, wpr] u32, box {4, 16}
@@ -346,6 +353,7 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                                               ~static_cast<uintptr_t>(1023));
   const uint32_t pool = smem_u32(smem);
   float *fin = reinterpret_cast<float *>(smem + kSkRedBytes);  // in the pool, after the partials
+  constexpr int kSkPool = sk_pool(kMaxNB16);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSkPool);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * kSkMaxStages;
@@ -463,11 +471,18 @@ __global__ void __launch_bounds__(kSkThreads, 2)
                                    : (p.mode == 0 ? static_cast<int64_t>(p.perm[g.row0 + rc]) : 0);
       }
     float *red = reinterpret_cast<float *>(smem);
-    switch (g.nn >> 4) {
-      case 1: shrink_consume<1>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
-      case 2: shrink_consume<2>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
-      case 3: shrink_consume<3>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
-      default: shrink_consume<4>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+    // the piece width nn is 16, 32, 48 or 64 (at most 16 * kMaxNB16: the host
+    // launches the small build only for such pieces)
+    if constexpr (kMaxNB16 <= 2) {
+      if (g.nn <= 16) shrink_consume<1>(w, p, g, orow, smem, abort_flag, red, warp, lane);
+      else shrink_consume<2>(w, p, g, orow, smem, abort_flag, red, warp, lane);
+    } else {
+      switch (g.nn >> 4) {
+        case 1: shrink_consume<1>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+        case 2: shrink_consume<2>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+        case 3: shrink_consume<3>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+        default: shrink_consume<4>(w, p, g, orow, smem, abort_flag, red, warp, lane); break;
+      }
     }
   }
 
