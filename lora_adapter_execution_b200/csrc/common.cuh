@@ -30,7 +30,6 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
-__device__ __forceinline__ uint32_t lane_id() { return threadIdx.x & 31u; }
 
 // ------------------------------------------------------------------ mbarrier
 __device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
@@ -248,16 +247,13 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t
 }
 
 // ------------------------------------------------------------------ dropout mask hash
-// Output number `n` (0-based) of a SplitMix64 generator seeded with `seed`
-// (Steele, Lea, Flood, OOPSLA 2014): the state advances by the golden-ratio
-// increment before each output, then a xor-shift / multiply finaliser mixes it.
-__host__ __device__ __forceinline__ uint64_t splitmix64_at(uint64_t seed, uint64_t n) {
-  uint64_t z = seed + (n + 1ull) * 0x9E3779B97F4A7C15ull;
-  z = (z ^ (z >> 30)) * 0xBF58476D1CE4E5B9ull;
-  z = (z ^ (z >> 27)) * 0x94D049BB133111EBull;
-  return z ^ (z >> 31);
-}
-// splitmix64 output of state z (the state after its increment) >= thr, i.e. the
+// SplitMix64 (Steele, Lea, Flood, OOPSLA 2014) seeded with `seed`: output n
+// (0-based) mixes the state z = seed + (n + 1) * 0x9E3779B97F4A7C15 (the state
+// after n + 1 golden-ratio increments) with x ^= x >> 30, x *= 0xBF58476D1CE4E5B9,
+// x ^= x >> 27, x *= 0x94D049BB133111EB, x ^= x >> 31. Element (t, col) of the
+// LoRA-branch input is dropped when output t * d_in + col is below thr = p * 2^64.
+//
+// keep_state: the output of state z (the state after its increment) >= thr (the state after its increment) >= thr, i.e. the
 // element is kept. The comparison needs only the high word of the output unless
 // it ties with the high word of thr (a 2^-32 event): the last product's low word
 // and the last shift's low half are formed only then.
@@ -281,7 +277,7 @@ __device__ __forceinline__ bool keep_elem(uint64_t seed, uint64_t thr, int64_t t
 }
 
 // Keep bits of 32 consecutive mask positions idx0 .. idx0+31 (bit i set if kept):
-// the same SplitMix64 outputs as splitmix64_at, with the state advanced by one
+// the same SplitMix64 outputs as keep_elem, with the state advanced by one
 // increment per position instead of recomputed.
 __device__ __forceinline__ uint32_t keep_mask32(uint64_t seed, uint64_t thr, uint64_t idx0) {
   if (thr == 0) return 0xFFFFFFFFu;
