@@ -53,7 +53,10 @@ WORKLOAD_TEXT = {
     "fleet": "fleet: T=4096, d_in=d_out=4096, 1000 adapters ranks 1..21, B rows x 1/k, Zipf(1.2) per token",
     "finetune": "finetune: T=16384, d_in=d_out=4096, 1 adapter rank 16, s=2, dropout 0.1; forward + backward",
 }
+# The fused GEMM, its launch and the plan tables that shape its work: a recorded
+# ncu figure for the GEMM holds while the code of these files is unchanged.
 KERNEL_SOURCES = ["lora_adapter_execution_b200/csrc/gemm.cuh", "lora_adapter_execution_b200/csrc/common.cuh",
+                  "lora_adapter_execution_b200/csrc/internal.h", "lora_adapter_execution_b200/csrc/plan.cpp",
                   "lora_adapter_execution_b200/csrc/lora_b200.cu"]
 
 

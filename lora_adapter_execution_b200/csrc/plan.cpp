@@ -189,6 +189,14 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
       }
     }
   }
+  // Launch order, longest first: one CTA (or cluster) takes one unit, and
+  // blocks start in index order as earlier ones finish, so the units with the
+  // most rows and rank columns per 64-column block go in the first wave and
+  // the short ones fill the tail. Units write disjoint parts of the image and
+  // of U_save, so their order is free.
+  std::stable_sort(hp.units.begin(), hp.units.end(), [](const UnitDesc &x, const UnitDesc &y) {
+    return ((x.r1 - x.r0 + 15) / 16) * 16 + x.nn > ((y.r1 - y.r0 + 15) / 16) * 16 + y.nn;
+  });
   return LORA_OK;
 }
 
