@@ -92,6 +92,9 @@ enum lora_status {
  *               synchronises it, so the plan is on the device on return (and
  *               the host arrays may be freed)
  *   out         receives the plan; unchanged on error
+ * The plan belongs to the device current at this call: lora_plan_rebuild,
+ * lora_linear_shrink, lora_fused_gemm and lora_linear_fwd return LORA_ERR_ARG
+ * when another device is current.
  * Errors: LORA_ERR_ARG, LORA_ERR_ID, LORA_ERR_RANK, LORA_ERR_NOMEM, LORA_ERR_CUDA.
  * ------------------------------------------------------------------------ */
 int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_host,

@@ -2,7 +2,10 @@
 
 Tensors are torch CUDA tensors (bf16 where the ABI says bf16); each call passes
 their raw device pointers and the current torch stream to the library. Nothing
-here computes any part of the layer.
+here computes any part of the layer. The ABI takes every size from the plan or
+from other arguments, so before a pointer crosses it the tensor's metadata is
+checked against those sizes (exact shape, dtype, contiguous, on the current
+CUDA device); a mismatch raises LoraError with LORA_ERR_ARG and calls nothing.
 """
 
 from __future__ import annotations
@@ -99,6 +102,39 @@ def _ptr(t):
     return None if t is None else ctypes.c_void_p(t.data_ptr())
 
 
+_BF16 = ("bfloat16",)
+_F32 = ("float32",)
+_I32 = ("int32", "uint32")
+
+
+def _args(what, *specs):
+    """Check (name, tensor, shape, dtype names, optional) for each tensor handed
+    to the library call `what`: first every tensor's shape, dtype and layout,
+    then every tensor's device."""
+    given = []
+    for name, t, shape, dtypes, optional in specs:
+        if t is None:
+            if optional:
+                continue
+            raise LoraError(-1, f"{what}: {name} is required")
+        if tuple(t.shape) != tuple(shape):
+            raise LoraError(-1, f"{what}: {name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+        if str(t.dtype).rsplit(".", 1)[-1] not in dtypes:
+            raise LoraError(-1, f"{what}: {name} has dtype {t.dtype}, expected {' or '.join(dtypes)}")
+        if not t.is_contiguous():
+            raise LoraError(-1, f"{what}: {name} is not contiguous")
+        given.append((name, t))
+    dev = None
+    for name, t in given:
+        if not t.is_cuda:
+            raise LoraError(-1, f"{what}: {name} is not a CUDA tensor")
+        if dev is None:
+            import torch
+            dev = torch.cuda.current_device()
+        if t.device.index != dev:
+            raise LoraError(-1, f"{what}: {name} is on {t.device}, the current device is cuda:{dev}")
+
+
 def _stream(stream):
     if stream is None:
         import torch
@@ -131,6 +167,13 @@ class Plan:
         _check(rc, "lora_plan_build")
         self._h = h
         self.T, self.d_in, self.d_out, self.n_adapters = T, d_in, d_out, n
+        self._sizes()
+
+    def _sizes(self):
+        # pool rows (all adapters' ranks) and U_save's row length (the largest
+        # rank among adapters with tokens), as the library reads them
+        self.pool_rows = int(self._ranks.astype(np.int64).sum())
+        self.r_max = int(self.info()["r_max"])
 
     def rebuild(self, ids, *, ranks=None, stream=None):
         """lora_plan_rebuild: the same plan object for a new batch (device buffers
@@ -145,6 +188,7 @@ class Plan:
                                                 self._ranks.ctypes.data_as(_vp), n, self.d_in, self.d_out,
                                                 _stream(stream)), "lora_plan_rebuild")
         self.T, self.n_adapters = T, n
+        self._sizes()
 
     @property
     def handle(self):
@@ -176,8 +220,19 @@ class Plan:
             pass
 
 
+def _fwd_args(plan, X, A_pool, scale, U_save, keep_bits):
+    T, di, R = plan.T, plan.d_in, plan.pool_rows
+    return (("X", X, (T, di), _BF16, False), ("A_pool", A_pool, (R, di), _BF16, False),
+            ("scale", scale, (plan.n_adapters,), _F32, False), ("U_save", U_save, (T, plan.r_max), _F32, True),
+            ("keep_bits", keep_bits, (T, -(-di // 32)), _I32, True))
+
+
 def linear_fwd(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.0, seed: int = 0,
                U_save=None, keep_bits=None, stream=None):
+    di, do, R = plan.d_in, plan.d_out, plan.pool_rows
+    _args("lora_linear_fwd", *_fwd_args(plan, X, A_pool, scale, U_save, keep_bits),
+          ("W", W, (di, do), _BF16, False), ("B_pool", B_pool, (R, do), _BF16, False),
+          ("Y", Y, (plan.T, do), _BF16, False))
     _check(load_library().lora_linear_fwd(plan.handle, _ptr(X), _ptr(W), _ptr(A_pool), _ptr(B_pool), _ptr(scale),
                                           float(p_drop), int(seed) & (2**64 - 1), _ptr(Y), _ptr(U_save),
                                           _ptr(keep_bits), _stream(stream)), "lora_linear_fwd")
@@ -185,6 +240,7 @@ def linear_fwd(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.
 
 def linear_shrink(plan: Plan, X, A_pool, scale, *, p_drop: float = 0.0, seed: int = 0, U_save=None,
                   keep_bits=None, stream=None):
+    _args("lora_linear_shrink", *_fwd_args(plan, X, A_pool, scale, U_save, keep_bits))
     _check(load_library().lora_linear_shrink(plan.handle, _ptr(X), _ptr(A_pool), _ptr(scale), float(p_drop),
                                              int(seed) & (2**64 - 1), _ptr(U_save), _ptr(keep_bits),
                                              _stream(stream)),
@@ -192,6 +248,9 @@ def linear_shrink(plan: Plan, X, A_pool, scale, *, p_drop: float = 0.0, seed: in
 
 
 def fused_gemm(plan: Plan, X, W, B_pool, Y, *, stream=None):
+    T, di, do = plan.T, plan.d_in, plan.d_out
+    _args("lora_fused_gemm", ("X", X, (T, di), _BF16, False), ("W", W, (di, do), _BF16, False),
+          ("B_pool", B_pool, (plan.pool_rows, do), _BF16, False), ("Y", Y, (T, do), _BF16, False))
     _check(load_library().lora_fused_gemm(plan.handle, _ptr(X), _ptr(W), _ptr(B_pool), _ptr(Y), _stream(stream)),
            "lora_fused_gemm")
 
@@ -199,6 +258,8 @@ def fused_gemm(plan: Plan, X, W, B_pool, Y, *, stream=None):
 def base_gemm(X, W, Y, *, stream=None):
     T, d_in = X.shape
     d_out = W.shape[1]
+    _args("lora_base_gemm", ("X", X, (T, d_in), _BF16, False), ("W", W, (d_in, d_out), _BF16, False),
+          ("Y", Y, (T, d_out), _BF16, False))
     _check(load_library().lora_base_gemm(_ptr(X), _ptr(W), _ptr(Y), T, d_in, d_out, _stream(stream)),
            "lora_base_gemm")
 
@@ -207,11 +268,24 @@ def bwd_workspace_size(T: int, d_in: int, d_out: int, r: int) -> int:
     return int(load_library().lora_linear_bwd_workspace_size(T, d_in, d_out, r))
 
 
+def _bwd_args(X, W, A, B, U_save, dY, dX, dA, dB, keep_bits):
+    T, di = X.shape
+    do = W.shape[1]
+    r = A.shape[0]
+    return (("X", X, (T, di), _BF16, False), ("W", W, (di, do), _BF16, False), ("A", A, (r, di), _BF16, False),
+            ("B", B, (r, do), _BF16, False), ("U_save", U_save, (T, r), _F32, False),
+            ("dY", dY, (T, do), _BF16, False), ("dX", dX, (T, di), _BF16, False),
+            ("dA", dA, (r, di), _F32, False), ("dB", dB, (r, do), _F32, False),
+            ("keep_bits", keep_bits, (T, -(-di // 32)), _I32, True))
+
+
 def linear_bwd(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, workspace, *, p_drop: float = 0.0,
                seed: int = 0, keep_bits=None, stream=None):
     T, d_in = X.shape
     d_out = W.shape[1]
     r = A.shape[0]
+    _args("lora_linear_bwd", *_bwd_args(X, W, A, B, U_save, dY, dX, dA, dB, keep_bits))
+    _args("lora_linear_bwd", ("workspace", workspace, tuple(workspace.shape), (str(workspace.dtype)[6:],), False))
     nbytes = workspace.numel() * workspace.element_size()
     _check(load_library().lora_linear_bwd(_ptr(X), _ptr(W), _ptr(A), _ptr(B), float(scale), float(p_drop),
                                           int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY), _ptr(dX), _ptr(dA),
@@ -228,6 +302,7 @@ def linear_bwd_static(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, *, p_dro
     T, d_in = X.shape
     d_out = W.shape[1]
     r = A.shape[0]
+    _args("lora_linear_bwd_static", *_bwd_args(X, W, A, B, U_save, dY, dX, dA, dB, keep_bits))
     _check(load_library().lora_linear_bwd_static(_ptr(X), _ptr(W), _ptr(A), _ptr(B), float(scale), float(p_drop),
                                                  int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY), _ptr(dX),
                                                  _ptr(dA), _ptr(dB), T, d_in, d_out, r, _ptr(keep_bits),
@@ -237,6 +312,7 @@ def linear_bwd_static(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, *, p_dro
 
 def dropout_mask(seed: int, p_drop: float, mask, *, stream=None):
     T, d_in = mask.shape
+    _args("lora_dropout_mask", ("mask", mask, (T, d_in), ("uint8",), False))
     _check(load_library().lora_dropout_mask(int(seed) & (2**64 - 1), float(p_drop), T, d_in, _ptr(mask),
                                             _stream(stream)), "lora_dropout_mask")
 
@@ -244,9 +320,8 @@ def dropout_mask(seed: int, p_drop: float, mask, *, stream=None):
 def dropout_keep_bits(seed: int, p_drop: float, bits, d_in: int, *, stream=None):
     """Write the dropout keep bits of a [T, d_in] input into `bits` (int32 device
     tensor [T, ceil(d_in / 32)]), for linear_fwd / linear_bwd's keep_bits."""
-    T, wpr = bits.shape
-    if wpr != -(-d_in // 32):
-        raise ValueError("bits must have ceil(d_in / 32) columns")
+    T = bits.shape[0]
+    _args("lora_dropout_keep_bits", ("bits", bits, (T, -(-d_in // 32)), _I32, False))
     _check(load_library().lora_dropout_keep_bits(int(seed) & (2**64 - 1), float(p_drop), T, d_in, _ptr(bits),
                                                  _stream(stream)), "lora_dropout_keep_bits")
 

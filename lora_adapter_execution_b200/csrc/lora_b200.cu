@@ -3,6 +3,7 @@
 #include <cudaTypedefs.h>
 
 #include <algorithm>
+#include <atomic>
 #include <queue>
 #include <utility>
 #include <cstdio>
@@ -20,7 +21,7 @@ namespace {
 constexpr int kMaxDevices = 64;
 
 struct DeviceState {
-  bool init = false;
+  std::atomic<bool> init{false};  // set once, after the fields below (release)
   int status = LORA_OK;
   int num_sms = 0;
 };
@@ -32,9 +33,9 @@ int device_state(DeviceState **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_ERR_CUDA;
   DeviceState &d = g_dev[dev];
-  if (!d.init) {
+  if (!d.init.load(std::memory_order_acquire)) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!d.init) {
+    if (!d.init.load(std::memory_order_relaxed)) {
       int major = 0, minor = 0;
       if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev) != cudaSuccess ||
           cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev) != cudaSuccess ||
@@ -68,7 +69,7 @@ int device_state(DeviceState **out) {
           if (!ok) d.status = LORA_ERR_CUDA;
         }
       }
-      d.init = true;
+      d.init.store(true, std::memory_order_release);
     }
   }
   *out = &d;
@@ -284,6 +285,15 @@ struct lora_plan {
   int device = 0;
 };
 
+namespace {
+// A plan's tables and scratch live on the device that was current when it was
+// built; calls on any other device are rejected.
+bool on_plan_device(const lora_plan *pl) {
+  int d = -1;
+  return cudaGetDevice(&d) == cudaSuccess && d == pl->device;
+}
+}  // namespace
+
 extern "C" {
 
 const char *lora_status_string(int code) {
@@ -444,7 +454,7 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
   int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, pl->hp);
   if (rc == LORA_OK) rc = upload_plan(pl, stream, true);
   if (rc != LORA_OK) {
-    delete pl;
+    lora_plan_destroy(pl);  // also frees the staging buffers and events an upload made
     return rc;
   }
   *out = pl;
@@ -453,7 +463,7 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
 
 int lora_plan_rebuild(lora_plan_t plan, const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
                       int32_t n_adapters, int64_t d_in, int64_t d_out, lora_stream_t stream) {
-  if (!plan || !plan->dev) return LORA_ERR_ARG;
+  if (!plan || !plan->dev || !on_plan_device(plan)) return LORA_ERR_ARG;
   HostPlan hp;
   int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, hp);
   if (rc != LORA_OK) return rc;  // the plan is unchanged
@@ -520,6 +530,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
                        double p_drop, uint64_t seed, float *U_save, const uint32_t *keep_bits,
                        lora_stream_t stream) {
   if (!plan || !plan->dev || !X || !A_pool || !scale) return LORA_ERR_ARG;
+  if (!on_plan_device(plan)) return LORA_ERR_ARG;
   if (!aligned16(X) || !aligned16(A_pool)) return LORA_ERR_ARG;
   if (reinterpret_cast<uintptr_t>(keep_bits) & 3u) return LORA_ERR_ARG;
   if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
@@ -610,6 +621,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
 int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *B_pool, uint16_t *Y,
                     lora_stream_t stream) {
   if (!plan || !plan->dev || !X || !W || !B_pool || !Y) return LORA_ERR_ARG;
+  if (!on_plan_device(plan)) return LORA_ERR_ARG;
   if (!aligned16(X) || !aligned16(W) || !aligned16(B_pool) || !aligned16(Y)) return LORA_ERR_ARG;
   DeviceState *ds = nullptr;
   int rc = device_state(&ds);

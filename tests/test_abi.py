@@ -93,3 +93,45 @@ def test_bwd_rejects_bad_rank_before_cuda():
     assert rc == -3
     rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 16, None, 0, None, None)
     assert rc == -8
+
+
+def test_binding_checks_tensor_metadata_before_the_call():
+    """The binding rejects a tensor whose shape, dtype, layout or device does not
+    match the sizes the library will read, before any library call (a host-only
+    plan and CPU tensors: nothing reaches CUDA)."""
+    import torch
+    T, d_in, d_out = 40, 64, 48
+    ids = np.arange(T, dtype=np.int32) % 3
+    ranks = np.array([4, 8, 16], dtype=np.int32)
+    plan = lora.Plan(ids, ranks, d_in, d_out, host_only=True)
+    assert plan.pool_rows == 28 and plan.r_max == 16
+    bf = torch.bfloat16
+    good = dict(X=torch.zeros(T, d_in, dtype=bf), W=torch.zeros(d_in, d_out, dtype=bf),
+                A_pool=torch.zeros(28, d_in, dtype=bf), B_pool=torch.zeros(28, d_out, dtype=bf),
+                scale=torch.ones(3, dtype=torch.float32), Y=torch.zeros(T, d_out, dtype=bf))
+
+    def fwd(**over):
+        a = dict(good, **over)
+        with pytest.raises(lora.LoraError) as e:
+            lora.linear_fwd(plan, a["X"], a["W"], a["A_pool"], a["B_pool"], a["scale"], a["Y"],
+                            U_save=a.get("U_save"), keep_bits=a.get("keep_bits"))
+        assert e.value.code == -1
+        return str(e.value)
+
+    assert "X has shape" in fwd(X=torch.zeros(T - 1, d_in, dtype=bf))
+    assert "A_pool has shape" in fwd(A_pool=torch.zeros(16, d_in, dtype=bf))
+    assert "scale has shape" in fwd(scale=torch.ones(2, dtype=torch.float32))
+    assert "U_save has shape" in fwd(U_save=torch.zeros(T, 8, dtype=torch.float32))
+    assert "keep_bits has shape" in fwd(keep_bits=torch.zeros(T, 1, dtype=torch.int32))
+    assert "W has dtype" in fwd(W=torch.zeros(d_in, d_out, dtype=torch.float16))
+    assert "Y is not contiguous" in fwd(Y=torch.zeros(d_out, T, dtype=bf).t())
+    assert "X is not a CUDA tensor" in fwd()
+    with pytest.raises(lora.LoraError, match="dB has shape"):
+        r = 8
+        lora.linear_bwd(good["X"], good["W"], torch.zeros(r, d_in, dtype=bf), torch.zeros(r, d_out, dtype=bf), 1.0,
+                        torch.zeros(T, r, dtype=torch.float32), torch.zeros(T, d_out, dtype=bf),
+                        torch.zeros(T, d_in, dtype=bf), torch.zeros(r, d_in, dtype=torch.float32),
+                        torch.zeros(r, d_in, dtype=torch.float32), torch.zeros(16, dtype=torch.uint8))
+    with pytest.raises(lora.LoraError, match="bits has shape"):
+        lora.dropout_keep_bits(0, 0.1, torch.zeros(T, 3, dtype=torch.int32), d_in)
+    plan.destroy()
