@@ -130,7 +130,7 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
     hp.tiles.push_back(td);
   }
   // Tiles whose tokens are not consecutive originals read X through a sorted
-  // copy that the shrink writes while it gathers the rows anyway.
+  // copy that the row gather writes into the scratch before the shrink runs.
   bool any_gathered = false;
   for (const TileDesc &td : hp.tiles) any_gathered |= td.contig < 0;
   if (any_gathered) {
