@@ -611,6 +611,12 @@ def run_lora(a):
 
 def main():
     a = parse()
+    rank, _, world = dist_env()
+    if a.gpus != world and rank == 0:
+        # one process per GPU: N GPUs need N processes (torchrun); the line
+        # reports the processes that ran
+        print(f"bench.py: --gpus {a.gpus} but {world} process(es) (WORLD_SIZE); "
+              f"launch N > 1 with torchrun --nproc-per-node N", file=sys.stderr)
     if a.impl == "reference":
         run_reference(a)
     else:
