@@ -84,3 +84,48 @@ def test_reference_arm_other_ranks_exit_quietly():
                         "--steps", "1", "--warmup", "3"], env=env, capture_output=True, text=True, timeout=300)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == ""
+
+
+def _rank_leaves(rank, world, port, q):
+    """Rank 1 leaves between steps (after one agreed step, before the next
+    all-reduce); rank 0 must learn of it through an error from its next
+    collective within the short process-group timeout, not wait for good."""
+    import datetime
+    import time
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=datetime.timedelta(seconds=5))
+    first = bench.max_over_ranks(1.0 + rank, world)
+    if rank == 1:
+        q.put((rank, first, "left"))
+        q.close()
+        q.join_thread()  # the message is out before the process ends
+        os._exit(0)  # leaves without joining the next step
+    t0 = time.monotonic()
+    try:
+        bench.max_over_ranks(1.0, world)
+        outcome = "no error"
+    except Exception as e:  # the backend's error type varies by version
+        outcome = type(e).__name__
+    q.put((rank, first, outcome, time.monotonic() - t0))
+    q.close()
+    q.join_thread()
+    os._exit(0)
+
+
+def test_rank_that_leaves_ends_the_next_collective_with_an_error():
+    world = 2
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_rank_leaves, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    got = sorted([q.get(timeout=120) for _ in range(world)], key=lambda g: g[0])
+    for p in procs:
+        p.join(timeout=60)
+    assert got[0][1] == got[1][1] == 2.0       # the step both ranks took agreed
+    assert got[1][2] == "left"
+    assert got[0][2] != "no error"             # rank 0's next collective failed ...
+    assert got[0][3] < 60.0                    # ... within the timeout's bound, not forever
