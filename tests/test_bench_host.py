@@ -1,0 +1,49 @@
+"""bench.py's host-side arithmetic, on CPU: the algorithmic bytes and flops that
+the roofline divides by, recomputed from the inputs alone (numpy over the ids
+and ranks, not the planner), and the planner's rank sums they use."""
+import os
+import sys
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+import lora_adapter_execution_b200 as lora  # noqa: E402
+from lora_adapter_execution_b200 import workloads as wl  # noqa: E402
+
+
+@pytest.mark.parametrize("name", ["tiny", "decode", "fleet"])
+def test_algorithmic_bytes_and_flops_from_first_principles(name):
+    inp = wl.make_inputs(name)
+    plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out, host_only=True)
+    info = plan.info()
+    used = np.unique(inp.ids)
+    r_used = int(inp.ranks[used].astype(np.int64).sum())
+    r_tok = int(inp.ranks[inp.ids].astype(np.int64).sum())
+    assert info["sum_r_used"] == r_used and info["sum_r_tokens"] == r_tok
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    # the fused GEMM touches X, W, the used adapters' B rows, the s·U image's
+    # source (counted with the shrink) and Y, each once, 2 bytes an element
+    elems = T * di + di * do + sum(int(inp.ranks[a]) * do for a in used) + T * do
+    # dense flops: the base product, then each token's rank-r expand
+    flops = 2 * T * di * do + sum(2 * do * int(inp.ranks[a]) for a in inp.ids)
+    gb, gf, lb, lf = bench.algorithmic(inp, info)
+    assert gb == 2 * elems and gf == flops
+    # the layer adds A's used rows and each token's rank-r shrink
+    assert lb == 2 * (elems + sum(int(inp.ranks[a]) * di for a in used))
+    assert lf == flops + sum(2 * di * int(inp.ranks[a]) for a in inp.ids)
+    plan.destroy()
+
+
+def test_decode_gemm_bytes_match_the_reported_figure():
+    """The decode line's algorithmic bytes per launch: 2 B x (X 256x4096 + W
+    4096x4096 + B rows of the used adapters x 4096 + Y 256x4096)."""
+    inp = wl.make_inputs("decode")
+    plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out, host_only=True)
+    gb = bench.algorithmic(inp, plan.info())[0]
+    r_used = int(inp.ranks[np.unique(inp.ids)].sum())
+    assert gb == 2 * (256 * 4096 + 4096 * 4096 + r_used * 4096 + 256 * 4096)
+    plan.destroy()
