@@ -15,9 +15,9 @@ import lora_adapter_execution_b200 as lora  # noqa: E402
 from lora_adapter_execution_b200 import workloads as wl  # noqa: E402
 
 
-@pytest.mark.parametrize("name", ["tiny", "decode", "fleet"])
-def test_algorithmic_bytes_and_flops_from_first_principles(name):
-    inp = wl.make_inputs(name)
+@pytest.mark.parametrize("name,kw", [("tiny", {}), ("decode", {}), ("fleet", {"d_in": 256, "d_out": 264})])
+def test_algorithmic_bytes_and_flops_from_first_principles(name, kw):
+    inp = wl.make_inputs(name, **kw)  # fleet's ids and ranks at narrow widths
     plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out, host_only=True)
     info = plan.info()
     used = np.unique(inp.ids)
