@@ -167,13 +167,16 @@ class Plan:
         _check(rc, "lora_plan_build")
         self._h = h
         self.T, self.d_in, self.d_out, self.n_adapters = T, d_in, d_out, n
-        self._sizes()
+        self._sizes(True)
 
-    def _sizes(self):
+    def _sizes(self, ranks_changed):
         # pool rows (all adapters' ranks) and U_save's row length (the largest
         # rank among adapters with tokens), as the library reads them
-        self.pool_rows = int(self._ranks.astype(np.int64).sum())
-        self.r_max = int(self.info()["r_max"])
+        if ranks_changed:
+            self.pool_rows = int(self._ranks.astype(np.int64).sum())
+        inf = _Info()
+        _check(load_library().lora_plan_info(self._h, ctypes.byref(inf)), "lora_plan_info")
+        self.r_max = int(inf.r_max)
 
     def rebuild(self, ids, *, ranks=None, stream=None):
         """lora_plan_rebuild: the same plan object for a new batch (device buffers
@@ -188,7 +191,7 @@ class Plan:
                                                 self._ranks.ctypes.data_as(_vp), n, self.d_in, self.d_out,
                                                 _stream(stream)), "lora_plan_rebuild")
         self.T, self.n_adapters = T, n
-        self._sizes()
+        self._sizes(ranks is not None)
 
     @property
     def handle(self):
