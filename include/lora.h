@@ -160,6 +160,9 @@ void lora_plan_destroy(lora_plan_t plan);
 
 /* ------------------------------------------------------------------------
  * lora_linear_fwd — Y = X·W + s_a·((D ⊙ X)·A_a)·B_a for every token.
+ * Source: the LoRA reparameterisation of the LoRAFusion explainer (section
+ * 解决什么真问题, item 1), applied per token with that token's adapter, the
+ * base part batched and no padding (S-LoRA article, section 批处理).
  *
  *   X       bf16 [T, d_in]     tokens in their original order
  *   W       bf16 [d_in, d_out] frozen base weight
@@ -197,6 +200,10 @@ int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
  * (lora_linear_fwd is exactly lora_linear_shrink followed by lora_fused_gemm
  * on one stream).
  *
+ * Source: the shrink (X·A) and expand (·B) halves of the same
+ * reparameterisation; the pages keep them as separate small kernels next to
+ * the base GEMM, here the expand is folded into the GEMM.
+ *
  * lora_linear_shrink: U = (D ⊙ X)·A_a for every token, written as s_a·U in
  * bf16 into the plan's scratch (in the layout the fused GEMM reads) and, if
  * U_save is not NULL, as U into U_save. When the plan's tiles are not runs of
@@ -214,14 +221,17 @@ int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
                     uint16_t *Y, lora_stream_t stream);
 
 /* Y = X·W only (no adapter term), through the same tcgen05 GEMM kernel: the
- * base-only reference the adapter overhead is measured against.
+ * base-only reference the adapter overhead is measured against (the frozen
+ * base term of the LoRAFusion explainer's reparameterisation).
  * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA. */
 int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T, int64_t d_in,
                    int64_t d_out, lora_stream_t stream);
 
 /* ------------------------------------------------------------------------
  * lora_linear_bwd — backward of the forward for one adapter (fine-tuning;
- * every token uses it), W frozen so no dW. Plain chain rule:
+ * every token uses it), W frozen so no dW. The pages fix the forward and that
+ * W is frozen (LoRAFusion explainer, section 解决什么真问题, item 1); the
+ * backward is its plain chain rule:
  *   dU = s·dY·B^T                       [T, r]
  *   dB = s·U^T·dY                       [r, d_out]
  *   dA = ((D ⊙ X)^T·dU)^T, stored [r, d_in] (row k = column k of dA)
@@ -286,7 +296,9 @@ int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t 
                            int64_t d_in, int64_t d_out, int32_t r, const uint32_t *keep_bits,
                            lora_stream_t stream);
 
-/* Test hook: write the dropout mask the forward and backward use.
+/* Test hook: write the dropout mask the forward and backward use (dropout on
+ * the LoRA-branch input, one of the small ops the LoRAFusion explainer lists in
+ * section 解决什么真问题, item 1; the drop rule is the one under lora_linear_fwd).
  *   mask_dev  uint8 [T, d_in] device: 1 where X[t, i] is dropped, else 0.
  * Errors: LORA_ERR_ARG, LORA_ERR_CUDA. */
 int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint8_t *mask_dev,
