@@ -1,26 +1,38 @@
 """Benchmark of the multi-adapter LoRA linear layer on B200.
 
-    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl lora|reference]
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config all|NAME] [--impl lora|reference]
 
 One step = one pass of the layer's whole hot path over one batch: the shrink
 (U = (D ⊙ X)·A_a per token) and the fused tcgen05 GEMM (Y = X·W + s_a·U·B_a)
-over a plan built once per batch (and, for the fine-tuning workload, the
-backward dU -> dX GEMM -> dA, dB). Inputs are resident in HBM; steps rotate
+over a plan built once per batch and, for the fine-tuning workload, the
+backward (dU -> dX GEMM -> dA, dB). Inputs are resident in HBM; steps rotate
 over several input copies whose total exceeds the 126 MB L2, so no step reads
-its operands from a warm L2. Steps are CUDA-graph replays (one graph per input
-copy) timed with CUDA events on the replay stream, max over ranks.
+its operands from a warm L2. Steps are CUDA-graph replays timed with CUDA
+events on the replay stream; a timed region is exactly K steps bracketed by a
+barrier and a device synchronisation, repeated until the clock sampler has
+seen it for a while, and the median region is reported (max over ranks).
 
-Prints one JSON line (rank 0). `value` = tokens of all ranks / max-over-ranks
-device time of the K timed steps. `e2e` is the same metric through the public
-API with host buffers: per step the plan is built from host ids, X is copied
-from pinned host memory, the forward runs, Y is copied back; consecutive steps
-overlap (copy-in, compute and copy-out streams over two slots of buffers).
+With no --config every workload runs in one process and rank 0 prints ONE
+JSON line: the fine-tuning workload (the largest single-GPU configuration,
+forward + backward) is the headline (`value`, `roofline`, `e2e`,
+`cpu_baseline`), and `configs` holds the same record for every workload.
+`roofline` is the fused forward GEMM (the kernel the layer is built around);
+`layer_roofline` is the whole step against the same peak.
 
-Under torchrun each rank processes its own batch of the same workload (weak
-scaling, no collective on the data path).
+`e2e` is the same metric through the public API with host buffers: per step
+the plan is built from host ids, X (and dY) are copied from pinned host
+memory, the layer runs, the result is copied back; consecutive steps overlap
+(copy-in, compute and copy-out streams over two slots of buffers).
+
+Multi-GPU: one process per GPU. Under torchrun each rank runs the layer on a
+batch of its own (weak scaling). For the fine-tuning workload the ranks'
+batches are shards of one global batch (data parallel): each step ends with
+one NCCL all-reduce (sum) of the adapter gradients dA, dB, and each rank's
+dropout mask is the global batch's mask at its rows. `--gpus N` without
+torchrun re-executes this script under torchrun with N processes.
 
 --impl reference times the CPU oracle (fp64 loops, all host cores) on a
-bounded sample of the same workload.
+bounded sample of the headline workload, with the same config record.
 """
 
 from __future__ import annotations
@@ -30,6 +42,7 @@ import hashlib
 import json
 import math
 import os
+import socket
 import subprocess
 import sys
 import threading
@@ -44,8 +57,12 @@ from lora_adapter_execution_b200 import workloads as wl  # noqa: E402
 
 METRIC = "tokens/s per fused multi-LoRA linear at 1 B200; % of bf16 TC peak / HBM roofline"
 L2_BYTES = 126 * 1024 * 1024
+ORDER = ("tiny", "decode", "prefill", "fleet", "finetune")
+HEADLINE = "finetune"
 DEFAULT_STEPS = {"tiny": 2000, "decode": 3000, "prefill": 200, "fleet": 1000, "finetune": 100}
 DEFAULT_WARMUP = 5
+MIN_REGION_S = 0.3  # a timed region is repeated until this much device time has passed
+CPU_BUDGET_S = {"headline": 12.0, "other": 5.0}
 WORKLOAD_TEXT = {
     "tiny": "tiny: T=64, d_in=d_out=256, 4 adapters ranks {4,8,8,16}, s=16/r, ids uniform",
     "decode": "decode: T=256, d_in=d_out=4096, 64 adapters rank 16, s=2, ids uniform (unsorted)",
@@ -60,22 +77,28 @@ KERNEL_SOURCES = ["lora_adapter_execution_b200/csrc/gemm.cuh", "lora_adapter_exe
                   "lora_adapter_execution_b200/csrc/lora_b200.cu"]
 
 
-def parse():
+def parse(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=DEFAULT_WARMUP)
-    ap.add_argument("--config", default="decode", choices=list(wl.WORKLOADS))
+    ap.add_argument("--config", default="all", choices=["all", *wl.WORKLOADS])
     ap.add_argument("--impl", default="lora", choices=["lora", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-layer", action="store_true",
                     help="time only the full step (no GEMM-alone, base or torch timings; for profiler runs)")
-    a = ap.parse_args()
-    if a.steps is None:
-        a.steps = DEFAULT_STEPS[a.config]
+    ap.add_argument("--once", action="store_true",
+                    help="one timed region per config, no repeats (for profiler runs)")
+    ap.add_argument("--dry-run", action="store_true",
+                    help="no GPU: exercise the ranks' start-up and collectives over gloo and print a line")
+    a = ap.parse_args(argv)
     a.warmup = max(3, a.warmup)
     return a
+
+
+def steps_for(a, name):
+    return a.steps if a.steps is not None else DEFAULT_STEPS[name]
 
 
 def dist_env():
@@ -94,10 +117,52 @@ def max_over_ranks(x: float, world: int, device=None) -> float:
     return float(t.item())
 
 
+def allreduce_grads(grad, world: int):
+    """Data-parallel fine-tuning's one exchange: sum the ranks' adapter gradients
+    (dA and dB, views of the one fp32 buffer `grad`) in place. Each rank's dA, dB
+    is a sum over its own tokens, so the sum over ranks is the gradient of the
+    global batch."""
+    if world <= 1:
+        return grad
+    import torch.distributed as dist
+    dist.all_reduce(grad, op=dist.ReduceOp.SUM)
+    return grad
+
+
+def rank_rows(rank: int, tokens_per_rank: int) -> int:
+    """First global row of rank `rank`'s shard of the global batch."""
+    return rank * tokens_per_rank
+
+
 def job_throughput(tokens_per_rank: int, steps: int, world: int, ms: float) -> float:
     """Whole-job tokens/s: every rank processed steps x tokens_per_rank tokens of
     its own batch (weak scaling) in ms, the max over ranks."""
     return world * tokens_per_rank * steps / (ms * 1e-3)
+
+
+def n_copies_for(per_copy: int) -> int:
+    return max(2, min(8, math.ceil(3 * L2_BYTES / per_copy)))
+
+
+def copy_bytes(inp) -> int:
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    per_copy = 2 * (T * di + di * do + T * do) + 2 * (di + do) * int(inp.offsets[-1])
+    if inp.dY is not None:
+        per_copy += 2 * (T * do + 2 * T * di)
+    return per_copy
+
+
+def config_record(name, inp, world):
+    """The `config` object of a line: what the workload is and how it is run.
+    Computed from the inputs alone, so both arms print the same record."""
+    per_copy = copy_bytes(inp)
+    n = n_copies_for(per_copy)
+    ft = inp.dY is not None
+    return {"workload": WORKLOAD_TEXT[name], "tokens_per_rank": inp.T,
+            "l2": f"inputs rotate over {n} copies ({n * per_copy / 2**20:.0f} MiB > 126 MiB L2)",
+            "parallelism": (f"dp{world} (shards of one global batch, all-reduce of dA, dB per step)" if ft
+                            else f"dp{world} (independent batches, no collective)"),
+            "plan": "built once per batch outside the timed region (reused by every layer)"}
 
 
 # ----------------------------------------------------------------------------- clocks
@@ -249,6 +314,16 @@ def algorithmic(inp, info):
     return gemm_bytes, gemm_flops, layer_bytes, layer_flops
 
 
+def algorithmic_bwd(inp, r):
+    """Algorithmic bytes and flops of the single-adapter backward: reads X, W, dY,
+    A, B, U, writes dX, dA, dB; flops of dU = s·dY·B^T, the dX GEMM with its adapter
+    term, dB = s·U^T·dY and dA = (D⊙X)^T·dU."""
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    nbytes = 2 * (T * di + di * do + T * do + r * (di + do)) + 4 * T * r + 2 * T * di + 4 * r * (di + do)
+    flops = 2 * T * do * di + 2 * T * r * (do + di + do + di)
+    return nbytes, flops
+
+
 # ----------------------------------------------------------------------------- reference arm
 def _oracle_runner(inp):
     """(run(n) -> seconds, what) for the oracle on n tokens of the workload: the
@@ -286,18 +361,24 @@ def oracle_sample(inp, budget_s: float):
     return n, dt, what.format(n=n)
 
 
+def reference_name(a):
+    return HEADLINE if a.config == "all" else a.config
+
+
 def run_reference(a):
     rank, _, world = dist_env()
     if rank != 0:
         return
     import oracle
-    inp = wl.make_inputs(a.config)
+    name = reference_name(a)
+    inp = wl.make_inputs(name)
     oracle.build()
     cores = oracle.num_threads()
     # the whole run (warm-up + K steps) takes about 90 s of oracle time: each
     # step is a bounded sample sized once from a calibration run
+    K = steps_for(a, name)
     run, what = _oracle_runner(inp)
-    per_step = 90.0 / max(1, a.steps + a.warmup)
+    per_step = 90.0 / max(1, K + a.warmup)
     n0 = 2
     dt0 = run(n0)
     n = int(max(1, min(inp.T, n0 * per_step / max(dt0, 1e-6))))
@@ -305,319 +386,434 @@ def run_reference(a):
         run(n)
     tok = 0
     secs = 0.0
-    for _ in range(a.steps):
+    for _ in range(K):
         secs += run(n)
         tok += n
     v = tok / secs
     sample = what.format(n=n)
     out = {"impl": "reference", "metric": METRIC, "value": v, "unit": "tokens/s", "n_gpus": world,
-           "steps": a.steps, "warmup": a.warmup, "ms_per_step": 1e3 * secs / a.steps,
+           "steps": K, "warmup": a.warmup, "ms_per_step": 1e3 * secs / K,
            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-           "config": {"workload": WORKLOAD_TEXT[a.config]},
+           "config": config_record(name, inp, world),
            "cpu_baseline": {"value": v, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
            "e2e": {"value": v, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(out), flush=True)
 
 
 # ----------------------------------------------------------------------------- lora arm
-def run_lora(a):
+class Ctx:
+    """What the per-workload measurements share: the device, the process group,
+    the replay stream and the arguments."""
+
+    def __init__(self, a):
+        import torch
+        import torch.distributed as dist
+        import lora_adapter_execution_b200 as lora
+        self.a = a
+        self.rank, self.local_rank, self.world = dist_env()
+        torch.cuda.set_device(self.local_rank)
+        self.dev = torch.device("cuda", self.local_rank)
+        if self.world > 1:
+            import datetime
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=self.dev)
+        lora.load_library()
+        self.stream = torch.cuda.Stream(device=self.dev)
+
+    def barrier(self):
+        if self.world > 1:
+            import torch.distributed as dist
+            dist.barrier()
+
+    def timed(self, step, K, repeats=True):
+        """Device ms of exactly K calls of step() (graph replays), each region
+        bracketed by a barrier and a synchronisation; repeated until MIN_REGION_S
+        of device time (at least 3 regions) unless repeats is False; returns the
+        median region, max over ranks."""
+        import torch
+        for i in range(self.a.warmup):
+            step(i)
+        torch.cuda.synchronize()
+        regions = []
+        total = 0.0
+        while True:
+            self.barrier()
+            torch.cuda.synchronize()
+            e0 = torch.cuda.Event(enable_timing=True)
+            e1 = torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(self.stream):
+                e0.record(self.stream)
+                for i in range(K):
+                    step(i)
+                e1.record(self.stream)
+            torch.cuda.synchronize()
+            self.barrier()
+            ms = e0.elapsed_time(e1)
+            regions.append(ms)
+            total += ms * 1e-3
+            # every rank takes the same decision (the max over ranks of the total)
+            done = (not repeats) or (len(regions) >= 3 and max_over_ranks(total, self.world, self.dev) >= MIN_REGION_S)
+            if done or len(regions) >= 2000:
+                break
+        return max_over_ranks(float(np.median(regions)), self.world, self.dev), len(regions)
+
+
+def measure(name, cx, cpu_budget):
+    """Every figure of one workload: the step's throughput, the fused GEMM's and
+    the layer's roofline fractions, e2e through the public API, the CPU baseline."""
     import torch
     import torch.distributed as dist
-
     import lora_adapter_execution_b200 as lora
 
-    rank, local_rank, world = dist_env()
-    torch.cuda.set_device(local_rank)
-    dev = torch.device("cuda", local_rank)
-    if world > 1:
-        import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=dev)
-    lora.load_library()
-
-    # each rank its own batch (tokens and ids) of the same layer
-    inp = wl.make_rank_inputs(a.config, rank)
+    a, dev, world, rank = cx.a, cx.dev, cx.world, cx.rank
+    inp = wl.make_rank_inputs(name, rank)
     T, di, do = inp.T, inp.d_in, inp.d_out
     finetune = inp.dY is not None
+    K = steps_for(a, name)
+    # data parallel: this rank's rows are global rows rank*T.. of one batch, so
+    # its dropout mask is the global mask there
+    mask_seed = lora.dropout_seed_for_rows(inp.mask_seed, rank_rows(rank, T), di) if finetune else inp.mask_seed
 
     def d(bits):
         return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
 
-    per_copy = 2 * (T * di + di * do + T * do) + 2 * (di + do) * int(inp.offsets[-1])
-    if finetune:
-        per_copy += 2 * (T * do + 2 * T * di)
-    n_copies = max(2, min(8, math.ceil(3 * L2_BYTES / per_copy)))
+    per_copy = copy_bytes(inp)
+    n_copies = n_copies_for(per_copy)
     plan = lora.Plan(inp.ids, inp.ranks, di, do)
     info = plan.info()
     r_max = info["r_max"]
     scale = torch.from_numpy(inp.scale).to(dev)
+    r = int(inp.ranks[0])
     copies = []
     for c in range(n_copies):
         cp = dict(X=d(inp.X), W=d(inp.W), A=d(inp.A_pool), B=d(inp.B_pool),
                   Y=torch.empty(T, do, dtype=torch.bfloat16, device=dev),
                   U=torch.empty(T, r_max, dtype=torch.float32, device=dev) if finetune else None)
         if finetune:
-            r = int(inp.ranks[0])
-            cp.update(dY=d(inp.dY), dX=torch.empty(T, di, dtype=torch.bfloat16, device=dev),
-                      dA=torch.empty(r, di, dtype=torch.float32, device=dev),
-                      dB=torch.empty(r, do, dtype=torch.float32, device=dev),
+            grad = torch.empty(r * (di + do), dtype=torch.float32, device=dev)  # dA | dB, one all-reduce
+            cp.update(dY=d(inp.dY), dX=torch.empty(T, di, dtype=torch.bfloat16, device=dev), grad=grad,
+                      dA=grad[: r * di].view(r, di), dB=grad[r * di:].view(r, do),
                       ws=torch.empty(lora.bwd_workspace_size(T, di, do, r), dtype=torch.uint8, device=dev),
                       bits=torch.empty(T, -(-di // 32), dtype=torch.int32, device=dev))
         copies.append(cp)
 
-    # one graph per copy; the plan (and its scratch) is shared, steps run in order.
-    # With dropout, copy c's batch has its own mask seed; its keep bits depend on
-    # the seed only, so each step writes the next copy's bits on a second stream
-    # while its own forward GEMM runs (the bits kernel needs no shared memory and
-    # fits beside the GEMM's CTAs), and joins that stream before it ends.
+    # One graph per copy; the plan (and its scratch) is shared, steps run in
+    # order. Copy c holds step c's batch; with dropout each copy's keep bits are
+    # written on a second stream during the previous step's forward GEMM (the
+    # bits kernel needs no shared memory and fits beside the GEMM's CTAs), and
+    # that stream is joined before the step ends.
     masked = finetune and inp.p_drop > 0
     side = torch.cuda.Stream(device=dev)
     ev_fork = torch.cuda.Event()
     ev_join = torch.cuda.Event()
 
-    def seed_of(c):
-        return inp.mask_seed + c
-
     def step(c):
         cp, nxt = copies[c], (c + 1) % len(copies)
         bits = cp["bits"] if masked else None
-        lora.linear_shrink(plan, cp["X"], cp["A"], scale, p_drop=inp.p_drop, seed=seed_of(c), U_save=cp["U"],
+        lora.linear_shrink(plan, cp["X"], cp["A"], scale, p_drop=inp.p_drop, seed=mask_seed, U_save=cp["U"],
                            keep_bits=bits)
         cur = torch.cuda.current_stream()
         if masked:
             ev_fork.record(cur)
             side.wait_event(ev_fork)
             with torch.cuda.stream(side):
-                lora.dropout_keep_bits(seed_of(nxt), inp.p_drop, copies[nxt]["bits"], di)
+                lora.dropout_keep_bits(mask_seed, inp.p_drop, copies[nxt]["bits"], di)
             ev_join.record(side)
         lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
         if finetune:
             lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"], cp["dX"],
-                            cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=seed_of(c), keep_bits=bits)
+                            cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=mask_seed, keep_bits=bits)
         if masked:
             cur.wait_event(ev_join)
 
-    # the forward: [row gather] + shrink + fused GEMM; the backward: dU, dX GEMM, 2 x (contraction + reduce)
-    launches_per_step = 2 + int(info["gathers_x"]) + (6 if finetune else 0) + (1 if finetune and inp.p_drop > 0 else 0)
-    stream = torch.cuda.Stream(device=dev)
+    # launches of this library per step: [row gather] + shrink + fused GEMM; the
+    # backward: dU shrink, [U padding copy], dX GEMM, 2 contractions per 64-rank
+    # group, 2 reductions; the keep bits of the next copy
+    n_groups = -(-r // 64)
+    launches_per_step = 2 + int(info["gathers_x"])
+    if finetune:
+        launches_per_step += 2 + int(r % 16 != 0) + 2 * n_groups + 2 + int(masked)
     torch.cuda.synchronize()
-    with torch.cuda.stream(stream):
+    with torch.cuda.stream(cx.stream):
         if masked:  # every copy's keep bits exist before its first step
             for c in range(len(copies)):
-                lora.dropout_keep_bits(seed_of(c), inp.p_drop, copies[c]["bits"], di)
-        step(0)  # first call sets kernel attributes outside any capture
+                lora.dropout_keep_bits(mask_seed, inp.p_drop, copies[c]["bits"], di)
+        step(0)  # the first call sets kernel attributes outside any capture
     torch.cuda.synchronize()
     graphs, ggraphs, bgraphs = [], [], []
     for c, cp in enumerate(copies):
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
+        with torch.cuda.graph(g, stream=cx.stream):
             step(c)
         graphs.append(g)
-        g2 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g2, stream=stream):
-            lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
-        ggraphs.append(g2)
-        g3 = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g3, stream=stream):
-            lora.base_gemm(cp["X"], cp["W"], cp["Y"])
-        bgraphs.append(g3)
+        if not a.no_layer:
+            g2 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g2, stream=cx.stream):
+                lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
+            ggraphs.append(g2)
+            g3 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g3, stream=cx.stream):
+                lora.base_gemm(cp["X"], cp["W"], cp["Y"])
+            bgraphs.append(g3)
     torch.cuda.synchronize()
     assert lora.device_status() == 0
 
-    def timed(gs, K, sampler_index=None):
-        for i in range(a.warmup):
+    def replay(gs, exchange=False):
+        def f(i):
             gs[i % len(gs)].replay()
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
-        e0 = torch.cuda.Event(enable_timing=True)
-        e1 = torch.cuda.Event(enable_timing=True)
-        with torch.cuda.stream(stream):
-            e0.record(stream)
-            for i in range(K):
-                gs[i % len(gs)].replay()
-            e1.record(stream)
-        torch.cuda.synchronize()
-        if world > 1:
-            dist.barrier()
-        return max_over_ranks(e0.elapsed_time(e1), world, dev)
+            if exchange:  # the data-parallel gradient exchange, on the replay stream
+                allreduce_grads(copies[i % len(gs)]["grad"], world)
+        return f
 
-    K = a.steps
-    with ClockSampler(local_rank) as clk:
-        ms_total = timed(graphs, K)
+    with ClockSampler(cx.local_rank) as clk:
+        ms_total, n_regions = cx.timed(replay(graphs, finetune and world > 1), K, repeats=not a.once)
     clocks = clk.summary()
-    if a.no_layer:
-        value = job_throughput(T, K, world, ms_total)
-        if rank == 0:
-            print(json.dumps({"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-                              "warmup": a.warmup, "ms_per_step": ms_total / K, "note": "--no-layer run"}))
-        del graphs, ggraphs, bgraphs
-        plan.destroy()
-        if world > 1:
-            dist.barrier()
-            dist.destroy_process_group()
-        return
-    ms_gemm = timed(ggraphs, K)
-    ms_base = timed(bgraphs, K)
-    assert lora.device_status() == 0
-
-    # torch.matmul base for the overhead reference (cuBLAS, same shape and rotation)
-    with torch.cuda.stream(stream):
-        torch.matmul(copies[0]["X"], copies[0]["W"], out=copies[0]["Y"])  # create the cuBLAS handle outside capture
-    torch.cuda.synchronize()
-    tgraphs = []
-    for cp in copies:
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            torch.matmul(cp["X"], cp["W"], out=cp["Y"])
-        tgraphs.append(g)
-    ms_torch = timed(tgraphs, K)
-
     value = job_throughput(T, K, world, ms_total)
+    entry = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
+             "warmup": a.warmup, "ms_per_step": ms_total / K, "higher_is_better": True, "scaling": "weak",
+             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+             "config": config_record(name, inp, world),
+             "timing": (f"CUDA-graph replays, CUDA events on the replay stream; median of {n_regions} regions of "
+                        f"exactly {K} steps, max over ranks"),
+             "gpu_launches": launches_per_step * K,
+             "clocks": clocks}
+
     hbm, tc_burst, tc_sust, src = peaks()
     gb, gf, lb, lf = algorithmic(inp, info)
-    t_gemm = ms_gemm * 1e-3 / K
-    if a.config in ("decode", "tiny"):
-        achieved = gb / t_gemm / 1e9
-        roof = {"bound": "hbm", "achieved": achieved, "peak": hbm, "unit": "GB/s", "frac": achieved / hbm,
-                "peak_kind": f"{src} hbm_gbs (burst copy)"}
+    t_step = ms_total * 1e-3 / K
+    if finetune:
+        bb, bfl = algorithmic_bwd(inp, r)
+        lb, lf = lb + bb, lf + bfl
+    if name in ("decode", "tiny"):
+        ach = lb / t_step / 1e9
+        entry["layer_roofline"] = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                                   "peak_kind": f"{src} hbm_gbs (copy)", "algorithmic_per_step": lb,
+                                   "what": "the whole step (all launches) against the layer's algorithmic bytes"}
     else:
-        achieved = gf / t_gemm / 1e12
-        roof = {"bound": "tensor", "achieved": achieved, "peak": tc_burst, "unit": "TFLOP/s",
-                "frac": achieved / tc_burst, "peak_kind": f"{src} bf16_tflops (burst)"}
-    roof.update({"traffic": recorded_traffic(a.config), "kernel": "lora_gemm_kernel (fused base + adapter GEMM)",
-                 "algorithmic_per_launch": gb if roof["bound"] == "hbm" else gf,
-                 "avg_launch_us": t_gemm * 1e6})
+        ach = lf / t_step / 1e12
+        entry["layer_roofline"] = {"bound": "tensor", "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",
+                                   "frac": ach / tc_burst, "frac_of_sustained": ach / tc_sust if tc_sust else None,
+                                   "peak_kind": f"{src} bf16_tflops (burst); sustained {tc_sust}",
+                                   "algorithmic_per_step": lf,
+                                   "what": "the whole step (all launches) against the layer's algorithmic flops"}
 
-    out = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
-           "warmup": a.warmup, "ms_per_step": ms_total / K, "higher_is_better": True, "scaling": "weak",
-           "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-           "config": {"workload": WORKLOAD_TEXT[a.config], "tokens_per_rank": T,
-                      "l2": f"inputs rotate over {n_copies} copies ({n_copies * per_copy / 2**20:.0f} MiB > 126 MiB L2)",
-                      "timing": "CUDA-graph replays, CUDA events on the replay stream, max over ranks",
-                      "parallelism": f"dp{world} (independent batches)",
-                      "plan": "built once per batch outside the timed region (reused by every layer)"},
-           "roofline": roof,
-           "gpu_launches": launches_per_step * K,
-           "clocks": clocks,
-           "layer": {"fused_gemm_us": t_gemm * 1e6, "base_gemm_us": ms_base * 1e3 / K,
-                     "torch_matmul_us": ms_torch * 1e3 / K, "step_us": ms_total * 1e3 / K,
-                     "overhead_vs_base": (ms_total / min(ms_base, ms_torch)) - 1.0 if not finetune else None,
-                     "layer_alg_bytes": lb, "layer_alg_flops": lf,
-                     "segments": info["n_segments"], "aug_k_total": info["aug_k_total"]}}
+    ms_torch = None
+    if not a.no_layer:
+        ms_gemm, _ = cx.timed(replay(ggraphs), K, repeats=not a.once)
+        ms_base, _ = cx.timed(replay(bgraphs), K, repeats=not a.once)
+        assert lora.device_status() == 0
+        # torch.matmul base for the overhead reference (cuBLAS, same shape and rotation)
+        with torch.cuda.stream(cx.stream):
+            torch.matmul(copies[0]["X"], copies[0]["W"], out=copies[0]["Y"])  # cuBLAS handle outside capture
+        torch.cuda.synchronize()
+        tgraphs = []
+        for cp in copies:
+            g = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g, stream=cx.stream):
+                torch.matmul(cp["X"], cp["W"], out=cp["Y"])
+            tgraphs.append(g)
+        ms_torch, _ = cx.timed(replay(tgraphs), K, repeats=not a.once)
+        t_gemm = ms_gemm * 1e-3 / K
+        if name in ("decode", "tiny"):
+            ach = gb / t_gemm / 1e9
+            roof = {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                    "peak_kind": f"{src} hbm_gbs (burst copy)"}
+        else:
+            ach = gf / t_gemm / 1e12
+            roof = {"bound": "tensor", "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s", "frac": ach / tc_burst,
+                    "peak_kind": f"{src} bf16_tflops (burst)"}
+        roof.update({"traffic": recorded_traffic(name), "kernel": "lora_gemm_kernel (fused base + adapter GEMM)",
+                     "algorithmic_per_launch": gb if roof["bound"] == "hbm" else gf,
+                     "avg_launch_us": t_gemm * 1e6,
+                     "layer_frac": entry["layer_roofline"]["frac"]})
+        entry["roofline"] = roof
+        base_fwd = min(ms_base, ms_torch) * 1e-3 / K
+        entry["layer"] = {"fused_gemm_us": t_gemm * 1e6, "base_gemm_us": ms_base * 1e3 / K,
+                          "torch_matmul_us": ms_torch * 1e3 / K, "step_us": t_step * 1e6,
+                          "overhead_vs_base": None if finetune else t_step / base_fwd - 1.0,
+                          "gemm_overhead_vs_own_base": ms_gemm / ms_base - 1.0,
+                          "layer_alg_bytes": lb, "layer_alg_flops": lf,
+                          "segments": info["n_segments"], "aug_k_total": info["aug_k_total"]}
+        del ggraphs, bgraphs, tgraphs
 
     # ---- end to end through the public API with host buffers
     if not a.no_e2e:
-        pin_X = torch.from_numpy(inp.X.view(np.int16)).view(torch.bfloat16).pin_memory()
-        pin_Y = torch.empty(T, do, dtype=torch.bfloat16).pin_memory()
-        cp = copies[0]
-        h2d = pin_X.numel() * 2 + inp.ids.nbytes
-        d2h = pin_Y.numel() * 2
-        extra = {}
-        if finetune:
-            pin_dY = torch.from_numpy(inp.dY.view(np.int16)).view(torch.bfloat16).pin_memory()
-            pin_dX = torch.empty(T, di, dtype=torch.bfloat16).pin_memory()
-            h2d += pin_dY.numel() * 2
-            d2h += pin_dX.numel() * 2
-        Ke = max(3, min(K, 200 if not finetune else 20))
-
-        # Steps run as a pipeline over two slots (device buffers, plan, pinned
-        # results): step i copies its inputs in on one stream, computes on a
-        # second and copies its results out on a third, so the copies of one step
-        # overlap the compute of its neighbours. Each step still builds its plan
-        # from the host ids and moves all of its own inputs and results.
-        s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
-        slots = copies[:2]
-        plans = [lora.Plan(inp.ids, inp.ranks, di, do, stream=s_in) for _ in range(2)]
-        pin_Ys = [pin_Y, torch.empty(T, do, dtype=torch.bfloat16).pin_memory()]
-        pin_dXs = [pin_dX, torch.empty(T, di, dtype=torch.bfloat16).pin_memory()] if finetune else None
-        ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "comp", "out")}
-
-        def e2e_step(i):
-            s = i % 2
-            c, p = slots[s], plans[s]
-            if i >= 2:
-                s_in.wait_event(ev["comp"][s])  # step i - 2 is done with this slot's inputs and plan
-            p.rebuild(inp.ids, stream=s_in)  # the batch's plan from its host ids (buffers reused)
-            with torch.cuda.stream(s_in):
-                c["X"].copy_(pin_X, non_blocking=True)
-                if finetune:
-                    c["dY"].copy_(pin_dY, non_blocking=True)
-                ev["in"][s].record(s_in)
-            s_comp.wait_event(ev["in"][s])
-            if i >= 2:
-                s_comp.wait_event(ev["out"][s])  # step i - 2's results have left this slot
-            with torch.cuda.stream(s_comp):
-                bits = None
-                if finetune and inp.p_drop > 0:
-                    bits = c["bits"]
-                    lora.dropout_keep_bits(inp.mask_seed, inp.p_drop, bits, di, stream=s_comp)
-                lora.linear_fwd(p, c["X"], c["W"], c["A"], c["B"], scale, c["Y"], p_drop=inp.p_drop,
-                                seed=inp.mask_seed, U_save=c["U"], keep_bits=bits)
-                if finetune:
-                    lora.linear_bwd(c["X"], c["W"], c["A"], c["B"], float(inp.scale[0]), c["U"], c["dY"],
-                                    c["dX"], c["dA"], c["dB"], c["ws"], p_drop=inp.p_drop, seed=inp.mask_seed,
-                                    keep_bits=bits)
-                ev["comp"][s].record(s_comp)
-            s_out.wait_event(ev["comp"][s])
-            with torch.cuda.stream(s_out):
-                pin_Ys[s].copy_(c["Y"], non_blocking=True)
-                if finetune:
-                    pin_dXs[s].copy_(c["dX"], non_blocking=True)
-                ev["out"][s].record(s_out)
-
-        def drain():
-            for st in (s_in, s_comp, s_out):
-                st.synchronize()
-
-        for i in range(2):
-            e2e_step(i)
-        drain()
-        if world > 1:
-            dist.barrier()
-        t0 = time.perf_counter()
-        for i in range(Ke):
-            e2e_step(2 + i)
-        drain()
-        dt = time.perf_counter() - t0
-        for p in plans:
-            p.destroy()
-        dt = max_over_ranks(dt, world, dev)
-        out["e2e"] = {"value": job_throughput(T, Ke, world, dt * 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
-                      "d2h_bytes_per_step": int(d2h), "steps": Ke,
-                      "what": "per step: plan from host ids + H2D of X (pinned) + forward" + (" + backward" if finetune else "")
-                              + " + D2H of the result; steps pipelined over two slots (copy-in, compute and"
-                              " copy-out streams); host wall clock over the steps"}
+        entry["e2e"] = measure_e2e(cx, inp, copies, scale, mask_seed, K)
 
     # ---- CPU baseline: the oracle on a bounded sample (rank 0, N=1 only)
     if rank == 0 and world == 1 and not a.no_cpu_baseline:
         import oracle
         oracle.build()
-        n, dt, sample = oracle_sample(inp, 15.0)
-        out["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
-                               "kind": "oracle", "sample": sample}
+        n, dt, sample = oracle_sample(inp, cpu_budget)
+        entry["cpu_baseline"] = {"value": n / dt, "unit": "tokens/s", "cores": oracle.num_threads(),
+                                 "kind": "oracle", "sample": sample}
 
     for cp in copies:
         cp.clear()
-    del graphs, ggraphs, bgraphs, tgraphs
+    del graphs
     plan.destroy()
-    if rank == 0:
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
+def measure_e2e(cx, inp, copies, scale, mask_seed, K):
+    """The metric through the public API with host buffers (see the module text)."""
+    import torch
+    import lora_adapter_execution_b200 as lora
+    dev, world = cx.dev, cx.world
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    finetune = inp.dY is not None
+    pin_X = torch.from_numpy(inp.X.view(np.int16)).view(torch.bfloat16).pin_memory()
+    h2d = pin_X.numel() * 2 + inp.ids.nbytes
+    d2h = T * do * 2
+    if finetune:
+        pin_dY = torch.from_numpy(inp.dY.view(np.int16)).view(torch.bfloat16).pin_memory()
+        h2d += pin_dY.numel() * 2
+        d2h += T * di * 2
+    Ke = max(3, min(K, 200 if not finetune else 20))
+
+    # Steps run as a pipeline over two slots (device buffers, plan, pinned
+    # results): step i copies its inputs in on one stream, computes on a second
+    # and copies its results out on a third, so the copies of one step overlap
+    # the compute of its neighbours. Each step still builds its plan from the
+    # host ids and moves all of its own inputs and results.
+    s_in, s_comp, s_out = (torch.cuda.Stream(device=dev) for _ in range(3))
+    slots = copies[:2]
+    plans = [lora.Plan(inp.ids, inp.ranks, di, do, stream=s_in) for _ in range(2)]
+    pin_Ys = [torch.empty(T, do, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+    pin_dXs = [torch.empty(T, di, dtype=torch.bfloat16).pin_memory() for _ in range(2)] if finetune else None
+    ev = {k: [torch.cuda.Event(), torch.cuda.Event()] for k in ("in", "comp", "out")}
+
+    def e2e_step(i):
+        s = i % 2
+        c, p = slots[s], plans[s]
+        if i >= 2:
+            s_in.wait_event(ev["comp"][s])  # step i - 2 is done with this slot's inputs and plan
+        p.rebuild(inp.ids, stream=s_in)  # the batch's plan from its host ids (buffers reused)
+        with torch.cuda.stream(s_in):
+            c["X"].copy_(pin_X, non_blocking=True)
+            if finetune:
+                c["dY"].copy_(pin_dY, non_blocking=True)
+            ev["in"][s].record(s_in)
+        s_comp.wait_event(ev["in"][s])
+        if i >= 2:
+            s_comp.wait_event(ev["out"][s])  # step i - 2's results have left this slot
+        with torch.cuda.stream(s_comp):
+            bits = None
+            if finetune and inp.p_drop > 0:
+                bits = c["bits"]
+                lora.dropout_keep_bits(mask_seed, inp.p_drop, bits, di, stream=s_comp)
+            lora.linear_fwd(p, c["X"], c["W"], c["A"], c["B"], scale, c["Y"], p_drop=inp.p_drop,
+                            seed=mask_seed, U_save=c["U"], keep_bits=bits)
+            if finetune:
+                lora.linear_bwd(c["X"], c["W"], c["A"], c["B"], float(inp.scale[0]), c["U"], c["dY"],
+                                c["dX"], c["dA"], c["dB"], c["ws"], p_drop=inp.p_drop, seed=mask_seed,
+                                keep_bits=bits)
+                allreduce_grads(c["grad"], world)
+            ev["comp"][s].record(s_comp)
+        s_out.wait_event(ev["comp"][s])
+        with torch.cuda.stream(s_out):
+            pin_Ys[s].copy_(c["Y"], non_blocking=True)
+            if finetune:
+                pin_dXs[s].copy_(c["dX"], non_blocking=True)
+            ev["out"][s].record(s_out)
+
+    def drain():
+        for st in (s_in, s_comp, s_out):
+            st.synchronize()
+
+    for i in range(2):
+        e2e_step(i)
+    drain()
+    cx.barrier()
+    t0 = time.perf_counter()
+    for i in range(Ke):
+        e2e_step(2 + i)
+    drain()
+    dt = time.perf_counter() - t0
+    for p in plans:
+        p.destroy()
+    dt = max_over_ranks(dt, world, dev)
+    return {"value": job_throughput(T, Ke, world, dt * 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": Ke,
+            "what": "per step: plan from host ids + H2D of X (pinned)" + (" and dY" if finetune else "")
+                    + " + forward" + (" + backward + gradient all-reduce" if finetune else "")
+                    + " + D2H of the result; steps pipelined over two slots (copy-in, compute and"
+                    " copy-out streams); host wall clock over the steps"}
+
+
+HEAD_KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
+             "vs_baseline", "dtype", "data", "config", "timing", "roofline", "layer_roofline", "gpu_launches",
+             "clocks", "layer", "e2e", "cpu_baseline")
+
+
+def run_lora(a):
+    cx = Ctx(a)
+    names = list(ORDER) if a.config == "all" else [a.config]
+    entries = {}
+    for name in names:
+        budget = CPU_BUDGET_S["headline" if name in (HEADLINE, a.config) else "other"]
+        entries[name] = measure(name, cx, budget)
+    head = entries[HEADLINE if a.config == "all" else a.config]
+    out = {k: head[k] for k in HEAD_KEYS if k in head}
+    if a.config == "all":
+        out["headline"] = f"{HEADLINE} (the largest single-GPU configuration); every workload under configs"
+        out["configs"] = entries
+    if cx.rank == 0:
         print(json.dumps(out), flush=True)
+    if cx.world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+# ----------------------------------------------------------------------------- launchers
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def torchrun_command(argv, n):
+    """The command that runs this script with n processes (one per GPU) under
+    torchrun on this node, with the same arguments."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1", f"--nproc-per-node={n}",
+            "--master-addr", "127.0.0.1", "--master-port", str(_free_port()), os.path.abspath(__file__), *argv]
+
+
+def run_dry(a):
+    """No GPU: each rank joins a gloo group, takes one data-parallel gradient
+    exchange and the max over ranks of a time, and rank 0 prints a line."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    rank, _, world = dist_env()
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+    g = torch.full((4,), float(rank + 1), dtype=torch.float32)
+    allreduce_grads(g, world)
+    ms = max_over_ranks(1.0 + rank, world)
+    if rank == 0:
+        print(json.dumps({"dry_run": True, "n_gpus": world, "grad_sum": float(g[0]), "max_ms": ms}), flush=True)
     if world > 1:
         dist.barrier()
         dist.destroy_process_group()
 
 
-def main():
-    a = parse()
+def main(argv=None):
+    argv = sys.argv[1:] if argv is None else argv
+    a = parse(argv)
     rank, _, world = dist_env()
+    if a.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        # one process per GPU: start N ranks of this script under torchrun
+        r = subprocess.run(torchrun_command(argv, a.gpus))
+        sys.exit(r.returncode)
     if a.gpus != world and rank == 0:
-        # one process per GPU: N GPUs need N processes (torchrun); the line
-        # reports the processes that ran
-        print(f"bench.py: --gpus {a.gpus} but {world} process(es) (WORLD_SIZE); "
-              f"launch N > 1 with torchrun --nproc-per-node N", file=sys.stderr)
-    if a.impl == "reference":
+        print(f"bench.py: --gpus {a.gpus} but {world} process(es) (WORLD_SIZE); the line reports the processes "
+              f"that ran", file=sys.stderr)
+    if a.dry_run:
+        run_dry(a)
+    elif a.impl == "reference":
         run_reference(a)
     else:
         run_lora(a)

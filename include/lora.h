@@ -133,6 +133,7 @@ int lora_plan_build_host(const int32_t *ids_host, int64_t T, const int32_t *rank
  *   seg_host    int32[n_seg*3] or NULL: (adapter, start, length) per segment, ascending
  *               adapter id, start = first sorted position; adapters without tokens have none
  *   n_seg       int32* or NULL: number of segments
+ * No counterpart in the pages (inspection of this library's plan).
  * Errors: LORA_ERR_ARG (null plan). */
 int lora_plan_get(lora_plan_t plan, int32_t *perm_host, int32_t *seg_host, int32_t *n_seg);
 
@@ -151,11 +152,13 @@ typedef struct lora_plan_info {
                                tokens): one more kernel launch per forward */
 } lora_plan_info_t;
 
-/* Errors: LORA_ERR_ARG. */
+/* The plan's sizes. No counterpart in the pages (inspection of this library's
+ * plan). Errors: LORA_ERR_ARG. */
 int lora_plan_info(lora_plan_t plan, lora_plan_info_t *info);
 
 /* Free the plan (waits for nothing; the caller must not free a plan that queued
- * work still uses). NULL is ignored. */
+ * work still uses). NULL is ignored. No counterpart in the pages (the plan's
+ * lifetime is this library's design). */
 void lora_plan_destroy(lora_plan_t plan);
 
 /* ------------------------------------------------------------------------
@@ -190,6 +193,14 @@ void lora_plan_destroy(lora_plan_t plan);
  *   stream  launch stream
  * The plan's scratch holds s_a·U rounded to bf16 between the two kernels, so
  * two forwards with one plan must not run concurrently.
+ * Adapter isolation: a token's output reads only its own adapter's factor rows
+ * and the factor rows of adapters whose tokens share its 128-token tile of the
+ * sorted order (the tile's adapter K slices form one block-diagonal
+ * contraction, where other adapters' rows meet zeros). Factor rows of adapters
+ * with no token in that tile never enter it, even where a rank is not a
+ * multiple of 16 (the rows past it are zeroed on chip). Non-finite values in
+ * an adapter's B rows therefore reach, as NaN, only tokens of tiles that adapter
+ * shares.
  * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA.
  * ------------------------------------------------------------------------ */
 int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
@@ -239,11 +250,13 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
  *
  *   X, W, A (bf16 [r, d_in], rows = columns of A), B (bf16 [r, d_out]),
  *   scale, p_drop, seed    as in the forward (same mask)
- *   U_save  f32 [T, r]     the forward's U_save
+ *   r       the adapter's rank, 1 .. LORA_MAX_RANK
+ *   U_save  f32 [T, r]     the forward's U_save (16-byte aligned when r % 16 == 0,
+ *                          else 4-byte aligned)
  *   dY      bf16 [T, d_out]
  *   dX      bf16 [T, d_in]  output
- *   dA      f32 [r, d_in]   output
- *   dB      f32 [r, d_out]  output
+ *   dA      f32 [r, d_in]   output (4-byte aligned)
+ *   dB      f32 [r, d_out]  output (4-byte aligned)
  *   workspace, workspace_bytes  device scratch of at least
  *           lora_linear_bwd_workspace_size(T, d_in, d_out, r) bytes, 256-byte
  *           aligned, owned by the caller; contents on entry are ignored.
@@ -316,6 +329,17 @@ int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uin
 int lora_dropout_keep_bits(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint32_t *bits_dev,
                            lora_stream_t stream);
 
+/* The seed that gives rows t0 .. t0+T-1 of a [T_global, d_in] input the dropout
+ * mask they have in the global input under `seed`: a data-parallel rank whose
+ * batch is those rows of a global batch passes it to lora_linear_fwd,
+ * lora_linear_bwd and lora_dropout_keep_bits and indexes its rows from 0. The
+ * mask's generator state for element index n is seed + (n + 1)·g (g the
+ * generator's increment, arithmetic mod 2^64), so shifting n by t0·d_in is
+ * adding t0·d_in·g to the seed. Host only (no CUDA call); t0 >= 0, d_in >= 1,
+ * else returns `seed` unchanged. No counterpart in the pages (the pages fix no
+ * generator and no sharding). */
+uint64_t lora_dropout_seed_for_rows(uint64_t seed, int64_t t0, int64_t d_in);
+
 /* Test hook for failure detection: launch one thread that waits on an mbarrier
  * nothing will complete, with a wait limit of `limit_us` microseconds (1 ..
  * 10^6). The wait runs out, sets LORA_DEV_TIMEOUT in the status word and the
@@ -326,12 +350,13 @@ int lora_dropout_keep_bits(uint64_t seed, double p_drop, int64_t T, int64_t d_in
 int lora_selftest_bounded_wait(uint32_t limit_us, int *waited_ok_dev, lora_stream_t stream);
 
 /* Synchronise `stream`, then read and clear the current device's status word.
+ * No counterpart in the pages (this library's failure reporting).
  *   status_host  receives the LORA_DEV_* bits (0 if all kernels ran cleanly); may be NULL
  * Returns LORA_OK if the word was 0, LORA_ERR_DEVICE if any bit was set,
  * LORA_ERR_CUDA if the synchronisation failed. */
 int lora_device_status(lora_stream_t stream, uint32_t *status_host);
 
-/* Static string for a status code (never NULL). */
+/* Static string for a status code (never NULL). No counterpart in the pages. */
 const char *lora_status_string(int code);
 
 #ifdef __cplusplus

@@ -83,6 +83,7 @@ def load_library():
         "lora_dropout_keep_bits": (ctypes.c_int, [_u64, _dbl, _i64, _i64, _vp, _vp]),
         "lora_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
         "lora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _vp, _vp]),
+        "lora_dropout_seed_for_rows": (_u64, [_u64, _i64, _i64]),
         "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -327,6 +328,12 @@ def dropout_keep_bits(seed: int, p_drop: float, bits, d_in: int, *, stream=None)
     _args("lora_dropout_keep_bits", ("bits", bits, (T, -(-d_in // 32)), _I32, False))
     _check(load_library().lora_dropout_keep_bits(int(seed) & (2**64 - 1), float(p_drop), T, d_in, _ptr(bits),
                                                  _stream(stream)), "lora_dropout_keep_bits")
+
+
+def dropout_seed_for_rows(seed: int, t0: int, d_in: int) -> int:
+    """lora_dropout_seed_for_rows: the seed that gives local rows 0.. the dropout
+    mask of global rows t0.. (host only)."""
+    return int(load_library().lora_dropout_seed_for_rows(int(seed) & (2**64 - 1), int(t0), int(d_in)))
 
 
 def device_status(stream=None) -> int:

@@ -253,8 +253,8 @@ __host__ __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t
 // x ^= x >> 27, x *= 0x94D049BB133111EB, x ^= x >> 31. Element (t, col) of the
 // LoRA-branch input is dropped when output t * d_in + col is below thr = p * 2^64.
 //
-// keep_state: the output of state z (the state after its increment) >= thr (the state after its increment) >= thr, i.e. the
-// element is kept. The comparison needs only the high word of the output unless
+// keep_state: whether the output of state z (the state after its increment) is
+// >= thr, i.e. the element is kept. The comparison needs only the high word of the output unless
 // it ties with the high word of thr (a 2^-32 event): the last product's low word
 // and the last shift's low half are formed only then.
 __device__ __forceinline__ bool keep_state(uint64_t z, uint64_t thr) {

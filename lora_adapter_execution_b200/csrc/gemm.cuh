@@ -2,11 +2,12 @@
 //
 //   Y_tile = X_tile · W_tile + Ũ_tile · B_tile
 //
-// The adapter term is an augmented-K contraction [X | s·U]·[W ; B_a]: after the
-// d_in-long base K loop, the same TMEM accumulator receives the tile's adapter
-// K slices (one per adapter present in the tile, each r_a rounded up to 16),
-// so the expand and the add happen in-tile and no intermediate Y goes back to
-// HBM. This is the "split at the GEMM boundary, consume the intermediate in
+// The adapter term is an augmented-K contraction [X | s·U]·[W ; B_a]: the same
+// TMEM accumulator receives the tile's adapter K slices (one per adapter present
+// in the tile, each 2·r_a rounded up to 16: the hi and lo bf16 parts of s·U),
+// issued before the d_in-long base K loop so that their scattered B_pool loads
+// overlap it, so the expand and the add happen in-tile and no intermediate Y
+// goes back to HBM. This is the "split at the GEMM boundary, consume the intermediate in
 // place" point of the kernel-layer section (Kernel 层：图分裂融合) of
 // "LoRAFusion：消除冗余内存访问的多 LoRA 高效微调系统", applied to the
 // multi-adapter batch of the batching section (批处理) of "S-LoRA：一个GPU运行
@@ -72,9 +73,10 @@ struct GemmParams {
                         // A tensor map), as written by the shrink; 0: tiles are consecutive originals
   __nv_bfloat16 *out;   // [T, N]
   // backward epilogue: out += keep(t, col) / (1 - p) * sum_k dU[t, k] * A[k, col]
-  const float *dU;      // [T, r]
+  const float *dU;      // [T, du_stride] (ranks past r are zero)
   const uint16_t *A;    // [r, N]
   int32_t r;
+  int32_t du_stride;
   uint64_t seed, thr;
   float inv_keep;
   const uint32_t *keep_bits;  // precomputed keep bits (null: hash), word t * wpr + col / 32
@@ -248,6 +250,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // per stage: the B slot each K step of an adapter block reads (2 bits per step)
   volatile uint32_t *bmap = tmem_slot + 2;
   const uint32_t recv_bar = full0 + 128;  // split-K: the other ranks' partials have landed
+  // per stage: the adapter block's slot count and each slot's rows that belong to
+  // its adapter (AugBlockDesc::valid | nslot << 20), for the MMA warp
+  volatile uint32_t *bvalid = reinterpret_cast<volatile uint32_t *>(bars) + 34;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -318,10 +323,11 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // blocks come first: block i < naug is adapter block q + i * S)
         const int na = br.naug();
         int4 nprow = make_int4(0, 0, 0, 0);
-        int ninfo = 0;
+        int ninfo = 0, nvalid = 0;
         if (na > 0) {
           nprow = __ldg(reinterpret_cast<const int4 *>(p.augblocks + td.aug0 + q));
           ninfo = __ldg(&p.augblocks[td.aug0 + q].info);
+          nvalid = __ldg(&p.augblocks[td.aug0 + q].valid);
         }
         for (int i = 0; i < nblk; ++i) {
           const int blk = br.block(i, KB);
@@ -345,11 +351,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const int prow_s[4] = {nprow.x, nprow.y, nprow.z, nprow.w};
             const int nslot = ninfo & 15;
             const uint32_t map = static_cast<uint32_t>(ninfo >> 4) & 0xFFu;
+            bvalid[stage] = static_cast<uint32_t>(nvalid) | (static_cast<uint32_t>(nslot) << 20);
             if (i + 1 < na) {
               nprow = __ldg(reinterpret_cast<const int4 *>(p.augblocks + td.aug0 + lb + S));
               ninfo = __ldg(&p.augblocks[td.aug0 + lb + S].info);
+              nvalid = __ldg(&p.augblocks[td.aug0 + lb + S].valid);
             }
-            bmap[stage] = map;  // published to the MMA thread by the release arrive below
+            bmap[stage] = map;  // published to the MMA warp by the release arrive below
             mbar_arrive_expect_tx(fb, kStageA + nslot * kBSlot);
             bulk_g2s(a_dst, p.uimg + td.uofs + static_cast<int64_t>(lb) * kAugBlockBytes, kAugBlockBytes,
                      fb);
@@ -410,66 +418,106 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     }
     __syncwarp();
   } else if (warp == 1) {
-    if (lane == 0) {
-      // ------------------------------------------------------------ MMA issuer
-      constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false, !B_KMAJOR);
-      // stage 0's descriptors: A K-major (SW128, 8-row groups 1 KB apart, a K16
-      // step 32 bytes on); B K-major likewise, or MN-major with 64-column blocks
-      // 8 KB apart and a K16 step 16 rows (2 KB) on
-      const uint64_t adesc0 = sdesc_sw128(stage0, 16, 1024);
-      const uint64_t bdesc0 = B_KMAJOR ? sdesc_sw128(stage0 + kStageA, 16, 1024)
-                                       : sdesc_sw128(stage0 + kStageA, 8192, 1024);
-      constexpr uint64_t kAStep = 32 >> 4;
-      constexpr uint64_t kBStep = B_KMAJOR ? (32 >> 4) : (2048 >> 4);
-      int stage = 0;
-      uint32_t phase = 0;
-      int acc = 0;
-      uint32_t aphase = 0;
-      int tile;
-      for (int k = 0; !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
-        int mt, nt;
-        tile_coords(tile, p, mt, nt);
-        const int kaug = has_plan ? p.tiles[mt].kaug : 0;
-        const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
-        const int nblk = br.count();
-        if (!mbar_wait(acce0 + 8 * acc, aphase ^ 1)) { *abort_flag = 1; break; }
+    // -------------------------------------------------------------- MMA warp
+    // Lane 0 issues every MMA. The whole warp waits on each stage so that, for an
+    // adapter block whose 16-row B slices run past the adapter's rank (the rows
+    // after it are the next adapter's), all 32 lanes can zero those rows in
+    // shared memory before the MMA reads them: a token then never multiplies
+    // factor values of an adapter that is absent from its tile.
+    constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false, !B_KMAJOR);
+    // stage 0's descriptors: A K-major (SW128, 8-row groups 1 KB apart, a K16
+    // step 32 bytes on); B K-major likewise, or MN-major with 64-column blocks
+    // 8 KB apart and a K16 step 16 rows (2 KB) on
+    const uint64_t adesc0 = sdesc_sw128(stage0, 16, 1024);
+    const uint64_t bdesc0 = B_KMAJOR ? sdesc_sw128(stage0 + kStageA, 16, 1024)
+                                     : sdesc_sw128(stage0 + kStageA, 8192, 1024);
+    constexpr uint64_t kAStep = 32 >> 4;
+    constexpr uint64_t kBStep = B_KMAJOR ? (32 >> 4) : (2048 >> 4);
+    int stage = 0;
+    uint32_t phase = 0;
+    int acc = 0;
+    uint32_t aphase = 0;
+    int tile;
+    for (int k = 0;; ++k) {
+      // lane 0's reading of the abort flag decides for the whole warp
+      const bool go = !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile);
+      if (!__shfl_sync(0xFFFFFFFFu, go ? 1 : 0, 0)) break;
+      int mt, nt;
+      tile_coords(tile, p, mt, nt);
+      const int kaug = has_plan ? p.tiles[mt].kaug : 0;
+      const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
+      const int nblk = br.count();
+      bool okw = true;
+      if (lane == 0) okw = mbar_wait(acce0 + 8 * acc, aphase ^ 1);
+      if (!__shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0)) {
+        if (lane == 0) *abort_flag = 1;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t d_tmem = tmem_base + acc * kBN;
+      bool ok = true;
+      for (int i = 0; i < nblk; ++i) {
+        const int blk = br.block(i, KB);
+        if (!__all_sync(0xFFFFFFFFu, mbar_wait(full0 + 8 * stage, phase))) {
+          if (lane == 0) *abort_flag = 1;
+          ok = false;
+          break;
+        }
         tc_fence_after();
-        const uint32_t d_tmem = tmem_base + acc * kBN;
-        bool ok = true;
-        for (int i = 0; i < nblk; ++i) {
-          const int blk = br.block(i, KB);
-          if (!mbar_wait(full0 + 8 * stage, phase)) { *abort_flag = 1; ok = false; break; }
-          tc_fence_after();
-          // One thread issues every MMA, so its instruction count per K block
-          // bounds the tensor pipe: the descriptors of a stage are the stage's
-          // base descriptors plus constants (address field in 16-byte units).
-          const uint64_t ad = adesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
-          const uint64_t bd = bdesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
-          if (blk < KB) {
+        // One thread issues every MMA, so its instruction count per K block
+        // bounds the tensor pipe: the descriptors of a stage are the stage's
+        // base descriptors plus constants (address field in 16-byte units).
+        const uint64_t ad = adesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
+        const uint64_t bd = bdesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
+        if (blk < KB) {
+          if (lane == 0) {
             umma_bf16(d_tmem, ad, bd, kIdesc, i > 0 ? 1u : 0u);
             umma_bf16_acc(d_tmem, ad + kAStep, bd + kBStep, kIdesc);
             umma_bf16_acc(d_tmem, ad + 2 * kAStep, bd + 2 * kBStep, kIdesc);
             umma_bf16_acc(d_tmem, ad + 3 * kAStep, bd + 3 * kBStep, kIdesc);
-          } else {
-            // adapter block (MN-major B slots [4 column blocks][16 rows][64 cols],
-            // column-block stride 2 KB; the slot of each K step from bmap)
-            const int steps = min(4, (kaug - (blk - KB) * kAugBlock) / 16);
-            const uint32_t map = bmap[stage];
-            const uint32_t b_s = stage0 + stage * kStageBytes + kStageA;
+          }
+        } else {
+          // adapter block (MN-major B slots [4 column blocks][16 rows][64 cols],
+          // column-block stride 2 KB; the slot of each K step from bmap)
+          const int steps = min(4, (kaug - (blk - KB) * kAugBlock) / 16);
+          const uint32_t map = bmap[stage];
+          const uint32_t b_s = stage0 + stage * kStageBytes + kStageA;
+          if (!B_KMAJOR) {
+            const uint32_t vw = bvalid[stage];
+            const int nsl = static_cast<int>(vw >> 20);
+            uint8_t *bsp = smem + stage * kStageBytes + kStageA;
+            bool zeroed = false;
+            for (int u = 0; u < nsl; ++u) {
+              const int v = static_cast<int>((vw >> (5 * u)) & 31u);
+              // rows v .. 15 of the slot in each of its 4 column blocks, as
+              // 16-byte pieces (8 per 128-byte row)
+              for (int e = lane; e < (16 - v) * 32; e += 32) {
+                const int r = v + (e >> 5);
+                const int j = (e >> 3) & 3;
+                *reinterpret_cast<uint4 *>(bsp + u * kBSlot + j * 2048 + r * 128 + (e & 7) * 16) =
+                    make_uint4(0u, 0u, 0u, 0u);
+              }
+              zeroed |= v < 16;
+            }
+            if (zeroed) fence_proxy_async_smem();  // the MMA reads through the async proxy
+            __syncwarp();
+          }
+          if (lane == 0) {
             for (int qq = 0; qq < steps; ++qq) {
               const uint64_t bq = B_KMAJOR ? bd + qq * kAStep
                                            : sdesc_sw128(b_s + ((map >> (2 * qq)) & 3u) * kBSlot, 2048, 1024);
               umma_bf16(d_tmem, ad + qq * kAStep, bq, kIdesc, (i > 0 || qq > 0) ? 1u : 0u);
             }
           }
-          umma_commit(empty0 + 8 * stage);
-          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
         }
-        if (!ok) break;
-        umma_commit(accf0 + 8 * acc);
-        if (++acc == 2) { acc = 0; aphase ^= 1; }
+        if (lane == 0) umma_commit(empty0 + 8 * stage);
+        if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
       }
+      if (!ok) break;
+      if (lane == 0) umma_commit(accf0 + 8 * acc);
+      if (++acc == 2) { acc = 0; aphase ^= 1; }
     }
+    __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue (warps 2..5)
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
@@ -524,7 +572,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       float du[kEpiRankRegs];  // backward: this row's dU, loaded once per tile (ranks <= kEpiRankRegs)
       if (EPI == kEpiBwdLora) {
 #pragma unroll
-        for (int k = 0; k < kEpiRankRegs; ++k) du[k] = (valid && k < p.r) ? p.dU[orig * p.r + k] : 0.f;
+        for (int k = 0; k < kEpiRankRegs; ++k) du[k] = (valid && k < p.r) ? p.dU[orig * p.du_stride + k] : 0.f;
       }
       for (int c = 0; c < kBN / 32; ++c) {
         uint32_t v[32];
@@ -571,7 +619,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
                 }
               }
             }
-            for (int k = kEpiRankRegs; k < p.r; ++k) add_rank(k, p.dU[orig * p.r + k]);
+            for (int k = kEpiRankRegs; k < p.r; ++k) add_rank(k, p.dU[orig * p.du_stride + k]);
             const uint32_t keep = p.keep_bits ? __ldg(p.keep_bits + orig * p.wpr + (col0 >> 5))
                                               : keep_mask32(p.seed, p.thr, static_cast<uint64_t>(orig * p.N + col0));
 #pragma unroll

@@ -33,7 +33,10 @@ struct TileDesc {
 struct AugBlockDesc {
   int32_t prow[4];  // first B_pool row of slot 0..nslot-1 (0 past nslot)
   int32_t info;     // nslot | slot of K step q at bits 4 + 2q | steps << 12
-  int32_t pad_[3];
+  int32_t valid;    // rows of slot u that belong to its adapter, 5 bits at bit 5u (1..16):
+                    // the rest of the 16-row slice is another adapter's rows and is
+                    // zeroed in shared memory before the MMA reads it
+  int32_t pad_[2];
 };
 
 // One adapter's run of rows inside one tile: its K slice of the augmented contraction.

@@ -711,7 +711,9 @@ int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T,
   return launch_fwd_gemm(ds, gp, mX128, mW, mW, stream);
 }
 
-// Workspace layout: dU f32 [T, r] | dB partial [S, r, d_out] | dA partial [S, r, d_in]
+// Workspace layout: dU f32 [T, rp] | (r % 16 != 0: U f32 [T, rp]) | dB partial
+// [S, r, d_out] | dA partial [S, r, d_in], rp = r rounded up to 16 (the token
+// contraction reads whole 16-rank groups; the padding columns are zero).
 // Token splits of the backward contractions: about two CTAs per SM of a B200
 // (148 SMs) over the wider of the two column ranges, at least 64 tokens each.
 static int64_t bwd_splits(int64_t T, int64_t d_in, int64_t d_out) {
@@ -721,11 +723,35 @@ static int64_t bwd_splits(int64_t T, int64_t d_in, int64_t d_out) {
   return std::max<int64_t>(1, std::min<int64_t>(s, 16));
 }
 
-size_t lora_linear_bwd_workspace_size(int64_t T, int64_t d_in, int64_t d_out, int32_t r) {
-  if (T <= 0 || d_in <= 0 || d_out <= 0 || r <= 0) return 0;
+namespace {
+struct BwdLayout {
+  int64_t S, rp;
+  int64_t off_dU, off_U, off_pdB, off_pdA, total;  // off_U < 0: U_save is read directly
+};
+BwdLayout bwd_layout(int64_t T, int64_t d_in, int64_t d_out, int32_t r) {
   auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
-  const int64_t S = bwd_splits(T, d_in, d_out);
-  return static_cast<size_t>(up(T * r * 4) + up(S * r * d_out * 4) + up(S * r * d_in * 4));
+  BwdLayout L{};
+  L.S = bwd_splits(T, d_in, d_out);
+  L.rp = (r + 15) / 16 * 16;
+  L.off_dU = 0;
+  int64_t o = up(T * L.rp * 4);
+  L.off_U = -1;
+  if (r % 16 != 0) {
+    L.off_U = o;
+    o += up(T * L.rp * 4);
+  }
+  L.off_pdB = o;
+  o += up(L.S * r * d_out * 4);
+  L.off_pdA = o;
+  o += up(L.S * r * d_in * 4);
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+size_t lora_linear_bwd_workspace_size(int64_t T, int64_t d_in, int64_t d_out, int32_t r) {
+  if (T <= 0 || d_in <= 0 || d_out <= 0 || r <= 0 || r > LORA_MAX_RANK) return 0;
+  return static_cast<size_t>(bwd_layout(T, d_in, d_out, r).total);
 }
 
 int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, const uint16_t *B, float scale,
@@ -736,54 +762,57 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
   if (reinterpret_cast<uintptr_t>(keep_bits) & 3u) return LORA_ERR_ARG;
   if (T <= 0 || d_in < 8 || d_out < 8 || (d_in % 8) || (d_out % 8)) return LORA_ERR_ARG;
   if (T > (int64_t)1 << 30 || d_in > (int64_t)1 << 30 || d_out > (int64_t)1 << 30) return LORA_ERR_ARG;
-  if (r < 8 || r > kTcMaxR || (r % 8)) return LORA_ERR_RANK;
+  if (r < 1 || r > LORA_MAX_RANK) return LORA_ERR_RANK;
   if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
-  if (!aligned16(X) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(U_save) ||
-      !aligned16(dY) || !aligned16(dX) || !aligned16(dA) || !aligned16(dB))
+  // U_save rows are r fp32 apart; a tensor map needs 16-byte row strides, so
+  // U_save itself is read only when r % 16 == 0 (else its padded copy)
+  if (!aligned16(X) || !aligned16(W) || !aligned16(A) || !aligned16(B) || !aligned16(dY) || !aligned16(dX) ||
+      (reinterpret_cast<uintptr_t>(U_save) & 3u) || (reinterpret_cast<uintptr_t>(dA) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dB) & 3u) || (r % 16 == 0 && !aligned16(U_save)))
     return LORA_ERR_ARG;
-  const size_t need = lora_linear_bwd_workspace_size(T, d_in, d_out, r);
-  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+  const BwdLayout Lw = bwd_layout(T, d_in, d_out, r);
+  if (!workspace || workspace_bytes < static_cast<size_t>(Lw.total) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
     return LORA_ERR_WORKSPACE;
   DeviceState *ds = nullptr;
   int rc = device_state(&ds);
   if (rc != LORA_OK) return rc;
 
-  auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
-  const int64_t S = bwd_splits(T, d_in, d_out);
+  const int64_t S = Lw.S;
+  const int rp = static_cast<int>(Lw.rp);
   uint8_t *ws = static_cast<uint8_t *>(workspace);
-  float *dU = reinterpret_cast<float *>(ws);
-  float *pdB = reinterpret_cast<float *>(ws + up(T * r * 4));
-  float *pdA = reinterpret_cast<float *>(ws + up(T * r * 4) + up(S * r * d_out * 4));
+  float *dU = reinterpret_cast<float *>(ws + Lw.off_dU);
+  float *Ug = Lw.off_U >= 0 ? reinterpret_cast<float *>(ws + Lw.off_U) : const_cast<float *>(U_save);
+  float *pdB = reinterpret_cast<float *>(ws + Lw.off_pdB);
+  float *pdA = reinterpret_cast<float *>(ws + Lw.off_pdA);
 
   const uint64_t thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
   const float inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
 
-  CUtensorMap mdY16, mB16, mdY128, mWt, mdY64, mU, mdU, mX64;
+  CUtensorMap mdY16, mB16, mdY128, mWt, mdY64, mX64;
   bool ok = true;
   ok &= make_map(&mdY16, dY, d_out, T, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mB16, B, d_out, r, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mdY128, dY, d_out, T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mWt, W, d_out, d_in, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B);
   ok &= make_map(&mdY64, dY, d_out, T, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
-  ok &= make_map_f32(&mU, U_save, r, T, r, 64);
-  ok &= make_map_f32(&mdU, dU, r, T, r, 64);
   ok &= make_map(&mX64, X, d_in, T, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return LORA_ERR_ARG;
 
-  // K3a: dU = s * dY * B^T  (fp32 and bf16 copies)
+  // K3a: dU = s * dY * B^T (fp32, rows padded to rp with zeros)
   {
     ShrinkParams sp{};
     sp.mode = 1;
     sp.T = static_cast<int32_t>(T);
     sp.K = static_cast<int32_t>(d_out);
     sp.r = r;
-    sp.npieces = (((r + 15) / 16) * 16 + kShrinkN - 1) / kShrinkN;
+    sp.npieces = (rp + kShrinkN - 1) / kShrinkN;
     sp.scale1 = scale;
     sp.x_sorted = 0;
     sp.dU = dU;
     const int n_units = static_cast<int>((T + kTileM - 1) / kTileM) * sp.npieces;
     int ks = 1;
-    const int max_nb16 = shrink_build(n_units, d_out, ds->num_sms, std::min(kShrinkN, ((r + 15) / 16) * 16), &ks);
+    const int max_nb16 = shrink_build(n_units, d_out, ds->num_sms, std::min(kShrinkN, rp), &ks);
     int64_t slice = (d_out + ks - 1) / ks;
     slice = (slice + kSkBK - 1) / kSkBK * kSkBK;
     sp.ksplit = ks;
@@ -806,6 +835,12 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
       return LORA_ERR_CUDA;
     }
   }
+  if (Lw.off_U >= 0) {
+    // U_save with its rows padded to rp columns, for the dB contraction's tensor map
+    const int64_t n = T * rp;
+    lora_pad_cols_kernel<<<static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 16 * ds->num_sms)), 256, 0,
+                           stream>>>(U_save, r, Ug, rp, T);
+  }
   // K3b: dX = dY * W^T + D ⊙ (dU * A^T)
   {
     GemmParams gp{};
@@ -819,6 +854,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.dU = dU;
     gp.A = A;
     gp.r = r;
+    gp.du_stride = rp;
     gp.seed = seed;
     gp.thr = thr;
     gp.keep_bits = thr ? keep_bits : nullptr;
@@ -830,7 +866,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmemBwd, stream>>>(mdY128, mWt, mWt, gp);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
-  // K3c: dB = s * U^T * dY and dA = (D ⊙ X)^T * dU, split over tokens, then reduced
+  // K3c: dB = s * U^T * dY and dA = (D ⊙ X)^T * dU, split over tokens, then
+  // reduced; one launch of each contraction per group of up to 64 ranks
   {
     const int64_t tsplit = ((T + S - 1) / S + kTcTok - 1) / kTcTok * kTcTok;
     // keep bits in the dA contraction need a 16-byte row stride (d_in % 128 == 0);
@@ -847,28 +884,37 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
         use_bits = false;
     }
-    TcParams tp{};
-    tp.T = static_cast<int32_t>(T);
-    tp.r = r;
-    tp.splits = static_cast<int32_t>(S);
-    tp.tsplit = static_cast<int32_t>(tsplit);
-    tp.N = static_cast<int32_t>(d_out);
-    tp.thr = 0;
-    tp.keep_bits = nullptr;
-    tp.partial = pdB;
-    dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
-    const int smem_b = 1024 + tc_stages(r, false) * tc_stage_bytes(r, false) + 2 * kTcMaxStages * 8;
-    lora_tcontract_kernel<<<grid_b, kTcThreads, smem_b, stream>>>(mdY64, mU, mBits, tp);
-    tp.N = static_cast<int32_t>(d_in);
-    tp.thr = thr;
-    tp.seed = seed;
-    // with keep bits, each stage's bits come through the copy engine with its tile
-    tp.keep_bits = use_bits ? keep_bits : nullptr;
-    const int smem_a = 1024 + tc_stages(r, use_bits) * tc_stage_bytes(r, use_bits) + 2 * kTcMaxStages * 8;
-    tp.wpr = (d_in + 31) / 32;
-    tp.partial = pdA;
-    dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
-    lora_tcontract_kernel<<<grid_a, kTcThreads, smem_a, stream>>>(mX64, mdU, mBits, tp);
+    const int64_t ustride = Lw.off_U >= 0 ? rp : r;  // r % 16 == 0 when U_save is read directly
+    for (int k0 = 0; k0 < r; k0 += kTcMaxR) {
+      const int w = std::min(kTcMaxR, rp - k0);  // a multiple of 16
+      CUtensorMap mU, mdU;
+      if (!make_map_f32(&mU, Ug, ustride, T, w, 64) || !make_map_f32(&mdU, dU, rp, T, w, 64)) return LORA_ERR_ARG;
+      TcParams tp{};
+      tp.T = static_cast<int32_t>(T);
+      tp.r = w;
+      tp.r_valid = std::min(w, r - k0);
+      tp.k0 = k0;
+      tp.r_total = r;
+      tp.splits = static_cast<int32_t>(S);
+      tp.tsplit = static_cast<int32_t>(tsplit);
+      tp.N = static_cast<int32_t>(d_out);
+      tp.thr = 0;
+      tp.keep_bits = nullptr;
+      tp.partial = pdB;
+      dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
+      const int smem_b = 1024 + tc_stages(w, false) * tc_stage_bytes(w, false) + 2 * kTcMaxStages * 8;
+      lora_tcontract_kernel<<<grid_b, kTcThreads, smem_b, stream>>>(mdY64, mU, mBits, tp);
+      tp.N = static_cast<int32_t>(d_in);
+      tp.thr = thr;
+      tp.seed = seed;
+      // with keep bits, each stage's bits come through the copy engine with its tile
+      tp.keep_bits = use_bits ? keep_bits : nullptr;
+      const int smem_a = 1024 + tc_stages(w, use_bits) * tc_stage_bytes(w, use_bits) + 2 * kTcMaxStages * 8;
+      tp.wpr = (d_in + 31) / 32;
+      tp.partial = pdA;
+      dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
+      lora_tcontract_kernel<<<grid_a, kTcThreads, smem_a, stream>>>(mX64, mdU, mBits, tp);
+    }
     const int64_t nb = static_cast<int64_t>(r) * d_out;
     const int64_t na = static_cast<int64_t>(r) * d_in;
     lora_reduce_splits_kernel<<<static_cast<unsigned>(std::min<int64_t>((nb + 255) / 256, 4096)), 256, 0, stream>>>(
@@ -885,7 +931,8 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
 // call; host code must not use its name as an address (that is a host-side
 // stand-in), so the device address is looked up once per device below.
 static __device__ __align__(256) uint8_t g_bwd_static_scratch[LORA_BWD_STATIC_SCRATCH_BYTES];
-static void *g_bwd_static_ptr[kMaxDevices];
+// its device address per device, published once (release) and read lock-free (acquire)
+static std::atomic<void *> g_bwd_static_ptr[kMaxDevices];
 
 extern "C" {
 
@@ -893,23 +940,26 @@ int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t 
                            float scale, double p_drop, uint64_t seed, const float *U_save, const uint16_t *dY,
                            uint16_t *dX, float *dA, float *dB, int64_t T, int64_t d_in, int64_t d_out, int32_t r,
                            const uint32_t *keep_bits, lora_stream_t stream) {
+  // The size check comes first and touches no pointer: an oversized request is
+  // rejected before any argument is read or any CUDA call is made.
   const size_t need = lora_linear_bwd_workspace_size(T, d_in, d_out, r);
   if (need > LORA_BWD_STATIC_SCRATCH_BYTES) return LORA_ERR_WORKSPACE;
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_ERR_CUDA;
-  if (!g_bwd_static_ptr[dev]) {
+  void *scratch = g_bwd_static_ptr[dev].load(std::memory_order_acquire);
+  if (!scratch) {
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_bwd_static_ptr[dev]) {
-      void *ptr = nullptr;
-      if (cudaGetSymbolAddress(&ptr, g_bwd_static_scratch) != cudaSuccess || !ptr) {
+    scratch = g_bwd_static_ptr[dev].load(std::memory_order_relaxed);
+    if (!scratch) {
+      if (cudaGetSymbolAddress(&scratch, g_bwd_static_scratch) != cudaSuccess || !scratch) {
         cudaGetLastError();
         return LORA_ERR_CUDA;
       }
-      g_bwd_static_ptr[dev] = ptr;
+      g_bwd_static_ptr[dev].store(scratch, std::memory_order_release);
     }
   }
-  return lora_linear_bwd(X, W, A, B, scale, p_drop, seed, U_save, dY, dX, dA, dB, T, d_in, d_out, r,
-                         g_bwd_static_ptr[dev], LORA_BWD_STATIC_SCRATCH_BYTES, keep_bits, stream);
+  return lora_linear_bwd(X, W, A, B, scale, p_drop, seed, U_save, dY, dX, dA, dB, T, d_in, d_out, r, scratch,
+                         LORA_BWD_STATIC_SCRATCH_BYTES, keep_bits, stream);
 }
 
 int lora_dropout_mask(uint64_t seed, double p_drop, int64_t T, int64_t d_in, uint8_t *mask_dev,
@@ -938,6 +988,11 @@ int lora_dropout_keep_bits(uint64_t seed, double p_drop, int64_t T, int64_t d_in
   const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 16 * ds->num_sms));
   lora_keep_bits_kernel<<<blocks, 256, 0, stream>>>(seed, thr, T, d_in, wpr, bits_dev);
   return launch_status();
+}
+
+uint64_t lora_dropout_seed_for_rows(uint64_t seed, int64_t t0, int64_t d_in) {
+  if (t0 < 0 || d_in < 1) return seed;
+  return seed + static_cast<uint64_t>(t0) * static_cast<uint64_t>(d_in) * 0x9E3779B97F4A7C15ull;
 }
 
 int lora_selftest_bounded_wait(uint32_t limit_us, int *waited_ok_dev, lora_stream_t stream) {

@@ -112,7 +112,10 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
           const int32_t prow = cd.pool_row + o;
           int32_t sl = 0;
           while (sl < nslot && ab.prow[sl] != prow) ++sl;
-          if (sl == nslot) ab.prow[nslot++] = prow;
+          if (sl == nslot) {
+            ab.valid |= std::min<int32_t>(16, cd.rank - o) << (5 * nslot);
+            ab.prow[nslot++] = prow;
+          }
           map |= sl << (2 * q);
         }
         ab.info = nslot | (map << 4) | (steps << 12);

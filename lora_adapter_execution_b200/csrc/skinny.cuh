@@ -73,7 +73,7 @@ struct ShrinkParams {
   int32_t r;
   int32_t npieces;
   float scale1;
-  float *dU;                 // [T, r] fp32
+  float *dU;                 // [T, 16 * ceil(r / 16)] fp32, zero past r
 };
 
 struct UnitGeom {
@@ -616,10 +616,13 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
       }
     }
   } else {
+    // rows of dU are padded to a multiple of 16 ranks with zeros, so that the
+    // token contraction reads whole 16-rank groups
     const int nw = static_cast<int>(blockDim.x) >> 5;
+    const int64_t stride = ((p.r + 15) / 16) * 16;
     for (int lr = lr0 + warp; lr < lr1; lr += nw) {
-      float *dst = p.dU + static_cast<int64_t>(g.row0 + lr) * p.r + g.n0;
-      for (int c = lane; c < g.nvalid; c += 32) dst[c] = fin[lr * kShrinkN + c] * p.scale1;
+      float *dst = p.dU + static_cast<int64_t>(g.row0 + lr) * stride + g.n0;
+      for (int c = lane; c < g.nn; c += 32) dst[c] = c < g.nvalid ? fin[lr * kShrinkN + c] * p.scale1 : 0.f;
     }
   }
 }
@@ -647,12 +650,17 @@ __host__ __device__ inline int tc_stages(int r, bool bits) {
 }
 
 struct TcParams {
-  int32_t T, N, r;
+  int32_t T, N;
+  int32_t r;               // ranks of this launch's group, a multiple of 16, <= kTcMaxR (G is
+                           // zero past the real ranks)
+  int32_t r_valid;         // real ranks of the group (<= r): rows written
+  int32_t k0;              // first rank of the group
+  int32_t r_total;         // ranks of the whole contraction (row count of a split's partial)
   int32_t splits, tsplit;  // token splits, tokens per split (multiple of 64)
   uint64_t seed, thr;      // mask on In (dA); thr = 0 for none
   const uint32_t *keep_bits;  // precomputed keep bits of In (null: hash), word t * wpr + col / 32
   int64_t wpr;
-  float *partial;          // [splits][r][N]
+  float *partial;          // [splits][r_total][N]
 };
 
 // split fp32 values into bf16 hi + lo (hi = rn(v), lo = rn(v - hi)), packed in pairs
@@ -678,7 +686,7 @@ __device__ __forceinline__ uint32_t keep_pair_t(uint32_t xa, uint32_t xb) {
 // transposed In fragments and, per 16 ranks, two G^T fragments and eight MMAs.
 __global__ void __launch_bounds__(kTcThreads, 2)
     lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N] bf16, box {64, 64}, swizzle 128B
-                          const __grid_constant__ CUtensorMap mapG,   // G [T, r] fp32, box {r, 64}, no swizzle
+                          const __grid_constant__ CUtensorMap mapG,   // G [T, >= k0 + r] fp32, box {r, 64}, no swizzle
                           const __grid_constant__ CUtensorMap mapBits,  // keep bits [T, wpr] u32, box {4, 64}
                           const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
@@ -729,7 +737,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         mbar_arrive_expect_tx(fb, in_bytes + g_bytes + bits_bytes);
         tma_load_2d(sb, &mapIn, fb, n0, t);
         tma_load_2d(sb + 8192, &mapIn, fb, n0 + 64, t);
-        tma_load_2d(sb + in_bytes, &mapG, fb, 0, t);
+        tma_load_2d(sb + in_bytes, &mapG, fb, p.k0, t);  // the launch's group of ranks
         if (bits) tma_load_2d(sb + in_bytes + g_pad, &mapBits, fb, n0 / 32, t);
         if (++stage == nstage) { stage = 0; phase ^= 1; }
       }
@@ -796,7 +804,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const int tp = item / q4;
         const int k4 = (item - tp * q4) * 4;
         float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (k4 < p.r) {  // r % 8 == 0: a group is all in or all out
+        if (k4 < p.r) {  // r % 16 == 0: a group is all in or all out
           v0 = *reinterpret_cast<const float4 *>(graw + (2 * tp) * p.r + k4);
           v1 = *reinterpret_cast<const float4 *>(graw + (2 * tp + 1) * p.r + k4);
         }
@@ -873,8 +881,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     if (lane == 0) mbar_arrive(empty0 + 8 * stage);
     if (++stage == nstage) { stage = 0; phase ^= 1; }
   }
-  // write partial[q][k][n]
-  float *out = p.partial + static_cast<int64_t>(blockIdx.y) * p.r * p.N;
+  // write partial[q][k0 + k][n] for the group's real ranks
+  float *out = p.partial + (static_cast<int64_t>(blockIdx.y) * p.r_total + p.k0) * p.N;
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     if (i >= mblocks) break;
@@ -885,11 +893,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const int k = i * 16 + (lane >> 2);
         const int c = n0 + cw + 16 * g + j * 8 + q2;
         if (c < p.N) {
-          if (k < p.r) {
+          if (k < p.r_valid) {
             out[static_cast<int64_t>(k) * p.N + c] = acc[i][g][j][0];
             out[static_cast<int64_t>(k) * p.N + c + 1] = acc[i][g][j][1];
           }
-          if (k + 8 < p.r) {
+          if (k + 8 < p.r_valid) {
             out[static_cast<int64_t>(k + 8) * p.N + c] = acc[i][g][j][2];
             out[static_cast<int64_t>(k + 8) * p.N + c + 1] = acc[i][g][j][3];
           }
@@ -912,6 +920,19 @@ __global__ void lora_gather_rows_kernel(const uint16_t *__restrict__ X, const in
     const int64_t i = e / per_row, c = e % per_row;
     const uint4 v = __ldg(reinterpret_cast<const uint4 *>(X + static_cast<int64_t>(perm[i]) * d) + c);
     reinterpret_cast<uint4 *>(Xs + i * d)[c] = v;
+  }
+}
+
+// dst[t][k] = src[t][k] for k < r, 0 for r <= k < rp: a copy of an fp32 [T, r]
+// matrix with rows padded to rp columns.
+__global__ void lora_pad_cols_kernel(const float *__restrict__ src, int r, float *__restrict__ dst, int rp,
+                                     int64_t T) {
+  const int64_t n = T * rp;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t t = e / rp;
+    const int k = static_cast<int>(e - t * rp);
+    dst[e] = k < r ? src[t * r + k] : 0.f;
   }
 }
 

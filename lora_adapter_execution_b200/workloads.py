@@ -16,7 +16,7 @@ Y[t] = X[t]·W + s_a·(X[t]·A_a)·B_a, where a is token t's adapter):
   finetune  T=16384, 4096x4096, 1 adapter of rank 16, s=2, dropout p=0.1,
             plus an upstream gradient dY ~ N(0,1)
 
-Readings where the pages are silent (each is also listed in the design doc):
+Readings where the pages are silent:
   * X ~ N(0,1), W ~ N(0,1/d_in), A ~ N(0,1/d_in), B_a ~ N(0,1/r_a) for every
     workload (only the tiny and decode workloads state it).
   * s_a = 16/r_a where no scale is given (prefill, fleet).
@@ -223,9 +223,11 @@ def integer_inputs(T: int, d_in: int, d_out: int, ranks, ids, seed: int = 0,
 
 def make_rank_inputs(spec: Spec | str, rank: int, **kw) -> Inputs:
     """Rank `rank`'s share of a data-parallel run: the same layer (ranks, scales,
-    W, A_pool, B_pool) on every rank, and a batch of its own (ids, X, dY and the
-    dropout seed) drawn with the workload's recipe. Rank 0's batch is the
-    workload's own draw."""
+    W, A_pool, B_pool) on every rank, and a batch of its own (ids, X, dY) drawn
+    with the workload's recipe. Rank 0's batch is the workload's own draw. The
+    ranks' batches are read as consecutive shards of one global batch (rank r
+    holds global rows r*T .. r*T + T - 1); the dropout seed stays the global
+    one, and the caller derives the seed of its rows from it."""
     if isinstance(spec, str):
         spec = SPECS[spec]
     base = make_inputs(spec, **kw)
@@ -236,4 +238,4 @@ def make_rank_inputs(spec: Spec | str, rank: int, **kw) -> Inputs:
     other = make_inputs(spec, **kw2)
     return Inputs(spec=spec, T=base.T, d_in=base.d_in, d_out=base.d_out, ranks=base.ranks, ids=other.ids,
                   scale=base.scale, X=other.X, W=base.W, A_pool=base.A_pool, B_pool=base.B_pool, dY=other.dY,
-                  p_drop=base.p_drop, mask_seed=base.mask_seed + rank, offsets=base.offsets)
+                  p_drop=base.p_drop, mask_seed=base.mask_seed, offsets=base.offsets)

@@ -89,10 +89,13 @@ def test_bwd_workspace_size_monotone():
 def test_bwd_rejects_bad_rank_before_cuda():
     L = abi.load_library()
     p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
-    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 12, p, 1 << 20, None, None)
-    assert rc == -3
+    for bad_rank in (0, -1, 257):
+        rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, bad_rank, p, 1 << 20, None, None)
+        assert rc == -3
     rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 16, None, 0, None, None)
     assert rc == -8
+    rc = L.lora_linear_bwd(p, p, p, p, 1.0, 0.0, 0, p, p, p, p, p, 64, 64, 64, 5, p, 64, None, None)
+    assert rc == -8  # a workspace smaller than the rank-5 layout needs
 
 
 def test_binding_checks_tensor_metadata_before_the_call():

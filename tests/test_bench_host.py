@@ -47,3 +47,31 @@ def test_decode_gemm_bytes_match_the_reported_figure():
     r_used = int(inp.ranks[np.unique(inp.ids)].sum())
     assert gb == 2 * (256 * 4096 + 4096 * 4096 + r_used * 4096 + 256 * 4096)
     plan.destroy()
+
+
+def test_reference_arm_prints_the_same_config_record():
+    """Both arms describe the headline workload with one config record, computed
+    from the inputs alone."""
+    inp = wl.make_inputs("tiny")
+    a = bench.config_record("tiny", inp, 1)
+    b = bench.config_record("tiny", wl.make_inputs("tiny"), 1)
+    assert a == b and a["workload"] == bench.WORKLOAD_TEXT["tiny"] and a["tokens_per_rank"] == 64
+
+
+def test_backward_algorithmic_flops_match_the_fine_tuning_figure():
+    """Fine-tuning: the base products of the forward and the dX GEMM (2 x 2·T·d²)
+    plus the rank-16 terms come to about 1112 GFLOP per step."""
+    inp = wl.make_inputs("finetune", with_dy=False, T=16384, d_in=64, d_out=64)
+    T, d, r = 16384, 4096, 16
+    inp.T, inp.d_in, inp.d_out = T, d, d
+    _, fl = bench.algorithmic_bwd(inp, r)
+    assert fl == 2 * T * d * d + 2 * T * r * 4 * d
+    fwd = 2 * T * d * d + 2 * (d + d) * r * T
+    assert abs((fl + fwd) / 1e9 - 1112.4) < 0.5
+
+
+def test_default_runs_every_workload_with_the_fine_tuning_headline():
+    a = bench.parse([])
+    assert a.config == "all" and bench.HEADLINE == "finetune"
+    assert set(bench.ORDER) == set(wl.WORKLOADS)
+    assert bench.steps_for(bench.parse(["--steps", "20"]), "decode") == 20

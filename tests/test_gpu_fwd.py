@@ -198,20 +198,98 @@ def test_plan_rebuild_matches_fresh_plan():
     assert lora.device_status() == 0
 
 
-def _sample_rows(T, n, seed=0):
+def tile_rows(inp, seed=0):
+    """Original rows that hit every 128-row tile of the plan's sorted order (one
+    random row per tile, plus the tile's first and last row), and every row of
+    the tile with the largest augmented K (the most adapters and ranks); the
+    grouping comes from the oracle's plan."""
+    perm, seg = oracle.plan(inp.ids, inp.n_adapters)
+    T = inp.T
+    n_tiles = -(-T // 128)
+    kaug = np.zeros(n_tiles, dtype=np.int64)
+    for a, start, length in seg:
+        kc = -(-int(inp.ranks[a]) // 16) * 16
+        for m in range(start // 128, (start + length - 1) // 128 + 1):
+            kaug[m] += 2 * kc
     rng = np.random.default_rng(seed)
-    edge = [0, 1, 127, 128, T - 1, T - 2, T // 2]
-    return np.unique(np.concatenate([edge, rng.choice(T, size=n, replace=False)])).astype(np.int64)
+    pos = [int(rng.integers(128 * m, min(T, 128 * m + 128))) for m in range(n_tiles)]
+    pos += [128 * m for m in range(n_tiles)] + [min(T, 128 * m + 128) - 1 for m in range(n_tiles)]
+    heavy = int(np.argmax(kaug))
+    pos += list(range(128 * heavy, min(T, 128 * heavy + 128)))
+    return np.unique(perm[np.array(pos)]).astype(np.int64), heavy, int(kaug[heavy])
 
 
-@pytest.mark.parametrize("name,nrows", [("decode", None), ("prefill", 48), ("fleet", 96), ("finetune", 32)])
-def test_fwd_full_size_vs_oracle(name, nrows):
+@pytest.mark.parametrize("name", ["decode", "prefill", "fleet", "finetune"])
+def test_fwd_full_size_vs_oracle(name):
     inp = wl.make_inputs(name, with_dy=False)
     Y, U = run_fwd(inp)
-    rows = np.arange(inp.T) if nrows is None else _sample_rows(inp.T, nrows)
+    if name == "decode":
+        rows = np.arange(inp.T)
+    else:
+        rows, heavy, kaug = tile_rows(inp)
+        assert len(rows) >= -(-inp.T // 128)
     Yr, Ur = oracle.forward(inp, rows=rows, want_u=True)
     check_close(Y[rows], Yr, f"{name} Y")
     check_close(U[rows], Ur[:, :U.shape[1]], f"{name} U")
+
+
+def test_fwd_full_size_matches_merged_weights():
+    """The merged form of the S-LoRA article's batching section: Y[t] equals
+    X[t]·(W + s_a·A_a·B_a) with the adapter merged into the weight (numpy fp64,
+    a different formula from the oracle's), on the decode batch's tokens of ten
+    adapters."""
+    inp = wl.make_inputs("decode")
+    Y, _ = run_fwd(inp, want_u=False)
+    X = wl.bf16_bits_to_f32(inp.X).astype(np.float64)
+    W = wl.bf16_bits_to_f32(inp.W).astype(np.float64)
+    A = wl.bf16_bits_to_f32(inp.A_pool).astype(np.float64)
+    B = wl.bf16_bits_to_f32(inp.B_pool).astype(np.float64)
+    for a in np.unique(inp.ids)[:10]:
+        o, r = int(inp.offsets[a]), int(inp.ranks[a])
+        Wm = W + float(inp.scale[a]) * A[o:o + r].T @ B[o:o + r]
+        rows = np.flatnonzero(inp.ids == a)
+        check_close(Y[rows], X[rows] @ Wm, f"merged adapter {a}")
+
+
+@pytest.mark.parametrize("T,d_in,d_out,ranks", [(1, 8, 8, [3]), (1, 4096, 4096, [16, 5]), (5, 8, 8, [1, 16, 2]),
+                                                (130, 8, 16, [4, 21])])
+def test_fwd_degenerate_sizes_vs_oracle(T, d_in, d_out, ranks):
+    """The boundary's smallest sizes: one token, and widths of 8."""
+    inp = wl.make_inputs("tiny", T=T, d_in=d_in, d_out=d_out, n_adapters=len(ranks))
+    ranks = np.array(ranks, dtype=np.int32)
+    off = np.concatenate([[0], np.cumsum(ranks)]).astype(np.int64)
+    rng = np.random.default_rng(11)
+    A = wl.f32_to_bf16_bits(rng.standard_normal((off[-1], d_in)).astype(np.float32) / np.sqrt(d_in))
+    B = wl.f32_to_bf16_bits(rng.standard_normal((off[-1], d_out)).astype(np.float32))
+    ids = rng.integers(0, len(ranks), size=T).astype(np.int32)
+    inp = dataclasses.replace(inp, ranks=ranks, ids=ids, A_pool=A, B_pool=B, offsets=off,
+                              scale=(16.0 / ranks).astype(np.float32))
+    Y, U = run_fwd(inp)
+    Yr, Ur = oracle.forward(inp, want_u=True)
+    check_close(Y, Yr, "Y")
+    check_close(U, Ur[:, :U.shape[1]], "U")
+
+
+def test_fwd_absent_adapter_factors_never_reach_a_token():
+    """Rank 4 and 7 adapters read 16-row slices of B_pool whose remaining rows are
+    the next adapters' rows; with Inf and NaN in those adapters (which have no
+    token in the batch) every output stays finite and matches the oracle."""
+    T, d_in, d_out = 300, 256, 264
+    ranks = np.array([4, 16, 7, 21, 5], dtype=np.int32)
+    off = np.concatenate([[0], np.cumsum(ranks)]).astype(np.int64)
+    rng = np.random.default_rng(4)
+    ids = rng.choice([0, 2, 4], size=T).astype(np.int32)  # adapters 1 and 3 have no tokens
+    inp = wl.make_inputs("tiny", T=T, d_in=d_in, d_out=d_out, n_adapters=5)
+    A = wl.f32_to_bf16_bits(rng.standard_normal((off[-1], d_in)).astype(np.float32) / 16)
+    Bf = rng.standard_normal((off[-1], d_out)).astype(np.float32) / 4
+    Bf[off[1]:off[2]] = np.inf
+    Bf[off[3]:off[4]] = np.nan
+    inp = dataclasses.replace(inp, ranks=ranks, ids=ids, A_pool=A, B_pool=wl.f32_to_bf16_bits(Bf), offsets=off,
+                              scale=np.full(5, 2.0, dtype=np.float32))
+    Y, U = run_fwd(inp)
+    assert np.isfinite(Y).all() and np.isfinite(U).all()
+    clean = dataclasses.replace(inp, B_pool=wl.f32_to_bf16_bits(np.nan_to_num(Bf, nan=0.0, posinf=0.0)))
+    check_close(Y, oracle.forward(clean), "Y next to non-finite absent adapters")
 
 
 def test_fwd_repeatable_bitwise():
