@@ -60,6 +60,8 @@ def lib():
         L.oracle_bwd.restype = None
         L.oracle_bwd.argtypes = [_i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _vp,
                                  _dbl, _u64, _vp, _vp, _i64, _vp, _vp, _vp]
+        L.oracle_switch.restype = None
+        L.oracle_switch.argtypes = [_i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
         L.oracle_num_threads.restype = ctypes.c_int
         L.oracle_num_threads.argtypes = []
         _lib = L
@@ -149,3 +151,18 @@ def backward(inp, rows=None, p=None, seed=None, dY=None, want_dAB=True):
                      _p(X), _p(W), _p(A), _p(B), float(p), seed, _p(dY), _p(rows), rows.shape[0],
                      _p(dX), _p(dA), _p(dB))
     return dX, dA, dB
+
+
+def switch(W, A_pool, B_pool, ranks, term_adapter, term_coef):
+    """Fused adapter switch of every layer (see oracle_switch): W uint16 bf16 bits
+    [L, d_in, d_out], A_pool [L, R, d_in], B_pool [L, R, d_out]; returns the
+    unrounded fp64 [L, d_in, d_out]."""
+    W = _c(W, np.uint16)
+    L, d_in, d_out = W.shape
+    ranks = _c(ranks, np.int32)
+    ta = _c(term_adapter, np.int32)
+    tc = _c(term_coef, np.float64)
+    out = np.empty((L, d_in, d_out), dtype=np.float64)
+    lib().oracle_switch(L, d_in, d_out, ranks.shape[0], _p(ranks), _p(W), _p(_c(A_pool, np.uint16)),
+                        _p(_c(B_pool, np.uint16)), ta.shape[0], _p(ta), _p(tc), _p(out))
+    return out

@@ -292,6 +292,45 @@ void oracle_bwd(int64_t T, int64_t d_in, int64_t d_out, int32_t n_adapters,
     free(off);
 }
 
+/* ---------------------------------------------------------------- adapter switch (merge path)
+ * Fused adapter switching of "AdaFuse: Accelerating Dynamic Adapter Inference
+ * via Token-Level Pre-Gating and Fused Kernel Optimization" (方法详解, 关键设计
+ * item 2): the previous token's active adapters are unmerged (negative
+ * weights) and the current token's merged (positive weights) in one update of
+ * every layer's weight, W_l <- W_l + DOWN·UP with DOWN the concatenation of the
+ * weighted A factors and UP the stacked B factors. Term j names adapter
+ * term_adapter[j] and its coefficient term_coef[j] (the caller's signed gate
+ * times the adapter's scale). For every layer l, row i, column j:
+ *   Wx[l,i,j] = W[l,i,j] + sum_terms c * sum_{k < r_a} A_pool_l[off_a + k][i] * B_pool_l[off_a + k][j]
+ * in fp64, exact inputs; Wx is the unrounded result (the caller rounds to the
+ * weight's precision). Layer l's pools are A_pool + l*R*d_in, B_pool + l*R*d_out
+ * (R = sum of all ranks), with the same adapter offsets in every layer. */
+void oracle_switch(int64_t L, int64_t d_in, int64_t d_out, int32_t n_adapters, const int32_t *ranks,
+                   const uint16_t *W, const uint16_t *A_pool, const uint16_t *B_pool,
+                   int32_t n_terms, const int32_t *term_adapter, const double *term_coef, double *Wx) {
+    int64_t *off = (int64_t *)malloc(sizeof(int64_t) * (size_t)(n_adapters + 1));
+    offsets_of(ranks, n_adapters, off);
+    int64_t R = off[n_adapters];
+#pragma omp parallel for schedule(static)
+    for (int64_t li = 0; li < L * d_in; ++li) {
+        int64_t l = li / d_in, i = li % d_in;
+        const uint16_t *Al = A_pool + l * R * d_in;
+        const uint16_t *Bl = B_pool + l * R * d_out;
+        for (int64_t j = 0; j < d_out; ++j) {
+            double acc = bf(W[(l * d_in + i) * d_out + j]);
+            for (int32_t q = 0; q < n_terms; ++q) {
+                int32_t a = term_adapter[q];
+                double dot = 0.0;
+                for (int32_t k = 0; k < ranks[a]; ++k)
+                    dot += bf(Al[(off[a] + k) * d_in + i]) * bf(Bl[(off[a] + k) * d_out + j]);
+                acc += term_coef[q] * dot;
+            }
+            Wx[(l * d_in + i) * d_out + j] = acc;
+        }
+    }
+    free(off);
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

@@ -332,3 +332,73 @@ def test_backward_single_adapter_closed_forms():
     dU = s * dY @ B.T
     assert np.allclose(dB, s * U.T @ dY, rtol=1e-12, atol=1e-12)
     assert np.allclose(dA, dU.T @ X, rtol=1e-12, atol=1e-12)
+
+
+# ------------------------------------------------------------------ adapter switch (merge path)
+def switch_inputs(L=2, d_in=24, d_out=16, ranks=(3, 5, 2, 4), seed=0, ints=False):
+    """Stacked per-layer weights and factor pools, each layer its own pool with
+    the same adapter offsets."""
+    rng = np.random.default_rng(seed)
+    ranks = np.asarray(ranks, dtype=np.int32)
+    R = int(ranks.sum())
+    if ints:
+        draw = lambda shape: bf(rng.integers(-3, 4, size=shape).astype(np.float32))  # noqa: E731
+    else:
+        draw = lambda shape: bf(rng.standard_normal(shape).astype(np.float32))  # noqa: E731
+    return ranks, draw((L, d_in, d_out)), draw((L, R, d_in)), draw((L, R, d_out))
+
+
+def test_switch_rank1_closed_form():
+    """A rank-1 adapter whose A column is e_i and B row is e_j changes exactly
+    W[l, i, j] by its coefficient, in every layer, and nothing else."""
+    ranks, W, A, B = switch_inputs(L=3, ranks=(1, 2))
+    A[:] = 0
+    B[:] = 0
+    A[:, 0, 5] = bf(1.0)
+    B[:, 0, 7] = bf(1.0)
+    out = oracle.switch(W, A, B, ranks, [0], [-2.5])
+    want = f32(W).copy()
+    want[:, 5, 7] -= 2.5
+    assert np.array_equal(out, want)
+
+
+def test_switch_matches_numpy_sum_of_outer_products():
+    """Per layer, W + sum_j c_j · A_j^T·B_j with A_j^T the pool rows of adapter j
+    transposed (numpy fp64 matmul, a different order of summation)."""
+    ranks, W, A, B = switch_inputs(L=3, d_in=40, d_out=28, ranks=(3, 5, 2, 4), seed=1)
+    terms, coefs = [1, 3, 0], [-0.75, 1.25, 0.5]
+    out = oracle.switch(W, A, B, ranks, terms, coefs)
+    off = np.concatenate([[0], np.cumsum(ranks)])
+    for l in range(3):
+        want = f32(W[l]).copy()
+        for a, c in zip(terms, coefs):
+            Al, Bl = f32(A[l, off[a]:off[a + 1]]), f32(B[l, off[a]:off[a + 1]])
+            want += c * (Al.T @ Bl)
+        np.testing.assert_allclose(out[l], want, rtol=1e-12, atol=1e-12)
+
+
+def test_switch_fused_equals_unmerge_then_merge_and_round_trip():
+    """The fused switch (unmerge the previous adapters with negative weights and
+    merge the current ones in one update) equals the two updates applied one
+    after the other; and unmerging what was merged gives W back. Integer inputs
+    make every step exact, so both hold bit for bit."""
+    ranks, W, A, B = switch_inputs(L=2, ranks=(3, 5, 2, 4), ints=True, seed=2)
+    prev, cur = ([0, 2], [2.0, 1.0]), ([1, 3], [1.0, 3.0])
+    fused = oracle.switch(W, A, B, ranks, prev[0] + cur[0], [-c for c in prev[1]] + cur[1])
+    step1 = oracle.switch(W, A, B, ranks, prev[0], [-c for c in prev[1]])
+    assert np.abs(step1).max() < 256  # exact in bf16
+    step2 = oracle.switch(bf(step1), A, B, ranks, cur[0], cur[1])
+    assert np.array_equal(fused, step2)
+    back = oracle.switch(bf(oracle.switch(W, A, B, ranks, *cur)), A, B, ranks, cur[0], [-c for c in cur[1]])
+    assert np.array_equal(back, f32(W))
+
+
+def test_switch_merged_weight_reproduces_the_unmerged_forward():
+    """Merging an adapter with coefficient s_a into W (one layer) and running the
+    plain product X·W' gives the oracle's unmerged forward for tokens of that
+    adapter (S-LoRA article, batching: formula 1 against formula 2). Integer
+    inputs: exact."""
+    inp = wl.integer_inputs(20, 32, 24, [4, 6], np.ones(20, dtype=np.int32), seed=3, lo=-2, hi=2)
+    inp = dataclasses.replace(inp, scale=np.array([1.0, 3.0], dtype=np.float32))
+    Wm = oracle.switch(inp.W[None], inp.A_pool[None], inp.B_pool[None], inp.ranks, [1], [3.0])[0]
+    assert np.array_equal(f32(inp.X) @ Wm, oracle.forward(inp))
