@@ -16,8 +16,11 @@ With no --config every workload runs in one process and rank 0 prints ONE
 JSON line: the fine-tuning workload (the largest single-GPU configuration,
 forward + backward) is the headline (`value`, `roofline`, `e2e`,
 `cpu_baseline`), and `configs` holds the same record for every workload.
-`roofline` is the fused forward GEMM (the kernel the layer is built around);
-`layer_roofline` is the whole step against the same peak.
+`roofline` is the fused forward GEMM (the kernel the layer is built around),
+timed alone in short bursts against the burst peak; `layer_roofline` is the
+whole step, timed over long back-to-back regions, against the sustained peak.
+`configs["switch"]` is the merge path (one fused adapter switch of a 32-layer
+stack per step).
 
 `e2e` is the same metric through the public API with host buffers: per step
 the plan is built from host ids, X (and dY) are copied from pinned host
@@ -424,11 +427,11 @@ class Ctx:
             import torch.distributed as dist
             dist.barrier()
 
-    def timed(self, step, K, repeats=True):
+    def timed(self, step, K, min_s=MIN_REGION_S):
         """Device ms of exactly K calls of step() (graph replays), each region
-        bracketed by a barrier and a synchronisation; repeated until MIN_REGION_S
-        of device time (at least 3 regions) unless repeats is False; returns the
-        median region, max over ranks."""
+        bracketed by a barrier and a synchronisation; at least 3 regions, repeated
+        until min_s seconds of device time have passed; returns the median region
+        (max over ranks) and the number of regions."""
         import torch
         for i in range(self.a.warmup):
             step(i)
@@ -451,7 +454,7 @@ class Ctx:
             regions.append(ms)
             total += ms * 1e-3
             # every rank takes the same decision (the max over ranks of the total)
-            done = (not repeats) or (len(regions) >= 3 and max_over_ranks(total, self.world, self.dev) >= MIN_REGION_S)
+            done = len(regions) >= 3 and max_over_ranks(total, self.world, self.dev) >= min_s
             if done or len(regions) >= 2000:
                 break
         return max_over_ranks(float(np.median(regions)), self.world, self.dev), len(regions)
@@ -565,7 +568,7 @@ def measure(name, cx, cpu_budget):
         return f
 
     with ClockSampler(cx.local_rank) as clk:
-        ms_total, n_regions = cx.timed(replay(graphs, finetune and world > 1), K, repeats=not a.once)
+        ms_total, n_regions = cx.timed(replay(graphs, finetune and world > 1), K, 0.0 if a.once else MIN_REGION_S)
     clocks = clk.summary()
     value = job_throughput(T, K, world, ms_total)
     entry = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -589,17 +592,22 @@ def measure(name, cx, cpu_budget):
                                    "peak_kind": f"{src} hbm_gbs (copy)", "algorithmic_per_step": lb,
                                    "what": "the whole step (all launches) against the layer's algorithmic bytes"}
     else:
+        # the step is timed over long back-to-back regions (the clock record shows
+        # the power cap), so its peak is the sustained one
         ach = lf / t_step / 1e12
-        entry["layer_roofline"] = {"bound": "tensor", "achieved": ach, "peak": tc_burst, "unit": "TFLOP/s",
-                                   "frac": ach / tc_burst, "frac_of_sustained": ach / tc_sust if tc_sust else None,
-                                   "peak_kind": f"{src} bf16_tflops (burst); sustained {tc_sust}",
+        peak = tc_sust or tc_burst
+        entry["layer_roofline"] = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                                   "frac": ach / peak, "frac_of_burst": ach / tc_burst,
+                                   "peak_kind": f"{src} bf16_tflops_sustained (the step runs {MIN_REGION_S} s and more "
+                                                f"back to back); burst {tc_burst}",
                                    "algorithmic_per_step": lf,
                                    "what": "the whole step (all launches) against the layer's algorithmic flops"}
 
     ms_torch = None
     if not a.no_layer:
-        ms_gemm, _ = cx.timed(replay(ggraphs), K, repeats=not a.once)
-        ms_base, _ = cx.timed(replay(bgraphs), K, repeats=not a.once)
+        # the kernels alone: three regions of K launches (a burst, timed alone)
+        ms_gemm, _ = cx.timed(replay(ggraphs), K, 0.0)
+        ms_base, _ = cx.timed(replay(bgraphs), K, 0.0)
         assert lora.device_status() == 0
         # torch.matmul base for the overhead reference (cuBLAS, same shape and rotation)
         with torch.cuda.stream(cx.stream):
@@ -611,7 +619,7 @@ def measure(name, cx, cpu_budget):
             with torch.cuda.graph(g, stream=cx.stream):
                 torch.matmul(cp["X"], cp["W"], out=cp["Y"])
             tgraphs.append(g)
-        ms_torch, _ = cx.timed(replay(tgraphs), K, repeats=not a.once)
+        ms_torch, _ = cx.timed(replay(tgraphs), K, 0.0)
         t_gemm = ms_gemm * 1e-3 / K
         if name in ("decode", "tiny"):
             ach = gb / t_gemm / 1e9
@@ -623,7 +631,7 @@ def measure(name, cx, cpu_budget):
                     "peak_kind": f"{src} bf16_tflops (burst)"}
         roof.update({"traffic": recorded_traffic(name), "kernel": "lora_gemm_kernel (fused base + adapter GEMM)",
                      "algorithmic_per_launch": gb if roof["bound"] == "hbm" else gf,
-                     "avg_launch_us": t_gemm * 1e6,
+                     "avg_launch_us": t_gemm * 1e6, "timed": f"alone, 3 regions of {K} launches (burst)",
                      "layer_frac": entry["layer_roofline"]["frac"]})
         entry["roofline"] = roof
         base_fwd = min(ms_base, ms_torch) * 1e-3 / K
@@ -742,6 +750,106 @@ def measure_e2e(cx, inp, copies, scale, mask_seed, K):
                     " copy-out streams); host wall clock over the steps"}
 
 
+SWITCH = dict(L=32, d=4096, n_adapters=8, rank=16, prev=(2, 5), cur=(0, 7), gates=((0.6, 0.4), (0.7, 0.3)),
+              scale=2.0)
+SWITCH_TEXT = ("adapter switch: 32 layers of 4096x4096 bf16 weights, 8 rank-16 adapters per layer (s=2); "
+               "unmerge the previous token's top-2 and merge the current top-2 in one pass (4 terms)")
+
+
+def switch_inputs(seed=0):
+    """The switch workload: weights W ~ N(0, 1/d) and factor pools drawn like the
+    layer's (A ~ N(0, 1/d), B ~ N(0, 1/r)), per layer, as bf16 bits."""
+    c = SWITCH
+    rng = np.random.default_rng(seed)
+    L, d, R = c["L"], c["d"], c["n_adapters"] * c["rank"]
+    W = wl.f32_to_bf16_bits(rng.standard_normal((L, d, d), dtype=np.float32) * np.float32(d ** -0.5))
+    A = wl.f32_to_bf16_bits(rng.standard_normal((L, R, d), dtype=np.float32) * np.float32(d ** -0.5))
+    B = wl.f32_to_bf16_bits(rng.standard_normal((L, R, d), dtype=np.float32) * np.float32(c["rank"] ** -0.5))
+    terms = list(c["prev"]) + list(c["cur"])
+    coefs = [-g * c["scale"] for g in c["gates"][0]] + [g * c["scale"] for g in c["gates"][1]]
+    return W, A, B, terms, coefs
+
+
+def measure_switch(cx, cpu_budget):
+    """The merge path: one fused adapter switch of a whole layer stack per step,
+    in place on the resident weights (HBM-bound: every weight is read and
+    written once)."""
+    import torch
+    import lora_adapter_execution_b200 as lora
+    a, dev = cx.a, cx.dev
+    c = SWITCH
+    K = a.steps if a.steps is not None else 50
+    W, A, B, terms, coefs = switch_inputs()
+    L, d, R = c["L"], c["d"], c["n_adapters"] * c["rank"]
+    ranks = np.full(c["n_adapters"], c["rank"], dtype=np.int32)
+
+    def dv(bits):
+        return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).to(dev).view(torch.bfloat16)
+    Wd, Ad, Bd = dv(W), dv(A), dv(B)
+    sw = lora.Switch(ranks, L, d, d, len(terms))
+    # the step alternates the switch and its inverse, so the weights stay near W
+    neg = [-x for x in coefs]
+
+    def step(i):
+        sw.apply(Wd, Ad, Bd, terms, coefs if i % 2 == 0 else neg)
+    with torch.cuda.stream(cx.stream):
+        step(0)
+        step(1)
+    torch.cuda.synchronize()
+    assert lora.device_status() == 0
+    with ClockSampler(cx.local_rank) as clk:
+        ms, n_regions = cx.timed(step, K, 0.0 if a.once else MIN_REGION_S)
+    t = ms * 1e-3 / K
+    hbm, _, _, src = peaks()
+    nbytes = 2 * 2 * L * d * d + 2 * L * len(terms) * c["rank"] * 2 * d
+    ach = nbytes / t / 1e9
+    entry = {"metric": "fused adapter switches/s (every layer of the stack per switch)", "value": 1.0 / t,
+             "unit": "switches/s", "n_gpus": cx.world, "steps": K, "warmup": a.warmup, "ms_per_step": t * 1e3,
+             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+             "config": {"workload": SWITCH_TEXT, "l2": f"weights {2 * L * d * d / 2**30:.1f} GiB > 126 MiB L2"},
+             "timing": (f"eager calls of lora_switch_apply, CUDA events on the stream; median of {n_regions} regions "
+                        f"of exactly {K} switches"),
+             "gpu_launches": 2 * K, "clocks": clk.summary(),
+             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                          "peak_kind": f"{src} hbm_gbs (copy)", "traffic": None,
+                          "kernel": "lora_switch_images_kernel + lora_gemm_kernel (merge mode), per switch",
+                          "algorithmic_per_launch": nbytes, "avg_launch_us": t * 1e6,
+                          "what": "bytes: every weight read and written once, the terms' factor rows read once"}}
+    # e2e: the host holds the term list (adapters, gates); the step copies it in,
+    # switches and reads one row of the last layer back
+    pin = torch.empty(d, dtype=torch.bfloat16).pin_memory()
+    torch.cuda.synchronize()
+    cx.barrier()
+    t0 = time.perf_counter()
+    Ke = max(3, min(K, 50))
+    for i in range(Ke):
+        step(i)
+        pin.copy_(Wd[L - 1, 0], non_blocking=True)
+    torch.cuda.synchronize()
+    dt = max_over_ranks(time.perf_counter() - t0, cx.world, dev)
+    entry["e2e"] = {"value": Ke / dt, "unit": "switches/s", "h2d_bytes_per_step": 8 * len(terms),
+                    "d2h_bytes_per_step": 2 * d, "steps": Ke,
+                    "what": "per step: lora_switch_apply from host term arrays (staged and copied in) + D2H of one "
+                            "weight row; host wall clock"}
+    if cx.rank == 0 and cx.world == 1 and not a.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        run_layers = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < cpu_budget and run_layers < L:
+            oracle.switch(W[run_layers:run_layers + 1], A[run_layers:run_layers + 1], B[run_layers:run_layers + 1],
+                          ranks, terms, coefs)
+            run_layers += 1
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": run_layers / L / dt, "unit": "switches/s", "cores": oracle.num_threads(),
+                                 "kind": "oracle", "sample": f"{run_layers} of the {L} layers, scaled to one switch"}
+    sw.destroy()
+    del Wd, Ad, Bd
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
 HEAD_KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
              "vs_baseline", "dtype", "data", "config", "timing", "roofline", "layer_roofline", "gpu_launches",
              "clocks", "layer", "e2e", "cpu_baseline")
@@ -754,6 +862,8 @@ def run_lora(a):
     for name in names:
         budget = CPU_BUDGET_S["headline" if name in (HEADLINE, a.config) else "other"]
         entries[name] = measure(name, cx, budget)
+    if a.config == "all":
+        entries["switch"] = measure_switch(cx, CPU_BUDGET_S["other"])
     head = entries[HEADLINE if a.config == "all" else a.config]
     out = {k: head[k] for k in HEAD_KEYS if k in head}
     if a.config == "all":

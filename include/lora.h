@@ -309,6 +309,60 @@ int lora_linear_bwd_static(const uint16_t *X, const uint16_t *W, const uint16_t 
                            int64_t d_in, int64_t d_out, int32_t r, const uint32_t *keep_bits,
                            lora_stream_t stream);
 
+/* ------------------------------------------------------------------------
+ * Fused adapter switching (the merge path): W_l <- W_l + sum_j c_j·A_{l,a_j}·B_{l,a_j}
+ * for every layer l of a stack, in place, in one pass over the weights.
+ *
+ * Source: "AdaFuse: Accelerating Dynamic Adapter Inference via Token-Level
+ * Pre-Gating and Fused Kernel Optimization", 方法详解, 关键设计 item 2 (fused
+ * adapter switching: unmerge the previous token's adapters with negative weights
+ * and merge the current ones with positive weights as one concatenated update)
+ * and item 3 (all layers' merges as one batched launch, added in place into
+ * the backbone).
+ *
+ * lora_switch_create — a switch context for a stack of L layers.
+ *   ranks_host  int32[n_adapters]: every layer holds the same adapters with these
+ *               ranks (1 .. LORA_MAX_RANK), in the pool layout of lora_linear_fwd
+ *   L, d_in, d_out   layers and each layer's weight shape (multiples of 8, >= 8;
+ *               L*d_in <= 2^30)
+ *   max_terms   most terms an apply may pass, 1 .. LORA_SWITCH_MAX_TERMS
+ * The context owns device scratch of about L*ceil(d_in/128)*ceil(K/64)*16 KB,
+ * K = 2*max_terms*(largest rank rounded up to 16), plus small tables and two
+ * pinned host staging buffers, until lora_switch_destroy. It belongs to the
+ * device current at this call.
+ * Errors: LORA_ERR_ARG, LORA_ERR_RANK, LORA_ERR_NOMEM, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA.
+ *
+ * lora_switch_apply — the update, asynchronous on `stream`.
+ *   W       bf16 [L, d_in, d_out] DEVICE, updated in place:
+ *           W[l,i,j] <- bf16(W[l,i,j] + sum_j c_j * sum_{k < r_a} A_pool_l[off_a + k][i] * B_pool_l[off_a + k][j])
+ *           with the sum in fp32 and one rounding (nearest even) to bf16
+ *   A_pool  bf16 [L, R, d_in]   layer l's pool at A_pool + l*R*d_in (R = sum of ranks)
+ *   B_pool  bf16 [L, R, d_out]  layer l's pool at B_pool + l*R*d_out
+ *   term_adapter_host int32[n_terms], term_coef_host float[n_terms] (host): term j
+ *           adds c_j·A_a·B_a of adapter a = term_adapter_host[j], c_j =
+ *           term_coef_host[j]; for a switch, the previous adapters with
+ *           c = -gate*scale and the current ones with c = +gate*scale. The same
+ *           terms apply to every layer.
+ *   n_terms 1 .. max_terms
+ * The host arrays may be freed on return (they are staged in pinned memory the
+ * context owns and copied on `stream`). Two applies with one context must be
+ * ordered (they share its scratch). c_j·A enters the tensor cores as a hi and a
+ * lo bf16 part, so the weighted factor keeps about 16 bits.
+ * Errors: LORA_ERR_ARG (null or misaligned pointer, n_terms out of range, another
+ * device current), LORA_ERR_ID (a term's adapter out of range), LORA_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+#define LORA_SWITCH_MAX_TERMS 64
+typedef struct lora_switch *lora_switch_t;
+
+int lora_switch_create(const int32_t *ranks_host, int32_t n_adapters, int64_t L, int64_t d_in, int64_t d_out,
+                       int32_t max_terms, lora_switch_t *out);
+int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, const uint16_t *B_pool,
+                      const int32_t *term_adapter_host, const float *term_coef_host, int32_t n_terms,
+                      lora_stream_t stream);
+/* Free the context (waits for its staging copies; the caller must not free a
+ * context that queued work still uses). NULL is ignored. */
+void lora_switch_destroy(lora_switch_t sw);
+
 /* Test hook: write the dropout mask the forward and backward use (dropout on
  * the LoRA-branch input, one of the small ops the LoRAFusion explainer lists in
  * section 解决什么真问题, item 1; the drop rule is the one under lora_linear_fwd).

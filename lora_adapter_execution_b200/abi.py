@@ -84,6 +84,9 @@ def load_library():
         "lora_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
         "lora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _vp, _vp]),
         "lora_dropout_seed_for_rows": (_u64, [_u64, _i64, _i64]),
+        "lora_switch_create": (ctypes.c_int, [_vp, _i32, _i64, _i64, _i64, _i32, ctypes.POINTER(_vp)]),
+        "lora_switch_apply": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]),
+        "lora_switch_destroy": (None, [_vp]),
         "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -349,3 +352,40 @@ def selftest_bounded_wait(limit_us: int, waited_ok, *, stream=None):
     """Run the bounded-wait self-test (see include/lora.h)."""
     _check(load_library().lora_selftest_bounded_wait(int(limit_us), _ptr(waited_ok), _stream(stream)),
            "lora_selftest_bounded_wait")
+
+
+class Switch:
+    """A fused adapter switch context for a stack of layers (lora_switch_create)."""
+
+    def __init__(self, ranks, L: int, d_in: int, d_out: int, max_terms: int):
+        self._ranks = _host_i32(ranks)
+        self.L, self.d_in, self.d_out, self.max_terms = L, d_in, d_out, max_terms
+        self.pool_rows = int(self._ranks.astype(np.int64).sum())
+        h = _vp()
+        _check(load_library().lora_switch_create(self._ranks.ctypes.data_as(_vp), self._ranks.shape[0], L, d_in, d_out,
+                                                 max_terms, ctypes.byref(h)), "lora_switch_create")
+        self._h = h
+
+    def apply(self, W, A_pool, B_pool, term_adapters, term_coefs, *, stream=None):
+        """W[l] += sum_j coef_j · A_a·B_a (a = term_adapters[j]) for every layer, in place."""
+        L, di, do, R = self.L, self.d_in, self.d_out, self.pool_rows
+        _args("lora_switch_apply", ("W", W, (L, di, do), _BF16, False), ("A_pool", A_pool, (L, R, di), _BF16, False),
+              ("B_pool", B_pool, (L, R, do), _BF16, False))
+        ta = _host_i32(term_adapters)
+        tc = np.ascontiguousarray(term_coefs, dtype=np.float32)
+        if ta.shape != tc.shape or ta.ndim != 1:
+            raise LoraError(-1, "lora_switch_apply: term_adapters and term_coefs differ in shape")
+        _check(load_library().lora_switch_apply(self._h, _ptr(W), _ptr(A_pool), _ptr(B_pool), ta.ctypes.data_as(_vp),
+                                                tc.ctypes.data_as(_vp), ta.shape[0], _stream(stream)),
+               "lora_switch_apply")
+
+    def destroy(self):
+        if getattr(self, "_h", None) is not None and self._h.value:
+            load_library().lora_switch_destroy(self._h)
+            self._h = _vp()
+
+    def __del__(self):
+        try:
+            self.destroy()
+        except Exception:
+            pass

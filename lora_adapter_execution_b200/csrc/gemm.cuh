@@ -13,7 +13,7 @@
 // multi-adapter batch of the batching section (批处理) of "S-LoRA：一个GPU运行
 // 数千大模型成为可能" without padding adapters to a common rank.
 //
-// Structure: persistent CTAs (one per SM), 7 warps:
+// Structure: persistent CTAs (one per SM), 8 warps:
 //   warp 0      TMA producer (lane 0): a 128-row box of X (original rows when a
 //               tile's tokens are consecutive, else the sorted copy of X the
 //               shrink wrote while gathering), then the tile's s·U images (bulk
@@ -22,12 +22,16 @@
 //               every SM loading, one thread's copies complete one after another
 //               (a few hundred ns each, nearly independent of their size), so
 //               two issuing threads double the rate at which stages fill
+//   warp 7      fix-up (with a plan): releases each landed stage to the MMA
+//               thread, after zeroing the B_pool rows of an adapter block that
+//               belong to another adapter (rows past the adapter's rank)
 //   warp 1      MMA issuer (one thread) + TMEM owner: 128x256 fp32 accumulator,
 //               double-buffered in TMEM (512 columns) so the epilogue of tile i
 //               overlaps the main loop of tile i+1
 //   warps 2..5  epilogue: TMEM -> registers -> bf16 -> global rows in the
 //               original token order; in backward mode also adds the dropout-
-//               masked adapter term D ⊙ (dU·A^T)
+//               masked adapter term D ⊙ (dU·A^T); in merge mode adds the
+//               accumulator to the weights in place
 // Every wait is bounded (mbar_wait); on a timeout the CTA flags the status
 // word, stops issuing work and still frees its TMEM.
 #pragma once
@@ -47,12 +51,13 @@ constexpr int kStageBytes = kStageA + kStageB;    // 48 KB
 // An adapter block's B operand: up to four 8 KB slots, each one 16-row slice of
 // B_pool over the tile's 256 columns, stored [4 column blocks][16 rows][64 cols].
 constexpr int kBSlot = 4 * 16 * 128;
-constexpr int kGemmThreads = 224;
+constexpr int kGemmThreads = 256;
 constexpr int kGemmWarpW = 6;  // the W-copy warp
+constexpr int kGemmWarpFix = 7;  // the warp that clears B rows of other adapters
 constexpr int kGemmBarBytes = 256;
 constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16;
 
-enum GemmEpi { kEpiStore = 0, kEpiBwdLora = 1 };
+enum GemmEpi { kEpiStore = 0, kEpiBwdLora = 1, kEpiMergeAdd = 2 };
 constexpr int kEpiRankRegs = 16;  // dU values per row kept in registers by the backward epilogue
 // backward epilogue: the tile's slice of A (ranks < kEpiRankRegs, 256 columns) as
 // fp32 in shared memory, behind the adapter tables
@@ -102,6 +107,17 @@ struct GemmParams {
   // xws + ((tile * S + src) * S + owner) * xslot_bytes(S); null: through
   // distributed shared memory
   uint8_t *xws;
+  // merge mode (merge_kaug > 0, EPI kEpiMergeAdd, K = 0): a stack of layers'
+  // weights, out = [layers * merge_rows, N], updated in place by the adapter
+  // blocks alone. m-tile mt is row block mt % mt_per_layer of layer
+  // mt / mt_per_layer; every tile has merge_kaug augmented columns whose images
+  // sit merge_img_bytes apart in uimg, and the same adapter blocks (augblocks
+  // 0..), whose B rows are offset by the layer's layer_brows rows.
+  int32_t merge_kaug;
+  int32_t mt_per_layer;
+  int32_t merge_rows;
+  int32_t layer_brows;
+  int64_t merge_img_bytes;
 };
 
 // Split-K exchange, inside the idle stage ring once every MMA of the cluster is
@@ -217,6 +233,22 @@ __device__ __forceinline__ bool epi_bar_or(bool v) {
 }
 __device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
 
+// m-tile mt of the merge mode: rows of one layer, all tiles alike
+__device__ __forceinline__ TileDesc merge_tile(const GemmParams &p, int mt) {
+  const int l = mt / p.mt_per_layer;
+  const int ml = mt - l * p.mt_per_layer;
+  TileDesc td;
+  td.row0 = l * p.merge_rows + ml * kBM;
+  td.rows = min(kBM, p.merge_rows - ml * kBM);
+  td.chunk0 = 0;
+  td.nchunk = 0;
+  td.kaug = p.merge_kaug;
+  td.contig = td.row0;
+  td.uofs = static_cast<int64_t>(mt) * p.merge_img_bytes;
+  td.aug0 = 0;
+  return td;
+}
+
 __device__ __forceinline__ TileDesc regular_tile(int mt, int T) {
   TileDesc td;
   td.row0 = mt * kBM;
@@ -251,8 +283,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   volatile uint32_t *bmap = tmem_slot + 2;
   const uint32_t recv_bar = full0 + 128;  // split-K: the other ranks' partials have landed
   // per stage: the adapter block's slot count and each slot's rows that belong to
-  // its adapter (AugBlockDesc::valid | nslot << 20), for the MMA warp
+  // its adapter (AugBlockDesc::valid | nslot << 20), for the fix-up warp
   volatile uint32_t *bvalid = reinterpret_cast<volatile uint32_t *>(bars) + 34;
+  // per stage: released by the fix-up warp once the stage is ready for the MMAs
+  const uint32_t fixed0 = full0 + 152;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -267,6 +301,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       mbar_init(acce0 + 8 * b, 128);
     }
     mbar_init(recv_bar, 1);
+    for (int s = 0; s < kGemmStages; ++s) mbar_init(fixed0 + 8 * s, 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -286,7 +321,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   const int n_tiles = p.n_mt * p.n_nt;
   const int KB = (p.K + kBK - 1) / kBK;
-  const bool has_plan = p.tiles != nullptr;
+  const bool merge = p.merge_kaug > 0;
+  const bool has_plan = p.tiles != nullptr || merge;
+  // the tile table of the plan, the merge mode's layer geometry, or plain row blocks
+  auto tile_desc = [&](int mt) -> TileDesc {
+    return merge ? merge_tile(p, mt) : (p.tiles ? p.tiles[mt] : regular_tile(mt, p.T));
+  };
   const bool split = p.ksplit > 1;
   const int S = split ? p.ksplit : 1;
   const int q = split ? static_cast<int>(cluster_rank()) : 0;
@@ -310,8 +350,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int k = 0; !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
       int mt, nt;
       tile_coords(tile, p, mt, nt);
-      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      const TileDesc td = tile_desc(mt);
       const int n0 = nt * kBN;
+      // merge mode: this tile's layer's rows of B_pool
+      const int brow_ofs = merge ? (mt / p.mt_per_layer) * p.layer_brows : 0;
       // A rows: the sorted copy written by the shrink (rows in tile order), or the
       // original rows when the tile's tokens are consecutive originals
       const int arow = p.a_sorted ? td.row0 : td.contig;
@@ -348,7 +390,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // distinct 16-row slice of B_pool is copied once, into its own slot
             // (the planner's descriptor lists the slices and each step's slot).
             const int lb = blk - KB;
-            const int prow_s[4] = {nprow.x, nprow.y, nprow.z, nprow.w};
+            const int prow_s[4] = {nprow.x + brow_ofs, nprow.y + brow_ofs, nprow.z + brow_ofs, nprow.w + brow_ofs};
             const int nslot = ninfo & 15;
             const uint32_t map = static_cast<uint32_t>(ninfo >> 4) & 0xFFu;
             bvalid[stage] = static_cast<uint32_t>(nvalid) | (static_cast<uint32_t>(nslot) << 20);
@@ -392,7 +434,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int k = 0; !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
         int mt, nt;
         tile_coords(tile, p, mt, nt);
-        const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+        const TileDesc td = tile_desc(mt);
         const int n0 = nt * kBN;
         const int arow = p.a_sorted ? td.row0 : td.contig;
         const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
@@ -417,72 +459,38 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 1) {
-    // -------------------------------------------------------------- MMA warp
-    // Lane 0 issues every MMA. The whole warp waits on each stage so that, for an
+  } else if (warp == kGemmWarpFix) {
+    // ------------------------------------------------------------- fix-up warp
+    // With a plan, every stage reaches the MMA thread through this warp: it waits
+    // for the stage's copies and releases the stage's `fixed` barrier. For an
     // adapter block whose 16-row B slices run past the adapter's rank (the rows
-    // after it are the next adapter's), all 32 lanes can zero those rows in
-    // shared memory before the MMA reads them: a token then never multiplies
-    // factor values of an adapter that is absent from its tile.
-    constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false, !B_KMAJOR);
-    // stage 0's descriptors: A K-major (SW128, 8-row groups 1 KB apart, a K16
-    // step 32 bytes on); B K-major likewise, or MN-major with 64-column blocks
-    // 8 KB apart and a K16 step 16 rows (2 KB) on
-    const uint64_t adesc0 = sdesc_sw128(stage0, 16, 1024);
-    const uint64_t bdesc0 = B_KMAJOR ? sdesc_sw128(stage0 + kStageA, 16, 1024)
-                                     : sdesc_sw128(stage0 + kStageA, 8192, 1024);
-    constexpr uint64_t kAStep = 32 >> 4;
-    constexpr uint64_t kBStep = B_KMAJOR ? (32 >> 4) : (2048 >> 4);
-    int stage = 0;
-    uint32_t phase = 0;
-    int acc = 0;
-    uint32_t aphase = 0;
-    int tile;
-    for (int k = 0;; ++k) {
-      // lane 0's reading of the abort flag decides for the whole warp
-      const bool go = !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile);
-      if (!__shfl_sync(0xFFFFFFFFu, go ? 1 : 0, 0)) break;
-      int mt, nt;
-      tile_coords(tile, p, mt, nt);
-      const int kaug = has_plan ? p.tiles[mt].kaug : 0;
-      const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
-      const int nblk = br.count();
-      bool okw = true;
-      if (lane == 0) okw = mbar_wait(acce0 + 8 * acc, aphase ^ 1);
-      if (!__shfl_sync(0xFFFFFFFFu, okw ? 1 : 0, 0)) {
-        if (lane == 0) *abort_flag = 1;
-        break;
-      }
-      tc_fence_after();
-      const uint32_t d_tmem = tmem_base + acc * kBN;
-      bool ok = true;
-      for (int i = 0; i < nblk; ++i) {
-        const int blk = br.block(i, KB);
-        if (!__all_sync(0xFFFFFFFFu, mbar_wait(full0 + 8 * stage, phase))) {
-          if (lane == 0) *abort_flag = 1;
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        // One thread issues every MMA, so its instruction count per K block
-        // bounds the tensor pipe: the descriptors of a stage are the stage's
-        // base descriptors plus constants (address field in 16-byte units).
-        const uint64_t ad = adesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
-        const uint64_t bd = bdesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
-        if (blk < KB) {
-          if (lane == 0) {
-            umma_bf16(d_tmem, ad, bd, kIdesc, i > 0 ? 1u : 0u);
-            umma_bf16_acc(d_tmem, ad + kAStep, bd + kBStep, kIdesc);
-            umma_bf16_acc(d_tmem, ad + 2 * kAStep, bd + 2 * kBStep, kIdesc);
-            umma_bf16_acc(d_tmem, ad + 3 * kAStep, bd + 3 * kBStep, kIdesc);
+    // after it are the next adapter's), it first zeroes those rows, so a token
+    // never multiplies factor values of an adapter absent from its tile. Being a
+    // warp of its own, the zeroing overlaps the MMAs of the blocks before; and
+    // since the MMA thread waits on every stage's release, this warp is never more
+    // than one phase behind a barrier, which keeps its parity waits exact.
+    if (has_plan) {
+      int stage = 0;
+      uint32_t phase = 0;
+      int tile;
+      for (int k = 0;; ++k) {
+        const bool go = !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile);
+        if (!__shfl_sync(0xFFFFFFFFu, go ? 1 : 0, 0)) break;
+        int mt, nt;
+        tile_coords(tile, p, mt, nt);
+        const TileDesc td = tile_desc(mt);
+        const int arow = p.a_sorted ? td.row0 : td.contig;
+        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const int nblk = arow < 0 ? 0 : br.count();
+        bool ok = true;
+        for (int i = 0; i < nblk; ++i) {
+          const int blk = br.block(i, KB);
+          if (!__all_sync(0xFFFFFFFFu, mbar_wait(full0 + 8 * stage, phase))) {
+            if (lane == 0) *abort_flag = 1;
+            ok = false;
+            break;
           }
-        } else {
-          // adapter block (MN-major B slots [4 column blocks][16 rows][64 cols],
-          // column-block stride 2 KB; the slot of each K step from bmap)
-          const int steps = min(4, (kaug - (blk - KB) * kAugBlock) / 16);
-          const uint32_t map = bmap[stage];
-          const uint32_t b_s = stage0 + stage * kStageBytes + kStageA;
-          if (!B_KMAJOR) {
+          if (!B_KMAJOR && blk >= KB) {
             const uint32_t vw = bvalid[stage];
             const int nsl = static_cast<int>(vw >> 20);
             uint8_t *bsp = smem + stage * kStageBytes + kStageA;
@@ -500,24 +508,78 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
               zeroed |= v < 16;
             }
             if (zeroed) fence_proxy_async_smem();  // the MMA reads through the async proxy
-            __syncwarp();
           }
-          if (lane == 0) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(fixed0 + 8 * stage);
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
+        }
+        if (!ok) break;
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------ MMA issuer
+      constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false, !B_KMAJOR);
+      // stage 0's descriptors: A K-major (SW128, 8-row groups 1 KB apart, a K16
+      // step 32 bytes on); B K-major likewise, or MN-major with 64-column blocks
+      // 8 KB apart and a K16 step 16 rows (2 KB) on
+      const uint64_t adesc0 = sdesc_sw128(stage0, 16, 1024);
+      const uint64_t bdesc0 = B_KMAJOR ? sdesc_sw128(stage0 + kStageA, 16, 1024)
+                                       : sdesc_sw128(stage0 + kStageA, 8192, 1024);
+      constexpr uint64_t kAStep = 32 >> 4;
+      constexpr uint64_t kBStep = B_KMAJOR ? (32 >> 4) : (2048 >> 4);
+      // with a plan a stage is ready once the fix-up warp has released it
+      const uint32_t ready0 = has_plan ? fixed0 : full0;
+      int stage = 0;
+      uint32_t phase = 0;
+      int acc = 0;
+      uint32_t aphase = 0;
+      int tile;
+      for (int k = 0; !*abort_flag && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
+        int mt, nt;
+        tile_coords(tile, p, mt, nt);
+        const int kaug = merge ? p.merge_kaug : (p.tiles ? p.tiles[mt].kaug : 0);
+        const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const int nblk = br.count();
+        if (!mbar_wait(acce0 + 8 * acc, aphase ^ 1)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const uint32_t d_tmem = tmem_base + acc * kBN;
+        bool ok = true;
+        for (int i = 0; i < nblk; ++i) {
+          const int blk = br.block(i, KB);
+          if (!mbar_wait(ready0 + 8 * stage, phase)) { *abort_flag = 1; ok = false; break; }
+          tc_fence_after();
+          // One thread issues every MMA, so its instruction count per K block
+          // bounds the tensor pipe: the descriptors of a stage are the stage's
+          // base descriptors plus constants (address field in 16-byte units).
+          const uint64_t ad = adesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
+          const uint64_t bd = bdesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
+          if (blk < KB) {
+            umma_bf16(d_tmem, ad, bd, kIdesc, i > 0 ? 1u : 0u);
+            umma_bf16_acc(d_tmem, ad + kAStep, bd + kBStep, kIdesc);
+            umma_bf16_acc(d_tmem, ad + 2 * kAStep, bd + 2 * kBStep, kIdesc);
+            umma_bf16_acc(d_tmem, ad + 3 * kAStep, bd + 3 * kBStep, kIdesc);
+          } else {
+            // adapter block (MN-major B slots [4 column blocks][16 rows][64 cols],
+            // column-block stride 2 KB; the slot of each K step from bmap)
+            const int steps = min(4, (kaug - (blk - KB) * kAugBlock) / 16);
+            const uint32_t map = bmap[stage];
+            const uint32_t b_s = stage0 + stage * kStageBytes + kStageA;
             for (int qq = 0; qq < steps; ++qq) {
               const uint64_t bq = B_KMAJOR ? bd + qq * kAStep
                                            : sdesc_sw128(b_s + ((map >> (2 * qq)) & 3u) * kBSlot, 2048, 1024);
               umma_bf16(d_tmem, ad + qq * kAStep, bq, kIdesc, (i > 0 || qq > 0) ? 1u : 0u);
             }
           }
+          umma_commit(empty0 + 8 * stage);
+          if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
         }
-        if (lane == 0) umma_commit(empty0 + 8 * stage);
-        if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
+        if (!ok) break;
+        umma_commit(accf0 + 8 * acc);
+        if (++acc == 2) { acc = 0; aphase ^= 1; }
       }
-      if (!ok) break;
-      if (lane == 0) umma_commit(accf0 + 8 * acc);
-      if (++acc == 2) { acc = 0; aphase ^= 1; }
     }
-    __syncwarp();
   } else {
     // -------------------------------------------------------------- epilogue (warps 2..5)
     const int quarter = warp & 3;  // TMEM lanes 32*quarter .. +31
@@ -529,7 +591,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       // the split-K tail's table entry and output row, loaded while the K loop runs
       int mt = 0, nt = 0;
       tile_coords(tile0 < n_tiles ? tile0 : 0, p, mt, nt);
-      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      const TileDesc td = tile_desc(mt);
       split_rows = td.rows;
       split_nt = nt;
       split_kaug = td.kaug;
@@ -543,7 +605,50 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     for (int k = 0; (EPI == kEpiBwdLora || !*abort_flag) && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
       int mt, nt;
       tile_coords(tile, p, mt, nt);
-      const TileDesc td = has_plan ? p.tiles[mt] : regular_tile(mt, p.T);
+      const TileDesc td = tile_desc(mt);
+      if constexpr (EPI == kEpiMergeAdd) {
+        // W <- bf16(W + accumulator), in place: this row's current weights are
+        // loaded before the accumulator is waited for, so the loads overlap the
+        // tile's MMAs (each element is read and written by this thread only)
+        const bool valid = row < td.rows;
+        const int64_t orow = static_cast<int64_t>(td.contig) + row;
+        uint4 wv[kBN / 8];
+#pragma unroll
+        for (int c8 = 0; c8 < kBN / 8; ++c8) {
+          const int col = nt * kBN + c8 * 8;
+          wv[c8] = (valid && col < p.N) ? *reinterpret_cast<const uint4 *>(p.out + orow * p.N + col)
+                                        : make_uint4(0u, 0u, 0u, 0u);
+        }
+        if (!mbar_wait(accf0 + 8 * acc, aphase)) { *abort_flag = 1; break; }
+        tc_fence_after();
+#pragma unroll
+        for (int c = 0; c < kBN / 32; ++c) {
+          uint32_t v[32];
+          tmem_ld32(tmem_base + ((quarter * 32) << 16) + acc * kBN + c * 32, v);
+          tmem_wait_ld();
+          const int col0 = nt * kBN + c * 32;
+          if (valid && col0 < p.N) {
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * p.N + col0);
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+              if (col0 + 8 * j < p.N) {
+                const uint4 w = wv[c * 4 + j];
+                const uint32_t *vv = v + 8 * j;
+                uint4 o;
+                o.x = pack_bf16x2(bf16_lo(w.x) + __uint_as_float(vv[0]), bf16_hi(w.x) + __uint_as_float(vv[1]));
+                o.y = pack_bf16x2(bf16_lo(w.y) + __uint_as_float(vv[2]), bf16_hi(w.y) + __uint_as_float(vv[3]));
+                o.z = pack_bf16x2(bf16_lo(w.z) + __uint_as_float(vv[4]), bf16_hi(w.z) + __uint_as_float(vv[5]));
+                o.w = pack_bf16x2(bf16_lo(w.w) + __uint_as_float(vv[6]), bf16_hi(w.w) + __uint_as_float(vv[7]));
+                dst[j] = o;
+              }
+            }
+          }
+        }
+        tc_fence_before();
+        mbar_arrive(acce0 + 8 * acc);
+        if (++acc == 2) { acc = 0; aphase ^= 1; }
+        continue;
+      }
       if (EPI == kEpiBwdLora) {
         // stage A[k][nt*256 .. +256) for k < min(r, 16) as fp32 (zero past r or N):
         // 8 threads per rank, 32 columns each

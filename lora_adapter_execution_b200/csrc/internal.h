@@ -76,6 +76,18 @@ struct alignas(16) UnitDesc {
   int64_t uofs;       // byte offset of the tile's s*U image in the plan scratch
 };
 
+// One term of a fused adapter switch: adapter rows [pool_row, pool_row + rank)
+// of every layer's pools, weighted by coef, as augmented columns
+// [kofs, kofs + 2*kc) of every tile (hi part, then lo part).
+struct alignas(16) SwitchTerm {
+  int32_t pool_row;
+  int32_t rank;
+  int32_t kc;    // rank rounded up to 16
+  int32_t kofs;
+  float coef;
+  int32_t pad_[3];
+};
+
 struct HostPlan {
   int64_t T = 0, d_in = 0, d_out = 0;
   int32_t n_adapters = 0;
@@ -93,6 +105,10 @@ struct HostPlan {
   int64_t xs_offset = -1;  // byte offset of the sorted copy of X in the scratch (-1: not needed)
   int32_t max_chunk_rows = 0;
 };
+
+// The adapter K blocks of one tile whose chunks (consecutive, kofs ascending,
+// each 2*kc augmented columns: hi part then lo part) span kaug columns.
+void append_aug_blocks(const ChunkDesc *chunks, int32_t nchunk, int32_t kaug, std::vector<AugBlockDesc> &out);
 
 // Returns LORA_OK or a LORA_ERR_* code; fills `hp` on success.
 int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t n_adapters,

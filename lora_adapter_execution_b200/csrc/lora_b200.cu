@@ -13,6 +13,7 @@
 
 #include "gemm.cuh"
 #include "skinny.cuh"
+#include "switch.cuh"
 
 using namespace lora;
 
@@ -60,6 +61,8 @@ int device_state(DeviceState **out) {
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_gemm_kernel<true, kEpiBwdLora>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBwd) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_gemm_kernel<false, kEpiMergeAdd>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_shrink_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sk_smem(4)) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_shrink_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -1012,6 +1015,191 @@ int lora_device_status(lora_stream_t stream, uint32_t *status_host) {
   if (v && cudaMemcpyToSymbol(g_status, &zero, sizeof(zero)) != cudaSuccess) return LORA_ERR_CUDA;
   if (status_host) *status_host = v;
   return v ? LORA_ERR_DEVICE : LORA_OK;
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ fused adapter switch
+struct lora_switch {
+  int64_t L = 0, d_in = 0, d_out = 0;
+  std::vector<int32_t> ranks;
+  std::vector<int64_t> off;  // n_adapters + 1
+  int32_t max_terms = 0;
+  int32_t max_kaug = 0;      // max_terms * 2 * (largest rank rounded up to 16)
+  int32_t mt_per_layer = 0;
+  int64_t n_tiles = 0;       // L * mt_per_layer
+  int64_t img_bytes = 0;     // one tile's images
+  uint8_t *img = nullptr;    // n_tiles * img_bytes
+  void *dev = nullptr;       // terms | adapter blocks
+  size_t dev_bytes = 0;
+  void *stage[2] = {nullptr, nullptr};
+  cudaEvent_t stage_ev[2] = {nullptr, nullptr};
+  int stage_next = 0;
+  int device = 0;
+};
+
+extern "C" {
+
+void lora_switch_destroy(lora_switch_t sw) {
+  if (!sw) return;
+  for (int k = 0; k < 2; ++k) {
+    if (sw->stage_ev[k]) {
+      cudaEventSynchronize(sw->stage_ev[k]);
+      cudaEventDestroy(sw->stage_ev[k]);
+    }
+    if (sw->stage[k]) cudaFreeHost(sw->stage[k]);
+  }
+  if (sw->dev) cudaFree(sw->dev);
+  if (sw->img) cudaFree(sw->img);
+  delete sw;
+}
+
+int lora_switch_create(const int32_t *ranks_host, int32_t n_adapters, int64_t L, int64_t d_in, int64_t d_out,
+                       int32_t max_terms, lora_switch_t *out) {
+  if (!out || !ranks_host || n_adapters < 1 || L < 1 || d_in < 8 || d_out < 8 || (d_in % 8) || (d_out % 8))
+    return LORA_ERR_ARG;
+  if (max_terms < 1 || max_terms > LORA_SWITCH_MAX_TERMS) return LORA_ERR_ARG;
+  if (L * d_in > ((int64_t)1 << 30) || d_out > ((int64_t)1 << 30)) return LORA_ERR_ARG;
+  int32_t rmax = 0;
+  for (int32_t a = 0; a < n_adapters; ++a) {
+    if (ranks_host[a] < 1 || ranks_host[a] > LORA_MAX_RANK) return LORA_ERR_RANK;
+    rmax = std::max(rmax, ranks_host[a]);
+  }
+  DeviceState *ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LORA_OK) return rc;
+  lora_switch *sw = new (std::nothrow) lora_switch();
+  if (!sw) return LORA_ERR_NOMEM;
+  sw->L = L;
+  sw->d_in = d_in;
+  sw->d_out = d_out;
+  sw->ranks.assign(ranks_host, ranks_host + n_adapters);
+  sw->off.assign(n_adapters + 1, 0);
+  for (int32_t a = 0; a < n_adapters; ++a) sw->off[a + 1] = sw->off[a] + ranks_host[a];
+  if (L * sw->off[n_adapters] >= ((int64_t)1 << 31) - 256) {
+    delete sw;
+    return LORA_ERR_ARG;
+  }
+  sw->max_terms = max_terms;
+  sw->max_kaug = max_terms * 2 * ((rmax + 15) / 16 * 16);
+  sw->mt_per_layer = static_cast<int32_t>((d_in + kTileM - 1) / kTileM);
+  sw->n_tiles = L * sw->mt_per_layer;
+  sw->img_bytes = static_cast<int64_t>((sw->max_kaug + kAugBlock - 1) / kAugBlock) * kAugBlockBytes;
+  const size_t nblk_max = static_cast<size_t>((sw->max_kaug + kAugBlock - 1) / kAugBlock);
+  sw->dev_bytes = ((sizeof(SwitchTerm) * max_terms + 255) & ~static_cast<size_t>(255)) + sizeof(AugBlockDesc) * nblk_max;
+  cudaGetDevice(&sw->device);
+  bool ok = cudaMalloc(reinterpret_cast<void **>(&sw->img), static_cast<size_t>(sw->n_tiles * sw->img_bytes)) ==
+            cudaSuccess;
+  ok = ok && cudaMalloc(&sw->dev, sw->dev_bytes) == cudaSuccess;
+  for (int k = 0; k < 2 && ok; ++k) {
+    ok &= cudaHostAlloc(&sw->stage[k], sw->dev_bytes, cudaHostAllocDefault) == cudaSuccess;
+    ok = ok && cudaEventCreateWithFlags(&sw->stage_ev[k], cudaEventDisableTiming) == cudaSuccess;
+  }
+  if (!ok) {
+    cudaGetLastError();
+    lora_switch_destroy(sw);
+    return LORA_ERR_NOMEM;
+  }
+  *out = sw;
+  return LORA_OK;
+}
+
+int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, const uint16_t *B_pool,
+                      const int32_t *term_adapter_host, const float *term_coef_host, int32_t n_terms,
+                      lora_stream_t stream) {
+  if (!sw || !W || !A_pool || !B_pool || !term_adapter_host || !term_coef_host) return LORA_ERR_ARG;
+  if (n_terms < 1 || n_terms > sw->max_terms) return LORA_ERR_ARG;
+  if (!aligned16(W) || !aligned16(A_pool) || !aligned16(B_pool)) return LORA_ERR_ARG;
+  {
+    int d = -1;
+    if (cudaGetDevice(&d) != cudaSuccess || d != sw->device) return LORA_ERR_ARG;
+  }
+  const int32_t n_adapters = static_cast<int32_t>(sw->ranks.size());
+  for (int32_t j = 0; j < n_terms; ++j)
+    if (term_adapter_host[j] < 0 || term_adapter_host[j] >= n_adapters) return LORA_ERR_ID;
+  DeviceState *ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LORA_OK) return rc;
+  // the terms' augmented columns (hi part, then lo part, per term) and the
+  // adapter blocks that read their B rows, the same for every tile
+  std::vector<SwitchTerm> terms(n_terms);
+  std::vector<ChunkDesc> chunks(n_terms);
+  int32_t kofs = 0;
+  for (int32_t j = 0; j < n_terms; ++j) {
+    const int32_t a = term_adapter_host[j];
+    SwitchTerm &t = terms[j];
+    t = SwitchTerm{};
+    t.pool_row = static_cast<int32_t>(sw->off[a]);
+    t.rank = sw->ranks[a];
+    t.kc = (t.rank + 15) / 16 * 16;
+    t.kofs = kofs;
+    t.coef = term_coef_host[j];
+    ChunkDesc &c = chunks[j];
+    c = ChunkDesc{};
+    c.adapter = a;
+    c.pool_row = t.pool_row;
+    c.rank = t.rank;
+    c.kc = t.kc;
+    c.kofs = kofs;
+    kofs += 2 * t.kc;
+  }
+  const int32_t kaug = kofs;
+  std::vector<AugBlockDesc> aug;
+  append_aug_blocks(chunks.data(), n_terms, kaug, aug);
+  const size_t b_terms = (sizeof(SwitchTerm) * sw->max_terms + 255) & ~static_cast<size_t>(255);
+  const size_t total = b_terms + sizeof(AugBlockDesc) * aug.size();
+  // one copy from one of two pinned staging buffers (refilled once its last
+  // copy has completed), stream-ordered before the kernels that read it
+  const int k = sw->stage_next;
+  if (cudaEventSynchronize(sw->stage_ev[k]) != cudaSuccess) return LORA_ERR_CUDA;
+  uint8_t *h = static_cast<uint8_t *>(sw->stage[k]);
+  std::memcpy(h, terms.data(), sizeof(SwitchTerm) * n_terms);
+  std::memcpy(h + b_terms, aug.data(), sizeof(AugBlockDesc) * aug.size());
+  uint8_t *dbase = static_cast<uint8_t *>(sw->dev);
+  if (cudaMemcpyAsync(dbase, h, total, cudaMemcpyHostToDevice, stream) != cudaSuccess ||
+      cudaEventRecord(sw->stage_ev[k], stream) != cudaSuccess) {
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  sw->stage_next = k ^ 1;
+  const int64_t R = sw->off[n_adapters];
+  // DOWN: c·A of every term, as the tiles' swizzled images
+  {
+    const int64_t n = sw->n_tiles * (kaug / 8) * kTileM;
+    const unsigned blocks = static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 32 * ds->num_sms));
+    lora_switch_images_kernel<<<blocks, 256, 0, stream>>>(A_pool, reinterpret_cast<const SwitchTerm *>(dbase),
+                                                          n_terms, R, sw->d_in, sw->mt_per_layer, sw->n_tiles, kaug,
+                                                          sw->img_bytes, sw->img);
+    if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+  }
+  // W += DOWN·UP on the tensor cores, every layer in one persistent launch
+  CUtensorMap mBl;
+  const bool b3d = sw->d_out % 64 == 0;
+  const bool ok = b3d ? make_map_blocks(&mBl, B_pool, sw->d_out, sw->L * R, 16, kBN / 64)
+                      : make_map(&mBl, B_pool, sw->d_out, sw->L * R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return LORA_ERR_ARG;
+  GemmParams gp{};
+  gp.b3d = b3d ? 1 : 0;
+  gp.T = static_cast<int32_t>(sw->L * sw->d_in);
+  gp.K = 0;
+  gp.N = static_cast<int32_t>(sw->d_out);
+  gp.n_mt = static_cast<int32_t>(sw->n_tiles);
+  gp.n_nt = static_cast<int32_t>((sw->d_out + kBN - 1) / kBN);
+  gp.uimg = sw->img;
+  gp.augblocks = reinterpret_cast<const AugBlockDesc *>(dbase + b_terms);
+  gp.out = reinterpret_cast<__nv_bfloat16 *>(W);
+  gp.group_m = 1;
+  gp.ksplit = 1;
+  gp.merge_kaug = kaug;
+  gp.mt_per_layer = sw->mt_per_layer;
+  gp.merge_rows = static_cast<int32_t>(sw->d_in);
+  gp.layer_brows = static_cast<int32_t>(R);
+  gp.merge_img_bytes = sw->img_bytes;
+  const int64_t n_tiles = static_cast<int64_t>(gp.n_mt) * gp.n_nt;
+  const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ds->num_sms, n_tiles));
+  // no base K blocks: the A and W maps are never used for copies
+  lora_gemm_kernel<false, kEpiMergeAdd><<<grid, kGemmThreads, kGemmSmem, stream>>>(mBl, mBl, mBl, gp);
+  return launch_status();
 }
 
 }  // extern "C"

@@ -16,6 +16,34 @@
 
 namespace lora {
 
+void append_aug_blocks(const ChunkDesc *chunks, int32_t nchunk, int32_t kaug, std::vector<AugBlockDesc> &out) {
+  // for each 16-wide K step its B_pool rows (the hi and lo steps of a chunk read
+  // the same rows); distinct row slices get slots
+  int32_t c = 0;
+  for (int32_t k0 = 0; k0 < kaug; k0 += kAugBlock) {
+    AugBlockDesc ab{};
+    const int32_t steps = std::min<int32_t>(4, (kaug - k0) / 16);
+    int32_t nslot = 0, map = 0;
+    for (int32_t q = 0; q < steps; ++q) {
+      const int32_t kq = k0 + q * 16;
+      while (c + 1 < nchunk && kq >= chunks[c].kofs + 2 * chunks[c].kc) ++c;
+      const ChunkDesc &cd = chunks[c];
+      int32_t o = kq - cd.kofs;
+      if (o >= cd.kc) o -= cd.kc;
+      const int32_t prow = cd.pool_row + o;
+      int32_t sl = 0;
+      while (sl < nslot && ab.prow[sl] != prow) ++sl;
+      if (sl == nslot) {
+        ab.valid |= std::min<int32_t>(16, cd.rank - o) << (5 * nslot);
+        ab.prow[nslot++] = prow;
+      }
+      map |= sl << (2 * q);
+    }
+    ab.info = nslot | (map << 4) | (steps << 12);
+    out.push_back(ab);
+  }
+}
+
 int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t n_adapters,
                     int64_t d_in, int64_t d_out, HostPlan &hp) {
   if (!ids || !ranks || T <= 0 || n_adapters <= 0 || d_in < 8 || d_out < 8 || (d_in % 8) ||
@@ -94,34 +122,9 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
     }
     td.nchunk = (int32_t)hp.chunks.size() - td.chunk0;
     td.kaug = kofs;
-    // adapter K blocks: for each 16-wide K step its B_pool rows (the hi and lo
-    // steps of a chunk read the same rows); distinct row slices get slots
+    // the tile's adapter K blocks
     td.aug0 = (int32_t)hp.augblocks.size();
-    {
-      int32_t c = td.chunk0;
-      for (int32_t k0 = 0; k0 < td.kaug; k0 += kAugBlock) {
-        AugBlockDesc ab{};
-        const int32_t steps = std::min<int32_t>(4, (td.kaug - k0) / 16);
-        int32_t nslot = 0, map = 0;
-        for (int32_t q = 0; q < steps; ++q) {
-          const int32_t kq = k0 + q * 16;
-          while (c + 1 < td.chunk0 + td.nchunk && kq >= hp.chunks[c].kofs + 2 * hp.chunks[c].kc) ++c;
-          const ChunkDesc &cd = hp.chunks[c];
-          int32_t o = kq - cd.kofs;
-          if (o >= cd.kc) o -= cd.kc;
-          const int32_t prow = cd.pool_row + o;
-          int32_t sl = 0;
-          while (sl < nslot && ab.prow[sl] != prow) ++sl;
-          if (sl == nslot) {
-            ab.valid |= std::min<int32_t>(16, cd.rank - o) << (5 * nslot);
-            ab.prow[nslot++] = prow;
-          }
-          map |= sl << (2 * q);
-        }
-        ab.info = nslot | (map << 4) | (steps << 12);
-        hp.augblocks.push_back(ab);
-      }
-    }
+    append_aug_blocks(hp.chunks.data() + td.chunk0, td.nchunk, td.kaug, hp.augblocks);
     // consecutive originals?
     bool contig = true;
     for (int32_t i = 1; i < td.rows && contig; ++i)
