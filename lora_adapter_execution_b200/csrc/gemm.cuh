@@ -359,6 +359,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int arow = p.a_sorted ? td.row0 : td.contig;
       if (lane == 0) {
         if (arow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; }
+        if (merge) {
+          // the epilogue will read this tile's weights: have L2 fetch them now,
+          // while the stages and the epilogue of the tiles before are in flight
+          const uint32_t bytes = static_cast<uint32_t>(min(kBN, p.N - n0)) * 2u;
+          for (int r = 0; r < td.rows; ++r)
+            bulk_prefetch_l2(p.out + (static_cast<int64_t>(td.contig) + r) * p.N + n0, bytes);
+        }
         const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
         const int nblk = arow < 0 ? 0 : br.count();
         // adapter block descriptors, one load ahead of their use (the adapter
