@@ -62,7 +62,7 @@ METRIC = "tokens/s per fused multi-LoRA linear at 1 B200; % of bf16 TC peak / HB
 L2_BYTES = 126 * 1024 * 1024
 ORDER = ("tiny", "decode", "prefill", "fleet", "finetune")
 HEADLINE = "finetune"
-DEFAULT_STEPS = {"tiny": 2000, "decode": 3000, "prefill": 200, "fleet": 1000, "finetune": 100}
+DEFAULT_STEPS = {"tiny": 2000, "decode": 3000, "prefill": 200, "fleet": 1000, "finetune": 100, "fleet_finetune": 200}
 DEFAULT_WARMUP = 5
 MIN_REGION_S = 0.3  # a timed region is repeated until this much device time has passed
 CPU_BUDGET_S = {"headline": 12.0, "other": 5.0}
@@ -72,6 +72,9 @@ WORKLOAD_TEXT = {
     "prefill": "prefill: T=8192, d_in=4096, d_out=11008, 200 adapters ranks {8,16,32,64}, Zipf(1.0) per 512-token request",
     "fleet": "fleet: T=4096, d_in=d_out=4096, 1000 adapters ranks 1..21, B rows x 1/k, Zipf(1.2) per token",
     "finetune": "finetune: T=16384, d_in=d_out=4096, 1 adapter rank 16, s=2, dropout 0.1; forward + backward",
+    "fleet_finetune": ("fleet_finetune: the fleet batch (T=4096, 4096x4096, 1000 adapters ranks 1..21, Zipf(1.2) per "
+                       "token) as one fine-tuning step of all its adapters, dropout 0.1; forward + multi-adapter "
+                       "backward"),
 }
 # The fused GEMM, its launch and the plan tables that shape its work: a recorded
 # ncu figure for the GEMM holds while the code of these files is unchanged.
@@ -317,6 +320,18 @@ def algorithmic(inp, info):
     return gemm_bytes, gemm_flops, layer_bytes, layer_flops
 
 
+def algorithmic_bwd_multi(inp, info):
+    """The multi-adapter backward: reads X, W, dY, the used adapters' A, B rows
+    and U, writes dX and the used gradient rows; flops of the dX GEMM and each
+    token's rank-r terms (dU, its dX term, its dB and dA shares)."""
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    R_used, R_tok = info["sum_r_used"], info["sum_r_tokens"]
+    nbytes = (2 * (T * di + di * do + T * do + R_used * (di + do)) + 4 * T * info["r_max"] + 2 * T * di
+              + 4 * R_used * (di + do))
+    flops = 2 * T * do * di + 4 * (di + do) * R_tok
+    return nbytes, flops
+
+
 def algorithmic_bwd(inp, r):
     """Algorithmic bytes and flops of the single-adapter backward: reads X, W, dY,
     A, B, U, writes dX, dA, dB; flops of dU = s·dY·B^T, the dX GEMM with its adapter
@@ -471,6 +486,7 @@ def measure(name, cx, cpu_budget):
     inp = wl.make_rank_inputs(name, rank)
     T, di, do = inp.T, inp.d_in, inp.d_out
     finetune = inp.dY is not None
+    multi = finetune and inp.n_adapters > 1  # every adapter of a mixed batch trained at once
     K = steps_for(a, name)
     # data parallel: this rank's rows are global rows rank*T.. of one batch, so
     # its dropout mask is the global mask there
@@ -491,7 +507,14 @@ def measure(name, cx, cpu_budget):
         cp = dict(X=d(inp.X), W=d(inp.W), A=d(inp.A_pool), B=d(inp.B_pool),
                   Y=torch.empty(T, do, dtype=torch.bfloat16, device=dev),
                   U=torch.empty(T, r_max, dtype=torch.float32, device=dev) if finetune else None)
-        if finetune:
+        if multi:
+            R = plan.pool_rows
+            grad = torch.empty(R * (di + do), dtype=torch.float32, device=dev)  # dA_pool | dB_pool
+            cp.update(dY=d(inp.dY), dX=torch.empty(T, di, dtype=torch.bfloat16, device=dev), grad=grad,
+                      dA=grad[: R * di].view(R, di), dB=grad[R * di:].view(R, do),
+                      ws=torch.empty(lora.bwd_multi_workspace_size(plan), dtype=torch.uint8, device=dev),
+                      bits=torch.empty(T, -(-di // 32), dtype=torch.int32, device=dev))
+        elif finetune:
             grad = torch.empty(r * (di + do), dtype=torch.float32, device=dev)  # dA | dB, one all-reduce
             cp.update(dY=d(inp.dY), dX=torch.empty(T, di, dtype=torch.bfloat16, device=dev), grad=grad,
                       dA=grad[: r * di].view(r, di), dB=grad[r * di:].view(r, do),
@@ -522,7 +545,10 @@ def measure(name, cx, cpu_budget):
                 lora.dropout_keep_bits(mask_seed, inp.p_drop, copies[nxt]["bits"], di)
             ev_join.record(side)
         lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
-        if finetune:
+        if multi:
+            lora.linear_bwd_multi(plan, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["U"], cp["dY"], cp["dX"],
+                                  cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=mask_seed, keep_bits=bits)
+        elif finetune:
             lora.linear_bwd(cp["X"], cp["W"], cp["A"], cp["B"], float(inp.scale[0]), cp["U"], cp["dY"], cp["dX"],
                             cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=mask_seed, keep_bits=bits)
         if masked:
@@ -533,7 +559,13 @@ def measure(name, cx, cpu_budget):
     # group, 2 reductions; the keep bits of the next copy
     n_groups = -(-r // 64)
     launches_per_step = 2 + int(info["gathers_x"])
-    if finetune:
+    if multi:
+        # [X, dY (, keep bits) sorted copies], U sorted, dU shrink, dX GEMM, 2
+        # contractions, [2 partial reductions], the keep bits
+        bits_gathered = info["gathers_x"] and masked and (-(-di // 32)) % 4 == 0
+        launches_per_step += (2 * info["gathers_x"] + int(bits_gathered) + 4 + 2 * int(plan_partial_rows(plan) > 0)
+                              + int(masked))
+    elif finetune:
         launches_per_step += 2 + int(r % 16 != 0) + 2 * n_groups + 2 + int(masked)
     torch.cuda.synchronize()
     with torch.cuda.stream(cx.stream):
@@ -574,7 +606,7 @@ def measure(name, cx, cpu_budget):
         def burst(gs):
             time.sleep(0.2)
             return cx.timed(replay(gs), K, 0.0)[0]
-        ms_step_burst = burst(graphs) if not (finetune and world > 1) else None
+        ms_step_burst = burst(graphs) if not (finetune and not multi and world > 1) else None
         ms_gemm = burst(ggraphs)
         ms_base = burst(bgraphs)
         assert lora.device_status() == 0
@@ -592,7 +624,8 @@ def measure(name, cx, cpu_budget):
         del ggraphs, bgraphs, tgraphs
 
     with ClockSampler(cx.local_rank) as clk:
-        ms_total, n_regions = cx.timed(replay(graphs, finetune and world > 1), K, 0.0 if a.once else MIN_REGION_S)
+        ms_total, n_regions = cx.timed(replay(graphs, finetune and not multi and world > 1), K,
+                                   0.0 if a.once else MIN_REGION_S)
     clocks = clk.summary()
     value = job_throughput(T, K, world, ms_total)
     entry = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world, "steps": K,
@@ -607,7 +640,10 @@ def measure(name, cx, cpu_budget):
     hbm, tc_burst, tc_sust, src = peaks()
     gb, gf, lb, lf = algorithmic(inp, info)
     t_step = ms_total * 1e-3 / K
-    if finetune:
+    if multi:
+        bb, bfl = algorithmic_bwd_multi(inp, info)
+        lb, lf = lb + bb, lf + bfl
+    elif finetune:
         bb, bfl = algorithmic_bwd(inp, r)
         lb, lf = lb + bb, lf + bfl
     if name in ("decode", "tiny"):
@@ -673,6 +709,20 @@ def measure(name, cx, cpu_budget):
     return entry
 
 
+def plan_partial_rows(plan):
+    """Whether the multi-adapter backward has segments of several pieces (then it
+    launches two more reductions): a segment longer than 1024 sorted tokens, or
+    one whose original tokens are not consecutive in a plan without a sorted copy."""
+    perm, seg = plan.grouping()
+    gathers = plan.info()["gathers_x"]
+    for _, start, length in seg:
+        if length > 1024:
+            return 1
+        if not gathers and length > 1 and np.any(np.diff(perm[start:start + length]) != 1):
+            return 1
+    return 0
+
+
 def measure_e2e(cx, inp, copies, scale, mask_seed, K):
     """The metric through the public API with host buffers (see the module text)."""
     import torch
@@ -722,7 +772,10 @@ def measure_e2e(cx, inp, copies, scale, mask_seed, K):
                 lora.dropout_keep_bits(mask_seed, inp.p_drop, bits, di, stream=s_comp)
             lora.linear_fwd(p, c["X"], c["W"], c["A"], c["B"], scale, c["Y"], p_drop=inp.p_drop,
                             seed=mask_seed, U_save=c["U"], keep_bits=bits)
-            if finetune:
+            if finetune and inp.n_adapters > 1:
+                lora.linear_bwd_multi(p, c["X"], c["W"], c["A"], c["B"], scale, c["U"], c["dY"], c["dX"],
+                                      c["dA"], c["dB"], c["ws"], p_drop=inp.p_drop, seed=mask_seed, keep_bits=bits)
+            elif finetune:
                 lora.linear_bwd(c["X"], c["W"], c["A"], c["B"], float(inp.scale[0]), c["U"], c["dY"],
                                 c["dX"], c["dA"], c["dB"], c["ws"], p_drop=inp.p_drop, seed=mask_seed,
                                 keep_bits=bits)
@@ -872,6 +925,7 @@ def run_lora(a):
         budget = CPU_BUDGET_S["headline" if name in (HEADLINE, a.config) else "other"]
         entries[name] = measure(name, cx, budget)
     if a.config == "all":
+        entries["fleet_finetune"] = measure("fleet_finetune", cx, CPU_BUDGET_S["other"])
         entries["switch"] = measure_switch(cx, CPU_BUDGET_S["other"])
     head = entries[HEADLINE if a.config == "all" else a.config]
     out = {k: head[k] for k in HEAD_KEYS if k in head}

@@ -274,6 +274,43 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
                     size_t workspace_bytes, const uint32_t *keep_bits, lora_stream_t stream);
 
 /* ------------------------------------------------------------------------
+ * lora_linear_bwd_multi — the backward of lora_linear_fwd for a batch that
+ * mixes adapters (multi-adapter fine-tuning: several jobs' adapters trained on
+ * one frozen base in one batch), W frozen. Source: the LoRAFusion explainer,
+ * section 解决什么真问题 (several LoRA jobs sharing one base model) and item 1
+ * (the reparameterisation whose chain rule this is); per token t with adapter a:
+ *   dU[t]  = s_a·dY[t]·B_a^T
+ *   dX[t]  = dY[t]·W^T + D[t] ⊙ (dU[t]·A_a^T)         D = keep mask / (1 - p)
+ *   dA_a   = sum over the tokens of a of (D ⊙ X)[t]^T·dU[t]   (pool layout, as A_pool)
+ *   dB_a   = s_a · sum over the tokens of a of U[t]^T·dY[t]  (pool layout, as B_pool)
+ *
+ *   plan, X, W, A_pool, B_pool, scale, p_drop, seed, keep_bits
+ *           as in lora_linear_fwd (the same plan and mask as the forward)
+ *   U_save  f32 [T, r_max]  the forward's U_save (4-byte aligned)
+ *   dY      bf16 [T, d_out]
+ *   dX      bf16 [T, d_in]   output, original token order
+ *   dA_pool f32 [R, d_in]    output: rows off_a .. off_a + r_a - 1 of every
+ *                            adapter with tokens in the batch (4-byte aligned);
+ *                            rows of adapters without tokens are not written
+ *   dB_pool f32 [R, d_out]   output, likewise
+ *   workspace, workspace_bytes  device scratch of at least
+ *           lora_linear_bwd_multi_workspace_size(plan) bytes, 256-byte aligned,
+ *           caller-owned; contents on entry are ignored
+ * Each adapter's gradient is summed over its tokens in pieces of at most 1024
+ * sorted tokens, in a fixed order: results are deterministic run to run. The
+ * call reads the plan's tables but not its scratch. A segment's last piece may
+ * share a 64-token stage with the next segment's tokens, which enter as zeros:
+ * inputs are assumed finite.
+ * Errors: LORA_ERR_ARG, LORA_ERR_WORKSPACE, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA.
+ * ------------------------------------------------------------------------ */
+size_t lora_linear_bwd_multi_workspace_size(lora_plan_t plan);
+
+int lora_linear_bwd_multi(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
+                          const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed,
+                          const float *U_save, const uint16_t *dY, uint16_t *dX, float *dA_pool, float *dB_pool,
+                          void *workspace, size_t workspace_bytes, const uint32_t *keep_bits, lora_stream_t stream);
+
+/* ------------------------------------------------------------------------
  * lora_linear_bwd_static — lora_linear_bwd without a caller workspace.
  *
  * No counterpart on the pages: this is an integration aid. Some callers cannot

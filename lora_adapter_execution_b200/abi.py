@@ -84,6 +84,9 @@ def load_library():
         "lora_device_status": (ctypes.c_int, [_vp, ctypes.POINTER(ctypes.c_uint32)]),
         "lora_selftest_bounded_wait": (ctypes.c_int, [ctypes.c_uint32, _vp, _vp]),
         "lora_dropout_seed_for_rows": (_u64, [_u64, _i64, _i64]),
+        "lora_linear_bwd_multi_workspace_size": (_sz, [_vp]),
+        "lora_linear_bwd_multi": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp, _vp, _vp,
+                                                 _vp, _sz, _vp, _vp]),
         "lora_switch_create": (ctypes.c_int, [_vp, _i32, _i64, _i64, _i64, _i32, ctypes.POINTER(_vp)]),
         "lora_switch_apply": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]),
         "lora_switch_destroy": (None, [_vp]),
@@ -299,6 +302,30 @@ def linear_bwd(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, workspace, *, p
                                           _ptr(dB), T, d_in, d_out, r, _ptr(workspace), nbytes, _ptr(keep_bits),
                                           _stream(stream)),
            "lora_linear_bwd")
+
+
+def bwd_multi_workspace_size(plan: Plan) -> int:
+    return int(load_library().lora_linear_bwd_multi_workspace_size(plan.handle))
+
+
+def linear_bwd_multi(plan: Plan, X, W, A_pool, B_pool, scale, U_save, dY, dX, dA_pool, dB_pool, workspace, *,
+                     p_drop: float = 0.0, seed: int = 0, keep_bits=None, stream=None):
+    """lora_linear_bwd_multi: the backward of a mixed-adapter batch over its plan
+    (dX, and the gradient rows of every adapter with tokens in dA_pool, dB_pool)."""
+    T, di, do, R = plan.T, plan.d_in, plan.d_out, plan.pool_rows
+    _args("lora_linear_bwd_multi", *_fwd_args(plan, X, A_pool, scale, U_save, keep_bits),
+          ("W", W, (di, do), _BF16, False), ("B_pool", B_pool, (R, do), _BF16, False),
+          ("dY", dY, (T, do), _BF16, False), ("dX", dX, (T, di), _BF16, False),
+          ("dA_pool", dA_pool, (R, di), _F32, False), ("dB_pool", dB_pool, (R, do), _F32, False),
+          ("workspace", workspace, tuple(workspace.shape), (str(workspace.dtype)[6:],), False))
+    if U_save is None:
+        raise LoraError(-1, "lora_linear_bwd_multi: U_save is required")
+    nbytes = workspace.numel() * workspace.element_size()
+    _check(load_library().lora_linear_bwd_multi(plan.handle, _ptr(X), _ptr(W), _ptr(A_pool), _ptr(B_pool), _ptr(scale),
+                                                float(p_drop), int(seed) & (2**64 - 1), _ptr(U_save), _ptr(dY),
+                                                _ptr(dX), _ptr(dA_pool), _ptr(dB_pool), _ptr(workspace), nbytes,
+                                                _ptr(keep_bits), _stream(stream)),
+           "lora_linear_bwd_multi")
 
 
 def linear_bwd_static(X, W, A, B, scale: float, U_save, dY, dX, dA, dB, *, p_drop: float = 0.0,

@@ -54,10 +54,19 @@ constexpr int kBSlot = 4 * 16 * 128;
 constexpr int kGemmThreads = 256;
 constexpr int kGemmWarpW = 6;  // the W-copy warp
 constexpr int kGemmWarpFix = 7;  // the warp that clears B rows of other adapters
+// merge mode: after its adapter blocks each tile's block sequence has two W
+// blocks, the tile's current weights (128 rows x 128 columns each, in the B part
+// of a stage), which the epilogue consumes and releases
+constexpr int kMergeWBlocks = 2;
 constexpr int kGemmBarBytes = 256;
 constexpr int kGemmSmem = 1024 + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16;
 
-enum GemmEpi { kEpiStore = 0, kEpiBwdLora = 1, kEpiMergeAdd = 2 };
+// kEpiStore: out = accumulator. kEpiBwdLora: single-adapter backward, out =
+// accumulator + D ⊙ (dU·A^T) on CUDA cores. kEpiMergeAdd: out += accumulator (in
+// place). kEpiBwdMulti: multi-adapter backward with dropout, out = base
+// accumulator + D ⊙ adapter accumulator (the adapter K blocks go to a second
+// accumulator at TMEM columns 256..511; one accumulator pair, no double buffer).
+enum GemmEpi { kEpiStore = 0, kEpiBwdLora = 1, kEpiMergeAdd = 2, kEpiBwdMulti = 3 };
 constexpr int kEpiRankRegs = 16;  // dU values per row kept in registers by the backward epilogue
 // backward epilogue: the tile's slice of A (ranks < kEpiRankRegs, 256 columns) as
 // fp32 in shared memory, behind the adapter tables
@@ -359,15 +368,9 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int arow = p.a_sorted ? td.row0 : td.contig;
       if (lane == 0) {
         if (arow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; }
-        if (merge) {
-          // the epilogue will read this tile's weights: have L2 fetch them now,
-          // while the stages and the epilogue of the tiles before are in flight
-          const uint32_t bytes = static_cast<uint32_t>(min(kBN, p.N - n0)) * 2u;
-          for (int r = 0; r < td.rows; ++r)
-            bulk_prefetch_l2(p.out + (static_cast<int64_t>(td.contig) + r) * p.N + n0, bytes);
-        }
         const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
-        const int nblk = arow < 0 ? 0 : br.count();
+        const int nmma = br.count();
+        const int nblk = arow < 0 ? 0 : nmma + (merge ? kMergeWBlocks : 0);
         // adapter block descriptors, one load ahead of their use (the adapter
         // blocks come first: block i < naug is adapter block q + i * S)
         const int na = br.naug();
@@ -379,12 +382,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           nvalid = __ldg(&p.augblocks[td.aug0 + q].valid);
         }
         for (int i = 0; i < nblk; ++i) {
-          const int blk = br.block(i, KB);
+          const int blk = i < nmma ? br.block(i, KB) : -1;
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
           const uint32_t a_dst = stage0 + stage * kStageBytes;
           const uint32_t b_dst = a_dst + kStageA;
           const uint32_t fb = full0 + 8 * stage;
-          if (blk < KB) {
+          if (blk < 0) {
+            // merge mode: W block i - nmma, the tile's weights in columns
+            // [n0 + 128h, n0 + 128h + 128) as two 64-column boxes of 128 rows
+            const int h = i - nmma;
+            mbar_arrive_expect_tx(fb, kStageB);
+            tma_load_2d(b_dst, &mapA, fb, n0 + 128 * h, td.contig);
+            tma_load_2d(b_dst + kStageB / 2, &mapA, fb, n0 + 128 * h + 64, td.contig);
+          } else if (blk < KB) {
             // the W tile of this stage comes from warp kGemmWarpW's copy; the
             // expected bytes cover both (a copy may land before this arrive:
             // the phase cannot complete while the arrival is pending)
@@ -445,9 +455,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const int n0 = nt * kBN;
         const int arow = p.a_sorted ? td.row0 : td.contig;
         const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
-        const int nblk = arow < 0 ? 0 : br.count();
+        const int nmma = br.count();
+        const int nblk = arow < 0 ? 0 : nmma + (merge ? kMergeWBlocks : 0);
         for (int i = 0; i < nblk; ++i) {
-          const int blk = br.block(i, KB);
+          const int blk = i < nmma ? br.block(i, KB) : KB;  // merge W blocks: nothing to copy here
           if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { *abort_flag = 1; break; }
           if (blk < KB) {
             const uint32_t b_dst = stage0 + stage * kStageBytes + kStageA;
@@ -488,16 +499,17 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const TileDesc td = tile_desc(mt);
         const int arow = p.a_sorted ? td.row0 : td.contig;
         const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
-        const int nblk = arow < 0 ? 0 : br.count();
+        const int nmma = br.count();
+        const int nblk = arow < 0 ? 0 : nmma + (merge ? kMergeWBlocks : 0);
         bool ok = true;
         for (int i = 0; i < nblk; ++i) {
-          const int blk = br.block(i, KB);
+          const int blk = i < nmma ? br.block(i, KB) : -1;
           if (!__all_sync(0xFFFFFFFFu, mbar_wait(full0 + 8 * stage, phase))) {
             if (lane == 0) *abort_flag = 1;
             ok = false;
             break;
           }
-          if (!B_KMAJOR && blk >= KB) {
+          if (blk >= KB) {
             const uint32_t vw = bvalid[stage];
             const int nsl = static_cast<int>(vw >> 20);
             uint8_t *bsp = smem + stage * kStageBytes + kStageA;
@@ -528,6 +540,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     if (lane == 0) {
       // ------------------------------------------------------------ MMA issuer
       constexpr uint32_t kIdesc = idesc_bf16(kBM, kBN, false, !B_KMAJOR);
+      constexpr uint32_t kIdescAug = idesc_bf16(kBM, kBN, false, true);  // adapter B slots are MN-major
+      constexpr bool kDual = EPI == kEpiBwdMulti;
       // stage 0's descriptors: A K-major (SW128, 8-row groups 1 KB apart, a K16
       // step 32 bytes on); B K-major likewise, or MN-major with 64-column blocks
       // 8 KB apart and a K16 step 16 rows (2 KB) on
@@ -548,12 +562,23 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tile_coords(tile, p, mt, nt);
         const int kaug = merge ? p.merge_kaug : (p.tiles ? p.tiles[mt].kaug : 0);
         const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
-        const int nblk = br.count();
+        const int nmma = br.count();
+        const int nblk = nmma + (merge ? kMergeWBlocks : 0);
         if (!mbar_wait(acce0 + 8 * acc, aphase ^ 1)) { *abort_flag = 1; break; }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * kBN;
+        const uint32_t d_aug = kDual ? tmem_base + kBN : d_tmem;
+        // the first base block starts the base accumulator (after the adapter
+        // blocks when they have their own)
+        const int first_base = kDual ? br.naug() : 0;
         bool ok = true;
         for (int i = 0; i < nblk; ++i) {
+          if (i >= nmma) {
+            // merge mode's W blocks: no MMA; the epilogue reads and releases them
+            if (!mbar_wait(ready0 + 8 * stage, phase)) { *abort_flag = 1; ok = false; break; }
+            if (++stage == kGemmStages) { stage = 0; phase ^= 1; }
+            continue;
+          }
           const int blk = br.block(i, KB);
           if (!mbar_wait(ready0 + 8 * stage, phase)) { *abort_flag = 1; ok = false; break; }
           tc_fence_after();
@@ -563,7 +588,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
           const uint64_t ad = adesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
           const uint64_t bd = bdesc0 + static_cast<uint64_t>(stage * (kStageBytes >> 4));
           if (blk < KB) {
-            umma_bf16(d_tmem, ad, bd, kIdesc, i > 0 ? 1u : 0u);
+            umma_bf16(d_tmem, ad, bd, kIdesc, i > first_base ? 1u : 0u);
             umma_bf16_acc(d_tmem, ad + kAStep, bd + kBStep, kIdesc);
             umma_bf16_acc(d_tmem, ad + 2 * kAStep, bd + 2 * kBStep, kIdesc);
             umma_bf16_acc(d_tmem, ad + 3 * kAStep, bd + 3 * kBStep, kIdesc);
@@ -574,9 +599,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             const uint32_t map = bmap[stage];
             const uint32_t b_s = stage0 + stage * kStageBytes + kStageA;
             for (int qq = 0; qq < steps; ++qq) {
-              const uint64_t bq = B_KMAJOR ? bd + qq * kAStep
-                                           : sdesc_sw128(b_s + ((map >> (2 * qq)) & 3u) * kBSlot, 2048, 1024);
-              umma_bf16(d_tmem, ad + qq * kAStep, bq, kIdesc, (i > 0 || qq > 0) ? 1u : 0u);
+              const uint64_t bq = sdesc_sw128(b_s + ((map >> (2 * qq)) & 3u) * kBSlot, 2048, 1024);
+              umma_bf16(d_aug, ad + qq * kAStep, bq, kIdescAug, (i > 0 || qq > 0) ? 1u : 0u);
             }
           }
           umma_commit(empty0 + 8 * stage);
@@ -584,7 +608,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         if (!ok) break;
         umma_commit(accf0 + 8 * acc);
-        if (++acc == 2) { acc = 0; aphase ^= 1; }
+        if (kDual) aphase ^= 1;  // one accumulator pair: buffer 0 every tile
+        else if (++acc == 2) { acc = 0; aphase ^= 1; }
       }
     }
   } else {
@@ -594,6 +619,8 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     float *as = reinterpret_cast<float *>(smem + kGemmStages * kStageBytes + kGemmBarBytes + kBM * 16);
     int acc = 0;
     uint32_t aphase = 0;
+    int ep_stage = 0;  // merge mode: the epilogue's walk of the stage ring
+    uint32_t ep_phase = 0;
     if (split) {
       // the split-K tail's table entry and output row, loaded while the K loop runs
       int mt = 0, nt = 0;
@@ -609,51 +636,107 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // the backward's warps leave together (epi_bar_or), so its loop ignores the
     // flag here and tests it at the barrier
     int tile;
-    for (int k = 0; (EPI == kEpiBwdLora || !*abort_flag) && cta_tile(p, k, tile0, tile_step, n_tiles, tile); ++k) {
+    for (int k = 0; (EPI == kEpiBwdLora || EPI == kEpiMergeAdd || !*abort_flag) &&
+                    cta_tile(p, k, tile0, tile_step, n_tiles, tile);
+         ++k) {
       int mt, nt;
       tile_coords(tile, p, mt, nt);
       const TileDesc td = tile_desc(mt);
       if constexpr (EPI == kEpiMergeAdd) {
-        // W <- bf16(W + accumulator), in place: this row's current weights are
-        // loaded before the accumulator is waited for, so the loads overlap the
-        // tile's MMAs (each element is read and written by this thread only)
+        // W <- bf16(W + accumulator), in place. The tile's current weights come
+        // through the stage ring as its two W blocks (after its adapter blocks):
+        // walk the ring as the producer fills it, wait for each W block, add,
+        // store, and release the stage.
+        const int nmma = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count();
+        for (int i = 0; i < nmma; ++i)
+          if (++ep_stage == kGemmStages) { ep_stage = 0; ep_phase ^= 1; }
         const bool valid = row < td.rows;
         const int64_t orow = static_cast<int64_t>(td.contig) + row;
-        uint4 wv[kBN / 8];
-#pragma unroll
-        for (int c8 = 0; c8 < kBN / 8; ++c8) {
-          const int col = nt * kBN + c8 * 8;
-          wv[c8] = (valid && col < p.N) ? *reinterpret_cast<const uint4 *>(p.out + orow * p.N + col)
-                                        : make_uint4(0u, 0u, 0u, 0u);
-        }
-        if (!mbar_wait(accf0 + 8 * acc, aphase)) { *abort_flag = 1; break; }
+        // every wait is agreed by the four warps (bar.red.or), so that none
+        // leaves while the others wait at the barrier below
+        if (epi_bar_or(!mbar_wait(accf0 + 8 * acc, aphase) || *abort_flag)) { *abort_flag = 1; break; }
         tc_fence_after();
+        bool ok = true;
+        for (int h = 0; h < kMergeWBlocks; ++h) {
+          if (epi_bar_or(!mbar_wait(full0 + 8 * ep_stage, ep_phase) || *abort_flag)) {
+            *abort_flag = 1;
+            ok = false;
+            break;
+          }
+          const uint8_t *wst = smem + ep_stage * kStageBytes + kStageA;  // [2 halves][128 rows][64 cols], SW128
 #pragma unroll
+          for (int cc = 0; cc < 4; ++cc) {
+            const int c = 4 * h + cc;
+            uint32_t v[32];
+            tmem_ld32(tmem_base + ((quarter * 32) << 16) + acc * kBN + c * 32, v);
+            tmem_wait_ld();
+            const int col0 = nt * kBN + c * 32;
+            if (valid && col0 < p.N) {
+              const uint8_t *wrow = wst + (cc >> 1) * (kStageB / 2);
+              uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * p.N + col0);
+#pragma unroll
+              for (int j = 0; j < 4; ++j) {
+                if (col0 + 8 * j < p.N) {
+                  const uint4 w = *reinterpret_cast<const uint4 *>(wrow + sw128_offset(row, (cc & 1) * 32 + 8 * j));
+                  const uint32_t *vv = v + 8 * j;
+                  uint4 o;
+                  o.x = pack_bf16x2(bf16_lo(w.x) + __uint_as_float(vv[0]), bf16_hi(w.x) + __uint_as_float(vv[1]));
+                  o.y = pack_bf16x2(bf16_lo(w.y) + __uint_as_float(vv[2]), bf16_hi(w.y) + __uint_as_float(vv[3]));
+                  o.z = pack_bf16x2(bf16_lo(w.z) + __uint_as_float(vv[4]), bf16_hi(w.z) + __uint_as_float(vv[5]));
+                  o.w = pack_bf16x2(bf16_lo(w.w) + __uint_as_float(vv[6]), bf16_hi(w.w) + __uint_as_float(vv[7]));
+                  dst[j] = o;
+                }
+              }
+            }
+          }
+          epi_bar();  // every thread's reads of the W block are done
+          if (threadIdx.x == 64) mbar_arrive(empty0 + 8 * ep_stage);
+          if (++ep_stage == kGemmStages) { ep_stage = 0; ep_phase ^= 1; }
+        }
+        if (!ok) break;
+        tc_fence_before();
+        mbar_arrive(acce0 + 8 * acc);
+        if (++acc == 2) { acc = 0; aphase ^= 1; }
+        continue;
+      }
+      if constexpr (EPI == kEpiBwdMulti) {
+        // dX = dY·W^T (TMEM columns of buffer 0) + keep / (1 - p) * sum over the
+        // row's adapter of dU·A^T (columns 256..511)
+        if (!mbar_wait(accf0, aphase)) { *abort_flag = 1; break; }
+        tc_fence_after();
+        const bool valid = row < td.rows;
+        int64_t orig = 0;
+        if (valid) orig = td.contig >= 0 ? td.contig + row : p.perm[td.row0 + row];
         for (int c = 0; c < kBN / 32; ++c) {
-          uint32_t v[32];
-          tmem_ld32(tmem_base + ((quarter * 32) << 16) + acc * kBN + c * 32, v);
+          uint32_t v[32], w[32];
+          tmem_ld32(tmem_base + ((quarter * 32) << 16) + c * 32, v);
+          tmem_ld32(tmem_base + ((quarter * 32) << 16) + kBN + c * 32, w);
           tmem_wait_ld();
           const int col0 = nt * kBN + c * 32;
           if (valid && col0 < p.N) {
-            uint4 *dst = reinterpret_cast<uint4 *>(p.out + orow * p.N + col0);
+            const uint32_t keep = p.keep_bits ? __ldg(p.keep_bits + orig * p.wpr + (col0 >> 5))
+                                              : keep_mask32(p.seed, p.thr, static_cast<uint64_t>(orig * p.N + col0));
+            float f[32];
+#pragma unroll
+            for (int i = 0; i < 32; ++i)
+              f[i] = __uint_as_float(v[i]) + (((keep >> i) & 1u) ? p.inv_keep * __uint_as_float(w[i]) : 0.f);
+            uint4 *dst = reinterpret_cast<uint4 *>(p.out + orig * p.N + col0);
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
               if (col0 + 8 * j < p.N) {
-                const uint4 w = wv[c * 4 + j];
-                const uint32_t *vv = v + 8 * j;
                 uint4 o;
-                o.x = pack_bf16x2(bf16_lo(w.x) + __uint_as_float(vv[0]), bf16_hi(w.x) + __uint_as_float(vv[1]));
-                o.y = pack_bf16x2(bf16_lo(w.y) + __uint_as_float(vv[2]), bf16_hi(w.y) + __uint_as_float(vv[3]));
-                o.z = pack_bf16x2(bf16_lo(w.z) + __uint_as_float(vv[4]), bf16_hi(w.z) + __uint_as_float(vv[5]));
-                o.w = pack_bf16x2(bf16_lo(w.w) + __uint_as_float(vv[6]), bf16_hi(w.w) + __uint_as_float(vv[7]));
+                o.x = pack_bf16x2(f[8 * j + 0], f[8 * j + 1]);
+                o.y = pack_bf16x2(f[8 * j + 2], f[8 * j + 3]);
+                o.z = pack_bf16x2(f[8 * j + 4], f[8 * j + 5]);
+                o.w = pack_bf16x2(f[8 * j + 6], f[8 * j + 7]);
                 dst[j] = o;
               }
             }
           }
         }
         tc_fence_before();
-        mbar_arrive(acce0 + 8 * acc);
-        if (++acc == 2) { acc = 0; aphase ^= 1; }
+        mbar_arrive(acce0);
+        aphase ^= 1;
         continue;
       }
       if (EPI == kEpiBwdLora) {

@@ -13,6 +13,7 @@ constexpr int kAugBlock = 64;    // augmented-K columns per shrink-output block
 constexpr int kAugBlockBytes = kTileM * kAugBlock * 2;  // 16 KB, one swizzled smem image
 constexpr int kShrinkN = 64;     // rank columns per shrink work unit
 constexpr int kUnitRows = 32;    // token rows per shrink work unit (a chunk's rows are split)
+constexpr int kPieceTokens = 1024;  // tokens per piece of a segment in the backward's per-adapter contractions
 
 // One 128-token output tile of the sorted order.
 struct TileDesc {
@@ -76,6 +77,23 @@ struct alignas(16) UnitDesc {
   int64_t uofs;       // byte offset of the tile's s*U image in the plan scratch
 };
 
+// A piece of one segment (consecutive sorted tokens of one adapter) for the
+// multi-adapter backward's contractions dA_a, dB_a: at most kPieceTokens tokens.
+// A segment of one piece writes its adapter's gradient rows itself; the pieces
+// of a longer segment write partial sums (partial_row = first row of this
+// piece's r_a rows in the partial buffer) that a reduction adds in piece order.
+struct alignas(16) PieceDesc {
+  int32_t start, len;   // sorted positions
+  int32_t in_row;       // row of the piece's first token in X / dY: its sorted position when the
+                        // plan gathers (the backward reads sorted copies), else its original
+                        // index (the piece is then a run of consecutive original tokens)
+  int32_t adapter, rank, pool_row;
+  int32_t seg_pieces;   // pieces of the segment (1: direct write)
+  int32_t first_piece;  // index of the segment's first piece
+  int32_t partial_row;  // -1 when seg_pieces == 1
+  int32_t pad_[3];
+};
+
 // One term of a fused adapter switch: adapter rows [pool_row, pool_row + rank)
 // of every layer's pools, weighted by coef, as augmented columns
 // [kofs, kofs + 2*kc) of every tile (hi part, then lo part).
@@ -99,6 +117,8 @@ struct HostPlan {
   std::vector<UnitDesc> units;
   std::vector<AugBlockDesc> augblocks;
   std::vector<int32_t> mt_order;  // m-tiles by decreasing adapter work (stable)
+  std::vector<PieceDesc> pieces;  // the backward's per-segment pieces, segment by segment
+  int64_t partial_rows = 0;       // rows of the partial buffer (pieces of multi-piece segments)
   int32_t r_max = 0;
   int64_t sum_r_used = 0, sum_r_tokens = 0, aug_k_total = 0;
   int64_t scratch_bytes = 0;

@@ -63,6 +63,10 @@ int device_state(DeviceState **out) {
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmemBwd) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_gemm_kernel<false, kEpiMergeAdd>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_gemm_kernel<true, kEpiStore>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_gemm_kernel<true, kEpiBwdMulti>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_shrink_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sk_smem(4)) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_shrink_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -276,6 +280,7 @@ struct lora_plan {
   const UnitDesc *d_units = nullptr;
   const int32_t *d_mt_order = nullptr;
   const AugBlockDesc *d_augblocks = nullptr;
+  const PieceDesc *d_pieces = nullptr;
   std::vector<int32_t> sched;           // the fused GEMM's per-CTA tiles (build_schedule), if persistent
   const int32_t *d_sched = nullptr;     // off[grid + 1] | tiles
   void *stage[2] = {nullptr, nullptr};  // pinned host staging of the tables, used in turn
@@ -294,6 +299,54 @@ namespace {
 bool on_plan_device(const lora_plan *pl) {
   int d = -1;
   return cudaGetDevice(&d) == cudaSuccess && d == pl->device;
+}
+
+// The shrink over the plan's units (one CTA cluster per unit): In rows by mIn
+// (box {64, 16}), factor rows by mF (box {64, 16}), sp.K the contraction length;
+// the caller fills the rest of sp (scale, mask, outputs). Launched with
+// programmatic stream serialization.
+int launch_unit_shrink(DeviceState *ds, const lora_plan *plan, const CUtensorMap &mIn, const CUtensorMap &mF,
+                       const CUtensorMap &mBits, ShrinkParams sp, lora_stream_t stream) {
+  const HostPlan &hp = plan->hp;
+  sp.mode = 0;
+  sp.T = static_cast<int32_t>(hp.T);
+  const int n_units = static_cast<int>(hp.units.size());
+  // the build (and cluster size) with the fewest stages on the critical path
+  int max_nn = 0;
+  for (const UnitDesc &u : hp.units) max_nn = std::max(max_nn, static_cast<int>(u.nn));
+  int ks = 1;
+  const int max_nb16 = shrink_build(n_units, sp.K, ds->num_sms, max_nn, &ks);
+  int64_t slice = (sp.K + ks - 1) / ks;
+  slice = (slice + kSkBK - 1) / kSkBK * kSkBK;
+  sp.ksplit = ks;
+  sp.kslice = static_cast<int32_t>(slice);
+  sp.units = plan->d_units;
+  sp.chunks = plan->d_chunks;
+  sp.tiles = plan->d_tiles;
+  sp.perm = plan->d_perm;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(n_units * ks));
+  cfg.blockDim = dim3(kSkThreads);
+  cfg.dynamicSmemBytes = sk_smem(max_nb16);
+  cfg.stream = stream;
+  // programmatic serialization: the shrink's setup (barriers, its plan entry)
+  // overlaps the end of the kernel before it; it waits in pdl_wait before
+  // touching its inputs or any output
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = ks;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  if (cudaLaunchKernelEx(&cfg, max_nb16 <= 2 ? lora_shrink_kernel<2> : lora_shrink_kernel<4>, mIn, mF, mBits,
+                         sp) != cudaSuccess) {
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  return LORA_OK;
 }
 }  // namespace
 
@@ -335,6 +388,7 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
   const size_t b_units = up(sizeof(UnitDesc) * hp.units.size());
   const size_t b_order = up(sizeof(int32_t) * hp.mt_order.size());
   const size_t b_aug = up(sizeof(AugBlockDesc) * hp.augblocks.size());
+  const size_t b_pieces = up(sizeof(PieceDesc) * hp.pieces.size());
   // the persistent fused GEMM's tile schedule (its grid and tile order as launched)
   pl->sched.clear();
   {
@@ -345,7 +399,7 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
       build_schedule(hp, std::min(ds->num_sms, n_tiles), default_group_m(n_mt, hp.d_in), pl->sched);
   }
   const size_t b_sched = up(sizeof(int32_t) * pl->sched.size());
-  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug + b_sched;
+  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug + b_pieces + b_sched;
   auto release = [&]() {
     if (pl->dev) cudaFree(pl->dev);
     if (pl->scratch) cudaFree(pl->scratch);
@@ -399,7 +453,9 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
   pl->d_mt_order = reinterpret_cast<const int32_t *>(base + b_perm + b_tiles + b_chunks + b_units);
   pl->d_augblocks =
       reinterpret_cast<const AugBlockDesc *>(base + b_perm + b_tiles + b_chunks + b_units + b_order);
-  uint8_t *sched_dst = base + b_perm + b_tiles + b_chunks + b_units + b_order + b_aug;
+  uint8_t *pieces_dst = base + b_perm + b_tiles + b_chunks + b_units + b_order + b_aug;
+  pl->d_pieces = reinterpret_cast<const PieceDesc *>(pieces_dst);
+  uint8_t *sched_dst = pieces_dst + b_pieces;
   pl->d_sched = pl->sched.empty() ? nullptr : reinterpret_cast<const int32_t *>(sched_dst);
   // The tables go to the device in one copy from one of the plan's two pinned
   // staging buffers, laid out as the device buffer. A staging buffer is refilled
@@ -432,6 +488,7 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
     put(b_perm + b_tiles + b_chunks + b_units, hp.mt_order.data(), sizeof(int32_t) * hp.mt_order.size());
     put(b_perm + b_tiles + b_chunks + b_units + b_order, hp.augblocks.data(),
         sizeof(AugBlockDesc) * hp.augblocks.size());
+    put(static_cast<size_t>(pieces_dst - base), hp.pieces.data(), sizeof(PieceDesc) * hp.pieces.size());
     put(static_cast<size_t>(sched_dst - base), pl->sched.data(), sizeof(int32_t) * pl->sched.size());
     ok &= cudaMemcpyAsync(base, h, total, cudaMemcpyHostToDevice, stream) == cudaSuccess;
     ok &= cudaEventRecord(pl->stage_ev[k], stream) == cudaSuccess;
@@ -550,22 +607,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   if (!ok) return LORA_ERR_ARG;
   ShrinkParams sp{};
   sp.mode = 0;
-  sp.T = static_cast<int32_t>(hp.T);
   sp.K = static_cast<int32_t>(hp.d_in);
-  const int n_units = static_cast<int>(hp.units.size());
-  // the build (and cluster size) with the fewest stages on the critical path
-  int max_nn = 0;
-  for (const UnitDesc &u : hp.units) max_nn = std::max(max_nn, static_cast<int>(u.nn));
-  int ks = 1;
-  const int max_nb16 = shrink_build(n_units, hp.d_in, ds->num_sms, max_nn, &ks);
-  int64_t slice = (hp.d_in + ks - 1) / ks;
-  slice = (slice + kSkBK - 1) / kSkBK * kSkBK;
-  sp.ksplit = ks;
-  sp.kslice = static_cast<int32_t>(slice);
-  sp.units = plan->d_units;
-  sp.chunks = plan->d_chunks;
-  sp.tiles = plan->d_tiles;
-  sp.perm = plan->d_perm;
   sp.scale = scale;
   sp.thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
   sp.keep_bits = sp.thr ? keep_bits : nullptr;  // no mask without dropout
@@ -589,23 +631,6 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
   sp.x_sorted = Xs ? 1 : 0;
   sp.U_save = U_save;
   sp.r_max = hp.r_max;
-  cudaLaunchConfig_t cfg{};
-  cfg.gridDim = dim3(static_cast<unsigned>(n_units * ks));
-  cfg.blockDim = dim3(kSkThreads);
-  cfg.dynamicSmemBytes = sk_smem(max_nb16);
-  cfg.stream = stream;
-  // programmatic serialization: the shrink's setup (barriers, its plan entry)
-  // overlaps the end of the kernel before it; it waits in pdl_wait before
-  // touching X or any output
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = ks;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[1].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
   if (Xs) {
     // sorted copy of X first (the shrink and the fused GEMM read token tiles from it)
     const int64_t pieces = hp.T * (hp.d_in / 8);
@@ -613,12 +638,7 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
     lora_gather_rows_kernel<<<blocks, 256, 0, stream>>>(X, plan->d_perm, Xs, hp.T, hp.d_in);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
-  if (cudaLaunchKernelEx(&cfg, max_nb16 <= 2 ? lora_shrink_kernel<2> : lora_shrink_kernel<4>, mX16, mA16, mBits16,
-                         sp) != cudaSuccess) {
-    cudaGetLastError();
-    return LORA_ERR_CUDA;
-  }
-  return LORA_OK;
+  return launch_unit_shrink(ds, plan, mX16, mA16, mBits16, sp, stream);
 }
 
 int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *B_pool, uint16_t *Y,
@@ -906,7 +926,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
       tp.partial = pdB;
       dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
       const int smem_b = 1024 + tc_stages(w, false) * tc_stage_bytes(w, false) + 2 * kTcMaxStages * 8;
-      lora_tcontract_kernel<<<grid_b, kTcThreads, smem_b, stream>>>(mdY64, mU, mBits, tp);
+      lora_tcontract_kernel<<<grid_b, kTcThreads, smem_b, stream>>>(mdY64, mU, mBits, mU, mU, mU, tp);
       tp.N = static_cast<int32_t>(d_in);
       tp.thr = thr;
       tp.seed = seed;
@@ -916,7 +936,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
       tp.wpr = (d_in + 31) / 32;
       tp.partial = pdA;
       dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
-      lora_tcontract_kernel<<<grid_a, kTcThreads, smem_a, stream>>>(mX64, mdU, mBits, tp);
+      lora_tcontract_kernel<<<grid_a, kTcThreads, smem_a, stream>>>(mX64, mdU, mBits, mdU, mdU, mdU, tp);
     }
     const int64_t nb = static_cast<int64_t>(r) * d_out;
     const int64_t na = static_cast<int64_t>(r) * d_in;
@@ -924,6 +944,238 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
         pdB, static_cast<int>(S), nb, scale, dB);
     lora_reduce_splits_kernel<<<static_cast<unsigned>(std::min<int64_t>((na + 255) / 256, 4096)), 256, 0, stream>>>(
         pdA, static_cast<int>(S), na, inv_keep, dA);
+  }
+  return launch_status();
+}
+
+
+// Workspace of lora_linear_bwd_multi, in this order (each part 256-byte aligned):
+// s·dU images (the plan's image layout) | sorted X, sorted dY, sorted keep bits
+// (when the plan gathers) | G = dY·B_a^T and U, both [T, rp] fp32 in sorted
+// order (rp = r_max rounded up to 16) | dA, dB partial rows of multi-piece
+// segments.
+namespace {
+struct BwdMultiLayout {
+  int64_t img, xs, dys, bits, g, u, pda, pdb, total;
+};
+BwdMultiLayout bwd_multi_layout(const HostPlan &hp) {
+  auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
+  const bool gathers = hp.xs_offset >= 0;
+  const int64_t rp = (hp.r_max + 15) / 16 * 16;
+  const int64_t wpr = (hp.d_in + 31) / 32;
+  BwdMultiLayout L{};
+  int64_t o = 0;
+  L.img = o;
+  o += up(gathers ? hp.xs_offset : hp.scratch_bytes);
+  L.xs = gathers ? o : -1;
+  if (gathers) o += up(hp.T * hp.d_in * 2);
+  L.dys = gathers ? o : -1;
+  if (gathers) o += up(hp.T * hp.d_out * 2);
+  L.bits = gathers ? o : -1;
+  if (gathers) o += up(hp.T * wpr * 4);
+  L.g = o;
+  o += up(hp.T * rp * 4);
+  L.u = o;
+  o += up(hp.T * rp * 4);
+  L.pda = o;
+  o += up(hp.partial_rows * hp.d_in * 4);
+  L.pdb = o;
+  o += up(hp.partial_rows * hp.d_out * 4);
+  L.total = o;
+  return L;
+}
+}  // namespace
+
+size_t lora_linear_bwd_multi_workspace_size(lora_plan_t plan) {
+  if (!plan) return 0;
+  return static_cast<size_t>(bwd_multi_layout(plan->hp).total);
+}
+
+int lora_linear_bwd_multi(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
+                          const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed,
+                          const float *U_save, const uint16_t *dY, uint16_t *dX, float *dA_pool, float *dB_pool,
+                          void *workspace, size_t workspace_bytes, const uint32_t *keep_bits, lora_stream_t stream) {
+  if (!plan || !plan->dev || !X || !W || !A_pool || !B_pool || !scale || !U_save || !dY || !dX || !dA_pool ||
+      !dB_pool)
+    return LORA_ERR_ARG;
+  if (!on_plan_device(plan)) return LORA_ERR_ARG;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(A_pool) || !aligned16(B_pool) || !aligned16(dY) ||
+      !aligned16(dX) || (reinterpret_cast<uintptr_t>(U_save) & 3u) || (reinterpret_cast<uintptr_t>(dA_pool) & 3u) ||
+      (reinterpret_cast<uintptr_t>(dB_pool) & 3u) || (reinterpret_cast<uintptr_t>(keep_bits) & 3u))
+    return LORA_ERR_ARG;
+  if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
+  const HostPlan &hp = plan->hp;
+  if (hp.pieces.size() > 65535) return LORA_ERR_ARG;  // one grid row per piece
+  const BwdMultiLayout Lw = bwd_multi_layout(hp);
+  if (!workspace || workspace_bytes < static_cast<size_t>(Lw.total) ||
+      (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return LORA_ERR_WORKSPACE;
+  DeviceState *ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LORA_OK) return rc;
+
+  const int64_t T = hp.T, d_in = hp.d_in, d_out = hp.d_out;
+  const int64_t R = hp.offsets[hp.n_adapters];
+  const int rp = (hp.r_max + 15) / 16 * 16;
+  const int64_t wpr = (d_in + 31) / 32;
+  const bool gathers = hp.xs_offset >= 0;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  uint8_t *img = ws + Lw.img;
+  const uint16_t *Xr = gathers ? reinterpret_cast<const uint16_t *>(ws + Lw.xs) : X;
+  const uint16_t *dYr = gathers ? reinterpret_cast<const uint16_t *>(ws + Lw.dys) : dY;
+  float *G = reinterpret_cast<float *>(ws + Lw.g);
+  float *Us = reinterpret_cast<float *>(ws + Lw.u);
+  float *pdA = reinterpret_cast<float *>(ws + Lw.pda);
+  float *pdB = reinterpret_cast<float *>(ws + Lw.pdb);
+  const uint64_t thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
+  const float inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
+  const uint32_t *bits = thr ? keep_bits : nullptr;
+  // keep bits for the dA contraction: rows in the order of its In rows (sorted
+  // when the plan gathers), staged through TMA when rows are 16-byte multiples
+  const bool bits_tc = bits && wpr % 4 == 0;
+  const uint32_t *bits_in = gathers && bits_tc ? reinterpret_cast<const uint32_t *>(ws + Lw.bits) : bits;
+
+  auto grid_for = [&](int64_t n) {
+    return static_cast<unsigned>(std::min<int64_t>((n + 255) / 256, 16 * ds->num_sms));
+  };
+  // sorted copies of X, dY (and the keep bits) when the plan's tiles are not runs
+  if (gathers) {
+    lora_gather_rows_kernel<<<grid_for(T * (d_in / 8)), 256, 0, stream>>>(X, plan->d_perm,
+                                                                         const_cast<uint16_t *>(Xr), T, d_in);
+    lora_gather_rows_kernel<<<grid_for(T * (d_out / 8)), 256, 0, stream>>>(dY, plan->d_perm,
+                                                                          const_cast<uint16_t *>(dYr), T, d_out);
+    if (bits_tc)
+      lora_gather_rows_kernel<<<grid_for(T * wpr / 4), 256, 0, stream>>>(
+          reinterpret_cast<const uint16_t *>(bits), plan->d_perm,
+          reinterpret_cast<uint16_t *>(const_cast<uint32_t *>(bits_in)), T, 2 * wpr);
+  }
+  // U in sorted order, rows padded to rp
+  lora_gather_pad_kernel<<<grid_for(T * rp), 256, 0, stream>>>(U_save, hp.r_max, plan->d_perm, Us, rp, T);
+  if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+
+  // dU: the plan's shrink units over dY against B_pool: s_a·dU images (hi/lo,
+  // the dX GEMM's adapter operand) and G = dY·B_a^T in sorted order
+  {
+    CUtensorMap mdY16, mB16;
+    if (!make_map(&mdY16, dYr, d_out, T, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mB16, B_pool, d_out, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B))
+      return LORA_ERR_ARG;
+    ShrinkParams sp{};
+    sp.K = static_cast<int32_t>(d_out);
+    sp.scale = scale;
+    sp.inv_keep = 1.0f;
+    sp.uimg = img;
+    sp.x_sorted = gathers ? 1 : 0;
+    sp.U_save = G;
+    sp.r_max = rp;
+    sp.u_sorted = 1;
+    rc = launch_unit_shrink(ds, plan, mdY16, mB16, mdY16, sp, stream);
+    if (rc != LORA_OK) return rc;
+  }
+  // dX = dY·W^T + D ⊙ (s_a·dU·A_a^T): the fused GEMM over the plan's tiles, W^T a
+  // K-major operand, the adapter blocks A_pool rows (into a second accumulator,
+  // masked in the epilogue, when there is dropout)
+  {
+    CUtensorMap mdY128, mWt, mAl;
+    const bool b3d = d_in % 64 == 0;
+    bool ok = make_map(&mdY128, dYr, d_out, T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              make_map(&mWt, W, d_out, d_in, 64, 256, CU_TENSOR_MAP_SWIZZLE_128B) &&
+              (b3d ? make_map_blocks(&mAl, A_pool, d_in, R, 16, kBN / 64)
+                   : make_map(&mAl, A_pool, d_in, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B));
+    if (!ok) return LORA_ERR_ARG;
+    GemmParams gp{};
+    gp.b3d = b3d ? 1 : 0;
+    gp.T = static_cast<int32_t>(T);
+    gp.K = static_cast<int32_t>(d_out);
+    gp.N = static_cast<int32_t>(d_in);
+    gp.n_mt = static_cast<int32_t>(hp.tiles.size());
+    gp.n_nt = static_cast<int32_t>((d_in + kBN - 1) / kBN);
+    gp.tiles = plan->d_tiles;
+    gp.chunks = plan->d_chunks;
+    gp.perm = plan->d_perm;
+    gp.uimg = img;
+    gp.mt_order = plan->d_mt_order;
+    gp.augblocks = plan->d_augblocks;
+    gp.a_sorted = gathers ? 1 : 0;
+    gp.out = reinterpret_cast<__nv_bfloat16 *>(dX);
+    gp.seed = seed;
+    gp.thr = thr;
+    gp.keep_bits = bits;
+    gp.wpr = wpr;
+    gp.inv_keep = inv_keep;
+    gp.ksplit = 1;
+    gp.group_m = default_group_m(gp.n_mt, gp.K);
+    const int n_tiles = gp.n_mt * gp.n_nt;
+    const int grid = std::min(ds->num_sms, n_tiles);
+    if (plan->d_sched && d_in == d_out && static_cast<int>(plan->sched.size()) - n_tiles - 1 == grid &&
+        default_group_m(gp.n_mt, d_in) == gp.group_m) {
+      gp.sched_off = plan->d_sched;  // the forward's per-CTA tile lists fit this grid and tile order
+      gp.sched_tiles = plan->d_sched + grid + 1;
+    }
+    if (thr)
+      lora_gemm_kernel<true, kEpiBwdMulti><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mAl, gp);
+    else
+      lora_gemm_kernel<true, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mAl, gp);
+    if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+  }
+  // dB_a = s_a·U^T·dY and dA_a = s_a·(D ⊙ X)^T·G over each segment's pieces, then
+  // the multi-piece segments' partial sums
+  {
+    CUtensorMap mIn64b, mIn64a, mBits = {};
+    if (!make_map(&mIn64b, dYr, d_out, T, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B) ||
+        !make_map(&mIn64a, Xr, d_in, T, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B))
+      return LORA_ERR_ARG;
+    CUtensorMap mU[4], mG[4];
+    for (int w = 0; w < 4; ++w)
+      if (!make_map_f32(&mU[w], Us, rp, T, 16 * (w + 1), 64) || !make_map_f32(&mG[w], G, rp, T, 16 * (w + 1), 64))
+        return LORA_ERR_ARG;
+    bool use_bits = bits_tc;
+    mBits = mIn64a;
+    if (use_bits) {
+      cuuint64_t dims[2] = {static_cast<cuuint64_t>(wpr), static_cast<cuuint64_t>(T)};
+      cuuint64_t strides[1] = {static_cast<cuuint64_t>(wpr) * 4};
+      cuuint32_t box[2] = {static_cast<cuuint32_t>(kTcCols / 32), static_cast<cuuint32_t>(kTcTok)};
+      cuuint32_t estr[2] = {1, 1};
+      if (g_encode(&mBits, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(bits_in), dims, strides, box,
+                   estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+        use_bits = false;
+    }
+    const unsigned n_pieces = static_cast<unsigned>(hp.pieces.size());
+    const unsigned groups = static_cast<unsigned>((rp + kTcMaxR - 1) / kTcMaxR);
+    const int smem = 1024 + kTcSmemBudget + 2 * kTcMaxStages * 8;
+    TcParams tp{};
+    tp.T = static_cast<int32_t>(T);
+    tp.pieces = plan->d_pieces;
+    tp.scale = scale;
+    // dB: In = dY, G = U, no mask
+    tp.N = static_cast<int32_t>(d_out);
+    tp.factor = 1.0f;
+    tp.out = dB_pool;
+    tp.partial = pdB;
+    dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), n_pieces, groups);
+    lora_tcontract_kernel<<<grid_b, kTcThreads, smem, stream>>>(mIn64b, mU[3], mBits, mU[0], mU[1], mU[2], tp);
+    // dA: In = X with the dropout mask, G = dY·B^T; the mask's 1/(1 - p) and s_a
+    // scale the sums
+    tp.N = static_cast<int32_t>(d_in);
+    tp.thr = thr;
+    tp.seed = seed;
+    tp.keep_bits = use_bits ? bits_in : nullptr;
+    tp.wpr = wpr;
+    tp.perm = gathers ? plan->d_perm : nullptr;
+    tp.factor = inv_keep;
+    tp.out = dA_pool;
+    tp.partial = pdA;
+    dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), n_pieces, groups);
+    lora_tcontract_kernel<<<grid_a, kTcThreads, smem, stream>>>(mIn64a, mG[3], mBits, mG[0], mG[1], mG[2], tp);
+    if (hp.partial_rows > 0) {
+      const unsigned gb = static_cast<unsigned>(std::min<int64_t>((hp.r_max * d_out + 255) / 256, 256));
+      const unsigned ga = static_cast<unsigned>(std::min<int64_t>((hp.r_max * d_in + 255) / 256, 256));
+      lora_reduce_pieces_kernel<<<dim3(gb, n_pieces), 256, 0, stream>>>(plan->d_pieces, pdB, d_out, scale, 1.0f,
+                                                                        dB_pool);
+      lora_reduce_pieces_kernel<<<dim3(ga, n_pieces), 256, 0, stream>>>(plan->d_pieces, pdA, d_in, scale, inv_keep,
+                                                                        dA_pool);
+    }
   }
   return launch_status();
 }
@@ -1173,10 +1425,12 @@ int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, con
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
   // W += DOWN·UP on the tensor cores, every layer in one persistent launch
-  CUtensorMap mBl;
+  CUtensorMap mBl, mW;
   const bool b3d = sw->d_out % 64 == 0;
-  const bool ok = b3d ? make_map_blocks(&mBl, B_pool, sw->d_out, sw->L * R, 16, kBN / 64)
-                      : make_map(&mBl, B_pool, sw->d_out, sw->L * R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  bool ok = b3d ? make_map_blocks(&mBl, B_pool, sw->d_out, sw->L * R, 16, kBN / 64)
+                : make_map(&mBl, B_pool, sw->d_out, sw->L * R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  // the weights as 128-row x 64-column boxes: each tile's W blocks
+  ok = ok && make_map(&mW, W, sw->d_out, sw->L * sw->d_in, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
   if (!ok) return LORA_ERR_ARG;
   GemmParams gp{};
   gp.b3d = b3d ? 1 : 0;
@@ -1197,8 +1451,8 @@ int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, con
   gp.merge_img_bytes = sw->img_bytes;
   const int64_t n_tiles = static_cast<int64_t>(gp.n_mt) * gp.n_nt;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ds->num_sms, n_tiles));
-  // no base K blocks: the A and W maps are never used for copies
-  lora_gemm_kernel<false, kEpiMergeAdd><<<grid, kGemmThreads, kGemmSmem, stream>>>(mBl, mBl, mBl, gp);
+  // no base K blocks: the A map carries the weights' W blocks, the W map is unused
+  lora_gemm_kernel<false, kEpiMergeAdd><<<grid, kGemmThreads, kGemmSmem, stream>>>(mW, mBl, mBl, gp);
   return launch_status();
 }
 

@@ -195,6 +195,37 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
       }
     }
   }
+  // The backward's per-adapter contractions: each segment in pieces of at most
+  // kPieceTokens sorted tokens, partial sums only for segments of several
+  // pieces. Without a sorted copy of X the backward reads original rows, so a
+  // piece is then also cut where the original index does not continue.
+  for (int32_t sidx = 0; sidx < n_seg; ++sidx) {
+    const int32_t a = hp.seg[3 * sidx], start = hp.seg[3 * sidx + 1], len = hp.seg[3 * sidx + 2];
+    const int32_t first = (int32_t)hp.pieces.size();
+    for (int32_t i = start; i < start + len;) {
+      int32_t n = std::min<int32_t>(kPieceTokens, start + len - i);
+      if (!any_gathered)
+        for (int32_t j = 1; j < n; ++j)
+          if (hp.perm[i + j] != hp.perm[i] + j) { n = j; break; }
+      PieceDesc pd{};
+      pd.start = i;
+      pd.len = n;
+      pd.in_row = any_gathered ? i : hp.perm[i];
+      pd.adapter = a;
+      pd.rank = ranks[a];
+      pd.pool_row = (int32_t)hp.offsets[a];
+      pd.first_piece = first;
+      hp.pieces.push_back(pd);
+      i += n;
+    }
+    const int32_t np = (int32_t)hp.pieces.size() - first;
+    for (int32_t q = first; q < first + np; ++q) {
+      hp.pieces[q].seg_pieces = np;
+      hp.pieces[q].partial_row = np > 1 ? (int32_t)hp.partial_rows : -1;
+      if (np > 1) hp.partial_rows += ranks[a];
+    }
+  }
+
   // Launch order, longest first: one CTA (or cluster) takes one unit, and
   // blocks start in index order as earlier ones finish, so the units with the
   // most rows and rank columns per 64-column block go in the first wave and

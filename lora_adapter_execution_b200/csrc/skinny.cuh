@@ -68,7 +68,8 @@ struct ShrinkParams {
   int32_t bits_tma;  // 1: units of consecutive tokens copy their bits with each stage (mapBits16)
   uint8_t *uimg;
   float *U_save;
-  int32_t r_max;
+  int32_t r_max;     // U_save's row length
+  int32_t u_sorted;  // 1: U_save rows in the plan's sorted order, else the original token order
   // backward
   int32_t r;
   int32_t npieces;
@@ -610,7 +611,8 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
       const int ncol = max(0, cend - g.n0);
       const int nw = static_cast<int>(blockDim.x) >> 5;
       for (int lr = lr0 + warp; lr < lr1; lr += nw) {
-        const int64_t orig = g.contig >= 0 ? static_cast<int64_t>(g.contig + lr) : p.perm[g.row0 + lr];
+        const int64_t orig = p.u_sorted ? static_cast<int64_t>(g.row0 + lr)
+                             : g.contig >= 0 ? static_cast<int64_t>(g.contig + lr) : p.perm[g.row0 + lr];
         float *dst = p.U_save + orig * p.r_max + g.n0;
         for (int c = lane; c < ncol; c += 32) dst[c] = c < g.nvalid ? fin[lr * kShrinkN + c] * p.inv_keep : 0.f;
       }
@@ -660,7 +662,17 @@ struct TcParams {
   uint64_t seed, thr;      // mask on In (dA); thr = 0 for none
   const uint32_t *keep_bits;  // precomputed keep bits of In (null: hash), word t * wpr + col / 32
   int64_t wpr;
-  float *partial;          // [splits][r_total][N]
+  float *partial;          // [splits][r_total][N]; piece mode: [partial rows][N]
+  // piece mode (pieces != null, multi-adapter backward): CTA (x, y, z) takes
+  // column block x of piece y, ranks [64z, 64z + 64) of the piece's adapter; its
+  // rank group's width selects the G map. A segment of one piece writes
+  // out[(pool_row + k) * N + n] = scale[adapter] * factor * sum; the pieces of a
+  // longer segment write partial rows (partial_row + k) for a later reduction.
+  const PieceDesc *pieces;
+  const float *scale;
+  float factor;
+  float *out;
+  const int32_t *perm;     // rows of In are sorted positions: the mask hash uses perm[row]
 };
 
 // split fp32 values into bf16 hi + lo (hi = rn(v), lo = rn(v - hi)), packed in pairs
@@ -688,19 +700,39 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N] bf16, box {64, 64}, swizzle 128B
                           const __grid_constant__ CUtensorMap mapG,   // G [T, >= k0 + r] fp32, box {r, 64}, no swizzle
                           const __grid_constant__ CUtensorMap mapBits,  // keep bits [T, wpr] u32, box {4, 64}
+                          const __grid_constant__ CUtensorMap mapG16,  // piece mode: G maps of boxes {16, 64},
+                          const __grid_constant__ CUtensorMap mapG32,  // {32, 64}, {48, 64} (mapG: {64, 64})
+                          const __grid_constant__ CUtensorMap mapG48,
                           const TcParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
+  // this CTA's ranks [k0, k0 + r) (r a multiple of 16; r_valid real ones) and tokens [t0, t1)
+  int r = p.r, r_valid = p.r_valid, k0 = p.k0, t0, t1;
+  PieceDesc pc{};
+  const CUtensorMap *gmap = &mapG;
+  if (p.pieces) {
+    pc = p.pieces[blockIdx.y];
+    k0 = static_cast<int>(blockIdx.z) * kTcMaxR;
+    if (k0 >= pc.rank) return;  // no barrier has been set up yet
+    r = min(kTcMaxR, (pc.rank + 15) / 16 * 16 - k0);
+    r_valid = min(r, pc.rank - k0);
+    gmap = r == 16 ? &mapG16 : r == 32 ? &mapG32 : r == 48 ? &mapG48 : &mapG;
+    t0 = pc.in_row;  // In (and keep-bit) rows; G rows are sorted positions from pc.start
+    t1 = pc.in_row + pc.len;
+  } else {
+    t0 = blockIdx.y * p.tsplit;
+    t1 = min(p.T, t0 + p.tsplit);
+  }
   const bool bits = p.keep_bits != nullptr;
-  const int mblocks = (p.r + 15) / 16;
+  const int mblocks = (r + 15) / 16;
   const int in_bytes = kTcTok * kTcCols * 2;    // 16 KB (two 8 KB halves)
-  const int g_bytes = kTcTok * p.r * 4;         // <= 16 KB
+  const int g_bytes = kTcTok * r * 4;           // <= 16 KB
   const int g_pad = (g_bytes + 1023) & ~1023;
   const int bits_bytes = bits ? 1024 : 0;       // the stage's keep bits
   const int conv_off = in_bytes + g_pad + bits_bytes;  // G^T hi, then lo (mblocks * 2 KB each)
-  const int stage_bytes = tc_stage_bytes(p.r, bits);
-  const int nstage = tc_stages(p.r, bits);
+  const int stage_bytes = tc_stage_bytes(r, bits);
+  const int nstage = tc_stages(r, bits);
   const uint32_t pool = smem_u32(smem);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + nstage * stage_bytes);
   const uint32_t full0 = smem_u32(bars);
@@ -709,9 +741,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kTcCols;
-  const int t0 = blockIdx.y * p.tsplit;
-  const int t1 = min(p.T, t0 + p.tsplit);
   const int nblk = t1 > t0 ? (t1 - t0 + kTcTok - 1) / kTcTok : 0;
+  const int g0 = p.pieces ? pc.start : t0;  // G row of token t0
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
@@ -725,7 +756,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   if (warp == kTcConsumerWarps) {
     if (lane == 0) {
       prefetch_tmap(&mapIn);
-      prefetch_tmap(&mapG);
+      prefetch_tmap(gmap);
       if (bits) prefetch_tmap(&mapBits);
       int stage = 0;
       uint32_t phase = 0;
@@ -737,7 +768,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         mbar_arrive_expect_tx(fb, in_bytes + g_bytes + bits_bytes);
         tma_load_2d(sb, &mapIn, fb, n0, t);
         tma_load_2d(sb + 8192, &mapIn, fb, n0 + 64, t);
-        tma_load_2d(sb + in_bytes, &mapG, fb, p.k0, t);  // the launch's group of ranks
+        tma_load_2d(sb + in_bytes, gmap, fb, k0, t - t0 + g0);  // this CTA's group of ranks
         if (bits) tma_load_2d(sb + in_bytes + g_pad, &mapBits, fb, n0 / 32, t);
         if (++stage == nstage) { stage = 0; phase ^= 1; }
       }
@@ -794,8 +825,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     // from k4): G[2tp][k4 .. k4 + 3] and G[2tp + 1][k4 .. k4 + 3] as two 16-byte
     // reads (consecutive threads take consecutive ranks, so the reads do not
     // collide on banks), written as (hi, lo) bf16 pairs at rank rows k4 .. k4 + 3,
-    // tokens 2tp and 2tp + 1. Rank rows from r to 16 * mblocks are zero.
+    // tokens 2tp and 2tp + 1. Rank rows from r to 16 * mblocks are zero, and so
+    // are the columns of tokens at or past t1 (in piece mode the stage's last
+    // rows can be the next segment's tokens, which must not enter the sums).
     {
+      const int tb = t0 + b * kTcTok;
       const float *graw = reinterpret_cast<const float *>(sbp + in_bytes);
       uint8_t *ghi = sbp + conv_off;
       uint8_t *glo = ghi + mblocks * 2048;
@@ -804,9 +838,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const int tp = item / q4;
         const int k4 = (item - tp * q4) * 4;
         float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (k4 < p.r) {  // r % 16 == 0: a group is all in or all out
-          v0 = *reinterpret_cast<const float4 *>(graw + (2 * tp) * p.r + k4);
-          v1 = *reinterpret_cast<const float4 *>(graw + (2 * tp + 1) * p.r + k4);
+        if (k4 < r) {  // r % 16 == 0: a group is all in or all out
+          if (tb + 2 * tp < t1) v0 = *reinterpret_cast<const float4 *>(graw + (2 * tp) * r + k4);
+          if (tb + 2 * tp + 1 < t1) v1 = *reinterpret_cast<const float4 *>(graw + (2 * tp + 1) * r + k4);
         }
         const float a0[4] = {v0.x, v0.y, v0.z, v0.w};
         const float a1[4] = {v1.x, v1.y, v1.z, v1.w};
@@ -851,14 +885,23 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             bf[g][3] &= keep_pair_t<0xDD99>(x8, x9);
           }
         } else {
+          // the mask is indexed by original token: rows past the token range are
+          // zero in the stage, their bits are never used
           const int tk = tbase + tl;
+          int64_t o0 = tk, o1 = tk + 1, o8 = tk + 8, o9 = tk + 9;
+          if (p.perm) {
+            o0 = p.perm[min(tk, t1 - 1)];
+            o1 = p.perm[min(tk + 1, t1 - 1)];
+            o8 = p.perm[min(tk + 8, t1 - 1)];
+            o9 = p.perm[min(tk + 9, t1 - 1)];
+          }
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
             const int c = n0 + cw + 16 * g + (lane >> 2);
-            bf[g][0] = mask_pair(bf[g][0], keep_elem(p.seed, p.thr, tk, c, p.N), keep_elem(p.seed, p.thr, tk + 1, c, p.N));
-            bf[g][1] = mask_pair(bf[g][1], keep_elem(p.seed, p.thr, tk + 8, c, p.N), keep_elem(p.seed, p.thr, tk + 9, c, p.N));
-            bf[g][2] = mask_pair(bf[g][2], keep_elem(p.seed, p.thr, tk, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 1, c + 8, p.N));
-            bf[g][3] = mask_pair(bf[g][3], keep_elem(p.seed, p.thr, tk + 8, c + 8, p.N), keep_elem(p.seed, p.thr, tk + 9, c + 8, p.N));
+            bf[g][0] = mask_pair(bf[g][0], keep_elem(p.seed, p.thr, o0, c, p.N), keep_elem(p.seed, p.thr, o1, c, p.N));
+            bf[g][1] = mask_pair(bf[g][1], keep_elem(p.seed, p.thr, o8, c, p.N), keep_elem(p.seed, p.thr, o9, c, p.N));
+            bf[g][2] = mask_pair(bf[g][2], keep_elem(p.seed, p.thr, o0, c + 8, p.N), keep_elem(p.seed, p.thr, o1, c + 8, p.N));
+            bf[g][3] = mask_pair(bf[g][3], keep_elem(p.seed, p.thr, o8, c + 8, p.N), keep_elem(p.seed, p.thr, o9, c + 8, p.N));
           }
         }
       }
@@ -881,8 +924,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     if (lane == 0) mbar_arrive(empty0 + 8 * stage);
     if (++stage == nstage) { stage = 0; phase ^= 1; }
   }
-  // write partial[q][k0 + k][n] for the group's real ranks
-  float *out = p.partial + (static_cast<int64_t>(blockIdx.y) * p.r_total + p.k0) * p.N;
+  // write partial[q][k0 + k][n] for the group's real ranks; piece mode: the
+  // adapter's gradient rows (scaled) or the piece's partial rows
+  float *out;
+  float f = 1.f;
+  if (p.pieces) {
+    if (pc.seg_pieces == 1) {
+      out = p.out + (static_cast<int64_t>(pc.pool_row) + k0) * p.N;
+      f = p.scale[pc.adapter] * p.factor;
+    } else {
+      out = p.partial + (static_cast<int64_t>(pc.partial_row) + k0) * p.N;
+    }
+  } else {
+    out = p.partial + (static_cast<int64_t>(blockIdx.y) * p.r_total + k0) * p.N;
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     if (i >= mblocks) break;
@@ -893,13 +948,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const int k = i * 16 + (lane >> 2);
         const int c = n0 + cw + 16 * g + j * 8 + q2;
         if (c < p.N) {
-          if (k < p.r_valid) {
-            out[static_cast<int64_t>(k) * p.N + c] = acc[i][g][j][0];
-            out[static_cast<int64_t>(k) * p.N + c + 1] = acc[i][g][j][1];
+          if (k < r_valid) {
+            out[static_cast<int64_t>(k) * p.N + c] = f * acc[i][g][j][0];
+            out[static_cast<int64_t>(k) * p.N + c + 1] = f * acc[i][g][j][1];
           }
-          if (k + 8 < p.r_valid) {
-            out[static_cast<int64_t>(k + 8) * p.N + c] = acc[i][g][j][2];
-            out[static_cast<int64_t>(k + 8) * p.N + c + 1] = acc[i][g][j][3];
+          if (k + 8 < r_valid) {
+            out[static_cast<int64_t>(k + 8) * p.N + c] = f * acc[i][g][j][2];
+            out[static_cast<int64_t>(k + 8) * p.N + c + 1] = f * acc[i][g][j][3];
           }
         }
       }
@@ -933,6 +988,41 @@ __global__ void lora_pad_cols_kernel(const float *__restrict__ src, int r, float
     const int64_t t = e / rp;
     const int k = static_cast<int>(e - t * rp);
     dst[e] = k < r ? src[t * r + k] : 0.f;
+  }
+}
+
+// The multi-adapter backward's segments of several pieces: for each such
+// segment (CTA row y = its first piece), row k < rank, column n:
+// out[(pool_row + k) * N + n] = scale[adapter] * factor * sum over the
+// segment's pieces, in piece order, of partial[(partial_row + k) * N + n].
+__global__ void lora_reduce_pieces_kernel(const PieceDesc *__restrict__ pieces, const float *__restrict__ partial,
+                                          int64_t N, const float *__restrict__ scale, float factor,
+                                          float *__restrict__ out) {
+  const PieceDesc pc = pieces[blockIdx.y];
+  if (pc.seg_pieces == 1 || pc.first_piece != static_cast<int>(blockIdx.y)) return;
+  const int64_t n = static_cast<int64_t>(pc.rank) * N;
+  const float f = scale[pc.adapter] * factor;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t k = e / N, c = e - k * N;
+    float s = 0.f;
+    for (int q = 0; q < pc.seg_pieces; ++q) s += partial[(pieces[pc.first_piece + q].partial_row + k) * N + c];
+    out[(pc.pool_row + k) * N + c] = f * s;
+  }
+}
+
+// dst[i][k] = src[row(i)][k] for k < r, 0 for r <= k < rp, row(i) = perm[i] (or
+// i without perm): rows of an fp32 [T, r] matrix in the plan's sorted order,
+// padded to rp columns.
+__global__ void lora_gather_pad_kernel(const float *__restrict__ src, int r, const int32_t *__restrict__ perm,
+                                       float *__restrict__ dst, int rp, int64_t T) {
+  const int64_t n = T * rp;
+  for (int64_t e = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; e < n;
+       e += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t i = e / rp;
+    const int k = static_cast<int>(e - i * rp);
+    const int64_t row = perm ? perm[i] : i;
+    dst[e] = k < r ? src[row * r + k] : 0.f;
   }
 }
 

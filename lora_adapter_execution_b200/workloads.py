@@ -15,6 +15,8 @@ Y[t] = X[t]·W + s_a·(X[t]·A_a)·B_a, where a is token t's adapter):
             scaled by 1/k, Zipf(1.2) adapter per token, s=16/r
   finetune  T=16384, 4096x4096, 1 adapter of rank 16, s=2, dropout p=0.1,
             plus an upstream gradient dY ~ N(0,1)
+  fleet_finetune  the fleet batch with dropout p=0.1 and dY ~ N(0,1): one
+            fine-tuning step of all its adapters at once
 
 Readings where the pages are silent:
   * X ~ N(0,1), W ~ N(0,1/d_in), A ~ N(0,1/d_in), B_a ~ N(0,1/r_a) for every
@@ -40,7 +42,7 @@ from dataclasses import dataclass, field
 
 import numpy as np
 
-WORKLOADS = ("tiny", "decode", "prefill", "fleet", "finetune")
+WORKLOADS = ("tiny", "decode", "prefill", "fleet", "finetune", "fleet_finetune")
 
 
 def f32_to_bf16_bits(a: np.ndarray) -> np.ndarray:
@@ -83,6 +85,9 @@ SPECS = {
                   "16/r", b_row_decay=True),
     "finetune": Spec("finetune", 16384, 4096, 4096, 1, ("fixed", 16), ("single",), 2.0,
                      p_drop=0.1, with_dy=True),
+    # the fleet batch as one multi-adapter fine-tuning step (every adapter trained)
+    "fleet_finetune": Spec("fleet_finetune", 4096, 4096, 4096, 1000, ("range", 1, 21), ("zipf_token", 1.2),
+                           "16/r", b_row_decay=True, p_drop=0.1, with_dy=True),
 }
 
 

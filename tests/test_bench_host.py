@@ -73,5 +73,5 @@ def test_backward_algorithmic_flops_match_the_fine_tuning_figure():
 def test_default_runs_every_workload_with_the_fine_tuning_headline():
     a = bench.parse([])
     assert a.config == "all" and bench.HEADLINE == "finetune"
-    assert set(bench.ORDER) == set(wl.WORKLOADS)
+    assert set(bench.ORDER) | {"fleet_finetune"} == set(wl.WORKLOADS)
     assert bench.steps_for(bench.parse(["--steps", "20"]), "decode") == 20
