@@ -72,7 +72,7 @@ int device_state(DeviceState **out) {
           ok &= cudaFuncSetAttribute(lora_shrink_kernel<2>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      sk_smem(2)) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_tcontract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     1024 + kTcSmemBudget + 2 * kTcMaxStages * 8) == cudaSuccess;
+                                     tc_smem(kTcMaxR)) == cudaSuccess;
           if (!ok) d.status = LORA_ERR_CUDA;
         }
       }
@@ -925,14 +925,14 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
       tp.keep_bits = nullptr;
       tp.partial = pdB;
       dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
-      const int smem_b = 1024 + tc_stages(w, false) * tc_stage_bytes(w, false) + 2 * kTcMaxStages * 8;
+      const int smem_b = tc_smem(w);
       lora_tcontract_kernel<<<grid_b, kTcThreads, smem_b, stream>>>(mdY64, mU, mBits, mU, mU, mU, tp);
       tp.N = static_cast<int32_t>(d_in);
       tp.thr = thr;
       tp.seed = seed;
       // with keep bits, each stage's bits come through the copy engine with its tile
       tp.keep_bits = use_bits ? keep_bits : nullptr;
-      const int smem_a = 1024 + tc_stages(w, use_bits) * tc_stage_bytes(w, use_bits) + 2 * kTcMaxStages * 8;
+      const int smem_a = tc_smem(w);
       tp.wpr = (d_in + 31) / 32;
       tp.partial = pdA;
       dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), static_cast<unsigned>(S));
@@ -1143,7 +1143,7 @@ int lora_linear_bwd_multi(lora_plan_t plan, const uint16_t *X, const uint16_t *W
     }
     const unsigned n_pieces = static_cast<unsigned>(hp.pieces.size());
     const unsigned groups = static_cast<unsigned>((rp + kTcMaxR - 1) / kTcMaxR);
-    const int smem = 1024 + kTcSmemBudget + 2 * kTcMaxStages * 8;
+    const int smem = tc_smem(std::min(rp, kTcMaxR));  // the widest rank group of any piece
     TcParams tp{};
     tp.T = static_cast<int32_t>(T);
     tp.pieces = plan->d_pieces;

@@ -14,8 +14,10 @@
 //    shared-memory image the fused GEMM's MMA reads, plus U for the backward.
 //  * lora_tcontract_kernel: partial[q][k][n] = sum_{t in split q} G[t, k] * In[t, n]
 //    (dB with G = U, In = dY; dA with G = dU, In = masked X), fixed token splits.
-//    G stays fp32 and enters the MMA as a hi + lo pair of bf16 (two MMAs), so the
-//    reduction over thousands of tokens keeps ~16 mantissa bits per term.
+//    G stays fp32 and enters the MMA as three bf16 parts (hi, mid, lo: three
+//    MMAs), about 24 mantissa bits, so each term carries fp32 precision: sums
+//    whose terms cancel (per-token terms of +-1e3 summing to 1e-3 occur in the
+//    fleet fine-tuning batch) keep an error at fp32-accumulation level.
 //  * lora_reduce_splits_kernel: sums the splits in a fixed order (deterministic).
 //  * lora_mask_kernel: the dropout mask itself (test hook).
 //
@@ -637,19 +639,25 @@ constexpr int kTcTok = 64;        // tokens per stage
 constexpr int kTcCols = 128;      // columns per CTA (32 per consumer warp)
 constexpr int kTcMaxR = 64;
 constexpr int kTcSmemBudget = 110 * 1024;  // stage ring per CTA: two CTAs share an SM
+constexpr int kTcSmemBudgetWide = 216 * 1024;  // rank groups wider than 32: one CTA per SM
+constexpr int kTcParts = 3;                 // bf16 parts of G (hi, mid, lo)
+__host__ __device__ inline int tc_budget(int r) { return r <= 32 ? kTcSmemBudget : kTcSmemBudgetWide; }
 
 // Bytes of one stage of the token contraction: In [64 tokens][128 columns] as two
 // 64-column halves (128-byte swizzle), G [64 tokens][r] fp32 as copied, the
-// stage's keep bits [64 tokens][4 words] when read, and G^T split into bf16 hi
-// and lo parts, [16 * mblocks ranks][64 tokens] each (128-byte rows, swizzled).
+// stage's keep bits [64 tokens][4 words] when read, and G^T split into bf16
+// parts (hi, mid, lo), [16 * mblocks ranks][64 tokens] each (128-byte rows,
+// swizzled).
 __host__ __device__ inline int tc_stage_bytes(int r, bool bits) {
   const int mblocks = (r + 15) / 16;
-  return kTcTok * kTcCols * 2 + ((kTcTok * r * 4 + 1023) & ~1023) + (bits ? 1024 : 0) + 2 * mblocks * 2048;
+  return kTcTok * kTcCols * 2 + ((kTcTok * r * 4 + 1023) & ~1023) + (bits ? 1024 : 0) + kTcParts * mblocks * 2048;
 }
 __host__ __device__ inline int tc_stages(int r, bool bits) {
-  const int n = kTcSmemBudget / tc_stage_bytes(r, bits);
+  const int n = tc_budget(r) / tc_stage_bytes(r, bits);
   return n < kTcMaxStages ? n : kTcMaxStages;
 }
+// dynamic shared memory of a launch whose rank groups are at most r wide
+__host__ __device__ inline int tc_smem(int r) { return 1024 + tc_budget(r) + 2 * kTcMaxStages * 8; }
 
 struct TcParams {
   int32_t T, N;
@@ -675,10 +683,13 @@ struct TcParams {
   const int32_t *perm;     // rows of In are sorted positions: the mask hash uses perm[row]
 };
 
-// split fp32 values into bf16 hi + lo (hi = rn(v), lo = rn(v - hi)), packed in pairs
-__device__ __forceinline__ void split_pair(float v0, float v1, uint32_t &hi, uint32_t &lo) {
+// split fp32 values into three bf16 parts, hi = rn(v), mid = rn(v - hi),
+// lo = rn(v - hi - mid) (each remainder exact in fp32), packed in pairs
+__device__ __forceinline__ void split3_pair(float v0, float v1, uint32_t &hi, uint32_t &mid, uint32_t &lo) {
   hi = pack_bf16x2(v0, v1);
-  lo = pack_bf16x2(v0 - bf16_lo(hi), v1 - bf16_hi(hi));
+  const float r0 = v0 - bf16_lo(hi), r1 = v1 - bf16_hi(hi);
+  mid = pack_bf16x2(r0, r1);
+  lo = pack_bf16x2(r0 - bf16_lo(mid), r1 - bf16_hi(mid));
 }
 
 // Mask of a transposed B fragment register: its two bf16 halves are tokens t
@@ -730,7 +741,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int g_bytes = kTcTok * r * 4;           // <= 16 KB
   const int g_pad = (g_bytes + 1023) & ~1023;
   const int bits_bytes = bits ? 1024 : 0;       // the stage's keep bits
-  const int conv_off = in_bytes + g_pad + bits_bytes;  // G^T hi, then lo (mblocks * 2 KB each)
+  const int conv_off = in_bytes + g_pad + bits_bytes;  // G^T hi, mid, lo (mblocks * 2 KB each)
   const int stage_bytes = tc_stage_bytes(r, bits);
   const int nstage = tc_stages(r, bits);
   const uint32_t pool = smem_u32(smem);
@@ -832,7 +843,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const int tb = t0 + b * kTcTok;
       const float *graw = reinterpret_cast<const float *>(sbp + in_bytes);
       uint8_t *ghi = sbp + conv_off;
-      uint8_t *glo = ghi + mblocks * 2048;
+      uint8_t *gmid = ghi + mblocks * 2048;
+      uint8_t *glo = gmid + mblocks * 2048;
       const int q4 = mblocks * 4;  // 4-rank groups per token pair
       for (int item = tid; item < 32 * q4; item += kTcConsumerWarps * 32) {
         const int tp = item / q4;
@@ -847,17 +859,19 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int k = k4 + u;
-          uint32_t hi, lo;
-          split_pair(a0[u], a1[u], hi, lo);
+          uint32_t hi, mid, lo;
+          split3_pair(a0[u], a1[u], hi, mid, lo);
           const uint32_t off = k * 128 + ((((tp >> 2) ^ (k & 7)) & 7) << 4) + (tp & 3) * 4;
           *reinterpret_cast<uint32_t *>(ghi + off) = hi;
+          *reinterpret_cast<uint32_t *>(gmid + off) = mid;
           *reinterpret_cast<uint32_t *>(glo + off) = lo;
         }
       }
     }
     asm volatile("bar.sync 1, %0;" ::"n"(kTcConsumerWarps * 32) : "memory");
     const uint32_t ghi_s = sb + conv_off;
-    const uint32_t glo_s = ghi_s + mblocks * 2048;
+    const uint32_t gmid_s = ghi_s + mblocks * 2048;
+    const uint32_t glo_s = gmid_s + mblocks * 2048;
     const uint32_t *bs = reinterpret_cast<const uint32_t *>(sbp + in_bytes + g_pad);
     const int tbase = t0 + b * kTcTok;
 #pragma unroll
@@ -908,15 +922,19 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         if (i >= mblocks) break;
-        uint32_t h0, h1, h2, h3, l0, l1, l2, l3;
+        uint32_t h0, h1, h2, h3, m0, m1, m2, m3, l0, l1, l2, l3;
         ldsm_x4(ghi_s + i * 2048 + aoff[ks], h0, h1, h2, h3);
+        ldsm_x4(gmid_s + i * 2048 + aoff[ks], m0, m1, m2, m3);
         ldsm_x4(glo_s + i * 2048 + aoff[ks], l0, l1, l2, l3);
 #pragma unroll
         for (int g = 0; g < 2; ++g) {
-          mma_bf16_16816(acc[i][g][0], h0, h1, h2, h3, bf[g][0], bf[g][1]);
-          mma_bf16_16816(acc[i][g][1], h0, h1, h2, h3, bf[g][2], bf[g][3]);
+          // smallest parts first, so the partial sums grow from the small end
           mma_bf16_16816(acc[i][g][0], l0, l1, l2, l3, bf[g][0], bf[g][1]);
           mma_bf16_16816(acc[i][g][1], l0, l1, l2, l3, bf[g][2], bf[g][3]);
+          mma_bf16_16816(acc[i][g][0], m0, m1, m2, m3, bf[g][0], bf[g][1]);
+          mma_bf16_16816(acc[i][g][1], m0, m1, m2, m3, bf[g][2], bf[g][3]);
+          mma_bf16_16816(acc[i][g][0], h0, h1, h2, h3, bf[g][0], bf[g][1]);
+          mma_bf16_16816(acc[i][g][1], h0, h1, h2, h3, bf[g][2], bf[g][3]);
         }
       }
     }
