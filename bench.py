@@ -96,6 +96,9 @@ def parse(argv=None):
                     help="time only the full step (no GEMM-alone, base or torch timings; for profiler runs)")
     ap.add_argument("--once", action="store_true",
                     help="one timed region per config, no repeats (for profiler runs)")
+    ap.add_argument("--fwd", default="auto", choices=["auto", "fused", "two"],
+                    help="the forward of the step: the faster of the two in a burst (auto), the one-launch fused "
+                         "forward, or the two kernels")
     ap.add_argument("--dry-run", action="store_true",
                     help="no GPU: exercise the ranks' start-up and collectives over gloo and print a line")
     a = ap.parse_args(argv)
@@ -532,11 +535,14 @@ def measure(name, cx, cpu_budget):
     ev_fork = torch.cuda.Event()
     ev_join = torch.cuda.Event()
 
-    def step(c):
+    def step(c, fused=False):
+        # the forward in two kernels (shrink, then the fused GEMM) or in one
+        # launch (lora_linear_fwd_fused)
         cp, nxt = copies[c], (c + 1) % len(copies)
         bits = cp["bits"] if masked else None
-        lora.linear_shrink(plan, cp["X"], cp["A"], scale, p_drop=inp.p_drop, seed=mask_seed, U_save=cp["U"],
-                           keep_bits=bits)
+        if not fused:
+            lora.linear_shrink(plan, cp["X"], cp["A"], scale, p_drop=inp.p_drop, seed=mask_seed, U_save=cp["U"],
+                               keep_bits=bits)
         cur = torch.cuda.current_stream()
         if masked:
             ev_fork.record(cur)
@@ -544,7 +550,11 @@ def measure(name, cx, cpu_budget):
             with torch.cuda.stream(side):
                 lora.dropout_keep_bits(mask_seed, inp.p_drop, copies[nxt]["bits"], di)
             ev_join.record(side)
-        lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
+        if fused:
+            lora.linear_fwd_fused(plan, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["Y"], p_drop=inp.p_drop,
+                                  seed=mask_seed, U_save=cp["U"], keep_bits=bits)
+        else:
+            lora.fused_gemm(plan, cp["X"], cp["W"], cp["B"], cp["Y"])
         if multi:
             lora.linear_bwd_multi(plan, cp["X"], cp["W"], cp["A"], cp["B"], scale, cp["U"], cp["dY"], cp["dX"],
                                   cp["dA"], cp["dB"], cp["ws"], p_drop=inp.p_drop, seed=mask_seed, keep_bits=bits)
@@ -574,12 +584,25 @@ def measure(name, cx, cpu_budget):
                 lora.dropout_keep_bits(mask_seed, inp.p_drop, copies[c]["bits"], di)
         step(0)  # the first call sets kernel attributes outside any capture
     torch.cuda.synchronize()
-    graphs, ggraphs, bgraphs = [], [], []
+    fused_error = None
+    try:
+        with torch.cuda.stream(cx.stream):
+            step(0, fused=True)
+        torch.cuda.synchronize()
+        assert lora.device_status() == 0
+    except Exception as e:  # the device refused the cooperative launch: two kernels only
+        fused_error = f"{type(e).__name__}: {e}"
+    graphs, fgraphs, ggraphs, bgraphs = [], [], [], []
     for c, cp in enumerate(copies):
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=cx.stream):
             step(c)
         graphs.append(g)
+        if fused_error is None:
+            g1 = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g1, stream=cx.stream):
+                step(c, fused=True)
+            fgraphs.append(g1)
         if not a.no_layer:
             g2 = torch.cuda.CUDAGraph()
             with torch.cuda.graph(g2, stream=cx.stream):
@@ -599,7 +622,7 @@ def measure(name, cx, cpu_budget):
                 allreduce_grads(copies[i % len(gs)]["grad"], world)
         return f
 
-    ms_torch = ms_gemm = ms_base = ms_step_burst = None
+    ms_torch = ms_gemm = ms_base = ms_step_burst = ms_fused_burst = None
     if not a.no_layer:
         # the kernels alone, first, on a GPU that has idled: three regions of K
         # launches each (a burst, as the burst peak was taken)
@@ -607,6 +630,7 @@ def measure(name, cx, cpu_budget):
             time.sleep(0.2)
             return cx.timed(replay(gs), K, 0.0)[0]
         ms_step_burst = burst(graphs) if not (finetune and not multi and world > 1) else None
+        ms_fused_burst = burst(fgraphs) if fgraphs and not (finetune and not multi and world > 1) else None
         ms_gemm = burst(ggraphs)
         ms_base = burst(bgraphs)
         assert lora.device_status() == 0
@@ -623,6 +647,13 @@ def measure(name, cx, cpu_budget):
         ms_torch = burst(tgraphs)
         del ggraphs, bgraphs, tgraphs
 
+    # the step's forward: whichever path ran faster in the burst (the same
+    # choice on every rank: the max over ranks of each path's time)
+    use_fused = (ms_fused_burst is not None and ms_step_burst is not None and ms_fused_burst < ms_step_burst)
+    if a.fwd != "auto":
+        use_fused = a.fwd == "fused" and bool(fgraphs)
+    if use_fused:
+        graphs, launches_per_step = fgraphs, launches_per_step - 1 - int(info["gathers_x"])
     with ClockSampler(cx.local_rank) as clk:
         ms_total, n_regions = cx.timed(replay(graphs, finetune and not multi and world > 1), K,
                                    0.0 if a.once else MIN_REGION_S)
@@ -635,6 +666,9 @@ def measure(name, cx, cpu_budget):
              "timing": (f"CUDA-graph replays, CUDA events on the replay stream; median of {n_regions} regions of "
                         f"exactly {K} steps, max over ranks"),
              "gpu_launches": launches_per_step * K,
+             "forward": ("one fused launch (lora_linear_fwd_fused)" if use_fused
+                         else "two kernels (lora_linear_shrink, lora_fused_gemm)"
+                         + (f"; fused launch unavailable: {fused_error}" if fused_error else "")),
              "clocks": clocks}
 
     hbm, tc_burst, tc_sust, src = peaks()
@@ -679,10 +713,11 @@ def measure(name, cx, cpu_budget):
                      "layer_frac": entry["layer_roofline"]["frac"]})
         entry["roofline"] = roof
         base_fwd = min(ms_base, ms_torch) * 1e-3 / K
-        t_sb = ms_step_burst * 1e-3 / K if ms_step_burst else None
+        t_sb = min(x for x in (ms_step_burst, ms_fused_burst) if x) * 1e-3 / K if ms_step_burst else None
         entry["layer"] = {"fused_gemm_us": t_gemm * 1e6, "base_gemm_us": ms_base * 1e3 / K,
                           "torch_matmul_us": ms_torch * 1e3 / K, "step_us": t_step * 1e6,
                           "step_burst_us": t_sb * 1e6 if t_sb else None,
+                          "step_burst_us_fused": ms_fused_burst * 1e3 / K if ms_fused_burst else None,
                           "overhead_vs_base": None if (finetune or not t_sb) else t_sb / base_fwd - 1.0,
                           "gemm_overhead_vs_own_base": ms_gemm / ms_base - 1.0,
                           "layer_alg_bytes": lb, "layer_alg_flops": lf,

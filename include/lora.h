@@ -231,6 +231,28 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
 int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *B_pool,
                     uint16_t *Y, lora_stream_t stream);
 
+/* lora_linear_fwd_fused — lora_linear_fwd in one launch (arguments and results
+ * as lora_linear_fwd). Source: the kernel-layer fusion of the LoRAFusion
+ * explainer (Kernel 层: split the graph only at real GEMM boundaries and keep
+ * the small ops' work next to the big GEMM), applied to the shrink and the row
+ * gather, which otherwise run as kernels of their own before the fused GEMM.
+ * The launch's CTAs first copy X's rows into the plan's sorted copy (when the
+ * plan gathers) and wait for every CTA's share, then run the plan's shrink units
+ * (one CTA per unit), each counting itself done for its 128-token tile, then the
+ * fused GEMM's tiles with the adapter K blocks last, a tile's first adapter
+ * block waiting (bounded) for its tile's count. The launch is cooperative, so
+ * every CTA is resident and every wait ends; the plan holds the lists of units
+ * per CTA for the launch's grid, and its counters are zeroed on `stream` before
+ * the launch (two fused forwards with one plan must not overlap). Results agree
+ * with lora_linear_fwd within rounding (each unit's contraction is summed by one
+ * CTA instead of a cluster, and the adapter blocks enter the accumulator after
+ * the base blocks instead of before).
+ * Errors: LORA_ERR_ARG, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA (also when the device
+ * refuses the cooperative launch). */
+int lora_linear_fwd_fused(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
+                          const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed, uint16_t *Y,
+                          float *U_save, const uint32_t *keep_bits, lora_stream_t stream);
+
 /* Y = X·W only (no adapter term), through the same tcgen05 GEMM kernel: the
  * base-only reference the adapter overhead is measured against (the frozen
  * base term of the LoRAFusion explainer's reparameterisation).

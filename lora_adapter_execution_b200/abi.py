@@ -71,6 +71,7 @@ def load_library():
         "lora_plan_info": (ctypes.c_int, [_vp, ctypes.POINTER(_Info)]),
         "lora_plan_destroy": (None, [_vp]),
         "lora_linear_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp, _vp]),
+        "lora_linear_fwd_fused": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp, _vp]),
         "lora_linear_shrink": (ctypes.c_int, [_vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp]),
         "lora_fused_gemm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
         "lora_base_gemm": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp]),
@@ -246,6 +247,19 @@ def linear_fwd(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.
     _check(load_library().lora_linear_fwd(plan.handle, _ptr(X), _ptr(W), _ptr(A_pool), _ptr(B_pool), _ptr(scale),
                                           float(p_drop), int(seed) & (2**64 - 1), _ptr(Y), _ptr(U_save),
                                           _ptr(keep_bits), _stream(stream)), "lora_linear_fwd")
+
+
+def linear_fwd_fused(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.0, seed: int = 0,
+                     U_save=None, keep_bits=None, stream=None):
+    """lora_linear_fwd_fused: the forward (row gather, shrink and fused GEMM) in one launch."""
+    di, do, R = plan.d_in, plan.d_out, plan.pool_rows
+    _args("lora_linear_fwd_fused", *_fwd_args(plan, X, A_pool, scale, U_save, keep_bits),
+          ("W", W, (di, do), _BF16, False), ("B_pool", B_pool, (R, do), _BF16, False),
+          ("Y", Y, (plan.T, do), _BF16, False))
+    _check(load_library().lora_linear_fwd_fused(plan.handle, _ptr(X), _ptr(W), _ptr(A_pool), _ptr(B_pool),
+                                                _ptr(scale), float(p_drop), int(seed) & (2**64 - 1), _ptr(Y),
+                                                _ptr(U_save), _ptr(keep_bits), _stream(stream)),
+           "lora_linear_fwd_fused")
 
 
 def linear_shrink(plan: Plan, X, A_pool, scale, *, p_drop: float = 0.0, seed: int = 0, U_save=None,

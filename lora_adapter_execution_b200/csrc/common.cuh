@@ -79,6 +79,31 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
   return mbar_wait_for(bar, parity, kWaitLimitNs);
 }
 
+// Wait until the global counter *cnt reaches `need` (an acquire load, so what the
+// counting threads wrote before their release is visible). Returns false (after
+// flagging LORA_DEV_TIMEOUT) if it has not within kWaitLimitNs.
+__device__ __forceinline__ bool wait_counter(const int *cnt, int need) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+  if (v >= need) return true;
+  const uint64_t t0 = globaltimer();
+  while (true) {
+    __nanosleep(64);
+    asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+    if (v >= need) return true;
+    if (globaltimer() - t0 > kWaitLimitNs) {
+      flag_status(LORA_DEV_TIMEOUT);
+      return false;
+    }
+  }
+}
+// Add one to a global counter after every write this thread made, or saw
+// through a barrier, before it (release at GPU scope).
+__device__ __forceinline__ void signal_counter(int *cnt) {
+  __threadfence();
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(cnt) : "memory");
+}
+
 // ------------------------------------------------------------------ programmatic dependent launch
 // Let the next kernel on the stream (launched with programmatic serialization)
 // start its prologue while this grid still runs.

@@ -38,6 +38,7 @@
 
 #include "common.cuh"
 #include "internal.h"
+#include "skinny.cuh"
 
 namespace lora {
 
@@ -127,6 +128,19 @@ struct GemmParams {
   int32_t merge_rows;
   int32_t layer_brows;
   int64_t merge_img_bytes;
+  // fused forward (the FUSED instance): the same launch first copies X's rows
+  // into the sorted copy (when a_sorted; then waits for every CTA's share),
+  // then runs its shrink units, each counting itself done for its m-tile, then
+  // the GEMM tiles with their adapter blocks last, each tile's first adapter
+  // block waiting for the tile's count
+  const int32_t *fz_unit_off;   // [grid + 1]: CTA b runs units fz_units[fz_unit_off[b] ..)
+  const int32_t *fz_units;      // indices into fz_sp.units
+  const int32_t *fz_tile_need;  // [n_mt]: units per m-tile
+  int32_t *fz_tile_cnt;         // [n_mt]: units done per m-tile (zero at launch)
+  int32_t *fz_grid_cnt;         // CTAs done with the row copy (zero at launch)
+  const uint16_t *fz_X;         // X in the original token order
+  uint16_t *fz_Xs;              // the plan's sorted copy of X
+  ShrinkParams fz_sp;           // the shrink's parameters (one CTA per unit)
 };
 
 // Split-K exchange, inside the idle stage ring once every MMA of the cluster is
@@ -153,24 +167,30 @@ __host__ __device__ constexpr uint32_t xswz(int row, int j) { return static_cast
 struct BlockRange {
   int kb_lo, nbase;  // base blocks kb_lo .. kb_lo + nbase - 1
   int q, S, nlb;     // adapter blocks q, q + S, ... < nlb
+  bool alast;        // adapter blocks after the base blocks (fused forward)
   __device__ __forceinline__ int naug() const { return q < nlb ? (nlb - q + S - 1) / S : 0; }
   __device__ __forceinline__ int count() const { return nbase + naug(); }
   // index into the tile's block sequence: < KB base, >= KB adapter block (blk - KB).
   // Adapter blocks come first: their scattered B-row loads then overlap the base
-  // K loop instead of draining the pipeline at the end of the tile.
+  // K loop instead of draining the pipeline at the end of the tile. In the fused
+  // forward they come last, when the shrink that writes their images is done.
   __device__ __forceinline__ int block(int i, int KB) const {
+    if (alast) return i < nbase ? kb_lo + i : KB + q + (i - nbase) * S;
     const int na = naug();
     return i < na ? KB + q + i * S : kb_lo + (i - na);
   }
+  // position of block i among the CTA's adapter blocks (i must be one)
+  __device__ __forceinline__ int aug_index(int i) const { return alast ? i - nbase : i; }
 };
 
-__device__ __forceinline__ BlockRange block_range(int KB, int nlb, int q, int S) {
+__device__ __forceinline__ BlockRange block_range(int KB, int nlb, int q, int S, bool alast = false) {
   BlockRange br;
   br.kb_lo = KB * q / S;
   br.nbase = KB * (q + 1) / S - br.kb_lo;
   br.q = q;
   br.S = S;
   br.nlb = nlb;
+  br.alast = alast;
   return br;
 }
 
@@ -271,11 +291,15 @@ __device__ __forceinline__ TileDesc regular_tile(int mt, int T) {
 }
 
 // B_KMAJOR: the B operand tile is K-major (backward: W^T); otherwise MN-major (W).
-template <bool B_KMAJOR, int EPI>
+// FUSED: the fused forward (GemmParams fz_*; the shrink's maps in mapS*).
+template <bool B_KMAJOR, int EPI, bool FUSED = false>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     lora_gemm_kernel(const __grid_constant__ CUtensorMap mapA,    // A rows (X, sorted X or dY), box {64, 128}
                      const __grid_constant__ CUtensorMap mapB,    // W (2-D or 3-D, see GemmParams::w3d)
                      const __grid_constant__ CUtensorMap mapBl,   // B_pool rows, box {64, 16(, 4)}
+                     const __grid_constant__ CUtensorMap mapSIn,    // fused: the shrink's X rows, box {64, 16}
+                     const __grid_constant__ CUtensorMap mapSF,     // fused: A_pool rows, box {64, 16}
+                     const __grid_constant__ CUtensorMap mapSBits,  // fused: keep bits, box {4, 16}
                      const GemmParams p) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -328,6 +352,44 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   // those kernels ran), so their warp starts streaming at once
   if (warp != kGemmWarpW) pdl_wait();
 
+  if constexpr (FUSED) {
+    // ---------------------------------------------------- fused forward, phase 0:
+    // X's rows into the plan's sorted copy (every CTA a share), then every CTA
+    // waits until all shares are written (the launch is cooperative: all CTAs
+    // are resident, so the wait ends)
+    if (p.a_sorted) {
+      const int64_t per_row = p.K / 8;
+      const int64_t n = static_cast<int64_t>(p.T) * per_row;
+      for (int64_t e = blockIdx.x * static_cast<int64_t>(kGemmThreads) + threadIdx.x; e < n;
+           e += static_cast<int64_t>(gridDim.x) * kGemmThreads) {
+        const int64_t i = e / per_row, c = e - (e / per_row) * per_row;
+        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.fz_X + static_cast<int64_t>(p.perm[i]) * p.K) + c);
+        reinterpret_cast<uint4 *>(p.fz_Xs + i * p.K)[c] = v;
+      }
+      __syncthreads();
+      if (threadIdx.x == 0) {
+        signal_counter(p.fz_grid_cnt);
+        if (!wait_counter(p.fz_grid_cnt, static_cast<int>(gridDim.x))) *abort_flag = 1;
+      }
+      __syncthreads();
+      fence_proxy_async_global();  // the copies (async proxy) read what the stores wrote
+    }
+    // phase 1: this CTA's shrink units, by warps 2..5 (consumers) and 7
+    // (producer) in the stage ring's memory; each unit then counts itself done
+    // for its m-tile (release), which the tile's adapter blocks wait for
+    const int lt = (warp >= 2 && warp <= 5) ? static_cast<int>(threadIdx.x) - 64 : (warp == kGemmWarpFix ? 128 + lane : -1);
+    if (lt >= 0 && !*abort_flag) {
+      uint64_t *sbars = reinterpret_cast<uint64_t *>(smem + sk_pool(4));
+      for (int j = p.fz_unit_off[blockIdx.x]; j < p.fz_unit_off[blockIdx.x + 1]; ++j) {
+        const int u = p.fz_units[j];
+        shrink_unit<4>(smem, sbars, mapSIn, mapSF, mapSBits, p.fz_sp, u, 0u, ShrinkRole{lt, 2, false});
+        asm volatile("bar.sync 2, 160;" ::: "memory");  // the unit's outputs are all written
+        if (lt == 0) signal_counter(p.fz_tile_cnt + p.fz_sp.units[u].tile);
+      }
+    }
+    __syncthreads();  // the stage ring is free again
+  }
+
   const int n_tiles = p.n_mt * p.n_nt;
   const int KB = (p.K + kBK - 1) / kBK;
   const bool merge = p.merge_kaug > 0;
@@ -368,7 +430,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       const int arow = p.a_sorted ? td.row0 : td.contig;
       if (lane == 0) {
         if (arow < 0) { flag_status(LORA_DEV_BOUNDS); *abort_flag = 1; }
-        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S, FUSED);
         const int nmma = br.count();
         const int nblk = arow < 0 ? 0 : nmma + (merge ? kMergeWBlocks : 0);
         // adapter block descriptors, one load ahead of their use (the adapter
@@ -407,11 +469,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
             // distinct 16-row slice of B_pool is copied once, into its own slot
             // (the planner's descriptor lists the slices and each step's slot).
             const int lb = blk - KB;
+            const int ai = br.aug_index(i);
+            if (FUSED && ai == 0) {
+              // the tile's shrink units are done (their images written) before
+              // the first of its images is copied
+              if (!wait_counter(p.fz_tile_cnt + mt, p.fz_tile_need[mt])) { *abort_flag = 1; break; }
+              fence_proxy_async_global();
+            }
             const int prow_s[4] = {nprow.x + brow_ofs, nprow.y + brow_ofs, nprow.z + brow_ofs, nprow.w + brow_ofs};
             const int nslot = ninfo & 15;
             const uint32_t map = static_cast<uint32_t>(ninfo >> 4) & 0xFFu;
             bvalid[stage] = static_cast<uint32_t>(nvalid) | (static_cast<uint32_t>(nslot) << 20);
-            if (i + 1 < na) {
+            if (ai + 1 < na) {
               nprow = __ldg(reinterpret_cast<const int4 *>(p.augblocks + td.aug0 + lb + S));
               ninfo = __ldg(&p.augblocks[td.aug0 + lb + S].info);
               nvalid = __ldg(&p.augblocks[td.aug0 + lb + S].valid);
@@ -454,7 +523,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const TileDesc td = tile_desc(mt);
         const int n0 = nt * kBN;
         const int arow = p.a_sorted ? td.row0 : td.contig;
-        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S, FUSED);
         const int nmma = br.count();
         const int nblk = arow < 0 ? 0 : nmma + (merge ? kMergeWBlocks : 0);
         for (int i = 0; i < nblk; ++i) {
@@ -498,7 +567,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tile_coords(tile, p, mt, nt);
         const TileDesc td = tile_desc(mt);
         const int arow = p.a_sorted ? td.row0 : td.contig;
-        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const BlockRange br = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S, FUSED);
         const int nmma = br.count();
         const int nblk = arow < 0 ? 0 : nmma + (merge ? kMergeWBlocks : 0);
         bool ok = true;
@@ -561,7 +630,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         int mt, nt;
         tile_coords(tile, p, mt, nt);
         const int kaug = merge ? p.merge_kaug : (p.tiles ? p.tiles[mt].kaug : 0);
-        const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S);
+        const BlockRange br = block_range(KB, (kaug + kAugBlock - 1) / kAugBlock, q, S, FUSED);
         const int nmma = br.count();
         const int nblk = nmma + (merge ? kMergeWBlocks : 0);
         if (!mbar_wait(acce0 + 8 * acc, aphase ^ 1)) { *abort_flag = 1; break; }
@@ -647,7 +716,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         // through the stage ring as its two W blocks (after its adapter blocks):
         // walk the ring as the producer fills it, wait for each W block, add,
         // store, and release the stage.
-        const int nmma = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S).count();
+        const int nmma = block_range(KB, (td.kaug + kAugBlock - 1) / kAugBlock, q, S, FUSED).count();
         for (int i = 0; i < nmma; ++i)
           if (++ep_stage == kGemmStages) { ep_stage = 0; ep_phase ^= 1; }
         const bool valid = row < td.rows;

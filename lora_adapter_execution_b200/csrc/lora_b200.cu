@@ -65,6 +65,8 @@ int device_state(DeviceState **out) {
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_gemm_kernel<true, kEpiStore>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_gemm_kernel<false, kEpiStore, true>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_gemm_kernel<true, kEpiBwdMulti>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, kGemmSmem) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_shrink_kernel<4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -261,7 +263,7 @@ int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const 
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = S == 1 ? 1 : 2;
-  if (cudaLaunchKernelEx(&cfg, lora_gemm_kernel<false, kEpiStore>, a, b, bl, gp) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, lora_gemm_kernel<false, kEpiStore>, a, b, bl, a, a, a, gp) != cudaSuccess) {
     cudaGetLastError();
     return LORA_ERR_CUDA;
   }
@@ -283,6 +285,13 @@ struct lora_plan {
   const PieceDesc *d_pieces = nullptr;
   std::vector<int32_t> sched;           // the fused GEMM's per-CTA tiles (build_schedule), if persistent
   const int32_t *d_sched = nullptr;     // off[grid + 1] | tiles
+  // the fused forward's launch (lora_linear_fwd_fused): its grid, the shrink
+  // units of each CTA (off[grid + 1] | units), units per m-tile, and its counters
+  // (per m-tile, then the row-copy count), zeroed before each launch
+  int fz_grid = 0;
+  std::vector<int32_t> fz_tab;          // off[grid + 1] | units | need[n_mt]
+  const int32_t *d_fz_off = nullptr, *d_fz_units = nullptr, *d_fz_need = nullptr;
+  int32_t *d_fz_cnt = nullptr;
   void *stage[2] = {nullptr, nullptr};  // pinned host staging of the tables, used in turn
   size_t stage_cap[2] = {0, 0};
   cudaEvent_t stage_ev[2] = {nullptr, nullptr};  // the last copy out of each staging buffer
@@ -399,7 +408,29 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
       build_schedule(hp, std::min(ds->num_sms, n_tiles), default_group_m(n_mt, hp.d_in), pl->sched);
   }
   const size_t b_sched = up(sizeof(int32_t) * pl->sched.size());
-  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug + b_pieces + b_sched;
+  // the fused forward: units dealt to the launch's CTAs in the plan's order
+  // (longest first), round robin; units per m-tile
+  pl->fz_tab.clear();
+  pl->fz_grid = 0;
+  {
+    const int n_mt = static_cast<int>(hp.tiles.size());
+    const int n_tiles = n_mt * static_cast<int>((hp.d_out + kBN - 1) / kBN);
+    const int KB = static_cast<int>((hp.d_in + kBK - 1) / kBK);
+    if (n_tiles > 0) {
+      const int S = fwd_ksplit(n_tiles, KB, ds->num_sms);
+      const int G = S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S;
+      const int nu = static_cast<int>(hp.units.size());
+      pl->fz_grid = G;
+      pl->fz_tab.assign(G + 1 + nu + n_mt, 0);
+      for (int b = 0; b < G; ++b) pl->fz_tab[b + 1] = pl->fz_tab[b] + (nu - b + G - 1) / G;
+      for (int b = 0; b < G; ++b)
+        for (int u = b, j = pl->fz_tab[b]; u < nu; u += G, ++j) pl->fz_tab[G + 1 + j] = u;
+      for (int u = 0; u < nu; ++u) ++pl->fz_tab[G + 1 + nu + hp.units[u].tile];
+    }
+  }
+  const size_t b_fz = up(sizeof(int32_t) * pl->fz_tab.size());
+  const size_t b_fzc = up(sizeof(int32_t) * (hp.tiles.size() + 1));
+  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug + b_pieces + b_sched + b_fz + b_fzc;
   auto release = [&]() {
     if (pl->dev) cudaFree(pl->dev);
     if (pl->scratch) cudaFree(pl->scratch);
@@ -457,6 +488,15 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
   pl->d_pieces = reinterpret_cast<const PieceDesc *>(pieces_dst);
   uint8_t *sched_dst = pieces_dst + b_pieces;
   pl->d_sched = pl->sched.empty() ? nullptr : reinterpret_cast<const int32_t *>(sched_dst);
+  uint8_t *fz_dst = sched_dst + b_sched;
+  {
+    const int G = pl->fz_grid, nu = static_cast<int>(hp.units.size());
+    const int32_t *f = reinterpret_cast<const int32_t *>(fz_dst);
+    pl->d_fz_off = f;
+    pl->d_fz_units = f + G + 1;
+    pl->d_fz_need = f + G + 1 + nu;
+    pl->d_fz_cnt = reinterpret_cast<int32_t *>(fz_dst + b_fz);
+  }
   // The tables go to the device in one copy from one of the plan's two pinned
   // staging buffers, laid out as the device buffer. A staging buffer is refilled
   // only after its previous copy has completed (its event), so consecutive
@@ -490,6 +530,7 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
         sizeof(AugBlockDesc) * hp.augblocks.size());
     put(static_cast<size_t>(pieces_dst - base), hp.pieces.data(), sizeof(PieceDesc) * hp.pieces.size());
     put(static_cast<size_t>(sched_dst - base), pl->sched.data(), sizeof(int32_t) * pl->sched.size());
+    put(static_cast<size_t>(fz_dst - base), pl->fz_tab.data(), sizeof(int32_t) * pl->fz_tab.size());
     ok &= cudaMemcpyAsync(base, h, total, cudaMemcpyHostToDevice, stream) == cudaSuccess;
     ok &= cudaEventRecord(pl->stage_ev[k], stream) == cudaSuccess;
     pl->stage_next = k ^ 1;
@@ -708,6 +749,129 @@ int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   return lora_fused_gemm(plan, X, W, B_pool, Y, stream);
 }
 
+int lora_linear_fwd_fused(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
+                          const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed, uint16_t *Y,
+                          float *U_save, const uint32_t *keep_bits, lora_stream_t stream) {
+  if (!plan || !plan->dev || !X || !W || !A_pool || !B_pool || !scale || !Y) return LORA_ERR_ARG;
+  if (!on_plan_device(plan)) return LORA_ERR_ARG;
+  if (!aligned16(X) || !aligned16(W) || !aligned16(A_pool) || !aligned16(B_pool) || !aligned16(Y)) return LORA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(keep_bits) & 3u) return LORA_ERR_ARG;
+  if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
+  DeviceState *ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LORA_OK) return rc;
+  const HostPlan &hp = plan->hp;
+  const int64_t R = hp.offsets[hp.n_adapters];
+  const bool sorted = hp.xs_offset >= 0;
+  uint16_t *Xs = sorted ? reinterpret_cast<uint16_t *>(plan->scratch + hp.xs_offset) : nullptr;
+  const void *Asrc = sorted ? static_cast<const void *>(Xs) : static_cast<const void *>(X);
+  // the GEMM's maps (as lora_fused_gemm) and the shrink's (as lora_linear_shrink)
+  CUtensorMap mX128, mW, mBl, mX16, mA16;
+  const bool b3d = hp.d_out % 64 == 0;
+  bool ok = make_map(&mX128, Asrc, hp.d_in, hp.T, 64, 128, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= b3d ? make_map_blocks(&mW, W, hp.d_out, hp.d_in, 64, kBN / 64)
+            : make_map(&mW, W, hp.d_out, hp.d_in, 64, 64, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= b3d ? make_map_blocks(&mBl, B_pool, hp.d_out, R, 16, kBN / 64)
+            : make_map(&mBl, B_pool, hp.d_out, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&mX16, Asrc, hp.d_in, hp.T, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  ok &= make_map(&mA16, A_pool, hp.d_in, R, 64, 16, CU_TENSOR_MAP_SWIZZLE_128B);
+  if (!ok) return LORA_ERR_ARG;
+  ShrinkParams sp{};
+  sp.mode = 0;
+  sp.T = static_cast<int32_t>(hp.T);
+  sp.K = static_cast<int32_t>(hp.d_in);
+  sp.ksplit = 1;  // one CTA per unit
+  sp.kslice = static_cast<int32_t>((hp.d_in + kSkBK - 1) / kSkBK * kSkBK);
+  sp.units = plan->d_units;
+  sp.chunks = plan->d_chunks;
+  sp.tiles = plan->d_tiles;
+  sp.perm = plan->d_perm;
+  sp.scale = scale;
+  sp.thr = p_drop > 0.0 ? static_cast<uint64_t>(ldexp(p_drop, 64)) : 0ull;
+  sp.keep_bits = sp.thr ? keep_bits : nullptr;
+  sp.wpr = (hp.d_in + 31) / 32;
+  CUtensorMap mBits16 = mX16;
+  if (sp.keep_bits && sp.wpr % 4 == 0) {
+    cuuint64_t dims[2] = {static_cast<cuuint64_t>(sp.wpr), static_cast<cuuint64_t>(hp.T)};
+    cuuint64_t strides[1] = {static_cast<cuuint64_t>(sp.wpr) * 4};
+    cuuint32_t box[2] = {4, 16};
+    cuuint32_t estr[2] = {1, 1};
+    sp.bits_tma = g_encode(&mBits16, CU_TENSOR_MAP_DATA_TYPE_UINT32, 2, const_cast<uint32_t *>(sp.keep_bits), dims,
+                           strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+    if (!sp.bits_tma) mBits16 = mX16;
+  }
+  sp.seed = seed;
+  sp.inv_keep = p_drop > 0.0 ? static_cast<float>(1.0 / (1.0 - p_drop)) : 1.0f;
+  sp.uimg = plan->scratch;
+  sp.x_sorted = sorted ? 1 : 0;
+  sp.U_save = U_save;
+  sp.r_max = hp.r_max;
+
+  GemmParams gp{};
+  gp.b3d = b3d ? 1 : 0;
+  gp.w3d = b3d ? 1 : 0;
+  gp.T = static_cast<int32_t>(hp.T);
+  gp.K = static_cast<int32_t>(hp.d_in);
+  gp.N = static_cast<int32_t>(hp.d_out);
+  gp.n_mt = static_cast<int32_t>(hp.tiles.size());
+  gp.n_nt = static_cast<int32_t>((hp.d_out + kBN - 1) / kBN);
+  gp.tiles = plan->d_tiles;
+  gp.chunks = plan->d_chunks;
+  gp.perm = plan->d_perm;
+  gp.uimg = plan->scratch;
+  gp.mt_order = plan->d_mt_order;
+  gp.augblocks = plan->d_augblocks;
+  gp.a_sorted = sorted ? 1 : 0;
+  gp.out = reinterpret_cast<__nv_bfloat16 *>(Y);
+  const int n_tiles = gp.n_mt * gp.n_nt;
+  const int KB = (gp.K + kBK - 1) / kBK;
+  gp.group_m = default_group_m(gp.n_mt, gp.K);
+  const int S = fwd_ksplit(n_tiles, KB, ds->num_sms);
+  gp.ksplit = S;
+  const int G = S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S;
+  if (G != plan->fz_grid) return LORA_ERR_ARG;  // the unit lists were dealt for this grid
+  if (S > 1 && plan->xws_S == S) gp.xws = plan->scratch + plan->xws_offset;
+  if (S == 1 && plan->d_sched && static_cast<int>(plan->sched.size()) - n_tiles - 1 == G) {
+    gp.sched_off = plan->d_sched;
+    gp.sched_tiles = plan->d_sched + G + 1;
+  }
+  gp.fz_unit_off = plan->d_fz_off;
+  gp.fz_units = plan->d_fz_units;
+  gp.fz_tile_need = plan->d_fz_need;
+  gp.fz_tile_cnt = plan->d_fz_cnt;
+  gp.fz_grid_cnt = plan->d_fz_cnt + hp.tiles.size();
+  gp.fz_X = X;
+  gp.fz_Xs = Xs;
+  gp.fz_sp = sp;
+  if (cudaMemsetAsync(plan->d_fz_cnt, 0, sizeof(int32_t) * (hp.tiles.size() + 1), stream) != cudaSuccess) {
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  // cooperative: every CTA is resident at once, so the waits for other CTAs'
+  // row copies and shrink units end
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(static_cast<unsigned>(G));
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = kGemmSmem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeCooperative;
+  attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeClusterDimension;
+  attr[1].val.clusterDim.x = S;
+  attr[1].val.clusterDim.y = 1;
+  attr[1].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = S == 1 ? 1 : 2;
+  if (cudaLaunchKernelEx(&cfg, lora_gemm_kernel<false, kEpiStore, true>, mX128, mW, mBl, mX16, mA16, mBits16, gp) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  return LORA_OK;
+}
+
 int lora_base_gemm(const uint16_t *X, const uint16_t *W, uint16_t *Y, int64_t T, int64_t d_in, int64_t d_out,
                    lora_stream_t stream) {
   if (!X || !W || !Y || T <= 0 || d_in < 8 || d_out < 8 || (d_in % 8) || (d_out % 8)) return LORA_ERR_ARG;
@@ -886,7 +1050,7 @@ int lora_linear_bwd(const uint16_t *X, const uint16_t *W, const uint16_t *A, con
     gp.ksplit = 1;
     gp.group_m = default_group_m(gp.n_mt, gp.K);
     const int grid = std::min(ds->num_sms, gp.n_mt * gp.n_nt);
-    lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmemBwd, stream>>>(mdY128, mWt, mWt, gp);
+    lora_gemm_kernel<true, kEpiBwdLora><<<grid, kGemmThreads, kGemmSmemBwd, stream>>>(mdY128, mWt, mWt, mWt, mWt, mWt, gp);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
   // K3c: dB = s * U^T * dY and dA = (D ⊙ X)^T * dU, split over tokens, then
@@ -1113,9 +1277,9 @@ int lora_linear_bwd_multi(lora_plan_t plan, const uint16_t *X, const uint16_t *W
       gp.sched_tiles = plan->d_sched + grid + 1;
     }
     if (thr)
-      lora_gemm_kernel<true, kEpiBwdMulti><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mAl, gp);
+      lora_gemm_kernel<true, kEpiBwdMulti><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mAl, mAl, mAl, mAl, gp);
     else
-      lora_gemm_kernel<true, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mAl, gp);
+      lora_gemm_kernel<true, kEpiStore><<<grid, kGemmThreads, kGemmSmem, stream>>>(mdY128, mWt, mAl, mAl, mAl, mAl, gp);
     if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
   }
   // dB_a = s_a·U^T·dY and dA_a = s_a·(D ⊙ X)^T·G over each segment's pieces, then
@@ -1452,7 +1616,7 @@ int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, con
   const int64_t n_tiles = static_cast<int64_t>(gp.n_mt) * gp.n_nt;
   const unsigned grid = static_cast<unsigned>(std::min<int64_t>(ds->num_sms, n_tiles));
   // no base K blocks: the A map carries the weights' W blocks, the W map is unused
-  lora_gemm_kernel<false, kEpiMergeAdd><<<grid, kGemmThreads, kGemmSmem, stream>>>(mW, mBl, mBl, gp);
+  lora_gemm_kernel<false, kEpiMergeAdd><<<grid, kGemmThreads, kGemmSmem, stream>>>(mW, mBl, mBl, mBl, mBl, mBl, gp);
   return launch_status();
 }
 

@@ -343,30 +343,37 @@ __device__ __forceinline__ void shrink_consume(const ShrinkWarp &w, const Shrink
   }
 }
 
-// Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
-// its rank q contracts columns [q*kslice, (q+1)*kslice).
+// Where the 160 threads that run one shrink unit sit in their CTA: thread lt
+// (0..159) is consumer warp lt / 32 (0..3) or, for lt >= 128, the producer warp.
+// bar_id names the barrier over the 160 (0: they are the whole CTA, and
+// __syncthreads serves); pdl: wait for the previous grid before touching X.
+struct ShrinkRole {
+  int lt;
+  int bar_id;
+  bool pdl;
+};
+
+__device__ __forceinline__ void shrink_bar_all(int bar_id) {
+  if (bar_id == 0) __syncthreads();
+  else asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(kSkThreads) : "memory");
+}
+
+// One shrink unit (one CTA of its cluster): smem is the 1024-aligned stage pool
+// (sk_pool(kMaxNB16) bytes), bars room for 2 * kSkMaxStages mbarriers and a flag.
 template <int kMaxNB16>
-__global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
-    lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows (X, sorted X or dY), box {64, 16}
-                       const __grid_constant__ CUtensorMap mapF16,   // F rows, box {64, 16}
-                       const __grid_constant__ CUtensorMap mapBits16,  // keep bits [T, wpr] u32, box {4, 16}
-                       const ShrinkParams p) {
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
-                                              ~static_cast<uintptr_t>(1023));
+__device__ __forceinline__ void shrink_unit(uint8_t *smem, uint64_t *bars, const CUtensorMap &mapIn16,
+                                            const CUtensorMap &mapF16, const CUtensorMap &mapBits16,
+                                            const ShrinkParams &p, int unit, uint32_t crank, const ShrinkRole role) {
   const uint32_t pool = smem_u32(smem);
   float *fin = reinterpret_cast<float *>(smem + kSkRedBytes);  // in the pool, after the partials
   constexpr int kSkPool = sk_pool(kMaxNB16);
-  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kSkPool);
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * kSkMaxStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kSkMaxStages);
 
-  const int warp = threadIdx.x >> 5;
-  const int lane = threadIdx.x & 31;
-  const int unit = blockIdx.x / p.ksplit;
-  const uint32_t crank = cluster_ctarank();
-  pdl_launch_dependents();  // the fused GEMM may set itself up meanwhile
+  const int tid = role.lt;
+  const int warp = tid >> 5;
+  const int lane = tid & 31;
   if (warp == kSkConsumerWarps && lane == 0) {
     prefetch_tmap(&mapIn16);
     prefetch_tmap(&mapF16);
@@ -400,7 +407,7 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
   const int NB = Rp <= 32 ? 4 : KW;
   const int nstage = min(kSkMaxStages, kSkPool / (NB * stage_bytes));
 
-  if (threadIdx.x == 0) {
+  if (tid == 0) {
     for (int s = 0; s < nstage; ++s) {
       mbar_init(full0 + 8 * s, 1);
       mbar_init(empty0 + 8 * s, kSkConsumerWarps);  // every consumer warp releases a stage
@@ -408,10 +415,10 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
     *abort_flag = 0;
     fence_mbar_init();
   }
-  __syncthreads();
+  shrink_bar_all(role.bar_id);
   // X (or its sorted copy from the row gather) and everything else the launch
   // reads or writes come after the previous kernel on the stream has completed
-  pdl_wait();
+  if (role.pdl) pdl_wait();
 
   if (warp == kSkConsumerWarps) {
     // -------------------------------------------------------------- producer
@@ -494,11 +501,11 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
   // the idle stage pool); fin[row][col] = the sum over the KW warps of a row.
   // Threads work on float4 column groups: nq per row, rpp rows per pass.
   float *red = reinterpret_cast<float *>(smem);
-  __syncthreads();
+  shrink_bar_all(role.bar_id);
   const int nq = g.nn >> 2;
-  const int rpp = static_cast<int>(blockDim.x) / nq;
-  const int tq = static_cast<int>(threadIdx.x) % nq;
-  const int tr = static_cast<int>(threadIdx.x) / nq;
+  const int rpp = kSkThreads / nq;
+  const int tq = tid % nq;
+  const int tr = tid / nq;
   int lmw = 0;
   while ((1 << lmw) < MW) ++lmw;
   if (tr < rpp) {
@@ -573,9 +580,9 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
     // outside the chunk; the chunk's other rows belong to its other pieces
     uint8_t *img = p.uimg + g.uofs;
     const int n8 = g.nn >> 3;
-    const int rp8 = static_cast<int>(blockDim.x) / n8;
-    const int t8 = static_cast<int>(threadIdx.x) % n8;
-    const int trow = static_cast<int>(threadIdx.x) / n8;
+    const int rp8 = kSkThreads / n8;
+    const int t8 = tid % n8;
+    const int trow = tid / n8;
     if (trow < rp8) {
       const int c8 = t8 * 8;
       for (int row = tr0 + trow; row < tr1; row += rp8) {
@@ -611,7 +618,7 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
       // past the adapter's rank up to r_max on the chunk's last piece)
       const int cend = g.last ? p.r_max : min(p.r_max, g.n0 + g.nn);
       const int ncol = max(0, cend - g.n0);
-      const int nw = static_cast<int>(blockDim.x) >> 5;
+      const int nw = kSkThreads >> 5;
       for (int lr = lr0 + warp; lr < lr1; lr += nw) {
         const int64_t orig = p.u_sorted ? static_cast<int64_t>(g.row0 + lr)
                              : g.contig >= 0 ? static_cast<int64_t>(g.contig + lr) : p.perm[g.row0 + lr];
@@ -622,13 +629,30 @@ __global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
   } else {
     // rows of dU are padded to a multiple of 16 ranks with zeros, so that the
     // token contraction reads whole 16-rank groups
-    const int nw = static_cast<int>(blockDim.x) >> 5;
+    const int nw = kSkThreads >> 5;
     const int64_t stride = ((p.r + 15) / 16) * 16;
     for (int lr = lr0 + warp; lr < lr1; lr += nw) {
       float *dst = p.dU + static_cast<int64_t>(g.row0 + lr) * stride + g.n0;
       for (int c = lane; c < g.nn; c += 32) dst[c] = c < g.nvalid ? fin[lr * kShrinkN + c] * p.scale1 : 0.f;
     }
   }
+}
+
+// Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
+// its rank q contracts columns [q*kslice, (q+1)*kslice).
+template <int kMaxNB16>
+__global__ void __launch_bounds__(kSkThreads, sk_ctas_per_sm(kMaxNB16))
+    lora_shrink_kernel(const __grid_constant__ CUtensorMap mapIn16,  // In rows (X, sorted X or dY), box {64, 16}
+                       const __grid_constant__ CUtensorMap mapF16,   // F rows, box {64, 16}
+                       const __grid_constant__ CUtensorMap mapBits16,  // keep bits [T, wpr] u32, box {4, 16}
+                       const ShrinkParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~static_cast<uintptr_t>(1023));
+  pdl_launch_dependents();  // the fused GEMM may set itself up meanwhile
+  shrink_unit<kMaxNB16>(smem, reinterpret_cast<uint64_t *>(smem + sk_pool(kMaxNB16)), mapIn16, mapF16, mapBits16, p,
+                        static_cast<int>(blockIdx.x) / p.ksplit, cluster_ctarank(),
+                        ShrinkRole{static_cast<int>(threadIdx.x), 0, true});
 }
 
 // ------------------------------------------------------------------ token contraction
