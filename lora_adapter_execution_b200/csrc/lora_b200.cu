@@ -292,6 +292,10 @@ struct lora_plan {
   std::vector<int32_t> fz_tab;          // off[grid + 1] | units | need[n_mt]
   const int32_t *d_fz_off = nullptr, *d_fz_units = nullptr, *d_fz_need = nullptr;
   int32_t *d_fz_cnt = nullptr;
+  // the multi-adapter backward's contraction: its pieces dealt into contiguous
+  // ranges of about equal stage counts, one range per grid row (off[P + 1])
+  std::vector<int32_t> ranges;
+  const int32_t *d_ranges = nullptr;
   void *stage[2] = {nullptr, nullptr};  // pinned host staging of the tables, used in turn
   size_t stage_cap[2] = {0, 0};
   cudaEvent_t stage_ev[2] = {nullptr, nullptr};  // the last copy out of each staging buffer
@@ -429,8 +433,28 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
     }
   }
   const size_t b_fz = up(sizeof(int32_t) * pl->fz_tab.size());
+  // about two CTAs per SM over the wider of the two contractions' column blocks
+  pl->ranges.clear();
+  {
+    const int np = static_cast<int>(hp.pieces.size());
+    const int64_t cols = (std::max(hp.d_in, hp.d_out) + kTcCols - 1) / kTcCols;
+    const int P = static_cast<int>(std::max<int64_t>(
+        1, std::min<int64_t>(std::max(np, 1), (2 * ds->num_sms + cols / 2) / std::max<int64_t>(1, cols))));
+    int64_t total = 0;
+    for (const PieceDesc &pd : hp.pieces) total += (pd.len + kTcTok - 1) / kTcTok;
+    pl->ranges.assign(P + 1, np);
+    pl->ranges[0] = 0;
+    int64_t cum = 0;
+    int k = 1;
+    for (int i = 0; i < np && k < P; ++i) {
+      cum += (hp.pieces[i].len + kTcTok - 1) / kTcTok;
+      while (k < P && cum * P >= total * k) pl->ranges[k++] = i + 1;
+    }
+  }
+  const size_t b_rng = up(sizeof(int32_t) * pl->ranges.size());
   const size_t b_fzc = up(sizeof(int32_t) * (hp.tiles.size() + 1));
-  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug + b_pieces + b_sched + b_fz + b_fzc;
+  const size_t total = b_perm + b_tiles + b_chunks + b_units + b_order + b_aug + b_pieces + b_sched + b_fz + b_fzc +
+                       b_rng;
   auto release = [&]() {
     if (pl->dev) cudaFree(pl->dev);
     if (pl->scratch) cudaFree(pl->scratch);
@@ -497,6 +521,8 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
     pl->d_fz_need = f + G + 1 + nu;
     pl->d_fz_cnt = reinterpret_cast<int32_t *>(fz_dst + b_fz);
   }
+  uint8_t *rng_dst = fz_dst + b_fz + b_fzc;
+  pl->d_ranges = reinterpret_cast<const int32_t *>(rng_dst);
   // The tables go to the device in one copy from one of the plan's two pinned
   // staging buffers, laid out as the device buffer. A staging buffer is refilled
   // only after its previous copy has completed (its event), so consecutive
@@ -531,6 +557,7 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
     put(static_cast<size_t>(pieces_dst - base), hp.pieces.data(), sizeof(PieceDesc) * hp.pieces.size());
     put(static_cast<size_t>(sched_dst - base), pl->sched.data(), sizeof(int32_t) * pl->sched.size());
     put(static_cast<size_t>(fz_dst - base), pl->fz_tab.data(), sizeof(int32_t) * pl->fz_tab.size());
+    put(static_cast<size_t>(rng_dst - base), pl->ranges.data(), sizeof(int32_t) * pl->ranges.size());
     ok &= cudaMemcpyAsync(base, h, total, cudaMemcpyHostToDevice, stream) == cudaSuccess;
     ok &= cudaEventRecord(pl->stage_ev[k], stream) == cudaSuccess;
     pl->stage_next = k ^ 1;
@@ -1169,7 +1196,7 @@ int lora_linear_bwd_multi(lora_plan_t plan, const uint16_t *X, const uint16_t *W
     return LORA_ERR_ARG;
   if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
   const HostPlan &hp = plan->hp;
-  if (hp.pieces.size() > 65535) return LORA_ERR_ARG;  // one grid row per piece
+  if (hp.pieces.size() > 65535) return LORA_ERR_ARG;  // one grid row of the reduction per piece
   const BwdMultiLayout Lw = bwd_multi_layout(hp);
   if (!workspace || workspace_bytes < static_cast<size_t>(Lw.total) ||
       (reinterpret_cast<uintptr_t>(workspace) & 255u))
@@ -1306,18 +1333,21 @@ int lora_linear_bwd_multi(lora_plan_t plan, const uint16_t *X, const uint16_t *W
         use_bits = false;
     }
     const unsigned n_pieces = static_cast<unsigned>(hp.pieces.size());
+    const unsigned n_ranges = static_cast<unsigned>(plan->ranges.size() - 1);
     const unsigned groups = static_cast<unsigned>((rp + kTcMaxR - 1) / kTcMaxR);
     const int smem = tc_smem(std::min(rp, kTcMaxR));  // the widest rank group of any piece
     TcParams tp{};
     tp.T = static_cast<int32_t>(T);
     tp.pieces = plan->d_pieces;
+    tp.range_off = plan->d_ranges;
+    tp.rp = rp;
     tp.scale = scale;
     // dB: In = dY, G = U, no mask
     tp.N = static_cast<int32_t>(d_out);
     tp.factor = 1.0f;
     tp.out = dB_pool;
     tp.partial = pdB;
-    dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), n_pieces, groups);
+    dim3 grid_b(static_cast<unsigned>((d_out + kTcCols - 1) / kTcCols), n_ranges, groups);
     lora_tcontract_kernel<<<grid_b, kTcThreads, smem, stream>>>(mIn64b, mU[3], mBits, mU[0], mU[1], mU[2], tp);
     // dA: In = X with the dropout mask, G = dY·B^T; the mask's 1/(1 - p) and s_a
     // scale the sums
@@ -1330,7 +1360,7 @@ int lora_linear_bwd_multi(lora_plan_t plan, const uint16_t *X, const uint16_t *W
     tp.factor = inv_keep;
     tp.out = dA_pool;
     tp.partial = pdA;
-    dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), n_pieces, groups);
+    dim3 grid_a(static_cast<unsigned>((d_in + kTcCols - 1) / kTcCols), n_ranges, groups);
     lora_tcontract_kernel<<<grid_a, kTcThreads, smem, stream>>>(mIn64a, mG[3], mBits, mG[0], mG[1], mG[2], tp);
     if (hp.partial_rows > 0) {
       const unsigned gb = static_cast<unsigned>(std::min<int64_t>((hp.r_max * d_out + 255) / 256, 256));

@@ -696,11 +696,15 @@ struct TcParams {
   int64_t wpr;
   float *partial;          // [splits][r_total][N]; piece mode: [partial rows][N]
   // piece mode (pieces != null, multi-adapter backward): CTA (x, y, z) takes
-  // column block x of piece y, ranks [64z, 64z + 64) of the piece's adapter; its
-  // rank group's width selects the G map. A segment of one piece writes
+  // column block x of pieces range_off[y] .. range_off[y + 1] - 1, one after
+  // another through one stage ring, ranks [64z, 64z + 64) of each piece's
+  // adapter (rp: the ranks rounded up to 16 of the widest adapter; the group's
+  // width selects the G map). A segment of one piece writes
   // out[(pool_row + k) * N + n] = scale[adapter] * factor * sum; the pieces of a
   // longer segment write partial rows (partial_row + k) for a later reduction.
   const PieceDesc *pieces;
+  const int32_t *range_off;
+  int32_t rp;
   const float *scale;
   float factor;
   float *out;
@@ -742,23 +746,35 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~static_cast<uintptr_t>(1023));
-  // this CTA's ranks [k0, k0 + r) (r a multiple of 16; r_valid real ones) and tokens [t0, t1)
-  int r = p.r, r_valid = p.r_valid, k0 = p.k0, t0, t1;
-  PieceDesc pc{};
+  // this CTA's ranks [k0, k0 + r) (r a multiple of 16) and its segments lo .. hi - 1:
+  // one token split, or a range of pieces
+  int r = p.r, k0 = p.k0, lo = 0, hi = 1;
   const CUtensorMap *gmap = &mapG;
   if (p.pieces) {
-    pc = p.pieces[blockIdx.y];
     k0 = static_cast<int>(blockIdx.z) * kTcMaxR;
-    if (k0 >= pc.rank) return;  // no barrier has been set up yet
-    r = min(kTcMaxR, (pc.rank + 15) / 16 * 16 - k0);
-    r_valid = min(r, pc.rank - k0);
+    r = min(kTcMaxR, p.rp - k0);
+    if (r <= 0) return;  // no barrier has been set up yet
     gmap = r == 16 ? &mapG16 : r == 32 ? &mapG32 : r == 48 ? &mapG48 : &mapG;
-    t0 = pc.in_row;  // In (and keep-bit) rows; G rows are sorted positions from pc.start
-    t1 = pc.in_row + pc.len;
-  } else {
-    t0 = blockIdx.y * p.tsplit;
-    t1 = min(p.T, t0 + p.tsplit);
+    lo = p.range_off[blockIdx.y];
+    hi = p.range_off[blockIdx.y + 1];
   }
+  // segment s: In (and keep-bit) rows [t0, t1), G rows from g0 (piece mode: the
+  // piece's sorted positions); false when the segment's adapter has no rank in
+  // this CTA's group
+  auto segment = [&](int s, int &t0, int &t1, int &g0) -> bool {
+    if (p.pieces) {
+      const PieceDesc pc = p.pieces[s];
+      if (pc.rank <= k0) return false;
+      t0 = pc.in_row;
+      t1 = pc.in_row + pc.len;
+      g0 = pc.start;
+    } else {
+      t0 = blockIdx.y * p.tsplit;
+      t1 = min(p.T, t0 + p.tsplit);
+      g0 = t0;
+    }
+    return true;
+  };
   const bool bits = p.keep_bits != nullptr;
   const int mblocks = (r + 15) / 16;
   const int in_bytes = kTcTok * kTcCols * 2;    // 16 KB (two 8 KB halves)
@@ -776,8 +792,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
   const int n0 = blockIdx.x * kTcCols;
-  const int nblk = t1 > t0 ? (t1 - t0 + kTcTok - 1) / kTcTok : 0;
-  const int g0 = p.pieces ? pc.start : t0;  // G row of token t0
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < nstage; ++s) {
@@ -795,17 +809,23 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       if (bits) prefetch_tmap(&mapBits);
       int stage = 0;
       uint32_t phase = 0;
-      for (int b = 0; b < nblk; ++b) {
-        if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) break;
-        const uint32_t fb = full0 + 8 * stage;
-        const uint32_t sb = pool + stage * stage_bytes;
-        const int t = t0 + b * kTcTok;
-        mbar_arrive_expect_tx(fb, in_bytes + g_bytes + bits_bytes);
-        tma_load_2d(sb, &mapIn, fb, n0, t);
-        tma_load_2d(sb + 8192, &mapIn, fb, n0 + 64, t);
-        tma_load_2d(sb + in_bytes, gmap, fb, k0, t - t0 + g0);  // this CTA's group of ranks
-        if (bits) tma_load_2d(sb + in_bytes + g_pad, &mapBits, fb, n0 / 32, t);
-        if (++stage == nstage) { stage = 0; phase ^= 1; }
+      bool ok = true;
+      for (int sg = lo; sg < hi && ok; ++sg) {
+        int t0, t1, g0;
+        if (!segment(sg, t0, t1, g0)) continue;
+        const int nblk = t1 > t0 ? (t1 - t0 + kTcTok - 1) / kTcTok : 0;
+        for (int b = 0; b < nblk; ++b) {
+          if (!mbar_wait(empty0 + 8 * stage, phase ^ 1)) { ok = false; break; }
+          const uint32_t fb = full0 + 8 * stage;
+          const uint32_t sb = pool + stage * stage_bytes;
+          const int t = t0 + b * kTcTok;
+          mbar_arrive_expect_tx(fb, in_bytes + g_bytes + bits_bytes);
+          tma_load_2d(sb, &mapIn, fb, n0, t);
+          tma_load_2d(sb + 8192, &mapIn, fb, n0 + 64, t);
+          tma_load_2d(sb + in_bytes, gmap, fb, k0, t - t0 + g0);  // this CTA's group of ranks
+          if (bits) tma_load_2d(sb + in_bytes + g_pad, &mapBits, fb, n0 / 32, t);
+          if (++stage == nstage) { stage = 0; phase ^= 1; }
+        }
       }
     }
     return;  // no block-wide barrier follows
@@ -829,8 +849,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const int chunk = (cin >> 3) + 2 * g + (mi >> 1);
       boff[ks][g] = half * 8192 + tr * 128 + (((chunk ^ (tr & 7)) & 7) << 4);
     }
-  // G^T fragments (ranks x tokens, row-major) from the hi / lo images: rank rows
-  // (q & 1)*8 + (lane & 7) of the 16-rank block, token chunk ks*2 + (q >> 1)
+  // G^T fragments (ranks x tokens, row-major) from the hi / mid / lo images:
+  // rank rows (q & 1)*8 + (lane & 7) of the 16-rank block, token chunk ks*2 + (q >> 1)
   uint32_t aoff[4];
 #pragma unroll
   for (int ks = 0; ks < 4; ++ks) {
@@ -840,166 +860,178 @@ __global__ void __launch_bounds__(kTcThreads, 2)
   const int q2 = 2 * (lane & 3);
   const int tid = static_cast<int>(threadIdx.x);  // 0 .. 127
 
-  float acc[4][2][2][4];  // [m-block][column group][n8][fragment]
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int g = 0; g < 2; ++g)
-#pragma unroll
-      for (int j = 0; j < 2; ++j)
-#pragma unroll
-        for (int e = 0; e < 4; ++e) acc[i][g][j][e] = 0.f;
-
   int stage = 0;
   uint32_t phase = 0;
-  for (int b = 0; b < nblk; ++b) {
-    if (!mbar_wait(full0 + 8 * stage, phase)) break;
-    const uint32_t sb = pool + stage * stage_bytes;
-    uint8_t *const sbp = smem + (sb - pool);
-    // G^T images of this stage. Work item = (token pair tp, 4 consecutive ranks
-    // from k4): G[2tp][k4 .. k4 + 3] and G[2tp + 1][k4 .. k4 + 3] as two 16-byte
-    // reads (consecutive threads take consecutive ranks, so the reads do not
-    // collide on banks), written as (hi, lo) bf16 pairs at rank rows k4 .. k4 + 3,
-    // tokens 2tp and 2tp + 1. Rank rows from r to 16 * mblocks are zero, and so
-    // are the columns of tokens at or past t1 (in piece mode the stage's last
-    // rows can be the next segment's tokens, which must not enter the sums).
-    {
-      const int tb = t0 + b * kTcTok;
-      const float *graw = reinterpret_cast<const float *>(sbp + in_bytes);
-      uint8_t *ghi = sbp + conv_off;
-      uint8_t *gmid = ghi + mblocks * 2048;
-      uint8_t *glo = gmid + mblocks * 2048;
-      const int q4 = mblocks * 4;  // 4-rank groups per token pair
-      for (int item = tid; item < 32 * q4; item += kTcConsumerWarps * 32) {
-        const int tp = item / q4;
-        const int k4 = (item - tp * q4) * 4;
-        float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
-        if (k4 < r) {  // r % 16 == 0: a group is all in or all out
-          if (tb + 2 * tp < t1) v0 = *reinterpret_cast<const float4 *>(graw + (2 * tp) * r + k4);
-          if (tb + 2 * tp + 1 < t1) v1 = *reinterpret_cast<const float4 *>(graw + (2 * tp + 1) * r + k4);
-        }
-        const float a0[4] = {v0.x, v0.y, v0.z, v0.w};
-        const float a1[4] = {v1.x, v1.y, v1.z, v1.w};
+  bool ok = true;
+  for (int sg = lo; sg < hi && ok; ++sg) {
+    int t0, t1, g0;
+    if (!segment(sg, t0, t1, g0)) continue;
+    const int nblk = t1 > t0 ? (t1 - t0 + kTcTok - 1) / kTcTok : 0;
+    float acc[4][2][2][4];  // [m-block][column group][n8][fragment]
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          const int k = k4 + u;
-          uint32_t hi, mid, lo;
-          split3_pair(a0[u], a1[u], hi, mid, lo);
-          const uint32_t off = k * 128 + ((((tp >> 2) ^ (k & 7)) & 7) << 4) + (tp & 3) * 4;
-          *reinterpret_cast<uint32_t *>(ghi + off) = hi;
-          *reinterpret_cast<uint32_t *>(gmid + off) = mid;
-          *reinterpret_cast<uint32_t *>(glo + off) = lo;
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int g = 0; g < 2; ++g)
+#pragma unroll
+        for (int j = 0; j < 2; ++j)
+#pragma unroll
+          for (int e = 0; e < 4; ++e) acc[i][g][j][e] = 0.f;
+
+    for (int b = 0; b < nblk; ++b) {
+      if (!mbar_wait(full0 + 8 * stage, phase)) { ok = false; break; }
+      const uint32_t sb = pool + stage * stage_bytes;
+      uint8_t *const sbp = smem + (sb - pool);
+      // G^T images of this stage. Work item = (token pair tp, 4 consecutive ranks
+      // from k4): G[2tp][k4 .. k4 + 3] and G[2tp + 1][k4 .. k4 + 3] as two 16-byte
+      // reads (consecutive threads take consecutive ranks, so the reads do not
+      // collide on banks), written as (hi, mid, lo) bf16 pairs at rank rows
+      // k4 .. k4 + 3, tokens 2tp and 2tp + 1. Rank rows from r to 16 * mblocks
+      // are zero, and so are the columns of tokens at or past t1 (in piece mode
+      // the stage's last rows can be the next segment's tokens, which must not
+      // enter the sums).
+      {
+        const int tb = t0 + b * kTcTok;
+        const float *graw = reinterpret_cast<const float *>(sbp + in_bytes);
+        uint8_t *ghi = sbp + conv_off;
+        uint8_t *gmid = ghi + mblocks * 2048;
+        uint8_t *glo = gmid + mblocks * 2048;
+        const int q4 = mblocks * 4;  // 4-rank groups per token pair
+        for (int item = tid; item < 32 * q4; item += kTcConsumerWarps * 32) {
+          const int tp = item / q4;
+          const int k4 = (item - tp * q4) * 4;
+          float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
+          if (k4 < r) {  // r % 16 == 0: a group is all in or all out
+            if (tb + 2 * tp < t1) v0 = *reinterpret_cast<const float4 *>(graw + (2 * tp) * r + k4);
+            if (tb + 2 * tp + 1 < t1) v1 = *reinterpret_cast<const float4 *>(graw + (2 * tp + 1) * r + k4);
+          }
+          const float a0[4] = {v0.x, v0.y, v0.z, v0.w};
+          const float a1[4] = {v1.x, v1.y, v1.z, v1.w};
+#pragma unroll
+          for (int u = 0; u < 4; ++u) {
+            const int k = k4 + u;
+            uint32_t hi, mid, lo;
+            split3_pair(a0[u], a1[u], hi, mid, lo);
+            const uint32_t off = k * 128 + ((((tp >> 2) ^ (k & 7)) & 7) << 4) + (tp & 3) * 4;
+            *reinterpret_cast<uint32_t *>(ghi + off) = hi;
+            *reinterpret_cast<uint32_t *>(gmid + off) = mid;
+            *reinterpret_cast<uint32_t *>(glo + off) = lo;
+          }
         }
       }
-    }
-    asm volatile("bar.sync 1, %0;" ::"n"(kTcConsumerWarps * 32) : "memory");
-    const uint32_t ghi_s = sb + conv_off;
-    const uint32_t gmid_s = ghi_s + mblocks * 2048;
-    const uint32_t glo_s = gmid_s + mblocks * 2048;
-    const uint32_t *bs = reinterpret_cast<const uint32_t *>(sbp + in_bytes + g_pad);
-    const int tbase = t0 + b * kTcTok;
+      asm volatile("bar.sync 1, %0;" ::"n"(kTcConsumerWarps * 32) : "memory");
+      const uint32_t ghi_s = sb + conv_off;
+      const uint32_t gmid_s = ghi_s + mblocks * 2048;
+      const uint32_t glo_s = gmid_s + mblocks * 2048;
+      const uint32_t *bs = reinterpret_cast<const uint32_t *>(sbp + in_bytes + g_pad);
+      const int tbase = t0 + b * kTcTok;
 #pragma unroll
-    for (int ks = 0; ks < 4; ++ks) {
-      uint32_t bf[2][4];
+      for (int ks = 0; ks < 4; ++ks) {
+        uint32_t bf[2][4];
 #pragma unroll
-      for (int g = 0; g < 2; ++g) ldsm_x4_t(sb + boff[ks][g], bf[g][0], bf[g][1], bf[g][2], bf[g][3]);
-      if (p.thr != 0) {
-        // bf[g][0]: tokens tl, tl + 1 of column c = n0 + cw + 16g + lane/4;
-        // [1]: tokens + 8; [2], [3]: column + 8
-        const int tl = ks * 16 + q2;
-        if (bits) {
-          // the stage's bits: [64 tokens][4 words] for its 128 columns; the
-          // warp's 32 columns are word cw / 32, and c, c + 8 share it
-          const int wd = cw >> 5;
-          const uint32_t w0 = bs[tl * 4 + wd], w1 = bs[(tl + 1) * 4 + wd];
-          const uint32_t w8 = bs[(tl + 8) * 4 + wd], w9 = bs[(tl + 9) * 4 + wd];
+        for (int g = 0; g < 2; ++g) ldsm_x4_t(sb + boff[ks][g], bf[g][0], bf[g][1], bf[g][2], bf[g][3]);
+        if (p.thr != 0) {
+          // bf[g][0]: tokens tl, tl + 1 of column c = n0 + cw + 16g + lane/4;
+          // [1]: tokens + 8; [2], [3]: column + 8
+          const int tl = ks * 16 + q2;
+          if (bits) {
+            // the stage's bits: [64 tokens][4 words] for its 128 columns; the
+            // warp's 32 columns are word cw / 32, and c, c + 8 share it
+            const int wd = cw >> 5;
+            const uint32_t w0 = bs[tl * 4 + wd], w1 = bs[(tl + 1) * 4 + wd];
+            const uint32_t w8 = bs[(tl + 8) * 4 + wd], w9 = bs[(tl + 9) * 4 + wd];
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const int sh = 16 * g + (lane >> 2);
+              const uint32_t x0 = w0 >> sh, x1 = w1 >> sh, x8 = w8 >> sh, x9 = w9 >> sh;
+              bf[g][0] &= keep_pair_t<0xCC88>(x0, x1);
+              bf[g][1] &= keep_pair_t<0xCC88>(x8, x9);
+              bf[g][2] &= keep_pair_t<0xDD99>(x0, x1);
+              bf[g][3] &= keep_pair_t<0xDD99>(x8, x9);
+            }
+          } else {
+            // the mask is indexed by original token: rows past the token range
+            // meet zero G columns, their bits are never used
+            const int tk = tbase + tl;
+            int64_t o0 = tk, o1 = tk + 1, o8 = tk + 8, o9 = tk + 9;
+            if (p.perm) {
+              o0 = p.perm[min(tk, t1 - 1)];
+              o1 = p.perm[min(tk + 1, t1 - 1)];
+              o8 = p.perm[min(tk + 8, t1 - 1)];
+              o9 = p.perm[min(tk + 9, t1 - 1)];
+            }
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              const int c = n0 + cw + 16 * g + (lane >> 2);
+              bf[g][0] = mask_pair(bf[g][0], keep_elem(p.seed, p.thr, o0, c, p.N), keep_elem(p.seed, p.thr, o1, c, p.N));
+              bf[g][1] = mask_pair(bf[g][1], keep_elem(p.seed, p.thr, o8, c, p.N), keep_elem(p.seed, p.thr, o9, c, p.N));
+              bf[g][2] = mask_pair(bf[g][2], keep_elem(p.seed, p.thr, o0, c + 8, p.N), keep_elem(p.seed, p.thr, o1, c + 8, p.N));
+              bf[g][3] = mask_pair(bf[g][3], keep_elem(p.seed, p.thr, o8, c + 8, p.N), keep_elem(p.seed, p.thr, o9, c + 8, p.N));
+            }
+          }
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          if (i >= mblocks) break;
+          uint32_t h0, h1, h2, h3, m0, m1, m2, m3, l0, l1, l2, l3;
+          ldsm_x4(ghi_s + i * 2048 + aoff[ks], h0, h1, h2, h3);
+          ldsm_x4(gmid_s + i * 2048 + aoff[ks], m0, m1, m2, m3);
+          ldsm_x4(glo_s + i * 2048 + aoff[ks], l0, l1, l2, l3);
 #pragma unroll
           for (int g = 0; g < 2; ++g) {
-            const int sh = 16 * g + (lane >> 2);
-            const uint32_t x0 = w0 >> sh, x1 = w1 >> sh, x8 = w8 >> sh, x9 = w9 >> sh;
-            bf[g][0] &= keep_pair_t<0xCC88>(x0, x1);
-            bf[g][1] &= keep_pair_t<0xCC88>(x8, x9);
-            bf[g][2] &= keep_pair_t<0xDD99>(x0, x1);
-            bf[g][3] &= keep_pair_t<0xDD99>(x8, x9);
-          }
-        } else {
-          // the mask is indexed by original token: rows past the token range are
-          // zero in the stage, their bits are never used
-          const int tk = tbase + tl;
-          int64_t o0 = tk, o1 = tk + 1, o8 = tk + 8, o9 = tk + 9;
-          if (p.perm) {
-            o0 = p.perm[min(tk, t1 - 1)];
-            o1 = p.perm[min(tk + 1, t1 - 1)];
-            o8 = p.perm[min(tk + 8, t1 - 1)];
-            o9 = p.perm[min(tk + 9, t1 - 1)];
-          }
-#pragma unroll
-          for (int g = 0; g < 2; ++g) {
-            const int c = n0 + cw + 16 * g + (lane >> 2);
-            bf[g][0] = mask_pair(bf[g][0], keep_elem(p.seed, p.thr, o0, c, p.N), keep_elem(p.seed, p.thr, o1, c, p.N));
-            bf[g][1] = mask_pair(bf[g][1], keep_elem(p.seed, p.thr, o8, c, p.N), keep_elem(p.seed, p.thr, o9, c, p.N));
-            bf[g][2] = mask_pair(bf[g][2], keep_elem(p.seed, p.thr, o0, c + 8, p.N), keep_elem(p.seed, p.thr, o1, c + 8, p.N));
-            bf[g][3] = mask_pair(bf[g][3], keep_elem(p.seed, p.thr, o8, c + 8, p.N), keep_elem(p.seed, p.thr, o9, c + 8, p.N));
+            // smallest parts first, so the partial sums grow from the small end
+            mma_bf16_16816(acc[i][g][0], l0, l1, l2, l3, bf[g][0], bf[g][1]);
+            mma_bf16_16816(acc[i][g][1], l0, l1, l2, l3, bf[g][2], bf[g][3]);
+            mma_bf16_16816(acc[i][g][0], m0, m1, m2, m3, bf[g][0], bf[g][1]);
+            mma_bf16_16816(acc[i][g][1], m0, m1, m2, m3, bf[g][2], bf[g][3]);
+            mma_bf16_16816(acc[i][g][0], h0, h1, h2, h3, bf[g][0], bf[g][1]);
+            mma_bf16_16816(acc[i][g][1], h0, h1, h2, h3, bf[g][2], bf[g][3]);
           }
         }
       }
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        if (i >= mblocks) break;
-        uint32_t h0, h1, h2, h3, m0, m1, m2, m3, l0, l1, l2, l3;
-        ldsm_x4(ghi_s + i * 2048 + aoff[ks], h0, h1, h2, h3);
-        ldsm_x4(gmid_s + i * 2048 + aoff[ks], m0, m1, m2, m3);
-        ldsm_x4(glo_s + i * 2048 + aoff[ks], l0, l1, l2, l3);
-#pragma unroll
-        for (int g = 0; g < 2; ++g) {
-          // smallest parts first, so the partial sums grow from the small end
-          mma_bf16_16816(acc[i][g][0], l0, l1, l2, l3, bf[g][0], bf[g][1]);
-          mma_bf16_16816(acc[i][g][1], l0, l1, l2, l3, bf[g][2], bf[g][3]);
-          mma_bf16_16816(acc[i][g][0], m0, m1, m2, m3, bf[g][0], bf[g][1]);
-          mma_bf16_16816(acc[i][g][1], m0, m1, m2, m3, bf[g][2], bf[g][3]);
-          mma_bf16_16816(acc[i][g][0], h0, h1, h2, h3, bf[g][0], bf[g][1]);
-          mma_bf16_16816(acc[i][g][1], h0, h1, h2, h3, bf[g][2], bf[g][3]);
-        }
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(empty0 + 8 * stage);
+      if (++stage == nstage) { stage = 0; phase ^= 1; }
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(empty0 + 8 * stage);
-    if (++stage == nstage) { stage = 0; phase ^= 1; }
-  }
-  // write partial[q][k0 + k][n] for the group's real ranks; piece mode: the
-  // adapter's gradient rows (scaled) or the piece's partial rows
-  float *out;
-  float f = 1.f;
-  if (p.pieces) {
-    if (pc.seg_pieces == 1) {
-      out = p.out + (static_cast<int64_t>(pc.pool_row) + k0) * p.N;
-      f = p.scale[pc.adapter] * p.factor;
+    if (!ok) break;
+    // write partial[q][k0 + k][n] for the group's real ranks; piece mode: the
+    // adapter's gradient rows (scaled) or the piece's partial rows. The stores
+    // overlap the copies of the next segment's stages.
+    float *out;
+    float f = 1.f;
+    int r_valid = p.r_valid;
+    if (p.pieces) {
+      const PieceDesc pc = p.pieces[sg];
+      r_valid = min(r, pc.rank - k0);
+      if (pc.seg_pieces == 1) {
+        out = p.out + (static_cast<int64_t>(pc.pool_row) + k0) * p.N;
+        f = p.scale[pc.adapter] * p.factor;
+      } else {
+        out = p.partial + (static_cast<int64_t>(pc.partial_row) + k0) * p.N;
+      }
     } else {
-      out = p.partial + (static_cast<int64_t>(pc.partial_row) + k0) * p.N;
+      out = p.partial + (static_cast<int64_t>(blockIdx.y) * p.r_total + k0) * p.N;
     }
-  } else {
-    out = p.partial + (static_cast<int64_t>(blockIdx.y) * p.r_total + k0) * p.N;
-  }
 #pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    if (i >= mblocks) break;
+    for (int i = 0; i < 4; ++i) {
+      if (i >= mblocks) break;
 #pragma unroll
-    for (int g = 0; g < 2; ++g)
+      for (int g = 0; g < 2; ++g)
 #pragma unroll
-      for (int j = 0; j < 2; ++j) {
-        const int k = i * 16 + (lane >> 2);
-        const int c = n0 + cw + 16 * g + j * 8 + q2;
-        if (c < p.N) {
-          if (k < r_valid) {
-            out[static_cast<int64_t>(k) * p.N + c] = f * acc[i][g][j][0];
-            out[static_cast<int64_t>(k) * p.N + c + 1] = f * acc[i][g][j][1];
-          }
-          if (k + 8 < r_valid) {
-            out[static_cast<int64_t>(k + 8) * p.N + c] = f * acc[i][g][j][2];
-            out[static_cast<int64_t>(k + 8) * p.N + c + 1] = f * acc[i][g][j][3];
+        for (int j = 0; j < 2; ++j) {
+          const int k = i * 16 + (lane >> 2);
+          const int c = n0 + cw + 16 * g + j * 8 + q2;
+          if (c < p.N) {
+            if (k < r_valid) {
+              out[static_cast<int64_t>(k) * p.N + c] = f * acc[i][g][j][0];
+              out[static_cast<int64_t>(k) * p.N + c + 1] = f * acc[i][g][j][1];
+            }
+            if (k + 8 < r_valid) {
+              out[static_cast<int64_t>(k + 8) * p.N + c] = f * acc[i][g][j][2];
+              out[static_cast<int64_t>(k + 8) * p.N + c + 1] = f * acc[i][g][j][3];
+            }
           }
         }
-      }
+    }
   }
 }
 

@@ -80,6 +80,8 @@ CASES = {
     # one adapter: long segment, several pieces and their reduction
     "single": dict(name="finetune", kw=dict(T=2600, d_in=264, d_out=200)),
     "decode_small": dict(name="decode", kw=dict(T=300, d_in=328, d_out=264, n_adapters=40)),
+    # ~200 short segments dealt into ~18 ranges: each CTA's range holds many pieces
+    "fleet_ranges": dict(name="fleet", kw=dict(T=1500, d_in=2048, d_out=1024, n_adapters=300)),
 }
 
 
