@@ -62,6 +62,8 @@ def lib():
                                  _dbl, _u64, _vp, _vp, _i64, _vp, _vp, _vp]
         L.oracle_switch.restype = None
         L.oracle_switch.argtypes = [_i64, _i64, _i64, _i32, _vp, _vp, _vp, _vp, _i32, _vp, _vp, _vp]
+        L.oracle_qr.restype = None
+        L.oracle_qr.argtypes = [_i64, _i64, _i64, _vp, _vp, _vp]
         L.oracle_num_threads.restype = ctypes.c_int
         L.oracle_num_threads.argtypes = []
         _lib = L
@@ -166,3 +168,18 @@ def switch(W, A_pool, B_pool, ranks, term_adapter, term_coef):
     lib().oracle_switch(L, d_in, d_out, ranks.shape[0], _p(ranks), _p(W), _p(_c(A_pool, np.uint16)),
                         _p(_c(B_pool, np.uint16)), ta.shape[0], _p(ta), _p(tc), _p(out))
     return out
+
+
+def qr(A, want_q=True):
+    """Householder QR of each matrix of A (fp64 [batch, m, n], or [m, n]): R
+    [batch, n, n] and Q [batch, m, n] (see oracle_qr)."""
+    A = np.asarray(A, dtype=np.float64)
+    single = A.ndim == 2
+    A = _c(A[None] if single else A, np.float64)
+    b, m, n = A.shape
+    R = np.empty((b, n, n), dtype=np.float64)
+    Q = np.empty((b, m, n), dtype=np.float64) if want_q else None
+    lib().oracle_qr(b, m, n, _p(A), _p(R), _p(Q))
+    if single:
+        return R[0], (Q[0] if want_q else None)
+    return R, Q

@@ -331,6 +331,65 @@ void oracle_switch(int64_t L, int64_t d_in, int64_t d_out, int32_t n_adapters, c
     free(off);
 }
 
+/* ---------------------------------------------------------------- tall-skinny QR (FlashTSQR)
+ * "LoRAForge：压缩与执行协同，让多LoRA服务更高效", FlashTSQR section: the
+ * factor construction of post-hoc compression runs a QR of many tall, skinny
+ * factor matrices (rows far more than columns), parallel across modules and
+ * across row blocks. The oracle is the QR itself, by Householder reflections
+ * on the whole matrix in fp64 (the textbook algorithm, column by column):
+ * for column j, x = A[j:, j], alpha = -sign(x_0)·||x||, v = x - alpha·e_0,
+ * A[j:, j:] -= 2·v·(v^T·A[j:, j:]) / (v^T·v). R is the upper n x n triangle of
+ * the result; Q (m x n) = H_0·H_1·...·H_{n-1} applied to the first n columns
+ * of the identity. For each of `batch` matrices A [m x n] (row-major), outputs
+ * R [n x n] (zeros below the diagonal) and Q [m x n] (NULL to skip). */
+void oracle_qr(int64_t batch, int64_t m, int64_t n, const double *A, double *R, double *Q) {
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t b = 0; b < batch; ++b) {
+        double *a = (double *)malloc(sizeof(double) * (size_t)(m * n));
+        double *V = (double *)calloc((size_t)(m * n), sizeof(double)); /* reflector j in column j */
+        double *vv = (double *)calloc((size_t)n, sizeof(double));      /* v_j^T v_j */
+        memcpy(a, A + b * m * n, sizeof(double) * (size_t)(m * n));
+        for (int64_t j = 0; j < n; ++j) {
+            double norm2 = 0.0;
+            for (int64_t i = j; i < m; ++i) norm2 += a[i * n + j] * a[i * n + j];
+            double norm = sqrt(norm2);
+            double x0 = a[j * n + j];
+            double alpha = x0 >= 0.0 ? -norm : norm;
+            for (int64_t i = j; i < m; ++i) V[i * n + j] = a[i * n + j];
+            V[j * n + j] = x0 - alpha;
+            double vtv = 0.0;
+            for (int64_t i = j; i < m; ++i) vtv += V[i * n + j] * V[i * n + j];
+            vv[j] = vtv;
+            if (vtv == 0.0) continue; /* the column is already zero below the diagonal */
+            for (int64_t c = j; c < n; ++c) {
+                double w = 0.0;
+                for (int64_t i = j; i < m; ++i) w += V[i * n + j] * a[i * n + c];
+                double f = 2.0 * w / vtv;
+                for (int64_t i = j; i < m; ++i) a[i * n + c] -= f * V[i * n + j];
+            }
+        }
+        for (int64_t i = 0; i < n; ++i)
+            for (int64_t c = 0; c < n; ++c) R[(b * n + i) * n + c] = c >= i ? a[i * n + c] : 0.0;
+        if (Q) {
+            double *q = Q + b * m * n;
+            for (int64_t i = 0; i < m; ++i)
+                for (int64_t c = 0; c < n; ++c) q[i * n + c] = i == c ? 1.0 : 0.0;
+            for (int64_t j = n - 1; j >= 0; --j) { /* Q = H_0 (H_1 (... (H_{n-1} E))) */
+                if (vv[j] == 0.0) continue;
+                for (int64_t c = 0; c < n; ++c) {
+                    double w = 0.0;
+                    for (int64_t i = j; i < m; ++i) w += V[i * n + j] * q[i * n + c];
+                    double f = 2.0 * w / vv[j];
+                    for (int64_t i = j; i < m; ++i) q[i * n + c] -= f * V[i * n + j];
+                }
+            }
+        }
+        free(a);
+        free(V);
+        free(vv);
+    }
+}
+
 int oracle_num_threads(void) {
 #ifdef _OPENMP
     extern int omp_get_max_threads(void);

@@ -402,3 +402,40 @@ def test_switch_merged_weight_reproduces_the_unmerged_forward():
     inp = dataclasses.replace(inp, scale=np.array([1.0, 3.0], dtype=np.float32))
     Wm = oracle.switch(inp.W[None], inp.A_pool[None], inp.B_pool[None], inp.ranks, [1], [3.0])[0]
     assert np.array_equal(f32(inp.X) @ Wm, oracle.forward(inp))
+
+
+# ------------------------------------------------------------------ tall-skinny QR (FlashTSQR)
+def test_qr_reconstructs_and_is_orthonormal():
+    """Q·R = A, Q^T·Q = I and R upper triangular, on tall random matrices."""
+    rng = np.random.default_rng(5)
+    A = rng.standard_normal((3, 300, 24))
+    R, Q = oracle.qr(A)
+    for b in range(3):
+        np.testing.assert_allclose(Q[b] @ R[b], A[b], atol=1e-12)
+        np.testing.assert_allclose(Q[b].T @ Q[b], np.eye(24), atol=1e-12)
+        assert np.all(np.tril(R[b], -1) == 0)
+
+
+def test_qr_matches_numpy_up_to_row_signs():
+    """R is unique up to the sign of each row (Q up to the sign of each column):
+    the oracle's R against numpy's (LAPACK) after making both diagonals positive."""
+    rng = np.random.default_rng(6)
+    A = rng.standard_normal((200, 17))
+    R, Q = oracle.qr(A)
+    Qn, Rn = np.linalg.qr(A)
+    s, sn = np.sign(np.diag(R)), np.sign(np.diag(Rn))
+    np.testing.assert_allclose(s[:, None] * R, sn[:, None] * Rn, atol=1e-12)
+    np.testing.assert_allclose(Q * s[None, :], Qn * sn[None, :], atol=1e-12)
+
+
+def test_qr_gram_identity_and_orthogonal_columns():
+    """R^T·R = A^T·A (the Gram matrix); and a matrix whose columns are orthogonal
+    with norms d_j has |R| = diag(d)."""
+    rng = np.random.default_rng(7)
+    A = rng.standard_normal((150, 12))
+    R, _ = oracle.qr(A, want_q=False)
+    np.testing.assert_allclose(R.T @ R, A.T @ A, rtol=1e-12, atol=1e-10)
+    Qo, _ = np.linalg.qr(rng.standard_normal((150, 12)))
+    d = np.arange(1, 13, dtype=np.float64)
+    R2, _ = oracle.qr(Qo * d[None, :], want_q=False)
+    np.testing.assert_allclose(np.abs(R2), np.diag(d), atol=1e-12)
