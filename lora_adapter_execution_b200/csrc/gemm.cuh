@@ -366,6 +366,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.fz_X + static_cast<int64_t>(p.perm[i]) * p.K) + c);
         reinterpret_cast<uint4 *>(p.fz_Xs + i * p.K)[c] = v;
       }
+      fence_proxy_async_global();  // other CTAs read the copy through TMA
       __syncthreads();
       if (threadIdx.x == 0) {
         signal_counter(p.fz_grid_cnt);
@@ -383,11 +384,13 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       for (int j = p.fz_unit_off[blockIdx.x]; j < p.fz_unit_off[blockIdx.x + 1]; ++j) {
         const int u = p.fz_units[j];
         shrink_unit<4>(smem, sbars, mapSIn, mapSF, mapSBits, p.fz_sp, u, 0u, ShrinkRole{lt, 2, false});
+        fence_proxy_async_global();  // the image is read by other CTAs' bulk copies
         asm volatile("bar.sync 2, 160;" ::: "memory");  // the unit's outputs are all written
         if (lt == 0) signal_counter(p.fz_tile_cnt + p.fz_sp.units[u].tile);
       }
     }
-    __syncthreads();  // the stage ring is free again
+    fence_proxy_async_smem();  // the shrink's generic stores precede the ring's TMA writes
+    __syncthreads();           // the stage ring is free again
   }
 
   const int n_tiles = p.n_mt * p.n_nt;

@@ -415,6 +415,9 @@ __device__ __forceinline__ void shrink_unit(uint8_t *smem, uint64_t *bars, const
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // the pool may hold what generic stores wrote before (a previous unit's sums,
+  // or another role of the CTA): order them before the ring's TMA writes
+  fence_proxy_async_smem();
   shrink_bar_all(role.bar_id);
   // X (or its sorted copy from the row gather) and everything else the launch
   // reads or writes come after the previous kernel on the stream has completed
@@ -570,6 +573,8 @@ __device__ __forceinline__ void shrink_unit(uint8_t *smem, uint64_t *bars, const
       }
     }
     cluster_sync_all();  // the peers' fin was read: every rank may go on and exit
+  } else {
+    shrink_bar_all(role.bar_id);  // fin is complete before any thread reads a row of it
   }
 
   if (p.mode == 0) {
@@ -735,6 +740,21 @@ __device__ __forceinline__ uint32_t keep_pair_t(uint32_t xa, uint32_t xb) {
 // 128. The consumer warps first turn the stage's fp32 G into its transposed hi
 // and lo bf16 images (once for all warps), then each k16 step takes two
 // transposed In fragments and, per 16 ranks, two G^T fragments and eight MMAs.
+// Barrier 1 over the consumer warps (kTcConsumerWarps * 32 threads): true for
+// every participant when all of them passed true.
+__device__ __forceinline__ bool tc_bar_and(bool v) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 q, %1, 0;\n\t"
+      "bar.red.and.pred p, 1, %2, q;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}\n"
+      : "=r"(r)
+      : "r"(static_cast<uint32_t>(v)), "n"(kTcConsumerWarps * 32)
+      : "memory");
+  return r != 0;
+}
+
 __global__ void __launch_bounds__(kTcThreads, 2)
     lora_tcontract_kernel(const __grid_constant__ CUtensorMap mapIn,  // In [T, N] bf16, box {64, 64}, swizzle 128B
                           const __grid_constant__ CUtensorMap mapG,   // G [T, >= k0 + r] fp32, box {r, 64}, no swizzle
@@ -878,7 +898,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           for (int e = 0; e < 4; ++e) acc[i][g][j][e] = 0.f;
 
     for (int b = 0; b < nblk; ++b) {
-      if (!mbar_wait(full0 + 8 * stage, phase)) { ok = false; break; }
+      // the stage's wait; the four warps agree on its outcome at the barrier
+      // below, so that none is left waiting there for a warp that gave up
+      const bool landed = mbar_wait(full0 + 8 * stage, phase);
       const uint32_t sb = pool + stage * stage_bytes;
       uint8_t *const sbp = smem + (sb - pool);
       // G^T images of this stage. Work item = (token pair tp, 4 consecutive ranks
@@ -896,7 +918,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         uint8_t *gmid = ghi + mblocks * 2048;
         uint8_t *glo = gmid + mblocks * 2048;
         const int q4 = mblocks * 4;  // 4-rank groups per token pair
-        for (int item = tid; item < 32 * q4; item += kTcConsumerWarps * 32) {
+        for (int item = landed ? tid : 32 * q4; item < 32 * q4; item += kTcConsumerWarps * 32) {
           const int tp = item / q4;
           const int k4 = (item - tp * q4) * 4;
           float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
@@ -918,7 +940,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
           }
         }
       }
-      asm volatile("bar.sync 1, %0;" ::"n"(kTcConsumerWarps * 32) : "memory");
+      if (!tc_bar_and(landed)) { ok = false; break; }
       const uint32_t ghi_s = sb + conv_off;
       const uint32_t gmid_s = ghi_s + mblocks * 2048;
       const uint32_t glo_s = gmid_s + mblocks * 2048;
