@@ -20,7 +20,8 @@ forward + backward) is the headline (`value`, `roofline`, `e2e`,
 timed alone in short bursts against the burst peak; `layer_roofline` is the
 whole step, timed over long back-to-back regions, against the sustained peak.
 `configs["switch"]` is the merge path (one fused adapter switch of a 32-layer
-stack per step).
+stack per step); `configs["factor_qr"]` the factor construction of post-hoc
+compression (one batched tall-skinny QR of 2048 adapter factors per step).
 
 `e2e` is the same metric through the public API with host buffers: per step
 the plan is built from host ids, X (and dY) are copied from pinned host
@@ -947,6 +948,102 @@ def measure_switch(cx, cpu_budget):
     return entry
 
 
+FACTOR = dict(batch=2048, m=4096, n=16, decay=0.97)
+FACTOR_TEXT = ("factor QR: 2048 adapter factors of 4096 x 16 (1024 rank-16 modules, A and B^T of each; bf16 pool "
+               "rows in, fp32 Q and R out)")
+
+
+def measure_tsqr(cx, cpu_budget):
+    """The factor construction of post-hoc compression: one batched tall-skinny
+    QR (Q and R) of every factor per step; beside it torch.linalg.qr of the same
+    matrices in fp32 (the matched library QR, context only)."""
+    import torch
+    import lora_adapter_execution_b200 as lora
+    a, dev = cx.a, cx.dev
+    c = FACTOR
+    b, m, n = c["batch"], c["m"], c["n"]
+    K = a.steps if a.steps is not None else 20
+    bits = wl.factor_stack(b, m, n, seed=3, decay=c["decay"])
+    F = torch.from_numpy(bits.view(np.int16)).to(dev).view(torch.bfloat16)
+    R = torch.empty(b, n, n, dtype=torch.float32, device=dev)
+    Q = torch.empty(b, n, m, dtype=torch.float32, device=dev)
+    ws = torch.empty(max(1, lora.tsqr_workspace_size(b, m, n, True)), dtype=torch.uint8, device=dev)
+    levels = 1
+    while (max(1, m // 128) if m >= 256 else 1) > (1 << (levels - 1)):
+        levels += 1
+
+    def step(i):
+        lora.tsqr(F, R, Q, ws)
+    with torch.cuda.stream(cx.stream):
+        step(0)
+    torch.cuda.synchronize()
+    assert lora.device_status() == 0
+    with ClockSampler(cx.local_rank) as clk:
+        ms, n_regions = cx.timed(step, K, 0.0 if a.once else MIN_REGION_S)
+    t = ms * 1e-3 / K
+    hbm, _, _, src = peaks()
+    nbytes = b * (m * n * 2 + m * n * 4 + n * n * 4)
+    ach = nbytes / t / 1e9
+    entry = {"metric": "adapter factors QR-factorised per second (Q and R)", "value": b / t, "unit": "factors/s",
+             "n_gpus": cx.world, "steps": K, "warmup": a.warmup, "ms_per_step": t * 1e3, "higher_is_better": True,
+             "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+             "config": {"workload": FACTOR_TEXT, "l2": f"factors {b * m * n * 2 / 2**20:.0f} MiB in, "
+                                                       f"Q {b * m * n * 4 / 2**20:.0f} MiB out (> 126 MiB L2)"},
+             "timing": (f"eager calls of lora_tsqr, CUDA events on the stream; median of {n_regions} regions of "
+                        f"exactly {K} calls"),
+             "gpu_launches": 2 * levels * K, "clocks": clk.summary(),
+             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                          "peak_kind": f"{src} hbm_gbs (copy)", "traffic": None,
+                          "kernel": "lora_qr_factor_kernel + lora_qr_apply_kernel, all levels, per call",
+                          "algorithmic_per_launch": nbytes, "avg_launch_us": t * 1e6,
+                          "what": "bytes: the bf16 factors read once, Q and R (fp32) written once"}}
+    # matched library QR: torch.linalg.qr of the same matrices (fp32, [b, m, n])
+    A32 = F.float().transpose(1, 2).contiguous()
+    try:
+        def lib_step(i):
+            torch.linalg.qr(A32, mode="reduced")
+        lms, _ = cx.timed(lib_step, max(3, K // 4), 0.0)
+        entry["library_qr"] = {"what": "torch.linalg.qr(mode='reduced') of the same factors as fp32 [b, m, n]",
+                               "ms_per_call": lms / max(3, K // 4), "factors_per_s": b / (lms * 1e-3 / max(3, K // 4))}
+    except Exception as e:  # pragma: no cover - context only
+        entry["library_qr"] = {"unavailable": str(e)[:200]}
+    del A32
+    # e2e: factors from pinned host memory, R back to the host
+    hF = torch.from_numpy(bits.view(np.int16)).pin_memory()
+    hR = torch.empty(b, n, n, dtype=torch.float32).pin_memory()
+    torch.cuda.synchronize()
+    cx.barrier()
+    Ke = max(3, min(K, 10))
+    t0 = time.perf_counter()
+    for i in range(Ke):
+        F.view(torch.int16).copy_(hF, non_blocking=True)
+        step(i)
+        hR.copy_(R, non_blocking=True)
+    torch.cuda.synchronize()
+    dt = max_over_ranks(time.perf_counter() - t0, cx.world, dev)
+    entry["e2e"] = {"value": b * Ke / dt, "unit": "factors/s", "h2d_bytes_per_step": b * m * n * 2,
+                    "d2h_bytes_per_step": b * n * n * 4, "steps": Ke,
+                    "what": "per step: H2D of the bf16 factors (pinned) + lora_tsqr + D2H of R; host wall clock"}
+    if cx.rank == 0 and cx.world == 1 and not a.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        cores = oracle.num_threads()
+        cap = min(b, 64 * cores)
+        A64 = wl.bf16_bits_to_f32(bits[:cap]).astype(np.float64).transpose(0, 2, 1)
+        done = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < cpu_budget and done < cap:
+            oracle.qr(A64[done:done + cores])  # one matrix per thread
+            done += cores
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": done / dt, "unit": "factors/s", "cores": cores, "kind": "oracle",
+                                 "sample": f"{done} of the {b} factors (Householder QR in fp64, Q and R)"}
+    del F, R, Q, ws
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
 HEAD_KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
              "vs_baseline", "dtype", "data", "config", "timing", "roofline", "layer_roofline", "gpu_launches",
              "clocks", "layer", "e2e", "cpu_baseline")
@@ -962,6 +1059,7 @@ def run_lora(a):
     if a.config == "all":
         entries["fleet_finetune"] = measure("fleet_finetune", cx, CPU_BUDGET_S["other"])
         entries["switch"] = measure_switch(cx, CPU_BUDGET_S["other"])
+        entries["factor_qr"] = measure_tsqr(cx, CPU_BUDGET_S["other"])
     head = entries[HEADLINE if a.config == "all" else a.config]
     out = {k: head[k] for k in HEAD_KEYS if k in head}
     if a.config == "all":

@@ -422,6 +422,38 @@ int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, con
  * context that queued work still uses). NULL is ignored. */
 void lora_switch_destroy(lora_switch_t sw);
 
+/* Batched tall-skinny QR of adapter factors: the FlashTSQR factor construction
+ * of post-hoc compression in "LoRAForge：压缩与执行协同，让多LoRA服务更高效"
+ * (FlashTSQR section and the terms note on TSQR: a QR of many matrices with far
+ * more rows than columns, each cut into row blocks whose local QRs are merged,
+ * parallel across modules and across row blocks). A = Q·R for each of `batch`
+ * matrices A (m x n): Q (m x n) with orthonormal columns, R (n x n) upper
+ * triangular with a non-negative diagonal (so the factorisation is the unique
+ * one when A has full column rank). fp32 arithmetic (Householder reflections
+ * on row tiles of 128, a binary tree of stacked R pairs above them).
+ *   F             bf16 DEVICE, read only: element (i, j) of matrix b (row i < m,
+ *                 column j < n) at F[b*batch_stride + j*ld + i], i.e. column j
+ *                 is a row of an adapter pool (A_pool or B_pool rows of one
+ *                 adapter of rank n: A's m = d_in, B^T's m = d_out)
+ *   ld            elements between consecutive columns, >= m
+ *   batch_stride  elements between consecutive matrices, >= 0
+ *   batch, m, n   1 <= n <= 64, n <= m <= 2^31, batch * m * n <= 2^40
+ *   R             fp32 DEVICE [batch][n][n] row-major (zeros below the diagonal), caller-owned
+ *   Q             fp32 DEVICE [batch][n][m], column j of matrix b at Q + (b*n + j)*m
+ *                 (the layout of F), caller-owned; NULL computes R only
+ *   workspace     DEVICE scratch of lora_tsqr_workspace_size(batch, m, n, Q != NULL)
+ *                 bytes (may be 0 bytes: then NULL is accepted), caller-owned;
+ *                 used until the call's kernels complete on `stream`
+ * Stream-ordered; returns once the launches are queued. A zero column gives a
+ * zero diagonal entry of R (and a column of Q that is still orthonormal to the
+ * others).
+ * Errors: LORA_ERR_ARG (null F or R, sizes out of range, ld < m),
+ * LORA_ERR_WORKSPACE (workspace missing or too small), LORA_ERR_UNSUPPORTED,
+ * LORA_ERR_CUDA. */
+size_t lora_tsqr_workspace_size(int64_t batch, int64_t m, int32_t n, int want_q);
+int lora_tsqr(const uint16_t *F, int64_t ld, int64_t batch_stride, int64_t batch, int64_t m, int32_t n, float *R,
+              float *Q, void *workspace, size_t workspace_bytes, lora_stream_t stream);
+
 /* Test hook: write the dropout mask the forward and backward use (dropout on
  * the LoRA-branch input, one of the small ops the LoRAFusion explainer lists in
  * section 解决什么真问题, item 1; the drop rule is the one under lora_linear_fwd).

@@ -91,6 +91,8 @@ def load_library():
         "lora_switch_create": (ctypes.c_int, [_vp, _i32, _i64, _i64, _i64, _i32, ctypes.POINTER(_vp)]),
         "lora_switch_apply": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _i32, _vp]),
         "lora_switch_destroy": (None, [_vp]),
+        "lora_tsqr_workspace_size": (_sz, [_i64, _i64, _i32, ctypes.c_int]),
+        "lora_tsqr": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),
         "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -430,3 +432,31 @@ class Switch:
             self.destroy()
         except Exception:
             pass
+
+
+def tsqr_workspace_size(batch: int, m: int, n: int, want_q: bool) -> int:
+    return int(load_library().lora_tsqr_workspace_size(int(batch), int(m), int(n), 1 if want_q else 0))
+
+
+def tsqr(F, R, Q=None, workspace=None, *, stream=None):
+    """lora_tsqr: A_b = Q_b·R_b for the matrices A_b[i, j] = F[b, j, i] (F bf16
+    [batch, n, m], unit stride along m, any strides along b and j: e.g. one
+    adapter's rows of a stack of pools, A_pool[:, off:off + r, :]). R fp32
+    [batch, n, n]; Q fp32 [batch, n, m] (Q[b, j] is column j) or None. The
+    workspace is allocated when not given."""
+    if F is None or F.dim() != 3:
+        raise LoraError(-1, "lora_tsqr: F must be a [batch, n, m] tensor")
+    batch, n, m = (int(v) for v in F.shape)
+    if str(F.dtype).rsplit(".", 1)[-1] not in _BF16 or F.stride(2) != 1:
+        raise LoraError(-1, "lora_tsqr: F must be bfloat16 with unit stride along m")
+    if not F.is_cuda:
+        raise LoraError(-1, "lora_tsqr: F is not a CUDA tensor")
+    _args("lora_tsqr", ("R", R, (batch, n, n), _F32, False), ("Q", Q, (batch, n, m), _F32, True))
+    need = tsqr_workspace_size(batch, m, n, Q is not None)
+    if workspace is None and need > 0:
+        import torch
+        workspace = torch.empty(need, dtype=torch.uint8, device=F.device)
+    nbytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    ptr = ctypes.c_void_p(F.data_ptr())
+    _check(load_library().lora_tsqr(ptr, F.stride(1), F.stride(0), batch, m, n, _ptr(R), _ptr(Q), _ptr(workspace),
+                                    nbytes, _stream(stream)), "lora_tsqr")

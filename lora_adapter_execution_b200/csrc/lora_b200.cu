@@ -14,6 +14,7 @@
 #include "gemm.cuh"
 #include "skinny.cuh"
 #include "switch.cuh"
+#include "tsqr.cuh"
 
 using namespace lora;
 
@@ -75,6 +76,10 @@ int device_state(DeviceState **out) {
                                      sk_smem(2)) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_tcontract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      tc_smem(kTcMaxR)) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_qr_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     qr_factor_smem(kQrMaxN)) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_qr_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     qr_apply_smem(kQrMaxN)) == cudaSuccess;
           if (!ok) d.status = LORA_ERR_CUDA;
         }
       }
@@ -1648,6 +1653,115 @@ int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, con
   // no base K blocks: the A map carries the weights' W blocks, the W map is unused
   lora_gemm_kernel<false, kEpiMergeAdd><<<grid, kGemmThreads, kGemmSmem, stream>>>(mW, mBl, mBl, mBl, mBl, mBl, gp);
   return launch_status();
+}
+
+}  // extern "C"
+
+// ------------------------------------------------------------------ batched tall-skinny QR
+namespace {
+// The tree's levels for m rows, and the workspace: the root's row signs, then
+// per level its stacked pairs (level >= 1), its reflector scalars and its
+// blocks of the way down (the last two only when Q is wanted).
+struct QrLayout {
+  std::vector<int32_t> nodes;
+  std::vector<int64_t> off_S, off_hv, off_C;  // byte offsets, -1 where absent
+  int64_t off_sign = -1, total = 0;
+};
+QrLayout qr_layout(int64_t batch, int64_t m, int32_t n, bool want_q) {
+  auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
+  QrLayout L;
+  L.nodes.push_back(qr_leaves(m));
+  while (L.nodes.back() > 1) L.nodes.push_back((L.nodes.back() + 1) / 2);
+  const int nl = static_cast<int>(L.nodes.size());
+  int64_t o = 0;
+  if (want_q) {
+    L.off_sign = o;
+    o += up(batch * n * 4);
+  }
+  L.off_S.assign(nl, -1);
+  L.off_hv.assign(nl, -1);
+  L.off_C.assign(nl, -1);
+  for (int l = 0; l < nl; ++l) {
+    const int64_t nodes = L.nodes[l];
+    if (l >= 1) {
+      L.off_S[l] = o;
+      o += up(batch * nodes * 2 * n * n * 4);
+    }
+    if (want_q) {
+      L.off_hv[l] = o;
+      o += up(batch * nodes * 2 * n * 4);
+      if (l + 1 < nl) {
+        L.off_C[l] = o;
+        o += up(batch * nodes * n * n * 4);
+      }
+    }
+  }
+  L.total = o;
+  return L;
+}
+bool qr_args_ok(int64_t batch, int64_t m, int32_t n) {
+  return batch >= 1 && n >= 1 && n <= kQrMaxN && m >= n && m <= (int64_t(1) << 31) &&
+         batch * qr_leaves(m) <= 0x7FFFFFFF && batch * m * n <= (int64_t(1) << 40);
+}
+}  // namespace
+
+extern "C" {
+
+size_t lora_tsqr_workspace_size(int64_t batch, int64_t m, int32_t n, int want_q) {
+  if (!qr_args_ok(batch, m, n)) return 0;
+  return static_cast<size_t>(qr_layout(batch, m, n, want_q != 0).total);
+}
+
+int lora_tsqr(const uint16_t *F, int64_t ld, int64_t batch_stride, int64_t batch, int64_t m, int32_t n, float *R,
+              float *Q, void *workspace, size_t workspace_bytes, lora_stream_t stream) {
+  if (!F || !R || !qr_args_ok(batch, m, n) || ld < m || batch_stride < 0) return LORA_ERR_ARG;
+  DeviceState *ds = nullptr;
+  int rc = device_state(&ds);
+  if (rc != LORA_OK) return rc;
+  const bool want_q = Q != nullptr;
+  const QrLayout L = qr_layout(batch, m, n, want_q);
+  if (L.total > 0 && (!workspace || workspace_bytes < static_cast<size_t>(L.total))) return LORA_ERR_WORKSPACE;
+  uint8_t *ws = static_cast<uint8_t *>(workspace);
+  auto at = [&](int64_t off) { return off < 0 ? nullptr : reinterpret_cast<float *>(ws + off); };
+  const int nl = static_cast<int>(L.nodes.size());
+  QrParams p{};
+  p.batch = batch;
+  p.m = m;
+  p.n = n;
+  p.ld = ld;
+  p.bstride = batch_stride;
+  p.F = F;
+  p.Q = Q;
+  p.R = R;
+  p.sign = at(L.off_sign);
+  auto level = [&](int l) {
+    QrLevel lv{};
+    lv.nodes = L.nodes[l];
+    lv.below = l >= 1 ? L.nodes[l - 1] : 0;
+    lv.up = l + 1 < nl ? L.nodes[l + 1] : 0;
+    lv.S = at(L.off_S[l]);
+    lv.S_up = l + 1 < nl ? at(L.off_S[l + 1]) : nullptr;
+    lv.hv = at(L.off_hv[l]);
+    lv.C = at(L.off_C[l]);
+    lv.C_down = l >= 1 ? at(L.off_C[l - 1]) : nullptr;
+    return lv;
+  };
+  // up the tree: every level's QR; then, for Q, down it
+  for (int l = 0; l < nl; ++l) {
+    p.level = l;
+    p.lv = level(l);
+    lora_qr_factor_kernel<<<static_cast<unsigned>(batch * L.nodes[l]), kQrThreads, qr_factor_smem(n), stream>>>(p);
+    if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+  }
+  if (want_q) {
+    for (int l = nl - 1; l >= 0; --l) {
+      p.level = l;
+      p.lv = level(l);
+      lora_qr_apply_kernel<<<static_cast<unsigned>(batch * L.nodes[l]), kQrThreads, qr_apply_smem(n), stream>>>(p);
+      if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+    }
+  }
+  return LORA_OK;
 }
 
 }  // extern "C"

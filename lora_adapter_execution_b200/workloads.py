@@ -244,3 +244,14 @@ def make_rank_inputs(spec: Spec | str, rank: int, **kw) -> Inputs:
     return Inputs(spec=spec, T=base.T, d_in=base.d_in, d_out=base.d_out, ranks=base.ranks, ids=other.ids,
                   scale=base.scale, X=other.X, W=base.W, A_pool=base.A_pool, B_pool=base.B_pool, dY=other.dY,
                   p_drop=base.p_drop, mask_seed=base.mask_seed, offsets=base.offsets)
+
+
+def factor_stack(batch: int, m: int, n: int, *, seed: int = 0, decay: float = 1.0) -> np.ndarray:
+    """Adapter factors as a stack of pools, for the tall-skinny QR: bf16 bit
+    patterns [batch, n, m], matrix b's column j in row [b, j] (an adapter pool's
+    row layout). Entries N(0, 1/m); column j scaled by decay**j (decay < 1 gives
+    the decaying spectrum of a trained factor: condition number about decay**(1-n))."""
+    rng = np.random.default_rng(seed)
+    F = rng.standard_normal((batch, n, m)).astype(np.float32) / np.float32(np.sqrt(m))
+    F *= (np.float32(decay) ** np.arange(n, dtype=np.float32))[None, :, None]
+    return f32_to_bf16_bits(F)
