@@ -383,7 +383,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       uint64_t *sbars = reinterpret_cast<uint64_t *>(smem + sk_pool(4));
       for (int j = p.fz_unit_off[blockIdx.x]; j < p.fz_unit_off[blockIdx.x + 1]; ++j) {
         const int u = p.fz_units[j];
-        shrink_unit<4>(smem, sbars, mapSIn, mapSF, mapSBits, p.fz_sp, u, 0u, ShrinkRole{lt, 2, false});
+        if (!shrink_unit<4>(smem, sbars, mapSIn, mapSF, mapSBits, p.fz_sp, u, 0u, ShrinkRole{lt, 2, false})) {
+          if (lt == 0) *abort_flag = 1;  // a wait gave up (all 160 threads see it and leave together)
+          break;
+        }
         fence_proxy_async_global();  // the image is read by other CTAs' bulk copies
         asm volatile("bar.sync 2, 160;" ::: "memory");  // the unit's outputs are all written
         if (lt == 0) signal_counter(p.fz_tile_cnt + p.fz_sp.units[u].tile);

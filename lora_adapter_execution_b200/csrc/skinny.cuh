@@ -361,7 +361,7 @@ __device__ __forceinline__ void shrink_bar_all(int bar_id) {
 // One shrink unit (one CTA of its cluster): smem is the 1024-aligned stage pool
 // (sk_pool(kMaxNB16) bytes), bars room for 2 * kSkMaxStages mbarriers and a flag.
 template <int kMaxNB16>
-__device__ __forceinline__ void shrink_unit(uint8_t *smem, uint64_t *bars, const CUtensorMap &mapIn16,
+__device__ __forceinline__ bool shrink_unit(uint8_t *smem, uint64_t *bars, const CUtensorMap &mapIn16,
                                             const CUtensorMap &mapF16, const CUtensorMap &mapBits16,
                                             const ShrinkParams &p, int unit, uint32_t crank, const ShrinkRole role) {
   const uint32_t pool = smem_u32(smem);
@@ -576,6 +576,16 @@ __device__ __forceinline__ void shrink_unit(uint8_t *smem, uint64_t *bars, const
   } else {
     shrink_bar_all(role.bar_id);  // fin is complete before any thread reads a row of it
   }
+  // every thread is past its last use of the ring's barriers: invalidate them, so
+  // that the next unit of a fused launch can initialise them afresh (and the
+  // GEMM's ring may overwrite their memory)
+  // (not after a wait gave up: a copy may still be in flight to the ring)
+  const bool unit_ok = !*abort_flag;
+  if (tid == 0 && unit_ok)
+    for (int s = 0; s < nstage; ++s) {
+      mbar_inval(full0 + 8 * s);
+      mbar_inval(empty0 + 8 * s);
+    }
 
   if (p.mode == 0) {
     const float s_a = p.scale[g.adapter] * p.inv_keep;
@@ -641,6 +651,7 @@ __device__ __forceinline__ void shrink_unit(uint8_t *smem, uint64_t *bars, const
       for (int c = lane; c < g.nn; c += 32) dst[c] = c < g.nvalid ? fin[lr * kShrinkN + c] * p.scale1 : 0.f;
     }
   }
+  return unit_ok;
 }
 
 // Grid: n_units * ksplit CTAs, clusters of ksplit along x. Cluster c handles unit c;
