@@ -133,6 +133,7 @@ struct GemmParams {
   // then runs its shrink units, each counting itself done for its m-tile, then
   // the GEMM tiles with their adapter blocks last, each tile's first adapter
   // block waiting for the tile's count
+  int32_t gemm_ctas;            // CTAs that run GEMM tiles (0: all); the fused launch's others only run units
   const int32_t *fz_unit_off;   // [grid + 1]: CTA b runs units fz_units[fz_unit_off[b] ..)
   const int32_t *fz_units;      // indices into fz_sp.units
   const int32_t *fz_tile_need;  // [n_mt]: units per m-tile
@@ -235,6 +236,7 @@ __device__ __forceinline__ void tile_coords(int tile, const GemmParams &p, int &
 // tiles blockIdx.x, blockIdx.x + gridDim.x, ...
 __device__ __forceinline__ bool cta_tile(const GemmParams &p, int k, int tile0, int tile_step, int n_tiles,
                                          int &tile) {
+  if (tile0 >= n_tiles) return false;  // a CTA without tiles
   if (p.sched_off) {
     const int i = p.sched_off[blockIdx.x] + k;
     if (i >= p.sched_off[blockIdx.x + 1]) return false;
@@ -358,13 +360,26 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // waits until all shares are written (the launch is cooperative: all CTAs
     // are resident, so the wait ends)
     if (p.a_sorted) {
-      const int64_t per_row = p.K / 8;
-      const int64_t n = static_cast<int64_t>(p.T) * per_row;
-      for (int64_t e = blockIdx.x * static_cast<int64_t>(kGemmThreads) + threadIdx.x; e < n;
-           e += static_cast<int64_t>(gridDim.x) * kGemmThreads) {
-        const int64_t i = e / per_row, c = e - (e / per_row) * per_row;
-        const uint4 v = __ldg(reinterpret_cast<const uint4 *>(p.fz_X + static_cast<int64_t>(p.perm[i]) * p.K) + c);
-        reinterpret_cast<uint4 *>(p.fz_Xs + i * p.K)[c] = v;
+      // one warp per row: the row's source index is read once, and each lane
+      // has up to 8 16-byte loads in flight before its stores
+      const int per_row = p.K / 8;
+      const int nwarps = static_cast<int>(gridDim.x) * (kGemmThreads / 32);
+      for (int i = static_cast<int>(blockIdx.x) * (kGemmThreads / 32) + warp; i < p.T; i += nwarps) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.fz_X + static_cast<int64_t>(__ldg(p.perm + i)) * p.K);
+        uint4 *dst = reinterpret_cast<uint4 *>(p.fz_Xs + static_cast<int64_t>(i) * p.K);
+        for (int c0 = 0; c0 < per_row; c0 += 8 * 32) {
+          uint4 v[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int c = c0 + u * 32 + lane;
+            if (c < per_row) v[u] = __ldg(src + c);
+          }
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int c = c0 + u * 32 + lane;
+            if (c < per_row) dst[c] = v[u];
+          }
+        }
       }
       fence_proxy_async_global();  // other CTAs read the copy through TMA
       __syncthreads();
@@ -380,15 +395,19 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     // for its m-tile (release), which the tile's adapter blocks wait for
     const int lt = (warp >= 2 && warp <= 5) ? static_cast<int>(threadIdx.x) - 64 : (warp == kGemmWarpFix ? 128 + lane : -1);
     if (lt >= 0 && !*abort_flag) {
-      uint64_t *sbars = reinterpret_cast<uint64_t *>(smem + sk_pool(4));
+      // the unit's ring takes the whole stage ring of the GEMM (a deeper ring
+      // than the standalone shrink's: the units run beside other CTAs' GEMM
+      // tiles, whose HBM traffic lengthens every copy's round trip)
+      constexpr int kPool = kGemmStages * kStageBytes - 4096;
+      uint64_t *sbars = reinterpret_cast<uint64_t *>(smem + kPool);
       for (int j = p.fz_unit_off[blockIdx.x]; j < p.fz_unit_off[blockIdx.x + 1]; ++j) {
         const int u = p.fz_units[j];
-        if (!shrink_unit<4>(smem, sbars, mapSIn, mapSF, mapSBits, p.fz_sp, u, 0u, ShrinkRole{lt, 2, false})) {
+        if (!shrink_unit<4, kPool>(smem, sbars, mapSIn, mapSF, mapSBits, p.fz_sp, u, 0u, ShrinkRole{lt, 2, false})) {
           if (lt == 0) *abort_flag = 1;  // a wait gave up (all 160 threads see it and leave together)
           break;
         }
         fence_proxy_async_global();  // the image is read by other CTAs' bulk copies
-        asm volatile("bar.sync 2, 160;" ::: "memory");  // the unit's outputs are all written
+        shrink_bar_all(2);  // the unit's outputs are all written
         if (lt == 0) signal_counter(p.fz_tile_cnt + p.fz_sp.units[u].tile);
       }
     }
@@ -407,8 +426,12 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   const bool split = p.ksplit > 1;
   const int S = split ? p.ksplit : 1;
   const int q = split ? static_cast<int>(cluster_rank()) : 0;
-  const int tile0 = split ? static_cast<int>(blockIdx.x) / S : static_cast<int>(blockIdx.x);
-  const int tile_step = split ? n_tiles : static_cast<int>(gridDim.x);
+  // CTAs past gemm_ctas (the fused forward's unit-only CTAs) have no tiles
+  const int gctas = p.gemm_ctas > 0 ? p.gemm_ctas : static_cast<int>(gridDim.x);
+  const int tile0 = static_cast<int>(blockIdx.x) >= gctas ? n_tiles
+                    : split                                ? static_cast<int>(blockIdx.x) / S
+                                                           : static_cast<int>(blockIdx.x);
+  const int tile_step = split ? n_tiles : gctas;
   // split-K tail inputs, set by the epilogue warps before their wait
   int split_rows = 0, split_nt = 0, split_kaug = 0;
   int64_t split_orig = 0;

@@ -26,6 +26,9 @@ struct DeviceState {
   std::atomic<bool> init{false};  // set once, after the fields below (release)
   int status = LORA_OK;
   int num_sms = 0;
+  // the fused forward's cooperative launch: most CTAs resident at once in
+  // clusters of S = 1, 2, 4 (index S)
+  int fz_max_ctas[5] = {0, 0, 0, 0, 0};
 };
 DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
@@ -81,6 +84,25 @@ int device_state(DeviceState **out) {
           ok &= cudaFuncSetAttribute(lora_qr_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      qr_apply_smem(kQrMaxN)) == cudaSuccess;
           if (!ok) d.status = LORA_ERR_CUDA;
+          for (int S = 1; ok && S <= 4; S *= 2) {
+            cudaLaunchConfig_t cfg{};
+            cfg.gridDim = dim3(static_cast<unsigned>(S));
+            cfg.blockDim = dim3(kGemmThreads);
+            cfg.dynamicSmemBytes = kGemmSmem;
+            cudaLaunchAttribute attr[1];
+            attr[0].id = cudaLaunchAttributeClusterDimension;
+            attr[0].val.clusterDim.x = S;
+            attr[0].val.clusterDim.y = 1;
+            attr[0].val.clusterDim.z = 1;
+            cfg.attrs = attr;
+            cfg.numAttrs = 1;
+            int clusters = 0;
+            if (cudaOccupancyMaxActiveClusters(&clusters, lora_gemm_kernel<false, kEpiStore, true>, &cfg) ==
+                cudaSuccess)
+              d.fz_max_ctas[S] = std::min(clusters * S, d.num_sms);
+            else
+              cudaGetLastError();  // no extra shrink CTAs then
+          }
         }
       }
       d.init.store(true, std::memory_order_release);
@@ -294,6 +316,7 @@ struct lora_plan {
   // units of each CTA (off[grid + 1] | units), units per m-tile, and its counters
   // (per m-tile, then the row-copy count), zeroed before each launch
   int fz_grid = 0;
+  int fz_gemm_ctas = 0;  // the first fz_gemm_ctas CTAs run GEMM tiles, the others only shrink units
   std::vector<int32_t> fz_tab;          // off[grid + 1] | units | need[n_mt]
   const int32_t *d_fz_off = nullptr, *d_fz_units = nullptr, *d_fz_need = nullptr;
   int32_t *d_fz_cnt = nullptr;
@@ -427,13 +450,33 @@ int upload_plan(lora_plan *pl, lora_stream_t stream, bool sync) {
     const int KB = static_cast<int>((hp.d_in + kBK - 1) / kBK);
     if (n_tiles > 0) {
       const int S = fwd_ksplit(n_tiles, KB, ds->num_sms);
-      const int G = S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S;
+      const int Gg = S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S;
       const int nu = static_cast<int>(hp.units.size());
+      // CTAs the GEMM leaves free (whole clusters, within what can be resident
+      // at once) take the units, so the GEMM CTAs start their K loops at once;
+      // with no room every CTA runs units first
+      int Gx = std::max(0, std::min(ds->fz_max_ctas[S] - Gg, (nu + S - 1) / S * S));
+      Gx = Gx / S * S;
+      const int G = Gg + Gx;
+      // the unit-only CTAs take the units when there are enough of them for
+      // about two each; otherwise every CTA takes units, the unit-only ones first
+      const bool only = Gx > 0 && 2 * Gx >= nu;
+      const int nw = only ? Gx : G;  // the CTAs that take units
       pl->fz_grid = G;
+      pl->fz_gemm_ctas = Gg;
       pl->fz_tab.assign(G + 1 + nu + n_mt, 0);
-      for (int b = 0; b < G; ++b) pl->fz_tab[b + 1] = pl->fz_tab[b] + (nu - b + G - 1) / G;
-      for (int b = 0; b < G; ++b)
-        for (int u = b, j = pl->fz_tab[b]; u < nu; u += G, ++j) pl->fz_tab[G + 1 + j] = u;
+      // dealing position w of CTA b: the unit-only CTAs come first in the
+      // rotation, so with every CTA taking units they get the extra ones
+      auto pos = [&](int b) { return only ? b - Gg : (b >= Gg ? b - Gg : b + Gx); };
+      for (int b = 0; b < G; ++b) {
+        const int w = pos(b);
+        pl->fz_tab[b + 1] = pl->fz_tab[b] + ((w >= 0 && w < nw) ? (nu - w + nw - 1) / nw : 0);
+      }
+      for (int b = 0; b < G; ++b) {
+        const int w = pos(b);
+        if (w < 0 || w >= nw) continue;
+        for (int u = w, j = pl->fz_tab[b]; u < nu; u += nw, ++j) pl->fz_tab[G + 1 + j] = u;
+      }
       for (int u = 0; u < nu; ++u) ++pl->fz_tab[G + 1 + nu + hp.units[u].tile];
     }
   }
@@ -861,10 +904,12 @@ int lora_linear_fwd_fused(lora_plan_t plan, const uint16_t *X, const uint16_t *W
   gp.group_m = default_group_m(gp.n_mt, gp.K);
   const int S = fwd_ksplit(n_tiles, KB, ds->num_sms);
   gp.ksplit = S;
-  const int G = S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S;
-  if (G != plan->fz_grid) return LORA_ERR_ARG;  // the unit lists were dealt for this grid
+  const int Gg = S == 1 ? std::min(ds->num_sms, n_tiles) : n_tiles * S;
+  if (Gg != plan->fz_gemm_ctas) return LORA_ERR_ARG;  // the unit lists were dealt for this grid
+  const int G = plan->fz_grid;
+  gp.gemm_ctas = Gg;
   if (S > 1 && plan->xws_S == S) gp.xws = plan->scratch + plan->xws_offset;
-  if (S == 1 && plan->d_sched && static_cast<int>(plan->sched.size()) - n_tiles - 1 == G) {
+  if (S == 1 && plan->d_sched && static_cast<int>(plan->sched.size()) - n_tiles - 1 == Gg) {
     gp.sched_off = plan->d_sched;
     gp.sched_tiles = plan->d_sched + G + 1;
   }
@@ -1699,6 +1744,32 @@ QrLayout qr_layout(int64_t batch, int64_t m, int32_t n, bool want_q) {
   L.total = o;
   return L;
 }
+// One level's launch: a warp per node for n <= 32 (the column bound NC and the
+// rows per lane RPL as templates: leaves hold 128 rows, stacked pairs 2n), a
+// CTA per node above.
+template <int NC, int RPL>
+bool launch_qr_warp(const QrParams &p, int64_t units, bool apply, cudaStream_t st) {
+  const unsigned grid = static_cast<unsigned>((units + kQrWarpThreads / 32 - 1) / (kQrWarpThreads / 32));
+  if (apply) lora_qr_apply_warp_kernel<NC, RPL><<<grid, kQrWarpThreads, 0, st>>>(p);
+  else lora_qr_factor_warp_kernel<NC, RPL><<<grid, kQrWarpThreads, 0, st>>>(p);
+  return cudaGetLastError() == cudaSuccess;
+}
+template <int NC>
+bool launch_qr_nc(const QrParams &p, int64_t units, int rows, bool apply, cudaStream_t st) {
+  if (rows <= 32) return launch_qr_warp<NC, 1>(p, units, apply, st);
+  if (rows <= 64) return launch_qr_warp<NC, 2>(p, units, apply, st);
+  return launch_qr_warp<NC, 4>(p, units, apply, st);
+}
+bool launch_qr(const QrParams &p, int64_t units, int rows, bool apply, lora_stream_t stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (p.n <= 8) return launch_qr_nc<8>(p, units, rows, apply, st);
+  if (p.n <= 16) return launch_qr_nc<16>(p, units, rows, apply, st);
+  if (p.n <= kQrWarpMaxN) return launch_qr_nc<32>(p, units, rows, apply, st);
+  if (apply) lora_qr_apply_kernel<<<static_cast<unsigned>(units), kQrThreads, qr_apply_smem(p.n), st>>>(p);
+  else lora_qr_factor_kernel<<<static_cast<unsigned>(units), kQrThreads, qr_factor_smem(p.n), st>>>(p);
+  return cudaGetLastError() == cudaSuccess;
+}
+
 bool qr_args_ok(int64_t batch, int64_t m, int32_t n) {
   return batch >= 1 && n >= 1 && n <= kQrMaxN && m >= n && m <= (int64_t(1) << 31) &&
          batch * qr_leaves(m) <= 0x7FFFFFFF && batch * m * n <= (int64_t(1) << 40);
@@ -1750,15 +1821,13 @@ int lora_tsqr(const uint16_t *F, int64_t ld, int64_t batch_stride, int64_t batch
   for (int l = 0; l < nl; ++l) {
     p.level = l;
     p.lv = level(l);
-    lora_qr_factor_kernel<<<static_cast<unsigned>(batch * L.nodes[l]), kQrThreads, qr_factor_smem(n), stream>>>(p);
-    if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+    if (!launch_qr(p, batch * L.nodes[l], l == 0 ? kQrTile : 2 * n, false, stream)) return LORA_ERR_CUDA;
   }
   if (want_q) {
     for (int l = nl - 1; l >= 0; --l) {
       p.level = l;
       p.lv = level(l);
-      lora_qr_apply_kernel<<<static_cast<unsigned>(batch * L.nodes[l]), kQrThreads, qr_apply_smem(n), stream>>>(p);
-      if (cudaGetLastError() != cudaSuccess) return LORA_ERR_CUDA;
+      if (!launch_qr(p, batch * L.nodes[l], l == 0 ? kQrTile : 2 * n, true, stream)) return LORA_ERR_CUDA;
     }
   }
   return LORA_OK;

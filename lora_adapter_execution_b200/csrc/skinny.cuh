@@ -326,7 +326,7 @@ __device__ __forceinline__ void shrink_consume(const ShrinkWarp &w, const Shrink
 
   // every consumer warp is past its last stage: every TMA of the ring has
   // landed and been read, so the pool may be overwritten
-  asm volatile("bar.sync %0, %1;" ::"n"(kSkConsumerBar), "n"(kSkConsumerWarps * 32) : "memory");
+  asm volatile("barrier.sync %0, %1;" ::"n"(kSkConsumerBar), "n"(kSkConsumerWarps * 32) : "memory");
   float *base = red + (warp * 32) * kShrinkN;
 #pragma unroll
   for (int i = 0; i < 2; ++i) {
@@ -353,20 +353,27 @@ struct ShrinkRole {
   bool pdl;
 };
 
+// The producer warp reaches these barriers diverged (lane 0 may still be in its
+// copy loop while lanes 1..31 arrive), so the named form is the non-aligned
+// `barrier.sync`, which counts threads one by one; `bar.sync` is the aligned
+// form, for warps that arrive converged (with a diverged warp it can complete
+// before every thread has arrived). __syncthreads counts per thread as well.
 __device__ __forceinline__ void shrink_bar_all(int bar_id) {
   if (bar_id == 0) __syncthreads();
-  else asm volatile("bar.sync %0, %1;" ::"r"(bar_id), "n"(kSkThreads) : "memory");
+  else asm volatile("barrier.sync %0, %1;" ::"r"(bar_id), "n"(kSkThreads) : "memory");
 }
 
 // One shrink unit (one CTA of its cluster): smem is the 1024-aligned stage pool
-// (sk_pool(kMaxNB16) bytes), bars room for 2 * kSkMaxStages mbarriers and a flag.
-template <int kMaxNB16>
+// (kPoolBytes, by default the standalone kernel's sk_pool(kMaxNB16)), bars room
+// for 2 * kSkMaxStages mbarriers and a flag.
+template <int kMaxNB16, int kPoolBytes = sk_pool(kMaxNB16)>
 __device__ __forceinline__ bool shrink_unit(uint8_t *smem, uint64_t *bars, const CUtensorMap &mapIn16,
                                             const CUtensorMap &mapF16, const CUtensorMap &mapBits16,
                                             const ShrinkParams &p, int unit, uint32_t crank, const ShrinkRole role) {
   const uint32_t pool = smem_u32(smem);
   float *fin = reinterpret_cast<float *>(smem + kSkRedBytes);  // in the pool, after the partials
-  constexpr int kSkPool = sk_pool(kMaxNB16);
+  constexpr int kSkPool = kPoolBytes;
+  static_assert(kSkRedBytes + kSkFinBytes <= kPoolBytes, "the reduction scratch must fit the pool");
   const uint32_t full0 = smem_u32(bars);
   const uint32_t empty0 = full0 + 8 * kSkMaxStages;
   volatile int *abort_flag = reinterpret_cast<volatile int *>(bars + 2 * kSkMaxStages);

@@ -77,8 +77,9 @@ def check_backward(A, R, Q, what):
 
 
 CASES = {
-    # (batch, m, n, decay): one leaf (m < 256) and m == n; leaves 128 + 172;
-    # 7 leaves (odd levels 7 -> 4 -> 2 -> 1) at n = 1; 5 leaves at n = 64
+    # (batch, m, n, decay): one leaf and m == n; leaves 128 + 72; 8 leaves at
+    # n = 1 (the warp build's narrowest columns); 6 leaves at n = 64 (the CTA
+    # build); odd leaf counts (9 -> 5 -> 3 -> 2 -> 1 at m = 1111)
     "square_64": (2, 64, 64, 1.0),
     "one_leaf": (3, 200, 24, 1.0),
     "two_leaves": (3, 300, 16, 1.0),
@@ -86,6 +87,11 @@ CASES = {
     "five_leaves_n64": (2, 700, 64, 1.0),
     "ragged_n": (5, 1111, 37, 1.0),
     "many": (64, 520, 16, 1.0),
+    # a last leaf of one row (m = 129) and one shorter than n on the CTA build
+    "short_leaf": (3, 129, 16, 1.0),
+    "short_leaf_cta": (2, 140, 33, 1.0),
+    "n8": (5, 1000, 8, 1.0),
+    "n32": (3, 2000, 32, 1.0),
 }
 
 
