@@ -12,6 +12,7 @@ is fp64 over exactly widened bf16 inputs. Parity pins live in
 from __future__ import annotations
 
 import ctypes
+import math
 import os
 import subprocess
 
@@ -183,3 +184,96 @@ def qr(A, want_q=True):
     if single:
         return R[0], (Q[0] if want_q else None)
     return R, Q
+
+
+# --------------------------------------------------------------------------- post-hoc compression
+# "LoRAForge：压缩与执行协同，让多LoRA服务更高效": post-hoc compression keeps a
+# module's update A·B (A: d_in x r, B: r x d_out) in a retained rank k (核心设计:
+# the explicit retained-rank representation; FlashTSQR section: the factor
+# construction by QR; the spectral-energy note: a module's singular values and
+# their cumulative energy). The steps below are that reading, in fp64.
+
+def compress_spectra(A_rows, B_rows):
+    """Factor construction and spectrum of each module: A_rows [n, r, d_in] and
+    B_rows [n, r, d_out] (bf16 bits, or floats), module b's A = A_rows[b]^T and
+    B = B_rows[b]. A = Q_A·R_A and B^T = Q_B·R_B (Householder, oracle_qr), so
+    A·B = Q_A·(R_A·R_B^T)·Q_B^T with orthonormal Q_A, Q_B: the singular values of
+    A·B are those of the r x r core M = R_A·R_B^T. Returns (sigma [n, r]
+    descending, U, V [n, r, r] with M = U·diag(sigma)·V^T, Q_A [n, d_in, r],
+    Q_B [n, d_out, r]). The SVD of the small core is numpy's (a library step)."""
+    def f64(a):
+        a = np.asarray(a)
+        if a.dtype == np.uint16:
+            a = (a.astype(np.uint32) << 16).view(np.float32)
+        return a.astype(np.float64)
+    A = f64(A_rows).transpose(0, 2, 1)
+    Bt = f64(B_rows).transpose(0, 2, 1)
+    RA, QA = qr(A)
+    RB, QB = qr(Bt)
+    M = RA @ RB.transpose(0, 2, 1)
+    U, s, Vt = np.linalg.svd(M)
+    return s, U, Vt.transpose(0, 2, 1), QA, QB
+
+
+def allocate(sigma, ranks, costs, policy: str, keep: float, k_floor: int):
+    """Retained ranks of n modules (LoRAForge article, 核心设计: LoRAForge-U, the
+    same retention ratio for every module; LoRAForge-S, a budget spent by each
+    module's cumulative spectral energy). The rule, in float32 arithmetic so that
+    a caller holding the same float32 singular values decides identically:
+      U: k_b = clamp(ceil(keep * r_b), floor_b, r_b), floor_b = min(k_floor, r_b).
+      S: the budget P = floor(keep * sum_b r_b * c_b) parameters (c_b = the
+         parameters per retained rank of module b, d_in + d_out); every module
+         first keeps floor_b ranks; each further rank i >= floor_b of module b
+         scores g = (sigma_bi^2 / E_b) / c_b, E_b = sum_j sigma_bj^2 (summed in
+         j order; g = 0 when E_b = 0); the ranks are taken in the order of g
+         (largest first; equal g by module, then by i) while their costs fit in
+         P - sum floor_b * c_b, up to the first that does not fit. g falls with
+         i, so a module keeps a prefix of its ranks.
+    sigma: float32 [n, r_max] (descending in each row, zeros past r_b); ranks,
+    costs: [n] integers. Returns k [n] (int32) and offsets [n + 1] (int64, the
+    exclusive prefix sum of k: each module's first row in the new pools)."""
+    sigma = np.asarray(sigma, dtype=np.float32)
+    ranks = np.asarray(ranks, dtype=np.int64)
+    costs = np.asarray(costs, dtype=np.int64)
+    n = sigma.shape[0]
+    floors = np.minimum(ranks, k_floor)
+    if policy == "U":
+        k = np.array([min(int(ranks[b]), max(int(floors[b]), math.ceil(keep * int(ranks[b]))))
+                      for b in range(n)], dtype=np.int64)
+    elif policy == "S":
+        budget = math.floor(keep * float(int((ranks * costs).sum())))
+        left = budget - int((floors * costs).sum())
+        items = []  # (key, b, i, cost)
+        for b in range(n):
+            e = np.float32(0.0)
+            for j in range(int(ranks[b])):
+                e = np.float32(e + np.float32(sigma[b, j]) * np.float32(sigma[b, j]))
+            for i in range(int(floors[b]), int(ranks[b])):
+                sq = np.float32(np.float32(sigma[b, i]) * np.float32(sigma[b, i]))
+                g = np.float32(np.float32(sq / e) / np.float32(costs[b])) if e > 0 else np.float32(0.0)
+                items.append((int(np.array(g, dtype=np.float32).view(np.uint32)), b, i, int(costs[b])))
+        k = floors.copy()
+        total = 0
+        for key, b, i, c in sorted(items, key=lambda t: (-t[0], t[1], t[2])):
+            if total + c > left:
+                break
+            total += c
+            k[b] += 1
+    else:
+        raise ValueError(policy)
+    offsets = np.concatenate([[0], np.cumsum(k)]).astype(np.int64)
+    return k.astype(np.int32), offsets
+
+
+def export(sigma, U, V, QA, QB, k):
+    """The truncated factors of each module: A'_b = Q_A·U_k·diag(sqrt(sigma_k))
+    (d_in x k) and B'_b = diag(sqrt(sigma_k))·V_k^T·Q_B^T (k x d_out), so that
+    A'_b·B'_b is the best rank-k approximation of A_b·B_b (Eckart-Young).
+    Returns lists of fp64 arrays, A' as pool rows [k, d_in], B' [k, d_out]."""
+    A_new, B_new = [], []
+    for b in range(sigma.shape[0]):
+        kb = int(k[b])
+        sq = np.sqrt(sigma[b, :kb])
+        A_new.append(((QA[b] @ U[b][:, :kb]) * sq[None, :]).T)
+        B_new.append(((QB[b] @ V[b][:, :kb]) * sq[None, :]).T)
+    return A_new, B_new

@@ -8,6 +8,7 @@ CPU only (no GPU marker)."""
 from __future__ import annotations
 
 import dataclasses
+import math
 import os
 from fractions import Fraction
 
@@ -439,3 +440,107 @@ def test_qr_gram_identity_and_orthogonal_columns():
     d = np.arange(1, 13, dtype=np.float64)
     R2, _ = oracle.qr(Qo * d[None, :], want_q=False)
     np.testing.assert_allclose(np.abs(R2), np.diag(d), atol=1e-12)
+
+
+# --------------------------------------------------------------------------- post-hoc compression
+def _factor_modules(n, r, d_in, d_out, seed, decay=0.8):
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((n, r, d_in)) / np.sqrt(d_in)
+    B = rng.standard_normal((n, r, d_out)) * (decay ** np.arange(r))[None, :, None]
+    return A, B
+
+
+def test_compress_spectra_equal_the_singular_values_of_the_dense_product():
+    # the QR-core route against numpy's SVD of the explicit d_in x d_out product
+    A, B = _factor_modules(3, 6, 50, 40, seed=1)
+    s, U, V, QA, QB = oracle.compress_spectra(A, B)
+    for b in range(3):
+        dense = A[b].T @ B[b]
+        ref = np.linalg.svd(dense, compute_uv=False)[:6]
+        assert np.allclose(s[b], ref, rtol=1e-10, atol=1e-12)
+        # the core's factors rebuild the product
+        assert np.allclose(QA[b] @ U[b] @ np.diag(s[b]) @ V[b].T @ QB[b].T, dense, atol=1e-12)
+
+
+def test_compress_export_full_rank_and_eckart_young():
+    A, B = _factor_modules(2, 8, 64, 48, seed=2)
+    s, U, V, QA, QB = oracle.compress_spectra(A, B)
+    for k in (8, 5, 1):
+        An, Bn = oracle.export(s, U, V, QA, QB, np.array([k, k]))
+        for b in range(2):
+            dense = A[b].T @ B[b]
+            approx = An[b].T @ Bn[b]
+            err2 = np.linalg.norm(dense - approx) ** 2
+            assert np.isclose(err2, float((s[b, k:] ** 2).sum()), rtol=1e-9, atol=1e-20)
+            # the factors are balanced: A'^T A' = B' B'^T = diag(sigma_k)
+            assert np.allclose(An[b] @ An[b].T, np.diag(s[b, :k]), atol=1e-12)
+            assert np.allclose(Bn[b] @ Bn[b].T, np.diag(s[b, :k]), atol=1e-12)
+
+
+def test_allocate_uniform_by_hand():
+    sig = np.ones((3, 16), dtype=np.float32)
+    k, off = oracle.allocate(sig, [16, 8, 5], [100, 100, 100], "U", 0.25, 1)
+    assert k.tolist() == [4, 2, 2] and off.tolist() == [0, 4, 6, 8]   # ceil(4), ceil(2), ceil(1.25)
+    k, _ = oracle.allocate(sig, [16, 8, 5], [100, 100, 100], "U", 0.25, 3)
+    assert k.tolist() == [4, 3, 3]
+    k, _ = oracle.allocate(sig, [16, 8, 5], [100, 100, 100], "U", 1.0, 1)
+    assert k.tolist() == [16, 8, 5]
+
+
+def _score(sig, b, i, cost):
+    e = np.float32(0)
+    for j in range(sig.shape[1]):
+        e = np.float32(e + np.float32(sig[b, j] * sig[b, j]))
+    return float(np.float32(np.float32(np.float32(sig[b, i] * sig[b, i]) / e) / np.float32(cost)))
+
+
+def test_allocate_spectral_is_the_best_energy_per_budget_by_brute_force():
+    # equal costs and no ties: the kept set must be the allocation of the
+    # largest total score among all allocations within the budget
+    import itertools
+    rng = np.random.default_rng(5)
+    for trial in range(25):
+        n = 3
+        ranks = rng.integers(2, 6, size=n)
+        sig = np.zeros((n, 5), dtype=np.float32)
+        for b in range(n):
+            sig[b, :ranks[b]] = np.sort(rng.uniform(0.05, 3.0, size=ranks[b]).astype(np.float32))[::-1]
+        costs = np.full(n, 10)
+        keep = float(rng.uniform(0.2, 0.9))
+        k, _ = oracle.allocate(sig, ranks, costs, "S", keep, 1)
+        budget = math.floor(keep * float(int((ranks * costs).sum())))
+        best, best_k = -1.0, None
+        for ks in itertools.product(*[range(1, int(r) + 1) for r in ranks]):
+            if sum(ks) * 10 > max(budget, n * 10):
+                continue
+            tot = sum(_score(sig, b, i, 10) for b in range(n) for i in range(1, ks[b]))
+            if tot > best + 1e-12:
+                best, best_k = tot, ks
+        got = sum(_score(sig, b, i, 10) for b in range(n) for i in range(1, k[b]))
+        assert np.isclose(got, best, rtol=0, atol=1e-9), (trial, k.tolist(), best_k)
+
+
+def test_allocate_spectral_invariants():
+    rng = np.random.default_rng(6)
+    n, r = 40, 16
+    ranks = rng.integers(4, r + 1, size=n)
+    costs = rng.integers(200, 900, size=n)
+    sig = np.zeros((n, r), dtype=np.float32)
+    for b in range(n):
+        sig[b, :ranks[b]] = np.sort(rng.exponential(1.0, size=ranks[b]).astype(np.float32))[::-1]
+    prev = None
+    for keep in (1 / 12, 0.2, 0.5, 0.9):
+        k, off = oracle.allocate(sig, ranks, costs, "S", keep, 1)
+        budget = math.floor(keep * float(int((ranks * costs).sum())))
+        assert (k >= np.minimum(ranks, 1)).all() and (k <= ranks).all()
+        assert int((k * costs).sum()) <= max(budget, int((np.minimum(ranks, 1) * costs).sum()))
+        assert off[0] == 0 and (np.diff(off) == k).all()
+        if prev is not None:
+            assert (k >= prev).all()  # a larger budget never removes a rank
+        prev = k
+    # concentrated energy keeps fewer ranks than a flat spectrum at the same budget
+    s2 = np.zeros((2, 8), dtype=np.float32)
+    s2[0] = [10, 0.1, 0.1, 0.1, 0.1, 0.1, 0.1, 0.1]
+    s2[1] = [1, 1, 1, 1, 1, 1, 1, 1]
+    k, _ = oracle.allocate(s2, [8, 8], [100, 100], "S", 0.5, 1)
+    assert k[0] < k[1]
