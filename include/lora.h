@@ -454,6 +454,65 @@ size_t lora_tsqr_workspace_size(int64_t batch, int64_t m, int32_t n, int want_q)
 int lora_tsqr(const uint16_t *F, int64_t ld, int64_t batch_stride, int64_t batch, int64_t m, int32_t n, float *R,
               float *Q, void *workspace, size_t workspace_bytes, lora_stream_t stream);
 
+/* Post-hoc compression of adapter modules ("LoRAForge：压缩与执行协同，让多LoRA
+ * 服务更高效": section 核心设计, the retained-rank representation and the
+ * LoRAForge-U / LoRAForge-S allocation policies; section FlashTSQR, the factor
+ * construction; the note on spectral energy). A module's update A·B (A: d_in x r,
+ * B: r x d_out) is, with A = Q_A·R_A and B^T = Q_B·R_B (lora_tsqr's QR),
+ * Q_A·M·Q_B^T with the r x r core M = R_A·R_B^T = U·diag(sigma)·V^T: sigma is the
+ * update's spectrum, and A'·B' with A' = Q_A·U_k·diag(sigma_k)^½ and
+ * B' = diag(sigma_k)^½·V_k^T·Q_B^T is its best rank-k approximation. Three
+ * stream-ordered calls:
+ *
+ * lora_compress_spectra: the factor QRs and the core SVD (one-sided Jacobi, fp32)
+ * of a group of n_modules modules that share d_in, d_out and r.
+ *   A_rows     bf16 DEVICE: module b's A as r pool rows of d_in at A_rows + b*a_bstride
+ *              (row j = column j of A, the layout of A_pool)
+ *   B_rows     bf16 DEVICE: module b's B as r pool rows of d_out at B_rows + b*b_bstride
+ *   r          1 .. 64, r <= d_in, r <= d_out
+ *   sigma      fp32 DEVICE [n_modules][r], caller-owned: the spectrum, descending
+ *   workspace  DEVICE, lora_compress_workspace_size(n_modules, d_in, d_out, r) bytes,
+ *              caller-owned: it holds the factorisation for lora_compress_export
+ *              (about 4·n_modules·r·(d_in + d_out) bytes); keep it until then
+ *
+ * lora_compress_allocate: the retained rank of each of n_modules modules (of any
+ * groups: sigma rows padded with zeros to r_max), on the device.
+ *   sigma [n_modules][r_max] fp32, ranks [n_modules] int32, costs [n_modules] int64
+ *              (parameters per retained rank, d_in + d_out): DEVICE
+ *   policy     0: LoRAForge-U, k_b = clamp(ceil(keep·r_b), min(k_floor, r_b), r_b);
+ *              1: LoRAForge-S, a budget of floor(keep·sum r_b·c_b) parameters:
+ *              every module first keeps min(k_floor, r_b) ranks, then ranks are
+ *              taken by the largest (sigma_bi² / sum_j sigma_bj²) / c_b (float32;
+ *              equal values by module, then rank index) while their costs fit,
+ *              up to the first that does not
+ *   keep       in [0, 1]; k_floor >= 0
+ *   k          int32 DEVICE [n_modules]; offsets int64 DEVICE [n_modules + 1] (the
+ *              exclusive prefix sum of k: each module's first row in new pools)
+ *   workspace  DEVICE, lora_compress_allocate_workspace_size(n_modules, r_max)
+ *              bytes (policy 1 only; may be NULL for policy 0)
+ *
+ * lora_compress_export: the truncated factors of a group, written rank-exact:
+ * module b's A' as k[b] rows (k[b] <= r; more are not written) of d_in at row
+ * offsets[b] of A_new, B' as k[b] rows
+ * of d_out at row offsets[b] of B_new (bf16, caller-owned DEVICE pools). sigma,
+ * k, offsets are this group's (pointers to its first module); the workspace
+ * is the one lora_compress_spectra filled for this group (it is not changed,
+ * so several exports may follow one spectra call).
+ *
+ * Errors: LORA_ERR_ARG (null pointers, sizes out of range, policy, keep),
+ * LORA_ERR_WORKSPACE, LORA_ERR_UNSUPPORTED, LORA_ERR_CUDA. */
+size_t lora_compress_workspace_size(int64_t n_modules, int64_t d_in, int64_t d_out, int32_t r);
+int lora_compress_spectra(const uint16_t *A_rows, int64_t a_bstride, const uint16_t *B_rows, int64_t b_bstride,
+                          int64_t n_modules, int64_t d_in, int64_t d_out, int32_t r, float *sigma, void *workspace,
+                          size_t workspace_bytes, lora_stream_t stream);
+size_t lora_compress_allocate_workspace_size(int64_t n_modules, int32_t r_max);
+int lora_compress_allocate(const float *sigma, const int32_t *ranks, const int64_t *costs, int64_t n_modules,
+                           int32_t r_max, int32_t policy, double keep, int32_t k_floor, int32_t *k, int64_t *offsets,
+                           void *workspace, size_t workspace_bytes, lora_stream_t stream);
+int lora_compress_export(const float *sigma, const int32_t *k, const int64_t *offsets, int64_t n_modules, int64_t d_in,
+                         int64_t d_out, int32_t r, uint16_t *A_new, uint16_t *B_new, void *workspace,
+                         size_t workspace_bytes, lora_stream_t stream);
+
 /* Test hook: write the dropout mask the forward and backward use (dropout on
  * the LoRA-branch input, one of the small ops the LoRAFusion explainer lists in
  * section 解决什么真问题, item 1; the drop rule is the one under lora_linear_fwd).

@@ -93,6 +93,12 @@ def load_library():
         "lora_switch_destroy": (None, [_vp]),
         "lora_tsqr_workspace_size": (_sz, [_i64, _i64, _i32, ctypes.c_int]),
         "lora_tsqr": (ctypes.c_int, [_vp, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),
+        "lora_compress_workspace_size": (_sz, [_i64, _i64, _i64, _i32]),
+        "lora_compress_spectra": (ctypes.c_int, [_vp, _i64, _vp, _i64, _i64, _i64, _i64, _i32, _vp, _vp, _sz, _vp]),
+        "lora_compress_allocate_workspace_size": (_sz, [_i64, _i32]),
+        "lora_compress_allocate": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i32, _i32, _dbl, _i32, _vp, _vp, _vp, _sz,
+                                                  _vp]),
+        "lora_compress_export": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _i32, _vp, _vp, _vp, _sz, _vp]),
         "lora_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     }
     for name, (res, args) in sig.items():
@@ -460,3 +466,66 @@ def tsqr(F, R, Q=None, workspace=None, *, stream=None):
     ptr = ctypes.c_void_p(F.data_ptr())
     _check(load_library().lora_tsqr(ptr, F.stride(1), F.stride(0), batch, m, n, _ptr(R), _ptr(Q), _ptr(workspace),
                                     nbytes, _stream(stream)), "lora_tsqr")
+
+
+def _pool_rows(name, t):
+    """A [n, r, d] bf16 view of module rows (unit stride along d, rows of d
+    consecutive, any stride between modules)."""
+    if t is None or t.dim() != 3 or str(t.dtype).rsplit(".", 1)[-1] not in _BF16 or t.stride(2) != 1 \
+            or t.stride(1) != t.shape[2] or not t.is_cuda:
+        raise LoraError(-1, f"{name}: a CUDA bfloat16 [n, r, d] tensor with rows of d consecutive is required")
+    return int(t.shape[0]), int(t.shape[1]), int(t.shape[2])
+
+
+class Compressor:
+    """Post-hoc compression of a group of modules sharing d_in, d_out and r
+    (lora_compress_spectra / lora_compress_export); the workspace holds the
+    factorisation between the two calls."""
+
+    def __init__(self, A_rows, B_rows, *, stream=None):
+        import torch
+        n, r, d_in = _pool_rows("A_rows", A_rows)
+        n2, r2, d_out = _pool_rows("B_rows", B_rows)
+        if (n2, r2) != (n, r):
+            raise LoraError(-1, "lora_compress_spectra: A_rows and B_rows differ in modules or rank")
+        self.n, self.r, self.d_in, self.d_out = n, r, d_in, d_out
+        need = int(load_library().lora_compress_workspace_size(n, d_in, d_out, r))
+        if need == 0:
+            raise LoraError(-1, "lora_compress_spectra: sizes out of range")
+        self.workspace = torch.empty(need, dtype=torch.uint8, device=A_rows.device)
+        self.sigma = torch.empty(n, r, dtype=torch.float32, device=A_rows.device)
+        _check(load_library().lora_compress_spectra(_ptr(A_rows), A_rows.stride(0), _ptr(B_rows), B_rows.stride(0), n,
+                                                    d_in, d_out, r, _ptr(self.sigma), _ptr(self.workspace), need,
+                                                    _stream(stream)), "lora_compress_spectra")
+
+    def export(self, k, offsets, A_new, B_new, *, stream=None):
+        """Write this group's truncated factors: k int32 [n], offsets int64 [n]
+        (device; each module's first row), A_new bf16 [rows, d_in], B_new [rows, d_out]."""
+        _args("lora_compress_export", ("k", k, (self.n,), _I32, False), ("offsets", offsets, (offsets.shape[0],),
+                                                                         ("int64",), False),
+              ("A_new", A_new, (A_new.shape[0], self.d_in), _BF16, False),
+              ("B_new", B_new, (B_new.shape[0], self.d_out), _BF16, False))
+        if offsets.shape[0] < self.n:
+            raise LoraError(-1, "lora_compress_export: offsets has fewer entries than modules")
+        _check(load_library().lora_compress_export(_ptr(self.sigma), _ptr(k), _ptr(offsets), self.n, self.d_in,
+                                                   self.d_out, self.r, _ptr(A_new), _ptr(B_new),
+                                                   _ptr(self.workspace), self.workspace.numel(), _stream(stream)),
+               "lora_compress_export")
+
+
+def compress_allocate(sigma, ranks, costs, policy: str, keep: float, k_floor: int, *, stream=None):
+    """lora_compress_allocate: sigma fp32 [n, r_max], ranks int32 [n], costs int64 [n]
+    (device). Returns (k int32 [n], offsets int64 [n + 1]) on the device."""
+    import torch
+    n, r_max = int(sigma.shape[0]), int(sigma.shape[1])
+    _args("lora_compress_allocate", ("sigma", sigma, (n, r_max), _F32, False), ("ranks", ranks, (n,), _I32, False),
+          ("costs", costs, (n,), ("int64",), False))
+    k = torch.empty(n, dtype=torch.int32, device=sigma.device)
+    off = torch.empty(n + 1, dtype=torch.int64, device=sigma.device)
+    need = int(load_library().lora_compress_allocate_workspace_size(n, r_max))
+    ws = torch.empty(max(need, 1), dtype=torch.uint8, device=sigma.device)
+    pol = {"U": 0, "S": 1}[policy]
+    _check(load_library().lora_compress_allocate(_ptr(sigma), _ptr(ranks), _ptr(costs), n, r_max, pol, float(keep),
+                                                 int(k_floor), _ptr(k), _ptr(off), _ptr(ws), need, _stream(stream)),
+           "lora_compress_allocate")
+    return k, off

@@ -60,6 +60,14 @@ struct QrParams {
   float *Q;             // [batch][n][m] fp32 column-major (NULL: R only); holds the leaves' reflectors in between
   float *R;             // [batch][n][n] row-major, upper triangular, diagonal >= 0
   float *sign;          // [batch][n]: the root's row signs (Q wanted)
+  // way down only: the root's block, [batch][n][n] column-major (NULL: the sign
+  // diagonal, giving Q); with it the leaves give Q·(that block's leading rows)
+  const float *root_c;
+  // way down only: the leaves write columns c < out_k[b] of their result as
+  // bf16 rows out_row0[b] + c of out_rows (row length m) instead of Q
+  uint16_t *out_rows;
+  const int32_t *out_k;
+  const int64_t *out_row0;
   QrLevel lv;
 };
 
@@ -73,6 +81,9 @@ __host__ __device__ inline void qr_leaf_rows(int64_t m, int leaves, int t, int64
 __host__ __device__ inline int qr_node_parts(int below, int k) { return min(2, below - 2 * k); }
 
 __device__ __forceinline__ float bf16_to_f32(uint16_t h) { return __uint_as_float(static_cast<uint32_t>(h) << 16); }
+__device__ __forceinline__ uint16_t f32_to_bf16_rn(float x) {
+  return __bfloat16_as_ushort(__float2bfloat16_rn(x));
+}
 
 // Householder step quantities of a column x (x_0 its diagonal entry, ||x||^2 =
 // norm2): alpha = -sign(x_0)·||x||, v_0 = x_0 - alpha = x_0 + sign(x_0)·||x||,
@@ -296,7 +307,12 @@ __global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr
 #pragma unroll
     for (int c = 0; c < NC; ++c) y[r][c] = 0.f;
   if (lane < n) {
-    if (p.lv.up == 0) {
+    if (p.lv.up == 0 && p.root_c) {
+      const float *cb = p.root_c + b * n * n + lane;
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+        if (c < n) y[0][c] = cb[c * n];
+    } else if (p.lv.up == 0) {
       const float d = p.sign[b * n + lane];
 #pragma unroll
       for (int c = 0; c < NC; ++c) y[0][c] = c == lane ? d : 0.f;
@@ -333,7 +349,17 @@ __global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr
 #pragma unroll
       for (int r = 0; r < RPL; ++r) y[r][c] -= t * v[r] * w[c];
   }
-  if (p.level == 0) {
+  if (p.level == 0 && p.out_rows) {
+    const int kb = min(p.out_k[b], n);
+    uint16_t *o = p.out_rows + p.out_row0[b] * p.m + r0;
+#pragma unroll
+    for (int r = 0; r < RPL; ++r)
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int i = 32 * r + lane;
+        if (c < kb && i < s) o[c * p.m + i] = f32_to_bf16_rn(y[r][c]);
+      }
+  } else if (p.level == 0) {
     float *q = p.Q + b * n * p.m + r0;
 #pragma unroll
     for (int r = 0; r < RPL; ++r)
@@ -532,12 +558,17 @@ __global__ void __launch_bounds__(kQrThreads) lora_qr_apply_kernel(const QrParam
   for (int c = 0; c < n; ++c)
     for (int i = threadIdx.x; i < rows; i += kQrThreads) {
       float val = 0.f;
-      if (i < n) val = root ? (i == c ? p.sign[b * n + i] : 0.f) : cblk[c * n + i];
+      if (i < n)
+        val = !root ? cblk[c * n + i] : p.root_c ? p.root_c[b * n * n + c * n + i] : (i == c ? p.sign[b * n + i] : 0.f);
       y[i * ld + c] = val;
     }
   __syncthreads();
   qr_apply(y, v, ld, rows, n, vh, tau, w);
-  if (p.level == 0) {
+  if (p.level == 0 && p.out_rows) {
+    uint16_t *o = p.out_rows + p.out_row0[b] * p.m + r0;
+    for (int c = 0; c < min(p.out_k[b], n); ++c)
+      for (int i = threadIdx.x; i < s; i += kQrThreads) o[c * p.m + i] = f32_to_bf16_rn(y[i * ld + c]);
+  } else if (p.level == 0) {
     float *q = p.Q + b * n * p.m + r0;
     for (int c = 0; c < n; ++c)
       for (int i = threadIdx.x; i < s; i += kQrThreads) q[c * p.m + i] = y[i * ld + c];

@@ -255,3 +255,17 @@ def factor_stack(batch: int, m: int, n: int, *, seed: int = 0, decay: float = 1.
     F = rng.standard_normal((batch, n, m)).astype(np.float32) / np.float32(np.sqrt(m))
     F *= (np.float32(decay) ** np.arange(n, dtype=np.float32))[None, :, None]
     return f32_to_bf16_bits(F)
+
+
+def module_factors(n: int, r: int, d_in: int, d_out: int, *, seed: int = 0, decay=(0.6, 0.95)):
+    """Trained-like factors of n modules for post-hoc compression, as bf16 bit
+    patterns in pool-row layout: A_rows [n, r, d_in] with entries N(0, 1/d_in)
+    (LoRA's A scale) and B_rows [n, r, d_out] with entries N(0, 1) times
+    decay_b**j on row j, decay_b uniform in `decay` per module, so the modules'
+    spectra fall off at different rates (the spread a spectral budget reads)."""
+    rng = np.random.default_rng(seed)
+    A = rng.standard_normal((n, r, d_in)).astype(np.float32) / np.float32(np.sqrt(d_in))
+    dec = rng.uniform(decay[0], decay[1], size=n).astype(np.float32)
+    B = rng.standard_normal((n, r, d_out)).astype(np.float32)
+    B *= dec[:, None, None] ** np.arange(r, dtype=np.float32)[None, :, None]
+    return f32_to_bf16_bits(A), f32_to_bf16_bits(B)
