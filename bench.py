@@ -21,7 +21,8 @@ timed alone in short bursts against the burst peak; `layer_roofline` is the
 whole step, timed over long back-to-back regions, against the sustained peak.
 `configs["switch"]` is the merge path (one fused adapter switch of a 32-layer
 stack per step); `configs["factor_qr"]` the factor construction of post-hoc
-compression (one batched tall-skinny QR of 2048 adapter factors per step).
+compression (one batched tall-skinny QR of 2048 adapter factors per step);
+`configs["compress"]` the whole LoRAForge-S export of 1024 modules per step.
 
 `e2e` is the same metric through the public API with host buffers: per step
 the plan is built from host ids, X (and dY) are copied from pinned host
@@ -89,7 +90,7 @@ def parse(argv=None):
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=None)
     ap.add_argument("--warmup", type=int, default=DEFAULT_WARMUP)
-    ap.add_argument("--config", default="all", choices=["all", *wl.WORKLOADS, "switch", "factor_qr"])
+    ap.add_argument("--config", default="all", choices=["all", *wl.WORKLOADS, "switch", "factor_qr", "compress"])
     ap.add_argument("--impl", default="lora", choices=["lora", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
@@ -1050,6 +1051,88 @@ def measure_tsqr(cx, cpu_budget):
     return entry
 
 
+COMPRESS = dict(n=1024, r=16, d=4096, keep=1 / 12, floor=1)
+COMPRESS_TEXT = ("post-hoc compression: 1024 rank-16 modules of 4096 x 4096 (32 layers x 4 projections x 8 "
+                 "adapters), LoRAForge-S rank-floored 1/12 spectral export: spectra, allocation, truncated factors")
+
+
+def measure_compress(cx, cpu_budget):
+    """Post-hoc compression of a fleet's modules per step: the factor QRs and
+    core SVDs (lora_compress_spectra), the spectral-budget allocation and the
+    export of the truncated factors into new pools."""
+    import torch
+    import lora_adapter_execution_b200 as lora
+    a, dev = cx.a, cx.dev
+    c = COMPRESS
+    n, r, d = c["n"], c["r"], c["d"]
+    K = a.steps if a.steps is not None else 10
+    A, B = wl.module_factors(n, r, d, d, seed=5)
+    Ad = torch.from_numpy(A.view(np.int16)).to(dev).view(torch.bfloat16)
+    Bd = torch.from_numpy(B.view(np.int16)).to(dev).view(torch.bfloat16)
+    ranks = torch.full((n,), r, dtype=torch.int32, device=dev)
+    costs = torch.full((n,), 2 * d, dtype=torch.int64, device=dev)
+    A_new = torch.empty(n * r, d, dtype=torch.bfloat16, device=dev)
+    B_new = torch.empty(n * r, d, dtype=torch.bfloat16, device=dev)
+    state = {}
+
+    def step(i):
+        comp = lora.Compressor(Ad, Bd)
+        k, off = lora.compress_allocate(comp.sigma, ranks, costs, "S", c["keep"], c["floor"])
+        comp.export(k, off[:n], A_new, B_new)
+        state["k"] = k
+        state["comp"] = comp
+    with torch.cuda.stream(cx.stream):
+        step(0)
+    torch.cuda.synchronize()
+    assert lora.device_status() == 0
+    kept = int(state["k"].sum().item())
+    # tree levels of a 4096-row factor (leaves of 128): each factor goes up and
+    # down them; + the core SVDs, the allocation and two root-block launches
+    levels, nodes = 1, -(-d // 128)
+    while nodes > 1:
+        nodes, levels = -(-nodes // 2), levels + 1
+    with ClockSampler(cx.local_rank) as clk:
+        ms, n_regions = cx.timed(step, K, 0.0 if a.once else MIN_REGION_S)
+    t = ms * 1e-3 / K
+    hbm, _, _, src = peaks()
+    nbytes = n * r * 2 * d * 2 + kept * 2 * d * 2
+    ach = nbytes / t / 1e9
+    entry = {"metric": "adapter modules compressed per second (spectra, allocation, export)", "value": n / t,
+             "unit": "modules/s", "n_gpus": cx.world, "steps": K, "warmup": a.warmup, "ms_per_step": t * 1e3,
+             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+             "config": {"workload": COMPRESS_TEXT, "kept_ranks": kept, "of_ranks": n * r,
+                        "l2": f"factors {n * r * 2 * d * 2 / 2**20:.0f} MiB in (> 126 MiB L2)"},
+             "timing": (f"eager calls (workspace allocation included), CUDA events on the stream; median of "
+                        f"{n_regions} regions of exactly {K} exports"),
+             "gpu_launches": (4 * levels + 4) * K, "clocks": clk.summary(),
+             "roofline": {"bound": "hbm", "achieved": ach, "peak": hbm, "unit": "GB/s", "frac": ach / hbm,
+                          "peak_kind": f"{src} hbm_gbs (copy)", "traffic": None,
+                          "kernel": "all kernels of the export (tall-skinny QRs both ways, core SVDs, allocation)",
+                          "algorithmic_per_launch": nbytes, "avg_launch_us": t * 1e6,
+                          "what": "bytes: the modules' bf16 factors read once, the kept factors written once"}}
+    if cx.rank == 0 and cx.world == 1 and not a.no_cpu_baseline:
+        import oracle
+        oracle.build()
+        done = 0
+        t0 = time.perf_counter()
+        while time.perf_counter() - t0 < cpu_budget and done < n:
+            Af = wl.bf16_bits_to_f32(A[done:done + 4]).astype(np.float64)
+            Bf = wl.bf16_bits_to_f32(B[done:done + 4]).astype(np.float64)
+            s_, U_, V_, QA_, QB_ = oracle.compress_spectra(Af, Bf)
+            kk, _ = oracle.allocate(s_.astype(np.float32), np.full(len(Af), r), np.full(len(Af), 2 * d), "S",
+                                    c["keep"], c["floor"])
+            oracle.export(s_, U_, V_, QA_, QB_, kk)
+            done += len(Af)
+        dt = time.perf_counter() - t0
+        entry["cpu_baseline"] = {"value": done / dt, "unit": "modules/s", "cores": oracle.num_threads(),
+                                 "kind": "oracle", "sample": f"{done} of the {n} modules (allocation within each "
+                                                             "batch of 4)"}
+    del Ad, Bd, A_new, B_new, state
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    return entry
+
+
 HEAD_KEYS = ("metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step", "higher_is_better", "scaling",
              "vs_baseline", "dtype", "data", "config", "timing", "roofline", "layer_roofline", "gpu_launches",
              "clocks", "layer", "e2e", "cpu_baseline")
@@ -1059,7 +1142,7 @@ def run_lora(a):
     cx = Ctx(a)
     names = list(ORDER) if a.config == "all" else [a.config]
     entries = {}
-    extra = {"switch": measure_switch, "factor_qr": measure_tsqr}
+    extra = {"switch": measure_switch, "factor_qr": measure_tsqr, "compress": measure_compress}
     for name in names:
         budget = CPU_BUDGET_S["headline" if name in (HEADLINE, a.config) else "other"]
         entries[name] = extra[name](cx, budget) if name in extra else measure(name, cx, budget)
@@ -1067,6 +1150,7 @@ def run_lora(a):
         entries["fleet_finetune"] = measure("fleet_finetune", cx, CPU_BUDGET_S["other"])
         entries["switch"] = measure_switch(cx, CPU_BUDGET_S["other"])
         entries["factor_qr"] = measure_tsqr(cx, CPU_BUDGET_S["other"])
+        entries["compress"] = measure_compress(cx, CPU_BUDGET_S["other"])
     head = entries[HEADLINE if a.config == "all" else a.config]
     out = {k: head[k] for k in HEAD_KEYS if k in head}
     if a.config == "all":
