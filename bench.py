@@ -1004,9 +1004,12 @@ def measure_tsqr(cx, cpu_budget):
                           "kernel": "lora_qr_factor_kernel + lora_qr_apply_kernel, all levels, per call",
                           "algorithmic_per_launch": nbytes, "avg_launch_us": t * 1e6,
                           "what": "bytes: the bf16 factors read once, Q and R (fp32) written once"}}
-    # matched library QR: torch.linalg.qr of the same matrices (fp32, [b, m, n])
-    A32 = F.float().transpose(1, 2).contiguous()
+    # matched library QR: torch.linalg.qr of the same matrices (fp32, [b, m, n]);
+    # not in profiler runs (--no-layer: it launches thousands of library kernels)
+    A32 = F.float().transpose(1, 2).contiguous() if not a.no_layer else None
     try:
+        if A32 is None:
+            raise RuntimeError("skipped (--no-layer)")
         def lib_step(i):
             torch.linalg.qr(A32, mode="reduced")
         lms, _ = cx.timed(lib_step, max(3, K // 4), 0.0)
@@ -1016,6 +1019,12 @@ def measure_tsqr(cx, cpu_budget):
         entry["library_qr"] = {"unavailable": str(e)[:200]}
     del A32
     # e2e: factors from pinned host memory, R back to the host
+    if a.no_e2e:
+        entry["e2e"] = None
+        del F, R, Q, ws
+        torch.cuda.synchronize()
+        torch.cuda.empty_cache()
+        return entry
     hF = torch.from_numpy(bits.view(np.int16)).pin_memory()
     hR = torch.empty(b, n, n, dtype=torch.float32).pin_memory()
     torch.cuda.synchronize()
