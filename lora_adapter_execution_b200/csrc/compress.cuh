@@ -168,14 +168,18 @@ __device__ __forceinline__ int64_t alloc_sum(int64_t v, int64_t *red) {
 // not. That order is the order of the 64-bit keys (bits of g, then the
 // complement of b·r_max + i), all distinct, so the taken ranks are those with
 // key >= K*, K* the smallest key whose ranks at or above it cost at most the
-// rest of the budget: a bisection over the keys. Offsets: the exclusive prefix
-// sum of k.
+// rest of the budget: a radix select over the keys. Offsets: the exclusive
+// prefix sum of k.
 __global__ void __launch_bounds__(kAllocThreads) lora_compress_alloc_kernel(
     const float *__restrict__ sigma, const int32_t *__restrict__ ranks, const int64_t *__restrict__ costs,
     int64_t n, int r_max, int policy, double keep, int k_floor, uint64_t *__restrict__ keys,
     int32_t *__restrict__ k, int64_t *__restrict__ offsets) {
   __shared__ int64_t red[32];
   __shared__ int64_t chunk_tot[kAllocThreads];
+  __shared__ int64_t whist[8 * 256];  // byte histograms of the radix select, one per 4 warps
+  __shared__ int64_t hist[256];
+  __shared__ int sel[1];
+  __shared__ int64_t sel_above[1];
   const int tid = threadIdx.x;
   if (policy == 0) {
     for (int64_t b = tid; b < n; b += kAllocThreads) {
@@ -211,36 +215,63 @@ __global__ void __launch_bounds__(kAllocThreads) lora_compress_alloc_kernel(
       }
     }
     __syncthreads();
-    // smallest K with cost(key >= K) <= left; keys are never 0 for real ranks
-    // (the complement term is at least 1 while b·r_max + i < 2^32 - 1)
-    uint64_t lo = 1, hi = ~0ull;  // cost(key >= hi + 1) = 0 <= left: the answer is in [lo, hi + 1]
+    // K*: the smallest key whose ranks at or above it cost at most `left`
+    // (keys are never 0 for real ranks: the complement term is at least 1 while
+    // b·r_max + i < 2^32 - 1). Radix select, 8 bits a pass from the top: the
+    // candidates are the keys with the prefix fixed so far; a pass histograms
+    // their next byte weighted by cost (a copy per 4 warps, then summed) and walks
+    // the bytes from the top while the cost of the keys above still fits; the
+    // byte where it stops joins the prefix. Keys are distinct, so after 8 passes
+    // the prefix is the first key that does not fit, k0, and K* = k0 + 1.
     bool none = left <= 0;
+    uint64_t kstar = ~0ull;
     if (!none) {
-      // does everything fit?
       int64_t all = 0;
-      for (int64_t e = tid; e < n * r_max; e += kAllocThreads) {
-        const uint64_t key = keys[e];
-        if (key) all += costs[e / r_max];
-      }
+      for (int64_t e = tid; e < n * r_max; e += kAllocThreads)
+        if (keys[e]) all += costs[e / r_max];
       all = alloc_sum(all, red);
       if (all <= left) {
-        hi = 0;  // every key >= 1 taken
+        kstar = 1;  // every rank fits
       } else {
-        // invariant: cost(key >= lo) > left, cost(key >= hi + 1) <= left. Keys
-        // are below 2^63 (g >= 0), so lo stays below it and the interval halves
-        // each step: 64 steps at most (the cap only bounds the loop)
-        for (int it = 0; it < 66 && lo <= hi; ++it) {
-          const uint64_t mid = lo + (hi - lo) / 2;
-          int64_t c = 0;
-          for (int64_t e = tid; e < n * r_max; e += kAllocThreads)
-            if (keys[e] >= mid) c += costs[e / r_max];
-          c = alloc_sum(c, red);
-          if (c <= left) hi = mid - 1;
-          else lo = mid + 1;
+        uint64_t prefix = 0;
+        int64_t above = 0;  // cost of the keys above the current prefix's range
+        for (int pass = 0; pass < 8; ++pass) {
+          const int shift = 56 - 8 * pass;
+          for (int e = tid; e < 8 * 256; e += kAllocThreads) whist[e] = 0;
+          __syncthreads();
+          unsigned long long *wh = reinterpret_cast<unsigned long long *>(whist) + (tid >> 7) * 256;
+          for (int64_t e = tid; e < n * r_max; e += kAllocThreads) {
+            const uint64_t key = keys[e];
+            if (!key) continue;
+            // the fixed bytes match (pass 0: everything)
+            if (pass > 0 && (key >> (shift + 8)) != prefix) continue;
+            atomicAdd(wh + ((key >> shift) & 0xFF), static_cast<unsigned long long>(costs[e / r_max]));
+          }
+          __syncthreads();
+          if (tid < 256) {
+            int64_t s = 0;
+            for (int w = 0; w < 8; ++w) s += whist[w * 256 + tid];
+            hist[tid] = s;
+          }
+          __syncthreads();
+          if (tid == 0) {
+            int64_t acc = above;
+            int d = 255;
+            for (; d > 0; --d) {
+              if (acc + hist[d] > left) break;
+              acc += hist[d];
+            }
+            sel[0] = d;
+            sel_above[0] = acc;
+          }
+          __syncthreads();
+          prefix = (prefix << 8) | static_cast<uint64_t>(sel[0]);
+          above = sel_above[0];
+          __syncthreads();
         }
+        kstar = prefix + 1;
       }
     }
-    const uint64_t kstar = none ? ~0ull : hi + 1;  // taken: 0 < key >= kstar
     for (int64_t b = tid; b < n; b += kAllocThreads) {
       const int r = ranks[b];
       int kb = min(k_floor, r);

@@ -86,6 +86,10 @@ int device_state(DeviceState **out) {
                                      qr_apply_smem(kQrMaxN)) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_core_svd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      svd_smem(kSvdMaxN)) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_qr_factor_leaf_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     qr_leaf_factor_smem<32>()) == cudaSuccess;
+          ok &= cudaFuncSetAttribute(lora_qr_apply_leaf_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     qr_leaf_apply_smem<16>()) == cudaSuccess;
           if (!ok) d.status = LORA_ERR_CUDA;
           for (int S = 1; ok && S <= 4; S *= 2) {
             cudaLaunchConfig_t cfg{};
@@ -1763,8 +1767,37 @@ bool launch_qr_nc(const QrParams &p, int64_t units, int rows, bool apply, cudaSt
   if (rows <= 64) return launch_qr_warp<NC, 2>(p, units, apply, st);
   return launch_qr_warp<NC, 4>(p, units, apply, st);
 }
-bool launch_qr(const QrParams &p, int64_t units, int rows, bool apply, lora_stream_t stream) {
+// the way up's leaf level, persistent with its next tile copied in the
+// background (16-byte rows needed), for n <= 32
+template <int NC>
+bool launch_qr_leaf(const QrParams &p, int64_t units, int sms, cudaStream_t st) {
+  const int per_sm = NC > 16 ? 2 : 4;
+  const int64_t want = (units + kQrWarpThreads / 32 - 1) / (kQrWarpThreads / 32);
+  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sms) * per_sm)));
+  lora_qr_factor_leaf_kernel<NC><<<grid, kQrWarpThreads, qr_leaf_factor_smem<NC>(), st>>>(p);
+  return cudaGetLastError() == cudaSuccess;
+}
+// the way down's leaf level likewise, for n <= 16 (reflector rows of 16 bytes)
+template <int NC>
+bool launch_qr_leaf_apply(const QrParams &p, int64_t units, int sms, cudaStream_t st) {
+  const int64_t want = (units + kQrWarpThreads / 32 - 1) / (kQrWarpThreads / 32);
+  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sms) * 3)));
+  lora_qr_apply_leaf_kernel<NC><<<grid, kQrWarpThreads, qr_leaf_apply_smem<NC>(), st>>>(p);
+  return cudaGetLastError() == cudaSuccess;
+}
+bool launch_qr(const QrParams &p, int64_t units, int rows, bool apply, lora_stream_t stream, int sms) {
   cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const bool rows16 = (reinterpret_cast<uintptr_t>(p.F) & 15) == 0 && p.ld % 8 == 0 && p.bstride % 8 == 0;
+  if (!apply && p.level == 0 && p.F && rows16 && sms > 0) {
+    if (p.n <= 8) return launch_qr_leaf<8>(p, units, sms, st);
+    if (p.n <= 16) return launch_qr_leaf<16>(p, units, sms, st);
+    if (p.n <= kQrWarpMaxN) return launch_qr_leaf<32>(p, units, sms, st);
+  }
+  const bool q16 = (reinterpret_cast<uintptr_t>(p.Q) & 15) == 0 && p.m % 4 == 0;
+  if (apply && p.level == 0 && p.Q && q16 && sms > 0) {
+    if (p.n <= 8) return launch_qr_leaf_apply<8>(p, units, sms, st);
+    if (p.n <= 16) return launch_qr_leaf_apply<16>(p, units, sms, st);
+  }
   if (p.n <= 8) return launch_qr_nc<8>(p, units, rows, apply, st);
   if (p.n <= 16) return launch_qr_nc<16>(p, units, rows, apply, st);
   if (p.n <= kQrWarpMaxN) return launch_qr_nc<32>(p, units, rows, apply, st);
@@ -1803,20 +1836,20 @@ QrLevel qr_level(const QrLayout &L, uint8_t *ws, int l) {
 }
 // up the tree: every level's QR (R at the root; with p.Q, the reflectors kept
 // in Q's buffer and the workspace for the way down)
-bool qr_up(QrParams p, const QrLayout &L, uint8_t *ws, lora_stream_t stream) {
+bool qr_up(QrParams p, const QrLayout &L, uint8_t *ws, lora_stream_t stream, int sms) {
   for (int l = 0; l < static_cast<int>(L.nodes.size()); ++l) {
     p.level = l;
     p.lv = qr_level(L, ws, l);
-    if (!launch_qr(p, p.batch * L.nodes[l], l == 0 ? kQrTile : 2 * p.n, false, stream)) return false;
+    if (!launch_qr(p, p.batch * L.nodes[l], l == 0 ? kQrTile : 2 * p.n, false, stream, sms)) return false;
   }
   return true;
 }
 // down the tree: Q (or, with p.root_c / p.out_rows, Q times the root block)
-bool qr_down(QrParams p, const QrLayout &L, uint8_t *ws, lora_stream_t stream) {
+bool qr_down(QrParams p, const QrLayout &L, uint8_t *ws, lora_stream_t stream, int sms) {
   for (int l = static_cast<int>(L.nodes.size()) - 1; l >= 0; --l) {
     p.level = l;
     p.lv = qr_level(L, ws, l);
-    if (!launch_qr(p, p.batch * L.nodes[l], l == 0 ? kQrTile : 2 * p.n, true, stream)) return false;
+    if (!launch_qr(p, p.batch * L.nodes[l], l == 0 ? kQrTile : 2 * p.n, true, stream, sms)) return false;
   }
   return true;
 }
@@ -1844,8 +1877,8 @@ int lora_tsqr(const uint16_t *F, int64_t ld, int64_t batch_stride, int64_t batch
   if (L.total > 0 && (!workspace || workspace_bytes < static_cast<size_t>(L.total))) return LORA_ERR_WORKSPACE;
   uint8_t *ws = static_cast<uint8_t *>(workspace);
   QrParams p = qr_params(L, F, ld, batch_stride, batch, m, n, R, Q, ws);
-  if (!qr_up(p, L, ws, stream)) return LORA_ERR_CUDA;
-  if (want_q && !qr_down(p, L, ws, stream)) return LORA_ERR_CUDA;
+  if (!qr_up(p, L, ws, stream, ds->num_sms)) return LORA_ERR_CUDA;
+  if (want_q && !qr_down(p, L, ws, stream, ds->num_sms)) return LORA_ERR_CUDA;
   return LORA_OK;
 }
 
@@ -1913,10 +1946,10 @@ int lora_compress_spectra(const uint16_t *A_rows, int64_t a_bstride, const uint1
   // A = Q_A·R_A (A's column j = row j of the module's A rows), B^T = Q_B·R_B
   QrParams pa = qr_params(C.LA, A_rows, d_in, a_bstride, n_modules, d_in, r, f(C.off_RA), f(C.off_reflA),
                           ws + C.off_treeA);
-  if (!qr_up(pa, C.LA, ws + C.off_treeA, stream)) return LORA_ERR_CUDA;
+  if (!qr_up(pa, C.LA, ws + C.off_treeA, stream, ds->num_sms)) return LORA_ERR_CUDA;
   QrParams pb = qr_params(C.LB, B_rows, d_out, b_bstride, n_modules, d_out, r, f(C.off_RB), f(C.off_reflB),
                           ws + C.off_treeB);
-  if (!qr_up(pb, C.LB, ws + C.off_treeB, stream)) return LORA_ERR_CUDA;
+  if (!qr_up(pb, C.LB, ws + C.off_treeB, stream, ds->num_sms)) return LORA_ERR_CUDA;
   lora_core_svd_kernel<<<static_cast<unsigned>(n_modules), kSvdThreads, svd_smem(r), stream>>>(
       f(C.off_RA), f(C.off_RB), r, sigma, f(C.off_U), f(C.off_V));
   return launch_status();
@@ -1969,12 +2002,12 @@ int lora_compress_export(const float *sigma, const int32_t *k, const int64_t *of
   pa.out_rows = A_new;
   pa.out_k = k;
   pa.out_row0 = offsets;
-  if (!qr_down(pa, C.LA, ws + C.off_treeA, stream)) return LORA_ERR_CUDA;
+  if (!qr_down(pa, C.LA, ws + C.off_treeA, stream, ds->num_sms)) return LORA_ERR_CUDA;
   pb.root_c = f(C.off_CB);
   pb.out_rows = B_new;
   pb.out_k = k;
   pb.out_row0 = offsets;
-  if (!qr_down(pb, C.LB, ws + C.off_treeB, stream)) return LORA_ERR_CUDA;
+  if (!qr_down(pb, C.LB, ws + C.off_treeB, stream, ds->num_sms)) return LORA_ERR_CUDA;
   return LORA_OK;
 }
 

@@ -196,42 +196,16 @@ __device__ __forceinline__ void warp_qr(float (&a)[RPL][NC], int n, float *hv) {
   }
 }
 
-// Factor the nodes of one level, one warp per node (blockIdx.x · 4 + warp =
-// matrix · nodes + node).
+// After a node's tile is in registers: its QR, the reflectors and their v_0,
+// tau for the way down (Q wanted), and its R (to the parent's stacked pair, or
+// at the root with a non-negative diagonal).
 template <int NC, int RPL>
-__global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr_factor_warp_kernel(const QrParams p) {
+__device__ __forceinline__ void warp_factor_node(const QrParams &p, float (&a)[RPL][NC], int64_t b, int k, int64_t r0,
+                                                 int s) {
   const int lane = threadIdx.x & 31;
   const int nodes = p.lv.nodes;
-  const int64_t g = static_cast<int64_t>(blockIdx.x) * (kQrWarpThreads / 32) + (threadIdx.x >> 5);
-  if (g >= p.batch * nodes) return;  // uniform per warp
-  const int64_t b = g / nodes;
-  const int k = static_cast<int>(g - b * nodes);
   const int n = p.n;
   const bool want_q = p.Q != nullptr;
-  float a[RPL][NC];
-  int s;
-  int64_t r0 = 0;
-  if (p.level == 0) {
-    qr_leaf_rows(p.m, nodes, k, r0, s);
-    const uint16_t *src = p.F + b * p.bstride + r0;
-#pragma unroll
-    for (int r = 0; r < RPL; ++r)
-#pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        const int i = 32 * r + lane;
-        a[r][c] = (c < n && i < s) ? bf16_to_f32(__ldg(src + c * p.ld + i)) : 0.f;
-      }
-  } else {
-    s = qr_node_parts(p.lv.below, k) * n;
-    const float *src = p.lv.S + (b * nodes + k) * 2 * n * n;
-#pragma unroll
-    for (int r = 0; r < RPL; ++r)
-#pragma unroll
-      for (int c = 0; c < NC; ++c) {
-        const int i = 32 * r + lane;
-        a[r][c] = (c < n && i < s) ? src[c * 2 * n + i] : 0.f;
-      }
-  }
   warp_qr<NC, RPL>(a, n, want_q ? p.lv.hv + (b * nodes + k) * 2 * n : nullptr);
   if (want_q) {
     // the reflectors (entries below the diagonal) and their v_0, tau
@@ -274,34 +248,121 @@ __global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr
   }
 }
 
-// Going down, one warp per node: y = H_0·...·H_{n-1}·[C; 0] (C the node's block
-// of its parent's result, the sign diagonal at the root), the reflectors read
-// column by column from where the factor pass stored them. The row blocks of y
-// go to the children's C or, at a leaf, to Q.
+// Factor the nodes of one level, one warp per node (blockIdx.x · 4 + warp =
+// matrix · nodes + node).
 template <int NC, int RPL>
-__global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr_apply_warp_kernel(const QrParams p) {
+__global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr_factor_warp_kernel(const QrParams p) {
   const int lane = threadIdx.x & 31;
   const int nodes = p.lv.nodes;
   const int64_t g = static_cast<int64_t>(blockIdx.x) * (kQrWarpThreads / 32) + (threadIdx.x >> 5);
-  if (g >= p.batch * nodes) return;
+  if (g >= p.batch * nodes) return;  // uniform per warp
   const int64_t b = g / nodes;
   const int k = static_cast<int>(g - b * nodes);
   const int n = p.n;
+  float a[RPL][NC];
   int s;
   int64_t r0 = 0;
-  const float *vsrc;
-  int64_t cstride;
   if (p.level == 0) {
     qr_leaf_rows(p.m, nodes, k, r0, s);
-    vsrc = p.Q + b * n * p.m + r0;
-    cstride = p.m;
+    const uint16_t *src = p.F + b * p.bstride + r0;
+#pragma unroll
+    for (int r = 0; r < RPL; ++r)
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int i = 32 * r + lane;
+        a[r][c] = (c < n && i < s) ? bf16_to_f32(__ldg(src + c * p.ld + i)) : 0.f;
+      }
   } else {
     s = qr_node_parts(p.lv.below, k) * n;
-    vsrc = p.lv.S + (b * nodes + k) * 2 * n * n;
-    cstride = 2 * n;
+    const float *src = p.lv.S + (b * nodes + k) * 2 * n * n;
+#pragma unroll
+    for (int r = 0; r < RPL; ++r)
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        const int i = 32 * r + lane;
+        a[r][c] = (c < n && i < s) ? src[c * 2 * n + i] : 0.f;
+      }
   }
-  const float *hv = p.lv.hv + (b * nodes + k) * 2 * n;
-  float y[RPL][NC];
+  warp_factor_node<NC, RPL>(p, a, b, k, r0, s);
+}
+
+// 16-byte copy global -> shared that does not wait (cp.async, L2 only), reading
+// src_bytes (0 .. 16) and zero-filling the rest; a commit closes a group, and
+// wait<N> returns once at most N of this thread's groups are in flight.
+__device__ __forceinline__ void cp_async16(void *dst, const void *src, int src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
+}
+
+// The leaf level, persistent: each warp takes leaves g, g + (all warps), ... and
+// copies the next leaf's tile (bf16, [NC columns][128 rows], zero past the
+// matrix's rows) into the other half of its shared-memory buffer while it
+// factors the current one, so the tile loads no longer stall the warp.
+// Needs 16-byte aligned rows: F, ld and bstride multiples of 8 elements.
+template <int NC>
+__host__ __device__ constexpr int qr_leaf_factor_smem() { return (kQrWarpThreads / 32) * 2 * NC * kQrTile * 2; }
+template <int NC>
+__global__ void __launch_bounds__(kQrWarpThreads, NC > 16 ? 2 : 4) lora_qr_factor_leaf_kernel(const QrParams p) {
+  extern __shared__ __align__(16) uint8_t qlf[];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  uint16_t *buf = reinterpret_cast<uint16_t *>(qlf) + wid * 2 * NC * kQrTile;
+  const int nodes = p.lv.nodes, n = p.n;
+  const int64_t total = p.batch * nodes;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * (kQrWarpThreads / 32);
+  int64_t g = static_cast<int64_t>(blockIdx.x) * (kQrWarpThreads / 32) + wid;
+  // chunk q of a tile: column q / 16, rows 8·(q % 16) .. + 7
+  auto issue = [&](int64_t gg, int st) {
+    const int64_t b = gg / nodes;
+    const int k = static_cast<int>(gg - b * nodes);
+    int64_t r0;
+    int s;
+    qr_leaf_rows(p.m, nodes, k, r0, s);
+    const uint16_t *src = p.F + b * p.bstride + r0;
+    uint16_t *dst = buf + st * NC * kQrTile;
+#pragma unroll
+    for (int t = 0; t < NC / 2; ++t) {
+      const int q = t * 32 + lane, c = q >> 4, r8 = (q & 15) * 8;
+      const int valid = c < n ? max(0, min(8, s - r8)) : 0;
+      cp_async16(dst + c * kQrTile + r8, valid > 0 ? static_cast<const void *>(src + c * p.ld + r8) : p.F,
+                 valid * 2);
+    }
+    cp_async_commit();
+  };
+  if (g < total) issue(g, 0);
+  for (int st = 0; g < total; g += step, st ^= 1) {
+    if (g + step < total) issue(g + step, st ^ 1);
+    else cp_async_commit();  // an empty group: the wait below still means "this tile is in"
+    cp_async_wait<1>();
+    __syncwarp();
+    const int64_t b = g / nodes;
+    const int k = static_cast<int>(g - b * nodes);
+    int64_t r0;
+    int s;
+    qr_leaf_rows(p.m, nodes, k, r0, s);
+    const uint16_t *t = buf + st * NC * kQrTile;
+    float a[4][NC];
+#pragma unroll
+    for (int r = 0; r < 4; ++r)
+#pragma unroll
+      for (int c = 0; c < NC; ++c) a[r][c] = c < n ? bf16_to_f32(t[c * kQrTile + 32 * r + lane]) : 0.f;
+    __syncwarp();  // the buffer half is read: the next issue may refill it
+    warp_factor_node<NC, 4>(p, a, b, k, r0, s);
+  }
+  cp_async_wait<0>();
+}
+
+// The way down's start for one node: y = [C; 0] with C the node's block of its
+// parent's result (at the root: the root block when given, else the sign
+// diagonal), rows i = 32·r + lane.
+template <int NC, int RPL>
+__device__ __forceinline__ void warp_apply_init(const QrParams &p, float (&y)[RPL][NC], int64_t b, int k) {
+  const int lane = threadIdx.x & 31;
+  const int n = p.n, nodes = p.lv.nodes;
 #pragma unroll
   for (int r = 0; r < RPL; ++r)
 #pragma unroll
@@ -323,32 +384,15 @@ __global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr
         if (c < n) y[0][c] = cb[c * n];
     }
   }
-#pragma unroll
-  for (int j = NC - 1; j >= 0; --j) {
-    if (j >= n) continue;  // uniform
-    const float t = hv[n + j];
-    if (t == 0.f) continue;  // uniform
-    const float v0 = hv[j];
-    float v[RPL];
-#pragma unroll
-    for (int r = 0; r < RPL; ++r) {
-      const int i = 32 * r + lane;
-      v[r] = (i > j && i < s) ? vsrc[j * cstride + i] : (i == j ? v0 : 0.f);
-    }
-    float w[NC];
-#pragma unroll
-    for (int c = 0; c < NC; ++c) {
-      float sum = 0.f;
-#pragma unroll
-      for (int r = 0; r < RPL; ++r) sum += v[r] * y[r][c];
-      w[c] = sum;
-    }
-    warp_allreduce<NC>(w);
-#pragma unroll
-    for (int c = 0; c < NC; ++c)
-#pragma unroll
-      for (int r = 0; r < RPL; ++r) y[r][c] -= t * v[r] * w[c];
-  }
+}
+
+// The way down's end for one node: a leaf writes its rows of Q (or the export's
+// bf16 rows), an inner node its row blocks into the children's C.
+template <int NC, int RPL>
+__device__ __forceinline__ void warp_apply_store(const QrParams &p, const float (&y)[RPL][NC], int64_t b, int k,
+                                                 int64_t r0, int s) {
+  const int lane = threadIdx.x & 31;
+  const int n = p.n;
   if (p.level == 0 && p.out_rows) {
     const int kb = min(p.out_k[b], n);
     uint16_t *o = p.out_rows + p.out_row0[b] * p.m + r0;
@@ -381,6 +425,146 @@ __global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr
         if (c < n) cb[c * n] = y[r][c];
     }
   }
+}
+
+// Going down, one warp per node: y = H_0·...·H_{n-1}·[C; 0] (C the node's block
+// of its parent's result, the sign diagonal at the root), the reflectors read
+// column by column from where the factor pass stored them. The row blocks of y
+// go to the children's C or, at a leaf, to Q.
+template <int NC, int RPL>
+__global__ void __launch_bounds__(kQrWarpThreads, NC * RPL > 64 ? 2 : 4) lora_qr_apply_warp_kernel(const QrParams p) {
+  const int lane = threadIdx.x & 31;
+  const int nodes = p.lv.nodes;
+  const int64_t g = static_cast<int64_t>(blockIdx.x) * (kQrWarpThreads / 32) + (threadIdx.x >> 5);
+  if (g >= p.batch * nodes) return;
+  const int64_t b = g / nodes;
+  const int k = static_cast<int>(g - b * nodes);
+  const int n = p.n;
+  int s;
+  int64_t r0 = 0;
+  const float *vsrc;
+  int64_t cstride;
+  if (p.level == 0) {
+    qr_leaf_rows(p.m, nodes, k, r0, s);
+    vsrc = p.Q + b * n * p.m + r0;
+    cstride = p.m;
+  } else {
+    s = qr_node_parts(p.lv.below, k) * n;
+    vsrc = p.lv.S + (b * nodes + k) * 2 * n * n;
+    cstride = 2 * n;
+  }
+  const float *hv = p.lv.hv + (b * nodes + k) * 2 * n;
+  float y[RPL][NC];
+  warp_apply_init<NC, RPL>(p, y, b, k);
+#pragma unroll
+  for (int j = NC - 1; j >= 0; --j) {
+    if (j >= n) continue;  // uniform
+    const float t = hv[n + j];
+    if (t == 0.f) continue;  // uniform
+    const float v0 = hv[j];
+    float v[RPL];
+#pragma unroll
+    for (int r = 0; r < RPL; ++r) {
+      const int i = 32 * r + lane;
+      v[r] = (i > j && i < s) ? vsrc[j * cstride + i] : (i == j ? v0 : 0.f);
+    }
+    float w[NC];
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      float sum = 0.f;
+#pragma unroll
+      for (int r = 0; r < RPL; ++r) sum += v[r] * y[r][c];
+      w[c] = sum;
+    }
+    warp_allreduce<NC>(w);
+#pragma unroll
+    for (int c = 0; c < NC; ++c)
+#pragma unroll
+      for (int r = 0; r < RPL; ++r) y[r][c] -= t * v[r] * w[c];
+  }
+  warp_apply_store<NC, RPL>(p, y, b, k, r0, s);
+}
+
+// The way down's leaf level, persistent: each warp takes leaves g, g + (all
+// warps), ... and copies the next leaf's reflectors (fp32, [NC columns][128
+// rows] of Q's buffer, zero past the matrix's rows) into the other half of its
+// shared-memory buffer while it applies the current ones; the leaf's v_0 and tau
+// are read once per leaf, lane c holding column c's, and passed out by shuffle.
+// Needs m a multiple of 4 (16-byte rows of Q's buffer).
+template <int NC>
+__host__ __device__ constexpr int qr_leaf_apply_smem() { return (kQrWarpThreads / 32) * 2 * NC * kQrTile * 4; }
+template <int NC>
+__global__ void __launch_bounds__(kQrWarpThreads, 3) lora_qr_apply_leaf_kernel(const QrParams p) {
+  extern __shared__ __align__(16) uint8_t qla[];
+  const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+  float *buf = reinterpret_cast<float *>(qla) + wid * 2 * NC * kQrTile;
+  const int nodes = p.lv.nodes, n = p.n;
+  const int64_t total = p.batch * nodes;
+  const int64_t step = static_cast<int64_t>(gridDim.x) * (kQrWarpThreads / 32);
+  int64_t g = static_cast<int64_t>(blockIdx.x) * (kQrWarpThreads / 32) + wid;
+  // chunk q of a tile: column q / 32, rows 4·(q % 32) .. + 3
+  auto issue = [&](int64_t gg, int st) {
+    const int64_t b = gg / nodes;
+    const int k = static_cast<int>(gg - b * nodes);
+    int64_t r0;
+    int s;
+    qr_leaf_rows(p.m, nodes, k, r0, s);
+    const float *src = p.Q + b * n * p.m + r0;
+    float *dst = buf + st * NC * kQrTile;
+#pragma unroll
+    for (int t = 0; t < NC; ++t) {
+      const int q = t * 32 + lane, c = q >> 5, r4 = (q & 31) * 4;
+      const int valid = c < n ? max(0, min(4, s - r4)) : 0;
+      cp_async16(dst + c * kQrTile + r4, valid > 0 ? static_cast<const void *>(src + c * p.m + r4) : p.Q, valid * 4);
+    }
+    cp_async_commit();
+  };
+  if (g < total) issue(g, 0);
+  for (int st = 0; g < total; g += step, st ^= 1) {
+    if (g + step < total) issue(g + step, st ^ 1);
+    else cp_async_commit();  // an empty group: the wait below still means "this tile is in"
+    const int64_t b = g / nodes;
+    const int k = static_cast<int>(g - b * nodes);
+    int64_t r0;
+    int s;
+    qr_leaf_rows(p.m, nodes, k, r0, s);
+    const float *hv = p.lv.hv + (b * nodes + k) * 2 * n;
+    const float my_v0 = lane < n ? hv[lane] : 0.f, my_tau = lane < n ? hv[n + lane] : 0.f;
+    float y[4][NC];
+    warp_apply_init<NC, 4>(p, y, b, k);
+    cp_async_wait<1>();
+    __syncwarp();
+    const float *t = buf + st * NC * kQrTile;
+#pragma unroll
+    for (int j = NC - 1; j >= 0; --j) {
+      if (j >= n) continue;  // uniform
+      const float tj = __shfl_sync(0xFFFFFFFFu, my_tau, j);
+      if (tj == 0.f) continue;  // uniform
+      const float v0 = __shfl_sync(0xFFFFFFFFu, my_v0, j);
+      float v[4];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int i = 32 * r + lane;
+        v[r] = i > j ? t[j * kQrTile + i] : (i == j ? v0 : 0.f);
+      }
+      float w[NC];
+#pragma unroll
+      for (int c = 0; c < NC; ++c) {
+        float sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sum += v[r] * y[r][c];
+        w[c] = sum;
+      }
+      warp_allreduce<NC>(w);
+#pragma unroll
+      for (int c = 0; c < NC; ++c)
+#pragma unroll
+        for (int r = 0; r < 4; ++r) y[r][c] -= tj * v[r] * w[c];
+    }
+    __syncwarp();  // the buffer half is read: the next issue may refill it
+    warp_apply_store<NC, 4>(p, y, b, k, r0, s);
+  }
+  cp_async_wait<0>();
 }
 
 // ------------------------------------------------------------------ CTA build (32 < n <= 64)
