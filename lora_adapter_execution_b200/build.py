@@ -18,7 +18,7 @@ ROOT = os.path.dirname(HERE)
 LIB = os.path.join(HERE, "liblora_b200.so")
 BUILD_DIR = os.path.join(ROOT, "_build")
 SOURCES = [os.path.join(CSRC, "lora_b200.cu"), os.path.join(CSRC, "plan.cpp")]
-DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("common.cuh", "gemm.cuh", "skinny.cuh", "switch.cuh", "tsqr.cuh", "compress.cuh", "internal.h")] + [
+DEPS = SOURCES + [os.path.join(CSRC, f) for f in ("common.cuh", "gemm.cuh", "skinny.cuh", "switch.cuh", "tsqr.cuh", "compress.cuh", "qr_api.inc", "internal.h")] + [
     os.path.join(ROOT, "include", "lora.h")]
 
 NVCC = os.environ.get("NVCC", "/usr/local/cuda/bin/nvcc")

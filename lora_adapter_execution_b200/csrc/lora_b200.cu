@@ -35,6 +35,8 @@ DeviceState g_dev[kMaxDevices];
 std::mutex g_mu;
 PFN_cuTensorMapEncodeTiled_v12000 g_encode = nullptr;
 
+bool qr_kernel_attributes();  // qr_api.inc
+
 int device_state(DeviceState **out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return LORA_ERR_CUDA;
@@ -80,16 +82,7 @@ int device_state(DeviceState **out) {
                                      sk_smem(2)) == cudaSuccess;
           ok &= cudaFuncSetAttribute(lora_tcontract_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      tc_smem(kTcMaxR)) == cudaSuccess;
-          ok &= cudaFuncSetAttribute(lora_qr_factor_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     qr_factor_smem(kQrMaxN)) == cudaSuccess;
-          ok &= cudaFuncSetAttribute(lora_qr_apply_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     qr_apply_smem(kQrMaxN)) == cudaSuccess;
-          ok &= cudaFuncSetAttribute(lora_core_svd_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     svd_smem(kSvdMaxN)) == cudaSuccess;
-          ok &= cudaFuncSetAttribute(lora_qr_factor_leaf_kernel<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     qr_leaf_factor_smem<32>()) == cudaSuccess;
-          ok &= cudaFuncSetAttribute(lora_qr_apply_leaf_kernel<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     qr_leaf_apply_smem<16>()) == cudaSuccess;
+          ok &= qr_kernel_attributes();
           if (!ok) d.status = LORA_ERR_CUDA;
           for (int S = 1; ok && S <= 4; S *= 2) {
             cudaLaunchConfig_t cfg{};
@@ -1709,306 +1702,6 @@ int lora_switch_apply(lora_switch_t sw, uint16_t *W, const uint16_t *A_pool, con
 
 }  // extern "C"
 
-// ------------------------------------------------------------------ batched tall-skinny QR
-namespace {
-// The tree's levels for m rows, and the workspace: the root's row signs, then
-// per level its stacked pairs (level >= 1), its reflector scalars and its
-// blocks of the way down (the last two only when Q is wanted).
-struct QrLayout {
-  std::vector<int32_t> nodes;
-  std::vector<int64_t> off_S, off_hv, off_C;  // byte offsets, -1 where absent
-  int64_t off_sign = -1, total = 0;
-};
-QrLayout qr_layout(int64_t batch, int64_t m, int32_t n, bool want_q) {
-  auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
-  QrLayout L;
-  L.nodes.push_back(qr_leaves(m));
-  while (L.nodes.back() > 1) L.nodes.push_back((L.nodes.back() + 1) / 2);
-  const int nl = static_cast<int>(L.nodes.size());
-  int64_t o = 0;
-  if (want_q) {
-    L.off_sign = o;
-    o += up(batch * n * 4);
-  }
-  L.off_S.assign(nl, -1);
-  L.off_hv.assign(nl, -1);
-  L.off_C.assign(nl, -1);
-  for (int l = 0; l < nl; ++l) {
-    const int64_t nodes = L.nodes[l];
-    if (l >= 1) {
-      L.off_S[l] = o;
-      o += up(batch * nodes * 2 * n * n * 4);
-    }
-    if (want_q) {
-      L.off_hv[l] = o;
-      o += up(batch * nodes * 2 * n * 4);
-      if (l + 1 < nl) {
-        L.off_C[l] = o;
-        o += up(batch * nodes * n * n * 4);
-      }
-    }
-  }
-  L.total = o;
-  return L;
-}
-// One level's launch: a warp per node for n <= 32 (the column bound NC and the
-// rows per lane RPL as templates: leaves hold 128 rows, stacked pairs 2n), a
-// CTA per node above.
-template <int NC, int RPL>
-bool launch_qr_warp(const QrParams &p, int64_t units, bool apply, cudaStream_t st) {
-  const unsigned grid = static_cast<unsigned>((units + kQrWarpThreads / 32 - 1) / (kQrWarpThreads / 32));
-  if (apply) lora_qr_apply_warp_kernel<NC, RPL><<<grid, kQrWarpThreads, 0, st>>>(p);
-  else lora_qr_factor_warp_kernel<NC, RPL><<<grid, kQrWarpThreads, 0, st>>>(p);
-  return cudaGetLastError() == cudaSuccess;
-}
-template <int NC>
-bool launch_qr_nc(const QrParams &p, int64_t units, int rows, bool apply, cudaStream_t st) {
-  if (rows <= 32) return launch_qr_warp<NC, 1>(p, units, apply, st);
-  if (rows <= 64) return launch_qr_warp<NC, 2>(p, units, apply, st);
-  return launch_qr_warp<NC, 4>(p, units, apply, st);
-}
-// the way up's leaf level, persistent with its next tile copied in the
-// background (16-byte rows needed), for n <= 32
-template <int NC>
-bool launch_qr_leaf(const QrParams &p, int64_t units, int sms, cudaStream_t st) {
-  const int per_sm = NC > 16 ? 2 : 4;
-  const int64_t want = (units + kQrWarpThreads / 32 - 1) / (kQrWarpThreads / 32);
-  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sms) * per_sm)));
-  lora_qr_factor_leaf_kernel<NC><<<grid, kQrWarpThreads, qr_leaf_factor_smem<NC>(), st>>>(p);
-  return cudaGetLastError() == cudaSuccess;
-}
-// the way down's leaf level likewise, for n <= 16 (reflector rows of 16 bytes)
-template <int NC>
-bool launch_qr_leaf_apply(const QrParams &p, int64_t units, int sms, cudaStream_t st) {
-  const int64_t want = (units + kQrWarpThreads / 32 - 1) / (kQrWarpThreads / 32);
-  const unsigned grid = static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(want, int64_t(sms) * 3)));
-  lora_qr_apply_leaf_kernel<NC><<<grid, kQrWarpThreads, qr_leaf_apply_smem<NC>(), st>>>(p);
-  return cudaGetLastError() == cudaSuccess;
-}
-bool launch_qr(const QrParams &p, int64_t units, int rows, bool apply, lora_stream_t stream, int sms) {
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const bool rows16 = (reinterpret_cast<uintptr_t>(p.F) & 15) == 0 && p.ld % 8 == 0 && p.bstride % 8 == 0;
-  if (!apply && p.level == 0 && p.F && rows16 && sms > 0) {
-    if (p.n <= 8) return launch_qr_leaf<8>(p, units, sms, st);
-    if (p.n <= 16) return launch_qr_leaf<16>(p, units, sms, st);
-    if (p.n <= kQrWarpMaxN) return launch_qr_leaf<32>(p, units, sms, st);
-  }
-  const bool q16 = (reinterpret_cast<uintptr_t>(p.Q) & 15) == 0 && p.m % 4 == 0;
-  if (apply && p.level == 0 && p.Q && q16 && sms > 0) {
-    if (p.n <= 8) return launch_qr_leaf_apply<8>(p, units, sms, st);
-    if (p.n <= 16) return launch_qr_leaf_apply<16>(p, units, sms, st);
-  }
-  if (p.n <= 8) return launch_qr_nc<8>(p, units, rows, apply, st);
-  if (p.n <= 16) return launch_qr_nc<16>(p, units, rows, apply, st);
-  if (p.n <= kQrWarpMaxN) return launch_qr_nc<32>(p, units, rows, apply, st);
-  if (apply) lora_qr_apply_kernel<<<static_cast<unsigned>(units), kQrThreads, qr_apply_smem(p.n), st>>>(p);
-  else lora_qr_factor_kernel<<<static_cast<unsigned>(units), kQrThreads, qr_factor_smem(p.n), st>>>(p);
-  return cudaGetLastError() == cudaSuccess;
-}
-
-QrParams qr_params(const QrLayout &L, const uint16_t *F, int64_t ld, int64_t bstride, int64_t batch, int64_t m,
-                   int32_t n, float *R, float *Q, uint8_t *ws) {
-  QrParams p{};
-  p.batch = batch;
-  p.m = m;
-  p.n = n;
-  p.ld = ld;
-  p.bstride = bstride;
-  p.F = F;
-  p.Q = Q;
-  p.R = R;
-  p.sign = L.off_sign < 0 ? nullptr : reinterpret_cast<float *>(ws + L.off_sign);
-  return p;
-}
-QrLevel qr_level(const QrLayout &L, uint8_t *ws, int l) {
-  auto at = [&](int64_t off) { return off < 0 ? nullptr : reinterpret_cast<float *>(ws + off); };
-  const int nl = static_cast<int>(L.nodes.size());
-  QrLevel lv{};
-  lv.nodes = L.nodes[l];
-  lv.below = l >= 1 ? L.nodes[l - 1] : 0;
-  lv.up = l + 1 < nl ? L.nodes[l + 1] : 0;
-  lv.S = at(L.off_S[l]);
-  lv.S_up = l + 1 < nl ? at(L.off_S[l + 1]) : nullptr;
-  lv.hv = at(L.off_hv[l]);
-  lv.C = at(L.off_C[l]);
-  lv.C_down = l >= 1 ? at(L.off_C[l - 1]) : nullptr;
-  return lv;
-}
-// up the tree: every level's QR (R at the root; with p.Q, the reflectors kept
-// in Q's buffer and the workspace for the way down)
-bool qr_up(QrParams p, const QrLayout &L, uint8_t *ws, lora_stream_t stream, int sms) {
-  for (int l = 0; l < static_cast<int>(L.nodes.size()); ++l) {
-    p.level = l;
-    p.lv = qr_level(L, ws, l);
-    if (!launch_qr(p, p.batch * L.nodes[l], l == 0 ? kQrTile : 2 * p.n, false, stream, sms)) return false;
-  }
-  return true;
-}
-// down the tree: Q (or, with p.root_c / p.out_rows, Q times the root block)
-bool qr_down(QrParams p, const QrLayout &L, uint8_t *ws, lora_stream_t stream, int sms) {
-  for (int l = static_cast<int>(L.nodes.size()) - 1; l >= 0; --l) {
-    p.level = l;
-    p.lv = qr_level(L, ws, l);
-    if (!launch_qr(p, p.batch * L.nodes[l], l == 0 ? kQrTile : 2 * p.n, true, stream, sms)) return false;
-  }
-  return true;
-}
-bool qr_args_ok(int64_t batch, int64_t m, int32_t n) {
-  return batch >= 1 && n >= 1 && n <= kQrMaxN && m >= n && m <= (int64_t(1) << 31) &&
-         batch * qr_leaves(m) <= 0x7FFFFFFF && batch * m * n <= (int64_t(1) << 40);
-}
-}  // namespace
-
-extern "C" {
-
-size_t lora_tsqr_workspace_size(int64_t batch, int64_t m, int32_t n, int want_q) {
-  if (!qr_args_ok(batch, m, n)) return 0;
-  return static_cast<size_t>(qr_layout(batch, m, n, want_q != 0).total);
-}
-
-int lora_tsqr(const uint16_t *F, int64_t ld, int64_t batch_stride, int64_t batch, int64_t m, int32_t n, float *R,
-              float *Q, void *workspace, size_t workspace_bytes, lora_stream_t stream) {
-  if (!F || !R || !qr_args_ok(batch, m, n) || ld < m || batch_stride < 0) return LORA_ERR_ARG;
-  DeviceState *ds = nullptr;
-  int rc = device_state(&ds);
-  if (rc != LORA_OK) return rc;
-  const bool want_q = Q != nullptr;
-  const QrLayout L = qr_layout(batch, m, n, want_q);
-  if (L.total > 0 && (!workspace || workspace_bytes < static_cast<size_t>(L.total))) return LORA_ERR_WORKSPACE;
-  uint8_t *ws = static_cast<uint8_t *>(workspace);
-  QrParams p = qr_params(L, F, ld, batch_stride, batch, m, n, R, Q, ws);
-  if (!qr_up(p, L, ws, stream, ds->num_sms)) return LORA_ERR_CUDA;
-  if (want_q && !qr_down(p, L, ws, stream, ds->num_sms)) return LORA_ERR_CUDA;
-  return LORA_OK;
-}
-
-}  // extern "C"
-
-// ------------------------------------------------------------------ post-hoc compression
-namespace {
-// A group of modules sharing d_in, d_out and r: the two factors' trees, their
-// reflectors (the tall-skinny QR's Q buffers), R, the cores' U, V and the
-// way-down root blocks, all in one workspace that lora_compress_spectra fills
-// and lora_compress_export reads.
-struct CompressLayout {
-  QrLayout LA, LB;
-  int64_t off_reflA = 0, off_reflB = 0, off_treeA = 0, off_treeB = 0;
-  int64_t off_RA = 0, off_RB = 0, off_U = 0, off_V = 0, off_CA = 0, off_CB = 0, total = 0;
-};
-CompressLayout compress_layout(int64_t n, int64_t d_in, int64_t d_out, int32_t r) {
-  auto up = [](int64_t b) { return (b + 255) & ~static_cast<int64_t>(255); };
-  CompressLayout C;
-  C.LA = qr_layout(n, d_in, r, true);
-  C.LB = qr_layout(n, d_out, r, true);
-  int64_t o = 0;
-  C.off_reflA = o;
-  o += up(n * r * d_in * 4);
-  C.off_reflB = o;
-  o += up(n * r * d_out * 4);
-  C.off_treeA = o;
-  o += up(C.LA.total);
-  C.off_treeB = o;
-  o += up(C.LB.total);
-  const int64_t rr = up(n * r * r * 4);
-  C.off_RA = o;
-  C.off_RB = o + rr;
-  C.off_U = o + 2 * rr;
-  C.off_V = o + 3 * rr;
-  C.off_CA = o + 4 * rr;
-  C.off_CB = o + 5 * rr;
-  C.total = o + 6 * rr;
-  return C;
-}
-bool compress_args_ok(int64_t n, int64_t d_in, int64_t d_out, int32_t r) {
-  return r >= 1 && r <= kSvdMaxN && qr_args_ok(n, d_in, r) && qr_args_ok(n, d_out, r) && n <= 0x7FFFFFFF;
-}
-}  // namespace
-
-extern "C" {
-
-size_t lora_compress_workspace_size(int64_t n_modules, int64_t d_in, int64_t d_out, int32_t r) {
-  if (!compress_args_ok(n_modules, d_in, d_out, r)) return 0;
-  return static_cast<size_t>(compress_layout(n_modules, d_in, d_out, r).total);
-}
-
-int lora_compress_spectra(const uint16_t *A_rows, int64_t a_bstride, const uint16_t *B_rows, int64_t b_bstride,
-                          int64_t n_modules, int64_t d_in, int64_t d_out, int32_t r, float *sigma, void *workspace,
-                          size_t workspace_bytes, lora_stream_t stream) {
-  if (!A_rows || !B_rows || !sigma || a_bstride < 0 || b_bstride < 0 || !compress_args_ok(n_modules, d_in, d_out, r))
-    return LORA_ERR_ARG;
-  DeviceState *ds = nullptr;
-  int rc = device_state(&ds);
-  if (rc != LORA_OK) return rc;
-  const CompressLayout C = compress_layout(n_modules, d_in, d_out, r);
-  if (!workspace || workspace_bytes < static_cast<size_t>(C.total)) return LORA_ERR_WORKSPACE;
-  uint8_t *ws = static_cast<uint8_t *>(workspace);
-  auto f = [&](int64_t off) { return reinterpret_cast<float *>(ws + off); };
-  // A = Q_A·R_A (A's column j = row j of the module's A rows), B^T = Q_B·R_B
-  QrParams pa = qr_params(C.LA, A_rows, d_in, a_bstride, n_modules, d_in, r, f(C.off_RA), f(C.off_reflA),
-                          ws + C.off_treeA);
-  if (!qr_up(pa, C.LA, ws + C.off_treeA, stream, ds->num_sms)) return LORA_ERR_CUDA;
-  QrParams pb = qr_params(C.LB, B_rows, d_out, b_bstride, n_modules, d_out, r, f(C.off_RB), f(C.off_reflB),
-                          ws + C.off_treeB);
-  if (!qr_up(pb, C.LB, ws + C.off_treeB, stream, ds->num_sms)) return LORA_ERR_CUDA;
-  lora_core_svd_kernel<<<static_cast<unsigned>(n_modules), kSvdThreads, svd_smem(r), stream>>>(
-      f(C.off_RA), f(C.off_RB), r, sigma, f(C.off_U), f(C.off_V));
-  return launch_status();
-}
-
-size_t lora_compress_allocate_workspace_size(int64_t n_modules, int32_t r_max) {
-  if (n_modules < 1 || r_max < 1 || n_modules * r_max >= 0xFFFFFFFFll) return 0;
-  return static_cast<size_t>(n_modules * r_max * 8);
-}
-
-int lora_compress_allocate(const float *sigma, const int32_t *ranks, const int64_t *costs, int64_t n_modules,
-                           int32_t r_max, int32_t policy, double keep, int32_t k_floor, int32_t *k, int64_t *offsets,
-                           void *workspace, size_t workspace_bytes, lora_stream_t stream) {
-  if (!sigma || !ranks || !costs || !k || !offsets || n_modules < 1 || r_max < 1 || r_max > kSvdMaxN ||
-      (policy != 0 && policy != 1) || !(keep >= 0.0 && keep <= 1.0) || k_floor < 0 ||
-      n_modules * r_max >= 0xFFFFFFFFll)
-    return LORA_ERR_ARG;
-  DeviceState *ds = nullptr;
-  int rc = device_state(&ds);
-  if (rc != LORA_OK) return rc;
-  const size_t need = static_cast<size_t>(n_modules * r_max * 8);
-  if (policy == 1 && (!workspace || workspace_bytes < need)) return LORA_ERR_WORKSPACE;
-  lora_compress_alloc_kernel<<<1, kAllocThreads, 0, stream>>>(sigma, ranks, costs, n_modules, r_max, policy, keep,
-                                                             k_floor, static_cast<uint64_t *>(workspace), k,
-                                                             offsets);
-  return launch_status();
-}
-
-int lora_compress_export(const float *sigma, const int32_t *k, const int64_t *offsets, int64_t n_modules, int64_t d_in,
-                         int64_t d_out, int32_t r, uint16_t *A_new, uint16_t *B_new, void *workspace,
-                         size_t workspace_bytes, lora_stream_t stream) {
-  if (!sigma || !k || !offsets || !A_new || !B_new || !compress_args_ok(n_modules, d_in, d_out, r))
-    return LORA_ERR_ARG;
-  DeviceState *ds = nullptr;
-  int rc = device_state(&ds);
-  if (rc != LORA_OK) return rc;
-  const CompressLayout C = compress_layout(n_modules, d_in, d_out, r);
-  if (!workspace || workspace_bytes < static_cast<size_t>(C.total)) return LORA_ERR_WORKSPACE;
-  uint8_t *ws = static_cast<uint8_t *>(workspace);
-  auto f = [&](int64_t off) { return reinterpret_cast<float *>(ws + off); };
-  const int64_t total = n_modules * r * r;
-  const unsigned grid = static_cast<unsigned>(std::min<int64_t>((total + 255) / 256, 4096));
-  QrParams pa = qr_params(C.LA, nullptr, d_in, 0, n_modules, d_in, r, f(C.off_RA), f(C.off_reflA), ws + C.off_treeA);
-  QrParams pb = qr_params(C.LB, nullptr, d_out, 0, n_modules, d_out, r, f(C.off_RB), f(C.off_reflB),
-                          ws + C.off_treeB);
-  lora_export_roots_kernel<<<grid, 256, 0, stream>>>(f(C.off_U), sigma, pa.sign, k, n_modules, r, f(C.off_CA));
-  lora_export_roots_kernel<<<grid, 256, 0, stream>>>(f(C.off_V), sigma, pb.sign, k, n_modules, r, f(C.off_CB));
-  if (launch_status() != LORA_OK) return LORA_ERR_CUDA;
-  pa.root_c = f(C.off_CA);
-  pa.out_rows = A_new;
-  pa.out_k = k;
-  pa.out_row0 = offsets;
-  if (!qr_down(pa, C.LA, ws + C.off_treeA, stream, ds->num_sms)) return LORA_ERR_CUDA;
-  pb.root_c = f(C.off_CB);
-  pb.out_rows = B_new;
-  pb.out_k = k;
-  pb.out_row0 = offsets;
-  if (!qr_down(pb, C.LB, ws + C.off_treeB, stream, ds->num_sms)) return LORA_ERR_CUDA;
-  return LORA_OK;
-}
-
-}  // extern "C"
+// The batched tall-skinny QR and post-hoc compression entry points (and their
+// kernels' launch attributes, qr_kernel_attributes).
+#include "qr_api.inc"
