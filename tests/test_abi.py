@@ -138,3 +138,38 @@ def test_binding_checks_tensor_metadata_before_the_call():
     with pytest.raises(lora.LoraError, match="bits has shape"):
         lora.dropout_keep_bits(0, 0.1, torch.zeros(T, 3, dtype=torch.int32), d_in)
     plan.destroy()
+
+
+def test_qr_and_compression_reject_bad_arguments_before_cuda():
+    """The tall-skinny QR and the compression calls validate their sizes and
+    pointers on the host first (LORA_ERR_ARG = -1), with no CUDA call; their
+    workspace-size queries return 0 for sizes out of range."""
+    L = abi.load_library()
+    vp = ctypes.c_void_p
+    fake = vp(0x1000)  # never dereferenced: every call below fails its checks first
+    # workspace sizes: n out of range, m < n
+    assert L.lora_tsqr_workspace_size(4, 100, 65, 1) == 0
+    assert L.lora_tsqr_workspace_size(4, 10, 16, 1) == 0
+    assert L.lora_tsqr_workspace_size(4, 4096, 16, 1) > L.lora_tsqr_workspace_size(4, 4096, 16, 0) > 0
+    assert L.lora_compress_workspace_size(8, 4096, 4096, 0) == 0
+    assert L.lora_compress_workspace_size(8, 4096, 4096, 65) == 0
+    assert L.lora_compress_workspace_size(8, 12, 4096, 16) == 0   # r > d_in
+    assert L.lora_compress_allocate_workspace_size(0, 16) == 0
+    # lora_tsqr: null F or R, n > 64, m < n, ld < m
+    assert L.lora_tsqr(None, 4096, 0, 1, 4096, 16, fake, None, None, 0, None) == -1
+    assert L.lora_tsqr(fake, 4096, 0, 1, 4096, 16, None, None, None, 0, None) == -1
+    assert L.lora_tsqr(fake, 4096, 0, 1, 4096, 65, fake, None, None, 0, None) == -1
+    assert L.lora_tsqr(fake, 4096, 0, 1, 8, 16, fake, None, None, 0, None) == -1
+    assert L.lora_tsqr(fake, 100, 0, 1, 4096, 16, fake, None, None, 0, None) == -1
+    # lora_compress_spectra: null factors or sigma, rank 0
+    assert L.lora_compress_spectra(None, 0, fake, 0, 2, 256, 256, 8, fake, fake, 1 << 30, None) == -1
+    assert L.lora_compress_spectra(fake, 0, fake, 0, 2, 256, 256, 8, None, fake, 1 << 30, None) == -1
+    assert L.lora_compress_spectra(fake, 0, fake, 0, 2, 256, 256, 0, fake, fake, 1 << 30, None) == -1
+    # lora_compress_allocate: policy, keep outside [0, 1], negative floor, r_max > 64
+    assert L.lora_compress_allocate(fake, fake, fake, 4, 16, 2, 0.5, 1, fake, fake, fake, 1024, None) == -1
+    assert L.lora_compress_allocate(fake, fake, fake, 4, 16, 1, 1.5, 1, fake, fake, fake, 1024, None) == -1
+    assert L.lora_compress_allocate(fake, fake, fake, 4, 16, 1, 0.5, -1, fake, fake, fake, 1024, None) == -1
+    assert L.lora_compress_allocate(fake, fake, fake, 4, 65, 1, 0.5, 1, fake, fake, fake, 1024, None) == -1
+    # lora_compress_export: null pools
+    assert L.lora_compress_export(fake, fake, fake, 2, 256, 256, 8, None, fake, fake, 1 << 30, None) == -1
+    assert L.lora_compress_export(fake, fake, fake, 2, 256, 256, 8, fake, None, fake, 1 << 30, None) == -1
