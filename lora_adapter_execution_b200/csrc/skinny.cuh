@@ -929,6 +929,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       // are zero, and so are the columns of tokens at or past t1 (in piece mode
       // the stage's last rows can be the next segment's tokens, which must not
       // enter the sums).
+      // Only the stage's 16-token steps that hold tokens of the segment take
+      // part (nk of them): a short piece (a few tokens of a small adapter)
+      // converts and multiplies one step instead of four; the steps left out
+      // would only add products of zero columns.
+      const int nk = (min(kTcTok, t1 - (t0 + b * kTcTok)) + 15) / 16;
       {
         const int tb = t0 + b * kTcTok;
         const float *graw = reinterpret_cast<const float *>(sbp + in_bytes);
@@ -936,7 +941,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         uint8_t *gmid = ghi + mblocks * 2048;
         uint8_t *glo = gmid + mblocks * 2048;
         const int q4 = mblocks * 4;  // 4-rank groups per token pair
-        for (int item = landed ? tid : 32 * q4; item < 32 * q4; item += kTcConsumerWarps * 32) {
+        const int items = 8 * nk * q4;  // token pairs of the steps taken
+        for (int item = landed ? tid : items; item < items; item += kTcConsumerWarps * 32) {
           const int tp = item / q4;
           const int k4 = (item - tp * q4) * 4;
           float4 v0 = make_float4(0.f, 0.f, 0.f, 0.f), v1 = v0;
@@ -966,6 +972,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
       const int tbase = t0 + b * kTcTok;
 #pragma unroll
       for (int ks = 0; ks < 4; ++ks) {
+        if (ks >= nk) break;  // uniform
         uint32_t bf[2][4];
 #pragma unroll
         for (int g = 0; g < 2; ++g) ldsm_x4_t(sb + boff[ks][g], bf[g][0], bf[g][1], bf[g][2], bf[g][3]);
