@@ -407,11 +407,12 @@ __device__ __forceinline__ bool shrink_unit(uint8_t *smem, uint64_t *bars, const
   int MW = 1;
   while (MW * 2 <= mb && MW < kSkConsumerWarps) MW *= 2;
   const int KW = kSkConsumerWarps / MW;
-  // a ring stage holds NB consecutive 64-column blocks: small units (at most 32
-  // rows) take four, shared out over the KW warp groups, so their copies come in
-  // groups (a lone 16-row block pair per barrier round trip kept too few bytes
-  // moving); larger units one
-  const int NB = Rp <= 32 ? 4 : KW;
+  // a ring stage holds NB consecutive 64-column blocks: small units take eight
+  // (at most 16 rows) or four (at most 32), shared out over the KW warp groups,
+  // so their copies come in groups (a lone 16-row block pair per barrier round
+  // trip kept too few bytes moving; eight measured 1.4 % faster than four on
+  // fleet, the same on decode); larger units one
+  const int NB = Rp <= 16 ? 8 : Rp <= 32 ? 4 : KW;
   const int nstage = min(kSkMaxStages, kSkPool / (NB * stage_bytes));
 
   if (tid == 0) {
