@@ -103,10 +103,13 @@ def export_group(comp, k, off, rows):
     return host_f64(A_new), host_f64(B_new)
 
 
-@pytest.mark.parametrize("policy,keep", [("S", 0.3), ("U", 1.0), ("S", 1 / 12)])
-def test_export_vs_oracle_truncation(policy, keep):
+@pytest.mark.parametrize("policy,keep,r", [("S", 0.3, 16), ("U", 1.0, 16), ("S", 1 / 12, 16),
+                                           # the way down's other builds: the warp build's widest
+                                           # columns (r <= 32) and the CTA build (r > 32)
+                                           ("S", 0.4, 24), ("U", 1.0, 40), ("S", 0.3, 64)])
+def test_export_vs_oracle_truncation(policy, keep, r):
     import lora_adapter_execution_b200 as lora
-    n, r, d_in, d_out = 5, 16, 520, 264
+    n, d_in, d_out = 5, 520, 264
     A, B = wl.module_factors(n, r, d_in, d_out, seed=11)
     comp = spectra(A, B)
     sig = comp.sigma.cpu().numpy()
