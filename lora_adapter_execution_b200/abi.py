@@ -123,31 +123,43 @@ _F32 = ("float32",)
 _I32 = ("int32", "uint32")
 
 
+_DTYPE_NAME = {}  # torch dtype -> its short name ("bfloat16", ...), filled as dtypes are seen
+
+
+def _dtype_name(dt):
+    n = _DTYPE_NAME.get(dt)
+    if n is None:
+        n = _DTYPE_NAME[dt] = str(dt).rsplit(".", 1)[-1]
+    return n
+
+
 def _args(what, *specs):
     """Check (name, tensor, shape, dtype names, optional) for each tensor handed
     to the library call `what`: first every tensor's shape, dtype and layout,
-    then every tensor's device."""
+    then every tensor's device. (Called on every launch: the checks use the
+    cheapest accessors, a cached dtype name and the device index as an int.)"""
     given = []
     for name, t, shape, dtypes, optional in specs:
         if t is None:
             if optional:
                 continue
             raise LoraError(-1, f"{what}: {name} is required")
-        if tuple(t.shape) != tuple(shape):
+        if t.shape != tuple(shape):
             raise LoraError(-1, f"{what}: {name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
-        if str(t.dtype).rsplit(".", 1)[-1] not in dtypes:
+        if _dtype_name(t.dtype) not in dtypes:
             raise LoraError(-1, f"{what}: {name} has dtype {t.dtype}, expected {' or '.join(dtypes)}")
         if not t.is_contiguous():
             raise LoraError(-1, f"{what}: {name} is not contiguous")
         given.append((name, t))
     dev = None
     for name, t in given:
-        if not t.is_cuda:
+        idx = t.get_device()  # -1 for a host tensor
+        if idx < 0:
             raise LoraError(-1, f"{what}: {name} is not a CUDA tensor")
         if dev is None:
             import torch
             dev = torch.cuda.current_device()
-        if t.device.index != dev:
+        if idx != dev:
             raise LoraError(-1, f"{what}: {name} is on {t.device}, the current device is cuda:{dev}")
 
 

@@ -4,11 +4,11 @@
 
 #include <algorithm>
 #include <atomic>
-#include <queue>
-#include <utility>
+#include <limits>
 #include <cstdio>
 #include <cstring>
 #include <mutex>
+#include <utility>
 #include <new>
 
 #include "gemm.cuh"
@@ -230,40 +230,75 @@ void build_schedule(const HostPlan &hp, int grid, int group_m, std::vector<int32
   const int n_nt = static_cast<int>((hp.d_out + kBN - 1) / kBN);
   const int KB = static_cast<int>((hp.d_in + kBK - 1) / kBK);
   const int n_tiles = n_mt * n_nt;
-  std::vector<std::vector<int32_t>> lists(grid);
-  using Load = std::pair<int64_t, int>;  // (work so far, CTA): ties go to the lowest CTA
-  std::priority_queue<Load, std::vector<Load>, std::greater<Load>> q;
-  for (int b = 0; b < grid; ++b) q.push({0, b});
-  for (int t = 0; t < n_tiles; ++t) {
-    int mi, nt;
-    tile_mn(t, n_mt, n_nt, group_m, mi, nt);
-    const int mt = hp.mt_order.empty() ? mi : hp.mt_order[mi];
-    const int naug = (hp.tiles[mt].kaug + kAugBlock - 1) / kAugBlock;
-    const Load l = q.top();
-    q.pop();
-    lists[l.second].push_back(t);
-    q.push({l.first + 10 * KB + 13 * naug, l.second});
+  out.clear();
+  if (grid <= 0 || grid > 65535 || n_tiles <= 0) return;
+  // per m-tile cost; the visiting order of tile_mn walked group by group (n
+  // index outer, m index inner inside a group), so no division per tile
+  std::vector<int64_t> mcost(n_mt);
+  for (int mt = 0; mt < n_mt; ++mt) mcost[mt] = 10 * KB + 13 * ((hp.tiles[mt].kaug + kAugBlock - 1) / kAugBlock);
+  // the round robin's loads first: when even a perfect split of whole tiles
+  // (at least the mean, the largest tile, and ceil(tiles / CTAs) of the
+  // cheapest tiles on one CTA) could not beat its heaviest CTA by 2 % the
+  // greedy pass is skipped (nearly uniform tiles: fine-tuning, prefill)
+  std::vector<int64_t> rr(grid, 0);
+  int64_t total = 0, cmax = 0, cmin = std::numeric_limits<int64_t>::max();
+  {
+    int brr = 0;
+    for (int m0 = 0; m0 < n_mt; m0 += group_m) {
+      const int gm = std::min(group_m, n_mt - m0);
+      for (int nt = 0; nt < n_nt; ++nt)
+        for (int r = 0; r < gm; ++r) {
+          const int mi = m0 + r;
+          const int64_t c = mcost[hp.mt_order.empty() ? mi : hp.mt_order[mi]];
+          rr[brr] += c;
+          total += c;
+          cmax = std::max(cmax, c);
+          cmin = std::min(cmin, c);
+          if (++brr == grid) brr = 0;
+        }
+    }
+  }
+  const int64_t rr_max = *std::max_element(rr.begin(), rr.end());
+  const int64_t bound =
+      std::max({cmax, (total + grid - 1) / grid, static_cast<int64_t>((n_tiles + grid - 1) / grid) * cmin});
+  if (bound * 100 > rr_max * 98) return;
+  // the loads as a binary min-heap of (work << 16 | CTA): ties go to the lowest CTA
+  std::vector<uint64_t> heap(grid);
+  for (int b = 0; b < grid; ++b) heap[b] = static_cast<uint64_t>(b);
+  std::vector<int32_t> owner(n_tiles);
+  int t = 0;
+  for (int m0 = 0; m0 < n_mt; m0 += group_m) {
+    const int gm = std::min(group_m, n_mt - m0);
+    for (int nt = 0; nt < n_nt; ++nt)
+      for (int r = 0; r < gm; ++r, ++t) {
+        const int mi = m0 + r;
+        const int64_t c = mcost[hp.mt_order.empty() ? mi : hp.mt_order[mi]];
+        // the least loaded CTA takes tile t; its load grows: sift the top down
+        const uint64_t top = heap[0];
+        owner[t] = static_cast<int32_t>(top & 0xFFFFu);
+        const uint64_t v = top + (static_cast<uint64_t>(c) << 16);
+        int h = 0;
+        while (true) {
+          const int l = 2 * h + 1;
+          if (l >= grid) break;
+          const int m = (l + 1 < grid && heap[l + 1] < heap[l]) ? l + 1 : l;
+          if (heap[m] >= v) break;
+          heap[h] = heap[m];
+          h = m;
+        }
+        heap[h] = v;
+      }
   }
   // keep it only where it shortens the heaviest CTA by more than 2 % against the
   // round robin (whose tile order keeps more operands shared through L2)
   int64_t greedy_max = 0;
-  while (!q.empty()) {
-    greedy_max = std::max(greedy_max, q.top().first);
-    q.pop();
-  }
-  std::vector<int64_t> rr(grid, 0);
-  for (int t = 0; t < n_tiles; ++t) {
-    int mi, nt;
-    tile_mn(t, n_mt, n_nt, group_m, mi, nt);
-    const int mt = hp.mt_order.empty() ? mi : hp.mt_order[mi];
-    rr[t % grid] += 10 * KB + 13 * ((hp.tiles[mt].kaug + kAugBlock - 1) / kAugBlock);
-  }
-  const int64_t rr_max = *std::max_element(rr.begin(), rr.end());
-  out.clear();
+  for (uint64_t v : heap) greedy_max = std::max<int64_t>(greedy_max, static_cast<int64_t>(v >> 16));
   if (greedy_max * 100 > rr_max * 98) return;
-  out.assign(grid + 1, 0);
-  for (int b = 0; b < grid; ++b) out[b + 1] = out[b] + static_cast<int32_t>(lists[b].size());
-  for (int b = 0; b < grid; ++b) out.insert(out.end(), lists[b].begin(), lists[b].end());
+  out.assign(grid + 1 + n_tiles, 0);
+  for (int u = 0; u < n_tiles; ++u) ++out[owner[u] + 1];
+  for (int b = 0; b < grid; ++b) out[b + 1] += out[b];
+  std::vector<int32_t> pos(out.begin(), out.begin() + grid);
+  for (int u = 0; u < n_tiles; ++u) out[grid + 1 + pos[owner[u]]++] = u;
 }
 
 int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const CUtensorMap &b,
@@ -301,6 +336,7 @@ int launch_fwd_gemm(DeviceState *ds, GemmParams gp, const CUtensorMap &a, const 
 
 struct lora_plan {
   HostPlan hp;
+  HostPlan spare;  // the table set a rebuild fills before it swaps it in (storage kept across batches)
   void *dev = nullptr;       // perm | tiles | chunks | units
   uint8_t *scratch = nullptr;
   const int32_t *d_perm = nullptr;
@@ -640,10 +676,10 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
 int lora_plan_rebuild(lora_plan_t plan, const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
                       int32_t n_adapters, int64_t d_in, int64_t d_out, lora_stream_t stream) {
   if (!plan || !plan->dev || !on_plan_device(plan)) return LORA_ERR_ARG;
-  HostPlan hp;
-  int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, hp);
+  // the new tables go into the spare set (the previous batch's storage, reused)
+  int rc = build_host_plan(ids_host, T, ranks_host, n_adapters, d_in, d_out, plan->spare);
   if (rc != LORA_OK) return rc;  // the plan is unchanged
-  plan->hp = std::move(hp);
+  std::swap(plan->hp, plan->spare);
   return upload_plan(plan, stream, false);
 }
 

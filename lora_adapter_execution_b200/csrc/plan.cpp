@@ -44,6 +44,26 @@ void append_aug_blocks(const ChunkDesc *chunks, int32_t nchunk, int32_t kaug, st
   }
 }
 
+// Empty every table of the plan but keep its storage: a rebuild for the next
+// batch then allocates nothing once the tables have reached their sizes.
+static void reset_plan(HostPlan &hp) {
+  hp.perm.clear();
+  hp.seg.clear();
+  hp.offsets.clear();
+  hp.tiles.clear();
+  hp.chunks.clear();
+  hp.units.clear();
+  hp.augblocks.clear();
+  hp.mt_order.clear();
+  hp.pieces.clear();
+  hp.partial_rows = 0;
+  hp.r_max = 0;
+  hp.sum_r_used = hp.sum_r_tokens = hp.aug_k_total = 0;
+  hp.scratch_bytes = 0;
+  hp.xs_offset = -1;
+  hp.max_chunk_rows = 0;
+}
+
 int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t n_adapters,
                     int64_t d_in, int64_t d_out, HostPlan &hp) {
   if (!ids || !ranks || T <= 0 || n_adapters <= 0 || d_in < 8 || d_out < 8 || (d_in % 8) ||
@@ -53,10 +73,14 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
     return LORA_ERR_ARG;
   for (int32_t a = 0; a < n_adapters; ++a)
     if (ranks[a] < 1 || ranks[a] > LORA_MAX_RANK) return LORA_ERR_RANK;
-  for (int64_t t = 0; t < T; ++t)
-    if (ids[t] < 0 || ids[t] >= n_adapters) return LORA_ERR_ID;
+  {
+    // one unsigned compare per id (negative ids wrap above n_adapters), no early exit
+    uint32_t bad = 0;
+    for (int64_t t = 0; t < T; ++t) bad |= static_cast<uint32_t>(ids[t]) >= static_cast<uint32_t>(n_adapters);
+    if (bad) return LORA_ERR_ID;
+  }
 
-  hp = HostPlan();
+  reset_plan(hp);
   hp.T = T;
   hp.d_in = d_in;
   hp.d_out = d_out;
@@ -66,15 +90,34 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
   for (int32_t a = 0; a < n_adapters; ++a) hp.offsets[a + 1] = hp.offsets[a] + ranks[a];
   if (hp.offsets[n_adapters] >= ((int64_t)1 << 31) - 256) return LORA_ERR_ARG;
 
-  // Stable counting sort by adapter id.
-  std::vector<int64_t> count(n_adapters + 1, 0);
-  for (int64_t t = 0; t < T; ++t) ++count[ids[t] + 1];
+  // Stable counting sort by adapter id (T < 2^30: positions fit int32). Both
+  // passes walk runs of equal ids with the run's counter in a register: a
+  // batch of whole requests has long runs, where one increment per token in
+  // memory would wait on the previous one.
+  static thread_local std::vector<int32_t> count, cursor;
+  count.assign(n_adapters + 1, 0);
+  for (int64_t t = 0; t < T;) {
+    const int32_t a = ids[t];
+    int64_t e = t + 1;
+    while (e < T && ids[e] == a) ++e;
+    count[a + 1] += static_cast<int32_t>(e - t);
+    t = e;
+  }
   for (int32_t a = 0; a < n_adapters; ++a) count[a + 1] += count[a];  // count[a] = start of a
-  std::vector<int64_t> cursor(count.begin(), count.end() - 1);
-  hp.perm.assign(T, 0);
-  for (int64_t t = 0; t < T; ++t) hp.perm[cursor[ids[t]]++] = (int32_t)t;
+  cursor.assign(count.begin(), count.end() - 1);
+  hp.perm.resize(T);
+  int32_t *perm = hp.perm.data();
+  int32_t *cur = cursor.data();
+  for (int64_t t = 0; t < T;) {
+    const int32_t a = ids[t];
+    int32_t c = cur[a];
+    do perm[c++] = static_cast<int32_t>(t++);
+    while (t < T && ids[t] == a);
+    cur[a] = c;
+  }
 
   // Segments, ascending adapter id, adapters without tokens skipped.
+  hp.seg.reserve(3 * static_cast<size_t>(std::min<int64_t>(n_adapters, T)));
   for (int32_t a = 0; a < n_adapters; ++a) {
     int64_t len = count[a + 1] - count[a];
     if (len == 0) continue;
@@ -92,6 +135,8 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
   // step: s*U enters the MMA as bf16 hi + lo parts against the same B rows,
   // so the adapter term keeps ~16 mantissa bits whatever the scale.
   const int64_t n_tiles = (T + kTileM - 1) / kTileM;
+  hp.tiles.reserve(n_tiles);
+  hp.chunks.reserve(n_tiles + n_seg);  // a chunk per segment, plus one per tile boundary a segment crosses
   int32_t s = 0;  // current segment
   int64_t uofs = 0;
   for (int64_t m = 0; m < n_tiles; ++m) {
@@ -230,10 +275,22 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
   // blocks start in index order as earlier ones finish, so the units with the
   // most rows and rank columns per 64-column block go in the first wave and
   // the short ones fill the tail. Units write disjoint parts of the image and
-  // of U_save, so their order is free.
-  std::stable_sort(hp.units.begin(), hp.units.end(), [](const UnitDesc &x, const UnitDesc &y) {
-    return ((x.r1 - x.r0 + 15) / 16) * 16 + x.nn > ((y.r1 - y.r0 + 15) / 16) * 16 + y.nn;
-  });
+  // of U_save, so their order is free. The key (rows rounded up to 16, plus
+  // the piece width) is at most kTileM + kShrinkN: a stable bucket sort by
+  // decreasing key.
+  {
+    constexpr int kKeys = kTileM + kShrinkN + 1;
+    auto key = [](const UnitDesc &u) { return ((u.r1 - u.r0 + 15) / 16) * 16 + u.nn; };
+    int32_t start[kKeys + 1] = {};
+    for (const UnitDesc &u : hp.units) ++start[kKeys - key(u)];  // bucket kKeys - key: largest key first
+    for (int k = 0; k < kKeys; ++k) start[k + 1] += start[k];
+    static thread_local std::vector<UnitDesc> sorted;
+    sorted.resize(hp.units.size());
+    int32_t pos[kKeys] = {};
+    for (int k = 0; k < kKeys; ++k) pos[k] = start[k];
+    for (const UnitDesc &u : hp.units) sorted[pos[kKeys - 1 - key(u)]++] = u;
+    hp.units.swap(sorted);
+  }
   return LORA_OK;
 }
 
