@@ -280,15 +280,18 @@ int build_host_plan(const int32_t *ids, int64_t T, const int32_t *ranks, int32_t
   // decreasing key.
   {
     constexpr int kKeys = kTileM + kShrinkN + 1;
-    auto key = [](const UnitDesc &u) { return ((u.r1 - u.r0 + 15) / 16) * 16 + u.nn; };
-    int32_t start[kKeys + 1] = {};
-    for (const UnitDesc &u : hp.units) ++start[kKeys - key(u)];  // bucket kKeys - key: largest key first
+    // bucket of a unit: kKeys - 1 - key, so the largest key comes first (the
+    // clamp only guards the arrays: rows <= kTileM and nn <= kShrinkN hold)
+    auto bucket = [](const UnitDesc &u) {
+      const int key = ((u.r1 - u.r0 + 15) / 16) * 16 + u.nn;
+      return kKeys - 1 - std::min(std::max(key, 0), kKeys - 1);
+    };
+    int32_t start[kKeys + 1] = {};  // start[b + 1] counts bucket b, then the prefix sums
+    for (const UnitDesc &u : hp.units) ++start[bucket(u) + 1];
     for (int k = 0; k < kKeys; ++k) start[k + 1] += start[k];
     static thread_local std::vector<UnitDesc> sorted;
     sorted.resize(hp.units.size());
-    int32_t pos[kKeys] = {};
-    for (int k = 0; k < kKeys; ++k) pos[k] = start[k];
-    for (const UnitDesc &u : hp.units) sorted[pos[kKeys - 1 - key(u)]++] = u;
+    for (const UnitDesc &u : hp.units) sorted[start[bucket(u)]++] = u;
     hp.units.swap(sorted);
   }
   return LORA_OK;
