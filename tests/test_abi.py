@@ -64,6 +64,8 @@ def test_plan_argument_errors():
     assert _host_plan([0, 3], [4, 4, 4]) == -2           # id out of range
     assert _host_plan([-1], [4]) == -2
     assert _host_plan([0] * 300 + [3], [4, 4, 4]) == -2   # last id of a long run of valid ones
+    assert _host_plan([], [4]) == -1                      # an empty batch (T = 0)
+    assert _host_plan([0], []) == -1                      # no adapters
     assert _host_plan([1] * 50 + [-2**31] + [1] * 50, [4, 4]) == -2
     assert _host_plan([0], [0]) == -3                     # rank 0
     assert _host_plan([0], [257]) == -3                   # rank above the maximum
