@@ -104,7 +104,10 @@ int lora_plan_build(const int32_t *ids_host, int64_t T, const int32_t *ranks_hos
 /* Refill an existing device plan with a new batch (arguments as in
  * lora_plan_build). The plan's device tables and scratch are reused when they
  * are large enough and reallocated otherwise, so a serving loop that builds one
- * plan per batch does not allocate device memory per batch. The tables are
+ * plan per batch does not allocate device memory per batch; its host tables are
+ * kept in two sets (the new batch is planned into the spare set, which becomes
+ * the plan's on success), so once they have grown a rebuild allocates no host
+ * memory either. The tables are
  * copied to the device on `stream` from one of two pinned host staging buffers
  * the plan owns (used in turn; a buffer is refilled only after its previous copy
  * has completed), and the call returns without waiting for that copy: work that
