@@ -782,6 +782,17 @@ def measure_e2e(cx, inp, copies, scale, mask_seed, K):
         d2h += T * di * 2
     Ke = max(3, min(K, 200 if not finetune else 20))
 
+    fallback_note = ""
+    if not finetune:
+        # the forward workloads: one C-ABI call per step with host buffers; it
+        # must first reproduce the device-buffer forward bit for bit on every
+        # rank, else (or on any error) the steps below run as the
+        # Python-orchestrated loop
+        r = e2e_host_step_loop(cx, inp, copies, scale, mask_seed, Ke, h2d, d2h)
+        if r is not None:
+            return r
+        fallback_note = "; the host-step call failed or did not reproduce the device forward, so this loop ran"
+
     # Steps run as a pipeline over two slots (device buffers, plan, pinned
     # results): step i copies its inputs in on one stream, computes on a second
     # and copies its results out on a third, so the copies of one step overlap
@@ -852,7 +863,77 @@ def measure_e2e(cx, inp, copies, scale, mask_seed, K):
             "what": "per step: plan from host ids + H2D of X (pinned)" + (" and dY" if finetune else "")
                     + " + forward" + (" + backward + gradient all-reduce" if finetune else "")
                     + " + D2H of the result; steps pipelined over two slots (copy-in, compute and"
-                    " copy-out streams); host wall clock over the steps"}
+                    " copy-out streams); host wall clock over the steps" + fallback_note}
+
+
+def e2e_host_step_loop(cx, inp, copies, scale, mask_seed, Ke, h2d, d2h):
+    """The forward workloads' e2e through lora_linear_fwd_host: each step is one
+    call with host buffers (the plan rebuilt from the host ids, X copied in from
+    pinned host memory, the forward, Y copied out to pinned host memory), steps
+    alternating over two streams with a plan and a buffer set each, so one
+    step's copies overlap the other's kernels. The ranks first agree that the
+    call's first result equals the device-buffer forward bit for bit on every
+    rank (an all-reduce, taken by every rank whatever happened before it);
+    otherwise it returns None and nothing is timed."""
+    import torch
+    import lora_adapter_execution_b200 as lora
+    dev, world = cx.dev, cx.world
+    T, di, do = inp.T, inp.d_in, inp.d_out
+    streams, plans, pin_Ys = [], [], []
+    slots = copies[:2]
+
+    def step(i):
+        s = i % 2
+        c = slots[s]
+        lora.linear_fwd_host(plans[s], inp.ids, pin_X, c["X"], c["W"], c["A"], c["B"], scale, c["Y"], pin_Ys[s],
+                             p_drop=inp.p_drop, seed=mask_seed, U_save=c["U"], stream=streams[s])
+
+    def drain():
+        for st in streams:
+            st.synchronize()
+
+    ok = False
+    try:
+        pin_X = torch.from_numpy(inp.X.view(np.int16)).view(torch.bfloat16).pin_memory()
+        streams = [torch.cuda.Stream(device=dev) for _ in range(2)]
+        plans = [lora.Plan(inp.ids, inp.ranks, di, do, stream=st) for st in streams]
+        pin_Ys = [torch.empty(T, do, dtype=torch.bfloat16).pin_memory() for _ in range(2)]
+        for i in range(2):
+            step(i)
+        drain()
+        # the first step's host result against the device-buffer forward of the same batch
+        ref_plan = lora.Plan(inp.ids, inp.ranks, di, do)
+        Y_ref = torch.empty(T, do, dtype=torch.bfloat16, device=dev)
+        lora.linear_fwd(ref_plan, slots[0]["X"], slots[0]["W"], slots[0]["A"], slots[0]["B"], scale, Y_ref,
+                        p_drop=inp.p_drop, seed=mask_seed)
+        torch.cuda.synchronize(dev)
+        ref_plan.destroy()
+        ok = torch.equal(pin_Ys[0].view(torch.int16), Y_ref.cpu().view(torch.int16)) and lora.device_status() == 0
+    except Exception:  # noqa: BLE001
+        ok = False
+    if max_over_ranks(0.0 if ok else 1.0, world, dev) > 0:
+        drain()
+        for p in plans:
+            p.destroy()
+        return None
+    try:
+        cx.barrier()
+        t0 = time.perf_counter()
+        for i in range(Ke):
+            step(2 + i)
+        drain()
+        dt = time.perf_counter() - t0
+    finally:
+        drain()
+        for p in plans:
+            p.destroy()
+    dt = max_over_ranks(dt, world, dev)
+    return {"value": job_throughput(T, Ke, world, dt * 1e3), "unit": "tokens/s", "h2d_bytes_per_step": int(h2d),
+            "d2h_bytes_per_step": int(d2h), "steps": Ke,
+            "what": "per step: one lora_linear_fwd_host call (plan from host ids, H2D of X from pinned host "
+                    "memory, forward, D2H of Y into pinned host memory) on one of two streams, each with its "
+                    "own plan and buffers; checked bit for bit against the device-buffer forward first; host "
+                    "wall clock over the steps"}
 
 
 SWITCH = dict(L=32, d=4096, n_adapters=8, rank=16, prev=(2, 5), cur=(0, 7), gates=((0.6, 0.4), (0.7, 0.3)),

@@ -234,6 +234,36 @@ int lora_linear_shrink(lora_plan_t plan, const uint16_t *X, const uint16_t *A_po
 int lora_fused_gemm(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *B_pool,
                     uint16_t *Y, lora_stream_t stream);
 
+/* lora_linear_fwd_host — one serving step from host memory: the batch's plan
+ * from its host ids (lora_plan_rebuild of `plan` with the plan's d_in, d_out),
+ * the copy of X from host to device, lora_linear_fwd, and the copy of Y from
+ * device to host, queued on `stream` in that order. The call returns once the
+ * work is queued: Y_host holds the step's result when `stream` has passed it
+ * (synchronise the stream or wait on an event recorded after the call). With
+ * pinned host buffers both copies run asynchronously, so steps queued on two
+ * streams with two plans and two sets of buffers overlap one step's copies with
+ * the other's kernels. No counterpart in the pages (the per-batch host-to-device
+ * path of a serving loop around the layer).
+ *
+ *   plan        a device plan (lora_plan_build); rebuilt for this batch, so work on
+ *               other streams that still uses its previous batch must be ordered first
+ *   ids_host, T, ranks_host, n_adapters   the batch, as in lora_plan_build
+ *   X_host      bf16 [T, d_in] host
+ *   X_dev       bf16 [T, d_in] device buffer the step copies X into (16-byte aligned)
+ *   W, A_pool, B_pool, scale, p_drop, seed, U_save, keep_bits   as in lora_linear_fwd
+ *   Y_dev       bf16 [T, d_out] device output of the forward (16-byte aligned)
+ *   Y_host      bf16 [T, d_out] host destination of the copy out
+ * The caller owns every buffer; the call allocates nothing (beyond what a plan
+ * rebuild does when the batch outgrows the plan's buffers).
+ * Errors: as lora_plan_rebuild (the plan is unchanged on LORA_ERR_ARG, _ID or
+ * _RANK from it) and lora_linear_fwd; LORA_ERR_ARG for a null or misaligned
+ * buffer before anything is queued; LORA_ERR_CUDA when a copy cannot be queued. */
+int lora_linear_fwd_host(lora_plan_t plan, const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
+                         int32_t n_adapters, const uint16_t *X_host, uint16_t *X_dev, const uint16_t *W,
+                         const uint16_t *A_pool, const uint16_t *B_pool, const float *scale, double p_drop,
+                         uint64_t seed, uint16_t *Y_dev, uint16_t *Y_host, float *U_save,
+                         const uint32_t *keep_bits, lora_stream_t stream);
+
 /* lora_linear_fwd_fused — lora_linear_fwd in one launch (arguments and results
  * as lora_linear_fwd). Source: the kernel-layer fusion of the LoRAFusion
  * explainer (Kernel 层: split the graph only at real GEMM boundaries and keep

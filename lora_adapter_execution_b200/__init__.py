@@ -9,6 +9,6 @@ no CPU fallback: if the library is missing, every call raises.
 from . import abi  # noqa: F401
 from .abi import (LoraError, Plan, base_gemm, bwd_workspace_size, device_status, dropout_keep_bits, dropout_mask,  # noqa: F401
                   dropout_seed_for_rows, Switch, bwd_multi_workspace_size, linear_bwd_multi, linear_fwd_fused,
-                  fused_gemm, linear_bwd, linear_bwd_static, linear_fwd, linear_shrink, load_library,
+                  fused_gemm, linear_bwd, linear_bwd_static, linear_fwd, linear_fwd_host, linear_shrink, load_library,
                   selftest_bounded_wait, tsqr, tsqr_workspace_size, Compressor,
                   compress_allocate)

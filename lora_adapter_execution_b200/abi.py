@@ -72,6 +72,8 @@ def load_library():
         "lora_plan_destroy": (None, [_vp]),
         "lora_linear_fwd": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp, _vp]),
         "lora_linear_fwd_fused": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp, _vp]),
+        "lora_linear_fwd_host": (ctypes.c_int, [_vp, _vp, _i64, _vp, _i32, _vp, _vp, _vp, _vp, _vp, _vp, _dbl, _u64,
+                                                _vp, _vp, _vp, _vp, _vp]),
         "lora_linear_shrink": (ctypes.c_int, [_vp, _vp, _vp, _vp, _dbl, _u64, _vp, _vp, _vp]),
         "lora_fused_gemm": (ctypes.c_int, [_vp, _vp, _vp, _vp, _vp, _vp]),
         "lora_base_gemm": (ctypes.c_int, [_vp, _vp, _vp, _i64, _i64, _i64, _vp]),
@@ -267,6 +269,42 @@ def linear_fwd(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.
     _check(load_library().lora_linear_fwd(plan.handle, _ptr(X), _ptr(W), _ptr(A_pool), _ptr(B_pool), _ptr(scale),
                                           float(p_drop), int(seed) & (2**64 - 1), _ptr(Y), _ptr(U_save),
                                           _ptr(keep_bits), _stream(stream)), "lora_linear_fwd")
+
+
+def linear_fwd_host(plan: Plan, ids, X_host, X_dev, W, A_pool, B_pool, scale, Y_dev, Y_host, *,
+                    p_drop: float = 0.0, seed: int = 0, U_save=None, keep_bits=None, stream=None):
+    """lora_linear_fwd_host: one step from host memory (the plan rebuilt from the
+    host ids with its current ranks, X_host copied into X_dev, the forward into
+    Y_dev, Y_dev copied into Y_host), queued on `stream` (default: the current
+    torch stream); Y_host holds the result once the stream has passed the call.
+    X_host and Y_host are host tensors (pinned for the copies to overlap)."""
+    ids = _host_i32(ids)
+    T = ids.shape[0]
+    di, do, R = plan.d_in, plan.d_out, plan.pool_rows
+    for name, t, shape in (("X_host", X_host, (T, di)), ("Y_host", Y_host, (T, do))):
+        if t.shape != shape or _dtype_name(t.dtype) not in _BF16 or not t.is_contiguous():
+            raise LoraError(-1, f"lora_linear_fwd_host: {name} must be a contiguous bfloat16 tensor of shape {shape}")
+        if t.get_device() >= 0:
+            raise LoraError(-1, f"lora_linear_fwd_host: {name} must be in host memory")
+    # U_save's rows are as long as the largest rank among the batch's adapters
+    # (ids out of range: the library reports them before anything is queued)
+    rmax = 0
+    if U_save is not None:
+        valid = T > 0 and ids.min() >= 0 and ids.max() < plan._ranks.shape[0]
+        rmax = int(plan._ranks[ids].max()) if valid else (U_save.shape[1] if U_save.dim() == 2 else 0)
+    _args("lora_linear_fwd_host", ("X_dev", X_dev, (T, di), _BF16, False), ("W", W, (di, do), _BF16, False),
+          ("A_pool", A_pool, (R, di), _BF16, False), ("B_pool", B_pool, (R, do), _BF16, False),
+          ("scale", scale, (plan.n_adapters,), _F32, False), ("Y_dev", Y_dev, (T, do), _BF16, False),
+          ("U_save", U_save, (T, rmax), _F32, True), ("keep_bits", keep_bits, (T, -(-di // 32)), _I32, True))
+    _check(load_library().lora_linear_fwd_host(plan.handle, ids.ctypes.data_as(_vp), T,
+                                               plan._ranks.ctypes.data_as(_vp), plan._ranks.shape[0],
+                                               _ptr(X_host), _ptr(X_dev), _ptr(W), _ptr(A_pool), _ptr(B_pool),
+                                               _ptr(scale), float(p_drop), int(seed) & (2**64 - 1), _ptr(Y_dev),
+                                               _ptr(Y_host), _ptr(U_save), _ptr(keep_bits), _stream(stream)),
+           "lora_linear_fwd_host")
+    plan._ids = ids
+    plan.T = T
+    plan._sizes(False)
 
 
 def linear_fwd_fused(plan: Plan, X, W, A_pool, B_pool, scale, Y, *, p_drop: float = 0.0, seed: int = 0,

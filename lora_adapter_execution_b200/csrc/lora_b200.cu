@@ -860,6 +860,35 @@ int lora_linear_fwd(lora_plan_t plan, const uint16_t *X, const uint16_t *W, cons
   return lora_fused_gemm(plan, X, W, B_pool, Y, stream);
 }
 
+int lora_linear_fwd_host(lora_plan_t plan, const int32_t *ids_host, int64_t T, const int32_t *ranks_host,
+                         int32_t n_adapters, const uint16_t *X_host, uint16_t *X_dev, const uint16_t *W,
+                         const uint16_t *A_pool, const uint16_t *B_pool, const float *scale, double p_drop,
+                         uint64_t seed, uint16_t *Y_dev, uint16_t *Y_host, float *U_save, const uint32_t *keep_bits,
+                         lora_stream_t stream) {
+  // every argument is checked before anything is queued
+  if (!plan || !plan->dev || !ids_host || !ranks_host || !X_host || !X_dev || !Y_dev || !Y_host) return LORA_ERR_ARG;
+  if (!W || !A_pool || !B_pool || !scale) return LORA_ERR_ARG;
+  if (!aligned16(X_dev) || !aligned16(W) || !aligned16(A_pool) || !aligned16(B_pool) || !aligned16(Y_dev))
+    return LORA_ERR_ARG;
+  if (reinterpret_cast<uintptr_t>(keep_bits) & 3u) return LORA_ERR_ARG;
+  if (!(p_drop >= 0.0 && p_drop < 1.0)) return LORA_ERR_ARG;
+  const int64_t d_in = plan->hp.d_in, d_out = plan->hp.d_out;
+  int rc = lora_plan_rebuild(plan, ids_host, T, ranks_host, n_adapters, d_in, d_out, stream);
+  if (rc != LORA_OK) return rc;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(X_dev, X_host, static_cast<size_t>(T * d_in) * 2, cudaMemcpyHostToDevice, st) != cudaSuccess) {
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  rc = lora_linear_fwd(plan, X_dev, W, A_pool, B_pool, scale, p_drop, seed, Y_dev, U_save, keep_bits, stream);
+  if (rc != LORA_OK) return rc;
+  if (cudaMemcpyAsync(Y_host, Y_dev, static_cast<size_t>(T * d_out) * 2, cudaMemcpyDeviceToHost, st) != cudaSuccess) {
+    cudaGetLastError();
+    return LORA_ERR_CUDA;
+  }
+  return LORA_OK;
+}
+
 int lora_linear_fwd_fused(lora_plan_t plan, const uint16_t *X, const uint16_t *W, const uint16_t *A_pool,
                           const uint16_t *B_pool, const float *scale, double p_drop, uint64_t seed, uint16_t *Y,
                           float *U_save, const uint32_t *keep_bits, lora_stream_t stream) {

@@ -81,6 +81,25 @@ def test_null_plan_calls():
     assert L.lora_plan_info(None, None) == -1
     L.lora_plan_destroy(None)  # ignored
     assert L.lora_linear_fwd(None, None, None, None, None, None, 0.0, 0, None, None, None, None) == -1
+    assert L.lora_linear_fwd_host(None, None, 0, None, 0, None, None, None, None, None, None, 0.0, 0, None, None,
+                                  None, None, None) == -1
+
+
+def test_fwd_host_step_rejects_a_host_only_plan_before_cuda():
+    """lora_linear_fwd_host checks its plan and buffers before it queues
+    anything: a host-only plan (no device tables) and null buffers are argument
+    errors, with no CUDA call made."""
+    L = abi.load_library()
+    ids = np.zeros(4, dtype=np.int32)
+    ranks = np.array([4], dtype=np.int32)
+    h = ctypes.c_void_p()
+    assert L.lora_plan_build_host(ids.ctypes.data_as(ctypes.c_void_p), 4, ranks.ctypes.data_as(ctypes.c_void_p), 1,
+                                  64, 64, ctypes.byref(h)) == 0
+    p = ctypes.c_void_p(256)  # never dereferenced: validation fails first
+    idp, rp = ids.ctypes.data_as(ctypes.c_void_p), ranks.ctypes.data_as(ctypes.c_void_p)
+    assert L.lora_linear_fwd_host(h, idp, 4, rp, 1, p, p, p, p, p, p, 0.0, 0, p, p, None, None, None) == -1
+    assert L.lora_linear_fwd_host(h, idp, 4, rp, 1, None, p, p, p, p, p, 0.0, 0, p, p, None, None, None) == -1
+    L.lora_plan_destroy(h)
 
 
 def test_bwd_workspace_size_monotone():

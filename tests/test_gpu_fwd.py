@@ -316,3 +316,36 @@ def test_fwd_argument_errors():
     with pytest.raises(lora.LoraError):
         lora.linear_fwd(host_plan, X, W, A, B, scale, Y)
     assert lora.device_status() == 0
+
+
+@pytest.mark.parametrize("name,kw", [("decode", dict(T=300, d_in=328, d_out=264, n_adapters=40)),
+                                     ("fleet", dict(T=700, d_in=320, d_out=296, n_adapters=200))])
+def test_fwd_host_step_matches_device_forward(name, kw):
+    """lora_linear_fwd_host (plan rebuilt from host ids, X copied in from pinned
+    host memory, the forward, Y copied out) on two different batches through one
+    plan: each step's host Y equals, bit for bit, lora_linear_fwd on device
+    buffers with a plan built for that batch, and matches the oracle."""
+    import lora_adapter_execution_b200 as lora
+    inp = wl.make_inputs(name, **kw)
+    W, A, B = dev_bf16(inp.W), dev_bf16(inp.A_pool), dev_bf16(inp.B_pool)
+    scale = torch.from_numpy(inp.scale).cuda()
+    step_plan = lora.Plan(inp.ids, inp.ranks, inp.d_in, inp.d_out)
+    X_dev = torch.empty(inp.T, inp.d_in, dtype=torch.bfloat16, device="cuda")
+    Y_dev = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+    rng = np.random.default_rng(9)
+    for it in range(2):
+        ids = inp.ids if it == 0 else rng.integers(0, inp.n_adapters, size=inp.T).astype(np.int32)
+        Xb = inp.X if it == 0 else wl.f32_to_bf16_bits(rng.standard_normal(inp.X.shape).astype(np.float32))
+        X_host = torch.from_numpy(np.ascontiguousarray(Xb).view(np.int16)).view(torch.bfloat16).pin_memory()
+        Y_host = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16).pin_memory()
+        lora.linear_fwd_host(step_plan, ids, X_host, X_dev, W, A, B, scale, Y_dev, Y_host)
+        torch.cuda.synchronize()
+        assert lora.device_status() == 0
+        ref_plan = lora.Plan(ids, inp.ranks, inp.d_in, inp.d_out)
+        Y_ref = torch.empty(inp.T, inp.d_out, dtype=torch.bfloat16, device="cuda")
+        lora.linear_fwd(ref_plan, dev_bf16(Xb), W, A, B, scale, Y_ref)
+        torch.cuda.synchronize()
+        ref_plan.destroy()
+        assert torch.equal(Y_host.view(torch.int16), Y_ref.cpu().view(torch.int16)), f"{name} batch {it}"
+        check_close(host_f64(Y_ref), oracle.forward(dataclasses.replace(inp, ids=ids, X=Xb)), f"{name} host step {it}")
+    step_plan.destroy()
